@@ -1,0 +1,224 @@
+"""fp64 CPU oracle for the SALA hybrid attention forward.
+
+TEST INFRASTRUCTURE ONLY: the test suite, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` are the only callers.  The product path (``hybrid_sparse_linear_b200``) never imports
+this package, and this package never imports the product.
+
+The arithmetic lives in ``sala_oracle.cpp`` (plain loops, fp64); this module only marshals numpy
+arrays through ctypes.  Every function takes float64 arrays in the row-major layouts documented in
+the C source: ``q, k, v`` are ``[B, heads, rows, dim]``.  ``from_tensor`` turns a torch tensor of
+any dtype the GPU path uses (bf16, fp32) into the exact float64 values it holds.
+
+Pinned by ``tests/test_oracle_*.py`` (closed forms, brute force, invariants between independent
+forms); see the module docstrings there for which pin covers which function.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "sala_oracle.cpp")
+_LIB_PATH = os.path.join(_HERE, "liborc.so")
+_lock = threading.Lock()
+_lib = None
+
+_D = ctypes.POINTER(ctypes.c_double)
+_I32 = ctypes.POINTER(ctypes.c_int32)
+_I64 = ctypes.POINTER(ctypes.c_int64)
+_i = ctypes.c_int
+_l = ctypes.c_int64
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with g++ (fp64, -O2, no fast-math) into ``oracle/liborc.so``."""
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(["g++", "-O2", "-std=c++17", "-fPIC", "-shared", "-pthread",
+                               "-fno-fast-math", "-ffp-contract=off", _SRC, "-o", tmp])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            lib.orc_round_bf16.restype = ctypes.c_double
+            lib.orc_round_bf16.argtypes = [ctypes.c_double]
+            lib.orc_linear_recurrent.argtypes = [_D, _D, _D, _D, _D, _D, _D, _i, _i, _i, _i, _i, _i]
+            lib.orc_linear_quadratic.argtypes = [_D, _D, _D, _D, _D, _D, _i, _i, _i, _i, _i, _I64, _l, _i]
+            lib.orc_linear_chunked.argtypes = [_D, _D, _D, _D, _D, _D, _D, _i, _i, _i, _i, _i, _i, _i]
+            lib.orc_linear_decode.argtypes = [_D, _D, _D, _D, _D, _D, _i, _i, _i, _i]
+            lib.orc_block_compress.argtypes = [_D, _D, _i, _i, _i, _i, _i, _i, _i, _i]
+            lib.orc_block_scores_at.argtypes = [_D, _D, _I64, _l, _D, _i, _i, _i, _i, _i]
+            lib.orc_block_select.argtypes = [_D, _D, _I32, _D, _i, _i, _i, _i, _i, _i, _i, _i, _i,
+                                             _i, _i, _i, _i]
+            lib.orc_sparse_attention.argtypes = [_D, _D, _D, _I32, _D, _i, _i, _i, _i, _i, _i, _i,
+                                                 _i, _i, ctypes.c_double, _I64, _l, _i]
+            lib.orc_dense_causal_attention.argtypes = [_D, _D, _D, _D, _i, _i, _i, _i, _i, _i, _i,
+                                                       ctypes.c_double, _i]
+            for name in ("orc_linear_recurrent", "orc_linear_quadratic", "orc_linear_chunked",
+                         "orc_linear_decode", "orc_block_compress", "orc_block_scores_at",
+                         "orc_block_select", "orc_sparse_attention", "orc_dense_causal_attention"):
+                getattr(lib, name).restype = None
+            _lib = lib
+    return _lib
+
+
+def default_threads() -> int:
+    return max(1, len(os.sched_getaffinity(0)))
+
+
+def from_tensor(t) -> np.ndarray:
+    """Exact float64 copy of a torch tensor (bf16 and fp32 values are exact in fp64)."""
+    import torch
+    return t.detach().to("cpu", torch.float64).contiguous().numpy()
+
+
+def _f64(a) -> np.ndarray:
+    return np.ascontiguousarray(a, dtype=np.float64)
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data_as(_D)
+
+
+def round_bf16(x):
+    """bf16 round-to-nearest-even of float64 values (elementwise)."""
+    lib = _load()
+    x = np.asarray(x, dtype=np.float64)
+    return np.vectorize(lib.orc_round_bf16, otypes=[np.float64])(x) if x.ndim else \
+        lib.orc_round_bf16(float(x))
+
+
+# ----------------------------------------------------------------------------------------------
+# Linear attention
+
+def _lin_args(q, k, v, lam, s_in):
+    q, k, v, lam = _f64(q), _f64(k), _f64(v), _f64(lam)
+    B, H, N, dk = q.shape
+    dv = v.shape[-1]
+    assert k.shape == (B, H, N, dk) and v.shape == (B, H, N, dv) and lam.shape == (H,)
+    s_in = None if s_in is None else _f64(s_in)
+    if s_in is not None:
+        assert s_in.shape == (B, H, dk, dv)
+    return q, k, v, lam, s_in, B, H, N, dk, dv
+
+
+def linear_recurrent(q, k, v, lam, s_in=None, threads=None):
+    """Recurrent form: S <- lambda S + k^T v; o = q S.  Returns (o, s_out)."""
+    q, k, v, lam, s_in, B, H, N, dk, dv = _lin_args(q, k, v, lam, s_in)
+    o = np.empty((B, H, N, dv)); s_out = np.empty((B, H, dk, dv))
+    _load().orc_linear_recurrent(_p(q), _p(k), _p(v), _p(lam), _p(s_in), _p(o), _p(s_out),
+                                 B, H, N, dk, dv, threads or default_threads())
+    return o, s_out
+
+
+def linear_quadratic(q, k, v, lam, s_in=None, rows=None, threads=None):
+    """Quadratic form.  rows: optional int array [n, 2] of (b*H + h, token); returns [n, dv]."""
+    q, k, v, lam, s_in, B, H, N, dk, dv = _lin_args(q, k, v, lam, s_in)
+    if rows is None:
+        o = np.empty((B, H, N, dv)); rp = None; n = 0
+    else:
+        rows = np.ascontiguousarray(rows, dtype=np.int64).reshape(-1, 2)
+        n = rows.shape[0]; o = np.empty((n, dv)); rp = rows.ctypes.data_as(_I64)
+    _load().orc_linear_quadratic(_p(q), _p(k), _p(v), _p(lam), _p(s_in), _p(o), B, H, N, dk, dv,
+                                 rp, n, threads or default_threads())
+    return o
+
+
+def linear_chunked(q, k, v, lam, chunk, s_in=None, threads=None):
+    """Chunked form (intra-chunk mask + carried state).  Returns (o, s_out)."""
+    q, k, v, lam, s_in, B, H, N, dk, dv = _lin_args(q, k, v, lam, s_in)
+    o = np.empty((B, H, N, dv)); s_out = np.empty((B, H, dk, dv))
+    _load().orc_linear_chunked(_p(q), _p(k), _p(v), _p(lam), _p(s_in), _p(o), _p(s_out),
+                               B, H, N, dk, dv, int(chunk), threads or default_threads())
+    return o, s_out
+
+
+def linear_decode(q, k, v, lam, state):
+    """One decode step.  q,k: [B,H,dk]; v: [B,H,dv]; state [B,H,dk,dv].  Returns (o, new_state)."""
+    q, k, v, lam = _f64(q), _f64(k), _f64(v), _f64(lam)
+    S = _f64(state).copy()
+    B, H, dk, dv = S.shape
+    o = np.empty((B, H, dv))
+    _load().orc_linear_decode(_p(q), _p(k), _p(v), _p(lam), _p(S), _p(o), B, H, dk, dv)
+    return o, S
+
+
+# ----------------------------------------------------------------------------------------------
+# Sparse attention
+
+def block_compress(k, block, first_block=0, n_blocks=None, round_to_bf16=True):
+    """Mean of each complete block of keys, rounded once to bf16.  k: [B,Hkv,N,d]."""
+    k = _f64(k)
+    B, Hkv, N, d = k.shape
+    if n_blocks is None:
+        n_blocks = N // block - first_block
+    assert 0 <= first_block and (first_block + n_blocks) * block <= N
+    out = np.empty((B, Hkv, n_blocks, d))
+    _load().orc_block_compress(_p(k), _p(out), B, Hkv, N, d, block, first_block, n_blocks,
+                               1 if round_to_bf16 else 0)
+    return out
+
+
+def block_select(q, kbar, block, topk, n_init, n_local, q_pos0=0, slots=None, threads=None):
+    """Per (batch, KV group, query row) block selection.  Returns (idx int32, kth_score)."""
+    q, kbar = _f64(q), _f64(kbar)
+    B, H, Nq, d = q.shape
+    Hkv, nb = kbar.shape[1], kbar.shape[2]
+    slots = slots or (n_init + n_local + topk)
+    idx = np.empty((B, Hkv, Nq, slots), dtype=np.int32)
+    kth = np.empty((B, Hkv, Nq))
+    _load().orc_block_select(_p(q), _p(kbar), idx.ctypes.data_as(_I32), _p(kth), B, H, Hkv, Nq,
+                             int(q_pos0), nb, d, block, topk, n_init, n_local, slots,
+                             threads or default_threads())
+    return idx, kth
+
+
+def block_scores_at(q, kbar, quads):
+    """Scores for (b, g, r, block) quadruples (int array [n, 4])."""
+    q, kbar = _f64(q), _f64(kbar)
+    B, H, Nq, d = q.shape
+    Hkv, nb = kbar.shape[1], kbar.shape[2]
+    quads = np.ascontiguousarray(quads, dtype=np.int64).reshape(-1, 4)
+    out = np.empty(quads.shape[0])
+    _load().orc_block_scores_at(_p(q), _p(kbar), quads.ctypes.data_as(_I64), quads.shape[0],
+                                _p(out), H, Hkv, Nq, nb, d)
+    return out
+
+
+def sparse_attention(q, k, v, idx, block, scale=None, q_pos0=0, rows=None, threads=None):
+    """Softmax attention over the selected blocks.  rows: optional [n, 2] of (b*H + h, r)."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H, Nq, d = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    slots = idx.shape[-1]
+    scale = (1.0 / np.sqrt(d)) if scale is None else float(scale)
+    if rows is None:
+        o = np.empty((B, H, Nq, d)); rp = None; n = 0
+    else:
+        rows = np.ascontiguousarray(rows, dtype=np.int64).reshape(-1, 2)
+        n = rows.shape[0]; o = np.empty((n, d)); rp = rows.ctypes.data_as(_I64)
+    _load().orc_sparse_attention(_p(q), _p(k), _p(v), idx.ctypes.data_as(_I32), _p(o), B, H, Hkv,
+                                 Nq, int(q_pos0), Nk, d, block, slots, scale, rp, n,
+                                 threads or default_threads())
+    return o
+
+
+def dense_causal_attention(q, k, v, scale=None, q_pos0=0, threads=None):
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H, Nq, d = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    scale = (1.0 / np.sqrt(d)) if scale is None else float(scale)
+    o = np.empty((B, H, Nq, d))
+    _load().orc_dense_causal_attention(_p(q), _p(k), _p(v), _p(o), B, H, Hkv, Nq, int(q_pos0), Nk,
+                                       d, scale, threads or default_threads())
+    return o

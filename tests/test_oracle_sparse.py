@@ -1,0 +1,254 @@
+"""Pins for the oracle's block-sparse (InfLLM-V2-style) attention.
+
+* bf16 rounding: hand-picked ties and torch's float32 -> bf16 conversion (a library routine,
+  exact for fp32-representable inputs);                                   [library / by hand]
+* block compression: constant blocks and arithmetic sequences give closed-form means;
+* selection: the defining properties (forced blocks present, k best candidates by
+  (score desc, index asc), nothing in the future, ascending, -1 padded) checked on every row,
+  plus a by-hand case (tests/golden/sparse_scalar.json) and the structural invariant that blocks
+  shifted along the query direction are always chosen when at most k are causally available;
+* attention: with top-k >= every block the sparse path equals dense causal softmax, which in turn
+  equals torch's scaled_dot_product_attention in fp64; all-equal keys give the mean of V over
+  the attended set; position 0 returns v_0.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# ------------------------------------------------------------------------------ bf16 rounding
+
+def test_round_bf16_ties_and_specials():
+    r = oracle.round_bf16
+    assert r(1.0 + 2 ** -8) == 1.0                     # tie -> even (1.0)
+    assert r(1.0 + 3 * 2 ** -8) == 1.0 + 2 ** -6        # tie -> even (mantissa 2)
+    assert r(1.0 + 2 ** -8 + 2 ** -30) == 1.0 + 2 ** -7  # just above the tie
+    assert r(-(1.0 + 2 ** -8)) == -1.0
+    assert r(0.0) == 0.0
+    assert r(2.0 ** -133) == 2.0 ** -133                # smallest bf16 subnormal
+    assert r(3.0 * 2.0 ** -135) == 2.0 ** -133
+    assert math.isinf(r(3.4e38))
+
+
+def test_round_bf16_matches_torch_on_fp32_values():
+    rng = np.random.default_rng(11)
+    x32 = (rng.standard_normal(20000) * np.exp(rng.uniform(-20, 20, 20000))).astype(np.float32)
+    expect = torch.from_numpy(x32).to(torch.bfloat16).to(torch.float64).numpy()
+    got = oracle.round_bf16(x32.astype(np.float64))
+    np.testing.assert_array_equal(got, expect)
+
+
+# ------------------------------------------------------------------------------ compression
+
+def test_block_compress_closed_forms():
+    B, Hkv, T, nb, d = 1, 2, 8, 5, 3
+    N = T * nb + 3  # a ragged tail that is never compressed
+    k = np.zeros((B, Hkv, N, d))
+    for g in range(Hkv):
+        for blk in range(nb):
+            k[0, g, blk * T:(blk + 1) * T, 0] = blk + 0.25 * g           # constant per block
+            k[0, g, blk * T:(blk + 1) * T, 1] = np.arange(T) + blk      # arithmetic sequence
+            k[0, g, blk * T:(blk + 1) * T, 2] = (-1.0) ** np.arange(T)  # alternating -> 0
+    kb = oracle.block_compress(k, T)
+    assert kb.shape == (B, Hkv, nb, d)
+    for g in range(Hkv):
+        for blk in range(nb):
+            assert kb[0, g, blk, 0] == blk + 0.25 * g
+            assert kb[0, g, blk, 1] == (T - 1) / 2 + blk
+            assert kb[0, g, blk, 2] == 0.0
+    part = oracle.block_compress(k, T, first_block=2, n_blocks=2)
+    np.testing.assert_array_equal(part, kb[:, :, 2:4])
+
+
+def test_block_compress_rounds_once():
+    # mean = 1 + 2^-8 + 2^-12 (just above a bf16 tie) must round up, not to even.
+    T = 4
+    k = np.full((1, 1, T, 1), 1.0 + 2 ** -8 + 2 ** -12)
+    assert oracle.block_compress(k, T)[0, 0, 0, 0] == 1.0 + 2 ** -7
+    assert oracle.block_compress(k, T, round_to_bf16=False)[0, 0, 0, 0] == 1.0 + 2 ** -8 + 2 ** -12
+
+
+# ------------------------------------------------------------------------------ selection
+
+def _check_selection_properties(q, kbar, idx, T, topk, n_init, n_local, q_pos0=0):
+    B, H, Nq, d = q.shape
+    Hkv = kbar.shape[1]
+    G = H // Hkv
+    qs = q.reshape(B, Hkv, G, Nq, d).sum(axis=2)                      # group sum per row
+    scores = np.einsum("bgnd,bgkd->bgnk", qs, kbar)
+    for b in range(B):
+        for g in range(Hkv):
+            for r in range(Nq):
+                pos = q_pos0 + r
+                c = pos // T
+                row = list(idx[b, g, r])
+                sel = [x for x in row if x >= 0]
+                assert row == sel + [-1] * (len(row) - len(sel))
+                assert sel == sorted(set(sel))
+                forced = set(range(min(n_init, c + 1))) | set(range(max(0, c - n_local + 1), c + 1))
+                assert forced <= set(sel)
+                cand = [x for x in range(n_init, c - n_local + 1)]
+                chosen = [x for x in sel if x not in forced]
+                assert set(chosen) <= set(cand)
+                assert len(chosen) == min(topk, len(cand))
+                rest = [x for x in cand if x not in chosen]
+                key = lambda x: (scores[b, g, r, x], -x)
+                if chosen and rest:
+                    assert min(key(x) for x in chosen) > max(key(x) for x in rest)
+
+
+@pytest.mark.parametrize("G,topk,n_init,n_local", [(1, 2, 1, 1), (4, 3, 1, 2), (2, 1, 2, 1),
+                                                   (3, 5, 0, 3)])
+def test_selection_properties(G, topk, n_init, n_local):
+    rng = np.random.default_rng(20 + G + topk)
+    B, Hkv, T, d = 2, 2, 4, 6
+    N = 14 * T + 3
+    q = rng.standard_normal((B, Hkv * G, N, d))
+    k = rng.standard_normal((B, Hkv, N, d))
+    kbar = oracle.block_compress(k, T)
+    idx, _ = oracle.block_select(q, kbar, T, topk, n_init, n_local)
+    _check_selection_properties(q, kbar, idx, T, topk, n_init, n_local)
+
+
+def test_selection_with_query_offset():
+    rng = np.random.default_rng(31)
+    B, H, Hkv, T, d = 1, 4, 2, 4, 5
+    N = 40
+    k = rng.standard_normal((B, Hkv, N, d))
+    q = rng.standard_normal((B, H, 3, d))
+    kbar = oracle.block_compress(k, T)
+    idx, _ = oracle.block_select(q, kbar, T, 2, 1, 2, q_pos0=N - 3)
+    _check_selection_properties(q, kbar, idx, T, 2, 1, 2, q_pos0=N - 3)
+
+
+def test_selection_ties_go_to_lower_index():
+    T, d = 2, 1
+    k = np.zeros((1, 1, 12, d))
+    k[0, 0, 2:4] = 1.0
+    k[0, 0, 4:6] = 1.0   # blocks 1, 2 and 3 tie at score 1
+    k[0, 0, 6:8] = 1.0
+    q = np.ones((1, 1, 12, d))
+    kbar = oracle.block_compress(k, T)
+    idx, kth = oracle.block_select(q, kbar, T, 2, 1, 1)
+    assert list(idx[0, 0, 11]) == [0, 1, 2, 5, ]
+    assert kth[0, 0, 11] == 1.0
+
+
+def test_selection_worked_example():
+    g = json.load(open(os.path.join(GOLD, "sparse_scalar.json")))
+    k = np.array(g["k"], float).reshape(1, 1, -1, 1)
+    q = np.ones((1, 1, 8, 1)) * g["q7"]
+    kbar = oracle.block_compress(k, 2)
+    np.testing.assert_array_equal(kbar.ravel(), g["kbar"])
+    idx, _ = oracle.block_select(q, kbar, 2, 1, 1, 1)
+    assert list(idx[0, 0, 7]) == g["selection_pos7"]
+    v = np.array(g["v"], float).reshape(1, 1, -1, 1)
+    o = oracle.sparse_attention(q, k, v, idx, 2, scale=1.0)
+    t = g["o7_numerator_terms"]
+    e = math.exp(t["shifted_logit"])
+    expect = (t["plain_v_sum"] + e * t["shifted_v_sum"]) / (t["plain_count"] + e * t["shifted_count"])
+    assert abs(o[0, 0, 7, 0] - expect) < 1e-13
+
+
+def test_shifted_blocks_always_selected():
+    # Blocks whose keys carry +3u for a query direction u score ~ 3 G |u|^2, far above the
+    # noise; every such block that is a candidate must be chosen while <= topk are available.
+    rng = np.random.default_rng(41)
+    B, H, Hkv, T, d, N = 1, 8, 2, 8, 16, 8 * 40
+    G = H // Hkv
+    u = rng.standard_normal((Hkv, d))
+    k = rng.standard_normal((B, Hkv, N, d))
+    shifted = {0: [3, 9, 17, 30], 1: [5, 6, 25]}
+    for g, blks in shifted.items():
+        for blk in blks:
+            k[0, g, blk * T:(blk + 1) * T] += 3 * u[g]
+    q = rng.standard_normal((B, H, N, d)) + np.repeat(u, G, axis=0)[None, :, None, :]
+    kbar = oracle.block_compress(k, T)
+    topk, n_init, n_local = 5, 1, 2
+    idx, _ = oracle.block_select(q, kbar, T, topk, n_init, n_local)
+    for g, blks in shifted.items():
+        for r in range(N):
+            c = r // T
+            avail = [x for x in blks if n_init <= x <= c - n_local]
+            assert set(avail) <= set(idx[0, g, r]), (g, r)
+
+
+# ------------------------------------------------------------------------------ attention
+
+def _sdpa(q, k, v, scale):
+    qt, kt, vt = (torch.from_numpy(x) for x in (q, k, v))
+    G = q.shape[1] // k.shape[1]
+    kt = kt.repeat_interleave(G, dim=1)
+    vt = vt.repeat_interleave(G, dim=1)
+    return torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, is_causal=True,
+                                                            scale=scale).numpy()
+
+
+def test_dense_matches_torch_sdpa():
+    rng = np.random.default_rng(51)
+    B, H, Hkv, N, d = 2, 4, 2, 33, 8
+    q = rng.standard_normal((B, H, N, d))
+    k = rng.standard_normal((B, Hkv, N, d))
+    v = rng.standard_normal((B, Hkv, N, d))
+    o = oracle.dense_causal_attention(q, k, v)
+    np.testing.assert_allclose(o, _sdpa(q, k, v, 1 / math.sqrt(d)), rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("T,n_init,n_local", [(4, 1, 1), (4, 1, 2), (8, 2, 1)])
+def test_sparse_with_all_blocks_is_dense(T, n_init, n_local):
+    rng = np.random.default_rng(52 + T)
+    B, H, Hkv, N, d = 1, 6, 2, 9 * T + 2, 8
+    q = rng.standard_normal((B, H, N, d))
+    k = rng.standard_normal((B, Hkv, N, d))
+    v = rng.standard_normal((B, Hkv, N, d))
+    kbar = oracle.block_compress(k, T)
+    idx, _ = oracle.block_select(q, kbar, T, topk=N // T + 1, n_init=n_init, n_local=n_local)
+    o_sparse = oracle.sparse_attention(q, k, v, idx, T)
+    o_dense = oracle.dense_causal_attention(q, k, v)
+    np.testing.assert_allclose(o_sparse, o_dense, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(o_sparse, _sdpa(q, k, v, 1 / math.sqrt(d)), rtol=0, atol=1e-12)
+
+
+def test_equal_keys_give_mean_of_selected_values():
+    rng = np.random.default_rng(53)
+    T, N, d = 4, 24, 3
+    k = np.ones((1, 1, N, d))
+    v = rng.standard_normal((1, 1, N, d))
+    q = rng.standard_normal((1, 1, N, d))
+    idx = np.full((1, 1, N, 3), -1, dtype=np.int32)
+    for r in range(N):
+        c = r // T
+        idx[0, 0, r, :2] = sorted({0, c})
+        if c >= 3:
+            idx[0, 0, r, :3] = [0, 2, c]
+    o = oracle.sparse_attention(q, k, v, idx, T)
+    for r in range(N):
+        J = [j for blk in set(x for x in idx[0, 0, r] if x >= 0)
+             for j in range(blk * T, (blk + 1) * T) if j <= r]
+        np.testing.assert_allclose(o[0, 0, r], v[0, 0, J].mean(axis=0), rtol=0, atol=1e-13)
+    np.testing.assert_allclose(o[0, 0, 0], v[0, 0, 0], rtol=0, atol=0)
+
+
+def test_sparse_rows_subset_and_empty_selection():
+    rng = np.random.default_rng(54)
+    B, H, Hkv, N, d, T = 1, 4, 2, 20, 4, 4
+    q = rng.standard_normal((B, H, N, d))
+    k = rng.standard_normal((B, Hkv, N, d))
+    v = rng.standard_normal((B, Hkv, N, d))
+    kbar = oracle.block_compress(k, T)
+    idx, _ = oracle.block_select(q, kbar, T, 1, 1, 1)
+    full = oracle.sparse_attention(q, k, v, idx, T)
+    rows = np.array([[0, 0], [3, 19], [2, 7]])
+    sub = oracle.sparse_attention(q, k, v, idx, T, rows=rows)
+    for n, (bh, r) in enumerate(rows):
+        np.testing.assert_array_equal(sub[n], full[0, bh, r])
+    empty = np.full_like(idx, -1)
+    assert np.all(oracle.sparse_attention(q, k, v, empty, T) == 0.0)
