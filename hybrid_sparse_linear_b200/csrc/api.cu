@@ -1,0 +1,338 @@
+// C ABI of libsala: host-side validation, dispatch to the kernels, and the status word.
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <atomic>
+#include <mutex>
+
+#include "../../include/sala.h"
+#include "kernels.h"
+
+namespace {
+
+// Per-device status word: kernels atomicOr fault bits into it; sala_check_status reads and
+// clears it.  It is the library's only global device state.
+__device__ unsigned g_status_word;
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+unsigned* g_status_ptr[kMaxDevices] = {};
+std::atomic<unsigned long long> g_wait_limit_ns{2000000000ull};
+thread_local char g_err[512] = "";
+
+sala_status fail(sala_status s, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof(g_err), fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+// Device context of the current device (address of its status word, wait limit).
+sala_status get_ctx(sala::DevCtx* ctx) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(SALA_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    if (dev < 0 || dev >= kMaxDevices) return fail(SALA_ERR_UNSUPPORTED, "device index %d", dev);
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_status_ptr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_status_word);
+        if (e != cudaSuccess)
+            return fail(SALA_ERR_CUDA, "cudaGetSymbolAddress(status): %s", cudaGetErrorString(e));
+        g_status_ptr[dev] = static_cast<unsigned*>(p);
+    }
+    ctx->status = g_status_ptr[dev];
+    ctx->wait_limit_ns = g_wait_limit_ns.load();
+    return SALA_OK;
+}
+
+sala_status launched(cudaError_t e, const char* what) {
+    if (e != cudaSuccess) return fail(SALA_ERR_CUDA, "%s launch: %s", what, cudaGetErrorString(e));
+    g_err[0] = 0;
+    return SALA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+#define REQUIRE(cond, code, ...) \
+    do {                         \
+        if (!(cond)) return fail(code, __VA_ARGS__); \
+    } while (0)
+
+#define REQ_PTR(p) REQUIRE((p) != nullptr && aligned16(p), SALA_ERR_INVALID_ARG, \
+                           "%s must be a non-NULL 16-byte aligned device pointer", #p)
+
+sala::DType to_dt(sala_dtype dt) { return dt == SALA_BF16 ? sala::DType::BF16 : sala::DType::F32; }
+
+}  // namespace
+
+extern "C" {
+
+int sala_version(void) { return 100; }
+
+const char* sala_status_string(sala_status s) {
+    switch (s) {
+        case SALA_OK: return "SALA_OK";
+        case SALA_ERR_INVALID_ARG: return "SALA_ERR_INVALID_ARG";
+        case SALA_ERR_UNSUPPORTED: return "SALA_ERR_UNSUPPORTED";
+        case SALA_ERR_CUDA: return "SALA_ERR_CUDA";
+        case SALA_ERR_TIMEOUT: return "SALA_ERR_TIMEOUT";
+        case SALA_ERR_BOUNDS: return "SALA_ERR_BOUNDS";
+    }
+    return "SALA_ERR_UNKNOWN";
+}
+
+const char* sala_last_error(void) { return g_err; }
+
+void sala_set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns.store(ns ? ns : 1); }
+
+sala_status sala_check_status(sala_stream stream) {
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail(SALA_ERR_CUDA, "stream sync: %s", cudaGetErrorString(e));
+    sala::DevCtx ctx;
+    sala_status s = get_ctx(&ctx);
+    if (s != SALA_OK) return s;
+    unsigned word = 0;
+    e = cudaMemcpy(&word, ctx.status, sizeof(word), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return fail(SALA_ERR_CUDA, "status read: %s", cudaGetErrorString(e));
+    if (word) {
+        const unsigned zero = 0;
+        e = cudaMemcpy(ctx.status, &zero, sizeof(zero), cudaMemcpyHostToDevice);
+        if (e != cudaSuccess) return fail(SALA_ERR_CUDA, "status clear: %s", cudaGetErrorString(e));
+    }
+    if (word & sala::kStatusTimeout) return fail(SALA_ERR_TIMEOUT, "a device-side wait expired");
+    if (word & sala::kStatusBounds) return fail(SALA_ERR_BOUNDS, "a device-side index was out of range");
+    g_err[0] = 0;
+    return SALA_OK;
+}
+
+sala_status sala_selftest_wait_timeout(sala_stream stream) {
+    sala::DevCtx ctx;
+    sala_status s = get_ctx(&ctx);
+    if (s != SALA_OK) return s;
+    return launched(sala::launch_selftest_wait(static_cast<cudaStream_t>(stream), ctx), "selftest");
+}
+
+// ----------------------------------------------------------------------------------------------
+sala_status sala_linear_prefill(const void* q, const void* k, const void* v, const float* decay,
+                                void* o, const float* state_in, float* state_out, int B, int H,
+                                int N, int d, int chunk, sala_dtype dt, sala_stream stream) {
+    REQUIRE(B >= 0 && H >= 0 && N >= 0, SALA_ERR_INVALID_ARG, "negative size (B=%d H=%d N=%d)", B, H, N);
+    REQUIRE(dt == SALA_F32 || dt == SALA_BF16, SALA_ERR_INVALID_ARG, "unknown dtype %d", (int)dt);
+    REQUIRE(d == 64 || d == 128, SALA_ERR_UNSUPPORTED, "head dim %d (supported: 64, 128)", d);
+    REQUIRE(chunk == 0 || chunk == 64, SALA_ERR_UNSUPPORTED, "chunk %d (supported: 0, 64)", chunk);
+    if (B == 0 || H == 0) return SALA_OK;
+    REQUIRE(decay != nullptr, SALA_ERR_INVALID_ARG, "decay must be a device pointer");
+    if (state_in) REQUIRE(aligned16(state_in), SALA_ERR_INVALID_ARG, "state_in must be 16-byte aligned");
+    if (state_out) REQUIRE(aligned16(state_out), SALA_ERR_INVALID_ARG, "state_out must be 16-byte aligned");
+    if (N > 0) {
+        REQ_PTR(q); REQ_PTR(k); REQ_PTR(v); REQ_PTR(o);
+    }
+    sala::DevCtx ctx;
+    sala_status s = get_ctx(&ctx);
+    if (s != SALA_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (dt == SALA_BF16 && N > 0 && sala::linear_prefill_tc_supported(d))
+        return launched(sala::launch_linear_prefill_tc(q, k, v, decay, o, state_in, state_out, B,
+                                                       H, N, d, st, ctx), "linear_prefill_tc");
+    return launched(sala::launch_linear_prefill_simt(to_dt(dt), q, k, v, decay, o, state_in,
+                                                     state_out, B, H, N, d, st, ctx),
+                    "linear_prefill");
+}
+
+sala_status sala_linear_decode(const void* q, const void* k, const void* v, const float* decay,
+                               float* state, void* o, int B, int H, int d, sala_dtype dt,
+                               sala_stream stream) {
+    REQUIRE(B >= 0 && H >= 0, SALA_ERR_INVALID_ARG, "negative size (B=%d H=%d)", B, H);
+    REQUIRE(dt == SALA_F32 || dt == SALA_BF16, SALA_ERR_INVALID_ARG, "unknown dtype %d", (int)dt);
+    REQUIRE(d == 64 || d == 128, SALA_ERR_UNSUPPORTED, "head dim %d (supported: 64, 128)", d);
+    if (B == 0 || H == 0) return SALA_OK;
+    REQ_PTR(q); REQ_PTR(k); REQ_PTR(v); REQ_PTR(o); REQ_PTR(state);
+    REQUIRE(decay != nullptr, SALA_ERR_INVALID_ARG, "decay must be a device pointer");
+    sala::DevCtx ctx;
+    sala_status s = get_ctx(&ctx);
+    if (s != SALA_OK) return s;
+    return launched(sala::launch_linear_decode(to_dt(dt), q, k, v, decay, state, o, B, H, d,
+                                               static_cast<cudaStream_t>(stream), ctx),
+                    "linear_decode");
+}
+
+// ----------------------------------------------------------------------------------------------
+sala_status sala_block_compress(const void* k, void* kbar, int B, int Hkv, int N, int d,
+                                int block, int first_block, int n_blocks, int nb_cap,
+                                sala_dtype dt, sala_stream stream) {
+    REQUIRE(B >= 0 && Hkv >= 0 && N >= 0 && first_block >= 0 && n_blocks >= 0,
+            SALA_ERR_INVALID_ARG, "negative size or block range");
+    REQUIRE(dt == SALA_F32 || dt == SALA_BF16, SALA_ERR_INVALID_ARG, "unknown dtype %d", (int)dt);
+    REQUIRE(d == 64 || d == 128, SALA_ERR_UNSUPPORTED, "head dim %d (supported: 64, 128)", d);
+    REQUIRE(block == 64, SALA_ERR_UNSUPPORTED, "block %d (supported: 64)", block);
+    REQUIRE((int64_t)(first_block + (int64_t)n_blocks) * block <= N, SALA_ERR_INVALID_ARG,
+            "blocks %d..%d are not complete within N=%d", first_block, first_block + n_blocks - 1, N);
+    REQUIRE(nb_cap >= first_block + n_blocks, SALA_ERR_INVALID_ARG,
+            "nb_cap %d < first_block + n_blocks = %d", nb_cap, first_block + n_blocks);
+    if (B == 0 || Hkv == 0 || n_blocks == 0) return SALA_OK;
+    REQ_PTR(k); REQ_PTR(kbar);
+    sala::DevCtx ctx;
+    sala_status s = get_ctx(&ctx);
+    if (s != SALA_OK) return s;
+    return launched(sala::launch_block_compress(to_dt(dt), k, kbar, B, Hkv, N, d, first_block,
+                                                n_blocks, nb_cap, static_cast<cudaStream_t>(stream),
+                                                ctx),
+                    "block_compress");
+}
+
+static sala_status check_select_args(int B, int H, int Hkv, int Nq, int q_pos0, int nb, int d,
+                                     int block, int topk, int n_init, int n_local,
+                                     sala_dtype dt) {
+    REQUIRE(B >= 0 && H >= 0 && Hkv > 0 && Nq >= 0 && q_pos0 >= 0 && nb >= 0,
+            SALA_ERR_INVALID_ARG, "bad sizes (B=%d H=%d Hkv=%d Nq=%d q_pos0=%d nb=%d)", B, H, Hkv,
+            Nq, q_pos0, nb);
+    REQUIRE(H % Hkv == 0, SALA_ERR_INVALID_ARG, "H=%d is not a multiple of Hkv=%d", H, Hkv);
+    REQUIRE(dt == SALA_F32 || dt == SALA_BF16, SALA_ERR_INVALID_ARG, "unknown dtype %d", (int)dt);
+    REQUIRE(d == 64 || d == 128, SALA_ERR_UNSUPPORTED, "head dim %d (supported: 64, 128)", d);
+    REQUIRE(block == 64, SALA_ERR_UNSUPPORTED, "block %d (supported: 64)", block);
+    REQUIRE(topk >= 0 && n_init >= 0 && n_local >= 1, SALA_ERR_INVALID_ARG,
+            "need topk >= 0, n_init >= 0, n_local >= 1");
+    REQUIRE(n_init + n_local + topk <= 1024, SALA_ERR_UNSUPPORTED, "more than 1024 slots");
+    if (Nq > 0 && B > 0) {
+        const int64_t last_pos = (int64_t)q_pos0 + Nq - 1;
+        const int64_t last_c = last_pos / block;
+        const int64_t need = last_c - n_local + 1;  // blocks 0 .. c - n_local must be compressed
+        REQUIRE(need <= nb, SALA_ERR_INVALID_ARG,
+                "kbar holds %d blocks but the last query (position %lld) needs %lld", nb,
+                (long long)last_pos, (long long)need);
+        const int64_t max_cand = last_c - n_local + 1 - n_init;
+        REQUIRE(topk <= 64 || max_cand <= topk, SALA_ERR_UNSUPPORTED,
+                "topk %d > 64 with up to %lld candidates", topk, (long long)max_cand);
+    }
+    return SALA_OK;
+}
+
+size_t sala_block_topk_workspace(int B, int Hkv, int Nq, int q_pos0, int nb, int block, int topk) {
+    (void)nb; (void)block;
+    if (B <= 0 || Hkv <= 0 || Nq <= 0) return 0;
+    if (Nq > 16) return 0;  // tiled path needs no scratch
+    return sala::rowwise_topk_workspace(B, Hkv, Nq, q_pos0, topk);
+}
+
+sala_status sala_block_topk(const void* q, const void* kbar, int32_t* idx, int B, int H, int Hkv,
+                            int Nq, int q_pos0, int nb, int d, int block, int topk, int n_init,
+                            int n_local, void* workspace, size_t workspace_bytes, sala_dtype dt,
+                            sala_stream stream) {
+    sala_status s = check_select_args(B, H, Hkv, Nq, q_pos0, nb, d, block, topk, n_init, n_local, dt);
+    if (s != SALA_OK) return s;
+    if (B == 0 || H == 0 || Nq == 0) return SALA_OK;
+    REQ_PTR(q); REQUIRE(idx != nullptr, SALA_ERR_INVALID_ARG, "idx must be a device pointer");
+    if (nb > 0) REQ_PTR(kbar);
+    sala::DevCtx ctx;
+    s = get_ctx(&ctx);
+    if (s != SALA_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const size_t need = sala_block_topk_workspace(B, Hkv, Nq, q_pos0, nb, block, topk);
+    if (need > 0) {
+        REQUIRE(workspace != nullptr && workspace_bytes >= need && aligned16(workspace),
+                SALA_ERR_INVALID_ARG, "workspace of %zu bytes (16-byte aligned) required, got %zu",
+                need, workspace_bytes);
+        return launched(sala::launch_block_topk_rowwise(to_dt(dt), q, kbar, idx, B, H, Hkv, Nq,
+                                                        q_pos0, nb, d, topk, n_init, n_local,
+                                                        workspace, st, ctx),
+                        "block_topk_rowwise");
+    }
+    return launched(sala::launch_block_topk_tiled(to_dt(dt), q, kbar, idx, B, H, Hkv, Nq, q_pos0,
+                                                  nb, d, topk, n_init, n_local, st, ctx),
+                    "block_topk");
+}
+
+// ----------------------------------------------------------------------------------------------
+sala_status sala_sparse_prefill(const void* q, const void* k, const void* v, const int32_t* idx,
+                                void* o, int B, int H, int Hkv, int N, int d, int block,
+                                int slots, float scale, sala_dtype dt, sala_stream stream) {
+    REQUIRE(B >= 0 && H >= 0 && Hkv > 0 && N >= 0 && slots >= 1, SALA_ERR_INVALID_ARG,
+            "bad sizes (B=%d H=%d Hkv=%d N=%d slots=%d)", B, H, Hkv, N, slots);
+    REQUIRE(H % Hkv == 0, SALA_ERR_INVALID_ARG, "H=%d is not a multiple of Hkv=%d", H, Hkv);
+    REQUIRE(dt == SALA_F32 || dt == SALA_BF16, SALA_ERR_INVALID_ARG, "unknown dtype %d", (int)dt);
+    REQUIRE(d == 64 || d == 128, SALA_ERR_UNSUPPORTED, "head dim %d (supported: 64, 128)", d);
+    REQUIRE(block == 64, SALA_ERR_UNSUPPORTED, "block %d (supported: 64)", block);
+    REQUIRE(slots <= 1024, SALA_ERR_UNSUPPORTED, "more than 1024 slots");
+    REQUIRE(isfinite(scale) && scale >= 0.f, SALA_ERR_INVALID_ARG, "scale must be finite and >= 0");
+    if (B == 0 || H == 0 || N == 0) return SALA_OK;
+    REQ_PTR(q); REQ_PTR(k); REQ_PTR(v); REQ_PTR(o);
+    REQUIRE(idx != nullptr, SALA_ERR_INVALID_ARG, "idx must be a device pointer");
+    if (scale == 0.f) scale = 1.0f / sqrtf((float)d);
+    sala::DevCtx ctx;
+    sala_status s = get_ctx(&ctx);
+    if (s != SALA_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (dt == SALA_BF16 && sala::sparse_prefill_tc_supported(H, Hkv, d))
+        return launched(sala::launch_sparse_prefill_tc(q, k, v, idx, o, B, H, Hkv, N, d, slots,
+                                                       scale, st, ctx), "sparse_prefill_tc");
+    return launched(sala::launch_sparse_prefill_simt(to_dt(dt), q, k, v, idx, o, B, H, Hkv, N, d,
+                                                     slots, scale, st, ctx),
+                    "sparse_prefill");
+}
+
+size_t sala_sparse_decode_workspace(int B, int H, int Hkv, int pos, int block, int topk,
+                                    int n_init, int n_local, int d) {
+    if (B <= 0 || H <= 0 || Hkv <= 0 || pos < 0 || block <= 0) return 0;
+    const int slots = n_init + n_local + topk;
+    size_t a = sala::sparse_decode_attn_workspace(B, H, Hkv, slots, d);
+    size_t sel = sala::rowwise_topk_workspace(B, Hkv, 1, pos, topk);
+    size_t idx_bytes = (size_t)B * Hkv * slots * sizeof(int32_t);
+    auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    return up(a) + up(sel) + up(idx_bytes);
+}
+
+sala_status sala_sparse_decode(const void* q, const void* kcache, const void* vcache,
+                               const void* kbar, const int32_t* idx_in, int32_t* idx_out, void* o,
+                               int B, int H, int Hkv, int pos, int Tmax, int nb_cap, int d,
+                               int block, int topk, int n_init, int n_local, float scale,
+                               void* workspace, size_t workspace_bytes, sala_dtype dt,
+                               sala_stream stream) {
+    REQUIRE(pos >= 0 && pos < Tmax, SALA_ERR_INVALID_ARG, "pos %d outside the cache (Tmax %d)", pos, Tmax);
+    sala_status s = check_select_args(B, H, Hkv, 1, pos, nb_cap, d, block, topk, n_init,
+                                      n_local, dt);
+    if (s != SALA_OK) return s;
+    REQUIRE(isfinite(scale) && scale >= 0.f, SALA_ERR_INVALID_ARG, "scale must be finite and >= 0");
+    if (B == 0 || H == 0) return SALA_OK;
+    REQ_PTR(q); REQ_PTR(kcache); REQ_PTR(vcache); REQ_PTR(o);
+    if (!idx_in && nb_cap > 0) REQ_PTR(kbar);
+    const size_t need = sala_sparse_decode_workspace(B, H, Hkv, pos, block, topk, n_init, n_local, d);
+    REQUIRE(workspace != nullptr && aligned16(workspace) && workspace_bytes >= need,
+            SALA_ERR_INVALID_ARG, "workspace of %zu bytes (16-byte aligned) required, got %zu",
+            need, workspace_bytes);
+    if (scale == 0.f) scale = 1.0f / sqrtf((float)d);
+    sala::DevCtx ctx;
+    s = get_ctx(&ctx);
+    if (s != SALA_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int slots = n_init + n_local + topk;
+    auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    char* w = static_cast<char*>(workspace);
+    void* ws_attn = w;
+    w += up(sala::sparse_decode_attn_workspace(B, H, Hkv, slots, d));
+    void* ws_sel = w;
+    w += up(sala::rowwise_topk_workspace(B, Hkv, 1, pos, topk));
+    int32_t* idx_ws = reinterpret_cast<int32_t*>(w);
+    const int32_t* idx_use = idx_in;
+    if (!idx_in) {
+        int32_t* dst = idx_out ? idx_out : idx_ws;
+        cudaError_t e = sala::launch_block_topk_rowwise(to_dt(dt), q, kbar, dst, B, H, Hkv, 1, pos,
+                                                        nb_cap, d, topk, n_init, n_local, ws_sel,
+                                                        st, ctx);
+        if (e != cudaSuccess) return launched(e, "sparse_decode select");
+        idx_use = dst;
+    } else if (idx_out) {
+        cudaError_t e = cudaMemcpyAsync(idx_out, idx_in, (size_t)B * Hkv * slots * sizeof(int32_t),
+                                        cudaMemcpyDeviceToDevice, st);
+        if (e != cudaSuccess) return launched(e, "sparse_decode idx copy");
+    }
+    return launched(sala::launch_sparse_decode_attn(to_dt(dt), q, kcache, vcache, idx_use, o, B, H,
+                                                    Hkv, pos, Tmax, d, slots, scale, ws_attn, st,
+                                                    ctx),
+                    "sparse_decode");
+}
+
+}  // extern "C"

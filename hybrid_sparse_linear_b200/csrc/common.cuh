@@ -1,0 +1,65 @@
+// Internal helpers shared by the CUDA kernels of libsala (not part of the C ABI).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace sala {
+
+// Bits of the per-device status word (read and cleared by sala_check_status).
+enum : unsigned { kStatusTimeout = 1u, kStatusBounds = 2u };
+
+// Passed by value to every kernel: where to record device-side faults, and how long a bounded
+// wait may spin before it gives up.
+struct DevCtx {
+    unsigned* status;
+    unsigned long long wait_limit_ns;
+};
+
+__device__ __forceinline__ void flag(const DevCtx& c, unsigned bits) { atomicOr(c.status, bits); }
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ float to_f(float x) { return x; }
+__device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T> __device__ __forceinline__ T from_f(float x);
+template <> __device__ __forceinline__ float from_f<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) {
+    return __float2bfloat16_rn(x);
+}
+
+// Correct rounding of an fp64 value to the element type: fp32 directly (round to nearest
+// even); bf16 through round-to-odd at fp32 followed by round-to-nearest-even at bf16, which is
+// exact-once rounding because fp32 carries more than two extra bits (Boldo & Melquiond,
+// "Emulation of FMA and correctly rounded sums: proved algorithms using rounding to odd").
+template <typename T> __device__ __forceinline__ T round_from_double(double x);
+template <> __device__ __forceinline__ float round_from_double<float>(double x) {
+    return __double2float_rn(x);
+}
+template <> __device__ __forceinline__ __nv_bfloat16 round_from_double<__nv_bfloat16>(double x) {
+    float f = __double2float_rz(x);
+    if ((double)f != x) f = __uint_as_float(__float_as_uint(f) | 1u);
+    return __float2bfloat16_rn(f);
+}
+
+// Monotone map of fp32 to uint32 (larger float -> larger integer).
+__device__ __forceinline__ uint32_t orderable(float s) {
+    uint32_t u = __float_as_uint(s);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Selection key: higher score first, then lower block index.  Key 0 means "empty".
+__device__ __forceinline__ uint64_t sel_key(float score, int blk) {
+    return ((uint64_t)orderable(score) << 32) | (uint32_t)(~(uint32_t)blk);
+}
+__device__ __forceinline__ int key_block(uint64_t key) { return (int)(~(uint32_t)(key & 0xffffffffu)); }
+
+__host__ __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+}  // namespace sala

@@ -1,0 +1,61 @@
+// Internal launchers of libsala.  Each returns the CUDA error of its launch(es).  Arguments are
+// validated by api.cu before any of these is called.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace sala {
+
+enum class DType { F32 = 0, BF16 = 1 };
+
+// Linear attention.
+cudaError_t launch_linear_prefill_simt(DType dt, const void* q, const void* k, const void* v,
+                                       const float* decay, void* o, const float* s_in,
+                                       float* s_out, int B, int H, int N, int d,
+                                       cudaStream_t st, DevCtx ctx);
+cudaError_t launch_linear_prefill_tc(const void* q, const void* k, const void* v,
+                                     const float* decay, void* o, const float* s_in,
+                                     float* s_out, int B, int H, int N, int d, cudaStream_t st,
+                                     DevCtx ctx);
+bool linear_prefill_tc_supported(int d);
+cudaError_t launch_linear_decode(DType dt, const void* q, const void* k, const void* v,
+                                 const float* decay, float* state, void* o, int B, int H, int d,
+                                 cudaStream_t st, DevCtx ctx);
+
+// Sparse attention.
+cudaError_t launch_block_compress(DType dt, const void* k, void* kbar, int B, int Hkv, int N,
+                                  int d, int first_block, int n_blocks, int nb_cap,
+                                  cudaStream_t st, DevCtx ctx);
+cudaError_t launch_block_topk_tiled(DType dt, const void* q, const void* kbar, int32_t* idx,
+                                    int B, int H, int Hkv, int Nq, int q_pos0, int nb, int d,
+                                    int topk, int n_init, int n_local, cudaStream_t st,
+                                    DevCtx ctx);
+// Row-wise selection for few query rows and many blocks: candidates split across CTAs, then a
+// merge.  Workspace = rowwise_topk_workspace(...) bytes.
+size_t rowwise_topk_workspace(int B, int Hkv, int Nq, int q_pos0, int topk);
+cudaError_t launch_block_topk_rowwise(DType dt, const void* q, const void* kbar, int32_t* idx,
+                                      int B, int H, int Hkv, int Nq, int q_pos0, int nb, int d,
+                                      int topk, int n_init, int n_local, void* ws,
+                                      cudaStream_t st, DevCtx ctx);
+cudaError_t launch_sparse_prefill_simt(DType dt, const void* q, const void* k, const void* v,
+                                       const int32_t* idx, void* o, int B, int H, int Hkv, int N,
+                                       int d, int slots, float scale, cudaStream_t st,
+                                       DevCtx ctx);
+cudaError_t launch_sparse_prefill_tc(const void* q, const void* k, const void* v,
+                                     const int32_t* idx, void* o, int B, int H, int Hkv, int N,
+                                     int d, int slots, float scale, cudaStream_t st, DevCtx ctx);
+bool sparse_prefill_tc_supported(int H, int Hkv, int d);
+size_t sparse_decode_attn_workspace(int B, int H, int Hkv, int slots, int d);
+cudaError_t launch_sparse_decode_attn(DType dt, const void* q, const void* kc, const void* vc,
+                                      const int32_t* idx, void* o, int B, int H, int Hkv,
+                                      int pos, int Tmax, int d, int slots, float scale, void* ws,
+                                      cudaStream_t st, DevCtx ctx);
+
+// Diagnostics.
+cudaError_t launch_selftest_wait(cudaStream_t st, DevCtx ctx);
+
+}  // namespace sala

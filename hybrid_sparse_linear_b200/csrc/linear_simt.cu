@@ -1,0 +1,227 @@
+// Linear (Lightning-style) attention on CUDA cores: the fp32 prefill and the decode step.
+//
+// Prefill is the chunked form of o_i = sum_{j<=i} lambda^{i-j} (q_i.k_j) v_j: per chunk of C
+// rows, an intra-chunk decay-masked product plus the carried d x d state.  One CTA owns one
+// (batch, head, slice of DV value columns) and walks the chunks in order; S[:, slice] evolves
+// independently of the other slices, so slices run in parallel with no communication.
+#include "kernels.h"
+
+namespace sala {
+namespace {
+
+constexpr int kC = 64;        // chunk rows
+constexpr int kThreads = 256;
+
+template <int D, int DV>
+struct PrefillSmem {
+    static constexpr int kQK = kC * (D + 1);
+    static constexpr size_t bytes =
+        sizeof(float) * (2 * kQK + kC * DV + kC * (kC + 1) + D * DV + (kC + 1));
+};
+
+template <typename T, int D, int DV>
+__global__ void __launch_bounds__(kThreads)
+linear_prefill_simt_kernel(const T* __restrict__ q, const T* __restrict__ k,
+                           const T* __restrict__ v, const float* __restrict__ decay,
+                           T* __restrict__ o, const float* s_in, float* s_out, int H, int N) {
+    extern __shared__ float sm[];
+    float* Qs = sm;                         // [C][D+1]
+    float* Ks = Qs + kC * (D + 1);          // [C][D+1]
+    float* Vs = Ks + kC * (D + 1);          // [C][DV]
+    float* As = Vs + kC * DV;               // [C][C+1]
+    float* Ss = As + kC * (kC + 1);         // [D][DV]  state slice
+    float* pw = Ss + D * DV;                // [C+1]    lambda^n
+
+    const int tid = threadIdx.x;
+    const int c0 = blockIdx.x * DV;         // first value column of this slice
+    const int64_t bh = blockIdx.y;
+    const int h = (int)(bh % H);
+    const float lam = decay[h];
+    for (int n = tid; n <= kC; n += kThreads) pw[n] = (float)pow((double)lam, (double)n);
+    for (int e = tid; e < D * DV; e += kThreads) {
+        const int a = e / DV, c = e % DV;
+        Ss[e] = s_in ? s_in[(bh * D + a) * D + c0 + c] : 0.f;
+    }
+    const T* qb = q + bh * (int64_t)N * D;
+    const T* kb = k + bh * (int64_t)N * D;
+    const T* vb = v + bh * (int64_t)N * D;
+    T* ob = o + bh * (int64_t)N * D;
+
+    for (int r0 = 0; r0 < N; r0 += kC) {
+        const int len = min(kC, N - r0);
+        __syncthreads();
+        for (int e = tid; e < kC * D; e += kThreads) {
+            const int t = e / D, a = e % D;
+            const bool ok = t < len;
+            Qs[t * (D + 1) + a] = ok ? to_f(qb[(int64_t)(r0 + t) * D + a]) : 0.f;
+            Ks[t * (D + 1) + a] = ok ? to_f(kb[(int64_t)(r0 + t) * D + a]) : 0.f;
+        }
+        for (int e = tid; e < kC * DV; e += kThreads) {
+            const int t = e / DV, c = e % DV;
+            Vs[e] = t < len ? to_f(vb[(int64_t)(r0 + t) * D + c0 + c]) : 0.f;
+        }
+        __syncthreads();
+        // Intra-chunk scores, decay-masked: A[t][s] = lambda^{t-s} q_t.k_s for s <= t.
+        {
+            const int t = tid >> 2;
+            for (int m = 0; m < kC / 4; ++m) {
+                const int s = (tid & 3) + 4 * m;
+                float acc = 0.f;
+                if (s <= t) {
+                    const float* qr = Qs + t * (D + 1);
+                    const float* kr = Ks + s * (D + 1);
+#pragma unroll 8
+                    for (int a = 0; a < D; ++a) acc = fmaf(qr[a], kr[a], acc);
+                    acc *= pw[t - s];
+                }
+                As[t * (kC + 1) + s] = acc;
+            }
+        }
+        __syncthreads();
+        // o_t = A[t,:] V + lambda^{t+1} q_t S.
+        {
+            const int t = tid >> 2;
+            if (t < len) {
+                for (int m = 0; m < DV / 4; ++m) {
+                    const int c = (tid & 3) + 4 * m;
+                    float intra = 0.f, inter = 0.f;
+                    for (int s = 0; s <= t; ++s) intra = fmaf(As[t * (kC + 1) + s], Vs[s * DV + c], intra);
+                    const float* qr = Qs + t * (D + 1);
+#pragma unroll 8
+                    for (int a = 0; a < D; ++a) inter = fmaf(qr[a], Ss[a * DV + c], inter);
+                    ob[(int64_t)(r0 + t) * D + c0 + c] = from_f<T>(intra + pw[t + 1] * inter);
+                }
+            }
+        }
+        __syncthreads();
+        // S <- lambda^len S + sum_s lambda^{len-1-s} k_s^T v_s.
+        {
+            constexpr int kPer = D * DV / kThreads;
+            const int a = (tid * kPer) / DV;
+            const int cb = (tid * kPer) % DV;
+            float acc[kPer];
+#pragma unroll
+            for (int j = 0; j < kPer; ++j) acc[j] = pw[len] * Ss[a * DV + cb + j];
+            for (int s = 0; s < len; ++s) {
+                const float w = pw[len - 1 - s] * Ks[s * (D + 1) + a];
+#pragma unroll
+                for (int j = 0; j < kPer; ++j) acc[j] = fmaf(w, Vs[s * DV + cb + j], acc[j]);
+            }
+#pragma unroll
+            for (int j = 0; j < kPer; ++j) Ss[a * DV + cb + j] = acc[j];
+        }
+    }
+    __syncthreads();
+    if (s_out)
+        for (int e = tid; e < D * DV; e += kThreads) {
+            const int a = e / DV, c = e % DV;
+            s_out[(bh * D + a) * D + c0 + c] = Ss[e];
+        }
+}
+
+template <typename T, int D>
+cudaError_t prefill_simt(const void* q, const void* k, const void* v, const float* decay, void* o,
+                         const float* s_in, float* s_out, int B, int H, int N, cudaStream_t st) {
+    constexpr int DV = 32;
+    auto kern = linear_prefill_simt_kernel<T, D, DV>;
+    const size_t smem = PrefillSmem<D, DV>::bytes;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid(D / DV, (unsigned)(B * H));
+    kern<<<grid, kThreads, smem, st>>>(static_cast<const T*>(q), static_cast<const T*>(k),
+                                       static_cast<const T*>(v), decay, static_cast<T*>(o), s_in,
+                                       s_out, H, N);
+    return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------------------------
+// Decode: S <- lambda S + k^T v ; o = q S.  One CTA per (batch*head, 16-column slice); thread
+// (a, half) owns row a of the slice, 8 columns, loaded and stored as two float4.
+template <typename T, int D>
+__global__ void __launch_bounds__(2 * D)
+linear_decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
+                     const float* __restrict__ decay, float* __restrict__ state,
+                     T* __restrict__ o, int H) {
+    constexpr int kCols = 16;
+    constexpr int kWarps = 2 * D / 32;
+    __shared__ float red[kWarps][kCols];
+    const int tid = threadIdx.x;
+    const int a = tid >> 1, half = tid & 1;
+    const int64_t bh = blockIdx.y;
+    const int c0 = blockIdx.x * kCols + half * 8;
+    const float lam = decay[bh % H];
+    const float ka = to_f(k[bh * D + a]);
+    const float qa = to_f(q[bh * D + a]);
+    float vv[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) vv[j] = to_f(v[bh * D + c0 + j]);
+    float4* row = reinterpret_cast<float4*>(state + (bh * D + a) * D + c0);
+    float4 s0 = row[0], s1 = row[1];
+    float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+    float part[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        sv[j] = fmaf(lam, sv[j], ka * vv[j]);
+        part[j] = qa * sv[j];
+    }
+    row[0] = make_float4(sv[0], sv[1], sv[2], sv[3]);
+    row[1] = make_float4(sv[4], sv[5], sv[6], sv[7]);
+    // Sum part[] over the 16 rows of this warp that share `half`, then over warps.
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+        for (int off = 2; off < 32; off <<= 1) part[j] += __shfl_xor_sync(0xffffffffu, part[j], off);
+    const int lane = tid & 31, w = tid >> 5;
+    if (lane < 2)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) red[w][lane * 8 + j] = part[j];
+    __syncthreads();
+    if (tid < kCols) {
+        float acc = 0.f;
+#pragma unroll
+        for (int ww = 0; ww < kWarps; ++ww) acc += red[ww][tid];
+        o[bh * D + blockIdx.x * kCols + tid] = from_f<T>(acc);
+    }
+}
+
+template <typename T, int D>
+cudaError_t decode_launch(const void* q, const void* k, const void* v, const float* decay,
+                          float* state, void* o, int B, int H, cudaStream_t st) {
+    dim3 grid(D / 16, (unsigned)(B * H));
+    linear_decode_kernel<T, D><<<grid, 2 * D, 0, st>>>(
+        static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), decay,
+        state, static_cast<T*>(o), H);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_linear_prefill_simt(DType dt, const void* q, const void* k, const void* v,
+                                       const float* decay, void* o, const float* s_in,
+                                       float* s_out, int B, int H, int N, int d, cudaStream_t st,
+                                       DevCtx) {
+    if (N == 0) {
+        // Nothing to attend to: the state passes through unchanged (or stays zero).
+        if (!s_out) return cudaSuccess;
+        const size_t bytes = (size_t)B * H * d * d * sizeof(float);
+        if (s_in) return s_in == s_out ? cudaSuccess
+                                       : cudaMemcpyAsync(s_out, s_in, bytes, cudaMemcpyDeviceToDevice, st);
+        return cudaMemsetAsync(s_out, 0, bytes, st);
+    }
+    if (dt == DType::F32)
+        return d == 64 ? prefill_simt<float, 64>(q, k, v, decay, o, s_in, s_out, B, H, N, st)
+                       : prefill_simt<float, 128>(q, k, v, decay, o, s_in, s_out, B, H, N, st);
+    return d == 64 ? prefill_simt<__nv_bfloat16, 64>(q, k, v, decay, o, s_in, s_out, B, H, N, st)
+                   : prefill_simt<__nv_bfloat16, 128>(q, k, v, decay, o, s_in, s_out, B, H, N, st);
+}
+
+cudaError_t launch_linear_decode(DType dt, const void* q, const void* k, const void* v,
+                                 const float* decay, float* state, void* o, int B, int H, int d,
+                                 cudaStream_t st, DevCtx) {
+    if (dt == DType::F32)
+        return d == 64 ? decode_launch<float, 64>(q, k, v, decay, state, o, B, H, st)
+                       : decode_launch<float, 128>(q, k, v, decay, state, o, B, H, st);
+    return d == 64 ? decode_launch<__nv_bfloat16, 64>(q, k, v, decay, state, o, B, H, st)
+                   : decode_launch<__nv_bfloat16, 128>(q, k, v, decay, state, o, B, H, st);
+}
+
+}  // namespace sala

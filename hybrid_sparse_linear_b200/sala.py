@@ -1,0 +1,223 @@
+"""ctypes binding of libsala (``include/sala.h``).
+
+Argument marshalling only: every function checks that the torch tensors it is given have the
+layout the C ABI documents, then passes raw device pointers and the current CUDA stream.  All
+computation happens in the library's CUDA kernels; there is no CPU or PyTorch fallback -- if the
+library is missing this module fails to import.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsala.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m hybrid_sparse_linear_b200.build`")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_BOUNDS = range(6)
+F32, BF16 = 0, 1
+
+_vp, _i, _st = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+_lib.sala_linear_prefill.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]
+_lib.sala_linear_decode.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp]
+_lib.sala_block_compress.argtypes = [_vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp]
+_lib.sala_block_topk.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp,
+                                 _st, _i, _vp]
+_lib.sala_block_topk_workspace.argtypes = [_i, _i, _i, _i, _i, _i, _i]
+_lib.sala_block_topk_workspace.restype = _st
+_lib.sala_sparse_prefill.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i,
+                                     ctypes.c_float, _i, _vp]
+_lib.sala_sparse_decode.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i,
+                                    _i, _i, _i, _i, ctypes.c_float, _vp, _st, _i, _vp]
+_lib.sala_sparse_decode_workspace.argtypes = [_i, _i, _i, _i, _i, _i, _i, _i, _i]
+_lib.sala_sparse_decode_workspace.restype = _st
+_lib.sala_check_status.argtypes = [_vp]
+_lib.sala_status_string.argtypes = [_i]
+_lib.sala_status_string.restype = ctypes.c_char_p
+_lib.sala_last_error.restype = ctypes.c_char_p
+_lib.sala_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+_lib.sala_selftest_wait_timeout.argtypes = [_vp]
+for _f in ("sala_linear_prefill", "sala_linear_decode", "sala_block_compress", "sala_block_topk",
+           "sala_sparse_prefill", "sala_sparse_decode", "sala_check_status",
+           "sala_selftest_wait_timeout"):
+    getattr(_lib, _f).restype = _i
+
+
+class SalaError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        msg = _lib.sala_last_error().decode()
+        super().__init__(f"{where}: {_lib.sala_status_string(code).decode()}: {msg}")
+
+
+def _check(code: int, where: str):
+    if code != OK:
+        raise SalaError(code, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float32:
+        return F32
+    raise TypeError(f"unsupported dtype {t.dtype} (bf16 or fp32)")
+
+
+def _need(t, name, shape=None, dtype=None):
+    if t is None:
+        return
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} has dtype {t.dtype}, expected {dtype}")
+
+
+# ----------------------------------------------------------------------------------------------
+def linear_prefill(q, k, v, decay, o=None, state_in=None, state_out=None, chunk=0, stream=None):
+    """Chunked decayed linear attention.  q,k,v: [B,H,N,d]; decay [H] fp32.  Returns o."""
+    B, H, N, d = q.shape
+    _need(q, "q"); _need(k, "k", q.shape, q.dtype); _need(v, "v", q.shape, q.dtype)
+    _need(decay, "decay", (H,), torch.float32)
+    if o is None:
+        o = torch.empty_like(q)
+    _need(o, "o", q.shape, q.dtype)
+    _need(state_in, "state_in", (B, H, d, d), torch.float32)
+    _need(state_out, "state_out", (B, H, d, d), torch.float32)
+    _check(_lib.sala_linear_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(decay), _ptr(o),
+                                    _ptr(state_in), _ptr(state_out), B, H, N, d, chunk, _dt(q),
+                                    _stream(stream)), "sala_linear_prefill")
+    return o
+
+
+def linear_decode(q, k, v, decay, state, o=None, stream=None):
+    """One decode step.  q,k,v: [B,H,d]; state [B,H,d,d] fp32 (updated in place).  Returns o."""
+    B, H, d = q.shape
+    _need(q, "q"); _need(k, "k", q.shape, q.dtype); _need(v, "v", q.shape, q.dtype)
+    _need(decay, "decay", (H,), torch.float32)
+    _need(state, "state", (B, H, d, d), torch.float32)
+    if o is None:
+        o = torch.empty_like(q)
+    _need(o, "o", q.shape, q.dtype)
+    _check(_lib.sala_linear_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(decay), _ptr(state), _ptr(o),
+                                   B, H, d, _dt(q), _stream(stream)), "sala_linear_decode")
+    return o
+
+
+def block_compress(k, kbar=None, block=64, first_block=0, n_blocks=None, stream=None):
+    """Mean-pooled block keys.  k: [B,Hkv,N,d] -> kbar [B,Hkv,nb_cap,d]."""
+    B, Hkv, N, d = k.shape
+    _need(k, "k")
+    if n_blocks is None:
+        n_blocks = N // block - first_block
+    if kbar is None:
+        kbar = torch.empty((B, Hkv, first_block + n_blocks, d), device=k.device, dtype=k.dtype)
+    _need(kbar, "kbar", dtype=k.dtype)
+    _check(_lib.sala_block_compress(_ptr(k), _ptr(kbar), B, Hkv, N, d, block, first_block,
+                                    n_blocks, kbar.shape[2], _dt(k), _stream(stream)),
+           "sala_block_compress")
+    return kbar
+
+
+def block_topk(q, kbar, topk, n_init=1, n_local=1, block=64, q_pos0=0, idx=None, workspace=None,
+               stream=None):
+    """Per (batch, KV group, query row) block selection -> idx [B,Hkv,Nq,slots] int32."""
+    B, H, Nq, d = q.shape
+    Hkv, nb = kbar.shape[1], kbar.shape[2]
+    _need(q, "q"); _need(kbar, "kbar", dtype=q.dtype)
+    slots = n_init + n_local + topk
+    if idx is None:
+        idx = torch.empty((B, Hkv, Nq, slots), device=q.device, dtype=torch.int32)
+    _need(idx, "idx", (B, Hkv, Nq, slots), torch.int32)
+    need = _lib.sala_block_topk_workspace(B, Hkv, Nq, q_pos0, nb, block, topk)
+    if need and workspace is None:
+        workspace = torch.empty(need, device=q.device, dtype=torch.uint8)
+    _check(_lib.sala_block_topk(_ptr(q), _ptr(kbar), _ptr(idx), B, H, Hkv, Nq, q_pos0, nb, d,
+                                block, topk, n_init, n_local, _ptr(workspace),
+                                0 if workspace is None else workspace.numel(), _dt(q),
+                                _stream(stream)), "sala_block_topk")
+    return idx
+
+
+def sparse_prefill(q, k, v, idx, o=None, block=64, scale=0.0, stream=None):
+    """Softmax attention over the selected blocks.  q: [B,H,N,d]; k,v: [B,Hkv,N,d]."""
+    B, H, N, d = q.shape
+    Hkv = k.shape[1]
+    _need(q, "q"); _need(k, "k", (B, Hkv, N, d), q.dtype); _need(v, "v", (B, Hkv, N, d), q.dtype)
+    _need(idx, "idx", dtype=torch.int32)
+    if idx.shape[:3] != (B, Hkv, N):
+        raise ValueError(f"idx has shape {tuple(idx.shape)}, expected ({B}, {Hkv}, {N}, slots)")
+    if o is None:
+        o = torch.empty_like(q)
+    _need(o, "o", q.shape, q.dtype)
+    _check(_lib.sala_sparse_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(idx), _ptr(o), B, H, Hkv, N, d,
+                                    block, idx.shape[3], float(scale), _dt(q), _stream(stream)),
+           "sala_sparse_prefill")
+    return o
+
+
+def sparse_decode_workspace_bytes(B, H, Hkv, pos, topk, n_init, n_local, d, block=64):
+    return _lib.sala_sparse_decode_workspace(B, H, Hkv, pos, block, topk, n_init, n_local, d)
+
+
+def sparse_decode(q, kcache, vcache, kbar, pos, topk, n_init=1, n_local=2, idx_in=None,
+                  idx_out=None, o=None, block=64, scale=0.0, workspace=None, stream=None):
+    """One query token per head at position pos over a dense KV cache.  q: [B,H,d]."""
+    B, H, d = q.shape
+    Hkv, Tmax = kcache.shape[1], kcache.shape[2]
+    _need(q, "q"); _need(kcache, "kcache", dtype=q.dtype); _need(vcache, "vcache", kcache.shape, q.dtype)
+    _need(kbar, "kbar", dtype=q.dtype)
+    slots = n_init + n_local + topk
+    _need(idx_in, "idx_in", (B, Hkv, slots), torch.int32)
+    _need(idx_out, "idx_out", (B, Hkv, slots), torch.int32)
+    if o is None:
+        o = torch.empty_like(q)
+    _need(o, "o", q.shape, q.dtype)
+    need = sparse_decode_workspace_bytes(B, H, Hkv, pos, topk, n_init, n_local, d, block)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), device=q.device, dtype=torch.uint8)
+    _check(_lib.sala_sparse_decode(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(kbar), _ptr(idx_in),
+                                   _ptr(idx_out), _ptr(o), B, H, Hkv, pos, Tmax, kbar.shape[2], d,
+                                   block, topk, n_init, n_local, float(scale), _ptr(workspace),
+                                   workspace.numel(), _dt(q), _stream(stream)),
+           "sala_sparse_decode")
+    return o
+
+
+def check_status(stream=None):
+    """Synchronise the stream and raise if a kernel recorded a device-side fault."""
+    _check(_lib.sala_check_status(_stream(stream)), "sala_check_status")
+
+
+def set_wait_limit_ns(ns: int):
+    _lib.sala_set_wait_limit_ns(int(ns))
+
+
+def selftest_wait_timeout(stream=None):
+    _check(_lib.sala_selftest_wait_timeout(_stream(stream)), "sala_selftest_wait_timeout")
+
+
+def default_scale(d: int) -> float:
+    return 1.0 / math.sqrt(d)
+
+
+raw = _lib  # the loaded C library, for callers that marshal pointers themselves

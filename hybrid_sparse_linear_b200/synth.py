@@ -15,6 +15,8 @@ Recipe (every draw is a standard normal from torch's Philox generator):
 * linear-attention layers: Q, K, V ~ N(0, 1) / sqrt(d); per-head decay
   ``lambda_h = exp(-2^(-8 (h+1) / H))`` (0.431 ... 0.9961 at H = 32), or the two fixed decays
   0.99 / 0.999 of the tiny fp32 case.
+* decode draws queries only for the last ``q_rows`` positions (a [.., q_rows, d] tensor seeded
+  like the others).
 * sparse-attention layers: K ~ N(0, 1); round(0.02 * n_blocks) complete blocks per (batch, KV
   head), chosen without replacement, get ``3 u`` added to every key row; Q ~ N(0, 1) + u for
   every query head of the group; V ~ N(0, 1); u ~ N(0, I_d), one per (layer, batch, KV head).
@@ -86,7 +88,8 @@ class SparseLayer:
 
 
 def sparse_layer(B, H, Hkv, N, d, dtype, device="cpu", layer=0, block=64, shift_frac=0.02,
-                 shift_mult=3.0, base=BASE_SEED) -> SparseLayer:
+                 shift_mult=3.0, base=BASE_SEED, q_rows=None) -> SparseLayer:
+    """q_rows: draw queries only for the last q_rows positions (decode), Q is [B, H, q_rows, d]."""
     G = H // Hkv
     nb = N // block
     gu = _gen("cpu", seed(layer, U, base))
@@ -106,7 +109,7 @@ def sparse_layer(B, H, Hkv, N, d, dtype, device="cpu", layer=0, block=64, shift_
             kk = k[b, g].index_select(0, rows).float() + shift
             k[b, g].index_copy_(0, rows, kk.to(dtype))
     uq = u.repeat_interleave(G, dim=1)  # [B, H, d]
-    q = normal((B, H, N, d), seed(layer, Q, base), device, dtype, 1.0, add=uq)
+    q = normal((B, H, q_rows or N, d), seed(layer, Q, base), device, dtype, 1.0, add=uq)
     v = normal((B, Hkv, N, d), seed(layer, V, base), device, dtype)
     return SparseLayer(q, k, v, shifted, u)
 

@@ -1,0 +1,195 @@
+/*
+ * sala.h -- C ABI of the SALA hybrid attention forward for NVIDIA B200 (sm_100a).
+ *
+ * MiniCPM-SALA mixes two attentions layer by layer, one sparse layer to three linear ones
+ * ("MiniCPM-SALA: Hybridizing Sparse and Linear Attention for Efficient Long-Context Modeling",
+ * abstract; gist.science technical summaries, section 2 "Method", subsection "hybrid attention"):
+ *   - Lightning Attention, a linear attention with a recursive O(N) form   -> sala_linear_*
+ *   - InfLLM-V2 sparse attention over a dense KV cache                       -> sala_block_*,
+ *                                                                               sala_sparse_*
+ * The pages give no formula for either; the operations below are the plain readings:
+ *   linear:  o_i = sum_{j<=i} lambda_h^{i-j} (q_i . k_j) v_j   (plus a carried d x d state)
+ *   sparse:  mean-pooled block keys, per-query top-k block selection that always keeps the init
+ *            and local blocks, then exact causal softmax attention over the selected blocks.
+ *
+ * Conventions shared by every call
+ *   - Tensors are dense, row-major [B, heads, rows, d] in device memory ("device pointer").
+ *     Query heads h of batch b use KV head h / (H / Hkv) (grouped-query attention).
+ *   - dt selects the element type of q/k/v/o/kbar: SALA_BF16 (tensor-core kernels, fp32
+ *     accumulation, bf16 output) or SALA_F32 (CUDA-core fp32 kernels).  Decays, linear states and
+ *     softmax statistics are always fp32.
+ *   - stream is a cudaStream_t (NULL = the legacy default stream).  Every call only enqueues
+ *     work and returns; results are ready when the stream reaches that point.
+ *   - Ownership: the caller allocates and frees every buffer, workspace included.  The library
+ *     keeps no allocation of its own; its only global state is one per-device status word.
+ *   - Errors: arguments are checked on the host before anything is launched.  A bad argument
+ *     returns SALA_ERR_INVALID_ARG, a valid but unimplemented case SALA_ERR_UNSUPPORTED, and in
+ *     both cases nothing is launched.  A failed launch returns SALA_ERR_CUDA.  Faults detected
+ *     on the device (a bounded wait that expired, an index out of range) are recorded in the
+ *     status word and reported by sala_check_status.  No call aborts or throws.
+ *     sala_last_error() gives a one-line explanation of the calling thread's last failure.
+ *   - Empty problems (B, H, N or Nq equal to 0) return SALA_OK and launch nothing.
+ */
+#ifndef SALA_H_
+#define SALA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SALA_OK = 0,
+    SALA_ERR_INVALID_ARG = 1,
+    SALA_ERR_UNSUPPORTED = 2,
+    SALA_ERR_CUDA = 3,
+    SALA_ERR_TIMEOUT = 4,
+    SALA_ERR_BOUNDS = 5
+} sala_status;
+
+typedef enum { SALA_F32 = 0, SALA_BF16 = 1 } sala_dtype;
+
+typedef void* sala_stream; /* a cudaStream_t */
+
+/* ------------------------------------------------------------------------------------------
+ * Linear attention prefill (Lightning-style, chunked).  Pages: abstract ("linear attention
+ * (Lightning Attention)"), DE technical summary section 2 ("recursive formulations", O(N)).
+ *
+ *   o_i     = sum_{j<=i} lambda_h^{i-j} (q_i . k_j) v_j  +  lambda_h^{i+1} q_i S_in
+ *   S_out   = lambda_h^N S_in + sum_{j<N} lambda_h^{N-1-j} k_j^T v_j
+ *
+ * q, k, v, o : [B, H, N, d] device, dt.  No feature map, no normalisation of o.
+ * decay      : [H] fp32 device, lambda_h in [0, 1].
+ * state_in   : [B, H, d, d] fp32 device or NULL (NULL = zero state).  Row index = key dim.
+ * state_out  : [B, H, d, d] fp32 device or NULL; may equal state_in (updated in place).
+ * chunk      : length of the intra-chunk masked product; 0 selects the kernel's native length.
+ *              The result does not depend on it beyond rounding.  Accepted: 0, 64.
+ * d          : 64 or 128.  All pointers 16-byte aligned.
+ */
+sala_status sala_linear_prefill(const void* q, const void* k, const void* v, const float* decay,
+                                void* o, const float* state_in, float* state_out, int B, int H,
+                                int N, int d, int chunk, sala_dtype dt, sala_stream stream);
+
+/* One decode step of the linear attention for every (batch, head): the state is updated first
+ * and then read, so the current token attends to itself with lambda^0:
+ *   S <- lambda_h S + k^T v ;  o = q S
+ * q, k, v, o : [B, H, d] device, dt.   state : [B, H, d, d] fp32 device, updated in place.
+ */
+sala_status sala_linear_decode(const void* q, const void* k, const void* v, const float* decay,
+                               float* state, void* o, int B, int H, int d, sala_dtype dt,
+                               sala_stream stream);
+
+/* ------------------------------------------------------------------------------------------
+ * Block compression of the keys of a sparse layer (mean pooling).  Pages: InfLLM-V2 selects
+ * the relevant context parts without extra parameters (JA technical summary section 2.1); the
+ * pooling itself is the plain reading of "mean-pooled block keys".
+ *
+ *   kbar[b, g, j] = round_dt( (1/block) * sum_{t < block} k[b, g, j*block + t] )
+ *
+ * computed exactly (fp64 sum) and rounded once to dt, for the complete blocks
+ * j = first_block .. first_block + n_blocks - 1 (they must end at or before row N).
+ * k    : [B, Hkv, N, d] device, dt.
+ * kbar : [B, Hkv, nb_cap, d] device, dt; block j is written at row j (nb_cap >= first_block +
+ *        n_blocks), other rows are untouched -- decode appends one block at a time.
+ * block: 64.
+ */
+sala_status sala_block_compress(const void* k, void* kbar, int B, int Hkv, int N, int d,
+                                int block, int first_block, int n_blocks, int nb_cap,
+                                sala_dtype dt, sala_stream stream);
+
+/* ------------------------------------------------------------------------------------------
+ * Block selection (scoring + top-k).  Query row r sits at absolute position p = q_pos0 + r in
+ * block c = p / block.  For KV group g:
+ *   forced     F = {0 .. n_init-1} U {max(0, c-n_local+1) .. c}          (init + local blocks)
+ *   candidates   = {n_init .. c-n_local}                                 (complete, past)
+ *   score(j)     = (sum over the group's query heads of q[b, h, r]) . kbar[b, g, j]
+ *   selection    = F U top_topk(candidates by score, ties to the lower block index)
+ * idx[b, g, r, :] receives the selection in ascending order, padded with -1, in
+ * slots = n_init + n_local + topk entries.
+ *
+ * q    : [B, H, Nq, d] device, dt.    kbar : [B, Hkv, nb, d] device, dt (nb >= c - n_local + 1
+ *        for every row).    idx : [B, Hkv, Nq, slots] int32 device.
+ * workspace: device scratch of at least sala_block_topk_workspace(...) bytes (may be NULL when
+ *        that is 0).  It must not be shared with a call that runs concurrently.
+ * Limits: topk <= 64 (or any value when every row has at most topk candidates), n_local >= 1,
+ *         n_init >= 0, block 64, d 64 or 128.
+ */
+sala_status sala_block_topk(const void* q, const void* kbar, int32_t* idx, int B, int H, int Hkv,
+                            int Nq, int q_pos0, int nb, int d, int block, int topk, int n_init,
+                            int n_local, void* workspace, size_t workspace_bytes, sala_dtype dt,
+                            sala_stream stream);
+size_t sala_block_topk_workspace(int B, int Hkv, int Nq, int q_pos0, int nb, int block, int topk);
+
+/* ------------------------------------------------------------------------------------------
+ * Sparse attention prefill: exact causal softmax over the selected blocks.  Pages: sparse
+ * layers compute on selected parts but keep the dense KV cache ("sparse compute, dense
+ * storage", JA technical summary section 1).
+ *
+ *   J(b,h,i) = { j <= i : j / block in idx[b, h / (H/Hkv), i, :] }
+ *   o[b,h,i] = sum_{j in J} softmax_j(scale * q[b,h,i] . k[b,g,j]) v[b,g,j]
+ *
+ * q, o : [B, H, N, d] device, dt.   k, v : [B, Hkv, N, d] device, dt.
+ * idx  : [B, Hkv, N, slots] int32 device, each row ascending and -1 padded (sala_block_topk's
+ *        output); entries must lie in [0, (N-1)/block].  An out-of-range entry is skipped and
+ *        flagged SALA_ERR_BOUNDS in the status word.
+ * scale: softmax scale; 0 selects 1/sqrt(d).   block 64; d 64 or 128 (bf16 tensor cores: 128).
+ */
+sala_status sala_sparse_prefill(const void* q, const void* k, const void* v, const int32_t* idx,
+                                void* o, int B, int H, int Hkv, int N, int d, int block,
+                                int slots, float scale, sala_dtype dt, sala_stream stream);
+
+/* ------------------------------------------------------------------------------------------
+ * Sparse attention decode: one query token per (batch, head) at absolute position pos, over
+ * a dense KV cache that holds rows 0 .. pos (capacity Tmax rows).
+ *
+ * q, o          : [B, H, d] device, dt.
+ * kcache, vcache: [B, Hkv, Tmax, d] device, dt.
+ * kbar          : [B, Hkv, nb_cap, d] device, dt; blocks 0 .. pos/block - n_local compressed.
+ * idx_in        : [B, Hkv, slots] int32 or NULL.  NULL = select here (scoring + top-k as in
+ *                 sala_block_topk, for q_pos0 = pos); otherwise attend to these blocks.
+ * idx_out       : [B, Hkv, slots] int32 or NULL; receives the selection that was used.
+ * workspace     : at least sala_sparse_decode_workspace(...) bytes of device scratch, not
+ *                 shared with a concurrent call.
+ */
+sala_status sala_sparse_decode(const void* q, const void* kcache, const void* vcache,
+                               const void* kbar, const int32_t* idx_in, int32_t* idx_out, void* o,
+                               int B, int H, int Hkv, int pos, int Tmax, int nb_cap, int d,
+                               int block, int topk, int n_init, int n_local, float scale,
+                               void* workspace, size_t workspace_bytes, sala_dtype dt,
+                               sala_stream stream);
+size_t sala_sparse_decode_workspace(int B, int H, int Hkv, int pos, int block, int topk,
+                                    int n_init, int n_local, int d);
+
+/* ------------------------------------------------------------------------------------------
+ * Status and diagnostics. */
+
+/* Synchronises `stream`, then reads and clears this device's status word: SALA_OK, or
+ * SALA_ERR_TIMEOUT / SALA_ERR_BOUNDS when a kernel recorded that fault since the last check,
+ * or SALA_ERR_CUDA when the synchronisation itself failed. */
+sala_status sala_check_status(sala_stream stream);
+
+/* Static string naming a status code. */
+const char* sala_status_string(sala_status status);
+
+/* One-line description of the calling thread's most recent failure ("" if none). */
+const char* sala_last_error(void);
+
+/* Upper bound, in nanoseconds, on every bounded wait inside the kernels (default 2e9).  A wait
+ * that runs past it gives up, records SALA_ERR_TIMEOUT and lets its kernel return. */
+void sala_set_wait_limit_ns(uint64_t ns);
+
+/* Self-test of the timeout path: launches one block that waits on a shared-memory barrier that
+ * nothing ever completes, bounded by sala_set_wait_limit_ns.  The kernel gives up, records
+ * SALA_ERR_TIMEOUT and returns; sala_check_status then reports it.  Launches on `stream`. */
+sala_status sala_selftest_wait_timeout(sala_stream stream);
+
+/* Library version (major * 10000 + minor * 100 + patch). */
+int sala_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SALA_H_ */

@@ -1,0 +1,146 @@
+"""GPU parity of the linear-attention calls (sala_linear_prefill / sala_linear_decode) against the
+fp64 oracle, through the C ABI.  Tolerances: see tests/parity.py."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from parity import assert_close
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def sala():
+    from hybrid_sparse_linear_b200 import sala as s
+    return s
+
+
+def _inputs(B, H, N, d, dtype, seed, layer=0):
+    from hybrid_sparse_linear_b200 import synth
+    q, k, v = synth.linear_layer(B, H, N, d, dtype, "cpu", layer=layer, base=seed)
+    return q, k, v
+
+
+def _f64(t):
+    return oracle.from_tensor(t)
+
+
+def test_tiny_fp32_prefill(sala):
+    from hybrid_sparse_linear_b200 import synth
+    w = synth.WORKLOADS["tiny_fp32_n512"]
+    q, k, v = _inputs(1, w["H"], w["N"], w["d"], torch.float32, 11)
+    lam = synth.decays(w["H"], "tiny")
+    so = torch.zeros((1, w["H"], w["d"], w["d"]), device="cuda")
+    o = sala.linear_prefill(q.cuda(), k.cuda(), v.cuda(), lam.cuda(), state_out=so, chunk=64)
+    sala.check_status()
+    ref, s_ref = oracle.linear_chunked(_f64(q), _f64(k), _f64(v), _f64(lam), 64)
+    assert_close(_f64(o), ref, "f32", "o")
+    assert_close(_f64(so), s_ref, "f32", "state_out")
+
+
+@pytest.mark.parametrize("d,N,B,H", [(128, 333, 2, 3), (64, 200, 1, 4), (128, 64, 1, 2),
+                                     (128, 1, 1, 2), (128, 1100, 1, 32)])
+def test_bf16_prefill_ragged_with_state(sala, d, N, B, H):
+    from hybrid_sparse_linear_b200 import synth
+    q, k, v = _inputs(B, H, N, d, torch.bfloat16, 100 + N)
+    lam = synth.decays(H)
+    g = torch.Generator().manual_seed(5)
+    s_in = torch.randn((B, H, d, d), generator=g) / d
+    so = torch.empty((B, H, d, d), device="cuda")
+    o = sala.linear_prefill(q.cuda(), k.cuda(), v.cuda(), lam.cuda(), state_in=s_in.cuda(),
+                            state_out=so)
+    sala.check_status()
+    ref, s_ref = oracle.linear_recurrent(_f64(q), _f64(k), _f64(v), _f64(lam), _f64(s_in))
+    assert_close(_f64(o), ref, "bf16", "o")
+    assert_close(_f64(so), s_ref, "bf16", "state_out")
+
+
+def test_fp32_prefill_split_resume(sala):
+    from hybrid_sparse_linear_b200 import synth
+    B, H, N, d = 1, 2, 300, 64
+    q, k, v = _inputs(B, H, N, d, torch.float32, 21)
+    lam = synth.decays(H, "tiny").cuda()
+    qc, kc, vc = q.cuda(), k.cuda(), v.cuda()
+    s_full = torch.empty((B, H, d, d), device="cuda")
+    o_full = sala.linear_prefill(qc, kc, vc, lam, state_out=s_full)
+    s1 = torch.empty_like(s_full)
+    o1 = sala.linear_prefill(qc[:, :, :131].contiguous(), kc[:, :, :131].contiguous(),
+                             vc[:, :, :131].contiguous(), lam, state_out=s1)
+    o2 = sala.linear_prefill(qc[:, :, 131:].contiguous(), kc[:, :, 131:].contiguous(),
+                             vc[:, :, 131:].contiguous(), lam, state_in=s1, state_out=s1)
+    sala.check_status()
+    ref, s_ref = oracle.linear_recurrent(_f64(q), _f64(k), _f64(v), _f64(lam.cpu()))
+    assert_close(_f64(torch.cat([o1, o2], dim=2)), ref, "f32", "resumed o")
+    assert_close(_f64(s1), s_ref, "f32", "resumed state")
+    assert_close(_f64(o_full), ref, "f32", "o")
+
+
+def test_prefill_empty_sequence_passes_state(sala):
+    B, H, d = 1, 2, 64
+    lam = torch.full((H,), 0.9, device="cuda")
+    s_in = torch.randn((B, H, d, d), device="cuda")
+    s_out = torch.zeros_like(s_in)
+    e = torch.empty((B, H, 0, d), device="cuda")
+    sala.linear_prefill(e, e, e, lam, o=e, state_in=s_in, state_out=s_out)
+    sala.check_status()
+    assert torch.equal(s_in, s_out)
+
+
+@pytest.mark.parametrize("dtype,d", [(torch.float32, 64), (torch.bfloat16, 128), (torch.float32, 128)])
+def test_decode_steps_match_oracle(sala, dtype, d):
+    from hybrid_sparse_linear_b200 import synth
+    B, H, steps = 2, 4, 5
+    lam = synth.decays(H)
+    g = torch.Generator().manual_seed(9)
+    S0 = (torch.randn((B, H, d, d), generator=g) / d).float()
+    S = S0.cuda().clone()
+    S_ref = _f64(S0)
+    q, k, v = _inputs(B, H, steps, d, dtype, 31)
+    kind = "bf16" if dtype == torch.bfloat16 else "f32"
+    for t in range(steps):
+        qt, kt, vt = (x[:, :, t].contiguous() for x in (q, k, v))
+        o = sala.linear_decode(qt.cuda(), kt.cuda(), vt.cuda(), lam.cuda(), S)
+        o_ref, S_ref = oracle.linear_decode(_f64(qt), _f64(kt), _f64(vt), _f64(lam), S_ref)
+        assert_close(_f64(o), o_ref, kind, f"o step {t}")
+    sala.check_status()
+    assert_close(_f64(S), S_ref, kind, "state")
+
+
+def test_decode_continues_prefill(sala):
+    # decode at position p reproduces prefill row p when started from the prefill state.
+    from hybrid_sparse_linear_b200 import synth
+    B, H, N, d = 1, 4, 129, 128
+    q, k, v = _inputs(B, H, N, d, torch.bfloat16, 41)
+    lam = synth.decays(H).cuda()
+    S = torch.empty((B, H, d, d), device="cuda")
+    o_pre = sala.linear_prefill(q.cuda(), k.cuda(), v.cuda(), lam)
+    sala.linear_prefill(q[:, :, :-1].contiguous().cuda(), k[:, :, :-1].contiguous().cuda(),
+                        v[:, :, :-1].contiguous().cuda(), lam, state_out=S)
+    o_dec = sala.linear_decode(q[:, :, -1].contiguous().cuda(), k[:, :, -1].contiguous().cuda(),
+                               v[:, :, -1].contiguous().cuda(), lam, S)
+    sala.check_status()
+    ref = oracle.linear_quadratic(_f64(q), _f64(k), _f64(v), _f64(lam.cpu()),
+                                  rows=np.array([[h, N - 1] for h in range(H)]))
+    assert_close(_f64(o_dec), ref.reshape(1, H, d), "bf16", "decode row")
+    assert_close(_f64(o_pre[:, :, -1]), ref.reshape(1, H, d), "bf16", "prefill row")
+
+
+def test_linear_prefill_full_size_sampled(sala):
+    """32 heads x 32768 tokens x d 128 (bf16), checked on sampled rows of four heads, including
+    the first and last rows and rows on both sides of 64- and 128-row boundaries."""
+    from hybrid_sparse_linear_b200 import synth
+    B, H, N, d = 1, 32, 32768, 128
+    q, k, v = synth.linear_layer(B, H, N, d, torch.bfloat16, "cuda", layer=0)
+    lam = synth.decays(H).cuda()
+    o = sala.linear_prefill(q, k, v, lam)
+    sala.check_status()
+    heads = [0, 7, 19, 31]
+    toks = [0, 1, 63, 64, 127, 128, 129, 4095, 4096, 20000, N - 129, N - 128, N - 2, N - 1]
+    sub = lambda t: oracle.from_tensor(t[:, heads])
+    rows = np.array([[hi, t] for hi in range(len(heads)) for t in toks])
+    ref = oracle.linear_quadratic(sub(q), sub(k), sub(v), _f64(lam.cpu()[heads]), rows=rows)
+    got = np.stack([_f64(o[0, heads[hi], t]) for hi, t in rows])
+    assert_close(got, ref, "bf16", "sampled rows")

@@ -1,0 +1,139 @@
+"""GPU parity of the block-sparse calls (sala_block_compress / sala_block_topk /
+sala_sparse_prefill / sala_sparse_decode) against the fp64 oracle, through the C ABI.
+
+Compression is checked bit for bit (both sides round the exact mean once).  Selection is checked
+with the near-tie rule of tests/parity.py.  Attention is checked on the GPU's own selection (the
+oracle re-evaluates the softmax over the blocks the GPU chose), so a legitimate near-tie swap does
+not move the output comparison."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from parity import assert_close, check_selection
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def sala():
+    from hybrid_sparse_linear_b200 import sala as s
+    return s
+
+
+def _f64(t):
+    return oracle.from_tensor(t)
+
+
+def _pipeline(sala, layer, kind, topk, n_init, n_local):
+    q, k, v = layer.q.cuda(), layer.k.cuda(), layer.v.cuda()
+    kbar = sala.block_compress(k)
+    idx = sala.block_topk(q, kbar, topk, n_init, n_local)
+    o = sala.sparse_prefill(q, k, v, idx)
+    sala.check_status()
+    q64, k64, v64 = _f64(layer.q), _f64(layer.k), _f64(layer.v)
+    kbar_ref = oracle.block_compress(k64, 64, round_to_bf16=(kind == "bf16"))
+    if kind == "f32":
+        kbar_ref = kbar_ref.astype(np.float32).astype(np.float64)
+    np.testing.assert_array_equal(_f64(kbar), kbar_ref)
+    idx_ref, kth = oracle.block_select(q64, kbar_ref, 64, topk, n_init, n_local)
+    ndiff = check_selection(idx.cpu().numpy(), idx_ref, q64, kbar_ref, kth, topk, n_init, n_local)
+    o_ref = oracle.sparse_attention(q64, k64, v64, idx.cpu().numpy(), 64)
+    assert_close(_f64(o), o_ref, kind, "o")
+    return ndiff
+
+
+def test_tiny_fp32_pipeline(sala):
+    from hybrid_sparse_linear_b200 import synth
+    w = synth.WORKLOADS["tiny_fp32_n512"]
+    layer = synth.tiny_sparse_layer(1, w["H"], w["Hkv"], w["N"], w["d"], torch.float32, layer=1)
+    _pipeline(sala, layer, "f32", w["topk"], w["n_init"], w["n_local"])
+
+
+@pytest.mark.parametrize("N,topk,n_local", [(64 * 70 + 17, 8, 2), (64 * 40, 64, 2), (64 * 9, 3, 1),
+                                             (100, 4, 2), (64 * 300, 16, 2)])
+def test_bf16_pipeline_gqa16(sala, N, topk, n_local):
+    from hybrid_sparse_linear_b200 import synth
+    layer = synth.sparse_layer(1, 32, 2, N, 128, torch.bfloat16, layer=2, shift_frac=0.05)
+    _pipeline(sala, layer, "bf16", topk, 1, n_local)
+
+
+def test_fp32_d128_pipeline_batch2(sala):
+    from hybrid_sparse_linear_b200 import synth
+    layer = synth.sparse_layer(2, 8, 2, 64 * 12 + 5, 128, torch.float32, layer=3, shift_frac=0.1)
+    _pipeline(sala, layer, "f32", 3, 1, 2)
+
+
+def test_shifted_blocks_are_selected(sala):
+    # Structural invariant on the GPU output: every shifted block that is a candidate is chosen
+    # while no more than top-k shifted blocks are causally available.
+    from hybrid_sparse_linear_b200 import synth
+    N, topk = 64 * 200, 16
+    layer = synth.sparse_layer(1, 32, 2, N, 128, torch.bfloat16, layer=4, shift_frac=0.05)
+    kbar = sala.block_compress(layer.k.cuda())
+    idx = sala.block_topk(layer.q.cuda(), kbar, topk, 1, 2).cpu().numpy()
+    for g in range(2):
+        shifted = layer.shifted[0][g]
+        for r in range(0, N, 61):
+            c = r // 64
+            avail = [x for x in shifted if 1 <= x <= c - 2]
+            if len(avail) <= topk:
+                assert set(avail) <= set(idx[0, g, r]), (g, r)
+
+
+def test_out_of_range_index_is_flagged(sala):
+    from hybrid_sparse_linear_b200 import synth
+    layer = synth.sparse_layer(1, 32, 2, 256, 128, torch.bfloat16, layer=5)
+    q, k, v = layer.q.cuda(), layer.k.cuda(), layer.v.cuda()
+    idx = torch.full((1, 2, 256, 3), -1, dtype=torch.int32)
+    idx[..., 0] = 0
+    idx[0, 0, 5, 1] = 3  # block 3 is in the future of row 5
+    o = sala.sparse_prefill(q, k, v, idx.cuda())
+    with pytest.raises(sala.SalaError) as ei:
+        sala.check_status()
+    assert ei.value.code == sala.ERR_BOUNDS
+    assert torch.isfinite(o.float()).all()
+    sala.check_status()  # the word was cleared
+
+
+# ---------------------------------------------------------------------------------------------
+def _decode_case(sala, T, topk, n_init, n_local, dtype, layer_id, given_idx=False):
+    from hybrid_sparse_linear_b200 import synth
+    H, Hkv, d = 32, 2, 128
+    layer = synth.sparse_layer(1, H, Hkv, T, d, dtype, device="cuda", layer=layer_id,
+                               shift_frac=0.05, q_rows=1)
+    pos = T - 1
+    kc, vc = layer.k, layer.v
+    kbar = sala.block_compress(kc)
+    qd = layer.q[:, :, 0].contiguous()
+    slots = n_init + n_local + topk
+    idx_out = torch.empty((1, Hkv, slots), dtype=torch.int32, device="cuda")
+    q64 = _f64(layer.q)
+    kind = "bf16" if dtype == torch.bfloat16 else "f32"
+    kbar_ref = oracle.block_compress(_f64(layer.k), 64, round_to_bf16=(kind == "bf16"))
+    if kind == "f32":
+        kbar_ref = kbar_ref.astype(np.float32).astype(np.float64)
+    idx_ref, kth = oracle.block_select(q64, kbar_ref, 64, topk, n_init, n_local, q_pos0=pos)
+    idx_in = torch.from_numpy(idx_ref[:, :, 0]).cuda() if given_idx else None
+    o = sala.sparse_decode(qd, kc, vc, kbar, pos, topk, n_init, n_local, idx_in=idx_in,
+                           idx_out=idx_out)
+    sala.check_status()
+    got = idx_out.cpu().numpy()[:, :, None, :]
+    check_selection(got, idx_ref, q64, kbar_ref, kth, topk, n_init, n_local, q_pos0=pos,
+                    row_ids=np.array([0]))
+    o_ref = oracle.sparse_attention(q64, _f64(layer.k), _f64(layer.v), got, 64, q_pos0=pos)
+    assert_close(_f64(o), o_ref[:, :, 0], kind, "decode o")
+
+
+@pytest.mark.parametrize("T", [64 * 300 + 5, 64 * 300, 64 * 3, 1, 70])
+def test_sparse_decode(sala, T):
+    _decode_case(sala, T, 16, 1, 2, torch.bfloat16, 6)
+
+
+def test_sparse_decode_given_idx_fp32(sala):
+    _decode_case(sala, 64 * 50 + 7, 8, 1, 2, torch.float32, 7, given_idx=True)
+
+
+def test_sparse_decode_1m_context(sala):
+    """One sparse layer at a 2^20-token cache: 16384 compressed blocks, top-64 + init + 2 local."""
+    _decode_case(sala, 1 << 20, 64, 1, 2, torch.bfloat16, 8)
