@@ -1,0 +1,549 @@
+#!/usr/bin/env python3
+"""Benchmark of the SALA hybrid attention forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {sala,reference}]
+
+One step = one attention prefill pass over a 262144-token sequence through the 32-layer hybrid
+stack: 24 linear-attention layers (sala_linear_prefill) and 8 sparse-attention layers
+(sala_block_compress -> sala_block_topk -> sala_sparse_prefill), sparse layers at 3, 7, ..., 31,
+each layer with its own seeded Q/K/V (all resident in HBM before timing; every tensor is 2 GiB or
+128 MiB, far larger than L2, so no flush is needed).  The printed JSON line reports whole-job
+tokens/s (device time, CUDA events, max over ranks), plus:
+  decode   : one decode token per step at a 2^20-token context through the same 32-layer stack
+             (24 x sala_linear_decode + 8 x sala_sparse_decode with in-kernel selection),
+             L2 flushed before every step, us/token;
+  e2e      : the prefill step through the same calls with the layer inputs streamed from pinned
+             host memory and the outputs copied back (copies inside the timed region);
+  roofline : the dominant kernel (sparse prefill, tensor-bound) -- algorithmic FLOPs per launch /
+             its mean launch time, against the measured bf16 peak;
+  cpu_baseline : the fp64 oracle on a bounded sample of the same workload, scaled to tokens/s.
+--impl reference times only the oracle (the CPU baseline arm) and prints its own line.
+With --gpus N > 1 (torchrun) every rank runs an independent replica (weak scaling).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+N_TOK = 262144
+H, HKV, D = 32, 2, 128
+TOPK, N_INIT, N_LOCAL, BLOCK = 64, 1, 2, 64
+N_LAYERS = 32
+SPARSE_LAYERS = [l for l in range(N_LAYERS) if l % 4 == 3]
+DECODE_T = 1 << 20
+METRIC = "SALA attn prefill tokens/s @256K; decode µs/token @1M; % of roofline"
+
+
+# ----------------------------------------------------------------------------------------------
+# algorithmic work (closed forms of the selection rule; independent of the GPU's output)
+
+def attended_keys(N: int, topk=TOPK, n_init=N_INIT, n_local=N_LOCAL, block=BLOCK) -> int:
+    """Sum over query tokens of |J_i| (keys each token attends to; shared by the group's heads)."""
+    total = 0
+    nblk = (N + block - 1) // block
+    for c in range(nblk):
+        rows = min(block, N - c * block)
+        ncand = max(0, c - n_local + 1 - n_init)
+        if ncand <= topk:
+            full_before = c                      # every block 0..c-1 plus the diagonal
+        else:
+            full_before = n_init + topk + (n_local - 1)
+        # token at offset t of block c attends full_before * block + (t + 1) keys
+        total += rows * full_before * block + rows * (rows + 1) // 2
+    return total
+
+
+def sparse_layer_flops(N: int) -> float:
+    return 4.0 * D * H * attended_keys(N)        # QK^T and PV, 2 FLOP per MAC each
+
+
+def linear_layer_bytes(N: int) -> float:
+    return 4.0 * H * N * D * 2                    # read Q, K, V and write O, bf16
+
+
+def decode_bytes(T: int) -> dict:
+    lin = H * D * D * 4 * 2 + 4 * H * D * 2       # state read + write, q/k/v/o
+    nb = T // BLOCK
+    sp = HKV * nb * D * 2 + HKV * (N_INIT + N_LOCAL + TOPK) * BLOCK * D * 2 * 2 + 2 * H * D * 2
+    return {"linear": lin, "sparse": sp, "step": 24 * lin + 8 * sp}
+
+
+# ----------------------------------------------------------------------------------------------
+# distributed plumbing (host-side only: barrier and max over ranks; no data-path collective)
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def init_dist(backend: str):
+    import torch.distributed as dist
+    ws, rank, _ = dist_env()
+    if ws > 1 and not dist.is_initialized():
+        import datetime
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=600))
+    return ws, rank
+
+
+def barrier():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+def max_over_ranks(x: float, device="cpu") -> float:
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------------------------
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled every 200 ms while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.reader = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.reader = threading.Thread(target=self._read, daemon=True)
+        self.reader.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.reader:
+            self.reader.join(timeout=2)
+        sm, smax, reasons, power = [], None, set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+                power.append(float(parts[3]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": smax, "reasons": ["no samples"]}
+        loaded = [s for s, p in zip(sm, power) if p > 300.0] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------------------------
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained", p["bf16_tflops"]),
+                "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+def run_prefill(sala, synth, torch, steps, warmup, stream):
+    """Device-timed hybrid prefill.  Returns timing dict."""
+    dev = torch.device("cuda")
+    lam = synth.decays(H).to(dev)
+    layers = []
+    for l in range(N_LAYERS):
+        if l in SPARSE_LAYERS:
+            sl = synth.sparse_layer(1, H, HKV, N_TOK, D, torch.bfloat16, dev, layer=l)
+            layers.append(("sparse", sl.q, sl.k, sl.v))
+        else:
+            q, k, v = synth.linear_layer(1, H, N_TOK, D, torch.bfloat16, dev, layer=l)
+            layers.append(("linear", q, k, v))
+    out = torch.empty((1, H, N_TOK, D), device=dev, dtype=torch.bfloat16)
+    nb = N_TOK // BLOCK
+    kbar = torch.empty((1, HKV, nb, D), device=dev, dtype=torch.bfloat16)
+    slots = N_INIT + N_LOCAL + TOPK
+    idx = torch.empty((1, HKV, N_TOK, slots), device=dev, dtype=torch.int32)
+    torch.cuda.synchronize()
+
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    sparse_ev, linear_ev, topk_ev = [], [], []
+
+    def one_step(record):
+        launches = 0
+        for kind, q, k, v in layers:
+            if kind == "linear":
+                e0, e1 = (ev(), ev()) if record else (None, None)
+                if record: e0.record(stream)
+                sala.linear_prefill(q, k, v, lam, o=out, stream=stream)
+                if record: e1.record(stream); linear_ev.append((e0, e1))
+                launches += 1
+            else:
+                t0, t1 = (ev(), ev()) if record else (None, None)
+                if record: t0.record(stream)
+                sala.block_compress(k, kbar, stream=stream)
+                sala.block_topk(q, kbar, TOPK, N_INIT, N_LOCAL, idx=idx, stream=stream)
+                if record: t1.record(stream); topk_ev.append((t0, t1))
+                e0, e1 = (ev(), ev()) if record else (None, None)
+                if record: e0.record(stream)
+                sala.sparse_prefill(q, k, v, idx, o=out, stream=stream)
+                if record: e1.record(stream); sparse_ev.append((e0, e1))
+                launches += 3
+        return launches
+
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            one_step(False)
+        sala.check_status(stream)
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        start, end = ev(), ev()
+        start.record(stream)
+        launches = 0
+        for _ in range(steps):
+            launches += one_step(True)
+        end.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    sala.check_status(stream)
+    total_ms = start.elapsed_time(end)
+    mean = lambda pairs: sum(a.elapsed_time(b) for a, b in pairs) / max(1, len(pairs))
+    res = {"total_ms": total_ms, "launches": launches,
+           "sparse_ms": mean(sparse_ev), "linear_ms": mean(linear_ev), "select_ms": mean(topk_ev)}
+    del layers, out, kbar, idx
+    torch.cuda.empty_cache()
+    return res
+
+
+def run_decode(sala, synth, torch, steps, warmup, stream):
+    """Decode at a 2^20-token context, 24 linear + 8 sparse layers per token, L2 flushed."""
+    dev = torch.device("cuda")
+    T = DECODE_T
+    pos = T - 1
+    lam = synth.decays(H).to(dev)
+    g = torch.Generator(device=dev)
+    lin = []
+    for l in range(N_LAYERS):
+        if l in SPARSE_LAYERS:
+            continue
+        g.manual_seed(synth.seed(l, synth.U) + 17)
+        S = torch.randn((1, H, D, D), generator=g, device=dev) / D
+        q, k, v = synth.linear_layer(1, H, 1, D, torch.bfloat16, dev, layer=l)
+        lin.append((S, q[:, :, 0].contiguous(), k[:, :, 0].contiguous(), v[:, :, 0].contiguous()))
+    sp = []
+    for l in SPARSE_LAYERS:
+        sl = synth.sparse_layer(1, H, HKV, T, D, torch.bfloat16, dev, layer=l, q_rows=1)
+        kbar = sala.block_compress(sl.k, stream=stream)
+        sp.append((sl.q[:, :, 0].contiguous(), sl.k, sl.v, kbar))
+    ws_bytes = sala.sparse_decode_workspace_bytes(1, H, HKV, pos, TOPK, N_INIT, N_LOCAL, D)
+    ws = torch.empty(max(ws_bytes, 16), device=dev, dtype=torch.uint8)
+    o = torch.empty((1, H, D), device=dev, dtype=torch.bfloat16)
+    flush = torch.empty(512 << 20, device=dev, dtype=torch.uint8)
+    torch.cuda.synchronize()
+
+    def one_token():
+        for l in range(N_LAYERS):
+            if l in SPARSE_LAYERS:
+                q, kc, vc, kbar = sp[SPARSE_LAYERS.index(l)]
+                sala.sparse_decode(q, kc, vc, kbar, pos, TOPK, N_INIT, N_LOCAL, o=o, workspace=ws,
+                                   stream=stream)
+            else:
+                S, q, k, v = lin[l - sum(1 for s in SPARSE_LAYERS if s < l)]
+                sala.linear_decode(q, k, v, lam, S, o=o, stream=stream)
+
+    times = []
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            one_token()
+        for _ in range(steps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            one_token()
+            b.record(stream)
+            times.append((a, b))
+        torch.cuda.synchronize()
+    sala.check_status(stream)
+    us = [a.elapsed_time(b) * 1000.0 for a, b in times]
+    del lin, sp, ws, flush
+    torch.cuda.empty_cache()
+    # launches per token: linear 1 each; sparse = select (2) + attention (2)
+    return {"us_per_token": statistics.median(us), "us_min": min(us), "samples": len(us),
+            "launches_per_token": 24 * 1 + 8 * 4}
+
+
+def run_e2e(sala, synth, torch, steps, warmup):
+    """Prefill step with every layer's inputs streamed from pinned host memory and the outputs
+    copied back, through the same calls.  One pinned host copy of a linear and of a sparse layer
+    is streamed for every layer of its kind (host RAM cannot hold 164 GiB of distinct inputs)."""
+    dev = torch.device("cuda")
+    lam = synth.decays(H).to(dev)
+    ql, kl, vl = synth.linear_layer(1, H, N_TOK, D, torch.bfloat16, dev, layer=0)
+    sl = synth.sparse_layer(1, H, HKV, N_TOK, D, torch.bfloat16, dev, layer=3)
+    host = {"linear": [t.cpu().pin_memory() for t in (ql, kl, vl)],
+            "sparse": [t.cpu().pin_memory() for t in (sl.q, sl.k, sl.v)]}
+    del ql, kl, vl, sl
+    dbuf = {"linear": [torch.empty((1, H, N_TOK, D), device=dev, dtype=torch.bfloat16) for _ in range(3)],
+            "sparse": [torch.empty((1, H, N_TOK, D), device=dev, dtype=torch.bfloat16),
+                       torch.empty((1, HKV, N_TOK, D), device=dev, dtype=torch.bfloat16),
+                       torch.empty((1, HKV, N_TOK, D), device=dev, dtype=torch.bfloat16)]}
+    out = torch.empty((1, H, N_TOK, D), device=dev, dtype=torch.bfloat16)
+    out_host = torch.empty((1, H, N_TOK, D), dtype=torch.bfloat16).pin_memory()
+    kbar = torch.empty((1, HKV, N_TOK // BLOCK, D), device=dev, dtype=torch.bfloat16)
+    idx = torch.empty((1, HKV, N_TOK, N_INIT + N_LOCAL + TOPK), device=dev, dtype=torch.int32)
+    stream = torch.cuda.current_stream()
+    h2d = d2h = 0
+
+    def step():
+        nonlocal h2d, d2h
+        for l in range(N_LAYERS):
+            kind = "sparse" if l in SPARSE_LAYERS else "linear"
+            for dst, src in zip(dbuf[kind], host[kind]):
+                dst.copy_(src, non_blocking=True)
+                h2d += src.numel() * 2
+            q, k, v = dbuf[kind]
+            if kind == "linear":
+                sala.linear_prefill(q, k, v, lam, o=out)
+            else:
+                sala.block_compress(k, kbar)
+                sala.block_topk(q, kbar, TOPK, N_INIT, N_LOCAL, idx=idx)
+                sala.sparse_prefill(q, k, v, idx, o=out)
+            out_host.copy_(out, non_blocking=True)
+            d2h += out.numel() * 2
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    h2d = d2h = 0
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    sala.check_status()
+    ms = a.elapsed_time(b) / steps
+    del host, dbuf, out, out_host, kbar, idx
+    torch.cuda.empty_cache()
+    return {"ms_per_step": ms, "h2d": h2d // steps, "d2h": d2h // steps}
+
+
+# ----------------------------------------------------------------------------------------------
+# CPU baseline: the fp64 oracle on a bounded sample, scaled to the full workload.
+
+def cpu_baseline(torch, synth, budget_s: float = 20.0):
+    import numpy as np
+    import oracle
+    cores = oracle.default_threads()
+    t_start = time.time()
+    # Linear layers: `cores` heads x n_lin tokens (the chunked form is O(N) per head).
+    n_lin = 16384
+    hs = min(cores, H)
+    q, k, v = synth.linear_layer(1, hs, n_lin, D, torch.bfloat16, "cpu", layer=0)
+    lam = synth.decays(H)[:hs]
+    f = oracle.from_tensor
+    t0 = time.perf_counter()
+    oracle.linear_chunked(f(q), f(k), f(v), f(lam), 64, threads=cores)
+    t_lin = time.perf_counter() - t0
+    lin_layer_s = t_lin * (H / hs) * (N_TOK / n_lin)
+    # Sparse layers: selection + attention for sampled query rows spread over the sequence; the
+    # attention cost is proportional to the attended keys, the selection cost to the candidates.
+    n_s = 32768
+    sl = synth.sparse_layer(1, H, HKV, n_s, D, torch.bfloat16, "cpu", layer=3)
+    q64, k64, v64 = f(sl.q), f(sl.k), f(sl.v)
+    kbar = oracle.block_compress(k64, BLOCK)
+    rng = np.random.default_rng(0)
+    rows_tok = np.sort(rng.choice(np.arange(n_s // 2, n_s), size=max(2 * cores, 48), replace=False))
+    t0 = time.perf_counter()
+    sel = []
+    for r in rows_tok:
+        ix, _ = oracle.block_select(q64[:, :, r:r + 1], kbar, BLOCK, TOPK, N_INIT, N_LOCAL,
+                                    q_pos0=int(r), threads=1)
+        sel.append(ix)
+    t_sel = time.perf_counter() - t0
+    idx = np.full((1, HKV, n_s, N_INIT + N_LOCAL + TOPK), -1, dtype=np.int32)
+    for r, ix in zip(rows_tok, sel):
+        idx[:, :, r] = ix[:, :, 0]
+    rows = np.array([[h, r] for r in rows_tok for h in range(H)])
+    t0 = time.perf_counter()
+    oracle.sparse_attention(q64, k64, v64, idx, BLOCK, rows=rows, threads=cores)
+    t_att = time.perf_counter() - t0
+    # scale: attention by attended keys, selection by candidate count
+    keys_sample = 0
+    cand_sample = 0
+    for r in rows_tok:
+        c = r // BLOCK
+        ncand = max(0, c - N_LOCAL + 1 - N_INIT)
+        full_before = c if ncand <= TOPK else N_INIT + TOPK + N_LOCAL - 1
+        keys_sample += full_before * BLOCK + (r % BLOCK) + 1
+        cand_sample += ncand
+    keys_full = attended_keys(N_TOK)
+    cand_full = sum(max(0, i // BLOCK - N_LOCAL + 1 - N_INIT) for i in range(0, N_TOK, BLOCK)) * BLOCK
+    sparse_layer_s = t_att * keys_full / keys_sample + t_sel * (cand_full * HKV) / (cand_sample * HKV)
+    step_s = 24 * lin_layer_s + 8 * sparse_layer_s
+    return {"value": N_TOK / step_s, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": (f"linear: {hs} heads x {n_lin} tokens (scaled x{H / hs:.0f} heads, "
+                       f"x{N_TOK // n_lin} length); sparse: selection + attention of {len(rows_tok)} "
+                       f"query tokens x {H} heads sampled from the second half of a {n_s}-token "
+                       f"layer (scaled by attended keys and candidate blocks); "
+                       f"{time.time() - t_start:.1f} s of CPU work"),
+            "step_s_extrapolated": step_s}
+
+
+# ----------------------------------------------------------------------------------------------
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["sala", "reference"], default="sala")
+    ap.add_argument("--phases", default="prefill,decode,e2e,cpu",
+                    help="comma list of prefill,decode,e2e,cpu (default: all)")
+    ap.add_argument("--decode-steps", type=int, default=50)
+    args = ap.parse_args()
+    phases = set(args.phases.split(","))
+
+    import torch
+    ws, rank, local = dist_env()
+
+    if args.impl == "reference":
+        if ws > 1:
+            init_dist("gloo")
+            if rank != 0:
+                barrier()
+                return
+        from hybrid_sparse_linear_b200 import synth
+        vals = []
+        for i in range(args.warmup + args.steps):
+            r = cpu_baseline(torch, synth)
+            if i >= args.warmup:
+                vals.append(r)
+        v = statistics.median(x["value"] for x in vals)
+        line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s",
+                "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": 1000.0 * N_TOK / v, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": {"workload": "hybrid_prefill_n256k: 24 linear + 8 sparse layers, "
+                                       "N=262144, 32 heads (2 KV heads in sparse layers), d=128",
+                           "global_batch": 1, "seq_len": N_TOK, "parallelism": "replicas"},
+                "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": vals[-1]["cores"],
+                                 "kind": "oracle", "sample": vals[-1]["sample"]},
+                "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        if ws > 1:
+            barrier()
+        return
+
+    if not torch.cuda.is_available():
+        print(json.dumps({"error": "no CUDA device"}))
+        sys.exit(1)
+    torch.cuda.set_device(local)
+    init_dist("nccl")
+    from hybrid_sparse_linear_b200 import sala, synth
+    stream = torch.cuda.Stream()
+    peaks = measured_peaks()
+    line = {"metric": METRIC, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded normal Q/K/V per layer)",
+            "config": {"workload": "hybrid_prefill_n256k: 24 linear + 8 sparse layers, N=262144, "
+                                   "32 heads (2 KV heads in sparse layers), d=128, chunk 64, "
+                                   "block 64, top-64 + init + 2 local",
+                       "global_batch": ws, "seq_len": N_TOK,
+                       "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU",
+                       "l2": "inputs larger than L2 (2 GiB per tensor); decode flushes L2 per step"}}
+    if "prefill" in phases:
+        vis = [x for x in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if x.strip()]
+        sampler = ClockSampler(vis[local] if local < len(vis) else str(local))
+        sampler.start()
+        pre = run_prefill(sala, synth, torch, args.steps, args.warmup, stream)
+        clocks = sampler.stop()
+        ms = max_over_ranks(pre["total_ms"], "cuda") / args.steps
+        line.update({"value": ws * N_TOK / (ms / 1000.0), "ms_per_step": ms,
+                     "gpu_launches": pre["launches"], "clocks": clocks})
+        fl = sparse_layer_flops(N_TOK)
+        achieved = fl / (pre["sparse_ms"] / 1000.0) / 1e12
+        peak = peaks["bf16_tflops_sustained"]
+        line["roofline"] = {"kernel": "sparse_prefill_tc_kernel", "bound": "tensor",
+                            "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                            "frac": achieved / peak, "traffic": None,
+                            "peak_source": f"{peaks['source']} bf16 sustained",
+                            "algorithmic_flops_per_launch": fl,
+                            "mean_launch_ms": pre["sparse_ms"]}
+        lin_gbs = linear_layer_bytes(N_TOK) / (pre["linear_ms"] / 1000.0) / 1e9
+        line["kernels"] = {
+            "linear_prefill": {"mean_ms": pre["linear_ms"], "achieved_gbs": lin_gbs,
+                               "hbm_frac": lin_gbs / peaks["hbm_gbs"]},
+            "sparse_prefill": {"mean_ms": pre["sparse_ms"], "achieved_tflops": achieved},
+            "compress_plus_select": {"mean_ms": pre["select_ms"]}}
+    if "decode" in phases:
+        dec = run_decode(sala, synth, torch, args.decode_steps, max(3, args.warmup), stream)
+        db = decode_bytes(DECODE_T)
+        gbs = db["step"] / (dec["us_per_token"] * 1e-6) / 1e9
+        line["decode"] = {"metric": "decode us/token @1M (24 linear + 8 sparse layers)",
+                          "us_per_token": dec["us_per_token"], "us_min": dec["us_min"],
+                          "bytes_per_token": db["step"], "achieved_gbs": gbs,
+                          "hbm_frac": gbs / peaks["hbm_gbs"],
+                          "launches_per_token": dec["launches_per_token"],
+                          "timing": "CUDA events per token, L2 flushed before each token, median"}
+    if "e2e" in phases:
+        e = run_e2e(sala, synth, torch, max(1, min(args.steps, 2)), 1)
+        line["e2e"] = {"value": ws * N_TOK / (max_over_ranks(e["ms_per_step"], "cuda") / 1000.0),
+                       "unit": "tokens/s", "h2d_bytes_per_step": e["h2d"],
+                       "d2h_bytes_per_step": e["d2h"],
+                       "note": "per layer: pinned host -> device copy of Q/K/V, the layer's calls, "
+                               "device -> pinned host copy of O"}
+    if "cpu" in phases and rank == 0 and ws == 1:
+        line["cpu_baseline"] = cpu_baseline(torch, synth)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    barrier()
+    import torch.distributed as dist
+    if dist.is_initialized():
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -123,7 +123,8 @@ sala_status sala_linear_prefill(const void* q, const void* k, const void* v, con
     REQUIRE(B >= 0 && H >= 0 && N >= 0, SALA_ERR_INVALID_ARG, "negative size (B=%d H=%d N=%d)", B, H, N);
     REQUIRE(dt == SALA_F32 || dt == SALA_BF16, SALA_ERR_INVALID_ARG, "unknown dtype %d", (int)dt);
     REQUIRE(d == 64 || d == 128, SALA_ERR_UNSUPPORTED, "head dim %d (supported: 64, 128)", d);
-    REQUIRE(chunk == 0 || chunk == 64, SALA_ERR_UNSUPPORTED, "chunk %d (supported: 0, 64)", chunk);
+    REQUIRE(chunk == 0 || chunk == 64 || chunk == 128, SALA_ERR_UNSUPPORTED,
+            "chunk %d (supported: 0, 64, 128)", chunk);
     if (B == 0 || H == 0) return SALA_OK;
     REQUIRE(decay != nullptr, SALA_ERR_INVALID_ARG, "decay must be a device pointer");
     if (state_in) REQUIRE(aligned16(state_in), SALA_ERR_INVALID_ARG, "state_in must be 16-byte aligned");

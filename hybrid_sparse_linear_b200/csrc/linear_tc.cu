@@ -1,0 +1,353 @@
+// Linear (Lightning-style) attention prefill on the 5th-generation tensor cores (sm_100a).
+//
+//   o_i = sum_{j<=i} lambda^{i-j} (q_i . k_j) v_j + lambda^{i+1} q_i S_in
+//
+// One CTA owns one (batch, head, 64-wide slice of the value columns): S[:, slice] and
+// o[:, slice] depend on no other slice, so the 2 slices of a head run on different SMs and only
+// re-read Q and K (which the sibling CTA pulls through L2 at the same time).  The CTA walks the
+// sequence in tiles of 128 rows; each tile is two 64-row chunks of the chunked form, with the
+// chunk-to-chunk term inside the tile computed directly instead of through the state (the same
+// sum, associated differently).  Per tile c (rows t, s in [0, 128), len valid):
+//   MMA1  A    = Q_c K_c^T                    M=128 N=128 K=128   (SMEM x SMEM -> TMEM)
+//   EPI   A'   = A * lambda^{t-s} [s <= t]    bf16, written back over A in TMEM
+//   MMA2  O1   = A' V_c[:, slice]             M=128 N=64  K=128   (TMEM x SMEM)
+//   MMA3  O2   = Q_c Sb                       M=128 N=64  K=128   (Sb = bf16 copy of S_{c-1})
+//   EPI   o_t  = O1_t + lambda^{t+1} O2_t     -> bf16 -> global
+//   EPI   V~   = diag(lambda^{len-1-s}) V_c   bf16 in SMEM
+//   MMA4  dS   = K_c^T V~                     M=128 N=64  K=128   (A read transposed)
+//   EPI   S    = lambda^len S + dS            fp32, one row of S per thread, in registers
+// Roles (192 threads): warps 0-3 epilogue (thread = row = TMEM lane), warp 4 TMA producer
+// (2-stage ring of Q/K/V tiles), warp 5 TMEM owner and MMA issuer.  MMA1 of tile c+1 overlaps
+// the epilogue of tile c.  Every wait is bounded (see ptx::mbar_wait).
+#include "kernels.h"
+#include "ptx.cuh"
+#include "tmap.cuh"
+
+namespace sala {
+namespace {
+
+using namespace ptx;
+
+constexpr int kD = 128, kC = 128, kDv = 64, kSlices = kD / kDv;
+constexpr int kThreads = 192;
+constexpr int kSub = kC * 128;                    // one [128 rows x 128 B] sub-tile: 16 KiB
+constexpr int kOffQ = 0, kOffK = 2 * kSub, kOffV = 4 * kSub;
+constexpr int kStageBytes = 5 * kSub;             // Q (2) + K (2) + V slice (1)
+constexpr int kOffVt = 2 * kStageBytes;           // V~ (decay-weighted V slice)
+constexpr int kOffSb = kOffVt + kSub;             // bf16 copy of the state slice
+constexpr int kSmemBytes = kOffSb + kSub + 1024;
+
+constexpr uint32_t kColA0 = 0, kColO1 = 256, kColO2 = 320, kColDS = 384, kTmemCols = 512;
+
+struct Bars {
+    uint64_t full[2], empty[2];
+    uint64_t qk_done[2], a_ready[2];
+    uint64_t v_ready, s_ready, o_free, ds_done, o_done, fin;
+    uint32_t tmem_base;
+    int abort;
+    float pw[kC + 1];  // lambda^n, n = 0..128
+};
+
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, const DevCtx& ctx,
+                                              volatile int* abort) {
+    if (*abort) return false;
+    if (!mbar_wait(bar, parity, ctx)) {
+        *abort = 1;
+        return false;
+    }
+    return true;
+}
+
+__device__ __forceinline__ float bf_lo(uint32_t x) { return __uint_as_float(x << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t x) { return __uint_as_float(x & 0xffff0000u); }
+
+__global__ void __launch_bounds__(kThreads, 1)
+linear_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
+                         const __grid_constant__ CUtensorMap tmK,
+                         const __grid_constant__ CUtensorMap tmV, const float* __restrict__ decay,
+                         __nv_bfloat16* __restrict__ out, const float* s_in, float* s_out, int H,
+                         int N, DevCtx ctx) {
+    extern __shared__ uint8_t smraw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smraw) + 1023) &
+                                             ~uintptr_t(1023));
+    __shared__ Bars bars;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int slice = blockIdx.x % kSlices;
+    const int64_t bh = blockIdx.x / kSlices;
+    const int n_tiles = (N + kC - 1) / kC;
+    volatile int* abort = &bars.abort;
+
+    if (warp == 5) {
+        tmem_alloc(&bars.tmem_base, kTmemCols);
+        tmem_relinquish();
+    }
+    if (tid == 0) {
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&bars.full[b], 1);
+            mbar_init(&bars.empty[b], 1);
+            mbar_init(&bars.qk_done[b], 1);
+            mbar_init(&bars.a_ready[b], 4);
+        }
+        mbar_init(&bars.v_ready, 4);
+        mbar_init(&bars.s_ready, 4);
+        mbar_init(&bars.o_free, 4);
+        mbar_init(&bars.ds_done, 1);
+        mbar_init(&bars.o_done, 1);
+        mbar_init(&bars.fin, 1);
+        bars.abort = 0;
+        fence_mbar_init();
+    }
+    {
+        const double lam = (double)decay[bh % H];
+        for (int n = tid; n <= kC; n += kThreads) bars.pw[n] = (float)pow(lam, (double)n);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bars.tmem_base;
+
+    if (warp == 4) {
+        // ------------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int issued[2] = {-1, -1};
+            for (int c = 0; c < n_tiles; ++c) {
+                const int s = c & 1, r = c >> 1;
+                if (r >= 1 && !wait_or_abort(&bars.empty[s], (r - 1) & 1, ctx, abort)) break;
+                uint8_t* st = sm + s * kStageBytes;
+                mbar_arrive_expect_tx(&bars.full[s], kStageBytes);
+                const int y = c * kC, z = (int)bh;
+                tma_load_3d(st + kOffQ, &tmQ, &bars.full[s], 0, y, z);
+                tma_load_3d(st + kOffQ + kSub, &tmQ, &bars.full[s], 64, y, z);
+                tma_load_3d(st + kOffK, &tmK, &bars.full[s], 0, y, z);
+                tma_load_3d(st + kOffK + kSub, &tmK, &bars.full[s], 64, y, z);
+                tma_load_3d(st + kOffV, &tmV, &bars.full[s], slice * kDv, y, z);
+                issued[s] = r;
+            }
+            for (int s = 0; s < 2; ++s)
+                if (issued[s] >= 0) (void)mbar_wait(&bars.full[s], issued[s] & 1, ctx);
+        }
+        __syncwarp();
+    } else if (warp == 5) {
+        // ------------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t idQK = idesc_bf16_f32(128, 128, false, false);
+            const uint32_t idO = idesc_bf16_f32(128, kDv, false, true);
+            const uint32_t idDS = idesc_bf16_f32(128, kDv, true, true);
+            const uint32_t vt = smem_u32(sm + kOffVt), sb = smem_u32(sm + kOffSb);
+            for (int c = 0; c <= n_tiles; ++c) {
+                if (c < n_tiles) {
+                    const int s = c & 1;
+                    if (!wait_or_abort(&bars.full[s], (c >> 1) & 1, ctx, abort)) break;
+                    tc_fence_after();
+                    const uint32_t q = smem_u32(sm + s * kStageBytes + kOffQ);
+                    const uint32_t k = smem_u32(sm + s * kStageBytes + kOffK);
+#pragma unroll
+                    for (int ks = 0; ks < kD / 16; ++ks) {
+                        const uint64_t a = sdesc_sw128(q + (ks >> 2) * kSub + (ks & 3) * 32, 16, 1024);
+                        const uint64_t b = sdesc_sw128(k + (ks >> 2) * kSub + (ks & 3) * 32, 16, 1024);
+                        mma_ss(tmem + kColA0 + s * 128, a, b, idQK, ks > 0);
+                    }
+                    mma_commit(&bars.qk_done[s]);
+                }
+                if (c >= 1) {
+                    const int j = c - 1, s = j & 1;
+                    const uint32_t q = smem_u32(sm + s * kStageBytes + kOffQ);
+                    const uint32_t k = smem_u32(sm + s * kStageBytes + kOffK);
+                    const uint32_t v = smem_u32(sm + s * kStageBytes + kOffV);
+                    if (!wait_or_abort(&bars.a_ready[s], (j >> 1) & 1, ctx, abort)) break;
+                    if (j >= 1 && !wait_or_abort(&bars.o_free, (j - 1) & 1, ctx, abort)) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int ks = 0; ks < kC / 16; ++ks)  // O1 = A' V  (A' from TMEM)
+                        mma_ts(tmem + kColO1, tmem + kColA0 + s * 128 + ks * 8,
+                               sdesc_sw128(v + ks * 16 * 128, 8192, 1024), idO, ks > 0);
+                    if (!wait_or_abort(&bars.s_ready, j & 1, ctx, abort)) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int ks = 0; ks < kD / 16; ++ks)  // O2 = Q Sb
+                        mma_ss(tmem + kColO2,
+                               sdesc_sw128(q + (ks >> 2) * kSub + (ks & 3) * 32, 16, 1024),
+                               sdesc_sw128(sb + ks * 16 * 128, 8192, 1024), idO, ks > 0);
+                    mma_commit(&bars.o_done);
+                    if (!wait_or_abort(&bars.v_ready, j & 1, ctx, abort)) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int ks = 0; ks < kC / 16; ++ks)  // dS = K^T V~  (A transposed)
+                        mma_ss(tmem + kColDS, sdesc_sw128(k + ks * 16 * 128, kSub, 1024),
+                               sdesc_sw128(vt + ks * 16 * 128, 8192, 1024), idDS, ks > 0);
+                    mma_commit(&bars.ds_done);
+                    mma_commit(&bars.empty[s]);
+                }
+            }
+            mma_commit(&bars.fin);
+            (void)mbar_wait(&bars.fin, 0, ctx);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------------ epilogue warps
+        const int t = tid;  // row of the tile = TMEM lane = row of the state slice
+        const uint32_t lb = tmem_lane_base(warp);
+        float S[kDv];
+        const float* sin_row = s_in ? s_in + (bh * kD + t) * kD + slice * kDv : nullptr;
+#pragma unroll
+        for (int j = 0; j < kDv; j += 4) {
+            float4 x = sin_row ? *reinterpret_cast<const float4*>(sin_row + j) : make_float4(0, 0, 0, 0);
+            S[j] = x.x; S[j + 1] = x.y; S[j + 2] = x.z; S[j + 3] = x.w;
+        }
+        uint8_t* sbrow = sm + kOffSb + t * 128;
+        auto write_sb = [&]() {  // bf16 copy of this thread's state row, 128-byte swizzle
+#pragma unroll
+            for (int cj = 0; cj < 8; ++cj) {
+                uint4 w;
+                w.x = pack_bf16x2(S[cj * 8 + 0], S[cj * 8 + 1]);
+                w.y = pack_bf16x2(S[cj * 8 + 2], S[cj * 8 + 3]);
+                w.z = pack_bf16x2(S[cj * 8 + 4], S[cj * 8 + 5]);
+                w.w = pack_bf16x2(S[cj * 8 + 6], S[cj * 8 + 7]);
+                *reinterpret_cast<uint4*>(sbrow + ((cj ^ (t & 7)) << 4)) = w;
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars.s_ready);
+        };
+        write_sb();
+        bool ok = true;
+        for (int c = 0; c < n_tiles && ok; ++c) {
+            const int s = c & 1;
+            const int len = min(kC, N - c * kC);
+            // (a) decay mask of Q K^T, written back as bf16 into the same TMEM columns.
+            if (!wait_or_abort(&bars.qk_done[s], (c >> 1) & 1, ctx, abort)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t colA = tmem + lb + kColA0 + s * 128;
+#pragma unroll 1
+            for (int k0 = 0; k0 < kC; k0 += 32) {
+                uint32_t x[32];
+                tmem_ld32(colA + k0, x);
+                tmem_ld_wait();
+                uint32_t pk[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const int s0 = k0 + 2 * j, s1 = s0 + 1;
+                    const float w0 = s0 <= t ? bars.pw[t - s0] : 0.f;
+                    const float w1 = s1 <= t ? bars.pw[t - s1] : 0.f;
+                    pk[j] = pack_bf16x2(__uint_as_float(x[2 * j]) * w0, __uint_as_float(x[2 * j + 1]) * w1);
+                }
+                tmem_st16(colA + k0 / 2, pk);
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars.a_ready[s]);
+            // (b) V~ = lambda^{len-1-s} V (row t of the V tile), same swizzled layout.
+            if (!wait_or_abort(&bars.full[s], (c >> 1) & 1, ctx, abort)) { ok = false; break; }
+            {
+                const float w = t < len ? bars.pw[len - 1 - t] : 0.f;
+                const uint8_t* vrow = sm + s * kStageBytes + kOffV + t * 128;
+                uint8_t* vtrow = sm + kOffVt + t * 128;
+#pragma unroll
+                for (int cj = 0; cj < 8; ++cj) {
+                    uint4 a = *reinterpret_cast<const uint4*>(vrow + cj * 16);
+                    uint4 b;
+                    b.x = pack_bf16x2(bf_lo(a.x) * w, bf_hi(a.x) * w);
+                    b.y = pack_bf16x2(bf_lo(a.y) * w, bf_hi(a.y) * w);
+                    b.z = pack_bf16x2(bf_lo(a.z) * w, bf_hi(a.z) * w);
+                    b.w = pack_bf16x2(bf_lo(a.w) * w, bf_hi(a.w) * w);
+                    *reinterpret_cast<uint4*>(vtrow + cj * 16) = b;
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars.v_ready);
+            }
+            // (c) S <- lambda^len S + dS, then its bf16 copy for the next tile.
+            if (!wait_or_abort(&bars.ds_done, c & 1, ctx, abort)) { ok = false; break; }
+            tc_fence_after();
+            {
+                uint32_t d0[32], d1[32];
+                tmem_ld32(tmem + lb + kColDS, d0);
+                tmem_ld32(tmem + lb + kColDS + 32, d1);
+                tmem_ld_wait();
+                const float decay_len = bars.pw[len];
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    S[j] = fmaf(decay_len, S[j], __uint_as_float(d0[j]));
+                    S[32 + j] = fmaf(decay_len, S[32 + j], __uint_as_float(d1[j]));
+                }
+                tc_fence_before();
+                write_sb();
+            }
+            // (d) o_t = O1 + lambda^{t+1} O2 for this tile's rows.
+            if (!wait_or_abort(&bars.o_done, c & 1, ctx, abort)) { ok = false; break; }
+            tc_fence_after();
+            {
+                uint32_t o1[32], o2[32];
+                const float wq = bars.pw[t + 1];
+                __nv_bfloat16* dst = out + ((bh * N) + (int64_t)c * kC + t) * kD + slice * kDv;
+#pragma unroll 1
+                for (int h0 = 0; h0 < kDv; h0 += 32) {
+                    tmem_ld32(tmem + lb + kColO1 + h0, o1);
+                    tmem_ld32(tmem + lb + kColO2 + h0, o2);
+                    tmem_ld_wait();
+                    if (t < len) {
+                        uint4 w[4];
+                        uint32_t* wp = reinterpret_cast<uint32_t*>(w);
+#pragma unroll
+                        for (int j = 0; j < 16; ++j)
+                            wp[j] = pack_bf16x2(fmaf(wq, __uint_as_float(o2[2 * j]), __uint_as_float(o1[2 * j])),
+                                                fmaf(wq, __uint_as_float(o2[2 * j + 1]), __uint_as_float(o1[2 * j + 1])));
+                        uint4* d4 = reinterpret_cast<uint4*>(dst + h0);
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) d4[j] = w[j];
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars.o_free);
+            }
+        }
+        if (ok && s_out) {
+            float* row = s_out + (bh * kD + t) * kD + slice * kDv;
+#pragma unroll
+            for (int j = 0; j < kDv; j += 4)
+                *reinterpret_cast<float4*>(row + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 5) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+}  // namespace
+
+bool linear_prefill_tc_supported(int d) { return d == kD; }
+
+cudaError_t launch_linear_prefill_tc(const void* q, const void* k, const void* v,
+                                     const float* decay, void* o, const float* s_in,
+                                     float* s_out, int B, int H, int N, int d, cudaStream_t st,
+                                     DevCtx ctx) {
+    if (d != kD) return cudaErrorNotSupported;
+    EncodeTiledFn fn = encode_tiled_fn();
+    if (!fn) return cudaErrorNotSupported;
+    auto make3 = [&](CUtensorMap* m, const void* base) -> bool {
+        cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)N, (cuuint64_t)B * H};
+        cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)kD * 2 * N};
+        cuuint32_t box[3] = {64, kC, 1};
+        cuuint32_t estr[3] = {1, 1, 1};
+        return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    };
+    CUtensorMap tmQ, tmK, tmV;
+    if (!make3(&tmQ, q) || !make3(&tmK, k) || !make3(&tmV, v)) return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(linear_prefill_tc_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    // If state_out aliases state_in, every CTA reads its slice before it writes it back, and no
+    // two CTAs share a slice, so in-place update is safe.
+    linear_prefill_tc_kernel<<<B * H * kSlices, kThreads, kSmemBytes, st>>>(
+        tmQ, tmK, tmV, decay, static_cast<__nv_bfloat16*>(o), s_in, s_out, H, N, ctx);
+    return cudaGetLastError();
+}
+
+}  // namespace sala

@@ -2,12 +2,13 @@
 // memory descriptor and TMEM paths the kernels use, so the tests can check each operand layout
 // in isolation against a host product.
 //
-//   sala_selftest_mma(A, B, D, N, K, b_mn_major, a_from_tmem, stream)
-//     A : [128, K] bf16, K contiguous.
+//   sala_selftest_mma(A, B, D, N, K, b_mn_major, a_mode, status, stream)
+//     A : a_mode 0/1 -> [128, K] bf16, K contiguous; a_mode 2 -> [K, 128] bf16, M contiguous
+//         (the MMA reads A transposed, "MN-major").
 //     B : b_mn_major == 0 -> [N, K] bf16, K contiguous, and D = A B^T
 //         b_mn_major == 1 -> [K, N] bf16, N contiguous, and D = A B
 //     D : [128, N] fp32.   N in {64, 128, 256}, K in {64, 128}.
-//     a_from_tmem: A is first copied into TMEM (bf16 pairs packed per 32-bit column) and the
+//     a_mode 1: A is first copied into TMEM (bf16 pairs packed per 32-bit column) and the
 //     MMA reads it from there instead of shared memory.
 //   Returns 0 on success, a negative value for bad arguments, or a CUDA error code.
 #include "ptx.cuh"
@@ -21,7 +22,8 @@ constexpr int kM = 128;
 __global__ void __launch_bounds__(128)
 selftest_mma_kernel(const __grid_constant__ CUtensorMap tA, const __grid_constant__ CUtensorMap tB,
                     const __nv_bfloat16* __restrict__ A, float* __restrict__ D, int N, int K,
-                    int b_mn_major, int a_tmem, DevCtx ctx) {
+                    int b_mn_major, int a_mode, DevCtx ctx) {
+    const int a_tmem = a_mode == 1, a_mn = a_mode == 2;
     extern __shared__ uint8_t smraw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
     uint8_t* sA = sm;                  // K/64 sub-tiles of [128 rows x 128 B]
@@ -49,7 +51,11 @@ selftest_mma_kernel(const __grid_constant__ CUtensorMap tA, const __grid_constan
     if (tid == 0) {
         const uint32_t bytes = (uint32_t)(kM * K * 2 + N * K * 2);
         ptx::mbar_arrive_expect_tx(&bar_tma, bytes);
-        for (int kb = 0; kb < K / 64; ++kb) ptx::tma_load_2d(sA + kb * kM * 128, &tA, &bar_tma, kb * 64, 0);
+        if (!a_mn) {
+            for (int kb = 0; kb < K / 64; ++kb) ptx::tma_load_2d(sA + kb * kM * 128, &tA, &bar_tma, kb * 64, 0);
+        } else {
+            for (int mb = 0; mb < kM / 64; ++mb) ptx::tma_load_2d(sA + mb * K * 128, &tA, &bar_tma, mb * 64, 0);
+        }
         if (!b_mn_major) {
             for (int kb = 0; kb < K / 64; ++kb) ptx::tma_load_2d(sB + kb * N * 128, &tB, &bar_tma, kb * 64, 0);
         } else {
@@ -75,7 +81,7 @@ selftest_mma_kernel(const __grid_constant__ CUtensorMap tA, const __grid_constan
 
     bool ok = ptx::mbar_wait(&bar_tma, 0, ctx);
     if (tid == 0 && ok) {
-        const uint32_t idesc = ptx::idesc_bf16_f32(kM, N, false, b_mn_major != 0);
+        const uint32_t idesc = ptx::idesc_bf16_f32(kM, N, a_mn != 0, b_mn_major != 0);
         const uint32_t a0 = ptx::smem_u32(sA), b0 = ptx::smem_u32(sB);
         for (int ks = 0; ks < K / 16; ++ks) {
             uint64_t bdesc;
@@ -85,6 +91,9 @@ selftest_mma_kernel(const __grid_constant__ CUtensorMap tA, const __grid_constan
                 bdesc = ptx::sdesc_sw128(b0 + ks * 16 * 128, (uint32_t)K * 128, 1024);
             if (a_tmem) {
                 ptx::mma_ts(tD, tA_cols + ks * 8, bdesc, idesc, ks > 0);
+            } else if (a_mn) {
+                const uint64_t adesc = ptx::sdesc_sw128(a0 + ks * 16 * 128, (uint32_t)K * 128, 1024);
+                ptx::mma_ss(tD, adesc, bdesc, idesc, ks > 0);
             } else {
                 const uint64_t adesc = ptx::sdesc_sw128(a0 + (ks / 4) * kM * 128 + (ks % 4) * 32, 16, 1024);
                 ptx::mma_ss(tD, adesc, bdesc, idesc, ks > 0);
@@ -112,13 +121,14 @@ selftest_mma_kernel(const __grid_constant__ CUtensorMap tA, const __grid_constan
 }  // namespace sala
 
 extern "C" int sala_selftest_mma(const void* A, const void* B, float* D, int N, int K,
-                                 int b_mn_major, int a_from_tmem, unsigned* status,
-                                 void* stream) {
+                                 int b_mn_major, int a_mode, unsigned* status, void* stream) {
     using namespace sala;
     if (!(N == 64 || N == 128 || N == 256) || !(K == 64 || K == 128) || !A || !B || !D || !status)
         return -1;
     CUtensorMap tA, tB;
-    cudaError_t e = make_tmap_bf16_2d(&tA, A, K, kM, K, 64, kM);
+    if (a_mode < 0 || a_mode > 2) return -1;
+    cudaError_t e = a_mode == 2 ? make_tmap_bf16_2d(&tA, A, kM, K, kM, 64, K)
+                                : make_tmap_bf16_2d(&tA, A, K, kM, K, 64, kM);
     if (e != cudaSuccess) return -2;
     if (!b_mn_major)
         e = make_tmap_bf16_2d(&tB, B, K, N, K, 64, N);
@@ -130,6 +140,6 @@ extern "C" int sala_selftest_mma(const void* A, const void* B, float* D, int N, 
     if (e != cudaSuccess) return (int)e;
     DevCtx ctx{status, 1000000000ull};
     selftest_mma_kernel<<<1, 128, smem, static_cast<cudaStream_t>(stream)>>>(
-        tA, tB, static_cast<const __nv_bfloat16*>(A), D, N, K, b_mn_major, a_from_tmem, ctx);
+        tA, tB, static_cast<const __nv_bfloat16*>(A), D, N, K, b_mn_major, a_mode, ctx);
     return (int)cudaGetLastError();
 }

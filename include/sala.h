@@ -64,8 +64,11 @@ typedef void* sala_stream; /* a cudaStream_t */
  * decay      : [H] fp32 device, lambda_h in [0, 1].
  * state_in   : [B, H, d, d] fp32 device or NULL (NULL = zero state).  Row index = key dim.
  * state_out  : [B, H, d, d] fp32 device or NULL; may equal state_in (updated in place).
- * chunk      : length of the intra-chunk masked product; 0 selects the kernel's native length.
- *              The result does not depend on it beyond rounding.  Accepted: 0, 64.
+ * chunk      : length of the chunks of the chunked form (0: the kernel's own).  The result does
+ *              not depend on it beyond rounding.  Accepted: 0, 64, 128.  The bf16 tensor-core
+ *              kernel (d = 128) always computes 128-row tiles -- two 64-row chunks per tile,
+ *              the chunk-to-chunk term inside a tile taken directly rather than through the
+ *              state; the fp32 CUDA-core kernel uses 64-row chunks.
  * d          : 64 or 128.  All pointers 16-byte aligned.
  */
 sala_status sala_linear_prefill(const void* q, const void* k, const void* v, const float* decay,

@@ -26,9 +26,9 @@ def st():
 @pytest.mark.parametrize("N", [64, 128, 256])
 @pytest.mark.parametrize("K", [64, 128])
 @pytest.mark.parametrize("b_mn_major", [0, 1])
-@pytest.mark.parametrize("a_tmem", [0, 1])
-def test_mma_tile(st, N, K, b_mn_major, a_tmem):
-    g = torch.Generator().manual_seed(N * 7 + K + 3 * b_mn_major + a_tmem)
+@pytest.mark.parametrize("a_mode", [0, 1, 2])  # A in SMEM K-major, in TMEM, in SMEM M-major
+def test_mma_tile(st, N, K, b_mn_major, a_mode):
+    g = torch.Generator().manual_seed(N * 7 + K + 3 * b_mn_major + a_mode)
     A = torch.randn((128, K), generator=g).to(torch.bfloat16)
     if b_mn_major:
         Bm = torch.randn((K, N), generator=g).to(torch.bfloat16)
@@ -36,10 +36,11 @@ def test_mma_tile(st, N, K, b_mn_major, a_tmem):
     else:
         Bm = torch.randn((N, K), generator=g).to(torch.bfloat16)
         ref = A.double() @ Bm.double().T
-    Ad, Bd = A.cuda(), Bm.cuda()
+    Ad = (A.T.contiguous() if a_mode == 2 else A).cuda()
+    Bd = Bm.cuda()
     D = torch.full((128, N), float("nan"), device="cuda")
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    r = st.sala_selftest_mma(Ad.data_ptr(), Bd.data_ptr(), D.data_ptr(), N, K, b_mn_major, a_tmem,
+    r = st.sala_selftest_mma(Ad.data_ptr(), Bd.data_ptr(), D.data_ptr(), N, K, b_mn_major, a_mode,
                              status.data_ptr(), torch.cuda.current_stream().cuda_stream)
     torch.cuda.synchronize()
     assert r == 0
