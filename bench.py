@@ -188,23 +188,35 @@ def measured_peaks():
                 "source": "fallback"}
 
 
-def run_prefill(sala, synth, torch, steps, warmup, stream):
-    """Device-timed hybrid prefill.  Returns timing dict."""
+# Prefill workloads: (sequence length, layer kinds).  The first is the benchmark; the single-layer
+# ones are the small cases used for kernel profiles.
+WORKLOADS = {
+    "hybrid_prefill_n256k": (N_TOK, ["sparse" if l in SPARSE_LAYERS else "linear" for l in range(N_LAYERS)]),
+    "sparse_prefill_n128k": (131072, ["sparse"]),
+    "linear_prefill_n32k": (32768, ["linear"]),
+    "sparse_prefill_n32k": (32768, ["sparse"]),
+    "linear_prefill_n256k": (N_TOK, ["linear"]),
+}
+
+
+def run_prefill(sala, synth, torch, steps, warmup, stream, workload="hybrid_prefill_n256k"):
+    """Device-timed prefill of a workload.  Returns timing dict."""
     dev = torch.device("cuda")
+    n_tok, kinds = WORKLOADS[workload]
     lam = synth.decays(H).to(dev)
     layers = []
-    for l in range(N_LAYERS):
-        if l in SPARSE_LAYERS:
-            sl = synth.sparse_layer(1, H, HKV, N_TOK, D, torch.bfloat16, dev, layer=l)
+    for l, kind in enumerate(kinds):
+        if kind == "sparse":
+            sl = synth.sparse_layer(1, H, HKV, n_tok, D, torch.bfloat16, dev, layer=l)
             layers.append(("sparse", sl.q, sl.k, sl.v))
         else:
-            q, k, v = synth.linear_layer(1, H, N_TOK, D, torch.bfloat16, dev, layer=l)
+            q, k, v = synth.linear_layer(1, H, n_tok, D, torch.bfloat16, dev, layer=l)
             layers.append(("linear", q, k, v))
-    out = torch.empty((1, H, N_TOK, D), device=dev, dtype=torch.bfloat16)
-    nb = N_TOK // BLOCK
+    out = torch.empty((1, H, n_tok, D), device=dev, dtype=torch.bfloat16)
+    nb = n_tok // BLOCK
     kbar = torch.empty((1, HKV, nb, D), device=dev, dtype=torch.bfloat16)
     slots = N_INIT + N_LOCAL + TOPK
-    idx = torch.empty((1, HKV, N_TOK, slots), device=dev, dtype=torch.int32)
+    idx = torch.empty((1, HKV, n_tok, slots), device=dev, dtype=torch.int32)
     torch.cuda.synchronize()
 
     ev = lambda: torch.cuda.Event(enable_timing=True)
@@ -442,7 +454,11 @@ def main():
     ap.add_argument("--phases", default="prefill,decode,e2e,cpu",
                     help="comma list of prefill,decode,e2e,cpu (default: all)")
     ap.add_argument("--decode-steps", type=int, default=50)
+    ap.add_argument("--workload", default="hybrid_prefill_n256k", choices=sorted(WORKLOADS),
+                    help="prefill workload (default: the 32-layer hybrid stack at 256K)")
     args = ap.parse_args()
+    if args.workload != "hybrid_prefill_n256k" and "--phases" not in " ".join(sys.argv):
+        args.phases = "prefill"
     phases = set(args.phases.split(","))
 
     import torch
@@ -498,26 +514,39 @@ def main():
         vis = [x for x in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if x.strip()]
         sampler = ClockSampler(vis[local] if local < len(vis) else str(local))
         sampler.start()
-        pre = run_prefill(sala, synth, torch, args.steps, args.warmup, stream)
+        pre = run_prefill(sala, synth, torch, args.steps, args.warmup, stream, args.workload)
         clocks = sampler.stop()
+        n_tok, kinds = WORKLOADS[args.workload]
         ms = max_over_ranks(pre["total_ms"], "cuda") / args.steps
-        line.update({"value": ws * N_TOK / (ms / 1000.0), "ms_per_step": ms,
+        line.update({"value": ws * n_tok / (ms / 1000.0), "ms_per_step": ms,
                      "gpu_launches": pre["launches"], "clocks": clocks})
-        fl = sparse_layer_flops(N_TOK)
-        achieved = fl / (pre["sparse_ms"] / 1000.0) / 1e12
-        peak = peaks["bf16_tflops_sustained"]
-        line["roofline"] = {"kernel": "sparse_prefill_tc_kernel", "bound": "tensor",
-                            "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                            "frac": achieved / peak, "traffic": None,
-                            "peak_source": f"{peaks['source']} bf16 sustained",
-                            "algorithmic_flops_per_launch": fl,
-                            "mean_launch_ms": pre["sparse_ms"]}
-        lin_gbs = linear_layer_bytes(N_TOK) / (pre["linear_ms"] / 1000.0) / 1e9
-        line["kernels"] = {
-            "linear_prefill": {"mean_ms": pre["linear_ms"], "achieved_gbs": lin_gbs,
-                               "hbm_frac": lin_gbs / peaks["hbm_gbs"]},
-            "sparse_prefill": {"mean_ms": pre["sparse_ms"], "achieved_tflops": achieved},
-            "compress_plus_select": {"mean_ms": pre["select_ms"]}}
+        if args.workload != "hybrid_prefill_n256k":
+            line["config"]["workload"] = f"{args.workload}: {len(kinds)} x {kinds[0]} layer, N={n_tok}"
+            line["config"]["seq_len"] = n_tok
+        line["kernels"] = {}
+        if "sparse" in kinds:
+            fl = sparse_layer_flops(n_tok)
+            achieved = fl / (pre["sparse_ms"] / 1000.0) / 1e12
+            peak = peaks["bf16_tflops_sustained"]
+            line["roofline"] = {"kernel": "sparse_prefill_tc_kernel", "bound": "tensor",
+                                "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                                "frac": achieved / peak, "traffic": None,
+                                "peak_source": f"{peaks['source']} bf16 sustained",
+                                "algorithmic_flops_per_launch": fl,
+                                "mean_launch_ms": pre["sparse_ms"]}
+            line["kernels"]["sparse_prefill"] = {"mean_ms": pre["sparse_ms"], "achieved_tflops": achieved}
+            line["kernels"]["compress_plus_select"] = {"mean_ms": pre["select_ms"]}
+        if "linear" in kinds:
+            lin_gbs = linear_layer_bytes(n_tok) / (pre["linear_ms"] / 1000.0) / 1e9
+            line["kernels"]["linear_prefill"] = {"mean_ms": pre["linear_ms"], "achieved_gbs": lin_gbs,
+                                                 "hbm_frac": lin_gbs / peaks["hbm_gbs"]}
+            if "sparse" not in kinds:
+                line["roofline"] = {"kernel": "linear_prefill_tc_kernel", "bound": "hbm",
+                                    "achieved": lin_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                    "frac": lin_gbs / peaks["hbm_gbs"], "traffic": None,
+                                    "peak_source": f"{peaks['source']} HBM copy",
+                                    "algorithmic_bytes_per_launch": linear_layer_bytes(n_tok),
+                                    "mean_launch_ms": pre["linear_ms"]}
     if "decode" in phases:
         dec = run_decode(sala, synth, torch, args.decode_steps, max(3, args.warmup), stream)
         db = decode_bytes(DECODE_T)
