@@ -69,6 +69,16 @@ sala::DType to_dt(sala_dtype dt) { return dt == SALA_BF16 ? sala::DType::BF16 : 
 
 }  // namespace
 
+namespace sala {
+// Lets entry points defined in other files report through sala_last_error().
+void set_last_error(const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof(g_err), fmt, ap);
+    va_end(ap);
+}
+}  // namespace sala
+
 extern "C" {
 
 int sala_version(void) { return 100; }

@@ -58,4 +58,7 @@ cudaError_t launch_sparse_decode_attn(DType dt, const void* q, const void* kc, c
 // Diagnostics.
 cudaError_t launch_selftest_wait(cudaStream_t st, DevCtx ctx);
 
+// Sets the calling thread's sala_last_error() message (printf-style).
+void set_last_error(const char* fmt, ...);
+
 }  // namespace sala

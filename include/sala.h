@@ -165,6 +165,32 @@ sala_status sala_sparse_decode(const void* q, const void* kcache, const void* vc
 size_t sala_sparse_decode_workspace(int B, int H, int Hkv, int pos, int block, int topk,
                                     int n_init, int n_local, int d);
 
+/* sala_sparse_decode for callers that cannot allocate device memory.  The pages have no
+ * counterpart; this is a property of the library, not of the method.
+ *
+ * Some callers may not allocate device memory once they are running -- a serving loop that sizes
+ * every buffer at start-up so no allocation can stall or fail mid-request, or a plug-in whose
+ * host application owns the whole device memory pool and exposes no allocator -- and so cannot
+ * provide the workspace sala_sparse_decode needs.  This call takes the same arguments minus the
+ * workspace and computes the same result with scratch space built into the library: a fixed
+ * 4 MiB area per GPU (a __device__ array that every GPU loading the library keeps until the
+ * process exits).  It allocates nothing itself and calls nothing that allocates.
+ *   - Problems whose sala_sparse_decode_workspace(...) exceeds 4 MiB are refused with
+ *     SALA_ERR_UNSUPPORTED (for example B * Hkv above 7 at a 2^20-token context with
+ *     32 query heads, d 128, top-64); nothing is launched.
+ *   - The first call on each GPU looks up the area's device address (cudaGetSymbolAddress, with
+ *     that GPU current) and caches it; make that first call before any stream capture.
+ *   - All calls on a GPU share the one area: calls that can run concurrently on the same GPU
+ *     race on it and must not be made.  The area keeps the previous call's contents; nothing in
+ *     it needs to start at zero.
+ * Other arguments, validation and errors are those of sala_sparse_decode. */
+sala_status sala_sparse_decode_noalloc(const void* q, const void* kcache, const void* vcache,
+                                       const void* kbar, const int32_t* idx_in, int32_t* idx_out,
+                                       void* o, int B, int H, int Hkv, int pos, int Tmax,
+                                       int nb_cap, int d, int block, int topk, int n_init,
+                                       int n_local, float scale, sala_dtype dt,
+                                       sala_stream stream);
+
 /* ------------------------------------------------------------------------------------------
  * Status and diagnostics. */
 
