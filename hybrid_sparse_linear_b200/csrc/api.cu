@@ -269,6 +269,7 @@ sala_status sala_sparse_prefill(const void* q, const void* k, const void* v, con
     REQUIRE(block == 64, SALA_ERR_UNSUPPORTED, "block %d (supported: 64)", block);
     REQUIRE(slots <= 1024, SALA_ERR_UNSUPPORTED, "more than 1024 slots");
     REQUIRE(isfinite(scale) && scale >= 0.f, SALA_ERR_INVALID_ARG, "scale must be finite and >= 0");
+    REQUIRE(H / Hkv <= 16, SALA_ERR_UNSUPPORTED, "more than 16 query heads per KV head");
     if (B == 0 || H == 0 || N == 0) return SALA_OK;
     REQ_PTR(q); REQ_PTR(k); REQ_PTR(v); REQ_PTR(o);
     REQUIRE(idx != nullptr, SALA_ERR_INVALID_ARG, "idx must be a device pointer");
@@ -307,6 +308,7 @@ sala_status sala_sparse_decode(const void* q, const void* kcache, const void* vc
                                       n_local, dt);
     if (s != SALA_OK) return s;
     REQUIRE(isfinite(scale) && scale >= 0.f, SALA_ERR_INVALID_ARG, "scale must be finite and >= 0");
+    REQUIRE(H / Hkv <= 16, SALA_ERR_UNSUPPORTED, "more than 16 query heads per KV head");
     if (B == 0 || H == 0) return SALA_OK;
     REQ_PTR(q); REQ_PTR(kcache); REQ_PTR(vcache); REQ_PTR(o);
     if (!idx_in && nb_cap > 0) REQ_PTR(kbar);

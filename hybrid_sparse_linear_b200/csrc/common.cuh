@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 namespace sala {
 
 // Bits of the per-device status word (read and cleared by sala_check_status).
@@ -61,5 +63,20 @@ __device__ __forceinline__ uint64_t sel_key(float score, int blk) {
 __device__ __forceinline__ int key_block(uint64_t key) { return (int)(~(uint32_t)(key & 0xffffffffu)); }
 
 __host__ __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+// Raises a kernel's dynamic shared memory limit once per device, so later launches (including
+// ones recorded into a CUDA graph) only enqueue work.
+template <auto Kern>
+cudaError_t ensure_smem(int bytes) {
+    static std::atomic<unsigned long long> done{0};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const unsigned long long bit = 1ull << (dev & 63);
+    if (done.load(std::memory_order_acquire) & bit) return cudaSuccess;
+    e = cudaFuncSetAttribute(Kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) done.fetch_or(bit, std::memory_order_release);
+    return e;
+}
 
 }  // namespace sala

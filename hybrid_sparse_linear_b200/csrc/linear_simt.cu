@@ -125,7 +125,7 @@ cudaError_t prefill_simt(const void* q, const void* k, const void* v, const floa
     constexpr int DV = 32;
     auto kern = linear_prefill_simt_kernel<T, D, DV>;
     const size_t smem = PrefillSmem<D, DV>::bytes;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = ensure_smem<linear_prefill_simt_kernel<T, D, DV>>((int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid(D / DV, (unsigned)(B * H));
     kern<<<grid, kThreads, smem, st>>>(static_cast<const T*>(q), static_cast<const T*>(k),

@@ -9,16 +9,19 @@
 // chunk-to-chunk term inside the tile computed directly instead of through the state (the same
 // sum, associated differently).  Per tile c (rows t, s in [0, 128), len valid):
 //   MMA1  A    = Q_c K_c^T                    M=128 N=128 K=128   (SMEM x SMEM -> TMEM)
-//   EPI   A'   = A * lambda^{t-s} [s <= t]    bf16, written back over A in TMEM
+//   EPI-A A'   = A * lambda^{t-s} [s <= t]    bf16, written back over A in TMEM
 //   MMA2  O1   = A' V_c[:, slice]             M=128 N=64  K=128   (TMEM x SMEM)
 //   MMA3  O2   = Q_c Sb                       M=128 N=64  K=128   (Sb = bf16 copy of S_{c-1})
-//   EPI   o_t  = O1_t + lambda^{t+1} O2_t     -> bf16 -> global
-//   EPI   V~   = diag(lambda^{len-1-s}) V_c   bf16 in SMEM
+//   EPI-A o_t  = O1_t + lambda^{t+1} O2_t     -> bf16 -> global
+//   EPI-S V~   = diag(lambda^{len-1-s}) V_c   bf16 in SMEM (double-buffered)
 //   MMA4  dS   = K_c^T V~                     M=128 N=64  K=128   (A read transposed)
-//   EPI   S    = lambda^len S + dS            fp32, one row of S per thread, in registers
-// Roles (192 threads): warps 0-3 epilogue (thread = row = TMEM lane), warp 4 TMA producer
-// (2-stage ring of Q/K/V tiles), warp 5 TMEM owner and MMA issuer.  MMA1 of tile c+1 overlaps
-// the epilogue of tile c.  Every wait is bounded (see ptx::mbar_wait).
+//   EPI-S S    = lambda^len S + dS            fp32, one row of S per thread, in registers
+// The only serial dependency between tiles is the state: MMA3(c) needs Sb(c-1) and the update of
+// S(c) needs MMA4(c).  The MMA issuer therefore issues MMA3 and MMA4 of a tile first, then MMA2
+// and the next tile's MMA1, so the tensor core works on MMA2/MMA1 while the state warps update S.
+// Roles (320 threads): warps 0-3 "EPI-A" (mask + output, thread = row = TMEM lane), warps 4-7
+// "EPI-S" (V~ + state, thread = row of S), warp 8 TMA producer (2-stage ring of Q/K/V tiles),
+// warp 9 TMEM owner and MMA issuer.  Every wait is bounded (see ptx::mbar_wait).
 #include "kernels.h"
 #include "ptx.cuh"
 #include "tmap.cuh"
@@ -29,20 +32,20 @@ namespace {
 using namespace ptx;
 
 constexpr int kD = 128, kC = 128, kDv = 64, kSlices = kD / kDv;
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
 constexpr int kSub = kC * 128;                    // one [128 rows x 128 B] sub-tile: 16 KiB
 constexpr int kOffQ = 0, kOffK = 2 * kSub, kOffV = 4 * kSub;
 constexpr int kStageBytes = 5 * kSub;             // Q (2) + K (2) + V slice (1)
-constexpr int kOffVt = 2 * kStageBytes;           // V~ (decay-weighted V slice)
-constexpr int kOffSb = kOffVt + kSub;             // bf16 copy of the state slice
+constexpr int kOffVt = 2 * kStageBytes;           // V~ (decay-weighted V slice), 2 buffers
+constexpr int kOffSb = kOffVt + 2 * kSub;         // bf16 copy of the state slice
 constexpr int kSmemBytes = kOffSb + kSub + 1024;
 
 constexpr uint32_t kColA0 = 0, kColO1 = 256, kColO2 = 320, kColDS = 384, kTmemCols = 512;
 
 struct Bars {
     uint64_t full[2], empty[2];
-    uint64_t qk_done[2], a_ready[2];
-    uint64_t v_ready, s_ready, o_free, ds_done, o_done, fin;
+    uint64_t qk_done[2], a_ready[2], v_ready[2];
+    uint64_t o_done, o_free, ds_done, s_ready, fin;
     uint32_t tmem_base;
     int abort;
     float pw[kC + 1];  // lambda^n, n = 0..128
@@ -77,7 +80,7 @@ linear_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
     const int n_tiles = (N + kC - 1) / kC;
     volatile int* abort = &bars.abort;
 
-    if (warp == 5) {
+    if (warp == 9) {
         tmem_alloc(&bars.tmem_base, kTmemCols);
         tmem_relinquish();
     }
@@ -87,12 +90,12 @@ linear_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
             mbar_init(&bars.empty[b], 1);
             mbar_init(&bars.qk_done[b], 1);
             mbar_init(&bars.a_ready[b], 4);
+            mbar_init(&bars.v_ready[b], 4);
         }
-        mbar_init(&bars.v_ready, 4);
-        mbar_init(&bars.s_ready, 4);
+        mbar_init(&bars.o_done, 1);
         mbar_init(&bars.o_free, 4);
         mbar_init(&bars.ds_done, 1);
-        mbar_init(&bars.o_done, 1);
+        mbar_init(&bars.s_ready, 4);
         mbar_init(&bars.fin, 1);
         bars.abort = 0;
         fence_mbar_init();
@@ -106,7 +109,7 @@ linear_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
     tc_fence_after();
     const uint32_t tmem = bars.tmem_base;
 
-    if (warp == 4) {
+    if (warp == 8) {
         // ------------------------------------------------------------------ TMA producer
         if (lane == 0) {
             int issued[2] = {-1, -1};
@@ -127,65 +130,133 @@ linear_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                 if (issued[s] >= 0) (void)mbar_wait(&bars.full[s], issued[s] & 1, ctx);
         }
         __syncwarp();
-    } else if (warp == 5) {
+    } else if (warp == 9) {
         // ------------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             const uint32_t idQK = idesc_bf16_f32(128, 128, false, false);
             const uint32_t idO = idesc_bf16_f32(128, kDv, false, true);
             const uint32_t idDS = idesc_bf16_f32(128, kDv, true, true);
-            const uint32_t vt = smem_u32(sm + kOffVt), sb = smem_u32(sm + kOffSb);
-            for (int c = 0; c <= n_tiles; ++c) {
-                if (c < n_tiles) {
-                    const int s = c & 1;
-                    if (!wait_or_abort(&bars.full[s], (c >> 1) & 1, ctx, abort)) break;
-                    tc_fence_after();
-                    const uint32_t q = smem_u32(sm + s * kStageBytes + kOffQ);
-                    const uint32_t k = smem_u32(sm + s * kStageBytes + kOffK);
+            const uint32_t sb = smem_u32(sm + kOffSb);
+            auto issue_qk = [&](int c) -> bool {
+                const int s = c & 1;
+                if (!wait_or_abort(&bars.full[s], (c >> 1) & 1, ctx, abort)) return false;
+                tc_fence_after();
+                const uint32_t q = smem_u32(sm + s * kStageBytes + kOffQ);
+                const uint32_t k = smem_u32(sm + s * kStageBytes + kOffK);
 #pragma unroll
-                    for (int ks = 0; ks < kD / 16; ++ks) {
-                        const uint64_t a = sdesc_sw128(q + (ks >> 2) * kSub + (ks & 3) * 32, 16, 1024);
-                        const uint64_t b = sdesc_sw128(k + (ks >> 2) * kSub + (ks & 3) * 32, 16, 1024);
-                        mma_ss(tmem + kColA0 + s * 128, a, b, idQK, ks > 0);
-                    }
-                    mma_commit(&bars.qk_done[s]);
+                for (int ks = 0; ks < kD / 16; ++ks) {
+                    const uint64_t a = sdesc_sw128(q + (ks >> 2) * kSub + (ks & 3) * 32, 16, 1024);
+                    const uint64_t b = sdesc_sw128(k + (ks >> 2) * kSub + (ks & 3) * 32, 16, 1024);
+                    mma_ss(tmem + kColA0 + s * 128, a, b, idQK, ks > 0);
                 }
-                if (c >= 1) {
-                    const int j = c - 1, s = j & 1;
-                    const uint32_t q = smem_u32(sm + s * kStageBytes + kOffQ);
-                    const uint32_t k = smem_u32(sm + s * kStageBytes + kOffK);
-                    const uint32_t v = smem_u32(sm + s * kStageBytes + kOffV);
-                    if (!wait_or_abort(&bars.a_ready[s], (j >> 1) & 1, ctx, abort)) break;
-                    if (j >= 1 && !wait_or_abort(&bars.o_free, (j - 1) & 1, ctx, abort)) break;
-                    tc_fence_after();
+                mma_commit(&bars.qk_done[s]);
+                return true;
+            };
+            bool ok = n_tiles > 0 ? issue_qk(0) : true;
+            for (int c = 0; c < n_tiles && ok; ++c) {
+                const int s = c & 1;
+                const uint32_t q = smem_u32(sm + s * kStageBytes + kOffQ);
+                const uint32_t k = smem_u32(sm + s * kStageBytes + kOffK);
+                const uint32_t v = smem_u32(sm + s * kStageBytes + kOffV);
+                const uint32_t vt = smem_u32(sm + kOffVt + s * kSub);
+                // MMA3: O2 = Q Sb(c-1)   (needs the state and a free O)
+                if (!wait_or_abort(&bars.s_ready, c & 1, ctx, abort)) break;
+                if (c >= 1 && !wait_or_abort(&bars.o_free, (c - 1) & 1, ctx, abort)) break;
+                tc_fence_after();
 #pragma unroll
-                    for (int ks = 0; ks < kC / 16; ++ks)  // O1 = A' V  (A' from TMEM)
-                        mma_ts(tmem + kColO1, tmem + kColA0 + s * 128 + ks * 8,
-                               sdesc_sw128(v + ks * 16 * 128, 8192, 1024), idO, ks > 0);
-                    if (!wait_or_abort(&bars.s_ready, j & 1, ctx, abort)) break;
-                    tc_fence_after();
+                for (int ks = 0; ks < kD / 16; ++ks)
+                    mma_ss(tmem + kColO2, sdesc_sw128(q + (ks >> 2) * kSub + (ks & 3) * 32, 16, 1024),
+                           sdesc_sw128(sb + ks * 16 * 128, 8192, 1024), idO, ks > 0);
+                // MMA4: dS = K^T V~
+                if (!wait_or_abort(&bars.v_ready[s], (c >> 1) & 1, ctx, abort)) break;
+                tc_fence_after();
 #pragma unroll
-                    for (int ks = 0; ks < kD / 16; ++ks)  // O2 = Q Sb
-                        mma_ss(tmem + kColO2,
-                               sdesc_sw128(q + (ks >> 2) * kSub + (ks & 3) * 32, 16, 1024),
-                               sdesc_sw128(sb + ks * 16 * 128, 8192, 1024), idO, ks > 0);
-                    mma_commit(&bars.o_done);
-                    if (!wait_or_abort(&bars.v_ready, j & 1, ctx, abort)) break;
-                    tc_fence_after();
+                for (int ks = 0; ks < kC / 16; ++ks)
+                    mma_ss(tmem + kColDS, sdesc_sw128(k + ks * 16 * 128, kSub, 1024),
+                           sdesc_sw128(vt + ks * 16 * 128, 8192, 1024), idDS, ks > 0);
+                mma_commit(&bars.ds_done);
+                // MMA2: O1 = A' V   (A' from TMEM)
+                if (!wait_or_abort(&bars.a_ready[s], (c >> 1) & 1, ctx, abort)) break;
+                tc_fence_after();
 #pragma unroll
-                    for (int ks = 0; ks < kC / 16; ++ks)  // dS = K^T V~  (A transposed)
-                        mma_ss(tmem + kColDS, sdesc_sw128(k + ks * 16 * 128, kSub, 1024),
-                               sdesc_sw128(vt + ks * 16 * 128, 8192, 1024), idDS, ks > 0);
-                    mma_commit(&bars.ds_done);
-                    mma_commit(&bars.empty[s]);
-                }
+                for (int ks = 0; ks < kC / 16; ++ks)
+                    mma_ts(tmem + kColO1, tmem + kColA0 + s * 128 + ks * 8,
+                           sdesc_sw128(v + ks * 16 * 128, 8192, 1024), idO, ks > 0);
+                mma_commit(&bars.o_done);
+                mma_commit(&bars.empty[s]);
+                // MMA1 of the next tile
+                if (c + 1 < n_tiles) ok = issue_qk(c + 1);
             }
             mma_commit(&bars.fin);
             (void)mbar_wait(&bars.fin, 0, ctx);
         }
         __syncwarp();
-    } else {
-        // ------------------------------------------------------------------ epilogue warps
-        const int t = tid;  // row of the tile = TMEM lane = row of the state slice
+    } else if (warp < 4) {
+        // ------------------------------------------------------------------ EPI-A: mask, output
+        const int t = tid;
+        const uint32_t lb = tmem_lane_base(warp);
+        const float wq = bars.pw[t + 1];
+        for (int c = 0; c < n_tiles; ++c) {
+            const int s = c & 1;
+            const int len = min(kC, N - c * kC);
+            if (!wait_or_abort(&bars.qk_done[s], (c >> 1) & 1, ctx, abort)) break;
+            tc_fence_after();
+            const uint32_t colA = tmem + lb + kColA0 + s * 128;
+            // s > t is masked; tiles never reach s >= 128, and rows/keys past len are zero.
+            const int kmax = (t >> 5) + 1;  // 32-column chunks holding some s <= t
+#pragma unroll 1
+            for (int kc = 0; kc < 4; ++kc) {
+                const int k0 = kc * 32;
+                uint32_t pk[16];
+                if (__any_sync(0xffffffffu, kc < kmax)) {
+                    uint32_t x[32];
+                    tmem_ld32(colA + k0, x);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const int s0 = k0 + 2 * j, s1 = s0 + 1;
+                        const float w0 = s0 <= t ? bars.pw[t - s0] : 0.f;
+                        const float w1 = s1 <= t ? bars.pw[t - s1] : 0.f;
+                        pk[j] = pack_bf16x2(__uint_as_float(x[2 * j]) * w0, __uint_as_float(x[2 * j + 1]) * w1);
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) pk[j] = 0u;
+                }
+                tmem_st16(colA + k0 / 2, pk);
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars.a_ready[s]);
+            // o_t = O1 + lambda^{t+1} O2
+            if (!wait_or_abort(&bars.o_done, c & 1, ctx, abort)) break;
+            tc_fence_after();
+            __nv_bfloat16* dst = out + ((bh * N) + (int64_t)c * kC + t) * kD + slice * kDv;
+            uint32_t o1[64], o2[64];
+            tmem_ld32(tmem + lb + kColO1, *reinterpret_cast<uint32_t(*)[32]>(&o1[0]));
+            tmem_ld32(tmem + lb + kColO1 + 32, *reinterpret_cast<uint32_t(*)[32]>(&o1[32]));
+            tmem_ld32(tmem + lb + kColO2, *reinterpret_cast<uint32_t(*)[32]>(&o2[0]));
+            tmem_ld32(tmem + lb + kColO2 + 32, *reinterpret_cast<uint32_t(*)[32]>(&o2[32]));
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars.o_free);
+            if (t < len) {
+                uint4 w[8];
+                uint32_t* wp = reinterpret_cast<uint32_t*>(w);
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    wp[j] = pack_bf16x2(fmaf(wq, __uint_as_float(o2[2 * j]), __uint_as_float(o1[2 * j])),
+                                        fmaf(wq, __uint_as_float(o2[2 * j + 1]), __uint_as_float(o1[2 * j + 1])));
+                uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) d4[j] = w[j];
+            }
+        }
+    } else if (warp < 8) {
+        // ------------------------------------------------------------------ EPI-S: V~, state
+        const int t = tid - 128;  // row of the V tile / of the state slice
         const uint32_t lb = tmem_lane_base(warp);
         float S[kDv];
         const float* sin_row = s_in ? s_in + (bh * kD + t) * kD + slice * kDv : nullptr;
@@ -214,35 +285,12 @@ linear_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
         for (int c = 0; c < n_tiles && ok; ++c) {
             const int s = c & 1;
             const int len = min(kC, N - c * kC);
-            // (a) decay mask of Q K^T, written back as bf16 into the same TMEM columns.
-            if (!wait_or_abort(&bars.qk_done[s], (c >> 1) & 1, ctx, abort)) { ok = false; break; }
-            tc_fence_after();
-            const uint32_t colA = tmem + lb + kColA0 + s * 128;
-#pragma unroll 1
-            for (int k0 = 0; k0 < kC; k0 += 32) {
-                uint32_t x[32];
-                tmem_ld32(colA + k0, x);
-                tmem_ld_wait();
-                uint32_t pk[16];
-#pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const int s0 = k0 + 2 * j, s1 = s0 + 1;
-                    const float w0 = s0 <= t ? bars.pw[t - s0] : 0.f;
-                    const float w1 = s1 <= t ? bars.pw[t - s1] : 0.f;
-                    pk[j] = pack_bf16x2(__uint_as_float(x[2 * j]) * w0, __uint_as_float(x[2 * j + 1]) * w1);
-                }
-                tmem_st16(colA + k0 / 2, pk);
-            }
-            tmem_st_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars.a_ready[s]);
-            // (b) V~ = lambda^{len-1-s} V (row t of the V tile), same swizzled layout.
+            // V~ = lambda^{len-1-s} V (row t of the V tile), same swizzled layout.
             if (!wait_or_abort(&bars.full[s], (c >> 1) & 1, ctx, abort)) { ok = false; break; }
             {
                 const float w = t < len ? bars.pw[len - 1 - t] : 0.f;
                 const uint8_t* vrow = sm + s * kStageBytes + kOffV + t * 128;
-                uint8_t* vtrow = sm + kOffVt + t * 128;
+                uint8_t* vtrow = sm + kOffVt + s * kSub + t * 128;
 #pragma unroll
                 for (int cj = 0; cj < 8; ++cj) {
                     uint4 a = *reinterpret_cast<const uint4*>(vrow + cj * 16);
@@ -255,9 +303,9 @@ linear_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&bars.v_ready);
+                if (lane == 0) mbar_arrive(&bars.v_ready[s]);
             }
-            // (c) S <- lambda^len S + dS, then its bf16 copy for the next tile.
+            // S <- lambda^len S + dS, then its bf16 copy for the next tile.
             if (!wait_or_abort(&bars.ds_done, c & 1, ctx, abort)) { ok = false; break; }
             tc_fence_after();
             {
@@ -274,34 +322,6 @@ linear_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                 tc_fence_before();
                 write_sb();
             }
-            // (d) o_t = O1 + lambda^{t+1} O2 for this tile's rows.
-            if (!wait_or_abort(&bars.o_done, c & 1, ctx, abort)) { ok = false; break; }
-            tc_fence_after();
-            {
-                uint32_t o1[32], o2[32];
-                const float wq = bars.pw[t + 1];
-                __nv_bfloat16* dst = out + ((bh * N) + (int64_t)c * kC + t) * kD + slice * kDv;
-#pragma unroll 1
-                for (int h0 = 0; h0 < kDv; h0 += 32) {
-                    tmem_ld32(tmem + lb + kColO1 + h0, o1);
-                    tmem_ld32(tmem + lb + kColO2 + h0, o2);
-                    tmem_ld_wait();
-                    if (t < len) {
-                        uint4 w[4];
-                        uint32_t* wp = reinterpret_cast<uint32_t*>(w);
-#pragma unroll
-                        for (int j = 0; j < 16; ++j)
-                            wp[j] = pack_bf16x2(fmaf(wq, __uint_as_float(o2[2 * j]), __uint_as_float(o1[2 * j])),
-                                                fmaf(wq, __uint_as_float(o2[2 * j + 1]), __uint_as_float(o1[2 * j + 1])));
-                        uint4* d4 = reinterpret_cast<uint4*>(dst + h0);
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) d4[j] = w[j];
-                    }
-                }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bars.o_free);
-            }
         }
         if (ok && s_out) {
             float* row = s_out + (bh * kD + t) * kD + slice * kDv;
@@ -312,7 +332,7 @@ linear_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == 9) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
@@ -340,8 +360,7 @@ cudaError_t launch_linear_prefill_tc(const void* q, const void* k, const void* v
     };
     CUtensorMap tmQ, tmK, tmV;
     if (!make3(&tmQ, q) || !make3(&tmK, k) || !make3(&tmV, v)) return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(linear_prefill_tc_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    cudaError_t e = ensure_smem<linear_prefill_tc_kernel>(kSmemBytes);
     if (e != cudaSuccess) return e;
     // If state_out aliases state_in, every CTA reads its slice before it writes it back, and no
     // two CTAs share a slice, so in-place update is safe.

@@ -209,7 +209,7 @@ cudaError_t tiled(const void* q, const void* kbar, int32_t* idx, int B, int H, i
                   int q_pos0, int nb, int topk, int n_init, int n_local, cudaStream_t st) {
     auto kern = topk_tiled_kernel<T, D>;
     const size_t smem = TopkSmem<D>::bytes;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = ensure_smem<topk_tiled_kernel<T, D>>((int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid(ceil_div(Nq, kRT), (unsigned)(B * Hkv));
     kern<<<grid, kTThreads, smem, st>>>(static_cast<const T*>(q), static_cast<const T*>(kbar), idx,

@@ -141,7 +141,7 @@ cudaError_t prefill(const void* q, const void* k, const void* v, const int32_t* 
     auto kern = sparse_prefill_simt_kernel<T, D>;
     const int G = H / Hkv;
     const size_t smem = BlockSmem<D>::bytes + sizeof(float) * G * D;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = ensure_smem<sparse_prefill_simt_kernel<T, D>>((int)(BlockSmem<D>::bytes + sizeof(float) * 2 * kWarps * D));
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)N, (unsigned)(B * Hkv));
     kern<<<grid, kWarps * 32, smem, st>>>(static_cast<const T*>(q), static_cast<const T*>(k),
@@ -235,7 +235,7 @@ cudaError_t decode(const void* q, const void* kc, const void* vc, const int32_t*
     auto kern = sparse_decode_partial_kernel<T, D>;
     const int G = H / Hkv;
     const size_t smem = BlockSmem<D>::bytes + sizeof(float) * G * D;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = ensure_smem<sparse_decode_partial_kernel<T, D>>((int)(BlockSmem<D>::bytes + sizeof(float) * 2 * kWarps * D));
     if (e != cudaSuccess) return e;
     float* part = static_cast<float*>(ws);
     kern<<<dim3(slots, B * Hkv), kWarps * 32, smem, st>>>(

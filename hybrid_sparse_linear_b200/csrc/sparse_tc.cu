@@ -6,21 +6,24 @@
 // share their query block (8 divides 64), hence the forced blocks and the diagonal; their
 // top-k choices differ, so the tile walks the UNION of the 8 selections (ascending) and each
 // row masks the blocks its token did not choose.  Executed FLOPs exceed the algorithmic ones by
-// the union overhead; the sum over the selected keys of each row is exact.
+// the union overhead; the sum over each row's own selected keys is exact.
 //
-// Per union block u (64 keys of the group's K/V, one TMA box per 64 columns):
-//   S_u  = Q K_u^T            M=128 N=64  K=128, A and B from shared memory -> TMEM (fp32)
-//   P_u  = online softmax of S_u, rows masked by selection and causality      (registers)
-//   O   += P_u V_u            M=128 N=128 K=64,  A = P_u from TMEM (bf16, aliasing S_u), B = V
-// S is double-buffered in TMEM so S_{u+1} runs on the tensor core while the softmax warps
-// process S_u.  O is rescaled only when a row's running max grows by more than 2^8 (the stale
-// max keeps exp2 below 256, far from overflow, and cancels in O / l).
+// The union is consumed two blocks at a time (a "pair", 128 keys):
+//   S    = Q [K_a; K_b]^T        M=128 N=128 K=128  (one MMA; the two K tiles sit back to back
+//                                                    in shared memory, so Q is read once)
+//   P    = online softmax of S, masked per row by each block's selection bit and, on the
+//          diagonal block, by causality                              (registers, fp32)
+//   O   += P [V_a; V_b]          M=128 N=128 K=128  (A = P from TMEM, bf16, aliasing S)
+// S is double-buffered in TMEM so the next pair's S runs on the tensor core while the softmax
+// warps work on this one.  O is rescaled only when a row's running max grows by more than 8 in
+// log2 units (the stale max keeps exp2 below 256 and cancels in O / l).
 //
 // Roles (192 threads, persistent: one CTA per SM walks tiles blockIdx.x, +gridDim.x, ...):
-// warps 0-3 softmax + epilogue (thread = row = TMEM lane); warp 4 builds the next tile's union
-// list and issues the TMA loads; warp 5 allocates TMEM and issues the MMAs (one thread).
-// Every wait is bounded; a timeout sets the status word, the roles wind down, and the kernel
-// waits (bounded) for its own copies and MMAs before it frees TMEM and returns.
+// warps 0-3 softmax + epilogue (thread = row = TMEM lane); warp 4 stages the next tile's
+// selection rows in shared memory with coalesced loads, merges them into the union list and
+// issues the TMA loads; warp 5 allocates TMEM and issues the MMAs (one thread).  Every wait is
+// bounded; a timeout sets the status word, the roles wind down, and the kernel waits (bounded)
+// for its own copies and MMAs before it frees TMEM and returns.
 #include "kernels.h"
 #include "ptx.cuh"
 #include "tmap.cuh"
@@ -34,28 +37,28 @@ constexpr int kD = 128;          // head dim
 constexpr int kG = 16;           // query heads per KV group
 constexpr int kTQ = 8;           // query tokens per tile
 constexpr int kBlk = 64;         // keys per block
-constexpr int kStages = 3;       // K/V pipeline depth
-constexpr int kMaxList = 1024;   // union capacity (8 x slots, slots <= 128)
+constexpr int kMaxSlots = 128;   // selection slots per row the kernel accepts
+constexpr int kMaxList = kTQ * kMaxSlots;
 constexpr int kThreads = 192;
 
-// Shared memory layout (offsets from a 1024-aligned base).
-constexpr int kQBytes = 128 * kD * 2;                 // 32 KiB: 2 sub-tiles [128 x 128 B]
-constexpr int kKBytes = kBlk * kD * 2;                // 16 KiB: 2 sub-tiles [64 x 128 B]
-constexpr int kVBytes = kBlk * kD * 2;                // 16 KiB: 2 sub-tiles [64 x 128 B]
+// Shared memory (offsets from a 1024-aligned base).
+constexpr int kQBytes = 128 * kD * 2;                 // 2 sub-tiles [128 rows x 128 B]
+constexpr int kHalfK = 8192;                          // one K box: [64 rows x 128 B]
+constexpr int kPairBytes = 8 * kHalfK;                // K_a|K_b (d 0-63), K_a|K_b (d 64-127), V_a, V_b
 constexpr int kOffQ = 0;
-constexpr int kOffKV = kOffQ + kQBytes;
-constexpr int kStageBytes = kKBytes + kVBytes;
-constexpr int kOffList = kOffKV + kStages * kStageBytes;   // 2 x kMaxList int32 + 2 x kMaxList u8
-constexpr int kListBytes = kMaxList * 5;
-constexpr int kSmemBytes = kOffList + 2 * kListBytes + 1024;
+constexpr int kOffKV = kQBytes;
+constexpr int kOffList = kOffKV + 2 * kPairBytes;
+constexpr int kListBytes = kMaxList * 5;              // int32 ids + uint8 token masks
+constexpr int kOffStage = kOffList + 2 * kListBytes;  // staged selection rows of one tile
+constexpr int kSmemBytes = kOffStage + kTQ * kMaxSlots * 4 + 1024;
 
-// TMEM columns: O [0,128), S buffers [128,192) and [192,256).
-constexpr uint32_t kTmemCols = 256;
+// TMEM columns: O [0,128), S buffers [128,256) and [256,384).
+constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 0, kColS0 = 128;
 
 struct Bars {
     uint64_t q_full, q_empty;
-    uint64_t kv_full[kStages], kv_empty[kStages];
+    uint64_t kv_full[2], kv_empty[2];
     uint64_t s_full[2], p_full[2], pv_done[2];
     uint64_t list_full[2], list_empty[2];
     uint64_t fin;
@@ -80,12 +83,41 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, co
     return true;
 }
 
+// Max of 64 values held as raw fp32 bit patterns, 8 independent chains.
+__device__ __forceinline__ float max64(const uint32_t* x) {
+    float m[8];
+#pragma unroll
+    for (int a = 0; a < 8; ++a) m[a] = __uint_as_float(x[a]);
+#pragma unroll
+    for (int j = 8; j < 64; j += 8)
+#pragma unroll
+        for (int a = 0; a < 8; ++a) m[a] = fmaxf(m[a], __uint_as_float(x[j + a]));
+    return fmaxf(fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3])), fmaxf(fmaxf(m[4], m[5]), fmaxf(m[6], m[7])));
+}
+
+// Softmax numerators of one 64-key half: p = 2^(x * sl2 - m), packed to bf16 pairs; returns the
+// sum of the fp32 p.  Keys j > lim are masked (lim = 63: none).
+__device__ __forceinline__ float exp_half(const uint32_t* x, float sl2, float neg_m, int lim,
+                                          uint32_t* pk) {
+    float s[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+        float p0 = ex2(fmaf(__uint_as_float(x[2 * j]), sl2, neg_m));
+        float p1 = ex2(fmaf(__uint_as_float(x[2 * j + 1]), sl2, neg_m));
+        p0 = (2 * j <= lim) ? p0 : 0.f;
+        p1 = (2 * j + 1 <= lim) ? p1 : 0.f;
+        s[j & 3] += p0 + p1;
+        pk[j] = pack_bf16x2(p0, p1);
+    }
+    return (s[0] + s[1]) + (s[2] + s[3]);
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 sparse_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                          const __grid_constant__ CUtensorMap tmK,
                          const __grid_constant__ CUtensorMap tmV,
                          const int32_t* __restrict__ idx, __nv_bfloat16* __restrict__ out, int H,
-                         int Hkv, int N, int slots, float scale_log2, int n_tiles, DevCtx ctx) {
+                         int Hkv, int N, int slots, float sl2, int n_tiles, DevCtx ctx) {
     extern __shared__ uint8_t smraw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smraw) + 1023) &
                                              ~uintptr_t(1023));
@@ -101,11 +133,9 @@ sparse_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
     if (tid == 0) {
         mbar_init(&bars.q_full, 1);
         mbar_init(&bars.q_empty, 1);
-        for (int s = 0; s < kStages; ++s) {
-            mbar_init(&bars.kv_full[s], 1);
-            mbar_init(&bars.kv_empty[s], 1);
-        }
         for (int b = 0; b < 2; ++b) {
+            mbar_init(&bars.kv_full[b], 1);
+            mbar_init(&bars.kv_empty[b], 1);
             mbar_init(&bars.s_full[b], 1);
             mbar_init(&bars.p_full[b], 4);
             mbar_init(&bars.pv_done[b], 1);
@@ -126,20 +156,24 @@ sparse_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
 
     if (warp == 4) {
         // ---------------------------------------------------------------- producer
-        int it = 0;     // tile iteration of this CTA
-        int gblk = 0;   // global block counter (pipeline position)
+        int32_t* stage = reinterpret_cast<int32_t*>(sm + kOffStage);
+        int it = 0, gp = 0;
         uint32_t q_issued = 0;
-        int last_phase[kStages];
-        for (int s = 0; s < kStages; ++s) last_phase[s] = -1;
+        int last_phase[2] = {-1, -1};
         for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
             const int lb = it & 1;
             if (it >= 2 && !wait_or_abort(&bars.list_empty[lb], ((it - 2) >> 1) & 1, ctx, abort)) break;
             const int64_t bg = tile / tiles_per_seq;
             const int i0 = (tile % tiles_per_seq) * kTQ;
             const int c = i0 / kBlk;
-            // Union of the (up to) 8 tokens' ascending selections: 8-way merge, one lane per token.
-            const int32_t* row = idx + (bg * N + i0 + lane) * (int64_t)slots;
-            const bool active = lane < kTQ && i0 + lane < N;
+            const int n_act = min(kTQ, N - i0);
+            // Stage the tile's selection rows (contiguous in memory) with coalesced loads.
+            const int32_t* src = idx + (bg * N + i0) * (int64_t)slots;
+            for (int e = lane; e < n_act * slots; e += 32) stage[e] = src[e];
+            __syncwarp();
+            // 8-way merge of the ascending rows, one lane per token.
+            const int32_t* row = stage + lane * slots;
+            const bool active = lane < n_act;
             int p = 0, n = 0, prev = -1;
             while (true) {
                 int head = 0x7fffffff;
@@ -151,7 +185,7 @@ sparse_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                 if (m == 0x7fffffff) break;
                 const unsigned msk = __ballot_sync(0xffffffffu, head == m);
                 if (head == m) ++p;
-                if (m > c) {  // a block in the future of every token of the tile
+                if (m > c) {  // in the future of every token of the tile
                     if (lane == 0) flag(ctx, kStatusBounds);
                     continue;
                 }
@@ -169,77 +203,82 @@ sparse_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
             }
             if (lane == 0) {
                 bars.list_n[lb] = n;
-                mbar_arrive(&bars.list_full[lb]);  // release: list writes precede the arrive
+                mbar_arrive(&bars.list_full[lb]);
             }
             __syncwarp();
-            if (lane == 0) {
-                // Q tile: 16 heads x 8 tokens x 128 columns (two boxes of 64 columns).
-                if (it >= 1 && !wait_or_abort(&bars.q_empty, (it - 1) & 1, ctx, abort)) break;
+            int stop = 0;
+            if (lane == 0 && it >= 1 && !wait_or_abort(&bars.q_empty, (it - 1) & 1, ctx, abort)) stop = 1;
+            if (lane == 0 && !stop) {
                 mbar_arrive_expect_tx(&bars.q_full, kQBytes);
                 const int z = (int)((bg / Hkv) * H + (bg % Hkv) * kG);
                 tma_load_3d(sm + kOffQ, &tmQ, &bars.q_full, 0, i0, z);
                 tma_load_3d(sm + kOffQ + kQBytes / 2, &tmQ, &bars.q_full, 64, i0, z);
                 q_issued = it + 1;
-                for (int u = 0; u < n; ++u, ++gblk) {
-                    const int s = gblk % kStages;
-                    const int r = gblk / kStages;
+                for (int u = 0; u < n; u += 2, ++gp) {
+                    const int s = gp & 1, r = gp >> 1;
                     if (r >= 1 && !wait_or_abort(&bars.kv_empty[s], (r - 1) & 1, ctx, abort)) break;
-                    const int blk = list_id[lb][u];
-                    uint8_t* st = sm + kOffKV + s * kStageBytes;
-                    mbar_arrive_expect_tx(&bars.kv_full[s], kStageBytes);
-                    tma_load_3d(st, &tmK, &bars.kv_full[s], 0, blk * kBlk, (int)bg);
-                    tma_load_3d(st + kKBytes / 2, &tmK, &bars.kv_full[s], 64, blk * kBlk, (int)bg);
-                    tma_load_3d(st + kKBytes, &tmV, &bars.kv_full[s], 0, blk * kBlk, (int)bg);
-                    tma_load_3d(st + kKBytes + kVBytes / 2, &tmV, &bars.kv_full[s], 64, blk * kBlk, (int)bg);
+                    const int nb = min(2, n - u);
+                    uint8_t* st = sm + kOffKV + s * kPairBytes;
+                    mbar_arrive_expect_tx(&bars.kv_full[s], nb * 4 * kHalfK);
+                    for (int e = 0; e < nb; ++e) {
+                        const int y = list_id[lb][u + e] * kBlk;
+                        tma_load_3d(st + e * kHalfK, &tmK, &bars.kv_full[s], 0, y, (int)bg);
+                        tma_load_3d(st + 2 * kHalfK + e * kHalfK, &tmK, &bars.kv_full[s], 64, y, (int)bg);
+                        tma_load_3d(st + 4 * kHalfK + e * 2 * kHalfK, &tmV, &bars.kv_full[s], 0, y, (int)bg);
+                        tma_load_3d(st + 5 * kHalfK + e * 2 * kHalfK, &tmV, &bars.kv_full[s], 64, y, (int)bg);
+                    }
                     last_phase[s] = r;
                 }
             }
-            gblk = __shfl_sync(0xffffffffu, gblk, 0);
-            if (*abort) break;
+            gp = __shfl_sync(0xffffffffu, gp, 0);
+            stop = __shfl_sync(0xffffffffu, stop, 0);
+            if (stop || *abort) break;
         }
-        // Wind down: wait (bounded) for every copy this warp issued.
         if (lane == 0) {
             if (q_issued) (void)mbar_wait(&bars.q_full, (q_issued - 1) & 1, ctx);
-            for (int s = 0; s < kStages; ++s)
+            for (int s = 0; s < 2; ++s)
                 if (last_phase[s] >= 0) (void)mbar_wait(&bars.kv_full[s], last_phase[s] & 1, ctx);
         }
     } else if (warp == 5) {
         // ---------------------------------------------------------------- MMA issuer
         if (lane == 0) {
-            const uint32_t idS = idesc_bf16_f32(128, kBlk, false, false);
+            const uint32_t idS2 = idesc_bf16_f32(128, 128, false, false);
+            const uint32_t idS1 = idesc_bf16_f32(128, 64, false, false);
             const uint32_t idPV = idesc_bf16_f32(128, kD, false, true);
             const uint32_t q0 = smem_u32(sm + kOffQ);
-            int it = 0, gblk = 0;
+            int it = 0, gp = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, ++it) {
                 const int lb = it & 1;
                 ok = wait_or_abort(&bars.list_full[lb], (it >> 1) & 1, ctx, abort);
                 if (!ok) break;
                 const int n = bars.list_n[lb];
+                const int np = (n + 1) >> 1;
                 mbar_arrive(&bars.list_empty[lb]);
                 ok = wait_or_abort(&bars.q_full, it & 1, ctx, abort);
                 if (!ok) break;
                 tc_fence_after();
-                auto issue_s = [&](int g) -> bool {
-                    const int s = g % kStages;
-                    if (!wait_or_abort(&bars.kv_full[s], (g / kStages) & 1, ctx, abort)) return false;
+                auto issue_s = [&](int j, int g) -> bool {
+                    const int s = g & 1;
+                    if (!wait_or_abort(&bars.kv_full[s], (g >> 1) & 1, ctx, abort)) return false;
                     tc_fence_after();
-                    const uint32_t kb = smem_u32(sm + kOffKV + s * kStageBytes);
-                    const uint32_t dS = tmem + kColS0 + (g & 1) * 64;
+                    const uint32_t kb = smem_u32(sm + kOffKV + s * kPairBytes);
+                    const uint32_t dS = tmem + kColS0 + s * 128;
+                    const uint32_t id = (2 * j + 1 < n) ? idS2 : idS1;
 #pragma unroll
                     for (int ks = 0; ks < kD / 16; ++ks) {
                         const uint64_t a = sdesc_sw128(q0 + (ks >> 2) * (kQBytes / 2) + (ks & 3) * 32, 16, 1024);
-                        const uint64_t b = sdesc_sw128(kb + (ks >> 2) * (kKBytes / 2) + (ks & 3) * 32, 16, 1024);
-                        mma_ss(dS, a, b, idS, ks > 0);
+                        const uint64_t b = sdesc_sw128(kb + (ks >> 2) * 2 * kHalfK + (ks & 3) * 32, 16, 1024);
+                        mma_ss(dS, a, b, id, ks > 0);
                     }
-                    mma_commit(&bars.s_full[g & 1]);
+                    mma_commit(&bars.s_full[s]);
                     return true;
                 };
-                if (n > 0) ok = issue_s(gblk);
-                for (int u = 0; u < n && ok; ++u) {
-                    const int g = gblk + u;
-                    if (u + 1 < n) {
-                        ok = issue_s(g + 1);
+                if (np > 0) ok = issue_s(0, gp);
+                for (int j = 0; j < np && ok; ++j) {
+                    const int g = gp + j;
+                    if (j + 1 < np) {
+                        ok = issue_s(j + 1, g + 1);
                         if (!ok) break;
                     } else {
                         mma_commit(&bars.q_empty);  // every S MMA of the tile has been issued
@@ -247,69 +286,79 @@ sparse_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                     ok = wait_or_abort(&bars.p_full[g & 1], (g >> 1) & 1, ctx, abort);
                     if (!ok) break;
                     tc_fence_after();
-                    const int s = g % kStages;
-                    const uint32_t vb = smem_u32(sm + kOffKV + s * kStageBytes + kKBytes);
-                    const uint32_t aP = tmem + kColS0 + (g & 1) * 64;
-#pragma unroll
-                    for (int ks = 0; ks < kBlk / 16; ++ks) {
-                        const uint64_t b = sdesc_sw128(vb + ks * 16 * 128, kVBytes / 2, 1024);
-                        mma_ts(tmem + kColO, aP + ks * 8, b, idPV, (u > 0 || ks > 0) ? 1u : 0u);
+                    const int s = g & 1;
+                    const uint32_t vb = smem_u32(sm + kOffKV + s * kPairBytes + 4 * kHalfK);
+                    const uint32_t aP = tmem + kColS0 + s * 128;
+                    const int ksteps = (2 * j + 1 < n) ? 8 : 4;
+                    for (int ks = 0; ks < ksteps; ++ks) {
+                        const uint64_t b = sdesc_sw128(vb + (ks >> 2) * 2 * kHalfK + (ks & 3) * 16 * 128, kHalfK, 1024);
+                        mma_ts(tmem + kColO, aP + ks * 8, b, idPV, (j > 0 || ks > 0) ? 1u : 0u);
                     }
                     mma_commit(&bars.kv_empty[s]);
-                    mma_commit(&bars.pv_done[g & 1]);
+                    mma_commit(&bars.pv_done[s]);
                 }
-                if (n == 0) mma_commit(&bars.q_empty);
-                gblk += n;
+                if (np == 0) mma_commit(&bars.q_empty);
+                gp += np;
             }
-            // Drain: every MMA this thread issued has completed before TMEM is released.
             mma_commit(&bars.fin);
             (void)mbar_wait(&bars.fin, 0, ctx);
         }
         __syncwarp();
     } else if (warp < 4) {
         // ---------------------------------------------------------------- softmax + epilogue
-        const int r = tid;                  // row = TMEM lane
+        const int r = tid;
         const int t = r % kTQ, hh = r / kTQ;
         const uint32_t lane_base = tmem_lane_base(warp);
-        int it = 0, gblk = 0;
+        int it = 0, gp = 0;
         for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
             const int lb = it & 1;
             if (!wait_or_abort(&bars.list_full[lb], (it >> 1) & 1, ctx, abort)) break;
             const int n = bars.list_n[lb];
+            const int np = (n + 1) >> 1;
             const int64_t bg = tile / tiles_per_seq;
             const int i0 = (tile % tiles_per_seq) * kTQ;
             const int c = i0 / kBlk;
             const int i = i0 + t;
-            float m_run = -INFINITY, l = 0.f;
-            bool o_live = false;  // O holds an accumulated value for this tile
+            float m_run = -INFINITY, l = 0.f;  // m_run in scaled log2 units
             bool ok = true;
-            for (int u = 0; u < n; ++u) {
-                const int g = gblk + u;
-                const int blk = list_id[lb][u];
-                const bool sel = (list_mask[lb][u] >> t) & 1;
-                if (!wait_or_abort(&bars.s_full[g & 1], (g >> 1) & 1, ctx, abort)) { ok = false; break; }
+            for (int j = 0; j < np; ++j) {
+                const int g = gp + j, s = g & 1;
+                const bool two = 2 * j + 1 < n;
+                const int blk_a = list_id[lb][2 * j];
+                const int blk_b = two ? list_id[lb][2 * j + 1] : -1;
+                const bool sel_a = (list_mask[lb][2 * j] >> t) & 1;
+                const bool sel_b = two && ((list_mask[lb][2 * j + 1] >> t) & 1);
+                // last visible key of each half (-1: none)
+                const int lim_a = !sel_a ? -1 : (blk_a == c ? i - blk_a * kBlk : kBlk - 1);
+                const int lim_b = !sel_b ? -1 : (blk_b == c ? i - blk_b * kBlk : kBlk - 1);
+                if (!wait_or_abort(&bars.s_full[s], (g >> 1) & 1, ctx, abort)) { ok = false; break; }
                 tc_fence_after();
-                const uint32_t colS = tmem + lane_base + kColS0 + (g & 1) * 64;
-                uint32_t sr[64];
-                tmem_ld32(colS, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-                tmem_ld32(colS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-                tmem_ld_wait();
-                const int lim = (blk == c) ? (i - blk * kBlk) : (kBlk - 1);  // last visible key
-                float mx = -INFINITY;
-#pragma unroll
-                for (int j = 0; j < 64; ++j) {
-                    float x = __uint_as_float(sr[j]) * scale_log2;
-                    x = (sel && j <= lim) ? x : -INFINITY;
-                    sr[j] = __float_as_uint(x);
-                    mx = fmaxf(mx, x);
+                const uint32_t colS = tmem + lane_base + kColS0 + s * 128;
+                uint32_t xa[64], xb[64];
+                tmem_ld32(colS, *reinterpret_cast<uint32_t(*)[32]>(&xa[0]));
+                tmem_ld32(colS + 32, *reinterpret_cast<uint32_t(*)[32]>(&xa[32]));
+                if (two) {
+                    tmem_ld32(colS + 64, *reinterpret_cast<uint32_t(*)[32]>(&xb[0]));
+                    tmem_ld32(colS + 96, *reinterpret_cast<uint32_t(*)[32]>(&xb[32]));
                 }
-                // Stale-max online softmax: rescale only when the max grows by more than 8.
+                tmem_ld_wait();
+                // Row max in raw units over the visible keys (diagonal block: masked first).
+                if (lim_a >= 0 && lim_a < kBlk - 1)
+#pragma unroll
+                    for (int jj = 0; jj < 64; ++jj) xa[jj] = jj <= lim_a ? xa[jj] : __float_as_uint(-INFINITY);
+                if (lim_b >= 0 && lim_b < kBlk - 1)
+#pragma unroll
+                    for (int jj = 0; jj < 64; ++jj) xb[jj] = jj <= lim_b ? xb[jj] : __float_as_uint(-INFINITY);
+                float mx = -INFINITY;
+                if (lim_a >= 0) mx = max64(xa);
+                if (lim_b >= 0) mx = fmaxf(mx, max64(xb));
+                mx *= sl2;
                 const bool grow = mx > m_run + 8.f;
-                const bool need_rescale = grow && o_live && l > 0.f;
+                const bool need_rescale = grow && l > 0.f;
                 if (__any_sync(0xffffffffu, need_rescale)) {
-                    if (u >= 1) {
-                        const int gp = g - 1;
-                        if (!wait_or_abort(&bars.pv_done[gp & 1], (gp >> 1) & 1, ctx, abort)) { ok = false; break; }
+                    if (j >= 1) {
+                        const int gq = g - 1;
+                        if (!wait_or_abort(&bars.pv_done[gq & 1], (gq >> 1) & 1, ctx, abort)) { ok = false; break; }
                     }
                     tc_fence_after();
                     const float alpha = need_rescale ? ex2(m_run - mx) : 1.f;
@@ -319,7 +368,7 @@ sparse_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                         tmem_ld32(tmem + lane_base + kColO + c0, orr);
                         tmem_ld_wait();
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) orr[j] = __float_as_uint(__uint_as_float(orr[j]) * alpha);
+                        for (int q = 0; q < 32; ++q) orr[q] = __float_as_uint(__uint_as_float(orr[q]) * alpha);
                         tmem_st16(tmem + lane_base + kColO + c0, *reinterpret_cast<uint32_t(*)[16]>(&orr[0]));
                         tmem_st16(tmem + lane_base + kColO + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&orr[16]));
                     }
@@ -329,33 +378,41 @@ sparse_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                     l = (m_run == -INFINITY) ? 0.f : l * ex2(m_run - mx);
                     m_run = mx;
                 }
-                uint32_t pk[32];
+                uint32_t pk[64];
                 float ps = 0.f;
+                if (lim_a >= 0) {
+                    ps += exp_half(xa, sl2, -m_run, lim_a, pk);
+                } else {
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const float x0 = __uint_as_float(sr[2 * j]), x1 = __uint_as_float(sr[2 * j + 1]);
-                    const float p0 = (x0 == -INFINITY) ? 0.f : ex2(x0 - m_run);
-                    const float p1 = (x1 == -INFINITY) ? 0.f : ex2(x1 - m_run);
-                    ps += p0 + p1;
-                    pk[j] = pack_bf16x2(p0, p1);
+                    for (int q = 0; q < 32; ++q) pk[q] = 0u;
+                }
+                if (two) {
+                    if (lim_b >= 0) {
+                        ps += exp_half(xb, sl2, -m_run, lim_b, pk + 32);
+                    } else {
+#pragma unroll
+                        for (int q = 32; q < 64; ++q) pk[q] = 0u;
+                    }
                 }
                 l += ps;
-                o_live = true;
                 tmem_st16(colS, *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
                 tmem_st16(colS + 16, *reinterpret_cast<uint32_t(*)[16]>(&pk[16]));
+                if (two) {
+                    tmem_st16(colS + 32, *reinterpret_cast<uint32_t(*)[16]>(&pk[32]));
+                    tmem_st16(colS + 48, *reinterpret_cast<uint32_t(*)[16]>(&pk[48]));
+                }
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&bars.p_full[g & 1]);
+                if (lane == 0) mbar_arrive(&bars.p_full[s]);
             }
             if (!ok) break;
-            // Epilogue: O / l -> bf16 -> global.
-            if (n > 0) {
-                const int gl = gblk + n - 1;
+            const int64_t orow = (((bg / Hkv) * H + (bg % Hkv) * kG + hh) * (int64_t)N + i) * kD;
+            if (np > 0) {
+                const int gl = gp + np - 1;
                 if (!wait_or_abort(&bars.pv_done[gl & 1], (gl >> 1) & 1, ctx, abort)) break;
                 tc_fence_after();
                 const float inv = l > 0.f ? 1.f / l : 0.f;
-                __nv_bfloat16* dst = out + (((bg / Hkv) * H + (bg % Hkv) * kG + hh) * (int64_t)N + i) * kD;
 #pragma unroll 1
                 for (int c0 = 0; c0 < kD; c0 += 32) {
                     uint32_t orr[32];
@@ -365,21 +422,20 @@ sparse_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                         uint4 w[4];
                         uint32_t* wp = reinterpret_cast<uint32_t*>(w);
 #pragma unroll
-                        for (int j = 0; j < 16; ++j)
-                            wp[j] = pack_bf16x2(__uint_as_float(orr[2 * j]) * inv,
-                                                __uint_as_float(orr[2 * j + 1]) * inv);
-                        uint4* d4 = reinterpret_cast<uint4*>(dst + c0);
+                        for (int q = 0; q < 16; ++q)
+                            wp[q] = pack_bf16x2(__uint_as_float(orr[2 * q]) * inv,
+                                                __uint_as_float(orr[2 * q + 1]) * inv);
+                        uint4* d4 = reinterpret_cast<uint4*>(out + orow + c0);
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) d4[j] = w[j];
+                        for (int q = 0; q < 4; ++q) d4[q] = w[q];
                     }
                 }
                 tc_fence_before();
             } else if (i < N) {
-                __nv_bfloat16* dst = out + (((bg / Hkv) * H + (bg % Hkv) * kG + hh) * (int64_t)N + i) * kD;
-                for (int j = 0; j < kD; ++j) dst[j] = __float2bfloat16_rn(0.f);
+                uint4* d4 = reinterpret_cast<uint4*>(out + orow);
+                for (int q = 0; q < kD / 8; ++q) d4[q] = make_uint4(0, 0, 0, 0);
             }
-            gblk += n;
-            // All four softmax warps are done with this list and with O.
+            gp += np;
             asm volatile("bar.sync 1, 128;" ::: "memory");
             if (tid == 0) mbar_arrive(&bars.list_empty[lb]);
         }
@@ -401,7 +457,7 @@ bool sparse_prefill_tc_supported(int H, int Hkv, int d) {
 cudaError_t launch_sparse_prefill_tc(const void* q, const void* k, const void* v,
                                      const int32_t* idx, void* o, int B, int H, int Hkv, int N,
                                      int d, int slots, float scale, cudaStream_t st, DevCtx ctx) {
-    if (d != kD || H != Hkv * kG || slots > kMaxList / kTQ) return cudaErrorNotSupported;
+    if (d != kD || H != Hkv * kG || slots > kMaxSlots) return cudaErrorNotSupported;
     CUtensorMap tmQ, tmK, tmV;
     EncodeTiledFn fn = encode_tiled_fn();
     if (!fn) return cudaErrorNotSupported;
@@ -426,16 +482,14 @@ cudaError_t launch_sparse_prefill_tc(const void* q, const void* k, const void* v
         cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
         if (num_sms <= 0) num_sms = 148;
     }
-    cudaError_t e = cudaFuncSetAttribute(sparse_prefill_tc_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    cudaError_t e = ensure_smem<sparse_prefill_tc_kernel>(kSmemBytes);
     if (e != cudaSuccess) return e;
     const int tiles_per_seq = (N + kTQ - 1) / kTQ;
     const int n_tiles = tiles_per_seq * B * Hkv;
     const int grid = n_tiles < num_sms ? n_tiles : num_sms;
-    const float scale_log2 = scale * 1.4426950408889634f;
+    const float sl2 = scale * 1.4426950408889634f;
     sparse_prefill_tc_kernel<<<grid, kThreads, kSmemBytes, st>>>(
-        tmQ, tmK, tmV, idx, static_cast<__nv_bfloat16*>(o), H, Hkv, N, slots, scale_log2, n_tiles,
-        ctx);
+        tmQ, tmK, tmV, idx, static_cast<__nv_bfloat16*>(o), H, Hkv, N, slots, sl2, n_tiles, ctx);
     return cudaGetLastError();
 }
 

@@ -137,7 +137,9 @@ size_t sala_block_topk_workspace(int B, int Hkv, int Nq, int q_pos0, int nb, int
  * idx  : [B, Hkv, N, slots] int32 device, each row ascending and -1 padded (sala_block_topk's
  *        output); entries must lie in [0, (N-1)/block].  An out-of-range entry is skipped and
  *        flagged SALA_ERR_BOUNDS in the status word.
- * scale: softmax scale; 0 selects 1/sqrt(d).   block 64; d 64 or 128 (bf16 tensor cores: 128).
+ * scale: softmax scale; 0 selects 1/sqrt(d).   block 64; d 64 or 128; H / Hkv <= 16.
+ *        bf16 with H / Hkv = 16 and d = 128 runs on the tensor cores; other shapes and fp32 run
+ *        on CUDA cores.
  */
 sala_status sala_sparse_prefill(const void* q, const void* k, const void* v, const int32_t* idx,
                                 void* o, int B, int H, int Hkv, int N, int d, int block,
