@@ -337,8 +337,10 @@ def run_decode(sala, synth, torch, steps, warmup, stream):
 
 def run_e2e(sala, synth, torch, steps, warmup):
     """Prefill step with every layer's inputs streamed from pinned host memory and the outputs
-    copied back, through the same calls.  One pinned host copy of a linear and of a sparse layer
-    is streamed for every layer of its kind (host RAM cannot hold 164 GiB of distinct inputs)."""
+    copied back, through the same calls.  Copies run on their own streams into double-buffered
+    device inputs, so the host->device copy of layer l+1 and the device->host copy of layer l-1
+    overlap the kernels of layer l.  One pinned host copy of a linear and of a sparse layer is
+    streamed for every layer of its kind (host RAM cannot hold 164 GiB of distinct inputs)."""
     dev = torch.device("cuda")
     lam = synth.decays(H).to(dev)
     ql, kl, vl = synth.linear_layer(1, H, N_TOK, D, torch.bfloat16, dev, layer=0)
@@ -346,49 +348,72 @@ def run_e2e(sala, synth, torch, steps, warmup):
     host = {"linear": [t.cpu().pin_memory() for t in (ql, kl, vl)],
             "sparse": [t.cpu().pin_memory() for t in (sl.q, sl.k, sl.v)]}
     del ql, kl, vl, sl
-    dbuf = {"linear": [torch.empty((1, H, N_TOK, D), device=dev, dtype=torch.bfloat16) for _ in range(3)],
-            "sparse": [torch.empty((1, H, N_TOK, D), device=dev, dtype=torch.bfloat16),
-                       torch.empty((1, HKV, N_TOK, D), device=dev, dtype=torch.bfloat16),
-                       torch.empty((1, HKV, N_TOK, D), device=dev, dtype=torch.bfloat16)]}
-    out = torch.empty((1, H, N_TOK, D), device=dev, dtype=torch.bfloat16)
+    torch.cuda.empty_cache()
+    shape = {"linear": [(1, H, N_TOK, D)] * 3,
+             "sparse": [(1, H, N_TOK, D), (1, HKV, N_TOK, D), (1, HKV, N_TOK, D)]}
+    dbuf = {kind: [[torch.empty(sh, device=dev, dtype=torch.bfloat16) for sh in shape[kind]]
+                   for _ in range(2)] for kind in ("linear", "sparse")}
+    outs = [torch.empty((1, H, N_TOK, D), device=dev, dtype=torch.bfloat16) for _ in range(2)]
     out_host = torch.empty((1, H, N_TOK, D), dtype=torch.bfloat16).pin_memory()
     kbar = torch.empty((1, HKV, N_TOK // BLOCK, D), device=dev, dtype=torch.bfloat16)
     idx = torch.empty((1, HKV, N_TOK, N_INIT + N_LOCAL + TOPK), device=dev, dtype=torch.int32)
-    stream = torch.cuda.current_stream()
-    h2d = d2h = 0
+    s_h2d, s_cmp, s_d2h = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event()
+    counts = {"h2d": 0, "d2h": 0}
+    # per buffer slot: inputs copied / inputs consumed; per output slot: written / read back
+    in_ready = {k: [None, None] for k in dbuf}
+    in_free = {k: [None, None] for k in dbuf}
+    out_ready, out_free = [None, None], [None, None]
+    use = {"linear": 0, "sparse": 0}
 
     def step():
-        nonlocal h2d, d2h
         for l in range(N_LAYERS):
             kind = "sparse" if l in SPARSE_LAYERS else "linear"
-            for dst, src in zip(dbuf[kind], host[kind]):
-                dst.copy_(src, non_blocking=True)
-                h2d += src.numel() * 2
-            q, k, v = dbuf[kind]
-            if kind == "linear":
-                sala.linear_prefill(q, k, v, lam, o=out)
-            else:
-                sala.block_compress(k, kbar)
-                sala.block_topk(q, kbar, TOPK, N_INIT, N_LOCAL, idx=idx)
-                sala.sparse_prefill(q, k, v, idx, o=out)
-            out_host.copy_(out, non_blocking=True)
-            d2h += out.numel() * 2
+            slot = use[kind] & 1
+            use[kind] += 1
+            with torch.cuda.stream(s_h2d):
+                if in_free[kind][slot] is not None:
+                    s_h2d.wait_event(in_free[kind][slot])
+                for dst, src in zip(dbuf[kind][slot], host[kind]):
+                    dst.copy_(src, non_blocking=True)
+                    counts["h2d"] += src.numel() * 2
+                e = ev(); e.record(s_h2d); in_ready[kind][slot] = e
+            o = outs[l & 1]
+            with torch.cuda.stream(s_cmp):
+                s_cmp.wait_event(in_ready[kind][slot])
+                if out_free[l & 1] is not None:
+                    s_cmp.wait_event(out_free[l & 1])
+                q, k, v = dbuf[kind][slot]
+                if kind == "linear":
+                    sala.linear_prefill(q, k, v, lam, o=o, stream=s_cmp)
+                else:
+                    sala.block_compress(k, kbar, stream=s_cmp)
+                    sala.block_topk(q, kbar, TOPK, N_INIT, N_LOCAL, idx=idx, stream=s_cmp)
+                    sala.sparse_prefill(q, k, v, idx, o=o, stream=s_cmp)
+                e = ev(); e.record(s_cmp); in_free[kind][slot] = e; out_ready[l & 1] = e
+            with torch.cuda.stream(s_d2h):
+                s_d2h.wait_event(out_ready[l & 1])
+                out_host.copy_(o, non_blocking=True)
+                counts["d2h"] += o.numel() * 2
+                e = ev(); e.record(s_d2h); out_free[l & 1] = e
 
     for _ in range(warmup):
         step()
     torch.cuda.synchronize()
-    h2d = d2h = 0
+    counts["h2d"] = counts["d2h"] = 0
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(stream)
+    a.record(s_h2d)
+    s_cmp.wait_event(a); s_d2h.wait_event(a)
     for _ in range(steps):
         step()
-    b.record(stream)
+    s_d2h.wait_stream(s_h2d); s_d2h.wait_stream(s_cmp)
+    b.record(s_d2h)
     torch.cuda.synchronize()
-    sala.check_status()
+    sala.check_status(s_cmp)
     ms = a.elapsed_time(b) / steps
-    del host, dbuf, out, out_host, kbar, idx
+    del host, dbuf, outs, out_host, kbar, idx
     torch.cuda.empty_cache()
-    return {"ms_per_step": ms, "h2d": h2d // steps, "d2h": d2h // steps}
+    return {"ms_per_step": ms, "h2d": counts["h2d"] // steps, "d2h": counts["d2h"] // steps}
 
 
 # ----------------------------------------------------------------------------------------------
@@ -573,7 +598,8 @@ def main():
                        "unit": "tokens/s", "h2d_bytes_per_step": e["h2d"],
                        "d2h_bytes_per_step": e["d2h"],
                        "note": "per layer: pinned host -> device copy of Q/K/V, the layer's calls, "
-                               "device -> pinned host copy of O"}
+                               "device -> pinned host copy of O; copies on their own streams, "
+                               "overlapping the neighbouring layers' kernels"}
     if "cpu" in phases and rank == 0 and ws == 1:
         line["cpu_baseline"] = cpu_baseline(torch, synth)
     if rank == 0:

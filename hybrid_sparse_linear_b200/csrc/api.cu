@@ -252,6 +252,10 @@ sala_status sala_block_topk(const void* q, const void* kbar, int32_t* idx, int B
                                                         workspace, st, ctx),
                         "block_topk_rowwise");
     }
+    if (dt == SALA_BF16 && sala::block_topk_tc_supported(H, Hkv, Nq, q_pos0, nb, d, topk))
+        return launched(sala::launch_block_topk_tc(q, kbar, idx, B, H, Hkv, Nq, nb, topk, n_init,
+                                                   n_local, st, ctx),
+                        "block_topk_tc");
     return launched(sala::launch_block_topk_tiled(to_dt(dt), q, kbar, idx, B, H, Hkv, Nq, q_pos0,
                                                   nb, d, topk, n_init, n_local, st, ctx),
                     "block_topk");

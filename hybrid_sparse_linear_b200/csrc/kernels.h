@@ -34,6 +34,11 @@ cudaError_t launch_block_topk_tiled(DType dt, const void* q, const void* kbar, i
                                     int B, int H, int Hkv, int Nq, int q_pos0, int nb, int d,
                                     int topk, int n_init, int n_local, cudaStream_t st,
                                     DevCtx ctx);
+// Tensor-core selection (bf16, d 128, prefill rows from position 0, topk <= 64).
+bool block_topk_tc_supported(int H, int Hkv, int Nq, int q_pos0, int nb, int d, int topk);
+cudaError_t launch_block_topk_tc(const void* q, const void* kbar, int32_t* idx, int B, int H,
+                                 int Hkv, int Nq, int nb, int topk, int n_init, int n_local,
+                                 cudaStream_t st, DevCtx ctx);
 // Row-wise selection for few query rows and many blocks: candidates split across CTAs, then a
 // merge.  Workspace = rowwise_topk_workspace(...) bytes.
 size_t rowwise_topk_workspace(int B, int Hkv, int Nq, int q_pos0, int topk);

@@ -16,9 +16,14 @@
 //   EPI-S V~   = diag(lambda^{len-1-s}) V_c   bf16 in SMEM (double-buffered)
 //   MMA4  dS   = K_c^T V~                     M=128 N=64  K=128   (A read transposed)
 //   EPI-S S    = lambda^len S + dS            fp32, one row of S per thread, in registers
-// The only serial dependency between tiles is the state: MMA3(c) needs Sb(c-1) and the update of
-// S(c) needs MMA4(c).  The MMA issuer therefore issues MMA3 and MMA4 of a tile first, then MMA2
-// and the next tile's MMA1, so the tensor core works on MMA2/MMA1 while the state warps update S.
+// The only serial dependency between tiles is the state: S(c) = lambda^len S(c-1) + dS(c), where
+// dS(c) needs no state at all.  The MMA issuer therefore computes dS one tile ahead (into a second
+// TMEM buffer): per tile it issues MMA3(c), MMA2(c) -- the last reader of stage c, which is then
+// released to the producer a full tile before it is needed again -- and MMA1(c+1), MMA4(c+1), so
+// the state warps find dS(c) already done and the tensor core always has independent work queued.
+// The bf16 state copy is double-buffered: Sb(c) lives in buffer (c+1)&1, MMA3(c) reads Sb(c-1)
+// from buffer c&1 and releases it through sb_free[c&1]; with one barrier per buffer no barrier
+// can run two phases ahead of its waiter.
 // Roles (320 threads): warps 0-3 "EPI-A" (mask + output, thread = row = TMEM lane), warps 4-7
 // "EPI-S" (V~ + state, thread = row of S), warp 8 TMA producer (2-stage ring of Q/K/V tiles),
 // warp 9 TMEM owner and MMA issuer.  Every wait is bounded (see ptx::mbar_wait).
@@ -37,15 +42,15 @@ constexpr int kSub = kC * 128;                    // one [128 rows x 128 B] sub-
 constexpr int kOffQ = 0, kOffK = 2 * kSub, kOffV = 4 * kSub;
 constexpr int kStageBytes = 5 * kSub;             // Q (2) + K (2) + V slice (1)
 constexpr int kOffVt = 2 * kStageBytes;           // V~ (decay-weighted V slice), 2 buffers
-constexpr int kOffSb = kOffVt + 2 * kSub;         // bf16 copy of the state slice
-constexpr int kSmemBytes = kOffSb + kSub + 1024;
+constexpr int kOffSb = kOffVt + 2 * kSub;         // bf16 copies of the state slice, 2 buffers
+constexpr int kSmemBytes = kOffSb + 2 * kSub + 1024;
 
-constexpr uint32_t kColA0 = 0, kColO1 = 256, kColO2 = 320, kColDS = 384, kTmemCols = 512;
+constexpr uint32_t kColA0 = 0, kColO1 = 256, kColO2 = 320, kColDS = 384, kTmemCols = 512;  // dS: 2 x 64
 
 struct Bars {
     uint64_t full[2], empty[2];
-    uint64_t qk_done[2], a_ready[2], v_ready[2];
-    uint64_t o_done, o_free, ds_done, s_ready, fin;
+    uint64_t qk_done[2], a_ready[2], v_ready[2], ds_done[2], s_ready[2], sb_free[2];
+    uint64_t o_done, o_free, fin;
     uint32_t tmem_base;
     int abort;
     float pw[kC + 1];  // lambda^n, n = 0..128
@@ -91,11 +96,12 @@ linear_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
             mbar_init(&bars.qk_done[b], 1);
             mbar_init(&bars.a_ready[b], 4);
             mbar_init(&bars.v_ready[b], 4);
+            mbar_init(&bars.ds_done[b], 1);
+            mbar_init(&bars.s_ready[b], 4);
+            mbar_init(&bars.sb_free[b], 1);
         }
         mbar_init(&bars.o_done, 1);
         mbar_init(&bars.o_free, 4);
-        mbar_init(&bars.ds_done, 1);
-        mbar_init(&bars.s_ready, 4);
         mbar_init(&bars.fin, 1);
         bars.abort = 0;
         fence_mbar_init();
@@ -136,7 +142,7 @@ linear_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
             const uint32_t idQK = idesc_bf16_f32(128, 128, false, false);
             const uint32_t idO = idesc_bf16_f32(128, kDv, false, true);
             const uint32_t idDS = idesc_bf16_f32(128, kDv, true, true);
-            const uint32_t sb = smem_u32(sm + kOffSb);
+            const uint32_t sb0 = smem_u32(sm + kOffSb);
             auto issue_qk = [&](int c) -> bool {
                 const int s = c & 1;
                 if (!wait_or_abort(&bars.full[s], (c >> 1) & 1, ctx, abort)) return false;
@@ -152,30 +158,38 @@ linear_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                 mma_commit(&bars.qk_done[s]);
                 return true;
             };
-            bool ok = n_tiles > 0 ? issue_qk(0) : true;
+            auto issue_ds = [&](int c) -> bool {  // MMA4: dS(c) = K^T V~  (A read transposed)
+                const int s = c & 1;
+                if (!wait_or_abort(&bars.full[s], (c >> 1) & 1, ctx, abort)) return false;
+                if (!wait_or_abort(&bars.v_ready[s], (c >> 1) & 1, ctx, abort)) return false;
+                tc_fence_after();
+                const uint32_t k = smem_u32(sm + s * kStageBytes + kOffK);
+                const uint32_t vt = smem_u32(sm + kOffVt + s * kSub);
+#pragma unroll
+                for (int ks = 0; ks < kC / 16; ++ks)
+                    mma_ss(tmem + kColDS + s * kDv, sdesc_sw128(k + ks * 16 * 128, kSub, 1024),
+                           sdesc_sw128(vt + ks * 16 * 128, 8192, 1024), idDS, ks > 0);
+                mma_commit(&bars.ds_done[s]);
+                return true;
+            };
+            bool ok = n_tiles > 0 ? (issue_qk(0) && issue_ds(0)) : true;
             for (int c = 0; c < n_tiles && ok; ++c) {
                 const int s = c & 1;
                 const uint32_t q = smem_u32(sm + s * kStageBytes + kOffQ);
-                const uint32_t k = smem_u32(sm + s * kStageBytes + kOffK);
                 const uint32_t v = smem_u32(sm + s * kStageBytes + kOffV);
-                const uint32_t vt = smem_u32(sm + kOffVt + s * kSub);
-                // MMA3: O2 = Q Sb(c-1)   (needs the state and a free O)
-                if (!wait_or_abort(&bars.s_ready, c & 1, ctx, abort)) break;
+                // MMA3: O2 = Q Sb(c-1), read from buffer c&1.  Sb(c-1) published also means
+                // dS(c-1) has been consumed, so its TMEM buffer is free for dS(c+1) below.
+                if (!wait_or_abort(&bars.s_ready[s], (c >> 1) & 1, ctx, abort)) break;
                 if (c >= 1 && !wait_or_abort(&bars.o_free, (c - 1) & 1, ctx, abort)) break;
                 tc_fence_after();
+                const uint32_t sb = sb0 + s * kSub;
 #pragma unroll
                 for (int ks = 0; ks < kD / 16; ++ks)
                     mma_ss(tmem + kColO2, sdesc_sw128(q + (ks >> 2) * kSub + (ks & 3) * 32, 16, 1024),
                            sdesc_sw128(sb + ks * 16 * 128, 8192, 1024), idO, ks > 0);
-                // MMA4: dS = K^T V~
-                if (!wait_or_abort(&bars.v_ready[s], (c >> 1) & 1, ctx, abort)) break;
-                tc_fence_after();
-#pragma unroll
-                for (int ks = 0; ks < kC / 16; ++ks)
-                    mma_ss(tmem + kColDS, sdesc_sw128(k + ks * 16 * 128, kSub, 1024),
-                           sdesc_sw128(vt + ks * 16 * 128, 8192, 1024), idDS, ks > 0);
-                mma_commit(&bars.ds_done);
-                // MMA2: O1 = A' V   (A' from TMEM)
+                mma_commit(&bars.sb_free[s]);
+                // MMA2: O1 = A' V   (A' from TMEM).  Last reader of stage c: release it so the
+                // producer can fetch tile c+2 while tile c+1 is being worked on.
                 if (!wait_or_abort(&bars.a_ready[s], (c >> 1) & 1, ctx, abort)) break;
                 tc_fence_after();
 #pragma unroll
@@ -184,8 +198,8 @@ linear_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                            sdesc_sw128(v + ks * 16 * 128, 8192, 1024), idO, ks > 0);
                 mma_commit(&bars.o_done);
                 mma_commit(&bars.empty[s]);
-                // MMA1 of the next tile
-                if (c + 1 < n_tiles) ok = issue_qk(c + 1);
+                // next tile: MMA1, then MMA4 (dS one tile ahead of the state update)
+                if (c + 1 < n_tiles) ok = issue_qk(c + 1) && issue_ds(c + 1);
             }
             mma_commit(&bars.fin);
             (void)mbar_wait(&bars.fin, 0, ctx);
@@ -265,8 +279,10 @@ linear_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
             float4 x = sin_row ? *reinterpret_cast<const float4*>(sin_row + j) : make_float4(0, 0, 0, 0);
             S[j] = x.x; S[j + 1] = x.y; S[j + 2] = x.z; S[j + 3] = x.w;
         }
-        uint8_t* sbrow = sm + kOffSb + t * 128;
-        auto write_sb = [&]() {  // bf16 copy of this thread's state row, 128-byte swizzle
+        // bf16 copy Sb(c) of this thread's state row (128-byte swizzle) into buffer (c+1)&1.
+        auto write_sb = [&](int c) {
+            const int b = (c + 1) & 1;
+            uint8_t* sbrow = sm + kOffSb + b * kSub + t * 128;
 #pragma unroll
             for (int cj = 0; cj < 8; ++cj) {
                 uint4 w;
@@ -278,50 +294,59 @@ linear_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
             }
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bars.s_ready);
+            if (lane == 0) mbar_arrive(&bars.s_ready[b]);
         };
-        write_sb();
-        bool ok = true;
+        // V~(c) = lambda^{len-1-s} V (row t of the V tile), same swizzled layout; the 16-byte
+        // chunks are visited in their physical order so a warp's 32 rows hit distinct banks.
+        auto make_vt = [&](int c) -> bool {
+            const int s = c & 1;
+            const int len = min(kC, N - c * kC);
+            if (!wait_or_abort(&bars.full[s], (c >> 1) & 1, ctx, abort)) return false;
+            const float w = t < len ? bars.pw[len - 1 - t] : 0.f;
+            const uint8_t* vrow = sm + s * kStageBytes + kOffV + t * 128;
+            uint8_t* vtrow = sm + kOffVt + s * kSub + t * 128;
+#pragma unroll
+            for (int cj = 0; cj < 8; ++cj) {
+                const int p = (cj ^ (t & 7)) << 4;
+                uint4 a = *reinterpret_cast<const uint4*>(vrow + p);
+                uint4 b;
+                b.x = pack_bf16x2(bf_lo(a.x) * w, bf_hi(a.x) * w);
+                b.y = pack_bf16x2(bf_lo(a.y) * w, bf_hi(a.y) * w);
+                b.z = pack_bf16x2(bf_lo(a.z) * w, bf_hi(a.z) * w);
+                b.w = pack_bf16x2(bf_lo(a.w) * w, bf_hi(a.w) * w);
+                *reinterpret_cast<uint4*>(vtrow + p) = b;
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars.v_ready[s]);
+            return true;
+        };
+        write_sb(-1);
+        bool ok = n_tiles > 0 ? make_vt(0) : true;
         for (int c = 0; c < n_tiles && ok; ++c) {
             const int s = c & 1;
             const int len = min(kC, N - c * kC);
-            // V~ = lambda^{len-1-s} V (row t of the V tile), same swizzled layout.
-            if (!wait_or_abort(&bars.full[s], (c >> 1) & 1, ctx, abort)) { ok = false; break; }
-            {
-                const float w = t < len ? bars.pw[len - 1 - t] : 0.f;
-                const uint8_t* vrow = sm + s * kStageBytes + kOffV + t * 128;
-                uint8_t* vtrow = sm + kOffVt + s * kSub + t * 128;
-#pragma unroll
-                for (int cj = 0; cj < 8; ++cj) {
-                    uint4 a = *reinterpret_cast<const uint4*>(vrow + cj * 16);
-                    uint4 b;
-                    b.x = pack_bf16x2(bf_lo(a.x) * w, bf_hi(a.x) * w);
-                    b.y = pack_bf16x2(bf_lo(a.y) * w, bf_hi(a.y) * w);
-                    b.z = pack_bf16x2(bf_lo(a.z) * w, bf_hi(a.z) * w);
-                    b.w = pack_bf16x2(bf_lo(a.w) * w, bf_hi(a.w) * w);
-                    *reinterpret_cast<uint4*>(vtrow + cj * 16) = b;
-                }
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bars.v_ready[s]);
-            }
-            // S <- lambda^len S + dS, then its bf16 copy for the next tile.
-            if (!wait_or_abort(&bars.ds_done, c & 1, ctx, abort)) { ok = false; break; }
+            if (c + 1 < n_tiles && !make_vt(c + 1)) { ok = false; break; }
+            // S <- lambda^len S + dS(c), then its bf16 copy for the next tile.
+            if (!wait_or_abort(&bars.ds_done[s], (c >> 1) & 1, ctx, abort)) { ok = false; break; }
             tc_fence_after();
-            {
-                uint32_t d0[32], d1[32];
-                tmem_ld32(tmem + lb + kColDS, d0);
-                tmem_ld32(tmem + lb + kColDS + 32, d1);
-                tmem_ld_wait();
-                const float decay_len = bars.pw[len];
+            uint32_t d0[32], d1[32];
+            tmem_ld32(tmem + lb + kColDS + s * kDv, d0);
+            tmem_ld32(tmem + lb + kColDS + s * kDv + 32, d1);
+            tmem_ld_wait();
+            const float decay_len = bars.pw[len];
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    S[j] = fmaf(decay_len, S[j], __uint_as_float(d0[j]));
-                    S[32 + j] = fmaf(decay_len, S[32 + j], __uint_as_float(d1[j]));
-                }
-                tc_fence_before();
-                write_sb();
+            for (int j = 0; j < 32; ++j) {
+                S[j] = fmaf(decay_len, S[j], __uint_as_float(d0[j]));
+                S[32 + j] = fmaf(decay_len, S[32 + j], __uint_as_float(d1[j]));
             }
+            tc_fence_before();
+            // Buffer (c+1)&1 last held Sb(c-2), read by MMA3(c-1): wait until that MMA is done.
+            if (c >= 1 && !wait_or_abort(&bars.sb_free[(c - 1) & 1], ((c - 1) >> 1) & 1, ctx, abort)) {
+                ok = false;
+                break;
+            }
+            write_sb(c);
         }
         if (ok && s_out) {
             float* row = s_out + (bh * kD + t) * kD + slice * kDv;

@@ -1,29 +1,33 @@
 // Block-sparse softmax attention prefill on the 5th-generation tensor cores (sm_100a).
 //
 // Work unit ("tile"): 8 consecutive query tokens x the 16 query heads of one KV group = 128 rows,
-// the M of one tcgen05 MMA.  Row r = head * 8 + token, so each head's 8 tokens are one 1024-byte
-// swizzle atom and the Q tile arrives with a single 3-D TMA box per 64 columns.  The 8 tokens
+// the M of one tcgen05 MMA (row r = head * 8 + token).  The Q tile lives in TMEM (A operand of the
+// S MMA), written one tile ahead by the softmax warps, so shared memory holds only K/V.  The 8 tokens
 // share their query block (8 divides 64), hence the forced blocks and the diagonal; their
 // top-k choices differ, so the tile walks the UNION of the 8 selections (ascending) and each
 // row masks the blocks its token did not choose.  Executed FLOPs exceed the algorithmic ones by
 // the union overhead; the sum over each row's own selected keys is exact.
 //
 // The union is consumed two blocks at a time (a "pair", 128 keys):
-//   S    = Q [K_a; K_b]^T        M=128 N=128 K=128  (one MMA; the two K tiles sit back to back
-//                                                    in shared memory, so Q is read once)
+//   S    = Q [K_a; K_b]^T        M=128 N=128 K=128  (A = Q from TMEM; the two K tiles sit back
+//                                                    to back in shared memory: one B operand)
 //   P    = online softmax of S, masked per row by each block's selection bit and, on the
 //          diagonal block, by causality                              (registers, fp32)
 //   O   += P [V_a; V_b]          M=128 N=128 K=128  (A = P from TMEM, bf16, aliasing S)
 // S is double-buffered in TMEM so the next pair's S runs on the tensor core while the softmax
-// warps work on this one.  O is rescaled only when a row's running max grows by more than 8 in
+// warps work on this one; K/V pairs stream through a 3-stage ring, so a pair's blocks are requested
+// two pairs before they are needed.  O is rescaled only when a row's running max grows by more than 8 in
 // log2 units (the stale max keeps exp2 below 256 and cancels in O / l).
 //
-// Roles (192 threads, persistent: one CTA per SM walks tiles blockIdx.x, +gridDim.x, ...):
-// warps 0-3 softmax + epilogue (thread = row = TMEM lane); warp 4 stages the next tile's
-// selection rows in shared memory with coalesced loads, merges them into the union list and
-// issues the TMA loads; warp 5 allocates TMEM and issues the MMAs (one thread).  Every wait is
-// bounded; a timeout sets the status word, the roles wind down, and the kernel waits (bounded)
-// for its own copies and MMAs before it frees TMEM and returns.
+// Roles (320 threads, persistent: one CTA per SM walks tiles blockIdx.x, +gridDim.x, ...):
+// warps 0-7 softmax + epilogue: warp w reads TMEM lanes 32(w%4).. (its 32 rows) and owns one
+// 64-key half of each pair (w < 4: the first block, w >= 4: the second), so every scheduler runs
+// two softmax warps; the two halves of a row exchange their maxima through shared memory and keep
+// one running max, two partial sums.  Warp 8 stages the next tile's selection rows in shared
+// memory with coalesced loads, merges them into the union list and issues the TMA loads; warp 9
+// allocates TMEM and issues the MMAs (one thread).  Every wait is bounded; a timeout sets the
+// status word, the roles wind down, and the kernel waits (bounded) for its own copies and MMAs
+// before it frees TMEM and returns.
 #include "kernels.h"
 #include "ptx.cuh"
 #include "tmap.cuh"
@@ -39,32 +43,35 @@ constexpr int kTQ = 8;           // query tokens per tile
 constexpr int kBlk = 64;         // keys per block
 constexpr int kMaxSlots = 128;   // selection slots per row the kernel accepts
 constexpr int kMaxList = kTQ * kMaxSlots;
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
+constexpr int kSoftmaxThreads = 256;
 
 // Shared memory (offsets from a 1024-aligned base).
-constexpr int kQBytes = 128 * kD * 2;                 // 2 sub-tiles [128 rows x 128 B]
+constexpr int kStages = 3;                            // K/V pair stages
 constexpr int kHalfK = 8192;                          // one K box: [64 rows x 128 B]
 constexpr int kPairBytes = 8 * kHalfK;                // K_a|K_b (d 0-63), K_a|K_b (d 64-127), V_a, V_b
-constexpr int kOffQ = 0;
-constexpr int kOffKV = kQBytes;
-constexpr int kOffList = kOffKV + 2 * kPairBytes;
+constexpr int kOffKV = 0;
+constexpr int kOffList = kOffKV + kStages * kPairBytes;
 constexpr int kListBytes = kMaxList * 5;              // int32 ids + uint8 token masks
 constexpr int kOffStage = kOffList + 2 * kListBytes;  // staged selection rows of one tile
 constexpr int kSmemBytes = kOffStage + kTQ * kMaxSlots * 4 + 1024;
 
-// TMEM columns: O [0,128), S buffers [128,256) and [256,384).
+// TMEM columns: O [0,128), S buffers [128,256) and [256,384), Q buffers [384,448) and [448,512).
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColO = 0, kColS0 = 128;
+constexpr uint32_t kColO = 0, kColS0 = 128, kColQ0 = 384;
 
 struct Bars {
-    uint64_t q_full, q_empty;
-    uint64_t kv_full[2], kv_empty[2];
+    uint64_t q_full, q_seen;
+    uint64_t kv_full[kStages], kv_empty[kStages];
     uint64_t s_full[2], p_full[2], pv_done[2];
     uint64_t list_full[2], list_empty[2];
     uint64_t fin;
     uint32_t tmem_base;
     int list_n[2];
     int abort;
+    float xmax[2][128];  // per-half row maxima of the current pair
+    float xl[128];       // second-half partial row sums, for the epilogue
+    int sm_stop;         // set by a softmax thread whose wait failed; read after a barrier
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -113,7 +120,7 @@ __device__ __forceinline__ float exp_half(const uint32_t* x, float sl2, float ne
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-sparse_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
+sparse_prefill_tc_kernel(const __nv_bfloat16* __restrict__ q,
                          const __grid_constant__ CUtensorMap tmK,
                          const __grid_constant__ CUtensorMap tmV,
                          const int32_t* __restrict__ idx, __nv_bfloat16* __restrict__ out, int H,
@@ -126,40 +133,42 @@ sparse_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
     const int tiles_per_seq = (N + kTQ - 1) / kTQ;
     volatile int* abort = &bars.abort;
 
-    if (warp == 5) {
+    if (warp == 9) {
         tmem_alloc(&bars.tmem_base, kTmemCols);
         tmem_relinquish();
     }
     if (tid == 0) {
-        mbar_init(&bars.q_full, 1);
-        mbar_init(&bars.q_empty, 1);
-        for (int b = 0; b < 2; ++b) {
+        mbar_init(&bars.q_full, 8);
+        mbar_init(&bars.q_seen, 1);
+        for (int b = 0; b < kStages; ++b) {
             mbar_init(&bars.kv_full[b], 1);
             mbar_init(&bars.kv_empty[b], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
             mbar_init(&bars.s_full[b], 1);
-            mbar_init(&bars.p_full[b], 4);
+            mbar_init(&bars.p_full[b], 8);
             mbar_init(&bars.pv_done[b], 1);
             mbar_init(&bars.list_full[b], 1);
             mbar_init(&bars.list_empty[b], 2);
         }
         mbar_init(&bars.fin, 1);
         bars.abort = 0;
+        bars.sm_stop = 0;
         fence_mbar_init();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = bars.tmem_base;
-    int32_t* list_id[2] = {reinterpret_cast<int32_t*>(sm + kOffList),
-                           reinterpret_cast<int32_t*>(sm + kOffList + kListBytes)};
-    uint8_t* list_mask[2] = {sm + kOffList + kMaxList * 4, sm + kOffList + kListBytes + kMaxList * 4};
+    auto list_id = [&](int lb) { return reinterpret_cast<int32_t*>(sm + kOffList + lb * kListBytes); };
+    auto list_mask = [&](int lb) { return sm + kOffList + lb * kListBytes + kMaxList * 4; };
 
-    if (warp == 4) {
+    if (warp == 8) {
         // ---------------------------------------------------------------- producer
         int32_t* stage = reinterpret_cast<int32_t*>(sm + kOffStage);
         int it = 0, gp = 0;
-        uint32_t q_issued = 0;
-        int last_phase[2] = {-1, -1};
+        int last_phase[kStages];
+        for (int e = 0; e < kStages; ++e) last_phase[e] = -1;
         for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
             const int lb = it & 1;
             if (it >= 2 && !wait_or_abort(&bars.list_empty[lb], ((it - 2) >> 1) & 1, ctx, abort)) break;
@@ -191,10 +200,10 @@ sparse_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                 }
                 if (lane == 0) {
                     if (m == prev) {
-                        list_mask[lb][n - 1] |= (uint8_t)msk;
+                        list_mask(lb)[n - 1] |= (uint8_t)msk;
                     } else if (n < kMaxList) {
-                        list_id[lb][n] = m;
-                        list_mask[lb][n] = (uint8_t)msk;
+                        list_id(lb)[n] = m;
+                        list_mask(lb)[n] = (uint8_t)msk;
                         ++n;
                     }
                 }
@@ -207,21 +216,18 @@ sparse_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
             }
             __syncwarp();
             int stop = 0;
-            if (lane == 0 && it >= 1 && !wait_or_abort(&bars.q_empty, (it - 1) & 1, ctx, abort)) stop = 1;
-            if (lane == 0 && !stop) {
-                mbar_arrive_expect_tx(&bars.q_full, kQBytes);
-                const int z = (int)((bg / Hkv) * H + (bg % Hkv) * kG);
-                tma_load_3d(sm + kOffQ, &tmQ, &bars.q_full, 0, i0, z);
-                tma_load_3d(sm + kOffQ + kQBytes / 2, &tmQ, &bars.q_full, 64, i0, z);
-                q_issued = it + 1;
+            if (lane == 0) {
                 for (int u = 0; u < n; u += 2, ++gp) {
-                    const int s = gp & 1, r = gp >> 1;
-                    if (r >= 1 && !wait_or_abort(&bars.kv_empty[s], (r - 1) & 1, ctx, abort)) break;
+                    const int s = gp % kStages, r = gp / kStages;
+                    if (r >= 1 && !wait_or_abort(&bars.kv_empty[s], (r - 1) & 1, ctx, abort)) {
+                        stop = 1;
+                        break;
+                    }
                     const int nb = min(2, n - u);
                     uint8_t* st = sm + kOffKV + s * kPairBytes;
                     mbar_arrive_expect_tx(&bars.kv_full[s], nb * 4 * kHalfK);
                     for (int e = 0; e < nb; ++e) {
-                        const int y = list_id[lb][u + e] * kBlk;
+                        const int y = list_id(lb)[u + e] * kBlk;
                         tma_load_3d(st + e * kHalfK, &tmK, &bars.kv_full[s], 0, y, (int)bg);
                         tma_load_3d(st + 2 * kHalfK + e * kHalfK, &tmK, &bars.kv_full[s], 64, y, (int)bg);
                         tma_load_3d(st + 4 * kHalfK + e * 2 * kHalfK, &tmV, &bars.kv_full[s], 0, y, (int)bg);
@@ -234,18 +240,15 @@ sparse_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
             stop = __shfl_sync(0xffffffffu, stop, 0);
             if (stop || *abort) break;
         }
-        if (lane == 0) {
-            if (q_issued) (void)mbar_wait(&bars.q_full, (q_issued - 1) & 1, ctx);
-            for (int s = 0; s < 2; ++s)
-                if (last_phase[s] >= 0) (void)mbar_wait(&bars.kv_full[s], last_phase[s] & 1, ctx);
-        }
-    } else if (warp == 5) {
+        if (lane == 0)
+            for (int e = 0; e < kStages; ++e)
+                if (last_phase[e] >= 0) (void)mbar_wait(&bars.kv_full[e], last_phase[e] & 1, ctx);
+    } else if (warp == 9) {
         // ---------------------------------------------------------------- MMA issuer
         if (lane == 0) {
             const uint32_t idS2 = idesc_bf16_f32(128, 128, false, false);
             const uint32_t idS1 = idesc_bf16_f32(128, 64, false, false);
             const uint32_t idPV = idesc_bf16_f32(128, kD, false, true);
-            const uint32_t q0 = smem_u32(sm + kOffQ);
             int it = 0, gp = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, ++it) {
@@ -255,23 +258,24 @@ sparse_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                 const int n = bars.list_n[lb];
                 const int np = (n + 1) >> 1;
                 mbar_arrive(&bars.list_empty[lb]);
-                ok = wait_or_abort(&bars.q_full, it & 1, ctx, abort);
+                ok = wait_or_abort(&bars.q_full, it & 1, ctx, abort);  // Q(tile) is in TMEM
                 if (!ok) break;
+                mbar_arrive(&bars.q_seen);
                 tc_fence_after();
+                const uint32_t aQ = tmem + kColQ0 + (it & 1) * 64;
                 auto issue_s = [&](int j, int g) -> bool {
-                    const int s = g & 1;
-                    if (!wait_or_abort(&bars.kv_full[s], (g >> 1) & 1, ctx, abort)) return false;
+                    const int st = g % kStages, b = g & 1;
+                    if (!wait_or_abort(&bars.kv_full[st], (g / kStages) & 1, ctx, abort)) return false;
                     tc_fence_after();
-                    const uint32_t kb = smem_u32(sm + kOffKV + s * kPairBytes);
-                    const uint32_t dS = tmem + kColS0 + s * 128;
+                    const uint32_t kb = smem_u32(sm + kOffKV + st * kPairBytes);
+                    const uint32_t dS = tmem + kColS0 + b * 128;
                     const uint32_t id = (2 * j + 1 < n) ? idS2 : idS1;
 #pragma unroll
                     for (int ks = 0; ks < kD / 16; ++ks) {
-                        const uint64_t a = sdesc_sw128(q0 + (ks >> 2) * (kQBytes / 2) + (ks & 3) * 32, 16, 1024);
-                        const uint64_t b = sdesc_sw128(kb + (ks >> 2) * 2 * kHalfK + (ks & 3) * 32, 16, 1024);
-                        mma_ss(dS, a, b, id, ks > 0);
+                        const uint64_t bd = sdesc_sw128(kb + (ks >> 2) * 2 * kHalfK + (ks & 3) * 32, 16, 1024);
+                        mma_ts(dS, aQ + ks * 8, bd, id, ks > 0);
                     }
-                    mma_commit(&bars.s_full[s]);
+                    mma_commit(&bars.s_full[b]);
                     return true;
                 };
                 if (np > 0) ok = issue_s(0, gp);
@@ -280,169 +284,226 @@ sparse_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                     if (j + 1 < np) {
                         ok = issue_s(j + 1, g + 1);
                         if (!ok) break;
-                    } else {
-                        mma_commit(&bars.q_empty);  // every S MMA of the tile has been issued
                     }
                     ok = wait_or_abort(&bars.p_full[g & 1], (g >> 1) & 1, ctx, abort);
                     if (!ok) break;
                     tc_fence_after();
-                    const int s = g & 1;
-                    const uint32_t vb = smem_u32(sm + kOffKV + s * kPairBytes + 4 * kHalfK);
+                    const int s = g & 1, st = g % kStages;
+                    const uint32_t vb = smem_u32(sm + kOffKV + st * kPairBytes + 4 * kHalfK);
                     const uint32_t aP = tmem + kColS0 + s * 128;
                     const int ksteps = (2 * j + 1 < n) ? 8 : 4;
                     for (int ks = 0; ks < ksteps; ++ks) {
                         const uint64_t b = sdesc_sw128(vb + (ks >> 2) * 2 * kHalfK + (ks & 3) * 16 * 128, kHalfK, 1024);
                         mma_ts(tmem + kColO, aP + ks * 8, b, idPV, (j > 0 || ks > 0) ? 1u : 0u);
                     }
-                    mma_commit(&bars.kv_empty[s]);
+                    mma_commit(&bars.kv_empty[st]);
                     mma_commit(&bars.pv_done[s]);
                 }
-                if (np == 0) mma_commit(&bars.q_empty);
                 gp += np;
             }
             mma_commit(&bars.fin);
             (void)mbar_wait(&bars.fin, 0, ctx);
         }
         __syncwarp();
-    } else if (warp < 4) {
+    } else {
         // ---------------------------------------------------------------- softmax + epilogue
-        const int r = tid;
+        // The 8 softmax warps meet at named barriers (bar.sync 2 / 1, 256 threads), which have
+        // no time limit.  So they never leave a loop one by one: a failed (timed-out) wait
+        // records sm_stop and the thread carries on without touching TMEM; after the next
+        // barrier every softmax thread reads the same sm_stop and they all leave together.
+        const int r = tid & 127;            // row = TMEM lane
+        const int half = tid >> 7;          // 0: first block of a pair, 1: second
         const int t = r % kTQ, hh = r / kTQ;
         const uint32_t lane_base = tmem_lane_base(warp);
+        // Q rows of a tile -> registers (this thread: row r, columns 64*half .. +63), then TMEM.
+        auto load_q = [&](int T, uint4 (&qv)[8]) {
+            const int64_t bgT = T / tiles_per_seq;
+            const int iT = (T % tiles_per_seq) * kTQ + t;
+            if (iT < N) {
+                const uint4* src = reinterpret_cast<const uint4*>(
+                    q + (((bgT / Hkv) * H + (bgT % Hkv) * kG + hh) * (int64_t)N + iT) * kD + half * 64);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) qv[e] = src[e];
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) qv[e] = make_uint4(0, 0, 0, 0);
+            }
+        };
+        auto store_q = [&](int buf, const uint4 (&qv)[8]) {
+            tmem_st32(tmem + lane_base + kColQ0 + buf * 64 + half * 32,
+                      *reinterpret_cast<const uint32_t(*)[32]>(&qv[0]));
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars.q_full);
+        };
+        {
+            uint4 qv[8];
+            load_q(blockIdx.x, qv);
+            store_q(0, qv);
+        }
+        // sm_stop holds the index of the first barrier after which everybody must leave: a
+        // failure before barrier k (nbar == k-1 completed) names k, one after it names k+1, so a
+        // thread that reads the flag right after barrier k never sees a later failure early.
+        volatile int* sm_stop = &bars.sm_stop;
+        int nbar = 0;                       // named barriers (id 2) passed so far
+        bool dead = false;                  // this thread saw a failed wait
+        auto fail = [&]() {
+            dead = true;
+            atomicCAS(&bars.sm_stop, 0, nbar + 1);
+            *abort = 1;
+        };
+        auto stop_now = [&]() { const int v = *sm_stop; return v != 0 && v <= nbar; };
         int it = 0, gp = 0;
         for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
             const int lb = it & 1;
-            if (!wait_or_abort(&bars.list_full[lb], (it >> 1) & 1, ctx, abort)) break;
+            if (!dead && !mbar_wait(&bars.list_full[lb], (it >> 1) & 1, ctx)) fail();
+            asm volatile("bar.sync 2, 256;" ::: "memory");
+            ++nbar;
+            if (stop_now()) break;
             const int n = bars.list_n[lb];
             const int np = (n + 1) >> 1;
+            const int32_t* ids = list_id(lb);
+            const uint8_t* msks = list_mask(lb);
             const int64_t bg = tile / tiles_per_seq;
             const int i0 = (tile % tiles_per_seq) * kTQ;
             const int c = i0 / kBlk;
             const int i = i0 + t;
-            float m_run = -INFINITY, l = 0.f;  // m_run in scaled log2 units
-            bool ok = true;
+            float m_run = -INFINITY, l = 0.f;  // running max (scaled log2 units), partial sum
+            bool stop = false;
+            // Q of this CTA's next tile: loaded now, written to TMEM after the first pair (by then
+            // the MMA thread has taken this tile's Q, see q_seen), into the other Q buffer.
+            const int next = tile + gridDim.x;
+            bool q_pending = next < n_tiles;
+            uint4 qv[8];
+            if (q_pending) load_q(next, qv);
+            auto flush_q = [&]() {
+                if (!q_pending) return;
+                q_pending = false;
+                if (!dead && !mbar_wait(&bars.q_seen, it & 1, ctx)) fail();
+                if (!__any_sync(0xffffffffu, dead)) store_q((it + 1) & 1, qv);
+            };
             for (int j = 0; j < np; ++j) {
                 const int g = gp + j, s = g & 1;
-                const bool two = 2 * j + 1 < n;
-                const int blk_a = list_id[lb][2 * j];
-                const int blk_b = two ? list_id[lb][2 * j + 1] : -1;
-                const bool sel_a = (list_mask[lb][2 * j] >> t) & 1;
-                const bool sel_b = two && ((list_mask[lb][2 * j + 1] >> t) & 1);
-                // last visible key of each half (-1: none)
-                const int lim_a = !sel_a ? -1 : (blk_a == c ? i - blk_a * kBlk : kBlk - 1);
-                const int lim_b = !sel_b ? -1 : (blk_b == c ? i - blk_b * kBlk : kBlk - 1);
-                if (!wait_or_abort(&bars.s_full[s], (g >> 1) & 1, ctx, abort)) { ok = false; break; }
+                const int u = 2 * j + half;     // this warp's union block
+                const bool has = u < n;
+                const int blk = has ? ids[u] : -1;
+                const bool sel = has && ((msks[u] >> t) & 1);
+                // last visible key of this half (-1: none)
+                const int lim = !sel ? -1 : (blk == c ? i - blk * kBlk : kBlk - 1);
+                if (!dead && !mbar_wait(&bars.s_full[s], (g >> 1) & 1, ctx)) fail();
                 tc_fence_after();
                 const uint32_t colS = tmem + lane_base + kColS0 + s * 128;
-                uint32_t xa[64], xb[64];
-                tmem_ld32(colS, *reinterpret_cast<uint32_t(*)[32]>(&xa[0]));
-                tmem_ld32(colS + 32, *reinterpret_cast<uint32_t(*)[32]>(&xa[32]));
-                if (two) {
-                    tmem_ld32(colS + 64, *reinterpret_cast<uint32_t(*)[32]>(&xb[0]));
-                    tmem_ld32(colS + 96, *reinterpret_cast<uint32_t(*)[32]>(&xb[32]));
+                uint32_t x[64];
+                const bool ld = __any_sync(0xffffffffu, has && !dead);
+                if (ld) {
+                    tmem_ld32(colS + half * 64, *reinterpret_cast<uint32_t(*)[32]>(&x[0]));
+                    tmem_ld32(colS + half * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&x[32]));
+                    tmem_ld_wait();
                 }
-                tmem_ld_wait();
-                // Row max in raw units over the visible keys (diagonal block: masked first).
-                if (lim_a >= 0 && lim_a < kBlk - 1)
+                if (lim >= 0 && lim < kBlk - 1)
 #pragma unroll
-                    for (int jj = 0; jj < 64; ++jj) xa[jj] = jj <= lim_a ? xa[jj] : __float_as_uint(-INFINITY);
-                if (lim_b >= 0 && lim_b < kBlk - 1)
-#pragma unroll
-                    for (int jj = 0; jj < 64; ++jj) xb[jj] = jj <= lim_b ? xb[jj] : __float_as_uint(-INFINITY);
-                float mx = -INFINITY;
-                if (lim_a >= 0) mx = max64(xa);
-                if (lim_b >= 0) mx = fmaxf(mx, max64(xb));
-                mx *= sl2;
+                    for (int jj = 0; jj < 64; ++jj) x[jj] = jj <= lim ? x[jj] : __float_as_uint(-INFINITY);
+                const float mh = (lim >= 0 && ld) ? max64(x) * sl2 : -INFINITY;
+                bars.xmax[half][r] = mh;
+                // Both halves have loaded their S columns before either overwrites S with P.
+                asm volatile("bar.sync 2, 256;" ::: "memory");
+                ++nbar;
+                if (stop_now()) { stop = true; break; }
+                const float mx = fmaxf(mh, bars.xmax[half ^ 1][r]);
                 const bool grow = mx > m_run + 8.f;
-                const bool need_rescale = grow && l > 0.f;
-                if (__any_sync(0xffffffffu, need_rescale)) {
-                    if (j >= 1) {
+                // O holds this row's earlier pairs once m_run is finite: rescale it (first half).
+                const bool need_rescale = grow && m_run != -INFINITY;
+                if (half == 0 && __any_sync(0xffffffffu, need_rescale)) {
+                    if (j >= 1 && !dead) {
                         const int gq = g - 1;
-                        if (!wait_or_abort(&bars.pv_done[gq & 1], (gq >> 1) & 1, ctx, abort)) { ok = false; break; }
+                        if (!mbar_wait(&bars.pv_done[gq & 1], (gq >> 1) & 1, ctx)) fail();
                     }
-                    tc_fence_after();
-                    const float alpha = need_rescale ? ex2(m_run - mx) : 1.f;
+                    if (!__any_sync(0xffffffffu, dead)) {
+                        tc_fence_after();
+                        const float alpha = need_rescale ? ex2(m_run - mx) : 1.f;
 #pragma unroll 1
-                    for (int c0 = 0; c0 < kD; c0 += 32) {
-                        uint32_t orr[32];
-                        tmem_ld32(tmem + lane_base + kColO + c0, orr);
-                        tmem_ld_wait();
+                        for (int c0 = 0; c0 < kD; c0 += 32) {
+                            uint32_t orr[32];
+                            tmem_ld32(tmem + lane_base + kColO + c0, orr);
+                            tmem_ld_wait();
 #pragma unroll
-                        for (int q = 0; q < 32; ++q) orr[q] = __float_as_uint(__uint_as_float(orr[q]) * alpha);
-                        tmem_st16(tmem + lane_base + kColO + c0, *reinterpret_cast<uint32_t(*)[16]>(&orr[0]));
-                        tmem_st16(tmem + lane_base + kColO + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&orr[16]));
+                            for (int q = 0; q < 32; ++q) orr[q] = __float_as_uint(__uint_as_float(orr[q]) * alpha);
+                            tmem_st16(tmem + lane_base + kColO + c0, *reinterpret_cast<uint32_t(*)[16]>(&orr[0]));
+                            tmem_st16(tmem + lane_base + kColO + c0 + 16, *reinterpret_cast<uint32_t(*)[16]>(&orr[16]));
+                        }
+                        tmem_st_wait();
                     }
-                    tmem_st_wait();
                 }
                 if (grow) {
                     l = (m_run == -INFINITY) ? 0.f : l * ex2(m_run - mx);
                     m_run = mx;
                 }
-                uint32_t pk[64];
-                float ps = 0.f;
-                if (lim_a >= 0) {
-                    ps += exp_half(xa, sl2, -m_run, lim_a, pk);
-                } else {
-#pragma unroll
-                    for (int q = 0; q < 32; ++q) pk[q] = 0u;
-                }
-                if (two) {
-                    if (lim_b >= 0) {
-                        ps += exp_half(xb, sl2, -m_run, lim_b, pk + 32);
+                if (ld && !__any_sync(0xffffffffu, dead)) {
+                    uint32_t pk[32];
+                    if (lim >= 0) {
+                        l += exp_half(x, sl2, -m_run, lim, pk);
                     } else {
 #pragma unroll
-                        for (int q = 32; q < 64; ++q) pk[q] = 0u;
+                        for (int q = 0; q < 32; ++q) pk[q] = 0u;
                     }
+                    tmem_st16(colS + half * 32, *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
+                    tmem_st16(colS + half * 32 + 16, *reinterpret_cast<uint32_t(*)[16]>(&pk[16]));
+                    tmem_st_wait();
                 }
-                l += ps;
-                tmem_st16(colS, *reinterpret_cast<uint32_t(*)[16]>(&pk[0]));
-                tmem_st16(colS + 16, *reinterpret_cast<uint32_t(*)[16]>(&pk[16]));
-                if (two) {
-                    tmem_st16(colS + 32, *reinterpret_cast<uint32_t(*)[16]>(&pk[32]));
-                    tmem_st16(colS + 48, *reinterpret_cast<uint32_t(*)[16]>(&pk[48]));
-                }
-                tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars.p_full[s]);
+                flush_q();
             }
-            if (!ok) break;
+            if (stop) break;
+            flush_q();
+            // Epilogue: l = sum of both halves; each half writes 64 of the 128 output columns.
+            if (half == 1) bars.xl[r] = l;
+            asm volatile("bar.sync 2, 256;" ::: "memory");
+            ++nbar;
+            if (half == 0) bars.xmax[0][r] = l + bars.xl[r];  // broadcast of the row total
+            asm volatile("bar.sync 2, 256;" ::: "memory");
+            ++nbar;
+            const float ltot = bars.xmax[0][r];
             const int64_t orow = (((bg / Hkv) * H + (bg % Hkv) * kG + hh) * (int64_t)N + i) * kD;
             if (np > 0) {
                 const int gl = gp + np - 1;
-                if (!wait_or_abort(&bars.pv_done[gl & 1], (gl >> 1) & 1, ctx, abort)) break;
-                tc_fence_after();
-                const float inv = l > 0.f ? 1.f / l : 0.f;
+                if (!dead && !mbar_wait(&bars.pv_done[gl & 1], (gl >> 1) & 1, ctx)) fail();
+                if (!__any_sync(0xffffffffu, dead)) {
+                    tc_fence_after();
+                    const float inv = ltot > 0.f ? 1.f / ltot : 0.f;
 #pragma unroll 1
-                for (int c0 = 0; c0 < kD; c0 += 32) {
-                    uint32_t orr[32];
-                    tmem_ld32(tmem + lane_base + kColO + c0, orr);
-                    tmem_ld_wait();
-                    if (i < N) {
-                        uint4 w[4];
-                        uint32_t* wp = reinterpret_cast<uint32_t*>(w);
+                    for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {
+                        uint32_t orr[32];
+                        tmem_ld32(tmem + lane_base + kColO + c0, orr);
+                        tmem_ld_wait();
+                        if (i < N) {
+                            uint4 w[4];
+                            uint32_t* wp = reinterpret_cast<uint32_t*>(w);
 #pragma unroll
-                        for (int q = 0; q < 16; ++q)
-                            wp[q] = pack_bf16x2(__uint_as_float(orr[2 * q]) * inv,
-                                                __uint_as_float(orr[2 * q + 1]) * inv);
-                        uint4* d4 = reinterpret_cast<uint4*>(out + orow + c0);
+                            for (int q = 0; q < 16; ++q)
+                                wp[q] = pack_bf16x2(__uint_as_float(orr[2 * q]) * inv,
+                                                    __uint_as_float(orr[2 * q + 1]) * inv);
+                            uint4* d4 = reinterpret_cast<uint4*>(out + orow + c0);
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) d4[q] = w[q];
+                            for (int q = 0; q < 4; ++q) d4[q] = w[q];
+                        }
                     }
+                    tc_fence_before();
                 }
-                tc_fence_before();
             } else if (i < N) {
-                uint4* d4 = reinterpret_cast<uint4*>(out + orow);
-                for (int q = 0; q < kD / 8; ++q) d4[q] = make_uint4(0, 0, 0, 0);
+                uint4* d4 = reinterpret_cast<uint4*>(out + orow + half * 64);
+                for (int q = 0; q < 8; ++q) d4[q] = make_uint4(0, 0, 0, 0);
             }
             gp += np;
-            asm volatile("bar.sync 1, 128;" ::: "memory");
+            asm volatile("bar.sync 1, 256;" ::: "memory");
             if (tid == 0) mbar_arrive(&bars.list_empty[lb]);
         }
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == 9) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
@@ -458,7 +519,7 @@ cudaError_t launch_sparse_prefill_tc(const void* q, const void* k, const void* v
                                      const int32_t* idx, void* o, int B, int H, int Hkv, int N,
                                      int d, int slots, float scale, cudaStream_t st, DevCtx ctx) {
     if (d != kD || H != Hkv * kG || slots > kMaxSlots) return cudaErrorNotSupported;
-    CUtensorMap tmQ, tmK, tmV;
+    CUtensorMap tmK, tmV;
     EncodeTiledFn fn = encode_tiled_fn();
     if (!fn) return cudaErrorNotSupported;
     auto make3 = [&](CUtensorMap* m, const void* base, uint64_t rows, uint64_t planes,
@@ -471,8 +532,7 @@ cudaError_t launch_sparse_prefill_tc(const void* q, const void* k, const void* v
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
     };
-    if (!make3(&tmQ, q, (uint64_t)N, (uint64_t)B * H, kTQ, kG) ||
-        !make3(&tmK, k, (uint64_t)N, (uint64_t)B * Hkv, kBlk, 1) ||
+    if (!make3(&tmK, k, (uint64_t)N, (uint64_t)B * Hkv, kBlk, 1) ||
         !make3(&tmV, v, (uint64_t)N, (uint64_t)B * Hkv, kBlk, 1))
         return cudaErrorInvalidValue;
     static int num_sms = 0;
@@ -489,7 +549,8 @@ cudaError_t launch_sparse_prefill_tc(const void* q, const void* k, const void* v
     const int grid = n_tiles < num_sms ? n_tiles : num_sms;
     const float sl2 = scale * 1.4426950408889634f;
     sparse_prefill_tc_kernel<<<grid, kThreads, kSmemBytes, st>>>(
-        tmQ, tmK, tmV, idx, static_cast<__nv_bfloat16*>(o), H, Hkv, N, slots, sl2, n_tiles, ctx);
+        static_cast<const __nv_bfloat16*>(q), tmK, tmV, idx, static_cast<__nv_bfloat16*>(o), H, Hkv,
+        N, slots, sl2, n_tiles, ctx);
     return cudaGetLastError();
 }
 

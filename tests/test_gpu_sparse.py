@@ -58,6 +58,20 @@ def test_bf16_pipeline_gqa16(sala, N, topk, n_local):
     _pipeline(sala, layer, "bf16", topk, 1, n_local)
 
 
+def test_bf16_d64_pipeline_cuda_core_paths(sala):
+    # d = 64 runs the CUDA-core selection and attention kernels in bf16.
+    from hybrid_sparse_linear_b200 import synth
+    layer = synth.sparse_layer(1, 8, 2, 64 * 30 + 3, 64, torch.bfloat16, layer=9, shift_frac=0.1)
+    _pipeline(sala, layer, "bf16", 5, 1, 2)
+
+
+def test_bf16_selection_batch2_k_below_64(sala):
+    # batch 2, k = 17 (lists shorter than their 64-entry capacity), tile of rows crossing N.
+    from hybrid_sparse_linear_b200 import synth
+    layer = synth.sparse_layer(2, 32, 2, 64 * 41 + 30, 128, torch.bfloat16, layer=10, shift_frac=0.05)
+    _pipeline(sala, layer, "bf16", 17, 1, 2)
+
+
 def test_fp32_d128_pipeline_batch2(sala):
     from hybrid_sparse_linear_b200 import synth
     layer = synth.sparse_layer(2, 8, 2, 64 * 12 + 5, 128, torch.float32, layer=3, shift_frac=0.1)
