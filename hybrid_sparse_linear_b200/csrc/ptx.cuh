@@ -220,5 +220,35 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// Three-input maximum (one instruction on sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// (x0, x1) * m + (c, c) on the packed two-wide fp32 FMA path.
+__device__ __forceinline__ void fma2_bcast(float& y0, float& y1, float x0, float x1, float m, float c) {
+    asm("{\n\t.reg .b64 xa, xm, xc, xd;\n\t"
+        "mov.b64 xa, {%2, %3};\n\t"
+        "mov.b64 xm, {%4, %4};\n\t"
+        "mov.b64 xc, {%5, %5};\n\t"
+        "fma.rn.f32x2 xd, xa, xm, xc;\n\t"
+        "mov.b64 {%0, %1}, xd;\n\t}"
+        : "=f"(y0), "=f"(y1)
+        : "f"(x0), "f"(x1), "f"(m), "f"(c));
+}
+
+// (a0, a1) += (b0, b1) on the packed two-wide fp32 add path.
+__device__ __forceinline__ void add2(float& a0, float& a1, float b0, float b1) {
+    asm("{\n\t.reg .b64 xa, xb;\n\t"
+        "mov.b64 xa, {%0, %1};\n\t"
+        "mov.b64 xb, {%2, %3};\n\t"
+        "add.rn.f32x2 xa, xa, xb;\n\t"
+        "mov.b64 {%0, %1}, xa;\n\t}"
+        : "+f"(a0), "+f"(a1)
+        : "f"(b0), "f"(b1));
+}
+
 }  // namespace ptx
 }  // namespace sala
