@@ -4,27 +4,30 @@
 // B (tokens 8-15) of 128 rows each (row = head * 8 + token, the 16 query heads of the group), the
 // M of one tcgen05 MMA.  The 16 tokens share their query block (16 divides 64), hence the forced
 // blocks and the diagonal; their top-k choices differ, so the unit walks the UNION of the 16
-// selections (ascending) and each row masks the blocks its token did not choose.  Executed FLOPs
-// exceed the algorithmic ones by that union overhead; each row's own sum over its selected keys
-// is exact.
+// selections (ascending).  K and V of each union block are loaded once for both tiles; a tile none
+// of whose 8 tokens chose the block skips it, and each row masks the blocks its own token did not
+// choose, so a row's sum runs over exactly its selected keys.
 //
-// The union is consumed two blocks at a time (a "pair", 128 keys), and the two tiles ping-pong on
-// the tensor core (the structure FlashAttention-4 uses on this architecture):
-//   S_X  = Q_X [K_a; K_b]^T      M=128 N=128 K=128  (X = A, B; Q from shared memory, the two K
-//                                                    tiles back to back in shared memory)
-//   P_X  = online softmax of S_X (per row: selection mask per block, causal mask on the diagonal)
-//   O_X += P_X [V_a; V_b]        M=128 N=128 K=128  (A = P_X from TMEM, aliasing S_X)
-// Issue order per pair: PV_A, S_A(next), PV_B, S_B(next), so the softmax of one tile overlaps the
-// MMAs of the other.  O_X is rescaled only when a row's running max grows by more than 8 in log2
-// units (the stale max keeps exp2 below 256 and cancels in O / l).
+// Per block b and active tile X:
+//   S_X  = Q_X K_b^T      M=128 N=64 K=128   (Q_X and K_b from shared memory)
+//   P_X  = online softmax of S_X (selection mask per row, causal mask on the diagonal block)
+//   O_X += P_X V_b        M=128 N=128 K=64   (A = P_X from TMEM, aliasing S_X; B = V_b)
+// Each tile's MMAs come from its own issuing thread, and each tile has two S buffers in TMEM, so
+// the S of the tile's next block runs while its softmax works on this one: per tile the chain is
+// softmax -> PV, and the two tiles' chains overlap each other's MMAs (the ping-pong
+// FlashAttention-4 uses on this architecture).  O_X is rescaled only when a row's running max
+// grows by more than 8 in log2 units (the stale max keeps exp2 below 256 and cancels in O / l).
 //
-// Roles (384 threads, persistent: one CTA per SM walks units blockIdx.x, +gridDim.x, ...):
-// warps 0-3 softmax + epilogue of tile A, warps 4-7 of tile B (thread = row = TMEM lane; each
-// thread owns its whole row, so the two warpgroups never wait for each other inside a unit);
-// warp 8 stages the next unit's 16 selection rows with coalesced loads, merges them into the union
-// list and issues the TMA loads (Q tiles, then a 2-stage ring of K/V pairs); warp 9 allocates TMEM
-// and issues the MMAs (one thread); warps 10-11 only complete the third warpgroup.  Every wait is bounded; a timeout sets the status word, the
-// roles wind down, and the kernel waits (bounded) for its own copies and MMAs before it frees TMEM.
+// Shared memory holds the unit's two Q tiles and a ring of four 32 KiB stages, each the K and V
+// of one block, loaded by TMA up to four blocks ahead.
+//
+// Roles (352 threads, persistent: one CTA per SM walks units blockIdx.x, +gridDim.x, ...):
+// warps 0-3 softmax + epilogue of tile A, warps 4-7 of tile B (thread = row = TMEM lane); warp 8
+// stages the next unit's 16 selection rows with coalesced loads, merges them into the union list
+// and issues the TMA loads (Q tiles, then the ring); warp 9 allocates TMEM and issues the MMAs of
+// tile A, warp 10 those of tile B (one thread each).  Every wait is bounded; a timeout sets the
+// status word, the roles wind down, and the kernel waits (bounded) for its own copies and MMAs
+// before it frees TMEM.
 #include "kernels.h"
 #include "ptx.cuh"
 #include "tmap.cuh"
@@ -41,35 +44,31 @@ constexpr int kUT = 16;          // query tokens per unit (two tiles)
 constexpr int kBlk = 64;         // keys per block
 constexpr int kMaxSlots = 80;    // selection slots per row the kernel accepts
 constexpr int kMaxList = kUT * kMaxSlots;
-constexpr int kThreads = 384;
-// Register split (setmaxnreg): the two softmax warpgroups hold a whole S row per thread; the
-// third warpgroup (producer, MMA issuer, two idle warps) needs little.  256 * 216 + 128 * 72 =
-// 384 * 168, the per-thread count the block is launched with.
-constexpr int kRegsLaunch = 168, kRegsSoftmax = 216, kRegsOther = 72;
-static_assert(256 * kRegsSoftmax + 128 * kRegsOther <= kThreads * kRegsLaunch, "register split");
-constexpr int kStages = 2;       // K/V pair stages
+constexpr int kThreads = 352;
+constexpr int kStages = 4;
 
-// Shared memory (offsets from a 1024-aligned base).
-constexpr int kQBytes = 128 * kD * 2;                 // one Q tile: 2 sub-tiles [128 rows x 128 B]
-constexpr int kHalfK = 8192;                          // one K box: [64 rows x 128 B]
-constexpr int kPairBytes = 8 * kHalfK;                // K_a|K_b (d 0-63), K_a|K_b (d 64-127), V_a, V_b
-constexpr int kOffQ = 0;                              // Q_A, Q_B
-constexpr int kOffKV = 2 * kQBytes;
-constexpr int kOffList = kOffKV + kStages * kPairBytes;
+// Shared memory (offsets from a 1024-aligned base): Q_A, Q_B (two [128 x 128 B] halves each,
+// d 0-63 and d 64-127), then the ring; a stage holds K_b (two [64 x 128 B] halves) then V_b.
+constexpr int kQBytes = 32768;
+constexpr int kHalfQ = 16384;                         // one [128 rows x 128 B] box
+constexpr int kStageBytes = 32768;
+constexpr int kHalfBlk = 8192;                        // one [64 rows x 128 B] box
+constexpr int kOffRing = 2 * kQBytes;
+constexpr int kOffList = kOffRing + kStages * kStageBytes;
 constexpr int kListBytes = kMaxList * 6;              // int32 ids + uint16 token masks
 constexpr int kOffStage = kOffList + 2 * kListBytes;  // staged selection rows of one unit
 constexpr int kSmemBytes = kOffStage + kUT * kMaxSlots * 4 + 1024;
 
-// TMEM columns: O_A [0,128), O_B [128,256), S_A [256,384), S_B [384,512).
+// TMEM columns: O_A [0,128), O_B [128,256), S_A two buffers [256,384), S_B two buffers [384,512).
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 0, kColS = 256;
 
 struct Bars {
-    uint64_t q_full, q_empty;
     uint64_t kv_full[kStages], kv_empty[kStages];
-    uint64_t s_full[2], p_full[2], pv_done[2];  // per tile
+    uint64_t s_full[2][2], p_full[2][2], pv_done[2][2];  // per tile and S buffer
+    uint64_t q_full, q_empty;
     uint64_t list_full[2], list_empty[2];
-    uint64_t fin;
+    uint64_t fin[2];
     uint32_t tmem_base;
     int list_n[2];
     int abort;
@@ -84,6 +83,7 @@ __device__ __forceinline__ float ex2(float x) {
 
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, const DevCtx& ctx,
                                               volatile int* abort) {
+    if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
     if (!mbar_wait(bar, parity, ctx)) {
         *abort = 1;
@@ -92,7 +92,7 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, co
     return true;
 }
 
-__device__ __forceinline__ uint32_t (&sub32(uint32_t (&a)[128], int k))[32] {
+__device__ __forceinline__ uint32_t (&sub32(uint32_t (&a)[64], int k))[32] {
     return *reinterpret_cast<uint32_t(*)[32]>(a + 32 * k);
 }
 
@@ -166,20 +166,22 @@ sparse_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
         tmem_relinquish();
     }
     if (tid == 0) {
-        mbar_init(&bars.q_full, 1);
-        mbar_init(&bars.q_empty, 1);
-        for (int b = 0; b < kStages; ++b) {
-            mbar_init(&bars.kv_full[b], 1);
-            mbar_init(&bars.kv_empty[b], 1);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&bars.kv_full[s], 1);
+            mbar_init(&bars.kv_empty[s], 2);  // released by both MMA issuers
         }
         for (int b = 0; b < 2; ++b) {
-            mbar_init(&bars.s_full[b], 1);
-            mbar_init(&bars.p_full[b], 4);
-            mbar_init(&bars.pv_done[b], 1);
+            for (int j = 0; j < 2; ++j) {
+                mbar_init(&bars.s_full[b][j], 1);
+                mbar_init(&bars.p_full[b][j], 4);
+                mbar_init(&bars.pv_done[b][j], 1);
+            }
             mbar_init(&bars.list_full[b], 1);
-            mbar_init(&bars.list_empty[b], 2);
+            mbar_init(&bars.list_empty[b], 3);
+            mbar_init(&bars.fin[b], 1);
         }
-        mbar_init(&bars.fin, 1);
+        mbar_init(&bars.q_full, 1);
+        mbar_init(&bars.q_empty, 2);  // both MMA issuers
         bars.abort = 0;
         bars.sm_stop = 0;
         fence_mbar_init();
@@ -192,171 +194,197 @@ sparse_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
     auto list_mask = [&](int lb) {
         return reinterpret_cast<uint16_t*>(sm + kOffList + lb * kListBytes + kMaxList * 4);
     };
+    // Ring entry e lives in stage e % kStages and is that stage's use number e / kStages.
+    auto stage_ptr = [&](uint32_t e) { return sm + kOffRing + (e % kStages) * kStageBytes; };
+    auto full_bar = [&](uint32_t e) { return &bars.kv_full[e % kStages]; };
+    auto empty_bar = [&](uint32_t e) { return &bars.kv_empty[e % kStages]; };
+    auto round_of = [](uint32_t e) { return (e / kStages) & 1u; };
 
-    if (warp >= 8) {
-        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsOther));
-        if (warp == 8) {
-            // ---------------------------------------------------------------- producer
-            int32_t* stage = reinterpret_cast<int32_t*>(sm + kOffStage);
-            int it = 0, gp = 0;
-            uint32_t q_issued = 0;
-            int last0 = -1, last1 = -1;
-            for (int unit = blockIdx.x; unit < n_units; unit += gridDim.x, ++it) {
-                const int lb = it & 1;
-                if (it >= 2 && !wait_or_abort(&bars.list_empty[lb], ((it - 2) >> 1) & 1, ctx, abort)) break;
-                const int64_t bg = unit / units_per_seq;
-                const int i0 = (unit % units_per_seq) * kUT;
-                const int c = i0 / kBlk;
-                const int n_act = min(kUT, N - i0);
-                // Stage the unit's selection rows (contiguous in memory) with coalesced loads.
-                const int32_t* src = idx + (bg * N + i0) * (int64_t)slots;
-                for (int e = lane; e < n_act * slots; e += 32) stage[e] = src[e];
-                __syncwarp();
-                // 16-way merge of the ascending rows, one lane per token.
-                const int32_t* row = stage + lane * slots;
-                const bool active = lane < n_act;
-                int p = 0, n = 0, prev = -1;
-                while (true) {
-                    int head = 0x7fffffff;
-                    if (active && p < slots) {
-                        const int v = row[p];
-                        if (v >= 0) head = v;
-                    }
-                    const int m = __reduce_min_sync(0xffffffffu, head);
-                    if (m == 0x7fffffff) break;
-                    const unsigned msk = __ballot_sync(0xffffffffu, head == m);
-                    if (head == m) ++p;
-                    if (m > c) {  // in the future of every token of the unit
-                        if (lane == 0) flag(ctx, kStatusBounds);
-                        continue;
-                    }
-                    if (lane == 0) {
-                        if (m == prev) {
-                            list_mask(lb)[n - 1] |= (uint16_t)msk;
-                        } else if (n < kMaxList) {
-                            list_id(lb)[n] = m;
-                            list_mask(lb)[n] = (uint16_t)msk;
-                            ++n;
-                        }
-                    }
-                    n = __shfl_sync(0xffffffffu, n, 0);
-                    prev = m;
+    if (warp == 8) {
+        // ---------------------------------------------------------------- producer
+        // A unit with a non-empty union loads its Q tiles, then one ring entry per union block.
+        int32_t* stage = reinterpret_cast<int32_t*>(sm + kOffStage);
+        int it = 0;
+        uint32_t rc = 0, kq = 0;  // ring entries issued, Q tile pairs issued
+        for (int unit = blockIdx.x; unit < n_units; unit += gridDim.x, ++it) {
+            const int lb = it & 1;
+            if (it >= 2 && !wait_or_abort(&bars.list_empty[lb], ((it - 2) >> 1) & 1, ctx, abort)) break;
+            const int64_t bg = unit / units_per_seq;
+            const int i0 = (unit % units_per_seq) * kUT;
+            const int c = i0 / kBlk;
+            const int n_act = min(kUT, N - i0);
+            // Stage the unit's selection rows (contiguous in memory) with coalesced loads.
+            const int32_t* src = idx + (bg * N + i0) * (int64_t)slots;
+            for (int e = lane; e < n_act * slots; e += 32) stage[e] = src[e];
+            __syncwarp();
+            // 16-way merge of the ascending rows, one lane per token.
+            const int32_t* row = stage + lane * slots;
+            const bool active = lane < n_act;
+            int p = 0, n = 0, prev = -1;
+            while (true) {
+                int head = 0x7fffffff;
+                if (active && p < slots) {
+                    const int v = row[p];
+                    if (v >= 0) head = v;
+                }
+                const int m = __reduce_min_sync(0xffffffffu, head);
+                if (m == 0x7fffffff) break;
+                const unsigned msk = __ballot_sync(0xffffffffu, head == m);
+                if (head == m) ++p;
+                if (m > c) {  // in the future of every token of the unit
+                    if (lane == 0) flag(ctx, kStatusBounds);
+                    continue;
                 }
                 if (lane == 0) {
-                    bars.list_n[lb] = n;
-                    mbar_arrive(&bars.list_full[lb]);
-                }
-                __syncwarp();
-                int stop = 0;
-                if (lane == 0) {
-                    // Q tiles A and B: 16 heads x 8 tokens x 128 columns each.
-                    if (it >= 1 && !wait_or_abort(&bars.q_empty, (it - 1) & 1, ctx, abort)) stop = 1;
-                    if (!stop) {
-                        mbar_arrive_expect_tx(&bars.q_full, 2 * kQBytes);
-                        const int z = (int)((bg / Hkv) * H + (bg % Hkv) * kG);
-                        for (int x = 0; x < 2; ++x) {
-                            uint8_t* qd = sm + kOffQ + x * kQBytes;
-                            tma_load_3d(qd, &tmQ, &bars.q_full, 0, i0 + x * kTQ, z);
-                            tma_load_3d(qd + kQBytes / 2, &tmQ, &bars.q_full, 64, i0 + x * kTQ, z);
-                        }
-                        q_issued = it + 1;
-                    }
-                    for (int u = 0; u < n && !stop; u += 2, ++gp) {
-                        const int s = gp & 1, r = gp >> 1;
-                        if (r >= 1 && !wait_or_abort(&bars.kv_empty[s], (r - 1) & 1, ctx, abort)) {
-                            stop = 1;
-                            break;
-                        }
-                        const int nb = min(2, n - u);
-                        uint8_t* st = sm + kOffKV + s * kPairBytes;
-                        mbar_arrive_expect_tx(&bars.kv_full[s], nb * 4 * kHalfK);
-                        for (int e = 0; e < nb; ++e) {
-                            const int y = list_id(lb)[u + e] * kBlk;
-                            tma_load_3d(st + e * kHalfK, &tmK, &bars.kv_full[s], 0, y, (int)bg);
-                            tma_load_3d(st + 2 * kHalfK + e * kHalfK, &tmK, &bars.kv_full[s], 64, y, (int)bg);
-                            tma_load_3d(st + 4 * kHalfK + e * 2 * kHalfK, &tmV, &bars.kv_full[s], 0, y, (int)bg);
-                            tma_load_3d(st + 5 * kHalfK + e * 2 * kHalfK, &tmV, &bars.kv_full[s], 64, y, (int)bg);
-                        }
-                        if (s == 0) last0 = r; else last1 = r;
+                    if (m == prev) {
+                        list_mask(lb)[n - 1] |= (uint16_t)msk;
+                    } else if (n < kMaxList) {
+                        list_id(lb)[n] = m;
+                        list_mask(lb)[n] = (uint16_t)msk;
+                        ++n;
                     }
                 }
-                gp = __shfl_sync(0xffffffffu, gp, 0);
-                stop = __shfl_sync(0xffffffffu, stop, 0);
-                if (stop || *abort) break;
+                n = __shfl_sync(0xffffffffu, n, 0);
+                prev = m;
             }
             if (lane == 0) {
-                if (q_issued) (void)mbar_wait(&bars.q_full, (q_issued - 1) & 1, ctx);
-                if (last0 >= 0) (void)mbar_wait(&bars.kv_full[0], last0 & 1, ctx);
-                if (last1 >= 0) (void)mbar_wait(&bars.kv_full[1], last1 & 1, ctx);
-            }
-        } else if (warp == 9) {
-            // ---------------------------------------------------------------- MMA issuer
-            if (lane == 0) {
-                const uint32_t idS2 = idesc_bf16_f32(128, 128, false, false);
-                const uint32_t idS1 = idesc_bf16_f32(128, 64, false, false);
-                const uint32_t idPV = idesc_bf16_f32(128, kD, false, true);
-                int it = 0, gp = 0;
-                bool ok = true;
-                for (int unit = blockIdx.x; unit < n_units && ok; unit += gridDim.x, ++it) {
-                    const int lb = it & 1;
-                    ok = wait_or_abort(&bars.list_full[lb], (it >> 1) & 1, ctx, abort);
-                    if (!ok) break;
-                    const int n = bars.list_n[lb];
-                    const int np = (n + 1) >> 1;
-                    mbar_arrive(&bars.list_empty[lb]);
-                    ok = wait_or_abort(&bars.q_full, it & 1, ctx, abort);
-                    if (!ok) break;
-                    tc_fence_after();
-                    // S_x(j) of tile x; waits for the pair's K/V only when asked.
-                    auto issue_s = [&](int x, int j, bool wait_kv) -> bool {
-                        const int g = gp + j, s = g & 1;
-                        if (wait_kv && !wait_or_abort(&bars.kv_full[s], (g >> 1) & 1, ctx, abort)) return false;
-                        tc_fence_after();
-                        const uint32_t q0 = smem_u32(sm + kOffQ + x * kQBytes);
-                        const uint32_t kb = smem_u32(sm + kOffKV + s * kPairBytes);
-                        const uint32_t id = (2 * j + 1 < n) ? idS2 : idS1;
-    #pragma unroll
-                        for (int ks = 0; ks < kD / 16; ++ks) {
-                            const uint64_t a = sdesc_sw128(q0 + (ks >> 2) * (kQBytes / 2) + (ks & 3) * 32, 16, 1024);
-                            const uint64_t b = sdesc_sw128(kb + (ks >> 2) * 2 * kHalfK + (ks & 3) * 32, 16, 1024);
-                            mma_ss(tmem + kColS + x * 128, a, b, id, ks > 0);
-                        }
-                        mma_commit(&bars.s_full[x]);
-                        return true;
-                    };
-                    auto issue_pv = [&](int x, int j) -> bool {
-                        const int g = gp + j, s = g & 1;
-                        if (!wait_or_abort(&bars.p_full[x], g & 1, ctx, abort)) return false;
-                        tc_fence_after();
-                        const uint32_t vb = smem_u32(sm + kOffKV + s * kPairBytes + 4 * kHalfK);
-                        const uint32_t aP = tmem + kColS + x * 128;
-                        const int ksteps = (2 * j + 1 < n) ? 8 : 4;
-                        for (int ks = 0; ks < ksteps; ++ks) {
-                            const uint64_t b = sdesc_sw128(vb + (ks >> 2) * 2 * kHalfK + (ks & 3) * 16 * 128, kHalfK, 1024);
-                            mma_ts(tmem + kColO + x * 128, aP + ks * 8, b, idPV, (j > 0 || ks > 0) ? 1u : 0u);
-                        }
-                        mma_commit(&bars.pv_done[x]);
-                        return true;
-                    };
-                    if (np > 0) ok = issue_s(0, 0, true) && issue_s(1, 0, false);
-                    for (int j = 0; j < np && ok; ++j) {
-                        const bool more = j + 1 < np;
-                        ok = issue_pv(0, j);
-                        if (ok && more) ok = issue_s(0, j + 1, true);
-                        if (ok) ok = issue_pv(1, j);
-                        if (ok) mma_commit(&bars.kv_empty[(gp + j) & 1]);
-                        if (ok && more) ok = issue_s(1, j + 1, false);
-                    }
-                    mma_commit(&bars.q_empty);  // every MMA reading this unit's Q has been issued
-                    gp += np;
-                }
-                mma_commit(&bars.fin);
-                (void)mbar_wait(&bars.fin, 0, ctx);
+                bars.list_n[lb] = n;
+                mbar_arrive(&bars.list_full[lb]);
             }
             __syncwarp();
+            int stop = 0;
+            if (lane == 0 && n > 0) {
+                // Q_A, Q_B: 16 heads x 8 tokens x 128 columns each, once both issuers are done
+                // with the previous unit's S MMAs.
+                if (kq >= 1 && !wait_or_abort(&bars.q_empty, (kq - 1) & 1, ctx, abort)) stop = 1;
+                if (!stop) {
+                    const int z = (int)((bg / Hkv) * H + (bg % Hkv) * kG);
+                    mbar_arrive_expect_tx(&bars.q_full, 2 * kQBytes);
+                    for (int q = 0; q < 2; ++q) {
+                        tma_load_3d(sm + q * kQBytes, &tmQ, &bars.q_full, 0, i0 + q * kTQ, z);
+                        tma_load_3d(sm + q * kQBytes + kHalfQ, &tmQ, &bars.q_full, 64, i0 + q * kTQ, z);
+                    }
+                    ++kq;
+                }
+                for (int e = 0; e < n && !stop; ++e, ++rc) {
+                    if (rc >= kStages && !wait_or_abort(empty_bar(rc), round_of(rc - kStages), ctx, abort)) {
+                        stop = 1;
+                        break;
+                    }
+                    uint8_t* st = stage_ptr(rc);
+                    uint64_t* fb = full_bar(rc);
+                    mbar_arrive_expect_tx(fb, kStageBytes);
+                    const int y = list_id(lb)[e] * kBlk;
+                    tma_load_3d(st, &tmK, fb, 0, y, (int)bg);
+                    tma_load_3d(st + kHalfBlk, &tmK, fb, 64, y, (int)bg);
+                    tma_load_3d(st + 2 * kHalfBlk, &tmV, fb, 0, y, (int)bg);
+                    tma_load_3d(st + 3 * kHalfBlk, &tmV, fb, 64, y, (int)bg);
+                }
+            }
+            rc = __shfl_sync(0xffffffffu, rc, 0);
+            kq = __shfl_sync(0xffffffffu, kq, 0);
+            stop = __shfl_sync(0xffffffffu, stop, 0);
+            if (stop || *abort) break;
         }
+        if (lane == 0) {  // drain: every copy this warp started has landed before the block exits
+            if (kq > 0) (void)mbar_wait(&bars.q_full, (kq - 1) & 1, ctx);
+            for (uint32_t e = rc > kStages ? rc - kStages : 0; e < rc; ++e)
+                (void)mbar_wait(full_bar(e), round_of(e), ctx);
+        }
+    } else if (warp >= 9) {
+        // ---------------------------------------------------------------- MMA issuers
+        // Warp 9 issues the MMAs of tile A, warp 10 those of tile B (one thread each): a single
+        // thread needs ~50 cycles per tcgen05.mma, more than the 32 of math in an N=64 S MMA, so
+        // two issuers keep the tensor pipe fed and the tiles' chains never wait on each other.
+        // Order per tile: S of round k+1 is issued before PV of round k (two S buffers), so the
+        // tensor core computes the next S while the softmax works on this one.  Each issuer
+        // observes every ring entry in order (so its parity waits never run two uses ahead of a
+        // stage) and returns each entry once: after the tile's PV for a block it used, right away
+        // for a block it did not.  Before it waits for an entry whose stage still holds a block of
+        // its own, it issues that block's PV, so it never holds a stage the producer needs.
+        const int x = warp - 9;
+        if (lane == 0) {
+            const uint32_t idS = idesc_bf16_f32(128, kBlk, false, false);
+            const uint32_t idPV = idesc_bf16_f32(128, kD, false, true);
+            const uint32_t dO = tmem + kColO + x * 128;
+            const uint64_t dQ = sdesc_sw128(smem_u32(sm + x * kQBytes), 16, 1024);
+            int it = 0;
+            uint32_t rc = 0, kq = 0, a = 0;  // ring entries seen, Q tile pairs used, S rounds issued
+            bool ok = true;
+            for (int unit = blockIdx.x; unit < n_units && ok; unit += gridDim.x, ++it) {
+                const int lb = it & 1;
+                ok = wait_or_abort(&bars.list_full[lb], (it >> 1) & 1, ctx, abort);
+                if (!ok) break;
+                const int n = bars.list_n[lb];
+                if (n > 0) {
+                    ok = wait_or_abort(&bars.q_full, kq & 1, ctx, abort);
+                    ++kq;
+                    tc_fence_after();
+                    // Rounds whose S is issued and whose PV is not: at most two, oldest first.
+                    int np = 0;
+                    uint32_t pe0 = 0, pk0 = 0, pe1 = 0, pk1 = 0;  // ring entry, round
+                    bool accum = false;
+                    auto flush_pv = [&]() -> bool {
+                        const uint32_t e = pe0, k = pk0;
+                        pe0 = pe1;
+                        pk0 = pk1;
+                        --np;
+                        if (!wait_or_abort(&bars.p_full[x][k & 1], (k >> 1) & 1, ctx, abort)) return false;
+                        tc_fence_after();
+                        const uint32_t aP = tmem + kColS + x * 128 + (k & 1) * 64;
+                        const uint64_t dV = sdesc_sw128(smem_u32(stage_ptr(e) + 2 * kHalfBlk), kHalfBlk, 1024);
+#pragma unroll
+                        for (int ks = 0; ks < kBlk / 16; ++ks)
+                            mma_ts(dO, aP + ks * 8, dV + (uint64_t)((ks * 16 * 128) >> 4), idPV,
+                                   (accum || ks > 0) ? 1u : 0u);
+                        mma_commit(&bars.pv_done[x][k & 1]);
+                        mma_commit(empty_bar(e));
+                        accum = true;
+                        return true;
+                    };
+                    for (int b = 0; b < n && ok; ++b) {
+                        const uint32_t e = rc + b;
+                        const bool act = ((list_mask(lb)[b] >> (8 * x)) & 0xffu) != 0;
+                        while (ok && np > 0 && pe0 + kStages <= e) ok = flush_pv();
+                        if (ok && np == 2) ok = flush_pv();
+                        if (!ok) break;
+                        if (!(ok = wait_or_abort(full_bar(e), round_of(e), ctx, abort))) break;
+                        if (!act) {  // no token of this tile chose the block
+                            mbar_arrive(empty_bar(e));
+                            continue;
+                        }
+                        tc_fence_after();
+                        const uint32_t dS = tmem + kColS + x * 128 + (a & 1) * 64;
+                        const uint64_t dK = sdesc_sw128(smem_u32(stage_ptr(e)), 16, 1024);
+#pragma unroll
+                        for (int ks = 0; ks < kD / 16; ++ks) {
+                            const uint32_t off = ((ks >> 2) * kHalfQ + (ks & 3) * 32) >> 4;
+                            const uint32_t offk = ((ks >> 2) * kHalfBlk + (ks & 3) * 32) >> 4;
+                            mma_ss(dS, dQ + off, dK + offk, idS, ks > 0 ? 1u : 0u);
+                        }
+                        mma_commit(&bars.s_full[x][a & 1]);
+                        if (np == 0) {
+                            pe0 = e;
+                            pk0 = a;
+                        } else {
+                            pe1 = e;
+                            pk1 = a;
+                        }
+                        ++np;
+                        ++a;
+                        if (np == 2) ok = flush_pv();
+                    }
+                    mma_commit(&bars.q_empty);  // every S MMA reading this unit's Q is issued
+                    while (ok && np > 0) ok = flush_pv();
+                    rc += n;
+                }
+                mbar_arrive(&bars.list_empty[lb]);
+            }
+            mma_commit(&bars.fin[x]);
+            (void)mbar_wait(&bars.fin[x], 0, ctx);
+        }
+        __syncwarp();
     } else {
-        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
         // ---------------------------------------------------------------- softmax + epilogue
         // Warpgroup x (0: tile A, 1: tile B); thread = row r of the tile = TMEM lane r.  The two
         // warpgroups meet only at one named barrier per unit (bar.sync 1, 256 threads).  A failed
@@ -368,7 +396,7 @@ sparse_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
         const int t = x * kTQ + r % kTQ, hh = r / kTQ;   // token within the unit, head
         const uint32_t lane_base = tmem_lane_base(warp);
         const uint32_t colO = tmem + lane_base + kColO + x * 128;
-        const uint32_t colS = tmem + lane_base + kColS + x * 128;
+        const uint32_t colS0 = tmem + lane_base + kColS + x * 128;  // + 64 for the second buffer
         volatile int* sm_stop = &bars.sm_stop;
         int nbar = 0;
         bool dead = false;
@@ -377,12 +405,12 @@ sparse_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
             atomicCAS(&bars.sm_stop, 0, nbar + 1);
             *abort = 1;
         };
-        int it = 0, gp = 0;
+        int it = 0;
+        uint32_t a = 0;  // rounds of this tile (one per active block), in the issuer's numbering
         for (int unit = blockIdx.x; unit < n_units; unit += gridDim.x, ++it) {
             const int lb = it & 1;
             if (!dead && !mbar_wait(&bars.list_full[lb], (it >> 1) & 1, ctx)) fail();
             const int n = dead ? 0 : bars.list_n[lb];
-            const int np = (n + 1) >> 1;
             const int32_t* ids = list_id(lb);
             const uint16_t* msks = list_mask(lb);
             const int64_t bg = unit / units_per_seq;
@@ -390,43 +418,25 @@ sparse_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
             const int c = i0 / kBlk;
             const int i = i0 + t;
             float m_run = -INFINITY, l = 0.f;  // running max (scaled log2 units), row sum
-            for (int j = 0; j < np; ++j) {
-                const int g = gp + j;
-                const bool two = 2 * j + 1 < n;
-                const int blk_a = ids[2 * j];
-                const int blk_b = two ? ids[2 * j + 1] : -1;
-                const bool sel_a = (msks[2 * j] >> t) & 1;
-                const bool sel_b = two && ((msks[2 * j + 1] >> t) & 1);
-                // last visible key of each block (-1: none)
-                const int lim_a = !sel_a ? -1 : (blk_a == c ? i - blk_a * kBlk : kBlk - 1);
-                const int lim_b = !sel_b ? -1 : (blk_b == c ? i - blk_b * kBlk : kBlk - 1);
-                if (!dead && !mbar_wait(&bars.s_full[x], g & 1, ctx)) fail();
+            int last = -1;
+            for (int b = 0; b < n; ++b) {
+                const unsigned msk = msks[b];
+                if (((msk >> (8 * x)) & 0xffu) == 0) continue;  // no token of this tile chose it
+                const int blk = ids[b];
+                const bool diag = blk == c;                      // uniform over the warpgroup
+                const bool sel = (msk >> t) & 1u;
+                const int lim = !sel ? -1 : (diag ? i - blk * kBlk : kBlk - 1);  // last visible key
+                const uint32_t j = a & 1u, colS = colS0 + j * 64;
+                if (!dead && !mbar_wait(&bars.s_full[x][j], (a >> 1) & 1u, ctx)) fail();
                 tc_fence_after();
                 const bool go = !__any_sync(0xffffffffu, dead);
-                // The pair's S row is read from TMEM once, into 128 registers.  Blocks the token did
-                // not select drop out through the exponent bias (2^-inf = 0); the causal mask inside
-                // the diagonal block, the one block a token sees in part, costs a select per element
-                // on the pair that holds it only.
-                const bool diag = (blk_a == c) || (blk_b == c);  // uniform over the CTA
-                uint32_t sr[128];
+                uint32_t sr[64];
                 float mx = -INFINITY;
                 if (go) {
                     tmem_ld32(colS, sub32(sr, 0));
                     tmem_ld32(colS + 32, sub32(sr, 1));
-                    if (two) {
-                        tmem_ld32(colS + 64, sub32(sr, 2));
-                        tmem_ld32(colS + 96, sub32(sr, 3));
-                    }
                     tmem_ld_wait();
-                    float ma, mb = -INFINITY;
-                    if (diag) {
-                        ma = max64_masked(sr, lim_a);
-                        if (two) mb = max64_masked(sr + 64, lim_b);
-                    } else {
-                        ma = lim_a >= 0 ? max64(sr) : -INFINITY;
-                        if (two && lim_b >= 0) mb = max64(sr + 64);
-                    }
-                    mx = fmaxf(ma, mb);
+                    mx = diag ? max64_masked(sr, lim) : (lim >= 0 ? max64(sr) : -INFINITY);
                 }
                 mx *= sl2;
                 const bool grow = mx > m_run + 8.f;
@@ -436,24 +446,19 @@ sparse_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                     l = (m_run == -INFINITY) ? 0.f : l * alpha;
                     m_run = mx;
                 }
-                // p = 2^(s * sl2 - m) as bf16 pairs over the first 64 columns of S (already read).
-                if (go && !__any_sync(0xffffffffu, dead)) {
-                    const float nb_a = lim_a >= 0 ? -m_run : -INFINITY;
-                    const float nb_b = lim_b >= 0 ? -m_run : -INFINITY;
+                // p = 2^(s * sl2 - m) as bf16 pairs over the first 32 columns of S (already read).
+                if (go) {
+                    const float nb = lim >= 0 ? -m_run : -INFINITY;
                     float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-                    if (diag) exp_block<true>(sr, sl2, nb_a, lim_a, colS, a0, a1, a2, a3);
-                    else exp_block<false>(sr, sl2, nb_a, lim_a, colS, a0, a1, a2, a3);
-                    if (two) {
-                        if (diag) exp_block<true>(sr + 64, sl2, nb_b, lim_b, colS + 32, a0, a1, a2, a3);
-                        else exp_block<false>(sr + 64, sl2, nb_b, lim_b, colS + 32, a0, a1, a2, a3);
-                    }
+                    if (diag) exp_block<true>(sr, sl2, nb, lim, colS, a0, a1, a2, a3);
+                    else exp_block<false>(sr, sl2, nb, lim, colS, a0, a1, a2, a3);
                     l += (a0 + a1) + (a2 + a3);
                 }
                 // Rescale O_x by 2^(m_old - m_new) where the max grew past the threshold (before
-                // this thread releases P, so before PV(j) can add into O_x).
+                // this thread releases P, so before this block's PV can add into O_x).
                 if (go && __any_sync(0xffffffffu, need_rescale)) {
-                    if (j >= 1) {  // the previous PV into O_x must be complete
-                        if (!dead && !mbar_wait(&bars.pv_done[x], (g - 1) & 1, ctx)) fail();
+                    if (last >= 0) {  // the tile's previous PV into O_x must be complete
+                        if (!dead && !mbar_wait(&bars.pv_done[x][last & 1], ((uint32_t)last >> 1) & 1u, ctx)) fail();
                     }
                     if (!__any_sync(0xffffffffu, dead)) {
                         tc_fence_after();
@@ -471,13 +476,14 @@ sparse_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&bars.p_full[x]);
+                if (lane == 0) mbar_arrive(&bars.p_full[x][j]);
+                last = (int)a;
+                ++a;
             }
-            // Epilogue: O_x / l -> bf16 -> global.
+            // Epilogue: O_x / l -> bf16 -> global (zeros when the tile saw no block).
             const int64_t orow = (((bg / Hkv) * H + (bg % Hkv) * kG + hh) * (int64_t)N + i) * kD;
-            if (np > 0) {
-                const int gl = gp + np - 1;
-                if (!dead && !mbar_wait(&bars.pv_done[x], gl & 1, ctx)) fail();
+            if (last >= 0) {
+                if (!dead && !mbar_wait(&bars.pv_done[x][last & 1], ((uint32_t)last >> 1) & 1u, ctx)) fail();
                 if (!__any_sync(0xffffffffu, dead)) {
                     tc_fence_after();
                     const float inv = l > 0.f ? 1.f / l : 0.f;
@@ -504,7 +510,6 @@ sparse_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                 uint4* d4 = reinterpret_cast<uint4*>(out + orow);
                 for (int q = 0; q < kD / 8; ++q) d4[q] = make_uint4(0, 0, 0, 0);
             }
-            gp += np;
             asm volatile("bar.sync 1, 256;" ::: "memory");
             ++nbar;
             if (tid == 0 && !dead) mbar_arrive(&bars.list_empty[lb]);
@@ -556,16 +561,6 @@ cudaError_t launch_sparse_prefill_tc(const void* q, const void* k, const void* v
     }
     cudaError_t e = ensure_smem<sparse_prefill_tc_kernel>(kSmemBytes);
     if (e != cudaSuccess) return e;
-    // setmaxnreg.inc waits until the block's pool has the registers, so launch only when the
-    // compiled per-thread count covers the split.
-    static int regs_ok = -1;
-    if (regs_ok < 0) {
-        cudaFuncAttributes fa;
-        e = cudaFuncGetAttributes(&fa, sparse_prefill_tc_kernel);
-        if (e != cudaSuccess) return e;
-        regs_ok = fa.numRegs * kThreads >= 256 * kRegsSoftmax + 128 * kRegsOther ? 1 : 0;
-    }
-    if (!regs_ok) return cudaErrorNotSupported;
     const int units_per_seq = (N + kUT - 1) / kUT;
     const int n_units = units_per_seq * B * Hkv;
     const int grid = n_units < num_sms ? n_units : num_sms;
