@@ -11,6 +11,11 @@
 //     a_mode 1: A is first copied into TMEM (bf16 pairs packed per 32-bit column) and the
 //     MMA reads it from there instead of shared memory.
 //   Returns 0 on success, a negative value for bad arguments, or a CUDA error code.
+//
+//   sala_selftest_exp2_poly(y, out, n, stream)
+//     out[i] = 2^y[i] through the FMA-pipe polynomial the softmax kernels use (fastexp.cuh), so
+//     the tests can check it against an exact 2^y.  y, out: n fp32 values on the device.
+#include "fastexp.cuh"
 #include "ptx.cuh"
 #include "tmap.cuh"
 
@@ -141,5 +146,24 @@ extern "C" int sala_selftest_mma(const void* A, const void* B, float* D, int N, 
     DevCtx ctx{status, 1000000000ull};
     selftest_mma_kernel<<<1, 128, smem, static_cast<cudaStream_t>(stream)>>>(
         tA, tB, static_cast<const __nv_bfloat16*>(A), D, N, K, b_mn_major, a_mode, ctx);
+    return (int)cudaGetLastError();
+}
+
+namespace {
+__global__ void exp2_poly_kernel(const float* __restrict__ y, float* __restrict__ out, int n) {
+    const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+    if (i >= n) return;
+    float a = y[i], b = i + 1 < n ? y[i + 1] : 0.f;
+    sala::exp2_poly2(a, b);
+    out[i] = a;
+    if (i + 1 < n) out[i + 1] = b;
+}
+}  // namespace
+
+extern "C" int sala_selftest_exp2_poly(const float* y, float* out, int n, void* stream) {
+    if (n < 0 || (n > 0 && (!y || !out))) return -1;
+    if (n == 0) return 0;
+    const int threads = 256, pairs = (n + 1) / 2;
+    exp2_poly_kernel<<<(pairs + threads - 1) / threads, threads, 0, (cudaStream_t)stream>>>(y, out, n);
     return (int)cudaGetLastError();
 }

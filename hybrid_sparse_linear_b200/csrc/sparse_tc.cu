@@ -28,6 +28,7 @@
 // tile A, warp 10 those of tile B (one thread each).  Every wait is bounded; a timeout sets the
 // status word, the roles wind down, and the kernel waits (bounded) for its own copies and MMAs
 // before it frees TMEM.
+#include "fastexp.cuh"
 #include "kernels.h"
 #include "ptx.cuh"
 #include "tmap.cuh"
@@ -119,9 +120,15 @@ __device__ __forceinline__ float max64_masked(const uint32_t* s, int lim) {
     return fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
 }
 
+// Which key pairs take the FMA-pipe exp2 instead of the multi-function unit (ex2.approx): one pair
+// in kPolyEvery, outside the diagonal block.  Per block both tiles' softmax warps on a scheduler
+// need 16384 exponentials, 1024 cycles of the multi-function unit at 16 per cycle, as long as the
+// block's MMAs; moving a quarter to the FMA pipe takes that unit off the critical path.
+constexpr int kPolyEvery = 4;
+
 // p = 2^(s * sl2 + nb) for 64 keys, packed to 32 bf16 pairs and stored to TMEM columns
 // taddr .. taddr+31 in two pieces of 16; sums added to a0..a3.  kMasked zeroes the keys past lim
-// (the causal edge).
+// (the causal edge) and uses ex2.approx throughout, so masked keys give exact zeros.
 template <bool kMasked>
 __device__ __forceinline__ void exp_block(const uint32_t* s, float sl2, float nb, int lim,
                                           uint32_t taddr, float& a0, float& a1, float& a2,
@@ -134,7 +141,15 @@ __device__ __forceinline__ void exp_block(const uint32_t* s, float sl2, float nb
             const int k = 32 * h + 2 * q;
             float y0, y1;
             fma2_bcast(y0, y1, __uint_as_float(s[k]), __uint_as_float(s[k + 1]), sl2, nb);
-            float p0 = ex2(y0), p1 = ex2(y1);
+            float p0, p1;
+            if (!kMasked && q % kPolyEvery == kPolyEvery - 1) {
+                p0 = y0;
+                p1 = y1;
+                exp2_poly2(p0, p1);
+            } else {
+                p0 = ex2(y0);
+                p1 = ex2(y1);
+            }
             if (kMasked) {
                 p0 = k <= lim ? p0 : 0.f;
                 p1 = k + 1 <= lim ? p1 : 0.f;
@@ -307,7 +322,12 @@ sparse_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
             const uint32_t idS = idesc_bf16_f32(128, kBlk, false, false);
             const uint32_t idPV = idesc_bf16_f32(128, kD, false, true);
             const uint32_t dO = tmem + kColO + x * 128;
-            const uint64_t dQ = sdesc_sw128(smem_u32(sm + x * kQBytes), 16, 1024);
+            // Shared-memory descriptors by halves: one high half for every operand here (stride
+            // 1024 B, 128-byte swizzle); low halves = address | leading offset, plus the K step.
+            const uint32_t dhi = sdesc_sw128_hi(1024);
+            const uint32_t q_lo = sdesc_sw128_lo(smem_u32(sm + x * kQBytes), 16);
+            const uint32_t ring_lo = sdesc_sw128_lo(smem_u32(sm + kOffRing), 16);
+            const uint32_t ring_v_lo = sdesc_sw128_lo(smem_u32(sm + kOffRing + 2 * kHalfBlk), kHalfBlk);
             int it = 0;
             uint32_t rc = 0, kq = 0, a = 0;  // ring entries seen, Q tile pairs used, S rounds issued
             bool ok = true;
@@ -332,11 +352,11 @@ sparse_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                         if (!wait_or_abort(&bars.p_full[x][k & 1], (k >> 1) & 1, ctx, abort)) return false;
                         tc_fence_after();
                         const uint32_t aP = tmem + kColS + x * 128 + (k & 1) * 64;
-                        const uint64_t dV = sdesc_sw128(smem_u32(stage_ptr(e) + 2 * kHalfBlk), kHalfBlk, 1024);
+                        const uint32_t v_lo = ring_v_lo + (e % kStages) * (kStageBytes >> 4);
 #pragma unroll
                         for (int ks = 0; ks < kBlk / 16; ++ks)
-                            mma_ts(dO, aP + ks * 8, dV + (uint64_t)((ks * 16 * 128) >> 4), idPV,
-                                   (accum || ks > 0) ? 1u : 0u);
+                            mma_ts_lohi(dO, aP + ks * 8, v_lo + ((ks * 16 * 128) >> 4), dhi, idPV,
+                                        (accum || ks > 0) ? 1u : 0u);
                         mma_commit(&bars.pv_done[x][k & 1]);
                         mma_commit(empty_bar(e));
                         accum = true;
@@ -355,13 +375,12 @@ sparse_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                         }
                         tc_fence_after();
                         const uint32_t dS = tmem + kColS + x * 128 + (a & 1) * 64;
-                        const uint64_t dK = sdesc_sw128(smem_u32(stage_ptr(e)), 16, 1024);
+                        const uint32_t k_lo = ring_lo + (e % kStages) * (kStageBytes >> 4);
 #pragma unroll
-                        for (int ks = 0; ks < kD / 16; ++ks) {
-                            const uint32_t off = ((ks >> 2) * kHalfQ + (ks & 3) * 32) >> 4;
-                            const uint32_t offk = ((ks >> 2) * kHalfBlk + (ks & 3) * 32) >> 4;
-                            mma_ss(dS, dQ + off, dK + offk, idS, ks > 0 ? 1u : 0u);
-                        }
+                        for (int ks = 0; ks < kD / 16; ++ks)
+                            mma_ss_lohi(dS, q_lo + (((ks >> 2) * kHalfQ + (ks & 3) * 32) >> 4),
+                                        k_lo + (((ks >> 2) * kHalfBlk + (ks & 3) * 32) >> 4), dhi, idS,
+                                        ks > 0 ? 1u : 0u);
                         mma_commit(&bars.s_full[x][a & 1]);
                         if (np == 0) {
                             pe0 = e;
@@ -486,7 +505,8 @@ sparse_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                 if (!dead && !mbar_wait(&bars.pv_done[x][last & 1], ((uint32_t)last >> 1) & 1u, ctx)) fail();
                 if (!__any_sync(0xffffffffu, dead)) {
                     tc_fence_after();
-                    const float inv = l > 0.f ? 1.f / l : 0.f;
+                    // No visible key (m_run = -inf): zeros (masked keys may have added 2^-125 terms).
+                    const float inv = (m_run != -INFINITY && l > 0.f) ? 1.f / l : 0.f;
 #pragma unroll 1
                     for (int c0 = 0; c0 < kD; c0 += 32) {
                         uint32_t orr[32];

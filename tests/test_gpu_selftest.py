@@ -20,6 +20,8 @@ def st():
     lib = ctypes.CDLL(SELFTEST)
     lib.sala_selftest_mma.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int] * 4 + [ctypes.c_void_p] * 2
     lib.sala_selftest_mma.restype = ctypes.c_int
+    lib.sala_selftest_exp2_poly.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p]
+    lib.sala_selftest_exp2_poly.restype = ctypes.c_int
     return lib
 
 
@@ -47,6 +49,33 @@ def test_mma_tile(st, N, K, b_mn_major, a_mode):
     assert int(status.item()) == 0, "device wait timed out"
     err = (D.double().cpu() - ref).abs().max().item()
     assert err <= 1e-4 * ref.abs().max().item(), f"max err {err}"
+
+
+def test_exp2_polynomial_against_exact(st):
+    """The FMA-pipe 2^y of the softmax: relative error within the fitted bound (7.5e-5, plus fp32
+    rounding of the argument reduction) against an exact 2^y, over the range the softmax feeds it
+    (y <= 8, including the stale-max excess) down to the clamp at -125; below the clamp (and at
+    -inf, a masked key) it returns 2^-125 scaled by the polynomial, a normal number far below any
+    ulp of the sums it enters."""
+    g = torch.Generator().manual_seed(11)
+    y = torch.cat([torch.linspace(-125.0, 8.0, 200001, dtype=torch.float64),
+                   torch.rand(100000, generator=g, dtype=torch.float64) * 40 - 32,
+                   torch.tensor([0.0, 0.5, -0.5, 1.0, -1.0, 7.999, 8.0, -124.999, -125.0])]).float()
+    yd = y.cuda()
+    out = torch.empty_like(yd)
+    assert st.sala_selftest_exp2_poly(yd.data_ptr(), out.data_ptr(), y.numel(),
+                                      torch.cuda.current_stream().cuda_stream) == 0
+    torch.cuda.synchronize()
+    ref = torch.exp2(y.double())
+    rel = ((out.cpu().double() - ref) / ref).abs()
+    assert rel.max().item() <= 8e-5, f"max rel err {rel.max().item()}"
+    low = torch.tensor([-126.0, -200.0, -1e30, float("-inf")]).cuda()
+    lo_out = torch.empty_like(low)
+    assert st.sala_selftest_exp2_poly(low.data_ptr(), lo_out.data_ptr(), 4,
+                                      torch.cuda.current_stream().cuda_stream) == 0
+    torch.cuda.synchronize()
+    v = lo_out.cpu().double()
+    assert bool(((v > 0) & (v <= 2.0 ** -125 * 1.0001)).all()), v
 
 
 def test_wait_timeout_is_reported_not_fatal():
