@@ -290,7 +290,7 @@ def run_decode(sala, synth, torch, steps, warmup, stream):
         kbar = sala.block_compress(sl.k, stream=stream)
         sp.append((sl.q[:, :, 0].contiguous(), sl.k, sl.v, kbar))
     ws_bytes = sala.sparse_decode_workspace_bytes(1, H, HKV, pos, TOPK, N_INIT, N_LOCAL, D)
-    ws = torch.empty(max(ws_bytes, 16), device=dev, dtype=torch.uint8)
+    ws = torch.zeros(max(ws_bytes, 256), device=dev, dtype=torch.uint8)  # counters start at 0
     o = torch.empty((1, H, D), device=dev, dtype=torch.bfloat16)
     flush = torch.empty(512 << 20, device=dev, dtype=torch.uint8)
     torch.cuda.synchronize()
@@ -328,11 +328,44 @@ def run_decode(sala, synth, torch, steps, warmup, stream):
         torch.cuda.synchronize()
     sala.check_status(stream)
     us = [a.elapsed_time(b) * 1000.0 for a, b in times]
+
+    def per_layer(kind):
+        # The same calls of one kind only, captured and replayed the same way: where the time goes.
+        calls = [l for l in range(N_LAYERS) if (l in SPARSE_LAYERS) == (kind == "sparse")]
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            with torch.cuda.graph(g, stream=stream):
+                for l in calls:
+                    if kind == "sparse":
+                        q, kc, vc, kbar = sp[SPARSE_LAYERS.index(l)]
+                        sala.sparse_decode(q, kc, vc, kbar, pos, TOPK, N_INIT, N_LOCAL, o=o,
+                                           workspace=ws, stream=stream)
+                    else:
+                        S, q, k, v = lin[l - sum(1 for s in SPARSE_LAYERS if s < l)]
+                        sala.linear_decode(q, k, v, lam, S, o=o, stream=stream)
+            for _ in range(warmup):
+                g.replay()
+            ts = []
+            for _ in range(steps):
+                flush.zero_()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                g.replay()
+                b.record(stream)
+                ts.append((a, b))
+            torch.cuda.synchronize()
+        del g
+        return statistics.median(a.elapsed_time(b) * 1000.0 for a, b in ts) / len(calls)
+
+    lin_us, sp_us = per_layer("linear"), per_layer("sparse")
+    sala.check_status(stream)
     del graph, lin, sp, ws, flush
     torch.cuda.empty_cache()
-    # launches per token: linear 1 each; sparse = select (2) + attention (2)
+    # launches per token: linear 1 each; sparse 1 each (scoring, top-k, attention and combine in
+    # one cooperative launch)
     return {"us_per_token": statistics.median(us), "us_min": min(us), "samples": len(us),
-            "launches_per_token": 24 * 1 + 8 * 4}
+            "launches_per_token": 24 * 1 + 8 * 1,
+            "us_per_linear_layer": lin_us, "us_per_sparse_layer": sp_us}
 
 
 def run_e2e(sala, synth, torch, steps, warmup):
@@ -590,8 +623,11 @@ def main():
                           "bytes_per_token": db["step"], "achieved_gbs": gbs,
                           "hbm_frac": gbs / peaks["hbm_gbs"],
                           "launches_per_token": dec["launches_per_token"],
+                          "us_per_linear_layer": dec["us_per_linear_layer"],
+                          "us_per_sparse_layer": dec["us_per_sparse_layer"],
                           "timing": "CUDA events around one CUDA-graph replay of a token's 32 layer "
-                                    "calls, L2 flushed before each token, median"}
+                                    "calls, L2 flushed before each token, median; per-layer figures "
+                                    "from graphs of one kind of call only"}
     if "e2e" in phases:
         e = run_e2e(sala, synth, torch, max(1, min(args.steps, 2)), 1)
         line["e2e"] = {"value": ws * N_TOK / (max_over_ranks(e["ms_per_step"], "cuda") / 1000.0),

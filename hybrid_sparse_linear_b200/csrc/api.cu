@@ -298,7 +298,10 @@ size_t sala_sparse_decode_workspace(int B, int H, int Hkv, int pos, int block, i
     size_t sel = sala::rowwise_topk_workspace(B, Hkv, 1, pos, topk);
     size_t idx_bytes = (size_t)B * Hkv * slots * sizeof(int32_t);
     auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
-    return up(a) + up(sel) + up(idx_bytes);
+    // [0, 256) holds the one-launch path's barrier words in every layout.
+    const size_t multi = 256 + up(a) + up(sel) + up(idx_bytes);
+    const size_t fused = up(sala::sparse_decode_fused_workspace(B, H, Hkv, pos, topk, n_init, n_local, d));
+    return multi > fused ? multi : fused;
 }
 
 sala_status sala_sparse_decode(const void* q, const void* kcache, const void* vcache,
@@ -325,9 +328,15 @@ sala_status sala_sparse_decode(const void* q, const void* kcache, const void* vc
     s = get_ctx(&ctx);
     if (s != SALA_OK) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    {
+        const cudaError_t e = sala::launch_sparse_decode_fused(
+            to_dt(dt), q, kcache, vcache, kbar, idx_in, idx_out, o, B, H, Hkv, pos, Tmax, nb_cap, d,
+            topk, n_init, n_local, scale, workspace, workspace_bytes, st, ctx);
+        if (e != cudaErrorNotSupported) return launched(e, "sparse_decode");
+    }
     const int slots = n_init + n_local + topk;
     auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
-    char* w = static_cast<char*>(workspace);
+    char* w = static_cast<char*>(workspace) + 256;  // [0, 256): the one-launch path's barrier words
     void* ws_attn = w;
     w += up(sala::sparse_decode_attn_workspace(B, H, Hkv, slots, d));
     void* ws_sel = w;

@@ -55,6 +55,19 @@ cudaError_t launch_sparse_prefill_tc(const void* q, const void* k, const void* v
                                      int d, int slots, float scale, cudaStream_t st, DevCtx ctx);
 bool sparse_prefill_tc_supported(int H, int Hkv, int d);
 size_t sparse_decode_attn_workspace(int B, int H, int Hkv, int slots, int d);
+// Sparse decode in one cooperative launch (scoring, top-k, attention, combine).  Returns
+// cudaErrorNotSupported, launching nothing, when the problem does not fit it (k > 64, more than
+// 80 slots, more than 16 heads per group, more than 8192 span-list keys, a grid that cannot be
+// resident at once, or a smaller workspace); the caller then uses the multi-kernel path.
+// Workspace: [0, 256) barrier words (zero before the first call, left zero), then its data.
+size_t sparse_decode_fused_workspace(int B, int H, int Hkv, int pos, int topk, int n_init,
+                                     int n_local, int d);
+cudaError_t launch_sparse_decode_fused(DType dt, const void* q, const void* kc, const void* vc,
+                                       const void* kbar, const int32_t* idx_in, int32_t* idx_out,
+                                       void* o, int B, int H, int Hkv, int pos, int Tmax,
+                                       int nb_cap, int d, int topk, int n_init, int n_local,
+                                       float scale, void* ws, size_t ws_bytes, cudaStream_t st,
+                                       DevCtx ctx);
 cudaError_t launch_sparse_decode_attn(DType dt, const void* q, const void* kc, const void* vc,
                                       const int32_t* idx, void* o, int B, int H, int Hkv,
                                       int pos, int Tmax, int d, int slots, float scale, void* ws,

@@ -12,8 +12,10 @@
 // The area is kNoallocScratchBytes (4 MiB) per GPU and exists on every GPU that loads the library
 // until the process exits.  All calls on a GPU share it, so two calls that may run at the same
 // time on that GPU (different streams, no ordering between them) race on it and must not be made.
-// The area keeps whatever the previous call left there; none of it needs to start at zero,
-// because every byte a call reads it has written earlier in the same call.
+// The area keeps whatever the previous call left there.  Its first 256 bytes are the counters of
+// the one-launch path's grid barrier: zero when the library loads (a __device__ array starts
+// zeroed) and put back to zero by every call that completes; every other byte a call reads it has
+// written earlier in the same call.
 #include <mutex>
 
 #include "../../include/sala.h"

@@ -1,0 +1,738 @@
+// Sparse decode in one launch: block scoring, top-k selection and attention for one query token
+// per (batch, KV group), at any context length the workspace covers.
+//
+// One query row per KV group meets a context of up to millions of keys, so every phase is a
+// memory stream with little arithmetic: the scores read the whole block-key table k_bar (8 MiB at
+// 2^20 tokens and 2 KV heads), the attention reads the ~67 selected K/V blocks (4 MiB).  Spread
+// over the GPU, each phase is one round of loads.  The kernel runs all of them in one cooperative
+// launch (all CTAs resident, so a grid-wide barrier is safe), with `cpg` CTAs per (batch, group):
+//   A  CTA j scores candidate span j (256 blocks): one thread per block, 256 bytes of k_bar each,
+//      then keeps the span's top-k keys (block-wide radix select on 64-bit keys).
+//   -- grid barrier --
+//   B  every CTA of the group merges all spans' lists into the group's top-k (the same
+//      deterministic result in each CTA, so no second exchange is needed) and forms the
+//      ascending slot list: init blocks, top-k, local blocks, -1 padding.
+//   C  CTA j attends slot j (and j + cpg, ...): K and V of the block staged in shared memory,
+//      G heads' logits, a per-head softmax partial (max, sum, sum of p v) written to workspace.
+//   -- grid barrier --
+//   D  CTA j combines the partials of one (head, 32-column) piece of the output.
+// Selection keys pack (orderable score << 32 | ~block): one unsigned compare orders by score,
+// then by lower block index, so the k-th largest key is unique and ties go to the lower block.
+//
+// The grid barrier counts arrivals in the low half of the workspace's first word, which must be
+// zero before the first call; the last CTA to arrive puts it back to zero, so every call that
+// completes leaves it as it found it.  Waits are bounded (the device status word records a
+// timeout).
+#include <atomic>
+#include <mutex>
+
+#include "kernels.h"
+
+namespace sala {
+namespace {
+
+constexpr int kBlk = 64;
+constexpr int kSpan = 256;
+constexpr int kThreads = 256;
+constexpr int kCap = 64;       // largest k
+constexpr int kMaxSlots = 80;  // n_init + n_local + k
+constexpr int kMaxG = 16;
+constexpr int kMergeE = 32;    // keys per thread in phase B: spans * k <= 8192
+
+__device__ __forceinline__ uint64_t sel_key_u(float score, int blk) { return sel_key(score, blk); }
+
+// Grid-wide barrier for a cooperative launch on one 32-bit word: arrivals of the current barrier
+// in the low 16 bits (zero between barriers), a generation count above.  The arrival's atomic
+// returns the generation it belongs to; the last arrival clears the count and bumps the generation
+// in one atomic.  Returns false after a timeout.
+__device__ bool grid_barrier(unsigned* word, unsigned nblocks, const DevCtx& ctx, int* s_ok) {
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int ok = 1;
+        __threadfence();
+        const unsigned old = atomicAdd(word, 1u);
+        if ((old & 0xFFFFu) == nblocks - 1) {
+            atomicAdd(word, 0x10000u - nblocks);
+        } else {
+            const unsigned g0 = old >> 16;
+            const uint64_t t0 = globaltimer_ns();
+            while ((*reinterpret_cast<volatile unsigned*>(word) >> 16) == g0) {
+                if (globaltimer_ns() - t0 > ctx.wait_limit_ns) {
+                    flag(ctx, kStatusTimeout);
+                    ok = 0;
+                    break;
+                }
+                __nanosleep(20);
+            }
+        }
+        __threadfence();
+        *s_ok = ok;
+    }
+    __syncthreads();
+    return *s_ok != 0;
+}
+
+struct SelSmem {
+    unsigned hist[256];
+    int d, above, eq, n;
+    int nvalid;
+};
+
+// Block-wide: finds the K-th largest nonzero key among the E keys per thread (keys distinct).  On
+// return, winner(key) = key != 0 && (key & mask) >= prefix picks exactly min(K, #nonzero) keys.
+template <int E>
+__device__ void block_kth(const uint64_t (&key)[E], int K, SelSmem& s, uint64_t& prefix,
+                          uint64_t& mask) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    int nv = 0;
+#pragma unroll
+    for (int e = 0; e < E; ++e) nv += key[e] != 0ull;
+    if (tid == 0) s.nvalid = 0;
+    __syncthreads();
+    nv = __reduce_add_sync(0xffffffffu, nv);
+    if (lane == 0 && nv) atomicAdd(&s.nvalid, nv);
+    __syncthreads();
+    prefix = 0;
+    mask = 0;
+    if (s.nvalid <= K) {  // every nonzero key wins
+        prefix = 1;
+        mask = ~0ull;
+        return;
+    }
+    int krem = K;
+    for (int shift = 56; shift >= 0; shift -= 8) {
+        s.hist[tid] = 0;
+        __syncthreads();
+        // Keys share their high bytes (nearby scores), so a plain atomic per key would serialize
+        // on one bin: lanes with the same digit add once, through their leader.
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            const bool m = key[e] && (key[e] & mask) == prefix;
+            if (!__any_sync(0xffffffffu, m)) continue;
+            const unsigned dig = m ? (unsigned)((key[e] >> shift) & 255u) : 256u;
+            const unsigned peers = __match_any_sync(0xffffffffu, dig);
+            if (m && lane == __ffs(peers) - 1) atomicAdd(&s.hist[dig], (unsigned)__popc(peers));
+        }
+        __syncthreads();
+        if (warp == 0) {
+            // lane l holds bins 255-8l .. 248-8l (descending order)
+            int cnt[8], sum = 0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                cnt[i] = (int)s.hist[255 - 8 * lane - i];
+                sum += cnt[i];
+            }
+            int incl = sum;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, incl, off);
+                if (lane >= off) incl += v;
+            }
+            const int excl = incl - sum;
+            if (excl < krem && krem <= incl) {
+                int run = excl;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    if (run + cnt[i] >= krem) {
+                        s.d = 255 - 8 * lane - i;
+                        s.above = run;
+                        s.eq = cnt[i];
+                        break;
+                    }
+                    run += cnt[i];
+                }
+            }
+        }
+        __syncthreads();
+        krem -= s.above;
+        prefix |= (uint64_t)s.d << shift;
+        mask |= 0xFFull << shift;
+        if (s.eq == krem) break;  // every key with this prefix is a winner
+    }
+}
+
+// Ascending bitonic sort of 64 ints held two per lane (position 2*lane + j).
+__device__ __forceinline__ void warp_sort64(int& x0, int& x1, int lane) {
+#pragma unroll
+    for (int k = 2; k <= 64; k <<= 1) {
+#pragma unroll
+        for (int s = k >> 1; s > 0; s >>= 1) {
+            if (s == 1) {
+                const bool asc = ((2 * lane) & k) == 0;
+                const int lo = min(x0, x1), hi = max(x0, x1);
+                x0 = asc ? lo : hi;
+                x1 = asc ? hi : lo;
+            } else {
+                const int lm = s >> 1;
+                const int y0 = __shfl_xor_sync(0xffffffffu, x0, lm);
+                const int y1 = __shfl_xor_sync(0xffffffffu, x1, lm);
+                const int p0 = 2 * lane, p1 = 2 * lane + 1;
+                const bool asc0 = (p0 & k) == 0, low0 = (p0 & s) == 0;
+                const bool asc1 = (p1 & k) == 0, low1 = (p1 & s) == 0;
+                x0 = (low0 == asc0) ? min(x0, y0) : max(x0, y0);
+                x1 = (low1 == asc1) ? min(x1, y1) : max(x1, y1);
+            }
+        }
+    }
+}
+
+// Descending bitonic sort of 64 keys held two per lane (position 2*lane + j).
+__device__ __forceinline__ void warp_sort64_desc(uint64_t& x0, uint64_t& x1, int lane) {
+#pragma unroll
+    for (int k = 2; k <= 64; k <<= 1) {
+#pragma unroll
+        for (int s = k >> 1; s > 0; s >>= 1) {
+            if (s == 1) {
+                const bool dsc = ((2 * lane) & k) == 0;
+                const uint64_t lo = x0 < x1 ? x0 : x1, hi = x0 < x1 ? x1 : x0;
+                x0 = dsc ? hi : lo;
+                x1 = dsc ? lo : hi;
+            } else {
+                const int lm = s >> 1;
+                const uint64_t y0 = __shfl_xor_sync(0xffffffffu, x0, lm);
+                const uint64_t y1 = __shfl_xor_sync(0xffffffffu, x1, lm);
+                const int p0 = 2 * lane, p1 = 2 * lane + 1;
+                const bool d0 = (p0 & k) == 0, low0 = (p0 & s) == 0;
+                const bool d1 = (p1 & k) == 0, low1 = (p1 & s) == 0;
+                x0 = (low0 == d0) ? (x0 > y0 ? x0 : y0) : (x0 < y0 ? x0 : y0);
+                x1 = (low1 == d1) ? (x1 > y1 ? x1 : y1) : (x1 < y1 ? x1 : y1);
+            }
+        }
+    }
+}
+
+template <int D>
+struct DecSmem {
+    float K[kBlk][D + 4];   // keys of the slot's block (rows padded: aligned and conflict-free)
+    float V[kBlk][D];
+    float Q[kMaxG][D];
+    float P[kMaxG][kBlk];   // logits, then probabilities
+    float m[kMaxG], l[kMaxG];
+    float qbar[D];
+    float sc[kSpan];
+    int sel[kMaxSlots];
+    int sel_top[kCap];
+    uint64_t cand[kThreads];
+    SelSmem ss;
+    int ok, overflow;
+    float cm[8][32], cl[8][32], co[8][32];  // phase D per-warp partials
+};
+
+template <typename T>
+__device__ __forceinline__ void load8(const T* p, float (&f)[8]);
+template <>
+__device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16* p, float (&f)[8]) {
+    const uint4 u = *reinterpret_cast<const uint4*>(p);
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 t = __bfloat1622float2(h[i]);
+        f[2 * i] = t.x;
+        f[2 * i + 1] = t.y;
+    }
+}
+template <>
+__device__ __forceinline__ void load8<float>(const float* p, float (&f)[8]) {
+    const float4 a = reinterpret_cast<const float4*>(p)[0], b = reinterpret_cast<const float4*>(p)[1];
+    f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+    f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+}
+
+// 16-byte raw loads, converted later: issuing every load of a phase before the first conversion
+// keeps them all in flight (converting each load as it arrives would serialize the round trips).
+__device__ __forceinline__ uint4 ld16(const void* p) { return *reinterpret_cast<const uint4*>(p); }
+template <typename T>
+__device__ __forceinline__ void cvt16(const uint4& u, float* f);  // sizeof(T) * ... elements
+template <>
+__device__ __forceinline__ void cvt16<__nv_bfloat16>(const uint4& u, float* f) {
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 t = __bfloat1622float2(h[i]);
+        f[2 * i] = t.x;
+        f[2 * i + 1] = t.y;
+    }
+}
+template <>
+__device__ __forceinline__ void cvt16<float>(const uint4& u, float* f) {
+    f[0] = __uint_as_float(u.x);
+    f[1] = __uint_as_float(u.y);
+    f[2] = __uint_as_float(u.z);
+    f[3] = __uint_as_float(u.w);
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kThreads)
+sparse_decode_fused_kernel(const T* __restrict__ q, const T* __restrict__ kc,
+                           const T* __restrict__ vc, const T* __restrict__ kbar,
+                           const int32_t* __restrict__ idx_in, int32_t* __restrict__ idx_out,
+                           T* __restrict__ o, int H, int Hkv, int pos, int Tmax, int nb_cap,
+                           int topk, int n_init, int n_local, int slots, float scale, int cpg,
+                           int nspan, unsigned* bar, uint64_t* part, float* rec, DevCtx ctx) {
+    extern __shared__ __align__(16) unsigned char dsm_raw[];
+    DecSmem<D>& sm = *reinterpret_cast<DecSmem<D>*>(dsm_raw);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int G = H / Hkv;
+    const int bg = blockIdx.x / cpg, j = blockIdx.x % cpg;
+    const int64_t b = bg / Hkv;
+    const int g = bg % Hkv;
+    const int c = pos / kBlk;
+    const int lo = n_init, hi = c - n_local;
+    const int ncand = hi - lo + 1;
+    const int K = topk;
+    const bool do_sel = idx_in == nullptr && ncand > K;
+    const T* qg = q + (b * H + (int64_t)g * G) * D;  // the group's G query rows
+    pdl_trigger();
+    pdl_wait();
+
+    // ---------------------------------------------------------------- A: span scores + top-k
+    // Rows of k_bar are read coalesced: kLPR lanes per row, 16 elements per lane.  Each span
+    // publishes its top-k keys sorted, largest first.
+    constexpr int kLPR = D / 16, kRPS = 32 / kLPR, kSteps = (kSpan / 8) / kRPS;
+    if (do_sel && K > 0) {
+        if (tid < D) {  // all G loads in flight at once (a runtime-G loop would issue them one by one)
+            float qv[kMaxG];
+#pragma unroll
+            for (int hh = 0; hh < kMaxG; ++hh) qv[hh] = hh < G ? to_f(qg[hh * D + tid]) : 0.f;
+            float s = 0.f;
+#pragma unroll
+            for (int hh = 0; hh < kMaxG; ++hh) s += qv[hh];
+            sm.qbar[tid] = s;
+        }
+        __syncthreads();
+        const T* kb = kbar + (int64_t)bg * nb_cap * D;
+        const int part16 = (lane % kLPR) * 16;
+        for (int span = j; span < nspan; span += cpg) {
+            const int base = lo + span * kSpan;
+            constexpr int kU = 16 * sizeof(T) / 16;   // 16-byte pieces per lane and row
+            constexpr int kEl = 16 / sizeof(T);        // elements per piece
+            uint4 raw[kSteps][kU];
+#pragma unroll
+            for (int st = 0; st < kSteps; ++st) {
+                const int blk = base + warp * (kSpan / 8) + st * kRPS + lane / kLPR;
+                const T* row = kb + (int64_t)blk * D + part16;
+#pragma unroll
+                for (int u = 0; u < kU; ++u)
+                    raw[st][u] = blk <= hi ? ld16(row + u * kEl) : make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
+            for (int st = 0; st < kSteps; ++st) {
+                float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+                for (int u = 0; u < kU; ++u) {
+                    float f[kEl];
+                    cvt16<T>(raw[st][u], f);
+#pragma unroll
+                    for (int i = 0; i < kEl; i += 2) {
+                        a0 = fmaf(sm.qbar[part16 + u * kEl + i], f[i], a0);
+                        a1 = fmaf(sm.qbar[part16 + u * kEl + i + 1], f[i + 1], a1);
+                    }
+                }
+                float d = a0 + a1;
+#pragma unroll
+                for (int off = 1; off < kLPR; off <<= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
+                if (lane % kLPR == 0) sm.sc[warp * (kSpan / 8) + st * kRPS + lane / kLPR] = d;
+            }
+            __syncthreads();
+            const int blk = base + tid;
+            uint64_t key[1] = {blk <= hi ? sel_key_u(sm.sc[tid], blk) : 0ull};
+            uint64_t prefix, mask;
+            block_kth<1>(key, K, sm.ss, prefix, mask);
+            if (tid == 0) sm.ss.n = 0;
+            if (tid < kCap) sm.cand[tid] = 0ull;
+            __syncthreads();
+            if (key[0] && (key[0] & mask) >= prefix) sm.cand[atomicAdd(&sm.ss.n, 1)] = key[0];
+            __syncthreads();
+            if (warp == 0) {  // the span's list, largest first (zeros, "no key", last)
+                uint64_t x0 = sm.cand[2 * lane], x1 = sm.cand[2 * lane + 1];
+                warp_sort64_desc(x0, x1, lane);
+                uint64_t* dst = part + ((int64_t)bg * nspan + span) * kCap;
+                dst[2 * lane] = x0;
+                dst[2 * lane + 1] = x1;
+            }
+            __syncthreads();
+        }
+    }
+    if (!grid_barrier(bar, gridDim.x, ctx, &sm.ok)) return;
+
+    // ---------------------------------------------------------------- B: the group's slot list
+    if (idx_in) {
+        for (int s = tid; s < slots; s += kThreads) {
+            int blk = idx_in[(int64_t)bg * slots + s];
+            if (blk > c) {
+                flag(ctx, kStatusBounds);
+                blk = -1;
+            }
+            sm.sel[s] = blk;
+        }
+    } else if (!do_sel) {
+        for (int s = tid; s < slots; s += kThreads) sm.sel[s] = s <= c ? s : -1;
+    } else {
+        if (K > 0) {
+            // The group's top-k from the spans' first kPre keys: if no span has all kPre of its
+            // loaded keys among the winners, no span can hide a winner further down its list, so
+            // the k-th largest loaded key is the group's k-th key.  Otherwise (rare) merge the
+            // spans' whole lists.
+            constexpr int kPre = 8, kPreE = kMergeE * kPre / kCap;  // prefix keys per thread (spans <= 128)
+            const unsigned long long* src =
+                reinterpret_cast<const unsigned long long*>(part) + (int64_t)bg * nspan * kCap;
+            uint64_t pk[kPreE];
+#pragma unroll
+            for (int e = 0; e < kPreE; ++e) {
+                const int i = e * kThreads + tid, span = i / kPre;
+                pk[e] = span < nspan ? __ldcg(src + span * kCap + i % kPre) : 0ull;
+            }
+            uint64_t prefix, mask;
+            block_kth<kPreE>(pk, K, sm.ss, prefix, mask);
+            if (tid == 0) {
+                sm.ss.n = 0;
+                sm.overflow = 0;
+            }
+            __syncthreads();
+#pragma unroll
+            for (int e = 0; e < kPreE; ++e) {
+                const int i = e * kThreads + tid;
+                if (pk[e] && (pk[e] & mask) >= prefix && i % kPre == kPre - 1) sm.overflow = 1;
+            }
+            __syncthreads();
+            if (!sm.overflow) {
+#pragma unroll
+                for (int e = 0; e < kPreE; ++e)
+                    if (pk[e] && (pk[e] & mask) >= prefix) sm.sel_top[atomicAdd(&sm.ss.n, 1)] = key_block(pk[e]);
+            } else {
+                uint64_t key[kMergeE];
+                const int nk = nspan * kCap;
+#pragma unroll
+                for (int e = 0; e < kMergeE; ++e) {
+                    const int i = e * kThreads + tid;
+                    key[e] = i < nk ? __ldcg(src + i) : 0ull;
+                }
+                block_kth<kMergeE>(key, K, sm.ss, prefix, mask);
+                if (tid == 0) sm.ss.n = 0;
+                __syncthreads();
+#pragma unroll
+                for (int e = 0; e < kMergeE; ++e)
+                    if (key[e] && (key[e] & mask) >= prefix) sm.sel_top[atomicAdd(&sm.ss.n, 1)] = key_block(key[e]);
+            }
+            __syncthreads();
+        }
+        if (warp == 0) {
+            int x0 = 2 * lane < K ? sm.sel_top[2 * lane] : 0x7fffffff;
+            int x1 = 2 * lane + 1 < K ? sm.sel_top[2 * lane + 1] : 0x7fffffff;
+            warp_sort64(x0, x1, lane);
+            for (int s = lane; s < n_init; s += 32) sm.sel[s] = s;
+            if (2 * lane < K) sm.sel[n_init + 2 * lane] = x0;
+            if (2 * lane + 1 < K) sm.sel[n_init + 2 * lane + 1] = x1;
+            for (int t = lane; t < n_local; t += 32) sm.sel[n_init + K + t] = c - n_local + 1 + t;
+            for (int s = n_init + K + n_local + lane; s < slots; s += 32) sm.sel[s] = -1;
+        }
+    }
+    __syncthreads();
+    if (idx_out && j == 0)
+        for (int s = tid; s < slots; s += kThreads) idx_out[(int64_t)bg * slots + s] = sm.sel[s];
+
+    // ---------------------------------------------------------------- C: per-slot partials
+    {
+        constexpr int kQIt = kMaxG * D / kThreads;
+        float qv[kQIt];
+#pragma unroll
+        for (int u = 0; u < kQIt; ++u) {
+            const int e = u * kThreads + tid;
+            qv[u] = e < G * D ? to_f(qg[e]) : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < kQIt; ++u) {
+            const int e = u * kThreads + tid;
+            if (e < G * D) sm.Q[e / D][e % D] = qv[u];
+        }
+    }
+    const T* kcg = kc + (int64_t)bg * Tmax * D;
+    const T* vcg = vc + (int64_t)bg * Tmax * D;
+    constexpr int kStage = kBlk * (D / 8) / kThreads;  // 8-element pieces of K (and V) per thread
+    for (int s = j; s < slots; s += cpg) {
+        const int blk = sm.sel[s];
+        float* r = rec + ((int64_t)bg * slots + s) * G * (D + 2);
+        if (blk < 0) {
+            for (int hh = tid; hh < G; hh += kThreads) {
+                r[hh * (D + 2)] = -INFINITY;
+                r[hh * (D + 2) + 1] = 0.f;
+            }
+            continue;
+        }
+        const int lim = min(kBlk - 1, pos - blk * kBlk);  // last visible key of the block
+        constexpr int kU = 8 * sizeof(T) / 16;  // 16-byte pieces per 8 elements
+        constexpr int kEl = 16 / sizeof(T);
+        uint4 rk[kStage][kU], rv[kStage][kU];
+#pragma unroll
+        for (int u = 0; u < kStage; ++u) {  // every load issued before the first use
+            const int e = u * kThreads + tid;
+            const int row = e / (D / 8), c8 = (e % (D / 8)) * 8;
+            const bool ok = row <= lim;
+            const T* pk = kcg + ((int64_t)blk * kBlk + row) * D + c8;
+            const T* pv = vcg + ((int64_t)blk * kBlk + row) * D + c8;
+#pragma unroll
+            for (int w = 0; w < kU; ++w) {
+                rk[u][w] = ok ? ld16(pk + w * kEl) : make_uint4(0u, 0u, 0u, 0u);
+                rv[u][w] = ok ? ld16(pv + w * kEl) : make_uint4(0u, 0u, 0u, 0u);
+            }
+        }
+        __syncthreads();  // the previous slot's readers are done with K, V, P
+#pragma unroll
+        for (int u = 0; u < kStage; ++u) {
+            const int e = u * kThreads + tid;
+            const int row = e / (D / 8), c8 = (e % (D / 8)) * 8;
+            float fk[8], fv[8];
+#pragma unroll
+            for (int w = 0; w < kU; ++w) {
+                cvt16<T>(rk[u][w], fk + w * kEl);
+                cvt16<T>(rv[u][w], fv + w * kEl);
+            }
+            *reinterpret_cast<float4*>(&sm.K[row][c8]) = make_float4(fk[0], fk[1], fk[2], fk[3]);
+            *reinterpret_cast<float4*>(&sm.K[row][c8 + 4]) = make_float4(fk[4], fk[5], fk[6], fk[7]);
+            *reinterpret_cast<float4*>(&sm.V[row][c8]) = make_float4(fv[0], fv[1], fv[2], fv[3]);
+            *reinterpret_cast<float4*>(&sm.V[row][c8 + 4]) = make_float4(fv[4], fv[5], fv[6], fv[7]);
+        }
+        __syncthreads();
+        // logits: thread = one key x four heads (K row read once for four heads)
+        {
+            const int key = tid % kBlk, h0 = (tid / kBlk) * 4;
+            if (h0 < G) {
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+                for (int dd = 0; dd < D; dd += 4) {
+                    const float4 k4 = *reinterpret_cast<const float4*>(&sm.K[key][dd]);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        if (h0 + i < G) {
+                            const float4 q4 = *reinterpret_cast<const float4*>(&sm.Q[h0 + i][dd]);
+                            acc[i] = fmaf(q4.x, k4.x, fmaf(q4.y, k4.y, fmaf(q4.z, k4.z, fmaf(q4.w, k4.w, acc[i]))));
+                        }
+                    }
+                }
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    if (h0 + i < G) sm.P[h0 + i][key] = key <= lim ? acc[i] * scale : -INFINITY;
+            }
+        }
+        __syncthreads();
+        for (int hh = warp; hh < G; hh += kThreads / 32) {
+            const float s0 = sm.P[hh][lane], s1 = sm.P[hh][lane + 32];
+            float m = fmaxf(s0, s1);
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+            const float p0 = expf(s0 - m), p1 = expf(s1 - m);  // lim >= 0, so m is finite
+            float l = p0 + p1;
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
+            sm.P[hh][lane] = p0;
+            sm.P[hh][lane + 32] = p1;
+            if (lane == 0) {
+                sm.m[hh] = m;
+                sm.l[hh] = l;
+            }
+        }
+        __syncthreads();
+        // p v: thread = four columns x the heads hp, hp + ngrp, ... (V read once for them)
+        {
+            constexpr int kQuads = D / 4, kGroups = kThreads / kQuads;
+            const int dq = tid % kQuads, hp = tid / kQuads;
+            for (int h0 = hp; h0 < G; h0 += 2 * kGroups) {
+                const int h1 = h0 + kGroups;
+                float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0;
+#pragma unroll 8
+                for (int key = 0; key < kBlk; ++key) {
+                    const float4 v4 = *reinterpret_cast<const float4*>(&sm.V[key][4 * dq]);
+                    const float p0 = sm.P[h0][key];
+                    a0.x = fmaf(p0, v4.x, a0.x); a0.y = fmaf(p0, v4.y, a0.y);
+                    a0.z = fmaf(p0, v4.z, a0.z); a0.w = fmaf(p0, v4.w, a0.w);
+                    if (h1 < G) {
+                        const float p1 = sm.P[h1][key];
+                        a1.x = fmaf(p1, v4.x, a1.x); a1.y = fmaf(p1, v4.y, a1.y);
+                        a1.z = fmaf(p1, v4.z, a1.z); a1.w = fmaf(p1, v4.w, a1.w);
+                    }
+                }
+                float* r0 = r + h0 * (D + 2);
+                r0[2 + 4 * dq] = a0.x; r0[3 + 4 * dq] = a0.y; r0[4 + 4 * dq] = a0.z; r0[5 + 4 * dq] = a0.w;
+                if (dq == 0) { r0[0] = sm.m[h0]; r0[1] = sm.l[h0]; }
+                if (h1 < G) {
+                    float* r1 = r + h1 * (D + 2);
+                    r1[2 + 4 * dq] = a1.x; r1[3 + 4 * dq] = a1.y; r1[4 + 4 * dq] = a1.z; r1[5 + 4 * dq] = a1.w;
+                    if (dq == 0) { r1[0] = sm.m[h1]; r1[1] = sm.l[h1]; }
+                }
+            }
+        }
+    }
+    if (!grid_barrier(bar, gridDim.x, ctx, &sm.ok)) return;
+
+    // ---------------------------------------------------------------- D: combine
+    // Warp w folds slots w, w + 8, ...; all of its records are loaded before the first use.
+    constexpr int kPerWarp = (kMaxSlots + 7) / 8;
+    for (int item = j; item < G * (D / 32); item += cpg) {
+        const int hh = item / (D / 32), d0 = (item % (D / 32)) * 32;
+        float ms[kPerWarp], ls[kPerWarp], os[kPerWarp];
+#pragma unroll
+        for (int i = 0; i < kPerWarp; ++i) {
+            const int s = warp + 8 * i;
+            if (s < slots) {
+                const float* r = rec + (((int64_t)bg * slots + s) * G + hh) * (D + 2);
+                ms[i] = __ldcg(r);
+                ls[i] = __ldcg(r + 1);
+                os[i] = __ldcg(r + 2 + d0 + lane);
+            } else {
+                ms[i] = -INFINITY;
+                ls[i] = os[i] = 0.f;
+            }
+        }
+        float M = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < kPerWarp; ++i) M = fmaxf(M, ms[i]);
+        float L = 0.f, acc = 0.f;
+        if (M != -INFINITY) {
+#pragma unroll
+            for (int i = 0; i < kPerWarp; ++i) {
+                if (ms[i] == -INFINITY) continue;
+                const float w8 = expf(ms[i] - M);
+                L = fmaf(ls[i], w8, L);
+                acc = fmaf(os[i], w8, acc);
+            }
+        }
+        sm.cm[warp][lane] = M;
+        sm.cl[warp][lane] = L;
+        sm.co[warp][lane] = acc;
+        __syncthreads();
+        if (warp == 0) {
+            float Mt = -INFINITY;
+#pragma unroll
+            for (int w = 0; w < kThreads / 32; ++w) Mt = fmaxf(Mt, sm.cm[w][lane]);
+            float Lt = 0.f, At = 0.f;
+            if (Mt != -INFINITY) {
+#pragma unroll
+                for (int w = 0; w < kThreads / 32; ++w) {
+                    if (sm.cm[w][lane] == -INFINITY) continue;
+                    const float a = expf(sm.cm[w][lane] - Mt);
+                    Lt += a * sm.cl[w][lane];
+                    At += a * sm.co[w][lane];
+                }
+            }
+            o[(b * H + (int64_t)g * G + hh) * D + d0 + lane] = from_f<T>(Lt > 0.f ? At / Lt : 0.f);
+        }
+        __syncthreads();
+    }
+}
+
+// Workspace of the one-launch path: [0, 256) barrier word, then per (batch, group, span) the span's
+// top-k keys, then the per-slot partial records.
+struct FusedLayout {
+    size_t part, rec, total;
+};
+FusedLayout fused_layout(int B, int H, int Hkv, int nspan, int slots, int d) {
+    auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    FusedLayout L;
+    L.part = 256;
+    L.rec = L.part + up((size_t)B * Hkv * nspan * kCap * sizeof(uint64_t));
+    L.total = L.rec + (size_t)B * Hkv * slots * (H / Hkv) * (d + 2) * sizeof(float);
+    return L;
+}
+
+template <typename T, int D>
+cudaError_t fused(const void* q, const void* kc, const void* vc, const void* kbar,
+                  const int32_t* idx_in, int32_t* idx_out, void* o, int B, int H, int Hkv, int pos,
+                  int Tmax, int nb_cap, int topk, int n_init, int n_local, float scale, void* ws,
+                  size_t ws_bytes, cudaStream_t st, DevCtx ctx) {
+    const int slots = n_init + n_local + topk;
+    const int G = H / Hkv;
+    const int c = pos / kBlk;
+    const int ncand = c - n_local - n_init + 1;
+    const int nspan = ncand > topk ? (ncand + kSpan - 1) / kSpan : 0;
+    if (topk > kCap || slots > kMaxSlots || G > kMaxG || nspan * kCap > kMergeE * kThreads)
+        return cudaErrorNotSupported;
+    auto kern = sparse_decode_fused_kernel<T, D>;
+    const int smem = (int)sizeof(DecSmem<D>);
+    static std::mutex mu;
+    static int occ_dev = -1, occ = 0, nsm = 0;
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        int dev = 0;
+        cudaGetDevice(&dev);
+        if (occ_dev != dev) {
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+            if (e != cudaSuccess) return e;
+            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kThreads, smem);
+            if (e != cudaSuccess) return e;
+            cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+            occ_dev = dev;
+        }
+    }
+    const int groups = B * Hkv;
+    const int cap = occ * nsm / groups;
+    const int want = max(max(nspan, slots), G * (D / 32));
+    const int cpg = min(cap, want);
+    if (cpg < 1) return cudaErrorNotSupported;
+    const FusedLayout lay = fused_layout(B, H, Hkv, nspan, slots, D);
+    if (lay.total > ws_bytes) return cudaErrorNotSupported;
+    unsigned char* w = static_cast<unsigned char*>(ws);
+    uint64_t* part = reinterpret_cast<uint64_t*>(w + lay.part);
+    float* rec = reinterpret_cast<float*>(w + lay.rec);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(groups * cpg));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    auto go = [&](int nattr) {
+        cfg.numAttrs = nattr;
+        return cudaLaunchKernelEx(&cfg, kern, static_cast<const T*>(q), static_cast<const T*>(kc),
+                                  static_cast<const T*>(vc), static_cast<const T*>(kbar), idx_in,
+                                  idx_out, static_cast<T*>(o), H, Hkv, pos, Tmax, nb_cap, topk,
+                                  n_init, n_local, slots, scale, cpg, nspan,
+                                  reinterpret_cast<unsigned*>(w), part, rec, ctx);
+    };
+    // Programmatic dependent launch together with the cooperative attribute is tried once, outside
+    // any stream capture; if the launch is refused, later launches use the cooperative attribute
+    // alone.
+    static std::atomic<int> pdl_ok{-1};
+    if (pdl_ok.load() == 1) return go(2);
+    if (pdl_ok.load() == 0) return go(1);
+    cudaStreamCaptureStatus capture = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(st, &capture) != cudaSuccess || capture != cudaStreamCaptureStatusNone)
+        return go(1);
+    cudaError_t e = go(2);
+    if (e == cudaSuccess) {
+        pdl_ok.store(1);
+        return e;
+    }
+    (void)cudaGetLastError();  // clear the refused launch's error
+    pdl_ok.store(0);
+    return go(1);
+}
+
+}  // namespace
+
+size_t sparse_decode_fused_workspace(int B, int H, int Hkv, int pos, int topk, int n_init,
+                                     int n_local, int d) {
+    if (B <= 0 || H <= 0 || Hkv <= 0 || pos < 0) return 0;
+    const int slots = n_init + n_local + topk;
+    const int ncand = pos / kBlk - n_local - n_init + 1;
+    const int nspan = ncand > topk ? (ncand + kSpan - 1) / kSpan : 0;
+    return fused_layout(B, H, Hkv, nspan, slots, d).total;
+}
+
+cudaError_t launch_sparse_decode_fused(DType dt, const void* q, const void* kc, const void* vc,
+                                       const void* kbar, const int32_t* idx_in, int32_t* idx_out,
+                                       void* o, int B, int H, int Hkv, int pos, int Tmax,
+                                       int nb_cap, int d, int topk, int n_init, int n_local,
+                                       float scale, void* ws, size_t ws_bytes, cudaStream_t st,
+                                       DevCtx ctx) {
+    if (dt == DType::F32)
+        return d == 64 ? fused<float, 64>(q, kc, vc, kbar, idx_in, idx_out, o, B, H, Hkv, pos, Tmax, nb_cap, topk, n_init, n_local, scale, ws, ws_bytes, st, ctx)
+                       : fused<float, 128>(q, kc, vc, kbar, idx_in, idx_out, o, B, H, Hkv, pos, Tmax, nb_cap, topk, n_init, n_local, scale, ws, ws_bytes, st, ctx);
+    return d == 64 ? fused<__nv_bfloat16, 64>(q, kc, vc, kbar, idx_in, idx_out, o, B, H, Hkv, pos, Tmax, nb_cap, topk, n_init, n_local, scale, ws, ws_bytes, st, ctx)
+                   : fused<__nv_bfloat16, 128>(q, kc, vc, kbar, idx_in, idx_out, o, B, H, Hkv, pos, Tmax, nb_cap, topk, n_init, n_local, scale, ws, ws_bytes, st, ctx);
+}
+
+}  // namespace sala

@@ -193,8 +193,8 @@ def sparse_decode(q, kcache, vcache, kbar, pos, topk, n_init=1, n_local=2, idx_i
         o = torch.empty_like(q)
     _need(o, "o", q.shape, q.dtype)
     need = sparse_decode_workspace_bytes(B, H, Hkv, pos, topk, n_init, n_local, d, block)
-    if workspace is None:
-        workspace = torch.empty(max(need, 16), device=q.device, dtype=torch.uint8)
+    if workspace is None:  # zero-filled: its first words are counters that must start at zero
+        workspace = torch.zeros(max(need, 256), device=q.device, dtype=torch.uint8)
     _check(_lib.sala_sparse_decode(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(kbar), _ptr(idx_in),
                                    _ptr(idx_out), _ptr(o), B, H, Hkv, pos, Tmax, kbar.shape[2], d,
                                    block, topk, n_init, n_local, float(scale), _ptr(workspace),

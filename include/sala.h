@@ -156,7 +156,15 @@ sala_status sala_sparse_prefill(const void* q, const void* k, const void* v, con
  *                 sala_block_topk, for q_pos0 = pos); otherwise attend to these blocks.
  * idx_out       : [B, Hkv, slots] int32 or NULL; receives the selection that was used.
  * workspace     : at least sala_sparse_decode_workspace(...) bytes of device scratch, not
- *                 shared with a concurrent call.
+ *                 shared with a concurrent call.  Its first 256 bytes hold the counters of a
+ *                 grid-wide barrier and must be zero before the first call (e.g. allocate it
+ *                 zero-filled once); every call that completes leaves them zero, so the same
+ *                 workspace can serve call after call and CUDA-graph replays.  After a call that
+ *                 reported an error (SALA_ERR_TIMEOUT from sala_check_status), zero them again.
+ *                 The rest needs no initial value.
+ * Implementation: when k <= 64, slots <= 80, H/Hkv <= 16 and the grid fits on the GPU at once,
+ * the whole step (scoring, top-k, attention over the selected blocks, combine) is one cooperative
+ * launch with two grid-wide barriers; otherwise it runs as four launches.
  */
 sala_status sala_sparse_decode(const void* q, const void* kcache, const void* vcache,
                                const void* kbar, const int32_t* idx_in, int32_t* idx_out, void* o,
@@ -183,8 +191,11 @@ size_t sala_sparse_decode_workspace(int B, int H, int Hkv, int pos, int block, i
  *   - The first call on each GPU looks up the area's device address (cudaGetSymbolAddress, with
  *     that GPU current) and caches it; make that first call before any stream capture.
  *   - All calls on a GPU share the one area: calls that can run concurrently on the same GPU
- *     race on it and must not be made.  The area keeps the previous call's contents; nothing in
- *     it needs to start at zero.
+ *     race on it and must not be made.  The area keeps the previous call's contents.  Its first
+ *     256 bytes are the barrier counters described under sala_sparse_decode: zero when the
+ *     library loads and left zero by every call that completes (a call that reported
+ *     SALA_ERR_TIMEOUT may leave them nonzero, after which later calls also time out instead of
+ *     completing); nothing else in it needs a starting value.
  * Other arguments, validation and errors are those of sala_sparse_decode. */
 sala_status sala_sparse_decode_noalloc(const void* q, const void* kcache, const void* vcache,
                                        const void* kbar, const int32_t* idx_in, int32_t* idx_out,

@@ -111,9 +111,9 @@ def test_out_of_range_index_is_flagged(sala):
 
 
 # ---------------------------------------------------------------------------------------------
-def _decode_case(sala, T, topk, n_init, n_local, dtype, layer_id, given_idx=False):
+def _decode_case(sala, T, topk, n_init, n_local, dtype, layer_id, given_idx=False, H=32, Hkv=2,
+                 d=128, workspace=None):
     from hybrid_sparse_linear_b200 import synth
-    H, Hkv, d = 32, 2, 128
     layer = synth.sparse_layer(1, H, Hkv, T, d, dtype, device="cuda", layer=layer_id,
                                shift_frac=0.05, q_rows=1)
     pos = T - 1
@@ -130,13 +130,14 @@ def _decode_case(sala, T, topk, n_init, n_local, dtype, layer_id, given_idx=Fals
     idx_ref, kth = oracle.block_select(q64, kbar_ref, 64, topk, n_init, n_local, q_pos0=pos)
     idx_in = torch.from_numpy(idx_ref[:, :, 0]).cuda() if given_idx else None
     o = sala.sparse_decode(qd, kc, vc, kbar, pos, topk, n_init, n_local, idx_in=idx_in,
-                           idx_out=idx_out)
+                           idx_out=idx_out, workspace=workspace)
     sala.check_status()
     got = idx_out.cpu().numpy()[:, :, None, :]
     check_selection(got, idx_ref, q64, kbar_ref, kth, topk, n_init, n_local, q_pos0=pos,
                     row_ids=np.array([0]))
     o_ref = oracle.sparse_attention(q64, _f64(layer.k), _f64(layer.v), got, 64, q_pos0=pos)
     assert_close(_f64(o), o_ref[:, :, 0], kind, "decode o")
+    return o, idx_out
 
 
 @pytest.mark.parametrize("T", [64 * 300 + 5, 64 * 300, 64 * 3, 1, 70])
@@ -151,3 +152,37 @@ def test_sparse_decode_given_idx_fp32(sala):
 def test_sparse_decode_1m_context(sala):
     """One sparse layer at a 2^20-token cache: 16384 compressed blocks, top-64 + init + 2 local."""
     _decode_case(sala, 1 << 20, 64, 1, 2, torch.bfloat16, 8)
+
+
+def test_sparse_decode_multi_launch_path(sala):
+    """k = 100 (103 slots) is past the one-launch kernel's limits: the four-launch path runs.  With
+    at most k candidates every block up to the query's is selected."""
+    _decode_case(sala, 64 * 90 + 3, 100, 1, 2, torch.bfloat16, 9)
+
+
+def test_sparse_decode_fp32_d64_one_head_per_group(sala):
+    _decode_case(sala, 64 * 200 + 17, 8, 1, 1, torch.float32, 10, H=2, Hkv=2, d=64)
+
+
+def test_sparse_decode_top0_forced_blocks_only(sala):
+    _decode_case(sala, 64 * 40 + 9, 0, 1, 2, torch.bfloat16, 12)
+
+
+def test_sparse_decode_workspace_reused_across_calls_and_shapes(sala):
+    """One zero-filled workspace serves call after call (the grid barrier's counters come back to
+    zero), also when the context length changes between calls."""
+    T_big, T_small = 64 * 2000 + 5, 64 * 300 + 5
+    need = max(sala.sparse_decode_workspace_bytes(1, 32, 2, T - 1, 64, 1, 2, 128)
+               for T in (T_big, T_small))
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    first = None
+    for T in (T_big, T_small, T_big, T_big):
+        o, idx = _decode_case(sala, T, 64, 1, 2, torch.bfloat16, 13, workspace=ws)
+        torch.cuda.synchronize()
+        word = int(ws[:4].view(torch.int32)[0].item())
+        assert word & 0xFFFF == 0, f"barrier count not restored: {word:#x}"  # low half: arrivals
+        if T == T_big:
+            if first is None:
+                first = (o.clone(), idx.clone())
+            else:
+                assert torch.equal(o, first[0]) and torch.equal(idx, first[1])
