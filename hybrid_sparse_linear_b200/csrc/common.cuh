@@ -21,14 +21,6 @@ struct DevCtx {
 
 __device__ __forceinline__ void flag(const DevCtx& c, unsigned bits) { atomicOr(c.status, bits); }
 
-// Programmatic dependent launch: a kernel launched with the programmatic-serialization attribute
-// may start while the previous kernel on its stream is still running.  pdl_trigger lets the next
-// such kernel start; pdl_wait blocks until the previous kernel has completed and its memory
-// writes are visible (a no-op for a kernel launched without the attribute).  Decode kernels call
-// both first thing, so only their launch latency overlaps the previous kernel, never their work.
-__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
-__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-
 __device__ __forceinline__ uint64_t globaltimer_ns() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

@@ -145,8 +145,6 @@ linear_decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* 
     constexpr int kCols = 16;
     constexpr int kWarps = 2 * D / 32;
     __shared__ float red[kWarps][kCols];
-    pdl_trigger();
-    pdl_wait();
     const int tid = threadIdx.x;
     const int a = tid >> 1, half = tid & 1;
     const int64_t bh = blockIdx.y;
@@ -188,18 +186,11 @@ linear_decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* 
 template <typename T, int D>
 cudaError_t decode_launch(const void* q, const void* k, const void* v, const float* decay,
                           float* state, void* o, int B, int H, cudaStream_t st) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(D / 16, (unsigned)(B * H));
-    cfg.blockDim = dim3(2 * D);
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, linear_decode_kernel<T, D>, static_cast<const T*>(q),
-                              static_cast<const T*>(k), static_cast<const T*>(v), decay, state,
-                              static_cast<T*>(o), H);
+    dim3 grid(D / 16, (unsigned)(B * H));
+    linear_decode_kernel<T, D><<<grid, 2 * D, 0, st>>>(
+        static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), decay,
+        state, static_cast<T*>(o), H);
+    return cudaGetLastError();
 }
 
 }  // namespace

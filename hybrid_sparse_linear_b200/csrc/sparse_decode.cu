@@ -6,14 +6,17 @@
 // 2^20 tokens and 2 KV heads), the attention reads the ~67 selected K/V blocks (4 MiB).  Spread
 // over the GPU, each phase is one round of loads.  The kernel runs all of them in one cooperative
 // launch (all CTAs resident, so a grid-wide barrier is safe), with `cpg` CTAs per (batch, group):
-//   A  CTA j scores candidate span j (256 blocks): one thread per block, 256 bytes of k_bar each,
-//      then keeps the span's top-k keys (block-wide radix select on 64-bit keys).
+//   A  CTA j scores candidate span j (256 blocks, 256 bytes of k_bar each, read coalesced) and
+//      publishes the span's top-k keys sorted largest first (a bitonic sort of the 256 keys).
 //   -- grid barrier --
-//   B  every CTA of the group merges all spans' lists into the group's top-k (the same
-//      deterministic result in each CTA, so no second exchange is needed) and forms the
-//      ascending slot list: init blocks, top-k, local blocks, -1 padding.
+//   B  every CTA of the group finds the group's top-k from the spans' first 8 keys (a radix
+//      select on 64-bit keys; exact unless some span's 8th key is itself a winner, in which case
+//      the spans' whole lists are merged), the same deterministic result in each CTA, so no
+//      second exchange is needed, and forms the ascending slot list: init blocks, top-k, local
+//      blocks, -1 padding.
 //   C  CTA j attends slot j (and j + cpg, ...): K and V of the block staged in shared memory,
-//      G heads' logits, a per-head softmax partial (max, sum, sum of p v) written to workspace.
+//      G heads' logits and p v (bf16: warp-level tensor-core tiles; fp32: CUDA cores), a per-head
+//      softmax partial (max, sum, sum of p v) written to workspace.
 //   -- grid barrier --
 //   D  CTA j combines the partials of one (head, 32-column) piece of the output.
 // Selection keys pack (orderable score << 32 | ~block): one unsigned compare orders by score,
@@ -23,8 +26,8 @@
 // zero before the first call; the last CTA to arrive puts it back to zero, so every call that
 // completes leaves it as it found it.  Waits are bounded (the device status word records a
 // timeout).
-#include <atomic>
 #include <mutex>
+#include <type_traits>
 
 #include "kernels.h"
 
@@ -176,36 +179,21 @@ __device__ __forceinline__ void warp_sort64(int& x0, int& x1, int lane) {
     }
 }
 
-// Descending bitonic sort of 64 keys held two per lane (position 2*lane + j).
-__device__ __forceinline__ void warp_sort64_desc(uint64_t& x0, uint64_t& x1, int lane) {
-#pragma unroll
-    for (int k = 2; k <= 64; k <<= 1) {
-#pragma unroll
-        for (int s = k >> 1; s > 0; s >>= 1) {
-            if (s == 1) {
-                const bool dsc = ((2 * lane) & k) == 0;
-                const uint64_t lo = x0 < x1 ? x0 : x1, hi = x0 < x1 ? x1 : x0;
-                x0 = dsc ? hi : lo;
-                x1 = dsc ? lo : hi;
-            } else {
-                const int lm = s >> 1;
-                const uint64_t y0 = __shfl_xor_sync(0xffffffffu, x0, lm);
-                const uint64_t y1 = __shfl_xor_sync(0xffffffffu, x1, lm);
-                const int p0 = 2 * lane, p1 = 2 * lane + 1;
-                const bool d0 = (p0 & k) == 0, low0 = (p0 & s) == 0;
-                const bool d1 = (p1 & k) == 0, low1 = (p1 & s) == 0;
-                x0 = (low0 == d0) ? (x0 > y0 ? x0 : y0) : (x0 < y0 ? x0 : y0);
-                x1 = (low1 == d1) ? (x1 > y1 ? x1 : y1) : (x1 < y1 ? x1 : y1);
-            }
-        }
-    }
-}
-
 template <int D>
 struct DecSmem {
-    float K[kBlk][D + 4];   // keys of the slot's block (rows padded: aligned and conflict-free)
-    float V[kBlk][D];
-    float Q[kMaxG][D];
+    union {
+        struct {                  // fp32 inputs: the slot's block and the queries as fp32
+            float K[kBlk][D + 4];  // rows padded: aligned and conflict-free
+            float V[kBlk][D];
+            float Q[kMaxG][D];
+        };
+        struct {                  // bf16 inputs: tensor-core operands (rows padded by 16 bytes)
+            __nv_bfloat16 Kb[kBlk][D + 8];
+            __nv_bfloat16 Vb[kBlk][D + 8];
+            __nv_bfloat16 Qb[kMaxG][D + 8];
+            __nv_bfloat16 Pb[kMaxG][kBlk + 8];
+        };
+    };
     float P[kMaxG][kBlk];   // logits, then probabilities
     float m[kMaxG], l[kMaxG];
     float qbar[D];
@@ -218,24 +206,28 @@ struct DecSmem {
     float cm[8][32], cl[8][32], co[8][32];  // phase D per-warp partials
 };
 
-template <typename T>
-__device__ __forceinline__ void load8(const T* p, float (&f)[8]);
-template <>
-__device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16* p, float (&f)[8]) {
-    const uint4 u = *reinterpret_cast<const uint4*>(p);
-    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const float2 t = __bfloat1622float2(h[i]);
-        f[2 * i] = t.x;
-        f[2 * i + 1] = t.y;
-    }
+// Warp-level bf16 tensor-core tile (m16n8k16, fp32 accumulate) and its shared-memory loaders.
+// Decode's products are 16 heads x 64 keys x d: far too small for the CTA-wide tensor-core path,
+// but on CUDA cores they cost thousands of shared-memory loads per thread.
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void* p) {
+    const uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(p));
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(a));
 }
-template <>
-__device__ __forceinline__ void load8<float>(const float* p, float (&f)[8]) {
-    const float4 a = reinterpret_cast<const float4*>(p)[0], b = reinterpret_cast<const float4*>(p)[1];
-    f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
-    f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+__device__ __forceinline__ void ldsm_x2(uint32_t (&r)[2], const void* p) {
+    const uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(p));
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];" : "=r"(r[0]), "=r"(r[1]) : "r"(a));
+}
+__device__ __forceinline__ void ldsm_x2_t(uint32_t (&r)[2], const void* p) {
+    const uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(p));
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];" : "=r"(r[0]), "=r"(r[1]) : "r"(a));
+}
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
 // 16-byte raw loads, converted later: issuing every load of a phase before the first conversion
@@ -282,8 +274,6 @@ sparse_decode_fused_kernel(const T* __restrict__ q, const T* __restrict__ kc,
     const int K = topk;
     const bool do_sel = idx_in == nullptr && ncand > K;
     const T* qg = q + (b * H + (int64_t)g * G) * D;  // the group's G query rows
-    pdl_trigger();
-    pdl_wait();
 
     // ---------------------------------------------------------------- A: span scores + top-k
     // Rows of k_bar are read coalesced: kLPR lanes per row, 16 elements per lane.  Each span
@@ -334,23 +324,28 @@ sparse_decode_fused_kernel(const T* __restrict__ q, const T* __restrict__ kc,
                 if (lane % kLPR == 0) sm.sc[warp * (kSpan / 8) + st * kRPS + lane / kLPR] = d;
             }
             __syncthreads();
+            // The span's keys sorted largest first (block-wide bitonic network, one key per
+            // thread; strides below 32 within the warp), then its first k written out.
             const int blk = base + tid;
-            uint64_t key[1] = {blk <= hi ? sel_key_u(sm.sc[tid], blk) : 0ull};
-            uint64_t prefix, mask;
-            block_kth<1>(key, K, sm.ss, prefix, mask);
-            if (tid == 0) sm.ss.n = 0;
-            if (tid < kCap) sm.cand[tid] = 0ull;
-            __syncthreads();
-            if (key[0] && (key[0] & mask) >= prefix) sm.cand[atomicAdd(&sm.ss.n, 1)] = key[0];
-            __syncthreads();
-            if (warp == 0) {  // the span's list, largest first (zeros, "no key", last)
-                uint64_t x0 = sm.cand[2 * lane], x1 = sm.cand[2 * lane + 1];
-                warp_sort64_desc(x0, x1, lane);
-                uint64_t* dst = part + ((int64_t)bg * nspan + span) * kCap;
-                dst[2 * lane] = x0;
-                dst[2 * lane + 1] = x1;
+            uint64_t x = blk <= hi ? sel_key_u(sm.sc[tid], blk) : 0ull;
+#pragma unroll
+            for (int kk = 2; kk <= kThreads; kk <<= 1) {
+#pragma unroll
+                for (int jj = kk >> 1; jj > 0; jj >>= 1) {
+                    uint64_t y;
+                    if (jj >= 32) {
+                        sm.cand[tid] = x;
+                        __syncthreads();
+                        y = sm.cand[tid ^ jj];
+                        __syncthreads();
+                    } else {
+                        y = __shfl_xor_sync(0xffffffffu, x, jj);
+                    }
+                    const bool dsc = (tid & kk) == 0, lower = (tid & jj) == 0;
+                    x = (lower == dsc) ? (x > y ? x : y) : (x < y ? x : y);
+                }
             }
-            __syncthreads();
+            if (tid < kCap) part[((int64_t)bg * nspan + span) * kCap + tid] = tid < K ? x : 0ull;
         }
     }
     if (!grid_barrier(bar, gridDim.x, ctx, &sm.ok)) return;
@@ -432,7 +427,15 @@ sparse_decode_fused_kernel(const T* __restrict__ q, const T* __restrict__ kc,
         for (int s = tid; s < slots; s += kThreads) idx_out[(int64_t)bg * slots + s] = sm.sel[s];
 
     // ---------------------------------------------------------------- C: per-slot partials
-    {
+    // bf16: the two products on the tensor cores (warp-level m16n8k16, heads padded to 16 rows);
+    // fp32: on CUDA cores in fp32.
+    constexpr bool kTC = std::is_same<T, __nv_bfloat16>::value;
+    if constexpr (kTC) {
+        for (int e = tid; e < kMaxG * (D / 8); e += kThreads) {
+            const int h = e / (D / 8), c8 = (e % (D / 8)) * 8;
+            *reinterpret_cast<uint4*>(&sm.Qb[h][c8]) = h < G ? ld16(qg + h * D + c8) : make_uint4(0u, 0u, 0u, 0u);
+        }
+    } else {
         constexpr int kQIt = kMaxG * D / kThreads;
         float qv[kQIt];
 #pragma unroll
@@ -481,20 +484,41 @@ sparse_decode_fused_kernel(const T* __restrict__ q, const T* __restrict__ kc,
         for (int u = 0; u < kStage; ++u) {
             const int e = u * kThreads + tid;
             const int row = e / (D / 8), c8 = (e % (D / 8)) * 8;
-            float fk[8], fv[8];
+            if constexpr (kTC) {
+                *reinterpret_cast<uint4*>(&sm.Kb[row][c8]) = rk[u][0];
+                *reinterpret_cast<uint4*>(&sm.Vb[row][c8]) = rv[u][0];
+            } else {
+                float fk[8], fv[8];
 #pragma unroll
-            for (int w = 0; w < kU; ++w) {
-                cvt16<T>(rk[u][w], fk + w * kEl);
-                cvt16<T>(rv[u][w], fv + w * kEl);
+                for (int w = 0; w < kU; ++w) {
+                    cvt16<T>(rk[u][w], fk + w * kEl);
+                    cvt16<T>(rv[u][w], fv + w * kEl);
+                }
+                *reinterpret_cast<float4*>(&sm.K[row][c8]) = make_float4(fk[0], fk[1], fk[2], fk[3]);
+                *reinterpret_cast<float4*>(&sm.K[row][c8 + 4]) = make_float4(fk[4], fk[5], fk[6], fk[7]);
+                *reinterpret_cast<float4*>(&sm.V[row][c8]) = make_float4(fv[0], fv[1], fv[2], fv[3]);
+                *reinterpret_cast<float4*>(&sm.V[row][c8 + 4]) = make_float4(fv[4], fv[5], fv[6], fv[7]);
             }
-            *reinterpret_cast<float4*>(&sm.K[row][c8]) = make_float4(fk[0], fk[1], fk[2], fk[3]);
-            *reinterpret_cast<float4*>(&sm.K[row][c8 + 4]) = make_float4(fk[4], fk[5], fk[6], fk[7]);
-            *reinterpret_cast<float4*>(&sm.V[row][c8]) = make_float4(fv[0], fv[1], fv[2], fv[3]);
-            *reinterpret_cast<float4*>(&sm.V[row][c8 + 4]) = make_float4(fv[4], fv[5], fv[6], fv[7]);
         }
         __syncthreads();
-        // logits: thread = one key x four heads (K row read once for four heads)
-        {
+        if constexpr (kTC) {
+            // logits: warp w owns keys 8w .. 8w+7; A = Q (16 heads x 16 d), B = K rows (keys x d)
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            const int n0 = 8 * warp;
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ++ks) {
+                uint32_t af[4], bf[2];
+                ldsm_x4(af, &sm.Qb[lane & 15][16 * ks + (lane >> 4) * 8]);
+                ldsm_x2(bf, &sm.Kb[n0 + (lane & 7)][16 * ks + ((lane >> 3) & 1) * 8]);
+                mma16816(acc, af, bf);
+            }
+            const int hr = lane >> 2, key = n0 + 2 * (lane & 3);
+            sm.P[hr][key] = key <= lim ? acc[0] * scale : -INFINITY;
+            sm.P[hr][key + 1] = key + 1 <= lim ? acc[1] * scale : -INFINITY;
+            sm.P[hr + 8][key] = key <= lim ? acc[2] * scale : -INFINITY;
+            sm.P[hr + 8][key + 1] = key + 1 <= lim ? acc[3] * scale : -INFINITY;
+        } else {
+            // logits: thread = one key x four heads (K row read once for four heads)
             const int key = tid % kBlk, h0 = (tid / kBlk) * 4;
             if (h0 < G) {
                 float acc[4] = {0.f, 0.f, 0.f, 0.f};
@@ -526,14 +550,57 @@ sparse_decode_fused_kernel(const T* __restrict__ q, const T* __restrict__ kc,
             for (int off = 16; off > 0; off >>= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
             sm.P[hh][lane] = p0;
             sm.P[hh][lane + 32] = p1;
+            if constexpr (kTC) {
+                sm.Pb[hh][lane] = __float2bfloat16_rn(p0);
+                sm.Pb[hh][lane + 32] = __float2bfloat16_rn(p1);
+            }
             if (lane == 0) {
                 sm.m[hh] = m;
                 sm.l[hh] = l;
             }
         }
+        if constexpr (kTC) {  // padding heads: zero probabilities (their rows are never written)
+            for (int e = tid; e < (kMaxG - G) * kBlk; e += kThreads)
+                sm.Pb[G + e / kBlk][e % kBlk] = __float2bfloat16_rn(0.f);
+        }
         __syncthreads();
-        // p v: thread = four columns x the heads hp, hp + ngrp, ... (V read once for them)
-        {
+        if constexpr (kTC) {
+            // p v: warp w owns columns 16w .. 16w+15 of d (two n-tiles; D = 64 uses warps 0-3);
+            // A = P (16 heads x 16 keys), B = V (16 keys x 8 columns, transposed on load)
+            constexpr int kNT = D / 8 / (kThreads / 32);  // n-tiles per warp
+            if (warp * kNT * 8 < D) {
+                float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+                for (int ks = 0; ks < kBlk / 16; ++ks) {
+                    uint32_t af[4];
+                    ldsm_x4(af, &sm.Pb[lane & 15][16 * ks + (lane >> 4) * 8]);
+#pragma unroll
+                    for (int t = 0; t < (kNT > 0 ? kNT : 1); ++t) {
+                        uint32_t bf[2];
+                        ldsm_x2_t(bf, &sm.Vb[16 * ks + (lane & 15)][(warp * kNT + t) * 8]);
+                        mma16816(acc[t], af, bf);
+                    }
+                }
+                const int hr = lane >> 2;
+#pragma unroll
+                for (int t = 0; t < (kNT > 0 ? kNT : 1); ++t) {
+                    const int col = (warp * kNT + t) * 8 + 2 * (lane & 3);
+                    if (hr < G) {
+                        r[hr * (D + 2) + 2 + col] = acc[t][0];
+                        r[hr * (D + 2) + 3 + col] = acc[t][1];
+                    }
+                    if (hr + 8 < G) {
+                        r[(hr + 8) * (D + 2) + 2 + col] = acc[t][2];
+                        r[(hr + 8) * (D + 2) + 3 + col] = acc[t][3];
+                    }
+                }
+            }
+            if (tid < G) {
+                r[tid * (D + 2)] = sm.m[tid];
+                r[tid * (D + 2) + 1] = sm.l[tid];
+            }
+        } else {
+            // p v: thread = four columns x the heads hp, hp + ngrp, ... (V read once for them)
             constexpr int kQuads = D / 4, kGroups = kThreads / kQuads;
             const int dq = tid % kQuads, hp = tid / kQuads;
             for (int h0 = hp; h0 < G; h0 += 2 * kGroups) {
@@ -678,37 +745,15 @@ cudaError_t fused(const void* q, const void* kc, const void* vc, const void* kba
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = (size_t)smem;
     cfg.stream = st;
-    cudaLaunchAttribute attr[2];
+    cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeCooperative;
     attr[0].val.cooperative = 1;
-    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    auto go = [&](int nattr) {
-        cfg.numAttrs = nattr;
-        return cudaLaunchKernelEx(&cfg, kern, static_cast<const T*>(q), static_cast<const T*>(kc),
-                                  static_cast<const T*>(vc), static_cast<const T*>(kbar), idx_in,
-                                  idx_out, static_cast<T*>(o), H, Hkv, pos, Tmax, nb_cap, topk,
-                                  n_init, n_local, slots, scale, cpg, nspan,
-                                  reinterpret_cast<unsigned*>(w), part, rec, ctx);
-    };
-    // Programmatic dependent launch together with the cooperative attribute is tried once, outside
-    // any stream capture; if the launch is refused, later launches use the cooperative attribute
-    // alone.
-    static std::atomic<int> pdl_ok{-1};
-    if (pdl_ok.load() == 1) return go(2);
-    if (pdl_ok.load() == 0) return go(1);
-    cudaStreamCaptureStatus capture = cudaStreamCaptureStatusNone;
-    if (cudaStreamIsCapturing(st, &capture) != cudaSuccess || capture != cudaStreamCaptureStatusNone)
-        return go(1);
-    cudaError_t e = go(2);
-    if (e == cudaSuccess) {
-        pdl_ok.store(1);
-        return e;
-    }
-    (void)cudaGetLastError();  // clear the refused launch's error
-    pdl_ok.store(0);
-    return go(1);
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<const T*>(q), static_cast<const T*>(kc),
+                              static_cast<const T*>(vc), static_cast<const T*>(kbar), idx_in, idx_out,
+                              static_cast<T*>(o), H, Hkv, pos, Tmax, nb_cap, topk, n_init, n_local,
+                              slots, scale, cpg, nspan, reinterpret_cast<unsigned*>(w), part, rec, ctx);
 }
 
 }  // namespace
