@@ -179,6 +179,41 @@ __device__ __forceinline__ void warp_sort64(int& x0, int& x1, int lane) {
     }
 }
 
+// Block-wide bitonic sort, largest first, of the E keys each thread holds (element E*tid + i).
+// Partners within a thread swap in registers, within a warp by shuffle, else through buf (one
+// slot per element, E * blockDim.x keys).
+template <int E>
+__device__ __forceinline__ void block_sort_desc(uint64_t (&x)[E], uint64_t* buf) {
+    const int tid = threadIdx.x;
+#pragma unroll
+    for (int kk = 2; kk <= E * kThreads; kk <<= 1) {
+#pragma unroll
+        for (int jj = kk >> 1; jj > 0; jj >>= 1) {
+            uint64_t y[E];
+            if (jj < E) {
+#pragma unroll
+                for (int i = 0; i < E; ++i) y[i] = x[i ^ jj];
+            } else if (jj < 32 * E) {
+#pragma unroll
+                for (int i = 0; i < E; ++i) y[i] = __shfl_xor_sync(0xffffffffu, x[i], jj / E);
+            } else {
+#pragma unroll
+                for (int i = 0; i < E; ++i) buf[E * tid + i] = x[i];
+                __syncthreads();
+#pragma unroll
+                for (int i = 0; i < E; ++i) y[i] = buf[(E * tid + i) ^ jj];
+                __syncthreads();
+            }
+#pragma unroll
+            for (int i = 0; i < E; ++i) {
+                const int e = E * tid + i;
+                const bool dsc = (e & kk) == 0, lower = (e & jj) == 0;
+                x[i] = (lower == dsc) ? (x[i] > y[i] ? x[i] : y[i]) : (x[i] < y[i] ? x[i] : y[i]);
+            }
+        }
+    }
+}
+
 template <int D>
 struct DecSmem {
     union {
@@ -200,7 +235,7 @@ struct DecSmem {
     float sc[kSpan];
     int sel[kMaxSlots];
     int sel_top[kCap];
-    uint64_t cand[kThreads];
+    uint64_t cand[2 * kThreads];
     SelSmem ss;
     int ok, overflow;
     float cm[8][32], cl[8][32], co[8][32];  // phase D per-warp partials
@@ -327,25 +362,9 @@ sparse_decode_fused_kernel(const T* __restrict__ q, const T* __restrict__ kc,
             // The span's keys sorted largest first (block-wide bitonic network, one key per
             // thread; strides below 32 within the warp), then its first k written out.
             const int blk = base + tid;
-            uint64_t x = blk <= hi ? sel_key_u(sm.sc[tid], blk) : 0ull;
-#pragma unroll
-            for (int kk = 2; kk <= kThreads; kk <<= 1) {
-#pragma unroll
-                for (int jj = kk >> 1; jj > 0; jj >>= 1) {
-                    uint64_t y;
-                    if (jj >= 32) {
-                        sm.cand[tid] = x;
-                        __syncthreads();
-                        y = sm.cand[tid ^ jj];
-                        __syncthreads();
-                    } else {
-                        y = __shfl_xor_sync(0xffffffffu, x, jj);
-                    }
-                    const bool dsc = (tid & kk) == 0, lower = (tid & jj) == 0;
-                    x = (lower == dsc) ? (x > y ? x : y) : (x < y ? x : y);
-                }
-            }
-            if (tid < kCap) part[((int64_t)bg * nspan + span) * kCap + tid] = tid < K ? x : 0ull;
+            uint64_t x[1] = {blk <= hi ? sel_key_u(sm.sc[tid], blk) : 0ull};
+            block_sort_desc<1>(x, sm.cand);
+            if (tid < kCap) part[((int64_t)bg * nspan + span) * kCap + tid] = tid < K ? x[0] : 0ull;
         }
     }
     if (!grid_barrier(bar, gridDim.x, ctx, &sm.ok)) return;
@@ -371,30 +390,55 @@ sparse_decode_fused_kernel(const T* __restrict__ q, const T* __restrict__ kc,
             constexpr int kPre = 8, kPreE = kMergeE * kPre / kCap;  // prefix keys per thread (spans <= 128)
             const unsigned long long* src =
                 reinterpret_cast<const unsigned long long*>(part) + (int64_t)bg * nspan * kCap;
-            uint64_t pk[kPreE];
-#pragma unroll
-            for (int e = 0; e < kPreE; ++e) {
-                const int i = e * kThreads + tid, span = i / kPre;
-                pk[e] = span < nspan ? __ldcg(src + span * kCap + i % kPre) : 0ull;
-            }
-            uint64_t prefix, mask;
-            block_kth<kPreE>(pk, K, sm.ss, prefix, mask);
             if (tid == 0) {
                 sm.ss.n = 0;
                 sm.overflow = 0;
             }
-            __syncthreads();
+            if (nspan * kPre <= 2 * kThreads) {
+                // up to 64 spans: sort the prefixes (two keys per thread); winners are the first k
+                uint64_t x[2], k8[2];
 #pragma unroll
-            for (int e = 0; e < kPreE; ++e) {
-                const int i = e * kThreads + tid;
-                if (pk[e] && (pk[e] & mask) >= prefix && i % kPre == kPre - 1) sm.overflow = 1;
-            }
-            __syncthreads();
-            if (!sm.overflow) {
+                for (int i = 0; i < 2; ++i) {
+                    const int e = 2 * tid + i, span = e / kPre;
+                    x[i] = span < nspan ? __ldcg(src + span * kCap + e % kPre) : 0ull;
+                    k8[i] = e % kPre == kPre - 1 ? x[i] : 0ull;  // a span's last loaded key
+                }
+                block_sort_desc<2>(x, sm.cand);
+                if (tid == (K - 1) / 2) sm.cand[0] = ((K - 1) & 1) ? x[1] : x[0];  // buf is free again
+                __syncthreads();
+                const uint64_t T = sm.cand[0];
+                if (T == 0ull || (k8[0] && k8[0] >= T) || (k8[1] && k8[1] >= T)) sm.overflow = 1;
+                __syncthreads();
+                if (!sm.overflow) {
 #pragma unroll
-                for (int e = 0; e < kPreE; ++e)
-                    if (pk[e] && (pk[e] & mask) >= prefix) sm.sel_top[atomicAdd(&sm.ss.n, 1)] = key_block(pk[e]);
+                    for (int i = 0; i < 2; ++i)
+                        if (2 * tid + i < K) sm.sel_top[2 * tid + i] = key_block(x[i]);
+                }
             } else {
+                uint64_t pk[kPreE];
+#pragma unroll
+                for (int e = 0; e < kPreE; ++e) {
+                    const int i = e * kThreads + tid, span = i / kPre;
+                    pk[e] = span < nspan ? __ldcg(src + span * kCap + i % kPre) : 0ull;
+                }
+                uint64_t prefix, mask;
+                block_kth<kPreE>(pk, K, sm.ss, prefix, mask);
+                if (tid == 0) sm.ss.n = 0;
+                __syncthreads();
+#pragma unroll
+                for (int e = 0; e < kPreE; ++e) {
+                    const int i = e * kThreads + tid;
+                    if (pk[e] && (pk[e] & mask) >= prefix && i % kPre == kPre - 1) sm.overflow = 1;
+                }
+                __syncthreads();
+                if (!sm.overflow) {
+#pragma unroll
+                    for (int e = 0; e < kPreE; ++e)
+                        if (pk[e] && (pk[e] & mask) >= prefix) sm.sel_top[atomicAdd(&sm.ss.n, 1)] = key_block(pk[e]);
+                }
+            }
+            if (sm.overflow) {
+                uint64_t prefix, mask;
                 uint64_t key[kMergeE];
                 const int nk = nspan * kCap;
 #pragma unroll
