@@ -217,6 +217,9 @@ def run_prefill(sala, synth, torch, steps, warmup, stream, workload="hybrid_pref
     kbar = torch.empty((1, HKV, nb, D), device=dev, dtype=torch.bfloat16)
     slots = N_INIT + N_LOCAL + TOPK
     idx = torch.empty((1, HKV, n_tok, slots), device=dev, dtype=torch.int32)
+    # scratch of the sequence-parallel linear prefill (the segments' states)
+    lws = torch.empty(max(sala.linear_prefill_workspace_bytes(1, H, n_tok, D), 16), device=dev,
+                      dtype=torch.uint8)
     torch.cuda.synchronize()
 
     ev = lambda: torch.cuda.Event(enable_timing=True)
@@ -228,7 +231,7 @@ def run_prefill(sala, synth, torch, steps, warmup, stream, workload="hybrid_pref
             if kind == "linear":
                 e0, e1 = (ev(), ev()) if record else (None, None)
                 if record: e0.record(stream)
-                sala.linear_prefill(q, k, v, lam, o=out, stream=stream)
+                sala.linear_prefill(q, k, v, lam, o=out, workspace=lws, stream=stream)
                 if record: e1.record(stream); linear_ev.append((e0, e1))
                 launches += 1
             else:
@@ -389,6 +392,8 @@ def run_e2e(sala, synth, torch, steps, warmup):
     outs = [torch.empty((1, H, N_TOK, D), device=dev, dtype=torch.bfloat16) for _ in range(2)]
     out_host = torch.empty((1, H, N_TOK, D), dtype=torch.bfloat16).pin_memory()
     kbar = torch.empty((1, HKV, N_TOK // BLOCK, D), device=dev, dtype=torch.bfloat16)
+    lws = torch.empty(max(sala.linear_prefill_workspace_bytes(1, H, N_TOK, D), 16), device=dev,
+                      dtype=torch.uint8)
     idx = torch.empty((1, HKV, N_TOK, N_INIT + N_LOCAL + TOPK), device=dev, dtype=torch.int32)
     s_h2d, s_cmp, s_d2h = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
     ev = lambda: torch.cuda.Event()
@@ -418,7 +423,7 @@ def run_e2e(sala, synth, torch, steps, warmup):
                     s_cmp.wait_event(out_free[l & 1])
                 q, k, v = dbuf[kind][slot]
                 if kind == "linear":
-                    sala.linear_prefill(q, k, v, lam, o=o, stream=s_cmp)
+                    sala.linear_prefill(q, k, v, lam, o=o, workspace=lws, stream=s_cmp)
                 else:
                     sala.block_compress(k, kbar, stream=s_cmp)
                     sala.block_topk(q, kbar, TOPK, N_INIT, N_LOCAL, idx=idx, stream=s_cmp)

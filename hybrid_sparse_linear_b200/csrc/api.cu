@@ -127,9 +127,11 @@ sala_status sala_selftest_wait_timeout(sala_stream stream) {
 }
 
 // ----------------------------------------------------------------------------------------------
-sala_status sala_linear_prefill(const void* q, const void* k, const void* v, const float* decay,
-                                void* o, const float* state_in, float* state_out, int B, int H,
-                                int N, int d, int chunk, sala_dtype dt, sala_stream stream) {
+static sala_status linear_prefill_impl(const void* q, const void* k, const void* v,
+                                       const float* decay, void* o, const float* state_in,
+                                       float* state_out, int B, int H, int N, int d, int chunk,
+                                       void* workspace, size_t workspace_bytes, sala_dtype dt,
+                                       sala_stream stream) {
     REQUIRE(B >= 0 && H >= 0 && N >= 0, SALA_ERR_INVALID_ARG, "negative size (B=%d H=%d N=%d)", B, H, N);
     REQUIRE(dt == SALA_F32 || dt == SALA_BF16, SALA_ERR_INVALID_ARG, "unknown dtype %d", (int)dt);
     REQUIRE(d == 64 || d == 128, SALA_ERR_UNSUPPORTED, "head dim %d (supported: 64, 128)", d);
@@ -139,6 +141,7 @@ sala_status sala_linear_prefill(const void* q, const void* k, const void* v, con
     REQUIRE(decay != nullptr, SALA_ERR_INVALID_ARG, "decay must be a device pointer");
     if (state_in) REQUIRE(aligned16(state_in), SALA_ERR_INVALID_ARG, "state_in must be 16-byte aligned");
     if (state_out) REQUIRE(aligned16(state_out), SALA_ERR_INVALID_ARG, "state_out must be 16-byte aligned");
+    if (workspace) REQUIRE(aligned16(workspace), SALA_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
     if (N > 0) {
         REQ_PTR(q); REQ_PTR(k); REQ_PTR(v); REQ_PTR(o);
     }
@@ -148,10 +151,31 @@ sala_status sala_linear_prefill(const void* q, const void* k, const void* v, con
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (dt == SALA_BF16 && N > 0 && sala::linear_prefill_tc_supported(d))
         return launched(sala::launch_linear_prefill_tc(q, k, v, decay, o, state_in, state_out, B,
-                                                       H, N, d, st, ctx), "linear_prefill_tc");
+                                                       H, N, d, workspace, workspace_bytes, st, ctx),
+                        "linear_prefill_tc");
     return launched(sala::launch_linear_prefill_simt(to_dt(dt), q, k, v, decay, o, state_in,
                                                      state_out, B, H, N, d, st, ctx),
                     "linear_prefill");
+}
+
+sala_status sala_linear_prefill(const void* q, const void* k, const void* v, const float* decay,
+                                void* o, const float* state_in, float* state_out, int B, int H,
+                                int N, int d, int chunk, sala_dtype dt, sala_stream stream) {
+    return linear_prefill_impl(q, k, v, decay, o, state_in, state_out, B, H, N, d, chunk, nullptr,
+                               0, dt, stream);
+}
+
+size_t sala_linear_prefill_workspace(int B, int H, int N, int d, sala_dtype dt) {
+    if (dt != SALA_BF16) return 0;
+    return sala::linear_prefill_tc_workspace(B, H, N, d);
+}
+
+sala_status sala_linear_prefill_ws(const void* q, const void* k, const void* v, const float* decay,
+                                   void* o, const float* state_in, float* state_out, int B, int H,
+                                   int N, int d, int chunk, void* workspace,
+                                   size_t workspace_bytes, sala_dtype dt, sala_stream stream) {
+    return linear_prefill_impl(q, k, v, decay, o, state_in, state_out, B, H, N, d, chunk,
+                               workspace, workspace_bytes, dt, stream);
 }
 
 sala_status sala_linear_decode(const void* q, const void* k, const void* v, const float* decay,

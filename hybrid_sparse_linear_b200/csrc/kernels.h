@@ -17,10 +17,14 @@ cudaError_t launch_linear_prefill_simt(DType dt, const void* q, const void* k, c
                                        const float* decay, void* o, const float* s_in,
                                        float* s_out, int B, int H, int N, int d,
                                        cudaStream_t st, DevCtx ctx);
+// bf16, d = 128.  With a workspace of linear_prefill_tc_workspace(...) bytes (0 = not needed) the
+// sequence is split into segments processed in parallel (state pass, chaining, output pass);
+// without it, or when one segment is best, a single pass over the whole sequence.
+size_t linear_prefill_tc_workspace(int B, int H, int N, int d);
 cudaError_t launch_linear_prefill_tc(const void* q, const void* k, const void* v,
                                      const float* decay, void* o, const float* s_in,
-                                     float* s_out, int B, int H, int N, int d, cudaStream_t st,
-                                     DevCtx ctx);
+                                     float* s_out, int B, int H, int N, int d, void* ws,
+                                     size_t ws_bytes, cudaStream_t st, DevCtx ctx);
 bool linear_prefill_tc_supported(int d);
 cudaError_t launch_linear_decode(DType dt, const void* q, const void* k, const void* v,
                                  const float* decay, float* state, void* o, int B, int H, int d,

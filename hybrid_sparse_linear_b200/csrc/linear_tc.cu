@@ -74,15 +74,21 @@ linear_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                          const __grid_constant__ CUtensorMap tmK,
                          const __grid_constant__ CUtensorMap tmV, const float* __restrict__ decay,
                          __nv_bfloat16* __restrict__ out, const float* s_in, float* s_out, int H,
-                         int N, DevCtx ctx) {
+                         int N, int seg_len, int n_seg, int64_t s_in_seg_stride, DevCtx ctx) {
     extern __shared__ uint8_t smraw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smraw) + 1023) &
                                              ~uintptr_t(1023));
     __shared__ Bars bars;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    // CTA = (batch*head, segment of the sequence, value slice); the segment's incoming state is
+    // s_in + seg * s_in_seg_stride (one segment: the whole sequence, stride 0).
     const int slice = blockIdx.x % kSlices;
-    const int64_t bh = blockIdx.x / kSlices;
-    const int n_tiles = (N + kC - 1) / kC;
+    const int seg = (blockIdx.x / kSlices) % n_seg;
+    const int64_t bh = blockIdx.x / kSlices / n_seg;
+    const int row0 = seg * seg_len;
+    const int Ns = min(seg_len, N - row0);  // rows of this segment
+    const int n_tiles = (Ns + kC - 1) / kC;
+    if (s_in) s_in += seg * s_in_seg_stride;
     volatile int* abort = &bars.abort;
 
     if (warp == 9) {
@@ -124,7 +130,7 @@ linear_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                 if (r >= 1 && !wait_or_abort(&bars.empty[s], (r - 1) & 1, ctx, abort)) break;
                 uint8_t* st = sm + s * kStageBytes;
                 mbar_arrive_expect_tx(&bars.full[s], kStageBytes);
-                const int y = c * kC, z = (int)bh;
+                const int y = row0 + c * kC, z = (int)bh;
                 tma_load_3d(st + kOffQ, &tmQ, &bars.full[s], 0, y, z);
                 tma_load_3d(st + kOffQ + kSub, &tmQ, &bars.full[s], 64, y, z);
                 tma_load_3d(st + kOffK, &tmK, &bars.full[s], 0, y, z);
@@ -212,7 +218,7 @@ linear_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
         const float wq = bars.pw[t + 1];
         for (int c = 0; c < n_tiles; ++c) {
             const int s = c & 1;
-            const int len = min(kC, N - c * kC);
+            const int len = min(kC, Ns - c * kC);
             if (!wait_or_abort(&bars.qk_done[s], (c >> 1) & 1, ctx, abort)) break;
             tc_fence_after();
             const uint32_t colA = tmem + lb + kColA0 + s * 128;
@@ -246,7 +252,7 @@ linear_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
             // o_t = O1 + lambda^{t+1} O2
             if (!wait_or_abort(&bars.o_done, c & 1, ctx, abort)) break;
             tc_fence_after();
-            __nv_bfloat16* dst = out + ((bh * N) + (int64_t)c * kC + t) * kD + slice * kDv;
+            __nv_bfloat16* dst = out + ((bh * N) + row0 + (int64_t)c * kC + t) * kD + slice * kDv;
             uint32_t o1[64], o2[64];
             tmem_ld32(tmem + lb + kColO1, *reinterpret_cast<uint32_t(*)[32]>(&o1[0]));
             tmem_ld32(tmem + lb + kColO1 + 32, *reinterpret_cast<uint32_t(*)[32]>(&o1[32]));
@@ -300,7 +306,7 @@ linear_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
         // chunks are visited in their physical order so a warp's 32 rows hit distinct banks.
         auto make_vt = [&](int c) -> bool {
             const int s = c & 1;
-            const int len = min(kC, N - c * kC);
+            const int len = min(kC, Ns - c * kC);
             if (!wait_or_abort(&bars.full[s], (c >> 1) & 1, ctx, abort)) return false;
             const float w = t < len ? bars.pw[len - 1 - t] : 0.f;
             const uint8_t* vrow = sm + s * kStageBytes + kOffV + t * 128;
@@ -325,7 +331,7 @@ linear_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
         bool ok = n_tiles > 0 ? make_vt(0) : true;
         for (int c = 0; c < n_tiles && ok; ++c) {
             const int s = c & 1;
-            const int len = min(kC, N - c * kC);
+            const int len = min(kC, Ns - c * kC);
             if (c + 1 < n_tiles && !make_vt(c + 1)) { ok = false; break; }
             // S <- lambda^len S + dS(c), then its bf16 copy for the next tile.
             if (!wait_or_abort(&bars.ds_done[s], (c >> 1) & 1, ctx, abort)) { ok = false; break; }
@@ -363,14 +369,271 @@ linear_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
     }
 }
 
+// ------------------------------------------------------------------------------------------------
+// Sequence-parallel prefill.  The state recursion S(c) = lambda^len S(c-1) + dS(c) is the only
+// serial dependency, and dS needs no state: so a sequence split into segments can first compute
+// each segment's own contribution S_seg (from a zero state, K and V only), then chain the segments'
+// incoming states in a tiny pass (S_in(p+1) = lambda^len(p) S_in(p) + S_seg(p)), then run the
+// output pass above on every segment at once.  K and V are read twice, but every SM has work.
+//
+// State pass, per CTA = (batch*head, segment, value slice): warp 4 streams K and the V slice
+// through a 3-stage ring, warp 5 issues dS = K^T V~ per tile into one of two TMEM buffers, and
+// warps 0-3 (thread = row of S) write V~ and fold dS into the fp32 state held in registers.
+constexpr int kStStages = 3;
+constexpr int kStStage = 3 * kSub;                     // K (2 sub-tiles) + V slice (1)
+constexpr int kStOffVt = kStStages * kStStage;         // V~, 2 buffers
+constexpr int kStSmem = kStOffVt + 2 * kSub + 1024;
+constexpr int kStThreads = 192;
+
+struct StBars {
+    uint64_t full[kStStages], empty[kStStages];
+    uint64_t v_ready[2], ds_done[2], ds_free[2];
+    uint64_t fin;
+    uint32_t tmem_base;
+    int abort;
+    float pw[kC + 1];
+};
+
+__global__ void __launch_bounds__(kStThreads, 1)
+linear_state_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                       const float* __restrict__ decay, float* __restrict__ s_seg, int H, int N,
+                       int seg_len, int n_seg, int64_t seg_stride, DevCtx ctx) {
+    extern __shared__ uint8_t smraw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smraw) + 1023) &
+                                             ~uintptr_t(1023));
+    __shared__ StBars bars;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int slice = blockIdx.x % kSlices;
+    const int seg = (blockIdx.x / kSlices) % n_seg;
+    const int64_t bh = blockIdx.x / kSlices / n_seg;
+    const int row0 = seg * seg_len;
+    const int Ns = min(seg_len, N - row0);
+    const int n_tiles = (Ns + kC - 1) / kC;
+    volatile int* abort = &bars.abort;
+    if (warp == 5) {
+        tmem_alloc(&bars.tmem_base, 128);
+        tmem_relinquish();
+    }
+    if (tid == 0) {
+        for (int s = 0; s < kStStages; ++s) {
+            mbar_init(&bars.full[s], 1);
+            mbar_init(&bars.empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&bars.v_ready[b], 4);
+            mbar_init(&bars.ds_done[b], 1);
+            mbar_init(&bars.ds_free[b], 4);
+        }
+        mbar_init(&bars.fin, 1);
+        bars.abort = 0;
+        fence_mbar_init();
+    }
+    {
+        const double lam = (double)decay[bh % H];
+        for (int n = tid; n <= kC; n += kStThreads) bars.pw[n] = (float)pow(lam, (double)n);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bars.tmem_base;
+
+    if (warp == 4) {
+        // ---------------------------------------------------------------- TMA producer
+        if (lane == 0) {
+            int last = -1;
+            for (int c = 0; c < n_tiles; ++c) {
+                const int s = c % kStStages, r = c / kStStages;
+                if (r >= 1 && !wait_or_abort(&bars.empty[s], (r - 1) & 1, ctx, abort)) break;
+                uint8_t* st = sm + s * kStStage;
+                mbar_arrive_expect_tx(&bars.full[s], kStStage);
+                const int y = row0 + c * kC, z = (int)bh;
+                tma_load_3d(st, &tmK, &bars.full[s], 0, y, z);
+                tma_load_3d(st + kSub, &tmK, &bars.full[s], 64, y, z);
+                tma_load_3d(st + 2 * kSub, &tmV, &bars.full[s], slice * kDv, y, z);
+                last = c;
+            }
+            for (int c = last - kStStages + 1; c <= last; ++c)  // drain: copies in flight land
+                if (c >= 0) (void)mbar_wait(&bars.full[c % kStStages], (c / kStStages) & 1, ctx);
+        }
+        __syncwarp();
+    } else if (warp == 5) {
+        // ---------------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            const uint32_t idDS = idesc_bf16_f32(128, kDv, true, true);
+            for (int c = 0; c < n_tiles; ++c) {
+                const int s = c % kStStages, b = c & 1;
+                if (!wait_or_abort(&bars.full[s], (c / kStStages) & 1, ctx, abort)) break;
+                if (!wait_or_abort(&bars.v_ready[b], (c >> 1) & 1, ctx, abort)) break;
+                if (c >= 2 && !wait_or_abort(&bars.ds_free[b], ((c - 2) >> 1) & 1, ctx, abort)) break;
+                tc_fence_after();
+                const uint32_t k = smem_u32(sm + s * kStStage);
+                const uint32_t vt = smem_u32(sm + kStOffVt + b * kSub);
+#pragma unroll
+                for (int ks = 0; ks < kC / 16; ++ks)
+                    mma_ss(tmem + b * kDv, sdesc_sw128(k + ks * 16 * 128, kSub, 1024),
+                           sdesc_sw128(vt + ks * 16 * 128, 8192, 1024), idDS, ks > 0);
+                mma_commit(&bars.ds_done[b]);
+                mma_commit(&bars.empty[s]);
+            }
+            mma_commit(&bars.fin);
+            (void)mbar_wait(&bars.fin, 0, ctx);
+        }
+        __syncwarp();
+    } else {
+        // ---------------------------------------------------------------- V~ and the state
+        const int t = tid;  // row of the V tile / of the state slice
+        const uint32_t lb = tmem_lane_base(warp);
+        float S[kDv];
+#pragma unroll
+        for (int j = 0; j < kDv; ++j) S[j] = 0.f;
+        auto make_vt = [&](int c) -> bool {
+            const int s = c % kStStages;
+            const int len = min(kC, Ns - c * kC);
+            if (!wait_or_abort(&bars.full[s], (c / kStStages) & 1, ctx, abort)) return false;
+            const float w = t < len ? bars.pw[len - 1 - t] : 0.f;
+            const uint8_t* vrow = sm + s * kStStage + 2 * kSub + t * 128;
+            uint8_t* vtrow = sm + kStOffVt + (c & 1) * kSub + t * 128;
+#pragma unroll
+            for (int cj = 0; cj < 8; ++cj) {
+                const int p = (cj ^ (t & 7)) << 4;
+                const uint4 a = *reinterpret_cast<const uint4*>(vrow + p);
+                uint4 o;
+                o.x = pack_bf16x2(bf_lo(a.x) * w, bf_hi(a.x) * w);
+                o.y = pack_bf16x2(bf_lo(a.y) * w, bf_hi(a.y) * w);
+                o.z = pack_bf16x2(bf_lo(a.z) * w, bf_hi(a.z) * w);
+                o.w = pack_bf16x2(bf_lo(a.w) * w, bf_hi(a.w) * w);
+                *reinterpret_cast<uint4*>(vtrow + p) = o;
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars.v_ready[c & 1]);
+            return true;
+        };
+        bool ok = n_tiles > 0 ? make_vt(0) : true;
+        for (int c = 0; c < n_tiles && ok; ++c) {
+            const int b = c & 1;
+            const int len = min(kC, Ns - c * kC);
+            if (c + 1 < n_tiles && !(ok = make_vt(c + 1))) break;
+            if (!(ok = wait_or_abort(&bars.ds_done[b], (c >> 1) & 1, ctx, abort))) break;
+            tc_fence_after();
+            uint32_t d0[32], d1[32];
+            tmem_ld32(tmem + lb + b * kDv, d0);
+            tmem_ld32(tmem + lb + b * kDv + 32, d1);
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars.ds_free[b]);
+            const float decay_len = bars.pw[len];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                S[j] = fmaf(decay_len, S[j], __uint_as_float(d0[j]));
+                S[32 + j] = fmaf(decay_len, S[32 + j], __uint_as_float(d1[j]));
+            }
+        }
+        if (ok) {
+            float* row = s_seg + seg * seg_stride + (bh * kD + t) * kD + slice * kDv;
+#pragma unroll
+            for (int j = 0; j < kDv; j += 4)
+                *reinterpret_cast<float4*>(row + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 5) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 128);
+    }
+}
+
+// Chains the segments' states, in place: on entry s_seg[p] holds segment p's own contribution, on
+// exit its incoming state S_in(p); S_in(0) = state_in (or 0), S_in(p+1) = lambda^len(p) S_in(p)
+// + S_seg(p).  state_out (if given) receives the state after the last segment.  Thread = one
+// state element of one head.
+constexpr int kMaxSeg = 64;
+__global__ void __launch_bounds__(256)
+linear_state_chain_kernel(float* __restrict__ s_seg, const float* __restrict__ state_in,
+                          float* __restrict__ state_out, const float* __restrict__ decay, int BH,
+                          int H, int N, int seg_len, int n_seg) {
+    const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;  // over BH * d * d
+    if (e >= (int64_t)BH * kD * kD) return;
+    const int64_t bh = e / (kD * kD);
+    const int64_t seg_stride = (int64_t)BH * kD * kD;
+    const double lam = (double)decay[bh % H];
+    const float w_full = (float)pow(lam, (double)seg_len);
+    const float w_last = (float)pow(lam, (double)(N - (n_seg - 1) * seg_len));
+    float s = state_in ? state_in[e] : 0.f;
+    for (int p0 = 0; p0 < n_seg; p0 += 8) {  // 8 segments' loads in flight, then their updates
+        float contrib[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) contrib[i] = p0 + i < n_seg ? s_seg[(p0 + i) * seg_stride + e] : 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int p = p0 + i;
+            if (p < n_seg) {
+                s_seg[p * seg_stride + e] = s;
+                s = fmaf(p + 1 < n_seg ? w_full : w_last, s, contrib[i]);
+            }
+        }
+    }
+    if (state_out) state_out[e] = s;
+}
+
 }  // namespace
 
 bool linear_prefill_tc_supported(int d) { return d == kD; }
 
+namespace {
+
+int sm_count() {
+    static int n = 0;
+    if (!n) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (n <= 0) n = 148;
+    }
+    return n;
+}
+
+// Segments for the sequence-parallel form: the count that minimises (waves of output-pass CTAs) x
+// (rows per segment) plus a per-segment cost for the state chaining (a segment boundary costs about
+// as much as 64 rows of output work).  Short sequences, or ones whose heads already fill the GPU,
+// stay in one segment.
+void pick_segments(int B, int H, int N, int* n_seg, int* seg_len) {
+    *n_seg = 1;
+    *seg_len = N;
+    const int64_t ctas1 = (int64_t)B * H * kSlices;
+    const int nsm = sm_count();
+    if (N < 8 * kC || ctas1 >= 2 * nsm) return;
+    double best = (double)((ctas1 + nsm - 1) / nsm) * N;
+    for (int n = 2; n <= kMaxSeg; ++n) {
+        const int len = ((N + n - 1) / n + kC - 1) / kC * kC;
+        const int ne = (N + len - 1) / len;
+        if (ne != n) continue;
+        const double waves = (double)((ctas1 * ne + nsm - 1) / nsm);
+        const double cost = waves * len + 64.0 * ne;
+        if (cost < best) {
+            best = cost;
+            *n_seg = ne;
+            *seg_len = len;
+        }
+    }
+}
+
+}  // namespace
+
+size_t linear_prefill_tc_workspace(int B, int H, int N, int d) {
+    if (d != kD || B <= 0 || H <= 0 || N <= 0) return 0;
+    int n_seg, seg_len;
+    pick_segments(B, H, N, &n_seg, &seg_len);
+    return n_seg > 1 ? (size_t)n_seg * B * H * kD * kD * sizeof(float) : 0;
+}
+
 cudaError_t launch_linear_prefill_tc(const void* q, const void* k, const void* v,
                                      const float* decay, void* o, const float* s_in,
-                                     float* s_out, int B, int H, int N, int d, cudaStream_t st,
-                                     DevCtx ctx) {
+                                     float* s_out, int B, int H, int N, int d, void* ws,
+                                     size_t ws_bytes, cudaStream_t st, DevCtx ctx) {
     if (d != kD) return cudaErrorNotSupported;
     EncodeTiledFn fn = encode_tiled_fn();
     if (!fn) return cudaErrorNotSupported;
@@ -387,10 +650,31 @@ cudaError_t launch_linear_prefill_tc(const void* q, const void* k, const void* v
     if (!make3(&tmQ, q) || !make3(&tmK, k) || !make3(&tmV, v)) return cudaErrorInvalidValue;
     cudaError_t e = ensure_smem<linear_prefill_tc_kernel>(kSmemBytes);
     if (e != cudaSuccess) return e;
-    // If state_out aliases state_in, every CTA reads its slice before it writes it back, and no
-    // two CTAs share a slice, so in-place update is safe.
+    int n_seg, seg_len;
+    pick_segments(B, H, N, &n_seg, &seg_len);
+    const int64_t seg_stride = (int64_t)B * H * kD * kD;
+    if (n_seg > 1 && ws && ws_bytes >= (size_t)n_seg * seg_stride * sizeof(float)) {
+        float* s_seg = static_cast<float*>(ws);
+        e = ensure_smem<linear_state_tc_kernel>(kStSmem);
+        if (e != cudaSuccess) return e;
+        linear_state_tc_kernel<<<B * H * n_seg * kSlices, kStThreads, kStSmem, st>>>(
+            tmK, tmV, decay, s_seg, H, N, seg_len, n_seg, seg_stride, ctx);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        const int64_t elems = seg_stride;
+        linear_state_chain_kernel<<<(unsigned)((elems + 255) / 256), 256, 0, st>>>(
+            s_seg, s_in, s_out, decay, B * H, H, N, seg_len, n_seg);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        linear_prefill_tc_kernel<<<B * H * n_seg * kSlices, kThreads, kSmemBytes, st>>>(
+            tmQ, tmK, tmV, decay, static_cast<__nv_bfloat16*>(o), s_seg, nullptr, H, N, seg_len,
+            n_seg, seg_stride, ctx);
+        return cudaGetLastError();
+    }
+    // One segment.  If state_out aliases state_in, every CTA reads its slice before it writes it
+    // back, and no two CTAs share a slice, so in-place update is safe.
     linear_prefill_tc_kernel<<<B * H * kSlices, kThreads, kSmemBytes, st>>>(
-        tmQ, tmK, tmV, decay, static_cast<__nv_bfloat16*>(o), s_in, s_out, H, N, ctx);
+        tmQ, tmK, tmV, decay, static_cast<__nv_bfloat16*>(o), s_in, s_out, H, N, N, 1, 0, ctx);
     return cudaGetLastError();
 }
 

@@ -26,6 +26,10 @@ F32, BF16 = 0, 1
 
 _vp, _i, _st = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
 _lib.sala_linear_prefill.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]
+_lib.sala_linear_prefill_ws.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp,
+                                        ctypes.c_size_t, _i, _vp]
+_lib.sala_linear_prefill_workspace.argtypes = [_i, _i, _i, _i, _i]
+_lib.sala_linear_prefill_workspace.restype = ctypes.c_size_t
 _lib.sala_linear_decode.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp]
 _lib.sala_block_compress.argtypes = [_vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp]
 _lib.sala_block_topk.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp,
@@ -93,8 +97,16 @@ def _need(t, name, shape=None, dtype=None):
 
 
 # ----------------------------------------------------------------------------------------------
-def linear_prefill(q, k, v, decay, o=None, state_in=None, state_out=None, chunk=0, stream=None):
-    """Chunked decayed linear attention.  q,k,v: [B,H,N,d]; decay [H] fp32.  Returns o."""
+def linear_prefill_workspace_bytes(B, H, N, d, dtype=torch.bfloat16):
+    return _lib.sala_linear_prefill_workspace(B, H, N, d, 1 if dtype == torch.bfloat16 else 0)
+
+
+def linear_prefill(q, k, v, decay, o=None, state_in=None, state_out=None, chunk=0, workspace=None,
+                   stream=None):
+    """Chunked decayed linear attention.  q,k,v: [B,H,N,d]; decay [H] fp32.  Returns o.
+    workspace: None = one pass (sala_linear_prefill); a uint8 device tensor of at least
+    linear_prefill_workspace_bytes(...) bytes lets long sequences run as parallel segments
+    (sala_linear_prefill_ws)."""
     B, H, N, d = q.shape
     _need(q, "q"); _need(k, "k", q.shape, q.dtype); _need(v, "v", q.shape, q.dtype)
     _need(decay, "decay", (H,), torch.float32)
@@ -103,9 +115,15 @@ def linear_prefill(q, k, v, decay, o=None, state_in=None, state_out=None, chunk=
     _need(o, "o", q.shape, q.dtype)
     _need(state_in, "state_in", (B, H, d, d), torch.float32)
     _need(state_out, "state_out", (B, H, d, d), torch.float32)
-    _check(_lib.sala_linear_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(decay), _ptr(o),
-                                    _ptr(state_in), _ptr(state_out), B, H, N, d, chunk, _dt(q),
-                                    _stream(stream)), "sala_linear_prefill")
+    if workspace is None:
+        _check(_lib.sala_linear_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(decay), _ptr(o),
+                                        _ptr(state_in), _ptr(state_out), B, H, N, d, chunk, _dt(q),
+                                        _stream(stream)), "sala_linear_prefill")
+    else:
+        _check(_lib.sala_linear_prefill_ws(_ptr(q), _ptr(k), _ptr(v), _ptr(decay), _ptr(o),
+                                           _ptr(state_in), _ptr(state_out), B, H, N, d, chunk,
+                                           _ptr(workspace), workspace.numel(), _dt(q),
+                                           _stream(stream)), "sala_linear_prefill_ws")
     return o
 
 

@@ -75,6 +75,24 @@ sala_status sala_linear_prefill(const void* q, const void* k, const void* v, con
                                 void* o, const float* state_in, float* state_out, int B, int H,
                                 int N, int d, int chunk, sala_dtype dt, sala_stream stream);
 
+/* sala_linear_prefill with device scratch, so that long sequences can be split into segments that
+ * run in parallel.  The pages have no counterpart; the split is the state recursion's own
+ * associativity: each segment's state contribution is computed from a zero state, the segments'
+ * incoming states are chained (S_in(p+1) = lambda^len(p) S_in(p) + S_seg(p)), then every
+ * segment's output is computed from its incoming state.  K and V are read twice; in exchange
+ * every SM has work when B * H alone would leave most of the GPU idle.  The result equals the
+ * one-pass result up to rounding (the state is associated differently).
+ * workspace       : at least sala_linear_prefill_workspace(B, H, N, d, dt) bytes of device
+ *                   scratch (16-byte aligned; no initial value needed), not shared with a
+ *                   concurrent call.  A size of 0 means this problem runs in one pass; with
+ *                   NULL or too small a workspace the call also runs in one pass.
+ * Other arguments, validation and errors are those of sala_linear_prefill. */
+sala_status sala_linear_prefill_ws(const void* q, const void* k, const void* v, const float* decay,
+                                   void* o, const float* state_in, float* state_out, int B, int H,
+                                   int N, int d, int chunk, void* workspace,
+                                   size_t workspace_bytes, sala_dtype dt, sala_stream stream);
+size_t sala_linear_prefill_workspace(int B, int H, int N, int d, sala_dtype dt);
+
 /* One decode step of the linear attention for every (batch, head): the state is updated first
  * and then read, so the current token attends to itself with lambda^0:
  *   S <- lambda_h S + k^T v ;  o = q S

@@ -128,14 +128,21 @@ def test_decode_continues_prefill(sala):
     assert_close(_f64(o_pre[:, :, -1]), ref.reshape(1, H, d), "bf16", "prefill row")
 
 
-def test_linear_prefill_full_size_sampled(sala):
+@pytest.mark.parametrize("segments", [False, True])
+def test_linear_prefill_full_size_sampled(sala, segments):
     """32 heads x 32768 tokens x d 128 (bf16), checked on sampled rows of four heads, including
-    the first and last rows and rows on both sides of 64- and 128-row boundaries."""
+    the first and last rows and rows on both sides of 64- and 128-row boundaries; in one pass and
+    split into parallel segments (then also on rows at segment boundaries)."""
     from hybrid_sparse_linear_b200 import synth
     B, H, N, d = 1, 32, 32768, 128
     q, k, v = synth.linear_layer(B, H, N, d, torch.bfloat16, "cuda", layer=0)
     lam = synth.decays(H).cuda()
-    o = sala.linear_prefill(q, k, v, lam)
+    ws = None
+    if segments:
+        nbytes = sala.linear_prefill_workspace_bytes(B, H, N, d)
+        assert nbytes > 0, "expected this shape to run as segments"
+        ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    o = sala.linear_prefill(q, k, v, lam, workspace=ws)
     sala.check_status()
     heads = [0, 7, 19, 31]
     toks = [0, 1, 63, 64, 127, 128, 129, 4095, 4096, 20000, N - 129, N - 128, N - 2, N - 1]
@@ -144,3 +151,33 @@ def test_linear_prefill_full_size_sampled(sala):
     ref = oracle.linear_quadratic(sub(q), sub(k), sub(v), _f64(lam.cpu()[heads]), rows=rows)
     got = np.stack([_f64(o[0, heads[hi], t]) for hi, t in rows])
     assert_close(got, ref, "bf16", "sampled rows")
+
+
+def test_bf16_prefill_segments_ragged_with_state(sala):
+    """The segment-parallel form on every row of a ragged length, with a carried-in state and the
+    state out (the chained state after the last segment) against the fp64 recurrence."""
+    from hybrid_sparse_linear_b200 import synth
+    B, H, N, d = 1, 32, 5000, 128
+    nbytes = sala.linear_prefill_workspace_bytes(B, H, N, d)
+    assert nbytes > 0, "expected this shape to run as segments"
+    q, k, v = _inputs(B, H, N, d, torch.bfloat16, 700)
+    lam = synth.decays(H)
+    g = torch.Generator().manual_seed(9)
+    s_in = torch.randn((B, H, d, d), generator=g) / d
+    so = torch.empty((B, H, d, d), device="cuda")
+    ws = torch.full((nbytes,), 0xFF, dtype=torch.uint8, device="cuda")  # no initial value needed
+    o = sala.linear_prefill(q.cuda(), k.cuda(), v.cuda(), lam.cuda(), state_in=s_in.cuda(),
+                            state_out=so, workspace=ws)
+    sala.check_status()
+    ref, s_ref = oracle.linear_recurrent(_f64(q), _f64(k), _f64(v), _f64(lam), _f64(s_in))
+    assert_close(_f64(o), ref, "bf16", "o")
+    assert_close(_f64(so), s_ref, "bf16", "state_out")
+
+
+def test_prefill_workspace_size_contract(sala):
+    """Short sequences need no workspace; fp32 never uses one; a NULL workspace falls back to one
+    pass (covered by the unsegmented runs above)."""
+    assert sala.linear_prefill_workspace_bytes(1, 32, 512, 128) == 0
+    assert sala.linear_prefill_workspace_bytes(1, 32, 32768, 128, torch.float32) == 0
+    n = sala.linear_prefill_workspace_bytes(1, 32, 32768, 128)
+    assert n > 0 and n % (32 * 128 * 128 * 4) == 0
