@@ -1,5 +1,5 @@
 // Block selection on the 5th-generation tensor cores (sm_100a): scores of 128 query rows against
-// 128 candidate blocks per MMA, exact per-row top-k with a provable floor.
+// 128 candidate blocks per MMA, exact per-row top-k behind a provable floor.
 //
 // Tile: 128 consecutive query rows (two query blocks) of one (batch, KV group).  The group-summed
 // query qbar_r = sum_{h in g} q_{h,r} is formed in fp32 and split into two bf16 terms
@@ -7,20 +7,23 @@
 // of qbar on bf16 tensor cores (kbar itself is bf16, exact).
 //
 // Floor: the pilot vector p = sum_r qbar_r ranks the candidates that every row of the tile may
-// take; its top-k become seeds.  For a row r with at least k seeds, its k-th best key is at least
-// the smallest key among its own k seed keys (k real candidates reach that key), so any candidate
-// whose key is below that floor can never enter row r's top-k and is skipped.  The seeds only
-// decide how much work is skipped, never the result: the selection is exact.
+// take; its best 2k become seeds.  Row r's k-th best score is at least the k-th best of its own
+// seed scores (k real candidates reach it), so a candidate scoring below that floor can never
+// enter row r's top-k.  The seeds only decide how much work is skipped, never the result: the
+// selection is exact.
 //
 // Main pass, per 128-candidate tile: MMA (2 x 8 K-steps, N = 128) -> TMEM (double-buffered) ->
-// warps 0-3 copy row r's 128 scores to shared memory -> warps 0-7 run the warp-level top-k of 16
-// rows each (best 64 keys per row in registers, two per lane; only candidates above both the
-// floor and the current k-th key are inserted).  Key = (orderable score, ~block), so ties go to
-// the lower block index.  Output as the CUDA-core path: init ids, sorted top-k ids, local ids.
+// one thread per query row reads its 128 scores straight from TMEM, compares each with the row's
+// floor, and appends the few that pass to the row's buffer in shared memory.  A full buffer is
+// cut back to its best k (the floor rises to the k-th); at the end each row's buffer is sorted
+// (one warp per row) and the best k taken.  Key = (orderable score, ~block), so ties go to the
+// lower block index.  Output as the CUDA-core path: init ids, sorted top-k ids, local ids.
 //
-// Roles (320 threads): warps 0-7 workers, warp 8 TMA producer (kbar tiles), warp 9 TMEM owner and
-// MMA issuer.  Every wait is bounded; the 8 workers leave their loops only together (see the
-// sparse prefill kernel for the same named-barrier discipline).
+// Roles (320 threads): warps 0-7 workers (the main pass runs on warps 0-3, thread = row = TMEM
+// lane), warp 8 TMA producer (kbar tiles), warp 9 TMEM owner and MMA issuer.  Every wait is
+// bounded; the 8 workers leave only together (the sparse prefill kernel's named-barrier
+// discipline).
+#include "blocksel.cuh"
 #include "kernels.h"
 #include "ptx.cuh"
 #include "tmap.cuh"
@@ -32,14 +35,24 @@ using namespace ptx;
 
 constexpr int kD = 128, kRows = 128, kCand = 128, kBlk = 64, kCap = 64;
 constexpr int kThreads = 320, kWorkers = 256;
+constexpr int kMaxG = 16;
+constexpr int kBufCap = 88;                            // buffered keys per row
 constexpr int kSub = 128 * 128;                        // [128 rows x 128 B] = 16 KiB
 constexpr int kOffAhi = 0, kOffAlo = 2 * kSub;         // A operands (hi, lo), 2 sub-tiles each
 constexpr int kOffKb = 4 * kSub;                       // kbar tiles, 2 stages x 2 sub-tiles
-constexpr int kOffSeedB = 8 * kSub;                    // seed kbar rows [64 x 128 d], 2 sub-tiles of 8 KiB
-constexpr int kSCStride = kCand + 4;                   // floats per row of the score tile
-constexpr int kOffSC = kOffSeedB + 2 * 8192;
-constexpr int kOffPList = kOffSC + kRows * kSCStride * 4;  // 8 warp lists x 64 keys
-constexpr int kSmemBytes = kOffPList + 8 * kCap * 8 + 1024;
+constexpr int kOffBuf = 8 * kSub;                      // row buffers [128][kBufCap] keys
+constexpr int kBufBytes = kRows * kBufCap * 8;
+constexpr int kSmemBytes = kOffBuf + kBufBytes + 1024;
+// Before the main pass the buffer area holds, in turn: the pilot partial sums, the pilot keys of
+// one chunk of candidates, and the seeds' kbar rows (the B operand of the seed MMA).
+constexpr int kOffPPart = kOffBuf;                     // [8][128] floats
+constexpr int kPilotChunk = 16 * kWorkers;             // keys per radix-select chunk
+constexpr int kOffPKeys = kOffBuf;                     // [kPilotChunk] keys
+constexpr int kSeeds = 2 * kCap;                       // pilot seeds (the floor uses the k-th)
+constexpr int kOffSeedB = kOffBuf + kPilotChunk * 8;   // [128 seeds x 128 d], 2 sub-tiles
+constexpr int kOffSeedSc = kOffBuf;  // [128 rows][kSeeds + 1] seed scores, once the seed MMA is done
+static_assert(kOffSeedB + 2 * kSub <= kOffBuf + kBufBytes, "buffer area too small");
+static_assert(kRows * (kSeeds + 1) * 4 <= kBufBytes, "buffer area too small for the seed scores");
 
 constexpr uint32_t kColS0 = 0, kColSeed = 256, kTmemCols = 512;
 
@@ -51,61 +64,13 @@ struct Bars {
     int abort;
     int sm_stop;
     float pilot[kD];
-    float ppart[8][kD];
-    uint64_t floor_key[kRows];
-    int seeds[kCap];
-    int n_seeds;
+    float floor_s[kRows];
+    int buf_n[kRows];
+    uint64_t carry[kSeeds];
+    int seeds[kSeeds];
+    int n_seeds, n_win;
+    RadixSelSmem rs;
 };
-
-__device__ __forceinline__ uint64_t shfl64(uint64_t x, int src) { return __shfl_sync(0xffffffffu, x, src); }
-
-__device__ __forceinline__ uint64_t kth_key(uint64_t l0, uint64_t l1, int K) {
-    return shfl64(((K - 1) & 1) ? l1 : l0, (K - 1) >> 1);
-}
-
-// Offer one key per lane to the warp's descending list (keeps the best K <= 64); keys at or below
-// `floor` are dropped.
-__device__ __forceinline__ void offer(uint64_t& l0, uint64_t& l1, uint64_t key, uint64_t floor,
-                                      int K, int lane) {
-    uint64_t thr = kth_key(l0, l1, K);
-    if (floor > thr) thr = floor - 1;  // a key equal to the floor may still enter
-    bool take = key > thr;
-    unsigned m = __ballot_sync(0xffffffffu, take);
-    while (m) {
-        const int src = __ffs(m) - 1;
-        const uint64_t kn = shfl64(key, src);
-        const int p = __popc(__ballot_sync(0xffffffffu, l0 > kn)) + __popc(__ballot_sync(0xffffffffu, l1 > kn));
-        const uint64_t prev1 = __shfl_up_sync(0xffffffffu, l1, 1);
-        const int q0 = 2 * lane, q1 = 2 * lane + 1;
-        const uint64_t n0 = q0 < p ? l0 : (q0 == p ? kn : prev1);
-        const uint64_t n1 = q1 < p ? l1 : (q1 == p ? kn : l0);
-        l0 = n0;
-        l1 = n1;
-        if (lane == src) take = false;
-        thr = kth_key(l0, l1, K);
-        if (floor > thr) thr = floor - 1;
-        m = __ballot_sync(0xffffffffu, take && key > thr);
-    }
-}
-
-// Top-64 (descending) of two descending 64-key lists held two per lane: elementwise max against
-// the reversed second list gives a bitonic sequence holding the top half, then a bitonic clean.
-__device__ __forceinline__ void merge_desc(uint64_t& a0, uint64_t& a1, uint64_t b0, uint64_t b1, int lane) {
-    const uint64_t r0 = shfl64(b1, 31 - lane), r1 = shfl64(b0, 31 - lane);  // reversed B
-    a0 = a0 > r0 ? a0 : r0;
-    a1 = a1 > r1 ? a1 : r1;
-#pragma unroll
-    for (int s = 32; s >= 2; s >>= 1) {
-        const int lm = s >> 1;
-        const uint64_t y0 = shfl64(a0, lane ^ lm), y1 = shfl64(a1, lane ^ lm);
-        const bool low = (lane & lm) == 0;  // this lane holds the lower position of the pair
-        a0 = low ? (a0 > y0 ? a0 : y0) : (a0 < y0 ? a0 : y0);
-        a1 = low ? (a1 > y1 ? a1 : y1) : (a1 < y1 ? a1 : y1);
-    }
-    const uint64_t hi = a0 > a1 ? a0 : a1, lo = a0 > a1 ? a1 : a0;
-    a0 = hi;
-    a1 = lo;
-}
 
 // Ascending bitonic sort of 64 ints held two per lane.
 __device__ __forceinline__ void sort64_asc(int& x0, int& x1, int lane) {
@@ -130,6 +95,42 @@ __device__ __forceinline__ void sort64_asc(int& x0, int& x1, int lane) {
             }
         }
     }
+}
+
+// Descending bitonic sort of 128 keys held four per lane (element 4*lane + i).
+__device__ __forceinline__ void sort128_desc(uint64_t (&x)[4], int lane) {
+#pragma unroll
+    for (int kk = 2; kk <= 128; kk <<= 1) {
+#pragma unroll
+        for (int jj = kk >> 1; jj > 0; jj >>= 1) {
+            uint64_t y[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                y[i] = jj < 4 ? x[i ^ jj] : __shfl_xor_sync(0xffffffffu, x[i], jj >> 2);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int e = 4 * lane + i;
+                const bool dsc = (e & kk) == 0, lower = (e & jj) == 0;
+                x[i] = (lower == dsc) ? (x[i] > y[i] ? x[i] : y[i]) : (x[i] < y[i] ? x[i] : y[i]);
+            }
+        }
+    }
+}
+
+// Cuts a full row buffer back to its k best keys (thread-serial; rare with a good floor) and
+// returns the new floor score (that of the k-th key).
+__device__ __forceinline__ float cut_buffer(uint64_t* buf, int n, int K) {
+    for (int i = 1; i < n; ++i) {  // insertion sort, descending
+        const uint64_t v = buf[i];
+        int j = i - 1;
+        while (j >= 0 && buf[j] < v) {
+            buf[j + 1] = buf[j];
+            --j;
+        }
+        buf[j + 1] = v;
+    }
+    const uint32_t o = (uint32_t)(buf[K - 1] >> 32);  // orderable score of the k-th key
+    return __uint_as_float((o & 0x80000000u) ? (o & 0x7fffffffu) : ~o);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -207,18 +208,18 @@ topk_tc_kernel(const __grid_constant__ CUtensorMap tmKb, const __nv_bfloat16* __
         if (lane == 0 && n_tiles > 0) {
             const uint32_t ahi = smem_u32(sm + kOffAhi), alo = smem_u32(sm + kOffAlo);
             bool ok = mbar_wait(&bars.a_ready, 0, ctx);
-            // Seed scores: [128 rows] x [64 seeds], only when the floor is used.
+            // Seed scores: [128 rows] x [128 seeds], only when the floor is used.
             if (ok) ok = mbar_wait(&bars.seed_ready, 0, ctx);
-            if (ok && bars.n_seeds == K) {
+            if (ok && bars.n_seeds == kSeeds) {
                 tc_fence_after();
                 const uint32_t sb = smem_u32(sm + kOffSeedB);
-                const uint32_t id64 = idesc_bf16_f32(128, 64, false, false);
+                const uint32_t idS = idesc_bf16_f32(128, kSeeds, false, false);
                 for (int part = 0; part < 2; ++part) {
                     const uint32_t a = part ? alo : ahi;
 #pragma unroll
                     for (int ks = 0; ks < kD / 16; ++ks)
                         mma_ss(tmem + kColSeed, sdesc_sw128(a + (ks >> 2) * kSub + (ks & 3) * 32, 16, 1024),
-                               sdesc_sw128(sb + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024), id64,
+                               sdesc_sw128(sb + (ks >> 2) * kSub + (ks & 3) * 32, 16, 1024), idS,
                                (part > 0 || ks > 0) ? 1u : 0u);
                 }
             }
@@ -263,191 +264,290 @@ topk_tc_kernel(const __grid_constant__ CUtensorMap tmKb, const __nv_bfloat16* __
         };
         auto stop_now = [&]() { const int v = *sm_stop; return v != 0 && v <= nbar; };
         // (1) group-summed queries -> A (hi, lo), pilot partial sums.  Warp w: rows 16w..16w+15,
-        // lane l: columns 4l..4l+3.
+        // two rows at a time with all their heads' loads in flight; lane l: columns 4l..4l+3.
         {
+            float* ppart = reinterpret_cast<float*>(sm + kOffPPart);
             float pp[4] = {0.f, 0.f, 0.f, 0.f};
             const int sub = lane >> 4, chunk = (lane & 15) >> 1, within = (lane & 1) * 8;
-            for (int rr = 0; rr < 16; ++rr) {
-                const int row = warp * 16 + rr;
-                float a[4] = {0.f, 0.f, 0.f, 0.f};
-                if (row < nrows) {
-                    for (int h = 0; h < G; ++h) {
-                        const uint2 v = *reinterpret_cast<const uint2*>(
-                            q + ((b * H + (int64_t)g * G + h) * Nq + r0 + row) * kD + 4 * lane);
-                        a[0] += __uint_as_float(v.x << 16);
-                        a[1] += __uint_as_float(v.x & 0xffff0000u);
-                        a[2] += __uint_as_float(v.y << 16);
-                        a[3] += __uint_as_float(v.y & 0xffff0000u);
+            for (int rr = 0; rr < 16; rr += 2) {
+                float a[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+                if (G <= kMaxG) {
+                    uint2 v[2][kMaxG];
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const int row = warp * 16 + rr + u;
+#pragma unroll
+                        for (int h = 0; h < kMaxG; ++h)
+                            v[u][h] = (row < nrows && h < G)
+                                          ? *reinterpret_cast<const uint2*>(
+                                                q + ((b * H + (int64_t)g * G + h) * Nq + r0 + row) * kD + 4 * lane)
+                                          : make_uint2(0u, 0u);
+                    }
+#pragma unroll
+                    for (int u = 0; u < 2; ++u)
+#pragma unroll
+                        for (int h = 0; h < kMaxG; ++h) {
+                            a[u][0] += __uint_as_float(v[u][h].x << 16);
+                            a[u][1] += __uint_as_float(v[u][h].x & 0xffff0000u);
+                            a[u][2] += __uint_as_float(v[u][h].y << 16);
+                            a[u][3] += __uint_as_float(v[u][h].y & 0xffff0000u);
+                        }
+                } else {
+                    for (int u = 0; u < 2; ++u) {
+                        const int row = warp * 16 + rr + u;
+                        if (row >= nrows) continue;
+                        for (int h = 0; h < G; ++h) {
+                            const uint2 w2 = *reinterpret_cast<const uint2*>(
+                                q + ((b * H + (int64_t)g * G + h) * Nq + r0 + row) * kD + 4 * lane);
+                            a[u][0] += __uint_as_float(w2.x << 16);
+                            a[u][1] += __uint_as_float(w2.x & 0xffff0000u);
+                            a[u][2] += __uint_as_float(w2.y << 16);
+                            a[u][3] += __uint_as_float(w2.y & 0xffff0000u);
+                        }
                     }
                 }
-                uint32_t hb[2], lb2[2];
 #pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const __nv_bfloat16 h0 = __float2bfloat16_rn(a[2 * e]), h1 = __float2bfloat16_rn(a[2 * e + 1]);
-                    const float r0f = a[2 * e] - __bfloat162float(h0), r1f = a[2 * e + 1] - __bfloat162float(h1);
-                    hb[e] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
-                    lb2[e] = pack_bf16x2(r0f, r1f);
+                for (int u = 0; u < 2; ++u) {
+                    const int row = warp * 16 + rr + u;
+                    uint32_t hb[2], lb2[2];
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const __nv_bfloat16 h0 = __float2bfloat16_rn(a[u][2 * e]), h1 = __float2bfloat16_rn(a[u][2 * e + 1]);
+                        const float d0 = a[u][2 * e] - __bfloat162float(h0), d1 = a[u][2 * e + 1] - __bfloat162float(h1);
+                        hb[e] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
+                        lb2[e] = pack_bf16x2(d0, d1);
+                    }
+                    const int off = sub * kSub + row * 128 + ((chunk ^ (row & 7)) << 4) + within;
+                    *reinterpret_cast<uint2*>(sm + kOffAhi + off) = make_uint2(hb[0], hb[1]);
+                    *reinterpret_cast<uint2*>(sm + kOffAlo + off) = make_uint2(lb2[0], lb2[1]);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) pp[e] += a[u][e];
                 }
-                const int off = sub * kSub + row * 128 + ((chunk ^ (row & 7)) << 4) + within;
-                *reinterpret_cast<uint2*>(sm + kOffAhi + off) = make_uint2(hb[0], hb[1]);
-                *reinterpret_cast<uint2*>(sm + kOffAlo + off) = make_uint2(lb2[0], lb2[1]);
-#pragma unroll
-                for (int e = 0; e < 4; ++e) pp[e] += a[e];
             }
 #pragma unroll
-            for (int e = 0; e < 4; ++e) bars.ppart[warp][4 * lane + e] = pp[e];
+            for (int e = 0; e < 4; ++e) ppart[warp * kD + 4 * lane + e] = pp[e];
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars.a_ready);
         }
         sync_workers();
         if (tid < kD) {
+            const float* ppart = reinterpret_cast<const float*>(sm + kOffPPart);
             float p = 0.f;
 #pragma unroll
-            for (int w = 0; w < 8; ++w) p += bars.ppart[w][tid];
+            for (int w = 0; w < 8; ++w) p += ppart[w * kD + tid];
             bars.pilot[tid] = p;
         }
         sync_workers();
-        // (2) seeds: top-K candidates of [lo, hi_all] by the pilot score (every row may take them).
-        const bool seeded = rank && ncand_all >= K;
+        // (2) seeds: the best kSeeds candidates of [lo, hi_all] by the pilot score (every row may
+        // take them).  Pilot scores of a chunk of candidates (coalesced kbar rows, 8 lanes per row,
+        // eight rows per lane in flight) plus the winners so far, then a radix select.
+        const bool seeded = rank && ncand_all >= kSeeds;
         if (seeded) {
-            uint64_t l0 = 0, l1 = 0;
-            const int nbatch = (ncand_all + 31) / 32;
-            for (int bt = warp; bt < nbatch; bt += 8) {
-                const int blk = lo + bt * 32 + lane;
-                uint64_t key = 0;
-                if (blk <= hi_all) {
-                    const uint4* row = reinterpret_cast<const uint4*>(kbar + (bg * nb + blk) * (int64_t)kD);
-                    float s = 0.f;
-#pragma unroll 4
-                    for (int c = 0; c < kD / 8; ++c) {
-                        const uint4 v = row[c];
-                        const float* pv = bars.pilot + 8 * c;
-                        s = fmaf(pv[0], __uint_as_float(v.x << 16), s);
-                        s = fmaf(pv[1], __uint_as_float(v.x & 0xffff0000u), s);
-                        s = fmaf(pv[2], __uint_as_float(v.y << 16), s);
-                        s = fmaf(pv[3], __uint_as_float(v.y & 0xffff0000u), s);
-                        s = fmaf(pv[4], __uint_as_float(v.z << 16), s);
-                        s = fmaf(pv[5], __uint_as_float(v.z & 0xffff0000u), s);
-                        s = fmaf(pv[6], __uint_as_float(v.w << 16), s);
-                        s = fmaf(pv[7], __uint_as_float(v.w & 0xffff0000u), s);
-                    }
-                    key = sel_key(s, blk);
-                }
-                offer(l0, l1, key, 0ull, K, lane);
-            }
-            uint64_t* pl = reinterpret_cast<uint64_t*>(sm + kOffPList) + warp * kCap;
-            pl[2 * lane] = l0;
-            pl[2 * lane + 1] = l1;
+            uint64_t* pkeys = reinterpret_cast<uint64_t*>(sm + kOffPKeys);
+            if (tid < kSeeds) bars.carry[tid] = 0ull;
             sync_workers();
+            constexpr int kNew = kPilotChunk - kSeeds, kBatch = 8;
+            const int part = lane & 7;
+            const float* pv = bars.pilot + part * 16;
+            for (int cb = 0; cb < ncand_all; cb += kNew) {
+                const int nc = min(kNew, ncand_all - cb);
+                for (int it0 = 0; it0 < nc; it0 += 32 * kBatch) {
+                    uint4 raw[kBatch][2];
 #pragma unroll
-            for (int span = 4; span >= 1; span >>= 1) {
-                if (warp < span) {
-                    uint64_t* pa = reinterpret_cast<uint64_t*>(sm + kOffPList) + warp * kCap;
-                    const uint64_t* pb = reinterpret_cast<const uint64_t*>(sm + kOffPList) + (warp + span) * kCap;
-                    uint64_t a0 = pa[2 * lane], a1 = pa[2 * lane + 1];
-                    merge_desc(a0, a1, pb[2 * lane], pb[2 * lane + 1], lane);
-                    pa[2 * lane] = a0;
-                    pa[2 * lane + 1] = a1;
+                    for (int st = 0; st < kBatch; ++st) {
+                        const int i = it0 + st * 32 + warp * 4 + (lane >> 3);
+                        const uint4* row = reinterpret_cast<const uint4*>(
+                            kbar + (bg * nb + lo + cb + i) * (int64_t)kD + part * 16);
+                        raw[st][0] = i < nc ? row[0] : make_uint4(0u, 0u, 0u, 0u);
+                        raw[st][1] = i < nc ? row[1] : make_uint4(0u, 0u, 0u, 0u);
+                    }
+#pragma unroll
+                    for (int st = 0; st < kBatch; ++st) {
+                        float d0 = 0.f, d1 = 0.f;
+#pragma unroll
+                        for (int u = 0; u < 2; ++u) {
+                            const uint4 v = raw[st][u];
+                            const float* p8 = pv + 8 * u;
+                            d0 = fmaf(p8[0], __uint_as_float(v.x << 16), d0);
+                            d1 = fmaf(p8[1], __uint_as_float(v.x & 0xffff0000u), d1);
+                            d0 = fmaf(p8[2], __uint_as_float(v.y << 16), d0);
+                            d1 = fmaf(p8[3], __uint_as_float(v.y & 0xffff0000u), d1);
+                            d0 = fmaf(p8[4], __uint_as_float(v.z << 16), d0);
+                            d1 = fmaf(p8[5], __uint_as_float(v.z & 0xffff0000u), d1);
+                            d0 = fmaf(p8[6], __uint_as_float(v.w << 16), d0);
+                            d1 = fmaf(p8[7], __uint_as_float(v.w & 0xffff0000u), d1);
+                        }
+                        float d = d0 + d1;
+                        d += __shfl_xor_sync(0xffffffffu, d, 1);
+                        d += __shfl_xor_sync(0xffffffffu, d, 2);
+                        d += __shfl_xor_sync(0xffffffffu, d, 4);
+                        const int i = it0 + st * 32 + warp * 4 + (lane >> 3);
+                        if (part == 0 && i < nc) pkeys[i] = sel_key(d, lo + cb + i);
+                    }
                 }
+                for (int i = nc + tid; i < kNew; i += kWorkers) pkeys[i] = 0ull;
+                if (tid < kSeeds) pkeys[kNew + tid] = bars.carry[tid];
+                sync_workers();
+                uint64_t key[kPilotChunk / kWorkers];
+#pragma unroll
+                for (int e = 0; e < kPilotChunk / kWorkers; ++e) key[e] = pkeys[e * kWorkers + tid];
+                uint64_t prefix, mask;
+                radix_kth<kPilotChunk / kWorkers>(key, kSeeds, bars.rs, prefix, mask, tid, sync_workers);
+                if (tid == 0) bars.n_win = 0;
+                sync_workers();
+#pragma unroll
+                for (int e = 0; e < kPilotChunk / kWorkers; ++e)
+                    if (key[e] && (key[e] & mask) >= prefix) bars.carry[atomicAdd(&bars.n_win, 1)] = key[e];
                 sync_workers();
             }
-            if (warp == 0) {
-                const uint64_t* pl0 = reinterpret_cast<const uint64_t*>(sm + kOffPList);
-                if (2 * lane < K) bars.seeds[2 * lane] = key_block(pl0[2 * lane]);
-                if (2 * lane + 1 < K) bars.seeds[2 * lane + 1] = key_block(pl0[2 * lane + 1]);
-                if (lane == 0) bars.n_seeds = K;
-            }
+            if (tid < kSeeds) bars.seeds[tid] = key_block(bars.carry[tid]);
+            if (tid == 0) bars.n_seeds = kSeeds;
             sync_workers();
-            // seed kbar rows -> B operand (K-major, 128-byte swizzle), zero rows past K
-            for (int e = tid; e < kCap * 16; e += kWorkers) {
-                const int j = e >> 4, cc = e & 15;
-                uint4 v = make_uint4(0, 0, 0, 0);
-                if (j < K) v = reinterpret_cast<const uint4*>(kbar + (bg * nb + bars.seeds[j]) * (int64_t)kD)[cc];
-                const int off = (cc >> 3) * 8192 + j * 128 + (((cc & 7) ^ (j & 7)) << 4);
-                *reinterpret_cast<uint4*>(sm + kOffSeedB + off) = v;
+            // seed kbar rows -> B operand (K-major, 128-byte swizzle); all loads in flight first
+            constexpr int kPer = kSeeds * 16 / kWorkers;
+            uint4 sv[kPer];
+#pragma unroll
+            for (int u = 0; u < kPer; ++u) {
+                const int e = u * kWorkers + tid, j = e >> 4, cc = e & 15;
+                sv[u] = reinterpret_cast<const uint4*>(kbar + (bg * nb + bars.seeds[j]) * (int64_t)kD)[cc];
+            }
+#pragma unroll
+            for (int u = 0; u < kPer; ++u) {
+                const int e = u * kWorkers + tid, j = e >> 4, cc = e & 15;
+                const int off = (cc >> 3) * kSub + j * 128 + (((cc & 7) ^ (j & 7)) << 4);
+                *reinterpret_cast<uint4*>(sm + kOffSeedB + off) = sv[u];
             }
             fence_proxy_async_smem();
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars.seed_ready);
-        // (3) per-row floors from the rows' own seed scores (warps 0-3 read TMEM lanes = rows).
-        if (warp < 4) {
-            uint64_t fk = 0;
-            if (seeded && n_tiles > 0) {
+        // (3) per-row floors: the k-th best of the row's own seed scores.  Warps 0-3 (thread = row)
+        // park the scores in shared memory (the seed operand is consumed by then); each worker warp
+        // then sorts 16 rows' scores.
+        if (seeded && n_tiles > 0) {
+            float* sc = reinterpret_cast<float*>(sm + kOffSeedSc);  // [128][kSeeds + 1]
+            if (warp < 4) {
                 if (!mbar_wait(&bars.seed_done, 0, ctx)) fail();
                 tc_fence_after();
                 if (!__any_sync(0xffffffffu, dead)) {
-                    uint32_t x[64];
                     const uint32_t lb = tmem_lane_base(warp);
-                    tmem_ld32(tmem + lb + kColSeed, *reinterpret_cast<uint32_t(*)[32]>(&x[0]));
-                    tmem_ld32(tmem + lb + kColSeed + 32, *reinterpret_cast<uint32_t(*)[32]>(&x[32]));
-                    tmem_ld_wait();
-                    fk = ~0ull;
+#pragma unroll 1
+                    for (int c = 0; c < kSeeds; c += 32) {
+                        uint32_t x[32];
+                        tmem_ld32(tmem + lb + kColSeed + c, x);
+                        tmem_ld_wait();
 #pragma unroll
-                    for (int j = 0; j < kCap; ++j) {
-                        if (j < K) {
-                            const uint64_t k2 = sel_key(__uint_as_float(x[j]), bars.seeds[j]);
-                            fk = k2 < fk ? k2 : fk;
-                        }
+                        for (int j = 0; j < 32; ++j) sc[tid * (kSeeds + 1) + c + j] = __uint_as_float(x[j]);
                     }
                 }
             }
-            bars.floor_key[tid] = fk;
+            sync_workers();
+            for (int i = 0; i < 16; ++i) {
+                const int row = warp * 16 + i;
+                uint64_t v[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    v[u] = (uint64_t)orderable(sc[row * (kSeeds + 1) + 4 * lane + u]) << 32;
+                sort128_desc(v, lane);
+                const int ii = (K - 1) & 3;
+                const uint64_t mine = ii == 0 ? v[0] : ii == 1 ? v[1] : ii == 2 ? v[2] : v[3];
+                const uint32_t o = (uint32_t)(__shfl_sync(0xffffffffu, mine, (K - 1) >> 2) >> 32);
+                if (lane == 0) bars.floor_s[row] = __uint_as_float((o & 0x80000000u) ? (o & 0x7fffffffu) : ~o);
+            }
+        } else if (tid < kRows) {
+            bars.floor_s[tid] = -INFINITY;
         }
         sync_workers();
         if (stop_now()) dead = true;
-        // (4) main pass
-        uint64_t L0[16], L1[16];
+        // (4) main pass, warps 0-3, thread = query row = TMEM lane: per 32-candidate chunk, the
+        // candidates at or above the row's floor go to the row's buffer.  A row whose buffer would
+        // overflow is first cut back to its best k by its whole warp (the floor rises).
+        if (warp < 4 && n_tiles > 0) {
+            const int row = tid;
+            const int lim = row < nrows ? (r0 + row) / kBlk - n_local : -1;
+            const bool act = lim - lo + 1 > topk;  // this row ranks its candidates
+            float fl = bars.floor_s[row];
+            int n = 0;
+            uint64_t* bufs = reinterpret_cast<uint64_t*>(sm + kOffBuf);
+            uint64_t* buf = bufs + row * kBufCap;
+            const uint32_t lb = tmem_lane_base(warp);
+            auto cut = [&](int src) {  // whole warp: row warp*32 + src back to its best K keys
+                const int nsrc = __shfl_sync(0xffffffffu, n, src);
+                uint64_t* b2 = bufs + (warp * 32 + src) * kBufCap;
+                uint64_t v[4];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) L0[i] = L1[i] = 0ull;
-        bool stop = dead;
-        for (int t = 0; t < n_tiles && !stop; ++t) {
-            const int s = t & 1, r = t >> 1;
-            if (warp < 4) {
+                for (int u = 0; u < 4; ++u) v[u] = 4 * lane + u < nsrc ? b2[4 * lane + u] : 0ull;
+                __syncwarp();
+                sort128_desc(v, lane);
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    if (4 * lane + u < K) b2[4 * lane + u] = v[u];
+                const int ii = (K - 1) & 3;
+                const uint64_t mine = ii == 0 ? v[0] : ii == 1 ? v[1] : ii == 2 ? v[2] : v[3];
+                const uint32_t o = (uint32_t)(__shfl_sync(0xffffffffu, mine, (K - 1) >> 2) >> 32);
+                if (lane == src) {
+                    n = K;
+                    fl = __uint_as_float((o & 0x80000000u) ? (o & 0x7fffffffu) : ~o);
+                }
+                __syncwarp();
+            };
+            for (int t = 0; t < n_tiles; ++t) {
+                const int s = t & 1, r = t >> 1;
                 if (!dead && !mbar_wait(&bars.s_full[s], r & 1, ctx)) fail();
                 tc_fence_after();
                 if (!__any_sync(0xffffffffu, dead)) {
-                    const uint32_t lb = tmem_lane_base(warp);
-                    float* dst = reinterpret_cast<float*>(sm + kOffSC) + tid * kSCStride;
+                    const int j0 = lo + t * kCand;
 #pragma unroll 1
-                    for (int c0 = 0; c0 < kCand; c0 += 32) {
+                    for (int c = 0; c < kCand; c += 32) {
                         uint32_t x[32];
-                        tmem_ld32(tmem + lb + kColS0 + s * kCand + c0, x);
+                        tmem_ld32(tmem + lb + kColS0 + s * kCand + c, x);
                         tmem_ld_wait();
+                        const int jmax = act ? min(32, lim - (j0 + c) + 1) : 0;  // visible candidates
+                        auto passing = [&](uint32_t keep) {
+                            uint32_t m = 0;
 #pragma unroll
-                        for (int j = 0; j < 32; j += 4)
-                            *reinterpret_cast<float4*>(dst + c0 + j) =
-                                make_float4(__uint_as_float(x[j]), __uint_as_float(x[j + 1]),
-                                            __uint_as_float(x[j + 2]), __uint_as_float(x[j + 3]));
+                            for (int j = 0; j < 32; ++j)
+                                m |= (j < jmax && __uint_as_float(x[j]) >= fl) ? (1u << j) : 0u;
+                            return m & keep;
+                        };
+                        auto append = [&](uint32_t m) {
+#pragma unroll
+                            for (int j = 0; j < 32; ++j)
+                                if ((m >> j) & 1u) buf[n++] = sel_key(__uint_as_float(x[j]), j0 + c + j);
+                        };
+                        const uint32_t pass = passing(~0u);
+                        if (__any_sync(0xffffffffu, n + __popc(pass) > kBufCap)) {
+                            // rare: some row would overflow.  Append in two halves of 16, cutting
+                            // the rows that would overflow before each half (a cut leaves k = 64
+                            // keys, so a half always fits afterwards).
+#pragma unroll 1
+                            for (int h = 0; h < 2; ++h) {
+                                const uint32_t half = h ? 0xffff0000u : 0x0000ffffu;
+                                unsigned need = __ballot_sync(0xffffffffu, n + __popc(passing(half)) > kBufCap);
+                                while (need) {
+                                    const int src = __ffs(need) - 1;
+                                    need &= need - 1;
+                                    cut(src);
+                                }
+                                append(passing(half));
+                            }
+                        } else {
+                            append(pass);
+                        }
                     }
                 }
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars.s_free[s]);
             }
-            sync_workers();
-            if (stop_now()) { stop = true; break; }
-            const int j0 = lo + t * kCand;
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const int row = warp * 16 + i;
-                const int lim = row < nrows ? (r0 + row) / kBlk - n_local : -1;
-                if (lim - lo + 1 <= topk) continue;  // row takes every candidate
-                const uint64_t fl = bars.floor_key[row];
-                const float* src = reinterpret_cast<const float*>(sm + kOffSC) + row * kSCStride;
-#pragma unroll
-                for (int qq = 0; qq < kCand / 32; ++qq) {
-                    const int blk = j0 + qq * 32 + lane;
-                    const uint64_t key = blk <= lim ? sel_key(src[qq * 32 + lane], blk) : 0ull;
-                    offer(L0[i], L1[i], key, fl, K, lane);
-                }
-            }
-            sync_workers();
+            bars.buf_n[row] = n;
         }
-        // (5) output rows: init ids, sorted top-k ids, local ids, -1 padding.
-        if (!stop) {
-#pragma unroll
+        sync_workers();
+        // (5) output rows: init ids, sorted top-k ids, local ids, -1 padding.  Warp w: rows
+        // 16w..16w+15; a ranked row's buffer is sorted by the warp and its best k taken.
+        if (!stop_now() && !dead) {
+            const uint64_t* bufs = reinterpret_cast<const uint64_t*>(sm + kOffBuf);
             for (int i = 0; i < 16; ++i) {
                 const int row = warp * 16 + i;
                 if (row >= nrows) continue;
@@ -459,8 +559,19 @@ topk_tc_kernel(const __grid_constant__ CUtensorMap tmKb, const __nv_bfloat16* __
                     for (int s = lane; s < slots; s += 32) out[s] = s <= c ? s : -1;
                     continue;
                 }
-                int x0 = (2 * lane < K && L0[i]) ? key_block(L0[i]) : 0x7fffffff;
-                int x1 = (2 * lane + 1 < K && L1[i]) ? key_block(L1[i]) : 0x7fffffff;
+                const int n = bars.buf_n[row];
+                uint64_t v[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) v[u] = 4 * lane + u < n ? bufs[row * kBufCap + 4 * lane + u] : 0ull;
+                sort128_desc(v, lane);
+                int id[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) id[u] = (4 * lane + u < K && v[u]) ? key_block(v[u]) : 0x7fffffff;
+                // positions 2*lane, 2*lane+1 of the sorted order live in lane (2*lane)/4
+                const int src = (2 * lane) >> 2;
+                const int a0 = __shfl_sync(0xffffffffu, id[0], src), a1 = __shfl_sync(0xffffffffu, id[1], src);
+                const int a2 = __shfl_sync(0xffffffffu, id[2], src), a3 = __shfl_sync(0xffffffffu, id[3], src);
+                int x0 = (lane & 1) ? a2 : a0, x1 = (lane & 1) ? a3 : a1;
                 sort64_asc(x0, x1, lane);
                 for (int s = lane; s < n_init; s += 32) out[s] = s;
                 if (2 * lane < K) out[n_init + 2 * lane] = x0;
@@ -481,7 +592,7 @@ topk_tc_kernel(const __grid_constant__ CUtensorMap tmKb, const __nv_bfloat16* __
 }  // namespace
 
 bool block_topk_tc_supported(int H, int Hkv, int Nq, int q_pos0, int nb, int d, int topk) {
-    (void)H; (void)Hkv;
+    (void)H; (void)Hkv; (void)nb;
     return d == kD && q_pos0 == 0 && Nq > 16 && topk <= kCap;
 }
 

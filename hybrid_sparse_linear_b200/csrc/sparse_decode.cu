@@ -29,6 +29,7 @@
 #include <mutex>
 #include <type_traits>
 
+#include "blocksel.cuh"
 #include "kernels.h"
 
 namespace sala {
@@ -73,85 +74,6 @@ __device__ bool grid_barrier(unsigned* word, unsigned nblocks, const DevCtx& ctx
     }
     __syncthreads();
     return *s_ok != 0;
-}
-
-struct SelSmem {
-    unsigned hist[256];
-    int d, above, eq, n;
-    int nvalid;
-};
-
-// Block-wide: finds the K-th largest nonzero key among the E keys per thread (keys distinct).  On
-// return, winner(key) = key != 0 && (key & mask) >= prefix picks exactly min(K, #nonzero) keys.
-template <int E>
-__device__ void block_kth(const uint64_t (&key)[E], int K, SelSmem& s, uint64_t& prefix,
-                          uint64_t& mask) {
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    int nv = 0;
-#pragma unroll
-    for (int e = 0; e < E; ++e) nv += key[e] != 0ull;
-    if (tid == 0) s.nvalid = 0;
-    __syncthreads();
-    nv = __reduce_add_sync(0xffffffffu, nv);
-    if (lane == 0 && nv) atomicAdd(&s.nvalid, nv);
-    __syncthreads();
-    prefix = 0;
-    mask = 0;
-    if (s.nvalid <= K) {  // every nonzero key wins
-        prefix = 1;
-        mask = ~0ull;
-        return;
-    }
-    int krem = K;
-    for (int shift = 56; shift >= 0; shift -= 8) {
-        s.hist[tid] = 0;
-        __syncthreads();
-        // Keys share their high bytes (nearby scores), so a plain atomic per key would serialize
-        // on one bin: lanes with the same digit add once, through their leader.
-#pragma unroll
-        for (int e = 0; e < E; ++e) {
-            const bool m = key[e] && (key[e] & mask) == prefix;
-            if (!__any_sync(0xffffffffu, m)) continue;
-            const unsigned dig = m ? (unsigned)((key[e] >> shift) & 255u) : 256u;
-            const unsigned peers = __match_any_sync(0xffffffffu, dig);
-            if (m && lane == __ffs(peers) - 1) atomicAdd(&s.hist[dig], (unsigned)__popc(peers));
-        }
-        __syncthreads();
-        if (warp == 0) {
-            // lane l holds bins 255-8l .. 248-8l (descending order)
-            int cnt[8], sum = 0;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                cnt[i] = (int)s.hist[255 - 8 * lane - i];
-                sum += cnt[i];
-            }
-            int incl = sum;
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const int v = __shfl_up_sync(0xffffffffu, incl, off);
-                if (lane >= off) incl += v;
-            }
-            const int excl = incl - sum;
-            if (excl < krem && krem <= incl) {
-                int run = excl;
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    if (run + cnt[i] >= krem) {
-                        s.d = 255 - 8 * lane - i;
-                        s.above = run;
-                        s.eq = cnt[i];
-                        break;
-                    }
-                    run += cnt[i];
-                }
-            }
-        }
-        __syncthreads();
-        krem -= s.above;
-        prefix |= (uint64_t)s.d << shift;
-        mask |= 0xFFull << shift;
-        if (s.eq == krem) break;  // every key with this prefix is a winner
-    }
 }
 
 // Ascending bitonic sort of 64 ints held two per lane (position 2*lane + j).
@@ -236,7 +158,8 @@ struct DecSmem {
     int sel[kMaxSlots];
     int sel_top[kCap];
     uint64_t cand[2 * kThreads];
-    SelSmem ss;
+    RadixSelSmem ss;
+    int sel_n;
     int ok, overflow;
     float cm[8][32], cl[8][32], co[8][32];  // phase D per-warp partials
 };
@@ -391,7 +314,7 @@ sparse_decode_fused_kernel(const T* __restrict__ q, const T* __restrict__ kc,
             const unsigned long long* src =
                 reinterpret_cast<const unsigned long long*>(part) + (int64_t)bg * nspan * kCap;
             if (tid == 0) {
-                sm.ss.n = 0;
+                sm.sel_n = 0;
                 sm.overflow = 0;
             }
             if (nspan * kPre <= 2 * kThreads) {
@@ -422,8 +345,8 @@ sparse_decode_fused_kernel(const T* __restrict__ q, const T* __restrict__ kc,
                     pk[e] = span < nspan ? __ldcg(src + span * kCap + i % kPre) : 0ull;
                 }
                 uint64_t prefix, mask;
-                block_kth<kPreE>(pk, K, sm.ss, prefix, mask);
-                if (tid == 0) sm.ss.n = 0;
+                radix_kth<kPreE>(pk, K, sm.ss, prefix, mask, tid, [] { __syncthreads(); });
+                if (tid == 0) sm.sel_n = 0;
                 __syncthreads();
 #pragma unroll
                 for (int e = 0; e < kPreE; ++e) {
@@ -434,7 +357,7 @@ sparse_decode_fused_kernel(const T* __restrict__ q, const T* __restrict__ kc,
                 if (!sm.overflow) {
 #pragma unroll
                     for (int e = 0; e < kPreE; ++e)
-                        if (pk[e] && (pk[e] & mask) >= prefix) sm.sel_top[atomicAdd(&sm.ss.n, 1)] = key_block(pk[e]);
+                        if (pk[e] && (pk[e] & mask) >= prefix) sm.sel_top[atomicAdd(&sm.sel_n, 1)] = key_block(pk[e]);
                 }
             }
             if (sm.overflow) {
@@ -446,12 +369,12 @@ sparse_decode_fused_kernel(const T* __restrict__ q, const T* __restrict__ kc,
                     const int i = e * kThreads + tid;
                     key[e] = i < nk ? __ldcg(src + i) : 0ull;
                 }
-                block_kth<kMergeE>(key, K, sm.ss, prefix, mask);
-                if (tid == 0) sm.ss.n = 0;
+                radix_kth<kMergeE>(key, K, sm.ss, prefix, mask, tid, [] { __syncthreads(); });
+                if (tid == 0) sm.sel_n = 0;
                 __syncthreads();
 #pragma unroll
                 for (int e = 0; e < kMergeE; ++e)
-                    if (key[e] && (key[e] & mask) >= prefix) sm.sel_top[atomicAdd(&sm.ss.n, 1)] = key_block(key[e]);
+                    if (key[e] && (key[e] & mask) >= prefix) sm.sel_top[atomicAdd(&sm.sel_n, 1)] = key_block(key[e]);
             }
             __syncthreads();
         }

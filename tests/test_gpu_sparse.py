@@ -78,6 +78,22 @@ def test_fp32_d128_pipeline_batch2(sala):
     _pipeline(sala, layer, "f32", 3, 1, 2)
 
 
+@pytest.mark.parametrize("topk", [64, 23])
+def test_bf16_selection_weak_pilot(sala, topk):
+    # Alternate rows negated: the tile's summed query nearly cancels, so the pilot seeds are close to
+    # random and most candidates clear the floor; the row buffers overflow and are cut many times.
+    from hybrid_sparse_linear_b200 import synth
+    layer = synth.sparse_layer(1, 32, 2, 64 * 600 + 40, 128, torch.bfloat16, layer=11, shift_frac=0.05)
+    q = layer.q.clone()
+    q[:, :, 1::2] = -q[:, :, 1::2]
+    kbar = sala.block_compress(layer.k.cuda())
+    idx = sala.block_topk(q.cuda(), kbar, topk, 1, 2)
+    sala.check_status()
+    kbar_ref = _f64(kbar)
+    idx_ref, kth = oracle.block_select(_f64(q), kbar_ref, 64, topk, 1, 2)
+    check_selection(idx.cpu().numpy(), idx_ref, _f64(q), kbar_ref, kth, topk, 1, 2)
+
+
 def test_shifted_blocks_are_selected(sala):
     # Structural invariant on the GPU output: every shifted block that is a candidate is chosen
     # while no more than top-k shifted blocks are causally available.
