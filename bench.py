@@ -67,6 +67,44 @@ def sparse_layer_flops(N: int) -> float:
     return 4.0 * D * H * attended_keys(N)        # QK^T and PV, 2 FLOP per MAC each
 
 
+# DRAM traffic of the sparse prefill kernel (dram__bytes_read.sum + dram__bytes_write.sum) from one
+# ncu capture of the single-layer N = 131072 case, 2.319e9 bytes per launch, scaled by the tokens
+# processed to N = 262144 (Q reads, O writes and the K/V re-reads per 16-token unit all grow with N).
+# Valid only for the kernel source it was taken on: any change to it reports null.
+SPARSE_TRAFFIC = {"bytes_per_token": 2.319232256e9 / 131072,
+                  "sources": {"sparse_tc.cu": "709e3ff2675006fb7cda0f2b626da9884f42750073917bf7e6d29f9a0499e15d",
+                              "fastexp.cuh": "b6d9ae064f35b9fd752ec893180eaf72ade6f0495d57f5699832618f42784c06"}}
+
+
+def sparse_traffic(N: int):
+    import hashlib
+    src = os.path.join(os.path.dirname(os.path.abspath(__file__)), "hybrid_sparse_linear_b200", "csrc")
+    for name, digest in SPARSE_TRAFFIC["sources"].items():
+        try:
+            with open(os.path.join(src, name), "rb") as f:
+                if hashlib.sha256(f.read()).hexdigest() != digest:
+                    return None
+        except OSError:
+            return None
+    return SPARSE_TRAFFIC["bytes_per_token"] * N
+
+
+# Tensor-core work the sparse prefill kernel executes per (8-token tile, block of the union of
+# the tile's 8 selections): S = Q K^T (M128 N64 K128) and O += P V (M128 N128 K64).
+EXEC_FLOPS_PER_TILE_BLOCK = 2.0 * 128 * 64 * 128 * 2
+
+
+def tile_union_blocks(torch, idx, tq: int = 8) -> int:
+    """Sum over 8-token tiles of |union of the tile's selections| (idx [B, Hkv, N, slots], -1 pad)."""
+    B, G, N, S = idx.shape
+    pad = (-N) % tq
+    if pad:
+        idx = torch.cat([idx, idx.new_full((B, G, pad, S), -1)], dim=2)
+    t, _ = torch.sort(idx.reshape(B, G, -1, tq * S), dim=-1)
+    n = ((t[..., 1:] != t[..., :-1]) & (t[..., 1:] >= 0)).sum() + (t[..., 0] >= 0).sum()
+    return int(n.item())
+
+
 def linear_layer_bytes(N: int) -> float:
     return 4.0 * H * N * D * 2                    # read Q, K, V and write O, bf16
 
@@ -267,15 +305,26 @@ def run_prefill(sala, synth, torch, steps, warmup, stream, workload="hybrid_pref
     mean = lambda pairs: sum(a.elapsed_time(b) for a, b in pairs) / max(1, len(pairs))
     res = {"total_ms": total_ms, "launches": launches,
            "sparse_ms": mean(sparse_ev), "linear_ms": mean(linear_ev), "select_ms": mean(topk_ev)}
+    # Executed tensor-core work of the sparse kernel, counted after the timed region from each
+    # sparse layer's selection (recomputed: the timed steps overwrite one shared buffer).
+    union, n_sp = 0, 0
+    with torch.cuda.stream(stream):
+        for kind, q, k, v in layers:
+            if kind == "sparse":
+                sala.block_compress(k, kbar, stream=stream)
+                sala.block_topk(q, kbar, TOPK, N_INIT, N_LOCAL, idx=idx, stream=stream)
+                union += tile_union_blocks(torch, idx)
+                n_sp += 1
+    res["sparse_exec_flops"] = EXEC_FLOPS_PER_TILE_BLOCK * union / max(1, n_sp)
     del layers, out, kbar, idx
     torch.cuda.empty_cache()
     return res
 
 
-def run_decode(sala, synth, torch, steps, warmup, stream):
-    """Decode at a 2^20-token context, 24 linear + 8 sparse layers per token, L2 flushed."""
+def run_decode(sala, synth, torch, steps, warmup, stream, T=DECODE_T):
+    """Decode at a T-token context (2^20 by default), 24 linear + 8 sparse layers per token, L2
+    flushed."""
     dev = torch.device("cuda")
-    T = DECODE_T
     pos = T - 1
     lam = synth.decays(H).to(dev)
     g = torch.Generator(device=dev)
@@ -526,6 +575,8 @@ def main():
     ap.add_argument("--phases", default="prefill,decode,e2e,cpu",
                     help="comma list of prefill,decode,e2e,cpu (default: all)")
     ap.add_argument("--decode-steps", type=int, default=50)
+    ap.add_argument("--decode-t", type=int, default=DECODE_T,
+                    help="decode context length (default 2^20, the benchmark; smaller only for profiles)")
     ap.add_argument("--workload", default="hybrid_prefill_n256k", choices=sorted(WORKLOADS),
                     help="prefill workload (default: the 32-layer hybrid stack at 256K)")
     args = ap.parse_args()
@@ -599,14 +650,18 @@ def main():
         if "sparse" in kinds:
             fl = sparse_layer_flops(n_tok)
             achieved = fl / (pre["sparse_ms"] / 1000.0) / 1e12
+            executed = pre["sparse_exec_flops"] / (pre["sparse_ms"] / 1000.0) / 1e12
             peak = peaks["bf16_tflops_sustained"]
             line["roofline"] = {"kernel": "sparse_prefill_tc_kernel", "bound": "tensor",
                                 "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                                "frac": achieved / peak, "traffic": None,
+                                "frac": achieved / peak, "traffic": sparse_traffic(n_tok),
                                 "peak_source": f"{peaks['source']} bf16 sustained",
                                 "algorithmic_flops_per_launch": fl,
-                                "mean_launch_ms": pre["sparse_ms"]}
-            line["kernels"]["sparse_prefill"] = {"mean_ms": pre["sparse_ms"], "achieved_tflops": achieved}
+                                "mean_launch_ms": pre["sparse_ms"],
+                                "executed_flops_per_launch": pre["sparse_exec_flops"],
+                                "executed_tflops": executed, "executed_frac": executed / peak}
+            line["kernels"]["sparse_prefill"] = {"mean_ms": pre["sparse_ms"], "achieved_tflops": achieved,
+                                                 "executed_tflops": executed}
             line["kernels"]["compress_plus_select"] = {"mean_ms": pre["select_ms"]}
         if "linear" in kinds:
             lin_gbs = linear_layer_bytes(n_tok) / (pre["linear_ms"] / 1000.0) / 1e9
@@ -620,10 +675,11 @@ def main():
                                     "algorithmic_bytes_per_launch": linear_layer_bytes(n_tok),
                                     "mean_launch_ms": pre["linear_ms"]}
     if "decode" in phases:
-        dec = run_decode(sala, synth, torch, args.decode_steps, max(3, args.warmup), stream)
-        db = decode_bytes(DECODE_T)
+        dec = run_decode(sala, synth, torch, args.decode_steps, max(3, args.warmup), stream, args.decode_t)
+        db = decode_bytes(args.decode_t)
         gbs = db["step"] / (dec["us_per_token"] * 1e-6) / 1e9
-        line["decode"] = {"metric": "decode us/token @1M (24 linear + 8 sparse layers)",
+        ctx = "1M" if args.decode_t == DECODE_T else str(args.decode_t)
+        line["decode"] = {"metric": f"decode us/token @{ctx} (24 linear + 8 sparse layers)",
                           "us_per_token": dec["us_per_token"], "us_min": dec["us_min"],
                           "bytes_per_token": db["step"], "achieved_gbs": gbs,
                           "hbm_frac": gbs / peaks["hbm_gbs"],
