@@ -143,10 +143,15 @@ topk_tc_kernel(const __grid_constant__ CUtensorMap tmKb, const __nv_bfloat16* __
     __shared__ Bars bars;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int G = H / Hkv;
-    const int64_t bg = blockIdx.y;
+    // Heaviest tiles first: a tile's work grows with its candidate count, i.e. with its row
+    // index, so the launch order walks row tiles from the last to the first (all groups of one
+    // row tile together) and the lightest tiles fill the tail.
+    const int n_rt = (Nq + kRows - 1) / kRows;
+    const int n_bg = (int)(gridDim.x / n_rt);
+    const int64_t bg = blockIdx.x % n_bg;
     const int64_t b = bg / Hkv;
     const int g = (int)(bg % Hkv);
-    const int r0 = blockIdx.x * kRows;
+    const int r0 = (n_rt - 1 - (int)(blockIdx.x / n_bg)) * kRows;
     const int nrows = min(kRows, Nq - r0);
     const int K = min(topk, kCap);
     // Candidate ranges: rows of the first query block of the tile (c0) and of the second (c0+1).
@@ -613,7 +618,7 @@ cudaError_t launch_block_topk_tc(const void* q, const void* kbar, int32_t* idx, 
         return cudaErrorInvalidValue;
     cudaError_t e = ensure_smem<topk_tc_kernel>(kSmemBytes);
     if (e != cudaSuccess) return e;
-    dim3 grid(ceil_div(Nq, kRows), (unsigned)(B * Hkv));
+    dim3 grid((unsigned)(ceil_div(Nq, kRows) * B * Hkv));
     topk_tc_kernel<<<grid, kThreads, kSmemBytes, st>>>(
         tm, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(kbar), idx, H,
         Hkv, Nq, nb, topk, n_init, n_local, n_init + n_local + topk, ctx);
