@@ -512,14 +512,23 @@ def cpu_baseline(torch, synth, budget_s: float = 20.0):
     cores = oracle.default_threads()
     t_start = time.time()
     # Linear layers: `cores` heads x n_lin tokens (the chunked form is O(N) per head).
-    n_lin = 16384
+    # A pilot of 4096 tokens sizes the sample to about 40 % of the budget (at most the full length).
     hs = min(cores, H)
-    q, k, v = synth.linear_layer(1, hs, n_lin, D, torch.bfloat16, "cpu", layer=0)
     lam = synth.decays(H)[:hs]
     f = oracle.from_tensor
-    t0 = time.perf_counter()
-    oracle.linear_chunked(f(q), f(k), f(v), f(lam), 64, threads=cores)
-    t_lin = time.perf_counter() - t0
+
+    def lin_sample(n):
+        q, k, v = synth.linear_layer(1, hs, n, D, torch.bfloat16, "cpu", layer=0)
+        t0 = time.perf_counter()
+        oracle.linear_chunked(f(q), f(k), f(v), f(lam), 64, threads=cores)
+        return time.perf_counter() - t0
+
+    n_lin = 4096
+    t_lin = lin_sample(n_lin)
+    grow = int(min(N_TOK // n_lin, max(1.0, 0.4 * budget_s / max(t_lin, 1e-6))))
+    if grow > 1:
+        n_lin *= 1 << (grow.bit_length() - 1)
+        t_lin = lin_sample(n_lin)
     lin_layer_s = t_lin * (H / hs) * (N_TOK / n_lin)
     # Sparse layers: selection + attention for sampled query rows spread over the sequence; the
     # attention cost is proportional to the attended keys, the selection cost to the candidates.
@@ -528,21 +537,29 @@ def cpu_baseline(torch, synth, budget_s: float = 20.0):
     q64, k64, v64 = f(sl.q), f(sl.k), f(sl.v)
     kbar = oracle.block_compress(k64, BLOCK)
     rng = np.random.default_rng(0)
-    rows_tok = np.sort(rng.choice(np.arange(n_s // 2, n_s), size=max(2 * cores, 48), replace=False))
-    t0 = time.perf_counter()
-    sel = []
-    for r in rows_tok:
-        ix, _ = oracle.block_select(q64[:, :, r:r + 1], kbar, BLOCK, TOPK, N_INIT, N_LOCAL,
-                                    q_pos0=int(r), threads=1)
-        sel.append(ix)
-    t_sel = time.perf_counter() - t0
-    idx = np.full((1, HKV, n_s, N_INIT + N_LOCAL + TOPK), -1, dtype=np.int32)
-    for r, ix in zip(rows_tok, sel):
-        idx[:, :, r] = ix[:, :, 0]
-    rows = np.array([[h, r] for r in rows_tok for h in range(H)])
-    t0 = time.perf_counter()
-    oracle.sparse_attention(q64, k64, v64, idx, BLOCK, rows=rows, threads=cores)
-    t_att = time.perf_counter() - t0
+
+    def sparse_sample(n_rows):
+        rows_tok = np.sort(rng.choice(np.arange(n_s // 2, n_s), size=n_rows, replace=False))
+        t0 = time.perf_counter()
+        sel = []
+        for r in rows_tok:
+            ix, _ = oracle.block_select(q64[:, :, r:r + 1], kbar, BLOCK, TOPK, N_INIT, N_LOCAL,
+                                        q_pos0=int(r), threads=1)
+            sel.append(ix)
+        t_sel = time.perf_counter() - t0
+        idx = np.full((1, HKV, n_s, N_INIT + N_LOCAL + TOPK), -1, dtype=np.int32)
+        for r, ix in zip(rows_tok, sel):
+            idx[:, :, r] = ix[:, :, 0]
+        rows = np.array([[h, r] for r in rows_tok for h in range(H)])
+        t0 = time.perf_counter()
+        oracle.sparse_attention(q64, k64, v64, idx, BLOCK, rows=rows, threads=cores)
+        return rows_tok, t_sel, time.perf_counter() - t0
+
+    n_rows = max(2 * cores, 32)
+    rows_tok, t_sel, t_att = sparse_sample(n_rows)
+    grow = int(min((n_s // 2) // n_rows, max(1.0, 0.4 * budget_s / max(t_sel + t_att, 1e-6))))
+    if grow > 1:
+        rows_tok, t_sel, t_att = sparse_sample(n_rows * grow)
     # scale: attention by attended keys, selection by candidate count
     keys_sample = 0
     cand_sample = 0
@@ -595,8 +612,10 @@ def main():
                 return
         from hybrid_sparse_linear_b200 import synth
         vals = []
+        # each step a bounded sample, so that the whole arm stays within a few minutes
+        budget = max(5.0, min(20.0, 150.0 / (args.warmup + args.steps)))
         for i in range(args.warmup + args.steps):
-            r = cpu_baseline(torch, synth)
+            r = cpu_baseline(torch, synth, budget)
             if i >= args.warmup:
                 vals.append(r)
         v = statistics.median(x["value"] for x in vals)
