@@ -37,6 +37,7 @@ constexpr int kD = 128, kRows = 128, kCand = 128, kBlk = 64, kCap = 64;
 constexpr int kThreads = 320, kWorkers = 256;
 constexpr int kMaxG = 16;
 constexpr int kBufCap = 88;                            // buffered keys per row
+static_assert(kBufCap <= 96, "keep_best reads three keys per lane");
 constexpr int kSub = 128 * 128;                        // [128 rows x 128 B] = 16 KiB
 constexpr int kOffAhi = 0, kOffAlo = 2 * kSub;         // A operands (hi, lo), 2 sub-tiles each
 constexpr int kOffKb = 4 * kSub;                       // kbar tiles, 2 stages x 2 sub-tiles
@@ -72,65 +73,78 @@ struct Bars {
     RadixSelSmem rs;
 };
 
-// Ascending bitonic sort of 64 ints held two per lane.
-__device__ __forceinline__ void sort64_asc(int& x0, int& x1, int lane) {
-#pragma unroll
-    for (int k = 2; k <= 64; k <<= 1) {
-#pragma unroll
-        for (int s = k >> 1; s > 0; s >>= 1) {
-            if (s == 1) {
-                const bool asc = ((2 * lane) & k) == 0;
-                const int lo = min(x0, x1), hi = max(x0, x1);
-                x0 = asc ? lo : hi;
-                x1 = asc ? hi : lo;
-            } else {
-                const int lm = s >> 1;
-                const int y0 = __shfl_xor_sync(0xffffffffu, x0, lm);
-                const int y1 = __shfl_xor_sync(0xffffffffu, x1, lm);
-                const int p0 = 2 * lane, p1 = 2 * lane + 1;
-                const bool asc0 = (p0 & k) == 0, low0 = (p0 & s) == 0;
-                const bool asc1 = (p1 & k) == 0, low1 = (p1 & s) == 0;
-                x0 = (low0 == asc0) ? min(x0, y0) : max(x0, y0);
-                x1 = (low1 == asc1) ? min(x1, y1) : max(x1, y1);
-            }
-        }
-    }
-}
-
-// Descending bitonic sort of 128 keys held four per lane (element 4*lane + i).
-__device__ __forceinline__ void sort128_desc(uint64_t (&x)[4], int lane) {
+// Descending bitonic sort of R independent 128-element arrays of orderable scores, four per lane
+// (element 4*lane + i).  The R sorts are interleaved so that each one's shuffle latency hides
+// behind the others'.
+template <int R>
+__device__ __forceinline__ void sort128u_desc(uint32_t (&x)[R][4], int lane) {
 #pragma unroll
     for (int kk = 2; kk <= 128; kk <<= 1) {
 #pragma unroll
         for (int jj = kk >> 1; jj > 0; jj >>= 1) {
-            uint64_t y[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-                y[i] = jj < 4 ? x[i ^ jj] : __shfl_xor_sync(0xffffffffu, x[i], jj >> 2);
+            for (int r = 0; r < R; ++r) {
+                uint32_t y[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int e = 4 * lane + i;
-                const bool dsc = (e & kk) == 0, lower = (e & jj) == 0;
-                x[i] = (lower == dsc) ? (x[i] > y[i] ? x[i] : y[i]) : (x[i] < y[i] ? x[i] : y[i]);
+                for (int i = 0; i < 4; ++i)
+                    y[i] = jj < 4 ? x[r][i ^ jj] : __shfl_xor_sync(0xffffffffu, x[r][i], jj >> 2);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int e = 4 * lane + i;
+                    const bool dsc = (e & kk) == 0, lower = (e & jj) == 0;
+                    x[r][i] = (lower == dsc) ? max(x[r][i], y[i]) : min(x[r][i], y[i]);
+                }
             }
         }
     }
 }
 
-// Cuts a full row buffer back to its k best keys (thread-serial; rare with a good floor) and
-// returns the new floor score (that of the k-th key).
-__device__ __forceinline__ float cut_buffer(uint64_t* buf, int n, int K) {
-    for (int i = 1; i < n; ++i) {  // insertion sort, descending
-        const uint64_t v = buf[i];
-        int j = i - 1;
-        while (j >= 0 && buf[j] < v) {
-            buf[j + 1] = buf[j];
-            --j;
-        }
-        buf[j + 1] = v;
-    }
-    const uint32_t o = (uint32_t)(buf[K - 1] >> 32);  // orderable score of the k-th key
+// Element `pos` of a sorted 128-element array held four per lane (every lane gets it).
+__device__ __forceinline__ uint32_t sorted_at(const uint32_t (&x)[4], int pos) {
+    const int ii = pos & 3;
+    const uint32_t mine = ii == 0 ? x[0] : ii == 1 ? x[1] : ii == 2 ? x[2] : x[3];
+    return __shfl_sync(0xffffffffu, mine, pos >> 2);
+}
+
+__device__ __forceinline__ float from_orderable(uint32_t o) {
     return __uint_as_float((o & 0x80000000u) ? (o & 0x7fffffffu) : ~o);
+}
+
+// The K best keys of a row buffer of n keys (n <= 96), in buffer order: those whose orderable
+// score beats s_k (the K-th best score), then the first K - #beating of those that tie with it.
+// Buffers are appended in ascending block order, so "first" is "lowest block", the tie rule of
+// the keys.  One warp; emit(pos, key) is called for the kept keys, pos = 0 .. kept-1 in order;
+// returns the number kept.  All reads happen before the first emit, so emit may write the
+// buffer in place.
+template <typename Emit>
+__device__ __forceinline__ int keep_best(const uint64_t* buf, int n, int K, uint32_t s_k, int lane,
+                                         Emit emit) {
+    uint64_t key[3];
+    bool gt[3], eq[3];
+    int n_gt = 0;
+#pragma unroll
+    for (int j = 0; j < 3; ++j) {
+        const int p = lane + 32 * j;
+        key[j] = p < n ? buf[p] : 0ull;
+        const uint32_t o = (uint32_t)(key[j] >> 32);
+        gt[j] = p < n && o > s_k;
+        eq[j] = p < n && o == s_k;
+        n_gt += __popc(__ballot_sync(0xffffffffu, gt[j]));
+    }
+    __syncwarp();
+    const int need = K - n_gt;
+    const unsigned below = (1u << lane) - 1u;
+    int base = 0, eq_base = 0;
+#pragma unroll
+    for (int j = 0; j < 3; ++j) {
+        const unsigned ue = __ballot_sync(0xffffffffu, eq[j]);
+        const bool take = gt[j] || (eq[j] && eq_base + __popc(ue & below) < need);
+        const unsigned ut = __ballot_sync(0xffffffffu, take);
+        if (take) emit(base + __popc(ut & below), key[j]);
+        base += __popc(ut);
+        eq_base += __popc(ue);
+    }
+    return base;
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -185,6 +199,7 @@ topk_tc_kernel(const __grid_constant__ CUtensorMap tmKb, const __nv_bfloat16* __
         bars.n_seeds = 0;
         fence_mbar_init();
     }
+    if (tid < kRows) bars.buf_n[tid] = 0;
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -448,17 +463,20 @@ topk_tc_kernel(const __grid_constant__ CUtensorMap tmKb, const __nv_bfloat16* __
                 }
             }
             sync_workers();
-            for (int i = 0; i < 16; ++i) {
-                const int row = warp * 16 + i;
-                uint64_t v[4];
+#pragma unroll 1
+            for (int i = 0; i < 16; i += 4) {
+                uint32_t v[4][4];
 #pragma unroll
-                for (int u = 0; u < 4; ++u)
-                    v[u] = (uint64_t)orderable(sc[row * (kSeeds + 1) + 4 * lane + u]) << 32;
-                sort128_desc(v, lane);
-                const int ii = (K - 1) & 3;
-                const uint64_t mine = ii == 0 ? v[0] : ii == 1 ? v[1] : ii == 2 ? v[2] : v[3];
-                const uint32_t o = (uint32_t)(__shfl_sync(0xffffffffu, mine, (K - 1) >> 2) >> 32);
-                if (lane == 0) bars.floor_s[row] = __uint_as_float((o & 0x80000000u) ? (o & 0x7fffffffu) : ~o);
+                for (int r = 0; r < 4; ++r)
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        v[r][u] = orderable(sc[(warp * 16 + i + r) * (kSeeds + 1) + 4 * lane + u]);
+                sort128u_desc<4>(v, lane);
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    const uint32_t o = sorted_at(v[r], K - 1);
+                    if (lane == 0) bars.floor_s[warp * 16 + i + r] = from_orderable(o);
+                }
             }
         } else if (tid < kRows) {
             bars.floor_s[tid] = -INFINITY;
@@ -480,22 +498,63 @@ topk_tc_kernel(const __grid_constant__ CUtensorMap tmKb, const __nv_bfloat16* __
             auto cut = [&](int src) {  // whole warp: row warp*32 + src back to its best K keys
                 const int nsrc = __shfl_sync(0xffffffffu, n, src);
                 uint64_t* b2 = bufs + (warp * 32 + src) * kBufCap;
-                uint64_t v[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) v[u] = 4 * lane + u < nsrc ? b2[4 * lane + u] : 0ull;
-                __syncwarp();
-                sort128_desc(v, lane);
+                uint32_t v[1][4];
 #pragma unroll
                 for (int u = 0; u < 4; ++u)
-                    if (4 * lane + u < K) b2[4 * lane + u] = v[u];
-                const int ii = (K - 1) & 3;
-                const uint64_t mine = ii == 0 ? v[0] : ii == 1 ? v[1] : ii == 2 ? v[2] : v[3];
-                const uint32_t o = (uint32_t)(__shfl_sync(0xffffffffu, mine, (K - 1) >> 2) >> 32);
+                    v[0][u] = 4 * lane + u < nsrc ? (uint32_t)(b2[4 * lane + u] >> 32) : 0u;
+                sort128u_desc<1>(v, lane);
+                const uint32_t s_k = sorted_at(v[0], K - 1);
+                keep_best(b2, nsrc, K, s_k, lane, [&](int pos, uint64_t key) { b2[pos] = key; });
+                __syncwarp();
                 if (lane == src) {
                     n = K;
-                    fl = __uint_as_float((o & 0x80000000u) ? (o & 0x7fffffffu) : ~o);
+                    fl = from_orderable(s_k);
                 }
-                __syncwarp();
+            };
+            // One 32-candidate chunk of this row's scores (candidates jb .. jb + 31).
+            // Whether any row of the warp has a visible candidate of the chunk at or above its floor.
+            auto worth = [&](const uint32_t (&x)[32], int jb) {
+                float m[8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    m[k] = fmax3(__uint_as_float(x[4 * k]), __uint_as_float(x[4 * k + 1]),
+                                 fmaxf(__uint_as_float(x[4 * k + 2]), __uint_as_float(x[4 * k + 3])));
+                const float mx = fmax3(fmax3(m[0], m[1], m[2]), fmax3(m[3], m[4], m[5]), fmaxf(m[6], m[7]));
+                return __any_sync(0xffffffffu, act && lim >= jb && mx >= fl);
+            };
+            auto filter = [&](const uint32_t (&x)[32], int jb) {
+                const int jmax = act ? min(32, lim - jb + 1) : 0;  // visible candidates
+                auto passing = [&](uint32_t keep) {
+                    uint32_t msk = 0;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        msk |= (j < jmax && __uint_as_float(x[j]) >= fl) ? (1u << j) : 0u;
+                    return msk & keep;
+                };
+                auto append = [&](uint32_t msk) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        if ((msk >> j) & 1u) buf[n++] = sel_key(__uint_as_float(x[j]), jb + j);
+                };
+                const uint32_t pass = passing(~0u);
+                if (__any_sync(0xffffffffu, n + __popc(pass) > kBufCap)) {
+                    // rare: some row would overflow.  Append in two halves of 16, cutting the
+                    // rows that would overflow before each half (a cut leaves k <= 64 keys, so a
+                    // half always fits afterwards).
+#pragma unroll 1
+                    for (int h = 0; h < 2; ++h) {
+                        const uint32_t half = h ? 0xffff0000u : 0x0000ffffu;
+                        unsigned need = __ballot_sync(0xffffffffu, n + __popc(passing(half)) > kBufCap);
+                        while (need) {
+                            const int src = __ffs(need) - 1;
+                            need &= need - 1;
+                            cut(src);
+                        }
+                        append(passing(half));
+                    }
+                } else {
+                    append(pass);
+                }
             };
             for (int t = 0; t < n_tiles; ++t) {
                 const int s = t & 1, r = t >> 1;
@@ -504,41 +563,25 @@ topk_tc_kernel(const __grid_constant__ CUtensorMap tmKb, const __nv_bfloat16* __
                 if (!__any_sync(0xffffffffu, dead)) {
                     const int j0 = lo + t * kCand;
 #pragma unroll 1
-                    for (int c = 0; c < kCand; c += 32) {
-                        uint32_t x[32];
-                        tmem_ld32(tmem + lb + kColS0 + s * kCand + c, x);
+                    for (int c = 0; c < kCand; c += 64) {
+                        // 64 columns per TMEM round trip; most chunks have nothing at or above
+                        // the floors.  The second chunk is loaded again after the first one's
+                        // filter, so that it is not held across it.
+                        const uint32_t col = tmem + lb + kColS0 + s * kCand + c;
+                        uint32_t xa[32], xb[32];
+                        tmem_ld32(col, xa);
+                        tmem_ld32(col + 32, xb);
                         tmem_ld_wait();
-                        const int jmax = act ? min(32, lim - (j0 + c) + 1) : 0;  // visible candidates
-                        auto passing = [&](uint32_t keep) {
-                            uint32_t m = 0;
-#pragma unroll
-                            for (int j = 0; j < 32; ++j)
-                                m |= (j < jmax && __uint_as_float(x[j]) >= fl) ? (1u << j) : 0u;
-                            return m & keep;
-                        };
-                        auto append = [&](uint32_t m) {
-#pragma unroll
-                            for (int j = 0; j < 32; ++j)
-                                if ((m >> j) & 1u) buf[n++] = sel_key(__uint_as_float(x[j]), j0 + c + j);
-                        };
-                        const uint32_t pass = passing(~0u);
-                        if (__any_sync(0xffffffffu, n + __popc(pass) > kBufCap)) {
-                            // rare: some row would overflow.  Append in two halves of 16, cutting
-                            // the rows that would overflow before each half (a cut leaves k = 64
-                            // keys, so a half always fits afterwards).
-#pragma unroll 1
-                            for (int h = 0; h < 2; ++h) {
-                                const uint32_t half = h ? 0xffff0000u : 0x0000ffffu;
-                                unsigned need = __ballot_sync(0xffffffffu, n + __popc(passing(half)) > kBufCap);
-                                while (need) {
-                                    const int src = __ffs(need) - 1;
-                                    need &= need - 1;
-                                    cut(src);
-                                }
-                                append(passing(half));
+                        const bool wa = worth(xa, j0 + c), wb = worth(xb, j0 + c + 32);
+                        if (wa) {
+                            filter(xa, j0 + c);
+                            if (wb) {
+                                tmem_ld32(col + 32, xb);
+                                tmem_ld_wait();
+                                filter(xb, j0 + c + 32);
                             }
-                        } else {
-                            append(pass);
+                        } else if (wb) {
+                            filter(xb, j0 + c + 32);
                         }
                     }
                 }
@@ -549,40 +592,44 @@ topk_tc_kernel(const __grid_constant__ CUtensorMap tmKb, const __nv_bfloat16* __
             bars.buf_n[row] = n;
         }
         sync_workers();
-        // (5) output rows: init ids, sorted top-k ids, local ids, -1 padding.  Warp w: rows
-        // 16w..16w+15; a ranked row's buffer is sorted by the warp and its best k taken.
+        // (5) output rows: init ids, the top-k ids in ascending order, local ids, -1 padding.
+        // Warp w: rows 16w..16w+15, four at a time; a ranked row's k-th best score comes from a
+        // sort of its buffer's scores, and its best k keys are taken in buffer (= block) order.
         if (!stop_now() && !dead) {
             const uint64_t* bufs = reinterpret_cast<const uint64_t*>(sm + kOffBuf);
-            for (int i = 0; i < 16; ++i) {
-                const int row = warp * 16 + i;
-                if (row >= nrows) continue;
-                const int rq = r0 + row;
-                const int c = rq / kBlk;
-                const int ncand = c - n_local - n_init + 1;
-                int32_t* out = idx + (bg * Nq + rq) * (int64_t)slots;
-                if (ncand <= topk) {
-                    for (int s = lane; s < slots; s += 32) out[s] = s <= c ? s : -1;
-                    continue;
+#pragma unroll 1
+            for (int i = 0; i < 16; i += 4) {
+                uint32_t v[4][4];
+                int nr[4];
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    const int row = warp * 16 + i + r;
+                    const bool ranked = row < nrows && (r0 + row) / kBlk - n_local - n_init + 1 > topk;
+                    nr[r] = ranked ? min(bars.buf_n[row], kBufCap) : 0;
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        v[r][u] = 4 * lane + u < nr[r] ? (uint32_t)(bufs[row * kBufCap + 4 * lane + u] >> 32) : 0u;
                 }
-                const int n = bars.buf_n[row];
-                uint64_t v[4];
+                sort128u_desc<4>(v, lane);
 #pragma unroll
-                for (int u = 0; u < 4; ++u) v[u] = 4 * lane + u < n ? bufs[row * kBufCap + 4 * lane + u] : 0ull;
-                sort128_desc(v, lane);
-                int id[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) id[u] = (4 * lane + u < K && v[u]) ? key_block(v[u]) : 0x7fffffff;
-                // positions 2*lane, 2*lane+1 of the sorted order live in lane (2*lane)/4
-                const int src = (2 * lane) >> 2;
-                const int a0 = __shfl_sync(0xffffffffu, id[0], src), a1 = __shfl_sync(0xffffffffu, id[1], src);
-                const int a2 = __shfl_sync(0xffffffffu, id[2], src), a3 = __shfl_sync(0xffffffffu, id[3], src);
-                int x0 = (lane & 1) ? a2 : a0, x1 = (lane & 1) ? a3 : a1;
-                sort64_asc(x0, x1, lane);
-                for (int s = lane; s < n_init; s += 32) out[s] = s;
-                if (2 * lane < K) out[n_init + 2 * lane] = x0;
-                if (2 * lane + 1 < K) out[n_init + 2 * lane + 1] = x1;
-                for (int u = lane; u < n_local; u += 32) out[n_init + K + u] = c - n_local + 1 + u;
-                for (int s = n_init + K + n_local + lane; s < slots; s += 32) out[s] = -1;
+                for (int r = 0; r < 4; ++r) {
+                    const int row = warp * 16 + i + r;
+                    if (row >= nrows) continue;
+                    const int rq = r0 + row;
+                    const int c = rq / kBlk;
+                    int32_t* out = idx + (bg * Nq + rq) * (int64_t)slots;
+                    if (c - n_local - n_init + 1 <= topk) {
+                        for (int sl = lane; sl < slots; sl += 32) out[sl] = sl <= c ? sl : -1;
+                        continue;
+                    }
+                    const uint32_t s_k = sorted_at(v[r], K - 1);
+                    const int kept = keep_best(bufs + row * kBufCap, nr[r], K, s_k, lane,
+                                               [&](int pos, uint64_t key) { out[n_init + pos] = key_block(key); });
+                    for (int u = kept + lane; u < K; u += 32) out[n_init + u] = -1;  // unreachable: >= k kept
+                    for (int sl = lane; sl < n_init; sl += 32) out[sl] = sl;
+                    for (int u = lane; u < n_local; u += 32) out[n_init + K + u] = c - n_local + 1 + u;
+                    for (int sl = n_init + K + n_local + lane; sl < slots; sl += 32) out[sl] = -1;
+                }
             }
         }
     }
@@ -598,7 +645,7 @@ topk_tc_kernel(const __grid_constant__ CUtensorMap tmKb, const __nv_bfloat16* __
 
 bool block_topk_tc_supported(int H, int Hkv, int Nq, int q_pos0, int nb, int d, int topk) {
     (void)H; (void)Hkv; (void)nb;
-    return d == kD && q_pos0 == 0 && Nq > 16 && topk <= kCap;
+    return d == kD && q_pos0 == 0 && Nq > 16 && topk >= 1 && topk <= kCap;
 }
 
 cudaError_t launch_block_topk_tc(const void* q, const void* kbar, int32_t* idx, int B, int H,

@@ -51,7 +51,7 @@ def test_tiny_fp32_pipeline(sala):
 
 
 @pytest.mark.parametrize("N,topk,n_local", [(64 * 70 + 17, 8, 2), (64 * 40, 64, 2), (64 * 9, 3, 1),
-                                             (100, 4, 2), (64 * 300, 16, 2)])
+                                             (100, 4, 2), (64 * 300, 16, 2), (64 * 20 + 5, 0, 2)])
 def test_bf16_pipeline_gqa16(sala, N, topk, n_local):
     from hybrid_sparse_linear_b200 import synth
     layer = synth.sparse_layer(1, 32, 2, N, 128, torch.bfloat16, layer=2, shift_frac=0.05)
