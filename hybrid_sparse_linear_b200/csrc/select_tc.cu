@@ -9,15 +9,17 @@
 // Floor: the pilot vector p = sum_r qbar_r ranks the candidates that every row of the tile may
 // take; its best 2k become seeds.  Row r's k-th best score is at least the k-th best of its own
 // seed scores (k real candidates reach it), so a candidate scoring below that floor can never
-// enter row r's top-k.  The seeds only decide how much work is skipped, never the result: the
-// selection is exact.
+// enter row r's top-k (the floor kept is that score rounded down to 16 bits of its orderable
+// form, a lower bound as well).  The seeds only decide how much work is skipped, never the
+// result: the selection is exact.
 //
 // Main pass, per 128-candidate tile: MMA (2 x 8 K-steps, N = 128) -> TMEM (double-buffered) ->
 // one thread per query row reads its 128 scores straight from TMEM, compares each with the row's
-// floor, and appends the few that pass to the row's buffer in shared memory.  A full buffer is
-// cut back to its best k (the floor rises to the k-th); at the end each row's buffer is sorted
-// (one warp per row) and the best k taken.  Key = (orderable score, ~block), so ties go to the
-// lower block index.  Output as the CUDA-core path: init ids, sorted top-k ids, local ids.
+// floor, and appends the few that pass to the row's buffer in shared memory, in ascending block
+// order.  A full buffer is cut back to its best k, order kept (the floor rises to the k-th
+// score); at the end each row's k-th best score is found by a bitwise select and the best k keys
+// are taken in buffer order.  Key = (orderable score, ~block), so ties go to the lower block
+// index.  Output as the CUDA-core path: init ids, top-k ids ascending, local ids.
 //
 // Roles (320 threads): warps 0-7 workers (the main pass runs on warps 0-3, thread = row = TMEM
 // lane), warp 8 TMA producer (kbar tiles), warp 9 TMEM owner and MMA issuer.  Every wait is
@@ -73,37 +75,26 @@ struct Bars {
     RadixSelSmem rs;
 };
 
-// Descending bitonic sort of R independent 128-element arrays of orderable scores, four per lane
-// (element 4*lane + i).  The R sorts are interleaved so that each one's shuffle latency hides
-// behind the others'.
-template <int R>
-__device__ __forceinline__ void sort128u_desc(uint32_t (&x)[R][4], int lane) {
+// K-th largest of R independent arrays of up to 128 orderable scores held four per lane (0 marks
+// an empty slot; every array holds at least K scores), returned to every lane: the largest t with
+// #(x >= t) >= K, decided one bit at a time from the top, one warp-wide count per bit.  The R rows
+// are interleaved so that each one's reduction latency hides behind the others'.  With kBits < 32
+// the low 32 - kBits bits of t stay zero: t is then the K-th largest with those bits cleared, a
+// lower bound of it (all a floor needs).
+template <int R, int kBits>
+__device__ __forceinline__ void kth_largest(const uint32_t (&x)[R][4], int K, uint32_t (&t)[R]) {
 #pragma unroll
-    for (int kk = 2; kk <= 128; kk <<= 1) {
+    for (int r = 0; r < R; ++r) t[r] = 0u;
+#pragma unroll 4
+    for (int bit = 31; bit >= 32 - kBits; --bit) {
 #pragma unroll
-        for (int jj = kk >> 1; jj > 0; jj >>= 1) {
-#pragma unroll
-            for (int r = 0; r < R; ++r) {
-                uint32_t y[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    y[i] = jj < 4 ? x[r][i ^ jj] : __shfl_xor_sync(0xffffffffu, x[r][i], jj >> 2);
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int e = 4 * lane + i;
-                    const bool dsc = (e & kk) == 0, lower = (e & jj) == 0;
-                    x[r][i] = (lower == dsc) ? max(x[r][i], y[i]) : min(x[r][i], y[i]);
-                }
-            }
+        for (int r = 0; r < R; ++r) {
+            const uint32_t c = t[r] | (1u << bit);
+            const int cnt = __reduce_add_sync(0xffffffffu, (int)(x[r][0] >= c) + (int)(x[r][1] >= c) +
+                                                               (int)(x[r][2] >= c) + (int)(x[r][3] >= c));
+            t[r] = cnt >= K ? c : t[r];
         }
     }
-}
-
-// Element `pos` of a sorted 128-element array held four per lane (every lane gets it).
-__device__ __forceinline__ uint32_t sorted_at(const uint32_t (&x)[4], int pos) {
-    const int ii = pos & 3;
-    const uint32_t mine = ii == 0 ? x[0] : ii == 1 ? x[1] : ii == 2 ? x[2] : x[3];
-    return __shfl_sync(0xffffffffu, mine, pos >> 2);
 }
 
 __device__ __forceinline__ float from_orderable(uint32_t o) {
@@ -471,12 +462,11 @@ topk_tc_kernel(const __grid_constant__ CUtensorMap tmKb, const __nv_bfloat16* __
 #pragma unroll
                     for (int u = 0; u < 4; ++u)
                         v[r][u] = orderable(sc[(warp * 16 + i + r) * (kSeeds + 1) + 4 * lane + u]);
-                sort128u_desc<4>(v, lane);
+                uint32_t t[4];
+                kth_largest<4, 16>(v, K, t);
 #pragma unroll
-                for (int r = 0; r < 4; ++r) {
-                    const uint32_t o = sorted_at(v[r], K - 1);
-                    if (lane == 0) bars.floor_s[warp * 16 + i + r] = from_orderable(o);
-                }
+                for (int r = 0; r < 4; ++r)
+                    if (lane == 0) bars.floor_s[warp * 16 + i + r] = from_orderable(t[r]);
             }
         } else if (tid < kRows) {
             bars.floor_s[tid] = -INFINITY;
@@ -502,8 +492,9 @@ topk_tc_kernel(const __grid_constant__ CUtensorMap tmKb, const __nv_bfloat16* __
 #pragma unroll
                 for (int u = 0; u < 4; ++u)
                     v[0][u] = 4 * lane + u < nsrc ? (uint32_t)(b2[4 * lane + u] >> 32) : 0u;
-                sort128u_desc<1>(v, lane);
-                const uint32_t s_k = sorted_at(v[0], K - 1);
+                uint32_t t[1];
+                kth_largest<1, 32>(v, K, t);
+                const uint32_t s_k = t[0];
                 keep_best(b2, nsrc, K, s_k, lane, [&](int pos, uint64_t key) { b2[pos] = key; });
                 __syncwarp();
                 if (lane == src) {
@@ -594,7 +585,8 @@ topk_tc_kernel(const __grid_constant__ CUtensorMap tmKb, const __nv_bfloat16* __
         sync_workers();
         // (5) output rows: init ids, the top-k ids in ascending order, local ids, -1 padding.
         // Warp w: rows 16w..16w+15, four at a time; a ranked row's k-th best score comes from a
-        // sort of its buffer's scores, and its best k keys are taken in buffer (= block) order.
+        // bitwise select over its buffer's scores, and its best k keys are taken in buffer (=
+        // block) order.
         if (!stop_now() && !dead) {
             const uint64_t* bufs = reinterpret_cast<const uint64_t*>(sm + kOffBuf);
 #pragma unroll 1
@@ -610,7 +602,8 @@ topk_tc_kernel(const __grid_constant__ CUtensorMap tmKb, const __nv_bfloat16* __
                     for (int u = 0; u < 4; ++u)
                         v[r][u] = 4 * lane + u < nr[r] ? (uint32_t)(bufs[row * kBufCap + 4 * lane + u] >> 32) : 0u;
                 }
-                sort128u_desc<4>(v, lane);
+                uint32_t kth[4];
+                kth_largest<4, 32>(v, K, kth);
 #pragma unroll
                 for (int r = 0; r < 4; ++r) {
                     const int row = warp * 16 + i + r;
@@ -622,7 +615,7 @@ topk_tc_kernel(const __grid_constant__ CUtensorMap tmKb, const __nv_bfloat16* __
                         for (int sl = lane; sl < slots; sl += 32) out[sl] = sl <= c ? sl : -1;
                         continue;
                     }
-                    const uint32_t s_k = sorted_at(v[r], K - 1);
+                    const uint32_t s_k = kth[r];
                     const int kept = keep_best(bufs + row * kBufCap, nr[r], K, s_k, lane,
                                                [&](int pos, uint64_t key) { out[n_init + pos] = key_block(key); });
                     for (int u = kept + lane; u < K; u += 32) out[n_init + u] = -1;  // unreachable: >= k kept
