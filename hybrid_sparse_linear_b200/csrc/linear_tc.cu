@@ -18,15 +18,17 @@
 //   EPI-S S    = lambda^len S + dS            fp32, one row of S per thread, in registers
 // The only serial dependency between tiles is the state: S(c) = lambda^len S(c-1) + dS(c), where
 // dS(c) needs no state at all.  The MMA issuer therefore computes dS one tile ahead (into a second
-// TMEM buffer): per tile it issues MMA3(c), MMA2(c) -- the last reader of stage c, which is then
-// released to the producer a full tile before it is needed again -- and MMA1(c+1), MMA4(c+1), so
-// the state warps find dS(c) already done and the tensor core always has independent work queued.
+// TMEM buffer): per tile, one thread issues MMA2(c) then MMA1(c+1) and the other MMA3(c) then
+// MMA4(c+1); after MMA2(c) and MMA3(c), the last readers of stage c, the stage goes back to the
+// producer a full tile before it is needed again, the state warps find dS(c) already done and the
+// tensor core always has independent work queued.
 // The bf16 state copy is double-buffered: Sb(c) lives in buffer (c+1)&1, MMA3(c) reads Sb(c-1)
 // from buffer c&1 and releases it through sb_free[c&1]; with one barrier per buffer no barrier
 // can run two phases ahead of its waiter.
-// Roles (320 threads): warps 0-3 "EPI-A" (mask + output, thread = row = TMEM lane), warps 4-7
+// Roles (352 threads): warps 0-3 "EPI-A" (mask + output, thread = row = TMEM lane), warps 4-7
 // "EPI-S" (V~ + state, thread = row of S), warp 8 TMA producer (2-stage ring of Q/K/V tiles),
-// warp 9 TMEM owner and MMA issuer.  Every wait is bounded (see ptx::mbar_wait).
+// warp 9 TMEM owner and issuer of MMA1/MMA2, warp 10 issuer of MMA3/MMA4 (one issuing thread
+// cannot keep four products per tile in flight).  Every wait is bounded (see ptx::mbar_wait).
 #include "kernels.h"
 #include "ptx.cuh"
 #include "tmap.cuh"
@@ -37,13 +39,15 @@ namespace {
 using namespace ptx;
 
 constexpr int kD = 128, kC = 128, kDv = 64, kSlices = kD / kDv;
-constexpr int kThreads = 320;
+constexpr int kThreads = 352;
 constexpr int kSub = kC * 128;                    // one [128 rows x 128 B] sub-tile: 16 KiB
 constexpr int kOffQ = 0, kOffK = 2 * kSub, kOffV = 4 * kSub;
 constexpr int kStageBytes = 5 * kSub;             // Q (2) + K (2) + V slice (1)
-constexpr int kOffVt = 2 * kStageBytes;           // V~ (decay-weighted V slice), 2 buffers
-constexpr int kOffSb = kOffVt + 2 * kSub;         // bf16 copies of the state slice, 2 buffers
-constexpr int kSmemBytes = kOffSb + 2 * kSub + 1024;
+constexpr int kOffVt = 2 * kStageBytes;           // V~ (decay-weighted V slice)
+constexpr int kOffSb = kOffVt + kSub;             // bf16 copies of the state slice, 2 buffers
+constexpr int kOffOst = kOffSb + 2 * kSub;        // output tile staged for its TMA store
+constexpr int kSmemBytes = kOffOst + kSub + 1024;
+static_assert(kSmemBytes <= 227 * 1024, "descriptor address fields (14 bits of 16-byte units) must not carry");
 
 constexpr uint32_t kColA0 = 0, kColO1 = 256, kColO2 = 320, kColDS = 384, kTmemCols = 512;  // dS: 2 x 64
 
@@ -72,8 +76,9 @@ __device__ __forceinline__ float bf_hi(uint32_t x) { return __uint_as_float(x & 
 __global__ void __launch_bounds__(kThreads, 1)
 linear_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                          const __grid_constant__ CUtensorMap tmK,
-                         const __grid_constant__ CUtensorMap tmV, const float* __restrict__ decay,
-                         __nv_bfloat16* __restrict__ out, const float* s_in, float* s_out, int H,
+                         const __grid_constant__ CUtensorMap tmV,
+                         const __grid_constant__ CUtensorMap tmO, const float* __restrict__ decay,
+                         const float* s_in, float* s_out, int H,
                          int N, int seg_len, int n_seg, int64_t s_in_seg_stride, DevCtx ctx) {
     extern __shared__ uint8_t smraw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smraw) + 1023) &
@@ -98,7 +103,7 @@ linear_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
     if (tid == 0) {
         for (int b = 0; b < 2; ++b) {
             mbar_init(&bars.full[b], 1);
-            mbar_init(&bars.empty[b], 1);
+            mbar_init(&bars.empty[b], 2);   // one commit per issuer
             mbar_init(&bars.qk_done[b], 1);
             mbar_init(&bars.a_ready[b], 4);
             mbar_init(&bars.v_ready[b], 4);
@@ -106,9 +111,9 @@ linear_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
             mbar_init(&bars.s_ready[b], 4);
             mbar_init(&bars.sb_free[b], 1);
         }
-        mbar_init(&bars.o_done, 1);
+        mbar_init(&bars.o_done, 2);  // O1 (warp 9) and O2 (warp 10)
         mbar_init(&bars.o_free, 4);
-        mbar_init(&bars.fin, 1);
+        mbar_init(&bars.fin, 2);
         bars.abort = 0;
         fence_mbar_init();
     }
@@ -142,70 +147,89 @@ linear_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                 if (issued[s] >= 0) (void)mbar_wait(&bars.full[s], issued[s] & 1, ctx);
         }
         __syncwarp();
-    } else if (warp == 9) {
-        // ------------------------------------------------------------------ MMA issuer
+    } else if (warp == 9 || warp == 10) {
+        // ------------------------------------------------------------------ MMA issuers
+        // Two issuing threads, so that one thread's issue latency does not serialise the four
+        // products: warp 9 issues the attention path (MMA1, MMA2), warp 10 the state path (MMA3,
+        // MMA4).  Each commits its own share of the stage release, of o_done and of fin.  The
+        // shared-memory descriptors are kept as 32-bit halves; a K-step adds to the low half.
         if (lane == 0) {
-            const uint32_t idQK = idesc_bf16_f32(128, 128, false, false);
-            const uint32_t idO = idesc_bf16_f32(128, kDv, false, true);
-            const uint32_t idDS = idesc_bf16_f32(128, kDv, true, true);
-            const uint32_t sb0 = smem_u32(sm + kOffSb);
-            auto issue_qk = [&](int c) -> bool {
-                const int s = c & 1;
-                if (!wait_or_abort(&bars.full[s], (c >> 1) & 1, ctx, abort)) return false;
-                tc_fence_after();
-                const uint32_t q = smem_u32(sm + s * kStageBytes + kOffQ);
-                const uint32_t k = smem_u32(sm + s * kStageBytes + kOffK);
+            const uint32_t hi = sdesc_sw128_hi(1024);
+            // Low halves for stage 0; stage st adds st * kStageBytes / 16 to the address field.
+            const uint32_t base = smem_u32(sm);
+            const uint32_t q_lo0 = sdesc_sw128_lo(base + kOffQ, 16);
+            const uint32_t k_lo0 = sdesc_sw128_lo(base + kOffK, 16);
+            const uint32_t kt_lo0 = sdesc_sw128_lo(base + kOffK, kSub);  // K read transposed (MMA4)
+            const uint32_t v_lo0 = sdesc_sw128_lo(base + kOffV, 8192);
+            auto at_stage = [](uint32_t lo, int st) -> uint32_t { return lo + (uint32_t)(st * (kStageBytes >> 4)); };
+            // K-major operand [128 x 128] in two 64-column sub-tiles: K-step ks starts at
+            // sub-tile ks / 4, byte 32 (ks % 4) of its rows.
+            auto kstep = [](int ks) -> uint32_t { return (uint32_t)(((ks >> 2) * kSub + (ks & 3) * 32) >> 4); };
+            if (warp == 9) {
+                const uint32_t idQK = idesc_bf16_f32(128, 128, false, false);
+                const uint32_t idO = idesc_bf16_f32(128, kDv, false, true);
+                auto issue_qk = [&](int c) -> bool {  // MMA1: A = Q K^T
+                    const int st = c & 1;
+                    if (!wait_or_abort(&bars.full[st], (c >> 1) & 1, ctx, abort)) return false;
+                    tc_fence_after();
 #pragma unroll
-                for (int ks = 0; ks < kD / 16; ++ks) {
-                    const uint64_t a = sdesc_sw128(q + (ks >> 2) * kSub + (ks & 3) * 32, 16, 1024);
-                    const uint64_t b = sdesc_sw128(k + (ks >> 2) * kSub + (ks & 3) * 32, 16, 1024);
-                    mma_ss(tmem + kColA0 + s * 128, a, b, idQK, ks > 0);
+                    for (int ks = 0; ks < kD / 16; ++ks)
+                        mma_ss_lohi(tmem + kColA0 + st * 128, at_stage(q_lo0, st) + kstep(ks), at_stage(k_lo0, st) + kstep(ks), hi,
+                                    idQK, ks > 0);
+                    mma_commit(&bars.qk_done[st]);
+                    return true;
+                };
+                bool ok = n_tiles > 0 ? issue_qk(0) : true;
+                for (int c = 0; c < n_tiles && ok; ++c) {
+                    const int st = c & 1;
+                    // MMA2: O1 = A' V (A' from TMEM) once the mask is done and O1 is free.
+                    if (!wait_or_abort(&bars.a_ready[st], (c >> 1) & 1, ctx, abort)) break;
+                    if (c >= 1 && !wait_or_abort(&bars.o_free, (c - 1) & 1, ctx, abort)) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int ks = 0; ks < kC / 16; ++ks)
+                        mma_ts_lohi(tmem + kColO1, tmem + kColA0 + st * 128 + ks * 8,
+                                    at_stage(v_lo0, st) + (uint32_t)((ks * 16 * 128) >> 4), hi, idO, ks > 0);
+                    mma_commit(&bars.o_done);
+                    mma_commit(&bars.empty[st]);  // this thread's last read of stage c
+                    if (c + 1 < n_tiles) ok = issue_qk(c + 1);
                 }
-                mma_commit(&bars.qk_done[s]);
-                return true;
-            };
-            auto issue_ds = [&](int c) -> bool {  // MMA4: dS(c) = K^T V~  (A read transposed)
-                const int s = c & 1;
-                if (!wait_or_abort(&bars.full[s], (c >> 1) & 1, ctx, abort)) return false;
-                if (!wait_or_abort(&bars.v_ready[s], (c >> 1) & 1, ctx, abort)) return false;
-                tc_fence_after();
-                const uint32_t k = smem_u32(sm + s * kStageBytes + kOffK);
-                const uint32_t vt = smem_u32(sm + kOffVt + s * kSub);
+            } else {
+                const uint32_t idO = idesc_bf16_f32(128, kDv, false, true);
+                const uint32_t idDS = idesc_bf16_f32(128, kDv, true, true);
+                const uint32_t sb_lo0 = sdesc_sw128_lo(smem_u32(sm + kOffSb), 8192);
+                const uint32_t vt_lo0 = sdesc_sw128_lo(smem_u32(sm + kOffVt), 8192);
+                auto issue_ds = [&](int c) -> bool {  // MMA4: dS(c) = K^T V~ (A read transposed)
+                    const int st = c & 1;
+                    if (!wait_or_abort(&bars.full[st], (c >> 1) & 1, ctx, abort)) return false;
+                    if (!wait_or_abort(&bars.v_ready[st], (c >> 1) & 1, ctx, abort)) return false;
+                    tc_fence_after();
+                    const uint32_t vt_lo = vt_lo0;
 #pragma unroll
-                for (int ks = 0; ks < kC / 16; ++ks)
-                    mma_ss(tmem + kColDS + s * kDv, sdesc_sw128(k + ks * 16 * 128, kSub, 1024),
-                           sdesc_sw128(vt + ks * 16 * 128, 8192, 1024), idDS, ks > 0);
-                mma_commit(&bars.ds_done[s]);
-                return true;
-            };
-            bool ok = n_tiles > 0 ? (issue_qk(0) && issue_ds(0)) : true;
-            for (int c = 0; c < n_tiles && ok; ++c) {
-                const int s = c & 1;
-                const uint32_t q = smem_u32(sm + s * kStageBytes + kOffQ);
-                const uint32_t v = smem_u32(sm + s * kStageBytes + kOffV);
-                // MMA3: O2 = Q Sb(c-1), read from buffer c&1.  Sb(c-1) published also means
-                // dS(c-1) has been consumed, so its TMEM buffer is free for dS(c+1) below.
-                if (!wait_or_abort(&bars.s_ready[s], (c >> 1) & 1, ctx, abort)) break;
-                if (c >= 1 && !wait_or_abort(&bars.o_free, (c - 1) & 1, ctx, abort)) break;
-                tc_fence_after();
-                const uint32_t sb = sb0 + s * kSub;
+                    for (int ks = 0; ks < kC / 16; ++ks)
+                        mma_ss_lohi(tmem + kColDS + st * kDv, at_stage(kt_lo0, st) + (uint32_t)((ks * 16 * 128) >> 4),
+                                    vt_lo + (uint32_t)((ks * 16 * 128) >> 4), hi, idDS, ks > 0);
+                    mma_commit(&bars.ds_done[st]);
+                    return true;
+                };
+                bool ok = n_tiles > 0 ? issue_ds(0) : true;
+                for (int c = 0; c < n_tiles && ok; ++c) {
+                    const int st = c & 1;
+                    // MMA3: O2 = Q Sb(c-1), read from buffer c&1.  Sb(c-1) published also means
+                    // dS(c-1) has been consumed, so its TMEM buffer is free for dS(c+1) below.
+                    if (!wait_or_abort(&bars.s_ready[st], (c >> 1) & 1, ctx, abort)) break;
+                    if (c >= 1 && !wait_or_abort(&bars.o_free, (c - 1) & 1, ctx, abort)) break;
+                    tc_fence_after();
+                    const uint32_t sb_lo = sb_lo0 + (uint32_t)((st * kSub) >> 4);
 #pragma unroll
-                for (int ks = 0; ks < kD / 16; ++ks)
-                    mma_ss(tmem + kColO2, sdesc_sw128(q + (ks >> 2) * kSub + (ks & 3) * 32, 16, 1024),
-                           sdesc_sw128(sb + ks * 16 * 128, 8192, 1024), idO, ks > 0);
-                mma_commit(&bars.sb_free[s]);
-                // MMA2: O1 = A' V   (A' from TMEM).  Last reader of stage c: release it so the
-                // producer can fetch tile c+2 while tile c+1 is being worked on.
-                if (!wait_or_abort(&bars.a_ready[s], (c >> 1) & 1, ctx, abort)) break;
-                tc_fence_after();
-#pragma unroll
-                for (int ks = 0; ks < kC / 16; ++ks)
-                    mma_ts(tmem + kColO1, tmem + kColA0 + s * 128 + ks * 8,
-                           sdesc_sw128(v + ks * 16 * 128, 8192, 1024), idO, ks > 0);
-                mma_commit(&bars.o_done);
-                mma_commit(&bars.empty[s]);
-                // next tile: MMA1, then MMA4 (dS one tile ahead of the state update)
-                if (c + 1 < n_tiles) ok = issue_qk(c + 1) && issue_ds(c + 1);
+                    for (int ks = 0; ks < kD / 16; ++ks)
+                        mma_ss_lohi(tmem + kColO2, at_stage(q_lo0, st) + kstep(ks), sb_lo + (uint32_t)((ks * 16 * 128) >> 4),
+                                    hi, idO, ks > 0);
+                    mma_commit(&bars.sb_free[st]);
+                    mma_commit(&bars.o_done);
+                    mma_commit(&bars.empty[st]);  // MMA4(c) came earlier: this thread is done with c
+                    if (c + 1 < n_tiles) ok = issue_ds(c + 1);  // dS one tile ahead
+                }
             }
             mma_commit(&bars.fin);
             (void)mbar_wait(&bars.fin, 0, ctx);
@@ -218,7 +242,6 @@ linear_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
         const float wq = bars.pw[t + 1];
         for (int c = 0; c < n_tiles; ++c) {
             const int s = c & 1;
-            const int len = min(kC, Ns - c * kC);
             if (!wait_or_abort(&bars.qk_done[s], (c >> 1) & 1, ctx, abort)) break;
             tc_fence_after();
             const uint32_t colA = tmem + lb + kColA0 + s * 128;
@@ -252,7 +275,6 @@ linear_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
             // o_t = O1 + lambda^{t+1} O2
             if (!wait_or_abort(&bars.o_done, c & 1, ctx, abort)) break;
             tc_fence_after();
-            __nv_bfloat16* dst = out + ((bh * N) + row0 + (int64_t)c * kC + t) * kD + slice * kDv;
             uint32_t o1[64], o2[64];
             tmem_ld32(tmem + lb + kColO1, *reinterpret_cast<uint32_t(*)[32]>(&o1[0]));
             tmem_ld32(tmem + lb + kColO1 + 32, *reinterpret_cast<uint32_t(*)[32]>(&o1[32]));
@@ -262,18 +284,30 @@ linear_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars.o_free);
-            if (t < len) {
-                uint4 w[8];
-                uint32_t* wp = reinterpret_cast<uint32_t*>(w);
+            uint4 w[8];
+            uint32_t* wp = reinterpret_cast<uint32_t*>(w);
 #pragma unroll
-                for (int j = 0; j < 32; ++j)
-                    wp[j] = pack_bf16x2(fmaf(wq, __uint_as_float(o2[2 * j]), __uint_as_float(o1[2 * j])),
-                                        fmaf(wq, __uint_as_float(o2[2 * j + 1]), __uint_as_float(o1[2 * j + 1])));
-                uint4* d4 = reinterpret_cast<uint4*>(dst);
+            for (int j = 0; j < 32; ++j)
+                wp[j] = pack_bf16x2(fmaf(wq, __uint_as_float(o2[2 * j]), __uint_as_float(o1[2 * j])),
+                                    fmaf(wq, __uint_as_float(o2[2 * j + 1]), __uint_as_float(o1[2 * j + 1])));
+            // The warp's 32 rows go out as one TMA store from its own 4 KiB of the staging tile
+            // (128-byte swizzle, as the tensor map reads it): the previous tile's store from the
+            // same rows must have read them first.  Rows past the sequence end are clipped by the
+            // tensor map; within a sequence every tile but the last is full.
+            uint8_t* stg = sm + kOffOst + warp * 32 * 128;
+            if (lane == 0) bulk_wait_read0();
+            __syncwarp();
 #pragma unroll
-                for (int j = 0; j < 8; ++j) d4[j] = w[j];
+            for (int cj = 0; cj < 8; ++cj)
+                *reinterpret_cast<uint4*>(stg + lane * 128 + ((cj ^ (lane & 7)) << 4)) = w[cj];
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0 && c * kC + warp * 32 < Ns) {  // no store starts past the end
+                tma_store_3d(&tmO, stg, slice * kDv, row0 + c * kC + warp * 32, (int)bh);
+                bulk_commit();
             }
         }
+        if (lane == 0) bulk_wait0();  // this warp's stores complete before the CTA retires
     } else if (warp < 8) {
         // ------------------------------------------------------------------ EPI-S: V~, state
         const int t = tid - 128;  // row of the V tile / of the state slice
@@ -310,7 +344,7 @@ linear_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
             if (!wait_or_abort(&bars.full[s], (c >> 1) & 1, ctx, abort)) return false;
             const float w = t < len ? bars.pw[len - 1 - t] : 0.f;
             const uint8_t* vrow = sm + s * kStageBytes + kOffV + t * 128;
-            uint8_t* vtrow = sm + kOffVt + s * kSub + t * 128;
+            uint8_t* vtrow = sm + kOffVt + t * 128;
 #pragma unroll
             for (int cj = 0; cj < 8; ++cj) {
                 const int p = (cj ^ (t & 7)) << 4;
@@ -332,8 +366,8 @@ linear_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
         for (int c = 0; c < n_tiles && ok; ++c) {
             const int s = c & 1;
             const int len = min(kC, Ns - c * kC);
-            if (c + 1 < n_tiles && !make_vt(c + 1)) { ok = false; break; }
-            // S <- lambda^len S + dS(c), then its bf16 copy for the next tile.
+            // S <- lambda^len S + dS(c), then its bf16 copy for the next tile; then V~(c+1) into
+            // the one V~ buffer, which MMA4(c) (done with dS(c)) has finished reading.
             if (!wait_or_abort(&bars.ds_done[s], (c >> 1) & 1, ctx, abort)) { ok = false; break; }
             tc_fence_after();
             uint32_t d0[32], d1[32];
@@ -353,6 +387,7 @@ linear_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                 break;
             }
             write_sb(c);
+            if (c + 1 < n_tiles && !make_vt(c + 1)) { ok = false; break; }
         }
         if (ok && s_out) {
             float* row = s_out + (bh * kD + t) * kD + slice * kDv;
@@ -637,17 +672,18 @@ cudaError_t launch_linear_prefill_tc(const void* q, const void* k, const void* v
     if (d != kD) return cudaErrorNotSupported;
     EncodeTiledFn fn = encode_tiled_fn();
     if (!fn) return cudaErrorNotSupported;
-    auto make3 = [&](CUtensorMap* m, const void* base) -> bool {
+    auto make3 = [&](CUtensorMap* m, const void* base, uint32_t box_rows) -> bool {
         cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)N, (cuuint64_t)B * H};
         cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)kD * 2 * N};
-        cuuint32_t box[3] = {64, kC, 1};
+        cuuint32_t box[3] = {64, box_rows, 1};
         cuuint32_t estr[3] = {1, 1, 1};
         return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
     };
-    CUtensorMap tmQ, tmK, tmV;
-    if (!make3(&tmQ, q) || !make3(&tmK, k) || !make3(&tmV, v)) return cudaErrorInvalidValue;
+    CUtensorMap tmQ, tmK, tmV, tmO;  // O: one warp's 32 rows per store
+    if (!make3(&tmQ, q, kC) || !make3(&tmK, k, kC) || !make3(&tmV, v, kC) || !make3(&tmO, o, 32))
+        return cudaErrorInvalidValue;
     cudaError_t e = ensure_smem<linear_prefill_tc_kernel>(kSmemBytes);
     if (e != cudaSuccess) return e;
     int n_seg, seg_len;
@@ -667,14 +703,13 @@ cudaError_t launch_linear_prefill_tc(const void* q, const void* k, const void* v
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
         linear_prefill_tc_kernel<<<B * H * n_seg * kSlices, kThreads, kSmemBytes, st>>>(
-            tmQ, tmK, tmV, decay, static_cast<__nv_bfloat16*>(o), s_seg, nullptr, H, N, seg_len,
-            n_seg, seg_stride, ctx);
+            tmQ, tmK, tmV, tmO, decay, s_seg, nullptr, H, N, seg_len, n_seg, seg_stride, ctx);
         return cudaGetLastError();
     }
     // One segment.  If state_out aliases state_in, every CTA reads its slice before it writes it
     // back, and no two CTAs share a slice, so in-place update is safe.
     linear_prefill_tc_kernel<<<B * H * kSlices, kThreads, kSmemBytes, st>>>(
-        tmQ, tmK, tmV, decay, static_cast<__nv_bfloat16*>(o), s_in, s_out, H, N, N, 1, 0, ctx);
+        tmQ, tmK, tmV, tmO, decay, s_in, s_out, H, N, N, 1, 0, ctx);
     return cudaGetLastError();
 }
 
