@@ -240,9 +240,11 @@ linear_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
         const int t = tid;
         const uint32_t lb = tmem_lane_base(warp);
         const float wq = bars.pw[t + 1];
-        for (int c = 0; c < n_tiles; ++c) {
+        // Tile c+1 is masked before tile c's output is written: MMA2(c) and MMA3(c) then run
+        // while this warp group works on the next tile's scores.
+        auto mask = [&](int c) -> bool {  // A' = A * lambda^{t-s} [s <= t], bf16, over A in TMEM
             const int s = c & 1;
-            if (!wait_or_abort(&bars.qk_done[s], (c >> 1) & 1, ctx, abort)) break;
+            if (!wait_or_abort(&bars.qk_done[s], (c >> 1) & 1, ctx, abort)) return false;
             tc_fence_after();
             const uint32_t colA = tmem + lb + kColA0 + s * 128;
             // s > t is masked; tiles never reach s >= 128, and rows/keys past len are zero.
@@ -272,8 +274,10 @@ linear_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars.a_ready[s]);
-            // o_t = O1 + lambda^{t+1} O2
-            if (!wait_or_abort(&bars.o_done, c & 1, ctx, abort)) break;
+            return true;
+        };
+        auto output = [&](int c) -> bool {  // o_t = O1 + lambda^{t+1} O2
+            if (!wait_or_abort(&bars.o_done, c & 1, ctx, abort)) return false;
             tc_fence_after();
             uint32_t o1[64], o2[64];
             tmem_ld32(tmem + lb + kColO1, *reinterpret_cast<uint32_t(*)[32]>(&o1[0]));
@@ -306,6 +310,12 @@ linear_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                 tma_store_3d(&tmO, stg, slice * kDv, row0 + c * kC + warp * 32, (int)bh);
                 bulk_commit();
             }
+            return true;
+        };
+        bool ok = n_tiles > 0 ? mask(0) : true;
+        for (int c = 0; c < n_tiles && ok; ++c) {
+            if (c + 1 < n_tiles && !mask(c + 1)) break;
+            ok = output(c);
         }
         if (lane == 0) bulk_wait0();  // this warp's stores complete before the CTA retires
     } else if (warp < 8) {
