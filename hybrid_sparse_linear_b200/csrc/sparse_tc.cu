@@ -21,11 +21,11 @@
 // Shared memory holds the unit's two Q tiles and a ring of four 32 KiB stages, each the K and V
 // of one block, loaded by TMA up to four blocks ahead.
 //
-// Roles (352 threads, persistent: one CTA per SM walks units blockIdx.x, +gridDim.x, ...):
-// warps 0-3 softmax + epilogue of tile A, warps 4-7 of tile B (thread = row = TMEM lane); warp 8
-// stages the next unit's 16 selection rows with coalesced loads, merges them into the union list
-// and issues the TMA loads (Q tiles, then the ring); warp 9 allocates TMEM and issues the MMAs of
-// tile A, warp 10 those of tile B (one thread each).  Every wait is bounded; a timeout sets the
+// Roles (384 threads, persistent: one CTA per SM walks units blockIdx.x, +gridDim.x, ...):
+// warps 0-3 softmax + epilogue of tile A, warps 4-7 of tile B (thread = row = TMEM lane); warp 11
+// stages the next unit's 16 selection rows and merges them into its union list (double-buffered,
+// one unit ahead); warp 8 issues the TMA loads (Q tiles, then the ring); warp 9 allocates TMEM and
+// issues the MMAs of tile A, warp 10 those of tile B (one thread each).  Every wait is bounded; a timeout sets the
 // status word, the roles wind down, and the kernel waits (bounded) for its own copies and MMAs
 // before it frees TMEM.
 #include "fastexp.cuh"
@@ -45,7 +45,7 @@ constexpr int kUT = 16;          // query tokens per unit (two tiles)
 constexpr int kBlk = 64;         // keys per block
 constexpr int kMaxSlots = 80;    // selection slots per row the kernel accepts
 constexpr int kMaxList = kUT * kMaxSlots;
-constexpr int kThreads = 352;
+constexpr int kThreads = 384;
 constexpr int kStages = 4;
 
 // Shared memory (offsets from a 1024-aligned base): Q_A, Q_B (two [128 x 128 B] halves each,
@@ -192,7 +192,7 @@ sparse_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                 mbar_init(&bars.pv_done[b][j], 1);
             }
             mbar_init(&bars.list_full[b], 1);
-            mbar_init(&bars.list_empty[b], 3);
+            mbar_init(&bars.list_empty[b], 4);  // producer, both issuers, softmax
             mbar_init(&bars.fin[b], 1);
         }
         mbar_init(&bars.q_full, 1);
@@ -215,12 +215,13 @@ sparse_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
     auto empty_bar = [&](uint32_t e) { return &bars.kv_empty[e % kStages]; };
     auto round_of = [](uint32_t e) { return (e / kStages) & 1u; };
 
-    if (warp == 8) {
-        // ---------------------------------------------------------------- producer
-        // A unit with a non-empty union loads its Q tiles, then one ring entry per union block.
+    if (warp == 11) {
+        // ---------------------------------------------------------------- union lists
+        // Builds unit u+1's union list (double-buffered) while unit u is being consumed, so the
+        // producer never stalls the ring on it: the unit's 16 selection rows (contiguous in
+        // memory) are staged with all loads in flight, then merged.
         int32_t* stage = reinterpret_cast<int32_t*>(sm + kOffStage);
         int it = 0;
-        uint32_t rc = 0, kq = 0;  // ring entries issued, Q tile pairs issued
         for (int unit = blockIdx.x; unit < n_units; unit += gridDim.x, ++it) {
             const int lb = it & 1;
             if (it >= 2 && !wait_or_abort(&bars.list_empty[lb], ((it - 2) >> 1) & 1, ctx, abort)) break;
@@ -228,9 +229,22 @@ sparse_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
             const int i0 = (unit % units_per_seq) * kUT;
             const int c = i0 / kBlk;
             const int n_act = min(kUT, N - i0);
-            // Stage the unit's selection rows (contiguous in memory) with coalesced loads.
+            const int total = n_act * slots;
             const int32_t* src = idx + (bg * N + i0) * (int64_t)slots;
-            for (int e = lane; e < n_act * slots; e += 32) stage[e] = src[e];
+            {
+                constexpr int kPer = kMaxList / 32;  // entries per lane at most
+                int32_t v[kPer];
+#pragma unroll
+                for (int j = 0; j < kPer; ++j) {
+                    const int e = lane + 32 * j;
+                    v[j] = e < total ? __ldg(src + e) : -1;
+                }
+#pragma unroll
+                for (int j = 0; j < kPer; ++j) {
+                    const int e = lane + 32 * j;
+                    if (e < total) stage[e] = v[j];
+                }
+            }
             __syncwarp();
             // 16-way merge of the ascending rows, one lane per token.
             const int32_t* row = stage + lane * slots;
@@ -262,39 +276,57 @@ sparse_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                 n = __shfl_sync(0xffffffffu, n, 0);
                 prev = m;
             }
+            __syncwarp();
             if (lane == 0) {
                 bars.list_n[lb] = n;
                 mbar_arrive(&bars.list_full[lb]);
             }
             __syncwarp();
+            if (*abort) break;
+        }
+    } else if (warp == 8) {
+        // ---------------------------------------------------------------- producer
+        // A unit with a non-empty union loads its Q tiles, then one ring entry per union block;
+        // its list buffer goes back to the list warp once the last entry is issued.
+        int it = 0;
+        uint32_t rc = 0, kq = 0;  // ring entries issued, Q tile pairs issued
+        for (int unit = blockIdx.x; unit < n_units; unit += gridDim.x, ++it) {
+            const int lb = it & 1;
             int stop = 0;
-            if (lane == 0 && n > 0) {
-                // Q_A, Q_B: 16 heads x 8 tokens x 128 columns each, once both issuers are done
-                // with the previous unit's S MMAs.
-                if (kq >= 1 && !wait_or_abort(&bars.q_empty, (kq - 1) & 1, ctx, abort)) stop = 1;
-                if (!stop) {
-                    const int z = (int)((bg / Hkv) * H + (bg % Hkv) * kG);
-                    mbar_arrive_expect_tx(&bars.q_full, 2 * kQBytes);
-                    for (int q = 0; q < 2; ++q) {
-                        tma_load_3d(sm + q * kQBytes, &tmQ, &bars.q_full, 0, i0 + q * kTQ, z);
-                        tma_load_3d(sm + q * kQBytes + kHalfQ, &tmQ, &bars.q_full, 64, i0 + q * kTQ, z);
+            if (lane == 0) {
+                if (!wait_or_abort(&bars.list_full[lb], (it >> 1) & 1, ctx, abort)) stop = 1;
+                const int n = stop ? 0 : bars.list_n[lb];
+                const int64_t bg = unit / units_per_seq;
+                const int i0 = (unit % units_per_seq) * kUT;
+                if (n > 0) {
+                    // Q_A, Q_B: 16 heads x 8 tokens x 128 columns each, once both issuers are
+                    // done with the previous unit's S MMAs.
+                    if (kq >= 1 && !wait_or_abort(&bars.q_empty, (kq - 1) & 1, ctx, abort)) stop = 1;
+                    if (!stop) {
+                        const int z = (int)((bg / Hkv) * H + (bg % Hkv) * kG);
+                        mbar_arrive_expect_tx(&bars.q_full, 2 * kQBytes);
+                        for (int q = 0; q < 2; ++q) {
+                            tma_load_3d(sm + q * kQBytes, &tmQ, &bars.q_full, 0, i0 + q * kTQ, z);
+                            tma_load_3d(sm + q * kQBytes + kHalfQ, &tmQ, &bars.q_full, 64, i0 + q * kTQ, z);
+                        }
+                        ++kq;
                     }
-                    ++kq;
-                }
-                for (int e = 0; e < n && !stop; ++e, ++rc) {
-                    if (rc >= kStages && !wait_or_abort(empty_bar(rc), round_of(rc - kStages), ctx, abort)) {
-                        stop = 1;
-                        break;
+                    for (int e = 0; e < n && !stop; ++e, ++rc) {
+                        if (rc >= kStages && !wait_or_abort(empty_bar(rc), round_of(rc - kStages), ctx, abort)) {
+                            stop = 1;
+                            break;
+                        }
+                        uint8_t* st = stage_ptr(rc);
+                        uint64_t* fb = full_bar(rc);
+                        mbar_arrive_expect_tx(fb, kStageBytes);
+                        const int y = list_id(lb)[e] * kBlk;
+                        tma_load_3d(st, &tmK, fb, 0, y, (int)bg);
+                        tma_load_3d(st + kHalfBlk, &tmK, fb, 64, y, (int)bg);
+                        tma_load_3d(st + 2 * kHalfBlk, &tmV, fb, 0, y, (int)bg);
+                        tma_load_3d(st + 3 * kHalfBlk, &tmV, fb, 64, y, (int)bg);
                     }
-                    uint8_t* st = stage_ptr(rc);
-                    uint64_t* fb = full_bar(rc);
-                    mbar_arrive_expect_tx(fb, kStageBytes);
-                    const int y = list_id(lb)[e] * kBlk;
-                    tma_load_3d(st, &tmK, fb, 0, y, (int)bg);
-                    tma_load_3d(st + kHalfBlk, &tmK, fb, 64, y, (int)bg);
-                    tma_load_3d(st + 2 * kHalfBlk, &tmV, fb, 0, y, (int)bg);
-                    tma_load_3d(st + 3 * kHalfBlk, &tmV, fb, 64, y, (int)bg);
                 }
+                if (!stop) mbar_arrive(&bars.list_empty[lb]);  // done reading the list
             }
             rc = __shfl_sync(0xffffffffu, rc, 0);
             kq = __shfl_sync(0xffffffffu, kq, 0);
@@ -306,7 +338,7 @@ sparse_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
             for (uint32_t e = rc > kStages ? rc - kStages : 0; e < rc; ++e)
                 (void)mbar_wait(full_bar(e), round_of(e), ctx);
         }
-    } else if (warp >= 9) {
+    } else if (warp == 9 || warp == 10) {
         // ---------------------------------------------------------------- MMA issuers
         // Warp 9 issues the MMAs of tile A, warp 10 those of tile B (one thread each): a single
         // thread needs ~50 cycles per tcgen05.mma, more than the 32 of math in an N=64 S MMA, so
