@@ -48,28 +48,33 @@ __device__ __forceinline__ uint64_t sel_key_u(float score, int blk) { return sel
 // Grid-wide barrier for a cooperative launch on one 32-bit word: arrivals of the current barrier
 // in the low 16 bits (zero between barriers), a generation count above.  The arrival's atomic
 // returns the generation it belongs to; the last arrival clears the count and bumps the generation
-// in one atomic.  Returns false after a timeout.
+// in one atomic.  Returns false after a timeout.  Ordering: the block barrier orders every thread's
+// writes before thread 0's arrival, an acquire-release atomic (the arrivals form one release
+// sequence), so the last arrival's release of the bump carries all CTAs' writes to each waiter's
+// acquire load; no full fence is needed on either side.
 __device__ bool grid_barrier(unsigned* word, unsigned nblocks, const DevCtx& ctx, int* s_ok) {
     __syncthreads();
     if (threadIdx.x == 0) {
         int ok = 1;
-        __threadfence();
-        const unsigned old = atomicAdd(word, 1u);
+        unsigned old;
+        asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(word) : "memory");
         if ((old & 0xFFFFu) == nblocks - 1) {
-            atomicAdd(word, 0x10000u - nblocks);
+            asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(word), "r"(0x10000u - nblocks)
+                         : "memory");
         } else {
             const unsigned g0 = old >> 16;
             const uint64_t t0 = globaltimer_ns();
-            while ((*reinterpret_cast<volatile unsigned*>(word) >> 16) == g0) {
+            while (true) {
+                unsigned v;
+                asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(word) : "memory");
+                if ((v >> 16) != g0) break;
                 if (globaltimer_ns() - t0 > ctx.wait_limit_ns) {
                     flag(ctx, kStatusTimeout);
                     ok = 0;
                     break;
                 }
-                __nanosleep(20);
             }
         }
-        __threadfence();
         *s_ok = ok;
     }
     __syncthreads();
@@ -238,6 +243,25 @@ sparse_decode_fused_kernel(const T* __restrict__ q, const T* __restrict__ kc,
     // publishes its top-k keys sorted, largest first.
     constexpr int kLPR = D / 16, kRPS = 32 / kLPR, kSteps = (kSpan / 8) / kRPS;
     if (do_sel && K > 0) {
+        const T* kb = kbar + (int64_t)bg * nb_cap * D;
+        const int part16 = (lane % kLPR) * 16;
+        constexpr int kU = 16 * sizeof(T) / 16;   // 16-byte pieces per lane and row
+        constexpr int kEl = 16 / sizeof(T);        // elements per piece
+        uint4 raw[kSteps][kU];
+        auto load_span = [&](int span) {  // every load of the span in flight at once
+            const int base = lo + span * kSpan;
+#pragma unroll
+            for (int st = 0; st < kSteps; ++st) {
+                const int blk = base + warp * (kSpan / 8) + st * kRPS + lane / kLPR;
+                const T* row = kb + (int64_t)blk * D + part16;
+#pragma unroll
+                for (int u = 0; u < kU; ++u)
+                    raw[st][u] = blk <= hi ? ld16(row + u * kEl) : make_uint4(0u, 0u, 0u, 0u);
+            }
+        };
+        // The first span's k_bar rows are requested before the query rows they are scored
+        // against, so the two memory round trips overlap.
+        if (j < nspan) load_span(j);
         if (tid < D) {  // all G loads in flight at once (a runtime-G loop would issue them one by one)
             float qv[kMaxG];
 #pragma unroll
@@ -248,21 +272,9 @@ sparse_decode_fused_kernel(const T* __restrict__ q, const T* __restrict__ kc,
             sm.qbar[tid] = s;
         }
         __syncthreads();
-        const T* kb = kbar + (int64_t)bg * nb_cap * D;
-        const int part16 = (lane % kLPR) * 16;
         for (int span = j; span < nspan; span += cpg) {
             const int base = lo + span * kSpan;
-            constexpr int kU = 16 * sizeof(T) / 16;   // 16-byte pieces per lane and row
-            constexpr int kEl = 16 / sizeof(T);        // elements per piece
-            uint4 raw[kSteps][kU];
-#pragma unroll
-            for (int st = 0; st < kSteps; ++st) {
-                const int blk = base + warp * (kSpan / 8) + st * kRPS + lane / kLPR;
-                const T* row = kb + (int64_t)blk * D + part16;
-#pragma unroll
-                for (int u = 0; u < kU; ++u)
-                    raw[st][u] = blk <= hi ? ld16(row + u * kEl) : make_uint4(0u, 0u, 0u, 0u);
-            }
+            if (span != j) load_span(span);
 #pragma unroll
             for (int st = 0; st < kSteps; ++st) {
                 float a0 = 0.f, a1 = 0.f;
