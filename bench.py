@@ -591,7 +591,7 @@ def main():
     ap.add_argument("--impl", choices=["sala", "reference"], default="sala")
     ap.add_argument("--phases", default="prefill,decode,e2e,cpu",
                     help="comma list of prefill,decode,e2e,cpu (default: all)")
-    ap.add_argument("--decode-steps", type=int, default=50)
+    ap.add_argument("--decode-steps", type=int, default=200)
     ap.add_argument("--decode-t", type=int, default=DECODE_T,
                     help="decode context length (default 2^20, the benchmark; smaller only for profiles)")
     ap.add_argument("--workload", default="hybrid_prefill_n256k", choices=sorted(WORKLOADS),

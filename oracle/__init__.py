@@ -55,6 +55,7 @@ def _load():
             lib.orc_linear_quadratic.argtypes = [_D, _D, _D, _D, _D, _D, _i, _i, _i, _i, _i, _I64, _l, _i]
             lib.orc_linear_chunked.argtypes = [_D, _D, _D, _D, _D, _D, _D, _i, _i, _i, _i, _i, _i, _i]
             lib.orc_linear_decode.argtypes = [_D, _D, _D, _D, _D, _D, _i, _i, _i, _i]
+            lib.orc_rope.argtypes = [_D, _i, _i, _i, _i, _l, ctypes.c_double]
             lib.orc_block_compress.argtypes = [_D, _D, _i, _i, _i, _i, _i, _i, _i, _i]
             lib.orc_block_scores_at.argtypes = [_D, _D, _I64, _l, _D, _i, _i, _i, _i, _i]
             lib.orc_block_select.argtypes = [_D, _D, _I32, _D, _i, _i, _i, _i, _i, _i, _i, _i, _i,
@@ -150,6 +151,22 @@ def linear_decode(q, k, v, lam, state):
     o = np.empty((B, H, dv))
     _load().orc_linear_decode(_p(q), _p(k), _p(v), _p(lam), _p(S), _p(o), B, H, dk, dv)
     return o, S
+
+
+def rope(x, pos0=0, base=10000.0):
+    """Rotary position embedding of x [B,H,N,d] (row r at position pos0 + r); a rotated copy.
+    The linear layers apply it to q and k before the linear attention (HyPE)."""
+    x = _f64(x).copy()
+    B, H, N, d = x.shape
+    assert d % 2 == 0
+    _load().orc_rope(_p(x), B, H, N, d, int(pos0), float(base))
+    return x
+
+
+def linear_chunked_rope(q, k, v, lam, chunk, pos0=0, base=10000.0, s_in=None):
+    """Linear attention of a linear (HyPE) layer: q and k rotated by position first.  Returns
+    (o, s_out) as linear_chunked."""
+    return linear_chunked(rope(q, pos0, base), rope(k, pos0, base), v, lam, chunk, s_in=s_in)
 
 
 # ----------------------------------------------------------------------------------------------

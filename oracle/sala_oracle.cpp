@@ -376,4 +376,27 @@ void orc_dense_causal_attention(const double* q, const double* k, const double* 
     });
 }
 
+// Rotary position embedding, in place on x [B, H, N, d] (d even), row r at position pos0 + r.
+// MiniCPM-SALA summaries, JA section 2.2 "positional encoding (HyPE)" and DE section 2 "HyPE": the
+// linear-attention layers rotate queries and keys by position (RoPE); the sparse layers do not.
+// The pages give no RoPE parameters; the reading taken is the rotate-half pairing (element i with
+// element i + d/2 for i < d/2), frequencies theta_i = base^(-2i/d), angle (pos0 + r) * theta_i:
+//   x'_i       = x_i cos(angle) - x_{i+d/2} sin(angle)
+//   x'_{i+d/2} = x_{i+d/2} cos(angle) + x_i sin(angle)
+void orc_rope(double* x, int B, int H, int N, int d, int64_t pos0, double base) {
+    const int half = d / 2;
+    for (int64_t bh = 0; bh < (int64_t)B * H; ++bh)
+        for (int r = 0; r < N; ++r) {
+            double* row = x + (bh * N + r) * d;
+            const double p = (double)(pos0 + r);
+            for (int i = 0; i < half; ++i) {
+                const double theta = std::pow(base, -2.0 * i / d);
+                const double c = std::cos(p * theta), s = std::sin(p * theta);
+                const double x0 = row[i], x1 = row[i + half];
+                row[i] = x0 * c - x1 * s;
+                row[i + half] = x1 * c + x0 * s;
+            }
+        }
+}
+
 }  // extern "C"

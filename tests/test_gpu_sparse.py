@@ -128,16 +128,16 @@ def test_out_of_range_index_is_flagged(sala):
 
 # ---------------------------------------------------------------------------------------------
 def _decode_case(sala, T, topk, n_init, n_local, dtype, layer_id, given_idx=False, H=32, Hkv=2,
-                 d=128, workspace=None):
+                 d=128, workspace=None, B=1):
     from hybrid_sparse_linear_b200 import synth
-    layer = synth.sparse_layer(1, H, Hkv, T, d, dtype, device="cuda", layer=layer_id,
+    layer = synth.sparse_layer(B, H, Hkv, T, d, dtype, device="cuda", layer=layer_id,
                                shift_frac=0.05, q_rows=1)
     pos = T - 1
     kc, vc = layer.k, layer.v
     kbar = sala.block_compress(kc)
     qd = layer.q[:, :, 0].contiguous()
     slots = n_init + n_local + topk
-    idx_out = torch.empty((1, Hkv, slots), dtype=torch.int32, device="cuda")
+    idx_out = torch.empty((B, Hkv, slots), dtype=torch.int32, device="cuda")
     q64 = _f64(layer.q)
     kind = "bf16" if dtype == torch.bfloat16 else "f32"
     kbar_ref = oracle.block_compress(_f64(layer.k), 64, round_to_bf16=(kind == "bf16"))
@@ -159,6 +159,13 @@ def _decode_case(sala, T, topk, n_init, n_local, dtype, layer_id, given_idx=Fals
 @pytest.mark.parametrize("T", [64 * 300 + 5, 64 * 300, 64 * 3, 1, 70])
 def test_sparse_decode(sala, T):
     _decode_case(sala, T, 16, 1, 2, torch.bfloat16, 6)
+
+
+@pytest.mark.parametrize("T,topk", [(64 * 700 + 9, 64), (64 * 120, 100)])
+def test_sparse_decode_batched(sala, T, topk):
+    # B = 3 sequences at one position: every (sequence, KV group) selects and attends on its own;
+    # k = 100 takes the four-launch path.
+    _decode_case(sala, T, topk, 1, 2, torch.bfloat16, 12, B=3)
 
 
 def test_sparse_decode_given_idx_fp32(sala):
