@@ -234,6 +234,8 @@ WORKLOADS = {
     "linear_prefill_n32k": (32768, ["linear"]),
     "sparse_prefill_n32k": (32768, ["sparse"]),
     "linear_prefill_n256k": (N_TOK, ["linear"]),
+    # a linear layer with its RoPE (HyPE) fused into the load path, base 10000, positions 0..N-1
+    "linear_rope_prefill_n256k": (N_TOK, ["linear_rope"]),
 }
 
 
@@ -249,7 +251,7 @@ def run_prefill(sala, synth, torch, steps, warmup, stream, workload="hybrid_pref
             layers.append(("sparse", sl.q, sl.k, sl.v))
         else:
             q, k, v = synth.linear_layer(1, H, n_tok, D, torch.bfloat16, dev, layer=l)
-            layers.append(("linear", q, k, v))
+            layers.append((kind, q, k, v))
     out = torch.empty((1, H, n_tok, D), device=dev, dtype=torch.bfloat16)
     nb = n_tok // BLOCK
     kbar = torch.empty((1, HKV, nb, D), device=dev, dtype=torch.bfloat16)
@@ -266,10 +268,14 @@ def run_prefill(sala, synth, torch, steps, warmup, stream, workload="hybrid_pref
     def one_step(record):
         launches = 0
         for kind, q, k, v in layers:
-            if kind == "linear":
+            if kind in ("linear", "linear_rope"):
                 e0, e1 = (ev(), ev()) if record else (None, None)
                 if record: e0.record(stream)
-                sala.linear_prefill(q, k, v, lam, o=out, workspace=lws, stream=stream)
+                if kind == "linear":
+                    sala.linear_prefill(q, k, v, lam, o=out, workspace=lws, stream=stream)
+                else:
+                    sala.linear_prefill(q, k, v, lam, o=out, workspace=lws, stream=stream,
+                                        rope_base=10000.0, pos0=0)
                 if record: e1.record(stream); linear_ev.append((e0, e1))
                 launches += 1
             else:
@@ -682,7 +688,7 @@ def main():
             line["kernels"]["sparse_prefill"] = {"mean_ms": pre["sparse_ms"], "achieved_tflops": achieved,
                                                  "executed_tflops": executed}
             line["kernels"]["compress_plus_select"] = {"mean_ms": pre["select_ms"]}
-        if "linear" in kinds:
+        if "linear" in kinds or "linear_rope" in kinds:
             lin_gbs = linear_layer_bytes(n_tok) / (pre["linear_ms"] / 1000.0) / 1e9
             line["kernels"]["linear_prefill"] = {"mean_ms": pre["linear_ms"], "achieved_gbs": lin_gbs,
                                                  "hbm_frac": lin_gbs / peaks["hbm_gbs"]}

@@ -130,8 +130,8 @@ sala_status sala_selftest_wait_timeout(sala_stream stream) {
 static sala_status linear_prefill_impl(const void* q, const void* k, const void* v,
                                        const float* decay, void* o, const float* state_in,
                                        float* state_out, int B, int H, int N, int d, int chunk,
-                                       void* workspace, size_t workspace_bytes, sala_dtype dt,
-                                       sala_stream stream) {
+                                       void* workspace, size_t workspace_bytes, sala::Rope rope,
+                                       sala_dtype dt, sala_stream stream) {
     REQUIRE(B >= 0 && H >= 0 && N >= 0, SALA_ERR_INVALID_ARG, "negative size (B=%d H=%d N=%d)", B, H, N);
     REQUIRE(dt == SALA_F32 || dt == SALA_BF16, SALA_ERR_INVALID_ARG, "unknown dtype %d", (int)dt);
     REQUIRE(d == 64 || d == 128, SALA_ERR_UNSUPPORTED, "head dim %d (supported: 64, 128)", d);
@@ -151,10 +151,11 @@ static sala_status linear_prefill_impl(const void* q, const void* k, const void*
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (dt == SALA_BF16 && N > 0 && sala::linear_prefill_tc_supported(d))
         return launched(sala::launch_linear_prefill_tc(q, k, v, decay, o, state_in, state_out, B,
-                                                       H, N, d, workspace, workspace_bytes, st, ctx),
+                                                       H, N, d, workspace, workspace_bytes, rope, st,
+                                                       ctx),
                         "linear_prefill_tc");
     return launched(sala::launch_linear_prefill_simt(to_dt(dt), q, k, v, decay, o, state_in,
-                                                     state_out, B, H, N, d, st, ctx),
+                                                     state_out, B, H, N, d, rope, st, ctx),
                     "linear_prefill");
 }
 
@@ -162,7 +163,7 @@ sala_status sala_linear_prefill(const void* q, const void* k, const void* v, con
                                 void* o, const float* state_in, float* state_out, int B, int H,
                                 int N, int d, int chunk, sala_dtype dt, sala_stream stream) {
     return linear_prefill_impl(q, k, v, decay, o, state_in, state_out, B, H, N, d, chunk, nullptr,
-                               0, dt, stream);
+                               0, sala::Rope{0.0, 0}, dt, stream);
 }
 
 size_t sala_linear_prefill_workspace(int B, int H, int N, int d, sala_dtype dt) {
@@ -175,12 +176,24 @@ sala_status sala_linear_prefill_ws(const void* q, const void* k, const void* v, 
                                    int N, int d, int chunk, void* workspace,
                                    size_t workspace_bytes, sala_dtype dt, sala_stream stream) {
     return linear_prefill_impl(q, k, v, decay, o, state_in, state_out, B, H, N, d, chunk,
-                               workspace, workspace_bytes, dt, stream);
+                               workspace, workspace_bytes, sala::Rope{0.0, 0}, dt, stream);
 }
 
-sala_status sala_linear_decode(const void* q, const void* k, const void* v, const float* decay,
-                               float* state, void* o, int B, int H, int d, sala_dtype dt,
-                               sala_stream stream) {
+sala_status sala_linear_prefill_rope(const void* q, const void* k, const void* v,
+                                     const float* decay, void* o, const float* state_in,
+                                     float* state_out, int B, int H, int N, int d, int64_t pos0,
+                                     double rope_base, void* workspace, size_t workspace_bytes,
+                                     sala_dtype dt, sala_stream stream) {
+    REQUIRE(pos0 >= 0, SALA_ERR_INVALID_ARG, "pos0 %lld is negative", (long long)pos0);
+    REQUIRE(rope_base > 1.0 && rope_base < 1e30, SALA_ERR_INVALID_ARG,
+            "rope_base %g (must lie in (1, 1e30))", rope_base);
+    return linear_prefill_impl(q, k, v, decay, o, state_in, state_out, B, H, N, d, 0, workspace,
+                               workspace_bytes, sala::Rope{rope_base, pos0}, dt, stream);
+}
+
+static sala_status linear_decode_impl(const void* q, const void* k, const void* v,
+                                      const float* decay, float* state, void* o, int B, int H,
+                                      int d, sala::Rope rope, sala_dtype dt, sala_stream stream) {
     REQUIRE(B >= 0 && H >= 0, SALA_ERR_INVALID_ARG, "negative size (B=%d H=%d)", B, H);
     REQUIRE(dt == SALA_F32 || dt == SALA_BF16, SALA_ERR_INVALID_ARG, "unknown dtype %d", (int)dt);
     REQUIRE(d == 64 || d == 128, SALA_ERR_UNSUPPORTED, "head dim %d (supported: 64, 128)", d);
@@ -191,8 +204,25 @@ sala_status sala_linear_decode(const void* q, const void* k, const void* v, cons
     sala_status s = get_ctx(&ctx);
     if (s != SALA_OK) return s;
     return launched(sala::launch_linear_decode(to_dt(dt), q, k, v, decay, state, o, B, H, d,
-                                               static_cast<cudaStream_t>(stream), ctx),
+                                               rope, static_cast<cudaStream_t>(stream), ctx),
                     "linear_decode");
+}
+
+sala_status sala_linear_decode(const void* q, const void* k, const void* v, const float* decay,
+                               float* state, void* o, int B, int H, int d, sala_dtype dt,
+                               sala_stream stream) {
+    return linear_decode_impl(q, k, v, decay, state, o, B, H, d, sala::Rope{0.0, 0}, dt, stream);
+}
+
+sala_status sala_linear_decode_rope(const void* q, const void* k, const void* v,
+                                    const float* decay, float* state, void* o, int B, int H,
+                                    int d, int64_t pos, double rope_base, sala_dtype dt,
+                                    sala_stream stream) {
+    REQUIRE(pos >= 0, SALA_ERR_INVALID_ARG, "pos %lld is negative", (long long)pos);
+    REQUIRE(rope_base > 1.0 && rope_base < 1e30, SALA_ERR_INVALID_ARG,
+            "rope_base %g (must lie in (1, 1e30))", rope_base);
+    return linear_decode_impl(q, k, v, decay, state, o, B, H, d, sala::Rope{rope_base, pos}, dt,
+                              stream);
 }
 
 // ----------------------------------------------------------------------------------------------

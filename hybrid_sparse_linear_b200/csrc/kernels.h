@@ -12,10 +12,15 @@ namespace sala {
 
 enum class DType { F32 = 0, BF16 = 1 };
 
-// Linear attention.
+// Linear attention.  rope: rotary position embedding of q and k (off when base <= 0); row r of
+// a prefill sits at position pos0 + r, a decode step at pos0.
+struct Rope {
+    double base;
+    int64_t pos0;
+};
 cudaError_t launch_linear_prefill_simt(DType dt, const void* q, const void* k, const void* v,
                                        const float* decay, void* o, const float* s_in,
-                                       float* s_out, int B, int H, int N, int d,
+                                       float* s_out, int B, int H, int N, int d, Rope rope,
                                        cudaStream_t st, DevCtx ctx);
 // bf16, d = 128.  With a workspace of linear_prefill_tc_workspace(...) bytes (0 = not needed) the
 // sequence is split into segments processed in parallel (state pass, chaining, output pass);
@@ -24,11 +29,11 @@ size_t linear_prefill_tc_workspace(int B, int H, int N, int d);
 cudaError_t launch_linear_prefill_tc(const void* q, const void* k, const void* v,
                                      const float* decay, void* o, const float* s_in,
                                      float* s_out, int B, int H, int N, int d, void* ws,
-                                     size_t ws_bytes, cudaStream_t st, DevCtx ctx);
+                                     size_t ws_bytes, Rope rope, cudaStream_t st, DevCtx ctx);
 bool linear_prefill_tc_supported(int d);
 cudaError_t launch_linear_decode(DType dt, const void* q, const void* k, const void* v,
                                  const float* decay, float* state, void* o, int B, int H, int d,
-                                 cudaStream_t st, DevCtx ctx);
+                                 Rope rope, cudaStream_t st, DevCtx ctx);
 
 // Sparse attention.
 cudaError_t launch_block_compress(DType dt, const void* k, void* kbar, int B, int Hkv, int N,

@@ -5,6 +5,7 @@
 // (batch, head, slice of DV value columns) and walks the chunks in order; S[:, slice] evolves
 // independently of the other slices, so slices run in parallel with no communication.
 #include "kernels.h"
+#include "rope.cuh"
 
 namespace sala {
 namespace {
@@ -15,7 +16,7 @@ constexpr int kThreads = 256;
 template <int D, int DV>
 struct PrefillSmem {
     static constexpr int kQK = kC * (D + 1);
-    static constexpr size_t bytes =
+    static constexpr size_t bytes = sizeof(double) * (D / 2) +  // RoPE turns per frequency
         sizeof(float) * (2 * kQK + kC * DV + kC * (kC + 1) + D * DV + (kC + 1));
 };
 
@@ -23,8 +24,11 @@ template <typename T, int D, int DV>
 __global__ void __launch_bounds__(kThreads)
 linear_prefill_simt_kernel(const T* __restrict__ q, const T* __restrict__ k,
                            const T* __restrict__ v, const float* __restrict__ decay,
-                           T* __restrict__ o, const float* s_in, float* s_out, int H, int N) {
-    extern __shared__ float sm[];
+                           T* __restrict__ o, const float* s_in, float* s_out, int H, int N,
+                           Rope rope) {
+    extern __shared__ double smd[];
+    double* turn = smd;                     // [D/2]  theta_i / 2pi (RoPE)
+    float* sm = reinterpret_cast<float*>(smd + D / 2);
     float* Qs = sm;                         // [C][D+1]
     float* Ks = Qs + kC * (D + 1);          // [C][D+1]
     float* Vs = Ks + kC * (D + 1);          // [C][DV]
@@ -38,6 +42,9 @@ linear_prefill_simt_kernel(const T* __restrict__ q, const T* __restrict__ k,
     const int h = (int)(bh % H);
     const float lam = decay[h];
     for (int n = tid; n <= kC; n += kThreads) pw[n] = (float)pow((double)lam, (double)n);
+    const bool use_rope = rope.base > 0.0;
+    if (use_rope)
+        for (int i = tid; i < D / 2; i += kThreads) turn[i] = rope_turn(rope.base, i, D);
     for (int e = tid; e < D * DV; e += kThreads) {
         const int a = e / DV, c = e % DV;
         Ss[e] = s_in ? s_in[(bh * D + a) * D + c0 + c] : 0.f;
@@ -50,11 +57,29 @@ linear_prefill_simt_kernel(const T* __restrict__ q, const T* __restrict__ k,
     for (int r0 = 0; r0 < N; r0 += kC) {
         const int len = min(kC, N - r0);
         __syncthreads();
-        for (int e = tid; e < kC * D; e += kThreads) {
-            const int t = e / D, a = e % D;
-            const bool ok = t < len;
-            Qs[t * (D + 1) + a] = ok ? to_f(qb[(int64_t)(r0 + t) * D + a]) : 0.f;
-            Ks[t * (D + 1) + a] = ok ? to_f(kb[(int64_t)(r0 + t) * D + a]) : 0.f;
+        if (use_rope) {  // rotate-half pairs (i, i + D/2) of q and k at position pos0 + row
+            for (int e = tid; e < kC * (D / 2); e += kThreads) {
+                const int t = e / (D / 2), i = e % (D / 2);
+                const bool ok = t < len;
+                const int64_t base = (int64_t)(r0 + t) * D;
+                float q0 = ok ? to_f(qb[base + i]) : 0.f, q1 = ok ? to_f(qb[base + i + D / 2]) : 0.f;
+                float k0 = ok ? to_f(kb[base + i]) : 0.f, k1 = ok ? to_f(kb[base + i + D / 2]) : 0.f;
+                float c, s;
+                rope_cs(turn[i], rope.pos0 + r0 + t, c, s);
+                rope_rot(q0, q1, c, s);
+                rope_rot(k0, k1, c, s);
+                Qs[t * (D + 1) + i] = q0;
+                Qs[t * (D + 1) + i + D / 2] = q1;
+                Ks[t * (D + 1) + i] = k0;
+                Ks[t * (D + 1) + i + D / 2] = k1;
+            }
+        } else {
+            for (int e = tid; e < kC * D; e += kThreads) {
+                const int t = e / D, a = e % D;
+                const bool ok = t < len;
+                Qs[t * (D + 1) + a] = ok ? to_f(qb[(int64_t)(r0 + t) * D + a]) : 0.f;
+                Ks[t * (D + 1) + a] = ok ? to_f(kb[(int64_t)(r0 + t) * D + a]) : 0.f;
+            }
         }
         for (int e = tid; e < kC * DV; e += kThreads) {
             const int t = e / DV, c = e % DV;
@@ -121,7 +146,8 @@ linear_prefill_simt_kernel(const T* __restrict__ q, const T* __restrict__ k,
 
 template <typename T, int D>
 cudaError_t prefill_simt(const void* q, const void* k, const void* v, const float* decay, void* o,
-                         const float* s_in, float* s_out, int B, int H, int N, cudaStream_t st) {
+                         const float* s_in, float* s_out, int B, int H, int N, Rope rope,
+                         cudaStream_t st) {
     constexpr int DV = 32;
     auto kern = linear_prefill_simt_kernel<T, D, DV>;
     const size_t smem = PrefillSmem<D, DV>::bytes;
@@ -130,7 +156,7 @@ cudaError_t prefill_simt(const void* q, const void* k, const void* v, const floa
     dim3 grid(D / DV, (unsigned)(B * H));
     kern<<<grid, kThreads, smem, st>>>(static_cast<const T*>(q), static_cast<const T*>(k),
                                        static_cast<const T*>(v), decay, static_cast<T*>(o), s_in,
-                                       s_out, H, N);
+                                       s_out, H, N, rope);
     return cudaGetLastError();
 }
 
@@ -141,7 +167,7 @@ template <typename T, int D>
 __global__ void __launch_bounds__(2 * D)
 linear_decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                      const float* __restrict__ decay, float* __restrict__ state,
-                     T* __restrict__ o, int H) {
+                     T* __restrict__ o, int H, Rope rope) {
     constexpr int kCols = 16;
     constexpr int kWarps = 2 * D / 32;
     __shared__ float red[kWarps][kCols];
@@ -150,8 +176,17 @@ linear_decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* 
     const int64_t bh = blockIdx.y;
     const int c0 = blockIdx.x * kCols + half * 8;
     const float lam = decay[bh % H];
-    const float ka = to_f(k[bh * D + a]);
-    const float qa = to_f(q[bh * D + a]);
+    float ka = to_f(k[bh * D + a]);
+    float qa = to_f(q[bh * D + a]);
+    if (rope.base > 0.0) {  // rotate-half pair (a, a +- D/2) at position pos0
+        const int i = a % (D / 2), partner = a < D / 2 ? a + D / 2 : a - D / 2;
+        const float kp = to_f(k[bh * D + partner]), qp = to_f(q[bh * D + partner]);
+        float c, s;
+        rope_cs(rope_turn(rope.base, i, D), rope.pos0, c, s);
+        if (a >= D / 2) s = -s;  // x'_hi = x_hi c + x_lo s;  x'_lo = x_lo c - x_hi s
+        ka = ka * c - kp * s;
+        qa = qa * c - qp * s;
+    }
     float vv[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) vv[j] = to_f(v[bh * D + c0 + j]);
@@ -185,11 +220,11 @@ linear_decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* 
 
 template <typename T, int D>
 cudaError_t decode_launch(const void* q, const void* k, const void* v, const float* decay,
-                          float* state, void* o, int B, int H, cudaStream_t st) {
+                          float* state, void* o, int B, int H, Rope rope, cudaStream_t st) {
     dim3 grid(D / 16, (unsigned)(B * H));
     linear_decode_kernel<T, D><<<grid, 2 * D, 0, st>>>(
         static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), decay,
-        state, static_cast<T*>(o), H);
+        state, static_cast<T*>(o), H, rope);
     return cudaGetLastError();
 }
 
@@ -197,8 +232,8 @@ cudaError_t decode_launch(const void* q, const void* k, const void* v, const flo
 
 cudaError_t launch_linear_prefill_simt(DType dt, const void* q, const void* k, const void* v,
                                        const float* decay, void* o, const float* s_in,
-                                       float* s_out, int B, int H, int N, int d, cudaStream_t st,
-                                       DevCtx) {
+                                       float* s_out, int B, int H, int N, int d, Rope rope,
+                                       cudaStream_t st, DevCtx) {
     if (N == 0) {
         // Nothing to attend to: the state passes through unchanged (or stays zero).
         if (!s_out) return cudaSuccess;
@@ -208,20 +243,20 @@ cudaError_t launch_linear_prefill_simt(DType dt, const void* q, const void* k, c
         return cudaMemsetAsync(s_out, 0, bytes, st);
     }
     if (dt == DType::F32)
-        return d == 64 ? prefill_simt<float, 64>(q, k, v, decay, o, s_in, s_out, B, H, N, st)
-                       : prefill_simt<float, 128>(q, k, v, decay, o, s_in, s_out, B, H, N, st);
-    return d == 64 ? prefill_simt<__nv_bfloat16, 64>(q, k, v, decay, o, s_in, s_out, B, H, N, st)
-                   : prefill_simt<__nv_bfloat16, 128>(q, k, v, decay, o, s_in, s_out, B, H, N, st);
+        return d == 64 ? prefill_simt<float, 64>(q, k, v, decay, o, s_in, s_out, B, H, N, rope, st)
+                       : prefill_simt<float, 128>(q, k, v, decay, o, s_in, s_out, B, H, N, rope, st);
+    return d == 64 ? prefill_simt<__nv_bfloat16, 64>(q, k, v, decay, o, s_in, s_out, B, H, N, rope, st)
+                   : prefill_simt<__nv_bfloat16, 128>(q, k, v, decay, o, s_in, s_out, B, H, N, rope, st);
 }
 
 cudaError_t launch_linear_decode(DType dt, const void* q, const void* k, const void* v,
                                  const float* decay, float* state, void* o, int B, int H, int d,
-                                 cudaStream_t st, DevCtx) {
+                                 Rope rope, cudaStream_t st, DevCtx) {
     if (dt == DType::F32)
-        return d == 64 ? decode_launch<float, 64>(q, k, v, decay, state, o, B, H, st)
-                       : decode_launch<float, 128>(q, k, v, decay, state, o, B, H, st);
-    return d == 64 ? decode_launch<__nv_bfloat16, 64>(q, k, v, decay, state, o, B, H, st)
-                   : decode_launch<__nv_bfloat16, 128>(q, k, v, decay, state, o, B, H, st);
+        return d == 64 ? decode_launch<float, 64>(q, k, v, decay, state, o, B, H, rope, st)
+                       : decode_launch<float, 128>(q, k, v, decay, state, o, B, H, rope, st);
+    return d == 64 ? decode_launch<__nv_bfloat16, 64>(q, k, v, decay, state, o, B, H, rope, st)
+                   : decode_launch<__nv_bfloat16, 128>(q, k, v, decay, state, o, B, H, rope, st);
 }
 
 }  // namespace sala

@@ -31,6 +31,7 @@
 // cannot keep four products per tile in flight).  Every wait is bounded (see ptx::mbar_wait).
 #include "kernels.h"
 #include "ptx.cuh"
+#include "rope.cuh"
 #include "tmap.cuh"
 
 namespace sala {
@@ -58,6 +59,7 @@ struct Bars {
     uint32_t tmem_base;
     int abort;
     float pw[kC + 1];  // lambda^n, n = 0..128
+    double turn[kD / 2];  // RoPE: theta_i / 2pi
 };
 
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, const DevCtx& ctx,
@@ -73,13 +75,45 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, co
 __device__ __forceinline__ float bf_lo(uint32_t x) { return __uint_as_float(x << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t x) { return __uint_as_float(x & 0xffff0000u); }
 
+// RoPE of row t of NT [128 x 128] bf16 tiles in place, each held as two 128-byte-swizzled
+// sub-tiles kSub apart (d 0-63, d 64-127), so the pair (i, i + 64) sits at the same offset in both
+// halves.  The tiles share the row's position, hence its cosines and sines.
+template <int NT>
+__device__ __forceinline__ void rope_rows(uint8_t* const (&tiles)[NT], int t, const double* turn,
+                                          int64_t pos) {
+#pragma unroll 1
+    for (int cj = 0; cj < 8; ++cj) {
+        const int off = t * 128 + ((cj ^ (t & 7)) << 4);
+        float cs[8], sn[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) rope_cs(turn[8 * cj + e], pos, cs[e], sn[e]);
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+            const uint4 a = *reinterpret_cast<const uint4*>(tiles[n] + off);
+            const uint4 b = *reinterpret_cast<const uint4*>(tiles[n] + kSub + off);
+            uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+                float x0 = bf_lo(av[w]), x1 = bf_hi(av[w]), y0 = bf_lo(bv[w]), y1 = bf_hi(bv[w]);
+                rope_rot(x0, y0, cs[2 * w], sn[2 * w]);
+                rope_rot(x1, y1, cs[2 * w + 1], sn[2 * w + 1]);
+                av[w] = pack_bf16x2(x0, x1);
+                bv[w] = pack_bf16x2(y0, y1);
+            }
+            *reinterpret_cast<uint4*>(tiles[n] + off) = make_uint4(av[0], av[1], av[2], av[3]);
+            *reinterpret_cast<uint4*>(tiles[n] + kSub + off) = make_uint4(bv[0], bv[1], bv[2], bv[3]);
+        }
+    }
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 linear_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                          const __grid_constant__ CUtensorMap tmK,
                          const __grid_constant__ CUtensorMap tmV,
                          const __grid_constant__ CUtensorMap tmO, const float* __restrict__ decay,
                          const float* s_in, float* s_out, int H,
-                         int N, int seg_len, int n_seg, int64_t s_in_seg_stride, DevCtx ctx) {
+                         int N, int seg_len, int n_seg, int64_t s_in_seg_stride, Rope rope,
+                         DevCtx ctx) {
     extern __shared__ uint8_t smraw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smraw) + 1023) &
                                              ~uintptr_t(1023));
@@ -120,7 +154,10 @@ linear_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
     {
         const double lam = (double)decay[bh % H];
         for (int n = tid; n <= kC; n += kThreads) bars.pw[n] = (float)pow(lam, (double)n);
+        if (rope.base > 0.0)
+            for (int i = tid; i < kD / 2; i += kThreads) bars.turn[i] = rope_turn(rope.base, i, kD);
     }
+    const bool use_rope = rope.base > 0.0;
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -171,6 +208,8 @@ linear_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                 auto issue_qk = [&](int c) -> bool {  // MMA1: A = Q K^T
                     const int st = c & 1;
                     if (!wait_or_abort(&bars.full[st], (c >> 1) & 1, ctx, abort)) return false;
+                    // with RoPE, Q and K are rotated in place together with V~ (v_ready)
+                    if (use_rope && !wait_or_abort(&bars.v_ready[st], (c >> 1) & 1, ctx, abort)) return false;
                     tc_fence_after();
 #pragma unroll
                     for (int ks = 0; ks < kD / 16; ++ks)
@@ -352,6 +391,10 @@ linear_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
             const int s = c & 1;
             const int len = min(kC, Ns - c * kC);
             if (!wait_or_abort(&bars.full[s], (c >> 1) & 1, ctx, abort)) return false;
+            if (use_rope) {  // row t of Q and K at position pos0 + row0 + c * kC + t
+                uint8_t* const qk[2] = {sm + s * kStageBytes + kOffQ, sm + s * kStageBytes + kOffK};
+                rope_rows<2>(qk, t, bars.turn, rope.pos0 + row0 + (int64_t)c * kC + t);
+            }
             const float w = t < len ? bars.pw[len - 1 - t] : 0.f;
             const uint8_t* vrow = sm + s * kStageBytes + kOffV + t * 128;
             uint8_t* vtrow = sm + kOffVt + t * 128;
@@ -437,12 +480,13 @@ struct StBars {
     uint32_t tmem_base;
     int abort;
     float pw[kC + 1];
+    double turn[kD / 2];  // RoPE: theta_i / 2pi
 };
 
 __global__ void __launch_bounds__(kStThreads, 1)
 linear_state_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                        const float* __restrict__ decay, float* __restrict__ s_seg, int H, int N,
-                       int seg_len, int n_seg, int64_t seg_stride, DevCtx ctx) {
+                       int seg_len, int n_seg, int64_t seg_stride, Rope rope, DevCtx ctx) {
     extern __shared__ uint8_t smraw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smraw) + 1023) &
                                              ~uintptr_t(1023));
@@ -476,6 +520,8 @@ linear_state_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
     {
         const double lam = (double)decay[bh % H];
         for (int n = tid; n <= kC; n += kStThreads) bars.pw[n] = (float)pow(lam, (double)n);
+        if (rope.base > 0.0)
+            for (int i = tid; i < kD / 2; i += kStThreads) bars.turn[i] = rope_turn(rope.base, i, kD);
     }
     tc_fence_before();
     __syncthreads();
@@ -535,6 +581,10 @@ linear_state_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
             const int s = c % kStStages;
             const int len = min(kC, Ns - c * kC);
             if (!wait_or_abort(&bars.full[s], (c / kStStages) & 1, ctx, abort)) return false;
+            if (rope.base > 0.0) {  // row t of K at position pos0 + row0 + c * kC + t
+                uint8_t* const kt[1] = {sm + s * kStStage};
+                rope_rows<1>(kt, t, bars.turn, rope.pos0 + row0 + (int64_t)c * kC + t);
+            }
             const float w = t < len ? bars.pw[len - 1 - t] : 0.f;
             const uint8_t* vrow = sm + s * kStStage + 2 * kSub + t * 128;
             uint8_t* vtrow = sm + kStOffVt + (c & 1) * kSub + t * 128;
@@ -678,7 +728,7 @@ size_t linear_prefill_tc_workspace(int B, int H, int N, int d) {
 cudaError_t launch_linear_prefill_tc(const void* q, const void* k, const void* v,
                                      const float* decay, void* o, const float* s_in,
                                      float* s_out, int B, int H, int N, int d, void* ws,
-                                     size_t ws_bytes, cudaStream_t st, DevCtx ctx) {
+                                     size_t ws_bytes, Rope rope, cudaStream_t st, DevCtx ctx) {
     if (d != kD) return cudaErrorNotSupported;
     EncodeTiledFn fn = encode_tiled_fn();
     if (!fn) return cudaErrorNotSupported;
@@ -704,7 +754,7 @@ cudaError_t launch_linear_prefill_tc(const void* q, const void* k, const void* v
         e = ensure_smem<linear_state_tc_kernel>(kStSmem);
         if (e != cudaSuccess) return e;
         linear_state_tc_kernel<<<B * H * n_seg * kSlices, kStThreads, kStSmem, st>>>(
-            tmK, tmV, decay, s_seg, H, N, seg_len, n_seg, seg_stride, ctx);
+            tmK, tmV, decay, s_seg, H, N, seg_len, n_seg, seg_stride, rope, ctx);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
         const int64_t elems = seg_stride;
@@ -713,13 +763,13 @@ cudaError_t launch_linear_prefill_tc(const void* q, const void* k, const void* v
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
         linear_prefill_tc_kernel<<<B * H * n_seg * kSlices, kThreads, kSmemBytes, st>>>(
-            tmQ, tmK, tmV, tmO, decay, s_seg, nullptr, H, N, seg_len, n_seg, seg_stride, ctx);
+            tmQ, tmK, tmV, tmO, decay, s_seg, nullptr, H, N, seg_len, n_seg, seg_stride, rope, ctx);
         return cudaGetLastError();
     }
     // One segment.  If state_out aliases state_in, every CTA reads its slice before it writes it
     // back, and no two CTAs share a slice, so in-place update is safe.
     linear_prefill_tc_kernel<<<B * H * kSlices, kThreads, kSmemBytes, st>>>(
-        tmQ, tmK, tmV, tmO, decay, s_in, s_out, H, N, N, 1, 0, ctx);
+        tmQ, tmK, tmV, tmO, decay, s_in, s_out, H, N, N, 1, 0, rope, ctx);
     return cudaGetLastError();
 }
 

@@ -31,6 +31,9 @@ _lib.sala_linear_prefill_ws.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _
 _lib.sala_linear_prefill_workspace.argtypes = [_i, _i, _i, _i, _i]
 _lib.sala_linear_prefill_workspace.restype = ctypes.c_size_t
 _lib.sala_linear_decode.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp]
+_lib.sala_linear_prefill_rope.argtypes = [_vp] * 7 + [_i] * 4 + [ctypes.c_int64, ctypes.c_double,
+                                                              _vp, _st, _i, _vp]
+_lib.sala_linear_decode_rope.argtypes = [_vp] * 6 + [_i] * 3 + [ctypes.c_int64, ctypes.c_double, _i, _vp]
 _lib.sala_block_compress.argtypes = [_vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp]
 _lib.sala_block_topk.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp,
                                  _st, _i, _vp]
@@ -48,7 +51,8 @@ _lib.sala_status_string.restype = ctypes.c_char_p
 _lib.sala_last_error.restype = ctypes.c_char_p
 _lib.sala_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
 _lib.sala_selftest_wait_timeout.argtypes = [_vp]
-for _f in ("sala_linear_prefill", "sala_linear_decode", "sala_block_compress", "sala_block_topk",
+for _f in ("sala_linear_prefill", "sala_linear_decode", "sala_linear_prefill_rope",
+           "sala_linear_decode_rope", "sala_block_compress", "sala_block_topk",
            "sala_sparse_prefill", "sala_sparse_decode", "sala_check_status",
            "sala_selftest_wait_timeout"):
     getattr(_lib, _f).restype = _i
@@ -102,11 +106,12 @@ def linear_prefill_workspace_bytes(B, H, N, d, dtype=torch.bfloat16):
 
 
 def linear_prefill(q, k, v, decay, o=None, state_in=None, state_out=None, chunk=0, workspace=None,
-                   stream=None):
+                   stream=None, rope_base=None, pos0=0):
     """Chunked decayed linear attention.  q,k,v: [B,H,N,d]; decay [H] fp32.  Returns o.
     workspace: None = one pass (sala_linear_prefill); a uint8 device tensor of at least
     linear_prefill_workspace_bytes(...) bytes lets long sequences run as parallel segments
-    (sala_linear_prefill_ws)."""
+    (sala_linear_prefill_ws).  rope_base: rotate q and k by position first, row r at pos0 + r
+    (sala_linear_prefill_rope; chunk is then the kernel's own)."""
     B, H, N, d = q.shape
     _need(q, "q"); _need(k, "k", q.shape, q.dtype); _need(v, "v", q.shape, q.dtype)
     _need(decay, "decay", (H,), torch.float32)
@@ -115,7 +120,13 @@ def linear_prefill(q, k, v, decay, o=None, state_in=None, state_out=None, chunk=
     _need(o, "o", q.shape, q.dtype)
     _need(state_in, "state_in", (B, H, d, d), torch.float32)
     _need(state_out, "state_out", (B, H, d, d), torch.float32)
-    if workspace is None:
+    if rope_base is not None:
+        _check(_lib.sala_linear_prefill_rope(_ptr(q), _ptr(k), _ptr(v), _ptr(decay), _ptr(o),
+                                             _ptr(state_in), _ptr(state_out), B, H, N, d, int(pos0),
+                                             float(rope_base), _ptr(workspace),
+                                             0 if workspace is None else workspace.numel(), _dt(q),
+                                             _stream(stream)), "sala_linear_prefill_rope")
+    elif workspace is None:
         _check(_lib.sala_linear_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(decay), _ptr(o),
                                         _ptr(state_in), _ptr(state_out), B, H, N, d, chunk, _dt(q),
                                         _stream(stream)), "sala_linear_prefill")
@@ -127,8 +138,9 @@ def linear_prefill(q, k, v, decay, o=None, state_in=None, state_out=None, chunk=
     return o
 
 
-def linear_decode(q, k, v, decay, state, o=None, stream=None):
-    """One decode step.  q,k,v: [B,H,d]; state [B,H,d,d] fp32 (updated in place).  Returns o."""
+def linear_decode(q, k, v, decay, state, o=None, stream=None, rope_base=None, pos=0):
+    """One decode step.  q,k,v: [B,H,d]; state [B,H,d,d] fp32 (updated in place).  Returns o.
+    rope_base: rotate q and k at position pos first (sala_linear_decode_rope)."""
     B, H, d = q.shape
     _need(q, "q"); _need(k, "k", q.shape, q.dtype); _need(v, "v", q.shape, q.dtype)
     _need(decay, "decay", (H,), torch.float32)
@@ -136,6 +148,11 @@ def linear_decode(q, k, v, decay, state, o=None, stream=None):
     if o is None:
         o = torch.empty_like(q)
     _need(o, "o", q.shape, q.dtype)
+    if rope_base is not None:
+        _check(_lib.sala_linear_decode_rope(_ptr(q), _ptr(k), _ptr(v), _ptr(decay), _ptr(state),
+                                            _ptr(o), B, H, d, int(pos), float(rope_base), _dt(q),
+                                            _stream(stream)), "sala_linear_decode_rope")
+        return o
     _check(_lib.sala_linear_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(decay), _ptr(state), _ptr(o),
                                    B, H, d, _dt(q), _stream(stream)), "sala_linear_decode")
     return o

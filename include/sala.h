@@ -102,6 +102,34 @@ sala_status sala_linear_decode(const void* q, const void* k, const void* v, cons
                                float* state, void* o, int B, int H, int d, sala_dtype dt,
                                sala_stream stream);
 
+/* The linear layers of the hybrid rotate queries and keys by position before the linear
+ * attention (HyPE: MiniCPM-SALA summaries, JA section 2.2 "positional encoding (HyPE)", DE
+ * section 2 "HyPE" -- rotary embeddings in the linear layers, none in the sparse layers).  The
+ * pages give no RoPE parameters; these calls take the rotate-half form: element i is paired with
+ * element i + d/2 (i < d/2), theta_i = rope_base^(-2i/d), and at position p
+ *   x'_i = x_i cos(p theta_i) - x_{i+d/2} sin(p theta_i)
+ *   x'_{i+d/2} = x_{i+d/2} cos(p theta_i) + x_i sin(p theta_i)
+ * for x = q and x = k (not v), then the linear attention above.  The rotation is fused into the
+ * kernels' load path (the rotated q and k are never written to memory); on the bf16 tensor-core
+ * path the rotated values are rounded to bf16 for the products.
+ * pos0      : position of row 0 (a continuation after state_out of an earlier call passes the
+ *             number of rows already processed); >= 0.
+ * rope_base : > 1 and < 1e30 (the usual value is 10000).
+ * workspace : as sala_linear_prefill_ws (NULL or too small: one pass).
+ * Other arguments, validation and errors are those of sala_linear_prefill (chunk: the kernel's
+ * own). */
+sala_status sala_linear_prefill_rope(const void* q, const void* k, const void* v,
+                                     const float* decay, void* o, const float* state_in,
+                                     float* state_out, int B, int H, int N, int d, int64_t pos0,
+                                     double rope_base, void* workspace, size_t workspace_bytes,
+                                     sala_dtype dt, sala_stream stream);
+
+/* sala_linear_decode with q and k rotated at position pos (>= 0), as sala_linear_prefill_rope. */
+sala_status sala_linear_decode_rope(const void* q, const void* k, const void* v,
+                                    const float* decay, float* state, void* o, int B, int H,
+                                    int d, int64_t pos, double rope_base, sala_dtype dt,
+                                    sala_stream stream);
+
 /* ------------------------------------------------------------------------------------------
  * Block compression of the keys of a sparse layer (mean pooling).  Pages: InfLLM-V2 selects
  * the relevant context parts without extra parameters (JA technical summary section 2.1); the

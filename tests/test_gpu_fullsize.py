@@ -63,3 +63,24 @@ def test_linear_layer_full_size():
                                   rows=rows)
     got = np.stack([oracle.from_tensor(o[0, heads[hi], t]) for hi, t in rows])
     assert_close(got, ref, "bf16", "linear N=262144 sampled rows")
+
+
+def test_linear_rope_layer_full_size():
+    # the RoPE linear layer at N = 262144 in the launch configuration the benchmark times
+    # (parallel segments), sampled rows against the oracle's quadratic form on rotated q, k
+    from hybrid_sparse_linear_b200 import sala, synth
+    N, H, d = 262144, 32, 128
+    q, k, v = synth.linear_layer(1, H, N, d, torch.bfloat16, "cuda", layer=2)
+    lam = synth.decays(H).cuda()
+    ws = torch.empty(max(sala.linear_prefill_workspace_bytes(1, H, N, d), 16), dtype=torch.uint8,
+                     device="cuda")
+    o = sala.linear_prefill(q, k, v, lam, workspace=ws, rope_base=10000.0, pos0=0)
+    sala.check_status()
+    heads = [0, 21]
+    toks = [0, 1, 127, 128, 16383, 16384, 131071, N - 129, N - 1]
+    sub = lambda t: oracle.from_tensor(t[:, heads])
+    rows = np.array([[hi, t] for hi in range(len(heads)) for t in toks])
+    ref = oracle.linear_quadratic(oracle.rope(sub(q), 0), oracle.rope(sub(k), 0), sub(v),
+                                  oracle.from_tensor(lam.cpu()[heads]), rows=rows)
+    got = np.stack([oracle.from_tensor(o[0, heads[hi], t]) for hi, t in rows])
+    assert_close(got, ref, "bf16", "RoPE linear N=262144 sampled rows")

@@ -181,3 +181,72 @@ def test_prefill_workspace_size_contract(sala):
     assert sala.linear_prefill_workspace_bytes(1, 32, 32768, 128, torch.float32) == 0
     n = sala.linear_prefill_workspace_bytes(1, 32, 32768, 128)
     assert n > 0 and n % (32 * 128 * 128 * 4) == 0
+
+
+# ---------------------------------------------------------------------------------------------
+# RoPE (the linear layers' half of HyPE): sala_linear_prefill_rope / sala_linear_decode_rope
+
+@pytest.mark.parametrize("d,N,B,H,pos0,ws,dtype", [
+    (128, 333, 2, 3, 0, False, torch.bfloat16),        # tensor cores, one pass, ragged tail
+    (128, 5000, 1, 4, 1234, True, torch.bfloat16),     # tensor cores, parallel segments
+    (128, 130, 1, 2, 2 ** 20 + 5, True, torch.bfloat16),  # positions past 2^20
+    (64, 200, 1, 4, 77, False, torch.bfloat16),        # CUDA cores, bf16
+    (64, 150, 2, 2, 9, False, torch.float32),          # CUDA cores, fp32
+])
+def test_rope_prefill_with_state(sala, d, N, B, H, pos0, ws, dtype):
+    from hybrid_sparse_linear_b200 import synth
+    q, k, v = _inputs(B, H, N, d, dtype, 300 + N)
+    lam = synth.decays(H)
+    g = torch.Generator().manual_seed(6)
+    s_in = torch.randn((B, H, d, d), generator=g) / d
+    so = torch.empty((B, H, d, d), device="cuda")
+    work = None
+    if ws:
+        nbytes = sala.linear_prefill_workspace_bytes(B, H, N, d)
+        work = torch.full((max(nbytes, 16),), 0xFF, dtype=torch.uint8, device="cuda")
+    o = sala.linear_prefill(q.cuda(), k.cuda(), v.cuda(), lam.cuda(), state_in=s_in.cuda(),
+                            state_out=so, workspace=work, rope_base=10000.0, pos0=pos0)
+    sala.check_status()
+    ref, s_ref = oracle.linear_chunked_rope(_f64(q), _f64(k), _f64(v), _f64(lam), 64, pos0=pos0,
+                                            s_in=_f64(s_in))
+    kind = "bf16" if dtype == torch.bfloat16 else "f32"
+    assert_close(_f64(o), ref, kind, "o")
+    assert_close(_f64(so), s_ref, kind, "state_out")
+
+
+def test_rope_decode_continues_prefill(sala):
+    # decode at position P + N - 1 from the rotated prefill's state reproduces that prefill row
+    from hybrid_sparse_linear_b200 import synth
+    B, H, N, d, P = 1, 4, 129, 128, 4000
+    q, k, v = _inputs(B, H, N, d, torch.bfloat16, 51)
+    lam = synth.decays(H).cuda()
+    S = torch.empty((B, H, d, d), device="cuda")
+    o_pre = sala.linear_prefill(q.cuda(), k.cuda(), v.cuda(), lam, rope_base=10000.0, pos0=P)
+    sala.linear_prefill(q[:, :, :-1].contiguous().cuda(), k[:, :, :-1].contiguous().cuda(),
+                        v[:, :, :-1].contiguous().cuda(), lam, state_out=S, rope_base=10000.0,
+                        pos0=P)
+    o_dec = sala.linear_decode(q[:, :, -1].contiguous().cuda(), k[:, :, -1].contiguous().cuda(),
+                               v[:, :, -1].contiguous().cuda(), lam, S, rope_base=10000.0,
+                               pos=P + N - 1)
+    sala.check_status()
+    ref, _ = oracle.linear_chunked_rope(_f64(q), _f64(k), _f64(v), _f64(lam.cpu()), 64, pos0=P)
+    assert_close(_f64(o_pre), ref, "bf16", "rope prefill")
+    assert_close(_f64(o_dec), ref[:, :, -1], "bf16", "rope decode row")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_rope_decode_fp32(sala, d):
+    from hybrid_sparse_linear_b200 import synth
+    B, H, pos = 2, 3, 123457
+    lam = synth.decays(H)
+    g = torch.Generator().manual_seed(8)
+    S0 = (torch.randn((B, H, d, d), generator=g) / d).float()
+    q, k, v = (x[:, :, 0].contiguous() for x in _inputs(B, H, 1, d, torch.float32, 61))
+    S = S0.cuda().clone()
+    o = sala.linear_decode(q.cuda(), k.cuda(), v.cuda(), lam.cuda(), S, rope_base=500000.0, pos=pos)
+    sala.check_status()
+    rq = oracle.rope(_f64(q)[:, :, None], pos, 500000.0)[:, :, 0]
+    rk = oracle.rope(_f64(k)[:, :, None], pos, 500000.0)[:, :, 0]
+    o_ref, s_ref = oracle.linear_decode(rq, rk, _f64(v), _f64(lam), _f64(S0))
+    assert_close(_f64(o), o_ref, "f32", "rope decode o")
+    assert_close(_f64(S), s_ref, "f32", "rope decode state")

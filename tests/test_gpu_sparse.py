@@ -161,10 +161,11 @@ def test_sparse_decode(sala, T):
     _decode_case(sala, T, 16, 1, 2, torch.bfloat16, 6)
 
 
-@pytest.mark.parametrize("T,topk", [(64 * 700 + 9, 64), (64 * 120, 100)])
+@pytest.mark.parametrize("T,topk", [(64 * 700 + 9, 64), (64 * 95, 100)])
 def test_sparse_decode_batched(sala, T, topk):
     # B = 3 sequences at one position: every (sequence, KV group) selects and attends on its own;
-    # k = 100 takes the four-launch path.
+    # k = 100 (past the one-launch kernel; accepted while every candidate is taken, here 92 of
+    # them) takes the four-launch path.
     _decode_case(sala, T, topk, 1, 2, torch.bfloat16, 12, B=3)
 
 
