@@ -25,10 +25,12 @@
 // The bf16 state copy is double-buffered: Sb(c) lives in buffer (c+1)&1, MMA3(c) reads Sb(c-1)
 // from buffer c&1 and releases it through sb_free[c&1]; with one barrier per buffer no barrier
 // can run two phases ahead of its waiter.
-// Roles (352 threads): warps 0-3 "EPI-A" (mask + output, thread = row = TMEM lane), warps 4-7
+// Roles (512 threads): warps 0-3 "EPI-A" (mask + output, thread = row = TMEM lane), warps 4-7
 // "EPI-S" (V~ + state, thread = row of S), warp 8 TMA producer (2-stage ring of Q/K/V tiles),
 // warp 9 TMEM owner and issuer of MMA1/MMA2, warp 10 issuer of MMA3/MMA4 (one issuing thread
-// cannot keep four products per tile in flight).  Every wait is bounded (see ptx::mbar_wait).
+// cannot keep four products per tile in flight), warp 11 idle, warps 12-15 RoPE (with a rotary
+// embedding: each stage's Q and K rotated in place, thread = row, before the stage's MMAs).
+// Every wait is bounded (see ptx::mbar_wait).
 #include "kernels.h"
 #include "ptx.cuh"
 #include "rope.cuh"
@@ -40,7 +42,12 @@ namespace {
 using namespace ptx;
 
 constexpr int kD = 128, kC = 128, kDv = 64, kSlices = kD / kDv;
-constexpr int kThreads = 352;
+constexpr int kThreads = 512;
+// Register split (setmaxnreg): the mask/output and V~/state warpgroups hold wide TMEM rows; the
+// producer/issuer warpgroup and the RoPE warpgroup need little.  256 * 168 + 256 * 88 = 512 * 128,
+// the per-thread count the block is launched with.
+constexpr int kRegsLaunch = 128, kRegsEpi = 168, kRegsOther = 88;
+static_assert(256 * kRegsEpi + 256 * kRegsOther == kThreads * kRegsLaunch, "register split");
 constexpr int kSub = kC * 128;                    // one [128 rows x 128 B] sub-tile: 16 KiB
 constexpr int kOffQ = 0, kOffK = 2 * kSub, kOffV = 4 * kSub;
 constexpr int kStageBytes = 5 * kSub;             // Q (2) + K (2) + V slice (1)
@@ -55,6 +62,7 @@ constexpr uint32_t kColA0 = 0, kColO1 = 256, kColO2 = 320, kColDS = 384, kTmemCo
 struct Bars {
     uint64_t full[2], empty[2];
     uint64_t qk_done[2], a_ready[2], v_ready[2], ds_done[2], s_ready[2], sb_free[2];
+    uint64_t rot_ready[2];  // RoPE: Q and K of the stage rotated in place
     uint64_t o_done, o_free, fin;
     uint32_t tmem_base;
     int abort;
@@ -75,18 +83,38 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, co
 __device__ __forceinline__ float bf_lo(uint32_t x) { return __uint_as_float(x << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t x) { return __uint_as_float(x & 0xffff0000u); }
 
-// RoPE of row t of NT [128 x 128] bf16 tiles in place, each held as two 128-byte-swizzled
-// sub-tiles kSub apart (d 0-63, d 64-127), so the pair (i, i + 64) sits at the same offset in both
-// halves.  The tiles share the row's position, hence its cosines and sines.
+// RoPE of row t (lane = t % 32) of NT [128 x 128] bf16 tiles in place, each held as two
+// 128-byte-swizzled sub-tiles kSub apart (d 0-63, d 64-127), so the pair (i, i + 64) sits at the
+// same offset in both halves.  The tile's rows sit at positions p0 + t and share frequencies: each
+// lane reduces p0 * theta_j / 2pi to a fraction of a turn in double precision for j = lane and
+// j = lane + 32, the warp shares them by shuffles, and row t adds t * theta_j / 2pi (at most ~21
+// turns, exact to ~2e-6 turns) in single precision before the final reduction and sine/cosine.
 template <int NT>
-__device__ __forceinline__ void rope_rows(uint8_t* const (&tiles)[NT], int t, const double* turn,
-                                          int64_t pos) {
+__device__ __forceinline__ void rope_rows(uint8_t* const (&tiles)[NT], int t, int lane,
+                                          const double* turn, int64_t p0) {
+    float fa, fb, ta, tb;
+    {
+        double x = (double)p0 * turn[lane];
+        double y = (double)p0 * turn[lane + 32];
+        fa = (float)(x - rint(x));
+        fb = (float)(y - rint(y));
+        ta = (float)turn[lane];
+        tb = (float)turn[lane + 32];
+    }
+    const float tr = (float)t;
 #pragma unroll 1
     for (int cj = 0; cj < 8; ++cj) {
         const int off = t * 128 + ((cj ^ (t & 7)) << 4);
         float cs[8], sn[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) rope_cs(turn[8 * cj + e], pos, cs[e], sn[e]);
+        for (int e = 0; e < 8; ++e) {
+            const int j = 8 * cj + e;  // frequency index
+            const float f0 = __shfl_sync(0xffffffffu, j < 32 ? fa : fb, j & 31);
+            const float tj = __shfl_sync(0xffffffffu, j < 32 ? ta : tb, j & 31);
+            float x = fmaf(tr, tj, f0);
+            x -= rintf(x);
+            __sincosf(x * 6.28318530717958647f, &sn[e], &cs[e]);
+        }
 #pragma unroll
         for (int n = 0; n < NT; ++n) {
             const uint4 a = *reinterpret_cast<const uint4*>(tiles[n] + off);
@@ -144,6 +172,7 @@ linear_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
             mbar_init(&bars.ds_done[b], 1);
             mbar_init(&bars.s_ready[b], 4);
             mbar_init(&bars.sb_free[b], 1);
+            mbar_init(&bars.rot_ready[b], 4);
         }
         mbar_init(&bars.o_done, 2);  // O1 (warp 9) and O2 (warp 10)
         mbar_init(&bars.o_free, 4);
@@ -162,7 +191,10 @@ linear_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = bars.tmem_base;
-
+    // Each warpgroup changes its register count at the top of its own role branch (ptxas then
+    // allocates the branch within the new count).
+    if (warp >= 8 && warp < 12) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsOther));
     if (warp == 8) {
         // ------------------------------------------------------------------ TMA producer
         if (lane == 0) {
@@ -208,8 +240,8 @@ linear_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                 auto issue_qk = [&](int c) -> bool {  // MMA1: A = Q K^T
                     const int st = c & 1;
                     if (!wait_or_abort(&bars.full[st], (c >> 1) & 1, ctx, abort)) return false;
-                    // with RoPE, Q and K are rotated in place together with V~ (v_ready)
-                    if (use_rope && !wait_or_abort(&bars.v_ready[st], (c >> 1) & 1, ctx, abort)) return false;
+                    // with RoPE, Q and K of the stage are rotated in place first
+                    if (use_rope && !wait_or_abort(&bars.rot_ready[st], (c >> 1) & 1, ctx, abort)) return false;
                     tc_fence_after();
 #pragma unroll
                     for (int ks = 0; ks < kD / 16; ++ks)
@@ -242,6 +274,8 @@ linear_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                     const int st = c & 1;
                     if (!wait_or_abort(&bars.full[st], (c >> 1) & 1, ctx, abort)) return false;
                     if (!wait_or_abort(&bars.v_ready[st], (c >> 1) & 1, ctx, abort)) return false;
+                    // with RoPE, Q (MMA3) and K (MMA4) of the stage rotated in place first
+                    if (use_rope && !wait_or_abort(&bars.rot_ready[st], (c >> 1) & 1, ctx, abort)) return false;
                     tc_fence_after();
                     const uint32_t vt_lo = vt_lo0;
 #pragma unroll
@@ -274,8 +308,26 @@ linear_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
             (void)mbar_wait(&bars.fin, 0, ctx);
         }
         __syncwarp();
+    }  // warp 11: idle
+    } else if (warp >= 12) {
+        // ------------------------------------------------------------------ RoPE of Q and K
+        // thread = row of the tile; each stage's Q and K rotated in place before its MMAs
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsOther));
+        if (use_rope) {
+            const int t = tid - 384;
+            for (int c = 0; c < n_tiles; ++c) {
+                const int s = c & 1;
+                if (!wait_or_abort(&bars.full[s], (c >> 1) & 1, ctx, abort)) break;
+                uint8_t* const qk[2] = {sm + s * kStageBytes + kOffQ, sm + s * kStageBytes + kOffK};
+                rope_rows<2>(qk, t, lane, bars.turn, rope.pos0 + row0 + (int64_t)c * kC);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars.rot_ready[s]);
+            }
+        }
     } else if (warp < 4) {
         // ------------------------------------------------------------------ EPI-A: mask, output
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsEpi));
         const int t = tid;
         const uint32_t lb = tmem_lane_base(warp);
         const float wq = bars.pw[t + 1];
@@ -359,6 +411,7 @@ linear_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
         if (lane == 0) bulk_wait0();  // this warp's stores complete before the CTA retires
     } else if (warp < 8) {
         // ------------------------------------------------------------------ EPI-S: V~, state
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsEpi));
         const int t = tid - 128;  // row of the V tile / of the state slice
         const uint32_t lb = tmem_lane_base(warp);
         float S[kDv];
@@ -391,10 +444,6 @@ linear_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
             const int s = c & 1;
             const int len = min(kC, Ns - c * kC);
             if (!wait_or_abort(&bars.full[s], (c >> 1) & 1, ctx, abort)) return false;
-            if (use_rope) {  // row t of Q and K at position pos0 + row0 + c * kC + t
-                uint8_t* const qk[2] = {sm + s * kStageBytes + kOffQ, sm + s * kStageBytes + kOffK};
-                rope_rows<2>(qk, t, bars.turn, rope.pos0 + row0 + (int64_t)c * kC + t);
-            }
             const float w = t < len ? bars.pw[len - 1 - t] : 0.f;
             const uint8_t* vrow = sm + s * kStageBytes + kOffV + t * 128;
             uint8_t* vtrow = sm + kOffVt + t * 128;
@@ -465,16 +514,17 @@ linear_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
 // output pass above on every segment at once.  K and V are read twice, but every SM has work.
 //
 // State pass, per CTA = (batch*head, segment, value slice): warp 4 streams K and the V slice
-// through a 3-stage ring, warp 5 issues dS = K^T V~ per tile into one of two TMEM buffers, and
-// warps 0-3 (thread = row of S) write V~ and fold dS into the fp32 state held in registers.
+// through a 3-stage ring, warp 5 issues dS = K^T V~ per tile into one of two TMEM buffers,
+// warps 0-3 (thread = row of S) write V~ and fold dS into the fp32 state held in registers, and
+// with RoPE warps 6-9 rotate each stage's K in place (thread = row of the tile).
 constexpr int kStStages = 3;
 constexpr int kStStage = 3 * kSub;                     // K (2 sub-tiles) + V slice (1)
 constexpr int kStOffVt = kStStages * kStStage;         // V~, 2 buffers
 constexpr int kStSmem = kStOffVt + 2 * kSub + 1024;
-constexpr int kStThreads = 192;
+constexpr int kStThreads = 320;  // warps 6-9 rotate K when RoPE is on (idle otherwise)
 
 struct StBars {
-    uint64_t full[kStStages], empty[kStStages];
+    uint64_t full[kStStages], empty[kStStages], rot_ready[kStStages];
     uint64_t v_ready[2], ds_done[2], ds_free[2];
     uint64_t fin;
     uint32_t tmem_base;
@@ -507,6 +557,7 @@ linear_state_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
         for (int s = 0; s < kStStages; ++s) {
             mbar_init(&bars.full[s], 1);
             mbar_init(&bars.empty[s], 1);
+            mbar_init(&bars.rot_ready[s], 4);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&bars.v_ready[b], 4);
@@ -555,6 +606,7 @@ linear_state_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
                 const int s = c % kStStages, b = c & 1;
                 if (!wait_or_abort(&bars.full[s], (c / kStStages) & 1, ctx, abort)) break;
                 if (!wait_or_abort(&bars.v_ready[b], (c >> 1) & 1, ctx, abort)) break;
+                if (rope.base > 0.0 && !wait_or_abort(&bars.rot_ready[s], (c / kStStages) & 1, ctx, abort)) break;
                 if (c >= 2 && !wait_or_abort(&bars.ds_free[b], ((c - 2) >> 1) & 1, ctx, abort)) break;
                 tc_fence_after();
                 const uint32_t k = smem_u32(sm + s * kStStage);
@@ -570,6 +622,21 @@ linear_state_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
             (void)mbar_wait(&bars.fin, 0, ctx);
         }
         __syncwarp();
+    } else if (warp >= 6) {
+        // ---------------------------------------------------------------- RoPE of K
+        // thread = row of the K tile; each stage's K rotated in place before its MMA
+        if (rope.base > 0.0) {
+            const int t = tid - 192;
+            for (int c = 0; c < n_tiles; ++c) {
+                const int s = c % kStStages;
+                if (!wait_or_abort(&bars.full[s], (c / kStStages) & 1, ctx, abort)) break;
+                uint8_t* const kt[1] = {sm + s * kStStage};
+                rope_rows<1>(kt, t, lane, bars.turn, rope.pos0 + row0 + (int64_t)c * kC);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars.rot_ready[s]);
+            }
+        }
     } else {
         // ---------------------------------------------------------------- V~ and the state
         const int t = tid;  // row of the V tile / of the state slice
@@ -581,10 +648,6 @@ linear_state_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
             const int s = c % kStStages;
             const int len = min(kC, Ns - c * kC);
             if (!wait_or_abort(&bars.full[s], (c / kStStages) & 1, ctx, abort)) return false;
-            if (rope.base > 0.0) {  // row t of K at position pos0 + row0 + c * kC + t
-                uint8_t* const kt[1] = {sm + s * kStStage};
-                rope_rows<1>(kt, t, bars.turn, rope.pos0 + row0 + (int64_t)c * kC + t);
-            }
             const float w = t < len ? bars.pw[len - 1 - t] : 0.f;
             const uint8_t* vrow = sm + s * kStStage + 2 * kSub + t * 128;
             uint8_t* vtrow = sm + kStOffVt + (c & 1) * kSub + t * 128;
@@ -746,6 +809,16 @@ cudaError_t launch_linear_prefill_tc(const void* q, const void* k, const void* v
         return cudaErrorInvalidValue;
     cudaError_t e = ensure_smem<linear_prefill_tc_kernel>(kSmemBytes);
     if (e != cudaSuccess) return e;
+    // setmaxnreg.inc waits until the block's pool holds the registers: launch only when the
+    // compiled per-thread count (the pool is that count times the threads) covers the split.
+    static int regs_ok = -1;
+    if (regs_ok < 0) {
+        cudaFuncAttributes fa;
+        e = cudaFuncGetAttributes(&fa, linear_prefill_tc_kernel);
+        if (e != cudaSuccess) return e;
+        regs_ok = fa.numRegs * kThreads >= 256 * kRegsEpi + 256 * kRegsOther ? 1 : 0;
+    }
+    if (!regs_ok) return cudaErrorNotSupported;
     int n_seg, seg_len;
     pick_segments(B, H, N, &n_seg, &seg_len);
     const int64_t seg_stride = (int64_t)B * H * kD * kD;
