@@ -194,121 +194,121 @@ linear_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
     // Each warpgroup changes its register count at the top of its own role branch (ptxas then
     // allocates the branch within the new count).
     if (warp >= 8 && warp < 12) {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsOther));
-    if (warp == 8) {
-        // ------------------------------------------------------------------ TMA producer
-        if (lane == 0) {
-            int issued[2] = {-1, -1};
-            for (int c = 0; c < n_tiles; ++c) {
-                const int s = c & 1, r = c >> 1;
-                if (r >= 1 && !wait_or_abort(&bars.empty[s], (r - 1) & 1, ctx, abort)) break;
-                uint8_t* st = sm + s * kStageBytes;
-                mbar_arrive_expect_tx(&bars.full[s], kStageBytes);
-                const int y = row0 + c * kC, z = (int)bh;
-                tma_load_3d(st + kOffQ, &tmQ, &bars.full[s], 0, y, z);
-                tma_load_3d(st + kOffQ + kSub, &tmQ, &bars.full[s], 64, y, z);
-                tma_load_3d(st + kOffK, &tmK, &bars.full[s], 0, y, z);
-                tma_load_3d(st + kOffK + kSub, &tmK, &bars.full[s], 64, y, z);
-                tma_load_3d(st + kOffV, &tmV, &bars.full[s], slice * kDv, y, z);
-                issued[s] = r;
-            }
-            for (int s = 0; s < 2; ++s)
-                if (issued[s] >= 0) (void)mbar_wait(&bars.full[s], issued[s] & 1, ctx);
-        }
-        __syncwarp();
-    } else if (warp == 9 || warp == 10) {
-        // ------------------------------------------------------------------ MMA issuers
-        // Two issuing threads, so that one thread's issue latency does not serialise the four
-        // products: warp 9 issues the attention path (MMA1, MMA2), warp 10 the state path (MMA3,
-        // MMA4).  Each commits its own share of the stage release, of o_done and of fin.  The
-        // shared-memory descriptors are kept as 32-bit halves; a K-step adds to the low half.
-        if (lane == 0) {
-            const uint32_t hi = sdesc_sw128_hi(1024);
-            // Low halves for stage 0; stage st adds st * kStageBytes / 16 to the address field.
-            const uint32_t base = smem_u32(sm);
-            const uint32_t q_lo0 = sdesc_sw128_lo(base + kOffQ, 16);
-            const uint32_t k_lo0 = sdesc_sw128_lo(base + kOffK, 16);
-            const uint32_t kt_lo0 = sdesc_sw128_lo(base + kOffK, kSub);  // K read transposed (MMA4)
-            const uint32_t v_lo0 = sdesc_sw128_lo(base + kOffV, 8192);
-            auto at_stage = [](uint32_t lo, int st) -> uint32_t { return lo + (uint32_t)(st * (kStageBytes >> 4)); };
-            // K-major operand [128 x 128] in two 64-column sub-tiles: K-step ks starts at
-            // sub-tile ks / 4, byte 32 (ks % 4) of its rows.
-            auto kstep = [](int ks) -> uint32_t { return (uint32_t)(((ks >> 2) * kSub + (ks & 3) * 32) >> 4); };
-            if (warp == 9) {
-                const uint32_t idQK = idesc_bf16_f32(128, 128, false, false);
-                const uint32_t idO = idesc_bf16_f32(128, kDv, false, true);
-                auto issue_qk = [&](int c) -> bool {  // MMA1: A = Q K^T
-                    const int st = c & 1;
-                    if (!wait_or_abort(&bars.full[st], (c >> 1) & 1, ctx, abort)) return false;
-                    // with RoPE, Q and K of the stage are rotated in place first
-                    if (use_rope && !wait_or_abort(&bars.rot_ready[st], (c >> 1) & 1, ctx, abort)) return false;
-                    tc_fence_after();
-#pragma unroll
-                    for (int ks = 0; ks < kD / 16; ++ks)
-                        mma_ss_lohi(tmem + kColA0 + st * 128, at_stage(q_lo0, st) + kstep(ks), at_stage(k_lo0, st) + kstep(ks), hi,
-                                    idQK, ks > 0);
-                    mma_commit(&bars.qk_done[st]);
-                    return true;
-                };
-                bool ok = n_tiles > 0 ? issue_qk(0) : true;
-                for (int c = 0; c < n_tiles && ok; ++c) {
-                    const int st = c & 1;
-                    // MMA2: O1 = A' V (A' from TMEM) once the mask is done and O1 is free.
-                    if (!wait_or_abort(&bars.a_ready[st], (c >> 1) & 1, ctx, abort)) break;
-                    if (c >= 1 && !wait_or_abort(&bars.o_free, (c - 1) & 1, ctx, abort)) break;
-                    tc_fence_after();
-#pragma unroll
-                    for (int ks = 0; ks < kC / 16; ++ks)
-                        mma_ts_lohi(tmem + kColO1, tmem + kColA0 + st * 128 + ks * 8,
-                                    at_stage(v_lo0, st) + (uint32_t)((ks * 16 * 128) >> 4), hi, idO, ks > 0);
-                    mma_commit(&bars.o_done);
-                    mma_commit(&bars.empty[st]);  // this thread's last read of stage c
-                    if (c + 1 < n_tiles) ok = issue_qk(c + 1);
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsOther));
+        if (warp == 8) {
+            // ------------------------------------------------------------------ TMA producer
+            if (lane == 0) {
+                int issued[2] = {-1, -1};
+                for (int c = 0; c < n_tiles; ++c) {
+                    const int s = c & 1, r = c >> 1;
+                    if (r >= 1 && !wait_or_abort(&bars.empty[s], (r - 1) & 1, ctx, abort)) break;
+                    uint8_t* st = sm + s * kStageBytes;
+                    mbar_arrive_expect_tx(&bars.full[s], kStageBytes);
+                    const int y = row0 + c * kC, z = (int)bh;
+                    tma_load_3d(st + kOffQ, &tmQ, &bars.full[s], 0, y, z);
+                    tma_load_3d(st + kOffQ + kSub, &tmQ, &bars.full[s], 64, y, z);
+                    tma_load_3d(st + kOffK, &tmK, &bars.full[s], 0, y, z);
+                    tma_load_3d(st + kOffK + kSub, &tmK, &bars.full[s], 64, y, z);
+                    tma_load_3d(st + kOffV, &tmV, &bars.full[s], slice * kDv, y, z);
+                    issued[s] = r;
                 }
-            } else {
-                const uint32_t idO = idesc_bf16_f32(128, kDv, false, true);
-                const uint32_t idDS = idesc_bf16_f32(128, kDv, true, true);
-                const uint32_t sb_lo0 = sdesc_sw128_lo(smem_u32(sm + kOffSb), 8192);
-                const uint32_t vt_lo0 = sdesc_sw128_lo(smem_u32(sm + kOffVt), 8192);
-                auto issue_ds = [&](int c) -> bool {  // MMA4: dS(c) = K^T V~ (A read transposed)
-                    const int st = c & 1;
-                    if (!wait_or_abort(&bars.full[st], (c >> 1) & 1, ctx, abort)) return false;
-                    if (!wait_or_abort(&bars.v_ready[st], (c >> 1) & 1, ctx, abort)) return false;
-                    // with RoPE, Q (MMA3) and K (MMA4) of the stage rotated in place first
-                    if (use_rope && !wait_or_abort(&bars.rot_ready[st], (c >> 1) & 1, ctx, abort)) return false;
-                    tc_fence_after();
-                    const uint32_t vt_lo = vt_lo0;
-#pragma unroll
-                    for (int ks = 0; ks < kC / 16; ++ks)
-                        mma_ss_lohi(tmem + kColDS + st * kDv, at_stage(kt_lo0, st) + (uint32_t)((ks * 16 * 128) >> 4),
-                                    vt_lo + (uint32_t)((ks * 16 * 128) >> 4), hi, idDS, ks > 0);
-                    mma_commit(&bars.ds_done[st]);
-                    return true;
-                };
-                bool ok = n_tiles > 0 ? issue_ds(0) : true;
-                for (int c = 0; c < n_tiles && ok; ++c) {
-                    const int st = c & 1;
-                    // MMA3: O2 = Q Sb(c-1), read from buffer c&1.  Sb(c-1) published also means
-                    // dS(c-1) has been consumed, so its TMEM buffer is free for dS(c+1) below.
-                    if (!wait_or_abort(&bars.s_ready[st], (c >> 1) & 1, ctx, abort)) break;
-                    if (c >= 1 && !wait_or_abort(&bars.o_free, (c - 1) & 1, ctx, abort)) break;
-                    tc_fence_after();
-                    const uint32_t sb_lo = sb_lo0 + (uint32_t)((st * kSub) >> 4);
-#pragma unroll
-                    for (int ks = 0; ks < kD / 16; ++ks)
-                        mma_ss_lohi(tmem + kColO2, at_stage(q_lo0, st) + kstep(ks), sb_lo + (uint32_t)((ks * 16 * 128) >> 4),
-                                    hi, idO, ks > 0);
-                    mma_commit(&bars.sb_free[st]);
-                    mma_commit(&bars.o_done);
-                    mma_commit(&bars.empty[st]);  // MMA4(c) came earlier: this thread is done with c
-                    if (c + 1 < n_tiles) ok = issue_ds(c + 1);  // dS one tile ahead
-                }
+                for (int s = 0; s < 2; ++s)
+                    if (issued[s] >= 0) (void)mbar_wait(&bars.full[s], issued[s] & 1, ctx);
             }
-            mma_commit(&bars.fin);
-            (void)mbar_wait(&bars.fin, 0, ctx);
-        }
-        __syncwarp();
-    }  // warp 11: idle
+            __syncwarp();
+        } else if (warp == 9 || warp == 10) {
+            // ------------------------------------------------------------------ MMA issuers
+            // Two issuing threads, so that one thread's issue latency does not serialise the four
+            // products: warp 9 issues the attention path (MMA1, MMA2), warp 10 the state path (MMA3,
+            // MMA4).  Each commits its own share of the stage release, of o_done and of fin.  The
+            // shared-memory descriptors are kept as 32-bit halves; a K-step adds to the low half.
+            if (lane == 0) {
+                const uint32_t hi = sdesc_sw128_hi(1024);
+                // Low halves for stage 0; stage st adds st * kStageBytes / 16 to the address field.
+                const uint32_t base = smem_u32(sm);
+                const uint32_t q_lo0 = sdesc_sw128_lo(base + kOffQ, 16);
+                const uint32_t k_lo0 = sdesc_sw128_lo(base + kOffK, 16);
+                const uint32_t kt_lo0 = sdesc_sw128_lo(base + kOffK, kSub);  // K read transposed (MMA4)
+                const uint32_t v_lo0 = sdesc_sw128_lo(base + kOffV, 8192);
+                auto at_stage = [](uint32_t lo, int st) -> uint32_t { return lo + (uint32_t)(st * (kStageBytes >> 4)); };
+                // K-major operand [128 x 128] in two 64-column sub-tiles: K-step ks starts at
+                // sub-tile ks / 4, byte 32 (ks % 4) of its rows.
+                auto kstep = [](int ks) -> uint32_t { return (uint32_t)(((ks >> 2) * kSub + (ks & 3) * 32) >> 4); };
+                if (warp == 9) {
+                    const uint32_t idQK = idesc_bf16_f32(128, 128, false, false);
+                    const uint32_t idO = idesc_bf16_f32(128, kDv, false, true);
+                    auto issue_qk = [&](int c) -> bool {  // MMA1: A = Q K^T
+                        const int st = c & 1;
+                        if (!wait_or_abort(&bars.full[st], (c >> 1) & 1, ctx, abort)) return false;
+                        // with RoPE, Q and K of the stage are rotated in place first
+                        if (use_rope && !wait_or_abort(&bars.rot_ready[st], (c >> 1) & 1, ctx, abort)) return false;
+                        tc_fence_after();
+    #pragma unroll
+                        for (int ks = 0; ks < kD / 16; ++ks)
+                            mma_ss_lohi(tmem + kColA0 + st * 128, at_stage(q_lo0, st) + kstep(ks), at_stage(k_lo0, st) + kstep(ks), hi,
+                                        idQK, ks > 0);
+                        mma_commit(&bars.qk_done[st]);
+                        return true;
+                    };
+                    bool ok = n_tiles > 0 ? issue_qk(0) : true;
+                    for (int c = 0; c < n_tiles && ok; ++c) {
+                        const int st = c & 1;
+                        // MMA2: O1 = A' V (A' from TMEM) once the mask is done and O1 is free.
+                        if (!wait_or_abort(&bars.a_ready[st], (c >> 1) & 1, ctx, abort)) break;
+                        if (c >= 1 && !wait_or_abort(&bars.o_free, (c - 1) & 1, ctx, abort)) break;
+                        tc_fence_after();
+    #pragma unroll
+                        for (int ks = 0; ks < kC / 16; ++ks)
+                            mma_ts_lohi(tmem + kColO1, tmem + kColA0 + st * 128 + ks * 8,
+                                        at_stage(v_lo0, st) + (uint32_t)((ks * 16 * 128) >> 4), hi, idO, ks > 0);
+                        mma_commit(&bars.o_done);
+                        mma_commit(&bars.empty[st]);  // this thread's last read of stage c
+                        if (c + 1 < n_tiles) ok = issue_qk(c + 1);
+                    }
+                } else {
+                    const uint32_t idO = idesc_bf16_f32(128, kDv, false, true);
+                    const uint32_t idDS = idesc_bf16_f32(128, kDv, true, true);
+                    const uint32_t sb_lo0 = sdesc_sw128_lo(smem_u32(sm + kOffSb), 8192);
+                    const uint32_t vt_lo0 = sdesc_sw128_lo(smem_u32(sm + kOffVt), 8192);
+                    auto issue_ds = [&](int c) -> bool {  // MMA4: dS(c) = K^T V~ (A read transposed)
+                        const int st = c & 1;
+                        if (!wait_or_abort(&bars.full[st], (c >> 1) & 1, ctx, abort)) return false;
+                        if (!wait_or_abort(&bars.v_ready[st], (c >> 1) & 1, ctx, abort)) return false;
+                        // with RoPE, Q (MMA3) and K (MMA4) of the stage rotated in place first
+                        if (use_rope && !wait_or_abort(&bars.rot_ready[st], (c >> 1) & 1, ctx, abort)) return false;
+                        tc_fence_after();
+                        const uint32_t vt_lo = vt_lo0;
+    #pragma unroll
+                        for (int ks = 0; ks < kC / 16; ++ks)
+                            mma_ss_lohi(tmem + kColDS + st * kDv, at_stage(kt_lo0, st) + (uint32_t)((ks * 16 * 128) >> 4),
+                                        vt_lo + (uint32_t)((ks * 16 * 128) >> 4), hi, idDS, ks > 0);
+                        mma_commit(&bars.ds_done[st]);
+                        return true;
+                    };
+                    bool ok = n_tiles > 0 ? issue_ds(0) : true;
+                    for (int c = 0; c < n_tiles && ok; ++c) {
+                        const int st = c & 1;
+                        // MMA3: O2 = Q Sb(c-1), read from buffer c&1.  Sb(c-1) published also means
+                        // dS(c-1) has been consumed, so its TMEM buffer is free for dS(c+1) below.
+                        if (!wait_or_abort(&bars.s_ready[st], (c >> 1) & 1, ctx, abort)) break;
+                        if (c >= 1 && !wait_or_abort(&bars.o_free, (c - 1) & 1, ctx, abort)) break;
+                        tc_fence_after();
+                        const uint32_t sb_lo = sb_lo0 + (uint32_t)((st * kSub) >> 4);
+    #pragma unroll
+                        for (int ks = 0; ks < kD / 16; ++ks)
+                            mma_ss_lohi(tmem + kColO2, at_stage(q_lo0, st) + kstep(ks), sb_lo + (uint32_t)((ks * 16 * 128) >> 4),
+                                        hi, idO, ks > 0);
+                        mma_commit(&bars.sb_free[st]);
+                        mma_commit(&bars.o_done);
+                        mma_commit(&bars.empty[st]);  // MMA4(c) came earlier: this thread is done with c
+                        if (c + 1 < n_tiles) ok = issue_ds(c + 1);  // dS one tile ahead
+                    }
+                }
+                mma_commit(&bars.fin);
+                (void)mbar_wait(&bars.fin, 0, ctx);
+            }
+            __syncwarp();
+        }  // warp 11: idle
     } else if (warp >= 12) {
         // ------------------------------------------------------------------ RoPE of Q and K
         // thread = row of the tile; each stage's Q and K rotated in place before its MMAs
