@@ -131,7 +131,7 @@ def init_dist(backend: str):
     ws, rank, _ = dist_env()
     if ws > 1 and not dist.is_initialized():
         import datetime
-        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=600))
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
     return ws, rank
 
 
@@ -595,6 +595,8 @@ def main():
     ap.add_argument("--steps", type=int, default=3)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["sala", "reference"], default="sala")
+    ap.add_argument("--cpu-budget", type=float, default=0.0,
+                    help="seconds of oracle work per CPU-baseline sample (0: the default sizing)")
     ap.add_argument("--phases", default="prefill,decode,e2e,cpu",
                     help="comma list of prefill,decode,e2e,cpu (default: all)")
     ap.add_argument("--decode-steps", type=int, default=200)
@@ -619,7 +621,7 @@ def main():
         from hybrid_sparse_linear_b200 import synth
         vals = []
         # each step a bounded sample, so that the whole arm stays within a few minutes
-        budget = max(5.0, min(20.0, 150.0 / (args.warmup + args.steps)))
+        budget = args.cpu_budget or max(5.0, min(20.0, 150.0 / (args.warmup + args.steps)))
         for i in range(args.warmup + args.steps):
             r = cpu_baseline(torch, synth, budget)
             if i >= args.warmup:
@@ -723,7 +725,7 @@ def main():
                                "device -> pinned host copy of O; copies on their own streams, "
                                "overlapping the neighbouring layers' kernels"}
     if "cpu" in phases and rank == 0 and ws == 1:
-        line["cpu_baseline"] = cpu_baseline(torch, synth)
+        line["cpu_baseline"] = cpu_baseline(torch, synth, args.cpu_budget or 20.0)
     if rank == 0:
         print(json.dumps(line), flush=True)
     barrier()
