@@ -385,7 +385,8 @@ sala_status sala_sparse_decode(const void* q, const void* kcache, const void* vc
     {
         const cudaError_t e = sala::launch_sparse_decode_fused(
             to_dt(dt), q, kcache, vcache, kbar, idx_in, idx_out, o, B, H, Hkv, pos, Tmax, nb_cap, d,
-            topk, n_init, n_local, scale, workspace, workspace_bytes, st, ctx);
+            topk, n_init, n_local, scale, workspace, workspace_bytes,
+            sala::DecodePaging{nullptr, nullptr, 0, 0}, st, ctx);
         if (e != cudaErrorNotSupported) return launched(e, "sparse_decode");
     }
     const int slots = n_init + n_local + topk;
@@ -413,6 +414,53 @@ sala_status sala_sparse_decode(const void* q, const void* kcache, const void* vc
                                                     Hkv, pos, Tmax, d, slots, scale, ws_attn, st,
                                                     ctx),
                     "sparse_decode");
+}
+
+size_t sala_sparse_decode_paged_workspace(int B, int H, int Hkv, int max_pos, int block, int topk,
+                                          int n_init, int n_local, int d) {
+    if (B <= 0 || H <= 0 || Hkv <= 0 || max_pos < 0 || block != 64) return 0;
+    auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    return up(sala::sparse_decode_fused_workspace(B, H, Hkv, max_pos, topk, n_init, n_local, d));
+}
+
+sala_status sala_sparse_decode_paged(const void* q, const void* k_pages, const void* v_pages,
+                                     int n_pages, const int32_t* page_table, int max_pages,
+                                     const void* kbar, int nb_cap, const int32_t* pos,
+                                     int max_pos, int32_t* idx_out, void* o, int B, int H,
+                                     int Hkv, int d, int block, int topk, int n_init, int n_local,
+                                     float scale, void* workspace, size_t workspace_bytes,
+                                     sala_dtype dt, sala_stream stream) {
+    REQUIRE(block == 64, SALA_ERR_UNSUPPORTED, "block %d (pages hold 64 tokens)", block);
+    REQUIRE(n_pages >= 0 && max_pages >= 0, SALA_ERR_INVALID_ARG, "negative page counts");
+    REQUIRE(max_pos >= 0 && (int64_t)max_pos < (int64_t)max_pages * 64, SALA_ERR_INVALID_ARG,
+            "max_pos %d outside the page table (%d pages of 64 tokens)", max_pos, max_pages);
+    sala_status s = check_select_args(B, H, Hkv, 1, max_pos, nb_cap, d, block, topk, n_init,
+                                      n_local, dt);
+    if (s != SALA_OK) return s;
+    REQUIRE(isfinite(scale) && scale >= 0.f, SALA_ERR_INVALID_ARG, "scale must be finite and >= 0");
+    REQUIRE(H / Hkv <= 16, SALA_ERR_UNSUPPORTED, "more than 16 query heads per KV head");
+    if (B == 0 || H == 0) return SALA_OK;
+    REQ_PTR(q); REQ_PTR(k_pages); REQ_PTR(v_pages); REQ_PTR(o); REQ_PTR(kbar);
+    REQUIRE(page_table != nullptr && pos != nullptr, SALA_ERR_INVALID_ARG,
+            "page_table and pos must be device pointers");
+    const size_t need = sala_sparse_decode_paged_workspace(B, H, Hkv, max_pos, block, topk, n_init,
+                                                           n_local, d);
+    REQUIRE(workspace != nullptr && aligned16(workspace) && workspace_bytes >= need,
+            SALA_ERR_INVALID_ARG, "workspace of %zu bytes (16-byte aligned) required, got %zu",
+            need, workspace_bytes);
+    if (scale == 0.f) scale = 1.0f / sqrtf((float)d);
+    sala::DevCtx ctx;
+    s = get_ctx(&ctx);
+    if (s != SALA_OK) return s;
+    const cudaError_t e = sala::launch_sparse_decode_fused(
+        to_dt(dt), q, k_pages, v_pages, kbar, nullptr, idx_out, o, B, H, Hkv, max_pos, 0, nb_cap, d,
+        topk, n_init, n_local, scale, workspace, workspace_bytes,
+        sala::DecodePaging{pos, page_table, max_pages, n_pages}, static_cast<cudaStream_t>(stream),
+        ctx);
+    if (e == cudaErrorNotSupported)
+        return fail(SALA_ERR_UNSUPPORTED, "paged decode runs only as one launch (top-k <= 64, at most "
+                    "80 slots, and a grid that fits the GPU)");
+    return launched(e, "sparse_decode_paged");
 }
 
 }  // extern "C"

@@ -71,11 +71,21 @@ size_t sparse_decode_attn_workspace(int B, int H, int Hkv, int slots, int d);
 // Workspace: [0, 256) barrier words (zero before the first call, left zero), then its data.
 size_t sparse_decode_fused_workspace(int B, int H, int Hkv, int pos, int topk, int n_init,
                                      int n_local, int d);
+// Paged KV cache and per-sequence positions for the one-launch decode (all null / 0: the dense
+// cache [B * Hkv][Tmax][d] and the launch's pos for every sequence).  pos_b: [B] device positions,
+// each at most the launch's pos; pages: [B][max_pages] device page ids, page p holding the 64 rows
+// of one block for every KV head, [n_pages][Hkv][64][d].
+struct DecodePaging {
+    const int32_t* pos_b;
+    const int32_t* pages;
+    int max_pages;
+    int n_pages;
+};
 cudaError_t launch_sparse_decode_fused(DType dt, const void* q, const void* kc, const void* vc,
                                        const void* kbar, const int32_t* idx_in, int32_t* idx_out,
                                        void* o, int B, int H, int Hkv, int pos, int Tmax,
                                        int nb_cap, int d, int topk, int n_init, int n_local,
-                                       float scale, void* ws, size_t ws_bytes, cudaStream_t st,
+                                       float scale, void* ws, size_t ws_bytes, DecodePaging pg, cudaStream_t st,
                                        DevCtx ctx);
 cudaError_t launch_sparse_decode_attn(DType dt, const void* q, const void* kc, const void* vc,
                                       const int32_t* idx, void* o, int B, int H, int Hkv,

@@ -163,7 +163,7 @@ cudaError_t prefill_simt(const void* q, const void* k, const void* v, const floa
 // ---------------------------------------------------------------------------------------------
 // Decode: S <- lambda S + k^T v ; o = q S.  One CTA per (batch*head, 16-column slice); thread
 // (a, half) owns row a of the slice, 8 columns, loaded and stored as two float4.
-template <typename T, int D>
+template <typename T, int D, bool kRope>
 __global__ void __launch_bounds__(2 * D)
 linear_decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                      const float* __restrict__ decay, float* __restrict__ state,
@@ -178,7 +178,7 @@ linear_decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* 
     const float lam = decay[bh % H];
     float ka = to_f(k[bh * D + a]);
     float qa = to_f(q[bh * D + a]);
-    if (rope.base > 0.0) {  // rotate-half pair (a, a +- D/2) at position pos0
+    if constexpr (kRope) {  // rotate-half pair (a, a +- D/2) at position pos0
         const int i = a % (D / 2), partner = a < D / 2 ? a + D / 2 : a - D / 2;
         const float kp = to_f(k[bh * D + partner]), qp = to_f(q[bh * D + partner]);
         float c, s;
@@ -222,9 +222,14 @@ template <typename T, int D>
 cudaError_t decode_launch(const void* q, const void* k, const void* v, const float* decay,
                           float* state, void* o, int B, int H, Rope rope, cudaStream_t st) {
     dim3 grid(D / 16, (unsigned)(B * H));
-    linear_decode_kernel<T, D><<<grid, 2 * D, 0, st>>>(
-        static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), decay,
-        state, static_cast<T*>(o), H, rope);
+    if (rope.base > 0.0)
+        linear_decode_kernel<T, D, true><<<grid, 2 * D, 0, st>>>(
+            static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), decay,
+            state, static_cast<T*>(o), H, rope);
+    else
+        linear_decode_kernel<T, D, false><<<grid, 2 * D, 0, st>>>(
+            static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), decay,
+            state, static_cast<T*>(o), H, rope);
     return cudaGetLastError();
 }
 

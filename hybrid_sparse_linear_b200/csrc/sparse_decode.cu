@@ -223,7 +223,9 @@ sparse_decode_fused_kernel(const T* __restrict__ q, const T* __restrict__ kc,
                            const int32_t* __restrict__ idx_in, int32_t* __restrict__ idx_out,
                            T* __restrict__ o, int H, int Hkv, int pos, int Tmax, int nb_cap,
                            int topk, int n_init, int n_local, int slots, float scale, int cpg,
-                           int nspan, unsigned* bar, uint64_t* part, float* rec, DevCtx ctx) {
+                           int span_stride, const int32_t* __restrict__ pos_b,
+                           const int32_t* __restrict__ pages, int max_pages, int n_pages,
+                           unsigned* bar, uint64_t* part, float* rec, DevCtx ctx) {
     extern __shared__ __align__(16) unsigned char dsm_raw[];
     DecSmem<D>& sm = *reinterpret_cast<DecSmem<D>*>(dsm_raw);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -231,11 +233,22 @@ sparse_decode_fused_kernel(const T* __restrict__ q, const T* __restrict__ kc,
     const int bg = blockIdx.x / cpg, j = blockIdx.x % cpg;
     const int64_t b = bg / Hkv;
     const int g = bg % Hkv;
-    const int c = pos / kBlk;
+    // This sequence's query position: the launch's pos for all, or its own (pos_b[b], at most pos;
+    // one out of range is flagged and clamped, so every CTA still reaches both grid barriers).
+    int pos_s = pos;
+    if (pos_b) {
+        pos_s = __ldg(pos_b + b);
+        if (pos_s < 0 || pos_s > pos) {
+            if (tid == 0) flag(ctx, kStatusBounds);
+            pos_s = pos_s < 0 ? 0 : pos;
+        }
+    }
+    const int c = pos_s / kBlk;
     const int lo = n_init, hi = c - n_local;
     const int ncand = hi - lo + 1;
     const int K = topk;
     const bool do_sel = idx_in == nullptr && ncand > K;
+    const int nspan = ncand > K ? (ncand + kSpan - 1) / kSpan : 0;  // this sequence's spans
     const T* qg = q + (b * H + (int64_t)g * G) * D;  // the group's G query rows
 
     // ---------------------------------------------------------------- A: span scores + top-k
@@ -299,7 +312,7 @@ sparse_decode_fused_kernel(const T* __restrict__ q, const T* __restrict__ kc,
             const int blk = base + tid;
             uint64_t x[1] = {blk <= hi ? sel_key_u(sm.sc[tid], blk) : 0ull};
             block_sort_desc<1>(x, sm.cand);
-            if (tid < kCap) part[((int64_t)bg * nspan + span) * kCap + tid] = tid < K ? x[0] : 0ull;
+            if (tid < kCap) part[((int64_t)bg * span_stride + span) * kCap + tid] = tid < K ? x[0] : 0ull;
         }
     }
     if (!grid_barrier(bar, gridDim.x, ctx, &sm.ok)) return;
@@ -324,7 +337,7 @@ sparse_decode_fused_kernel(const T* __restrict__ q, const T* __restrict__ kc,
             // spans' whole lists.
             constexpr int kPre = 8, kPreE = kMergeE * kPre / kCap;  // prefix keys per thread (spans <= 128)
             const unsigned long long* src =
-                reinterpret_cast<const unsigned long long*>(part) + (int64_t)bg * nspan * kCap;
+                reinterpret_cast<const unsigned long long*>(part) + (int64_t)bg * span_stride * kCap;
             if (tid == 0) {
                 sm.sel_n = 0;
                 sm.overflow = 0;
@@ -428,12 +441,30 @@ sparse_decode_fused_kernel(const T* __restrict__ q, const T* __restrict__ kc,
             if (e < G * D) sm.Q[e / D][e % D] = qv[u];
         }
     }
-    const T* kcg = kc + (int64_t)bg * Tmax * D;
-    const T* vcg = vc + (int64_t)bg * Tmax * D;
     constexpr int kStage = kBlk * (D / 8) / kThreads;  // 8-element pieces of K (and V) per thread
     for (int s = j; s < slots; s += cpg) {
-        const int blk = sm.sel[s];
+        int blk = sm.sel[s];
         float* r = rec + ((int64_t)bg * slots + s) * G * (D + 2);
+        // the block's 64 K and V rows: in the dense cache [B * Hkv][Tmax][D], or in the page the
+        // sequence's table names for it ([n_pages][Hkv][64][D]); a bad page id is flagged and the
+        // slot left empty
+        const T* kblk = nullptr;
+        const T* vblk = nullptr;
+        if (blk >= 0) {
+            if (pages) {
+                const int pg = blk < max_pages ? __ldg(pages + b * max_pages + blk) : -1;
+                if (pg < 0 || pg >= n_pages) {
+                    if (tid == 0) flag(ctx, kStatusBounds);
+                    blk = -1;
+                } else {
+                    kblk = kc + ((int64_t)pg * Hkv + g) * kBlk * D;
+                    vblk = vc + ((int64_t)pg * Hkv + g) * kBlk * D;
+                }
+            } else {
+                kblk = kc + ((int64_t)bg * Tmax + (int64_t)blk * kBlk) * D;
+                vblk = vc + ((int64_t)bg * Tmax + (int64_t)blk * kBlk) * D;
+            }
+        }
         if (blk < 0) {
             for (int hh = tid; hh < G; hh += kThreads) {
                 r[hh * (D + 2)] = -INFINITY;
@@ -441,7 +472,7 @@ sparse_decode_fused_kernel(const T* __restrict__ q, const T* __restrict__ kc,
             }
             continue;
         }
-        const int lim = min(kBlk - 1, pos - blk * kBlk);  // last visible key of the block
+        const int lim = min(kBlk - 1, pos_s - blk * kBlk);  // last visible key of the block
         constexpr int kU = 8 * sizeof(T) / 16;  // 16-byte pieces per 8 elements
         constexpr int kEl = 16 / sizeof(T);
         uint4 rk[kStage][kU], rv[kStage][kU];
@@ -450,8 +481,8 @@ sparse_decode_fused_kernel(const T* __restrict__ q, const T* __restrict__ kc,
             const int e = u * kThreads + tid;
             const int row = e / (D / 8), c8 = (e % (D / 8)) * 8;
             const bool ok = row <= lim;
-            const T* pk = kcg + ((int64_t)blk * kBlk + row) * D + c8;
-            const T* pv = vcg + ((int64_t)blk * kBlk + row) * D + c8;
+            const T* pk = kblk + (int64_t)row * D + c8;
+            const T* pv = vblk + (int64_t)row * D + c8;
 #pragma unroll
             for (int w = 0; w < kU; ++w) {
                 rk[u][w] = ok ? ld16(pk + w * kEl) : make_uint4(0u, 0u, 0u, 0u);
@@ -684,7 +715,7 @@ template <typename T, int D>
 cudaError_t fused(const void* q, const void* kc, const void* vc, const void* kbar,
                   const int32_t* idx_in, int32_t* idx_out, void* o, int B, int H, int Hkv, int pos,
                   int Tmax, int nb_cap, int topk, int n_init, int n_local, float scale, void* ws,
-                  size_t ws_bytes, cudaStream_t st, DevCtx ctx) {
+                  size_t ws_bytes, DecodePaging pg, cudaStream_t st, DevCtx ctx) {
     const int slots = n_init + n_local + topk;
     const int G = H / Hkv;
     const int c = pos / kBlk;
@@ -732,7 +763,8 @@ cudaError_t fused(const void* q, const void* kc, const void* vc, const void* kba
     return cudaLaunchKernelEx(&cfg, kern, static_cast<const T*>(q), static_cast<const T*>(kc),
                               static_cast<const T*>(vc), static_cast<const T*>(kbar), idx_in, idx_out,
                               static_cast<T*>(o), H, Hkv, pos, Tmax, nb_cap, topk, n_init, n_local,
-                              slots, scale, cpg, nspan, reinterpret_cast<unsigned*>(w), part, rec, ctx);
+                              slots, scale, cpg, nspan, pg.pos_b, pg.pages, pg.max_pages, pg.n_pages,
+                              reinterpret_cast<unsigned*>(w), part, rec, ctx);
 }
 
 }  // namespace
@@ -750,13 +782,13 @@ cudaError_t launch_sparse_decode_fused(DType dt, const void* q, const void* kc, 
                                        const void* kbar, const int32_t* idx_in, int32_t* idx_out,
                                        void* o, int B, int H, int Hkv, int pos, int Tmax,
                                        int nb_cap, int d, int topk, int n_init, int n_local,
-                                       float scale, void* ws, size_t ws_bytes, cudaStream_t st,
-                                       DevCtx ctx) {
+                                       float scale, void* ws, size_t ws_bytes, DecodePaging pg,
+                                       cudaStream_t st, DevCtx ctx) {
     if (dt == DType::F32)
-        return d == 64 ? fused<float, 64>(q, kc, vc, kbar, idx_in, idx_out, o, B, H, Hkv, pos, Tmax, nb_cap, topk, n_init, n_local, scale, ws, ws_bytes, st, ctx)
-                       : fused<float, 128>(q, kc, vc, kbar, idx_in, idx_out, o, B, H, Hkv, pos, Tmax, nb_cap, topk, n_init, n_local, scale, ws, ws_bytes, st, ctx);
-    return d == 64 ? fused<__nv_bfloat16, 64>(q, kc, vc, kbar, idx_in, idx_out, o, B, H, Hkv, pos, Tmax, nb_cap, topk, n_init, n_local, scale, ws, ws_bytes, st, ctx)
-                   : fused<__nv_bfloat16, 128>(q, kc, vc, kbar, idx_in, idx_out, o, B, H, Hkv, pos, Tmax, nb_cap, topk, n_init, n_local, scale, ws, ws_bytes, st, ctx);
+        return d == 64 ? fused<float, 64>(q, kc, vc, kbar, idx_in, idx_out, o, B, H, Hkv, pos, Tmax, nb_cap, topk, n_init, n_local, scale, ws, ws_bytes, pg, st, ctx)
+                       : fused<float, 128>(q, kc, vc, kbar, idx_in, idx_out, o, B, H, Hkv, pos, Tmax, nb_cap, topk, n_init, n_local, scale, ws, ws_bytes, pg, st, ctx);
+    return d == 64 ? fused<__nv_bfloat16, 64>(q, kc, vc, kbar, idx_in, idx_out, o, B, H, Hkv, pos, Tmax, nb_cap, topk, n_init, n_local, scale, ws, ws_bytes, pg, st, ctx)
+                   : fused<__nv_bfloat16, 128>(q, kc, vc, kbar, idx_in, idx_out, o, B, H, Hkv, pos, Tmax, nb_cap, topk, n_init, n_local, scale, ws, ws_bytes, pg, st, ctx);
 }
 
 }  // namespace sala

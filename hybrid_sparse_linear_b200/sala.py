@@ -45,6 +45,11 @@ _lib.sala_sparse_decode.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _
                                     _i, _i, _i, _i, ctypes.c_float, _vp, _st, _i, _vp]
 _lib.sala_sparse_decode_workspace.argtypes = [_i, _i, _i, _i, _i, _i, _i, _i, _i]
 _lib.sala_sparse_decode_workspace.restype = _st
+_lib.sala_sparse_decode_paged.argtypes = [_vp, _vp, _vp, _i, _vp, _i, _vp, _i, _vp, _i, _vp, _vp,
+                                          _i, _i, _i, _i, _i, _i, _i, _i, ctypes.c_float, _vp, _st,
+                                          _i, _vp]
+_lib.sala_sparse_decode_paged_workspace.argtypes = [_i] * 9
+_lib.sala_sparse_decode_paged_workspace.restype = _st
 _lib.sala_check_status.argtypes = [_vp]
 _lib.sala_status_string.argtypes = [_i]
 _lib.sala_status_string.restype = ctypes.c_char_p
@@ -52,7 +57,8 @@ _lib.sala_last_error.restype = ctypes.c_char_p
 _lib.sala_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
 _lib.sala_selftest_wait_timeout.argtypes = [_vp]
 for _f in ("sala_linear_prefill", "sala_linear_decode", "sala_linear_prefill_rope",
-           "sala_linear_decode_rope", "sala_block_compress", "sala_block_topk",
+           "sala_linear_decode_rope", "sala_sparse_decode_paged", "sala_block_compress",
+           "sala_block_topk",
            "sala_sparse_prefill", "sala_sparse_decode", "sala_check_status",
            "sala_selftest_wait_timeout"):
     getattr(_lib, _f).restype = _i
@@ -235,6 +241,41 @@ def sparse_decode(q, kcache, vcache, kbar, pos, topk, n_init=1, n_local=2, idx_i
                                    block, topk, n_init, n_local, float(scale), _ptr(workspace),
                                    workspace.numel(), _dt(q), _stream(stream)),
            "sala_sparse_decode")
+    return o
+
+
+def sparse_decode_paged_workspace_bytes(B, H, Hkv, max_pos, topk, n_init, n_local, d, block=64):
+    return _lib.sala_sparse_decode_paged_workspace(B, H, Hkv, max_pos, block, topk, n_init, n_local, d)
+
+
+def sparse_decode_paged(q, k_pages, v_pages, page_table, kbar, pos, max_pos, topk, n_init, n_local,
+                        idx_out=None, o=None, scale=0.0, workspace=None, stream=None):
+    """One query token per head for each of B sequences at its own position pos[b] (an int32
+    device tensor, each <= max_pos), the KV cache in pages: k_pages, v_pages [n_pages, Hkv, 64, d],
+    page_table [B, max_pages] int32.  q: [B, H, d]; kbar [B, Hkv, nb_cap, d].  Returns o."""
+    B, H, d = q.shape
+    n_pages, Hkv = k_pages.shape[0], k_pages.shape[1]
+    _need(q, "q"); _need(k_pages, "k_pages", dtype=q.dtype)
+    _need(v_pages, "v_pages", k_pages.shape, q.dtype)
+    assert k_pages.shape[2:] == (64, d), k_pages.shape
+    _need(page_table, "page_table", dtype=torch.int32)
+    assert page_table.dim() == 2 and page_table.shape[0] == B
+    _need(pos, "pos", (B,), torch.int32)
+    _need(kbar, "kbar", dtype=q.dtype)
+    slots = n_init + n_local + topk
+    _need(idx_out, "idx_out", (B, Hkv, slots), torch.int32)
+    if o is None:
+        o = torch.empty_like(q)
+    _need(o, "o", q.shape, q.dtype)
+    need = sparse_decode_paged_workspace_bytes(B, H, Hkv, max_pos, topk, n_init, n_local, d)
+    if workspace is None:
+        workspace = torch.zeros(max(need, 256), dtype=torch.uint8, device=q.device)
+    _check(_lib.sala_sparse_decode_paged(_ptr(q), _ptr(k_pages), _ptr(v_pages), n_pages,
+                                         _ptr(page_table), page_table.shape[1], _ptr(kbar),
+                                         kbar.shape[2], _ptr(pos), int(max_pos), _ptr(idx_out),
+                                         _ptr(o), B, H, Hkv, d, 64, topk, n_init, n_local,
+                                         ctypes.c_float(scale), _ptr(workspace), workspace.numel(),
+                                         _dt(q), _stream(stream)), "sala_sparse_decode_paged")
     return o
 
 

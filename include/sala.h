@@ -221,6 +221,36 @@ sala_status sala_sparse_decode(const void* q, const void* kcache, const void* vc
 size_t sala_sparse_decode_workspace(int B, int H, int Hkv, int pos, int block, int topk,
                                     int n_init, int n_local, int d);
 
+/* sala_sparse_decode for a batch of sequences that each decode at their own position, with the
+ * KV cache held in pages of one block.  The pages have no counterpart (the method stores the
+ * whole KV cache densely); paging is how a server keeps many sequences' caches in one pool.
+ * k_pages, v_pages : [n_pages, Hkv, 64, d] device, dt.  Page p holds the 64 key (value) rows of
+ *                    one block of one sequence, for every KV head.
+ * page_table       : [B, max_pages] int32 device.  Entry [b][j] is the page of block j of
+ *                    sequence b; only the blocks a sequence attends to are read, and an entry
+ *                    outside [0, n_pages) is flagged (SALA_ERR_BOUNDS through
+ *                    sala_check_status) and its block left out.
+ * kbar             : [B, Hkv, nb_cap, d] device, each sequence's compressed blocks (dense).
+ * pos              : [B] int32 device, sequence b's query position (its cache holds pos[b] + 1
+ *                    tokens); each in [0, max_pos] (outside: flagged and clamped).
+ * max_pos          : the largest position, < max_pages * 64 (sizes the launch and workspace).
+ * block            : 64 (the page size).  Selection happens here (no idx_in); idx_out: as
+ *                    sala_sparse_decode.
+ * workspace        : at least sala_sparse_decode_paged_workspace(...) bytes; its first 256
+ *                    bytes follow the rule of sala_sparse_decode's workspace.
+ * Runs as the one-launch kernel only: top-k <= 64, n_init + n_local + topk <= 80, at most 16
+ * query heads per KV head, d in {64, 128}; otherwise SALA_ERR_UNSUPPORTED.  Other arguments,
+ * validation and errors are those of sala_sparse_decode. */
+sala_status sala_sparse_decode_paged(const void* q, const void* k_pages, const void* v_pages,
+                                     int n_pages, const int32_t* page_table, int max_pages,
+                                     const void* kbar, int nb_cap, const int32_t* pos,
+                                     int max_pos, int32_t* idx_out, void* o, int B, int H,
+                                     int Hkv, int d, int block, int topk, int n_init, int n_local,
+                                     float scale, void* workspace, size_t workspace_bytes,
+                                     sala_dtype dt, sala_stream stream);
+size_t sala_sparse_decode_paged_workspace(int B, int H, int Hkv, int max_pos, int block, int topk,
+                                          int n_init, int n_local, int d);
+
 /* sala_sparse_decode for callers that cannot allocate device memory.  The pages have no
  * counterpart; this is a property of the library, not of the method.
  *

@@ -210,3 +210,78 @@ def test_sparse_decode_workspace_reused_across_calls_and_shapes(sala):
                 first = (o.clone(), idx.clone())
             else:
                 assert torch.equal(o, first[0]) and torch.equal(idx, first[1])
+
+
+# ---------------------------------------------------------------------------------------------
+# Paged KV cache, one position per sequence (sala_sparse_decode_paged)
+
+def _paged_batch(sala, lengths, H=32, Hkv=2, d=128, seed=0, layer0=20):
+    """Each sequence drawn dense at its own length, its blocks scattered over a shuffled page
+    pool (with unused pages in between).  Returns the paged tensors and the dense originals."""
+    from hybrid_sparse_linear_b200 import synth
+    B = len(lengths)
+    layers = [synth.sparse_layer(1, H, Hkv, n, d, torch.bfloat16, "cpu", layer=layer0 + b,
+                                 shift_frac=0.05, q_rows=1) for b, n in enumerate(lengths)]
+    nblk = [(n + 63) // 64 for n in lengths]
+    max_pages = max(nblk)
+    n_pages = sum(nblk) + 7
+    rng = np.random.default_rng(seed)
+    perm = rng.permutation(n_pages)
+    table = np.full((B, max_pages), -1, dtype=np.int32)
+    k_pages = torch.zeros((n_pages, Hkv, 64, d), dtype=torch.bfloat16)
+    v_pages = torch.zeros_like(k_pages)
+    nxt = 0
+    for b, (sl, n) in enumerate(zip(layers, lengths)):
+        for j in range(nblk[b]):
+            p = int(perm[nxt]); nxt += 1
+            table[b, j] = p
+            rows = min(64, n - 64 * j)
+            k_pages[p, :, :rows] = sl.k[0, :, 64 * j:64 * j + rows]
+            v_pages[p, :, :rows] = sl.v[0, :, 64 * j:64 * j + rows]
+    nb_cap = max(n // 64 for n in lengths)
+    kbar = torch.zeros((B, Hkv, max(nb_cap, 1), d), dtype=torch.bfloat16, device="cuda")
+    for b, sl in enumerate(layers):
+        nb = lengths[b] // 64
+        if nb:
+            kbar[b, :, :nb] = sala.block_compress(sl.k.cuda())[0, :, :nb]
+    q = torch.stack([sl.q[0, :, 0] for sl in layers]).contiguous()
+    pos = torch.tensor([n - 1 for n in lengths], dtype=torch.int32)
+    return (q.cuda(), k_pages.cuda(), v_pages.cuda(), torch.from_numpy(table).cuda(), kbar,
+            pos.cuda(), layers)
+
+
+def test_sparse_decode_paged_per_sequence_positions(sala):
+    lengths = [64 * 300 + 5, 64 * 40, 64 * 3 + 1, 64 * 128]
+    topk, n_init, n_local = 64, 1, 2
+    q, kp, vp, table, kbar, pos, layers = _paged_batch(sala, lengths)
+    B, Hkv = len(lengths), kp.shape[1]
+    idx_out = torch.empty((B, Hkv, n_init + n_local + topk), dtype=torch.int32, device="cuda")
+    o = sala.sparse_decode_paged(q, kp, vp, table, kbar, pos, max(lengths) - 1, topk, n_init,
+                                 n_local, idx_out=idx_out)
+    sala.check_status()
+    got = idx_out.cpu().numpy()
+    for b, (sl, n) in enumerate(zip(layers, lengths)):
+        p = n - 1
+        q64, k64, v64 = _f64(sl.q), _f64(sl.k), _f64(sl.v)
+        kbar_ref = oracle.block_compress(k64, 64, round_to_bf16=True) if n >= 64 else \
+            np.zeros((1, Hkv, 0, q64.shape[-1]))
+        idx_ref, kth = oracle.block_select(q64, kbar_ref, 64, topk, n_init, n_local, q_pos0=p)
+        gb = got[b:b + 1, :, None, :]
+        check_selection(gb, idx_ref, q64, kbar_ref, kth, topk, n_init, n_local, q_pos0=p,
+                        row_ids=np.array([0]))
+        o_ref = oracle.sparse_attention(q64, k64, v64, gb, 64, q_pos0=p)
+        assert_close(_f64(o[b:b + 1]), o_ref[:, :, 0], "bf16", f"paged decode sequence {b}")
+
+
+def test_sparse_decode_paged_bad_page_is_flagged(sala):
+    lengths = [64 * 50 + 3, 64 * 20]
+    q, kp, vp, table, kbar, pos, _ = _paged_batch(sala, lengths, seed=1)
+    table[0, 0] = kp.shape[0] + 5          # block 0 (always attended) names no page
+    sala.sparse_decode_paged(q, kp, vp, table, kbar, pos, max(lengths) - 1, 16, 1, 2)
+    with pytest.raises(sala.SalaError) as e:
+        sala.check_status()
+    assert e.value.code == sala.ERR_BOUNDS
+    # the context stays usable: a good call afterwards succeeds
+    table[0, 0] = 0 if int(table[1, 0]) != 0 else 1
+    sala.sparse_decode_paged(q, kp, vp, table, kbar, pos, max(lengths) - 1, 16, 1, 2)
+    sala.check_status()
