@@ -327,6 +327,71 @@ def run_prefill(sala, synth, torch, steps, warmup, stream, workload="hybrid_pref
     return res
 
 
+def run_decode_paged(sala, synth, torch, steps, warmup, stream, B=8):
+    """One sparse layer's decode for B sequences at their own positions (64K .. 256K tokens), the
+    KV cache in pages of one block scattered over a pool; CUDA-graph replays, L2 flushed."""
+    import numpy as np
+    dev = torch.device("cuda")
+    lengths = [int(n) // 64 * 64 + 17 for n in np.linspace(1 << 16, 1 << 18, B)]
+    nblk = [(n + 63) // 64 for n in lengths]
+    max_pages, n_pages = max(nblk), sum(nblk)
+    perm = torch.randperm(n_pages, generator=torch.Generator().manual_seed(5))
+    k_pages = torch.empty((n_pages, HKV, BLOCK, D), dtype=torch.bfloat16, device=dev)
+    v_pages = torch.empty_like(k_pages)
+    table = torch.full((B, max_pages), -1, dtype=torch.int32)
+    nb_cap = max(n // BLOCK for n in lengths)
+    kbar = torch.zeros((B, HKV, nb_cap, D), dtype=torch.bfloat16, device=dev)
+    qs, at = [], 0
+    for b, n in enumerate(lengths):
+        sl = synth.sparse_layer(1, H, HKV, n, D, torch.bfloat16, dev, layer=40 + b, q_rows=1)
+        pad = nblk[b] * BLOCK - n
+        kk = torch.nn.functional.pad(sl.k[0], (0, 0, 0, pad)).view(HKV, nblk[b], BLOCK, D)
+        vv = torch.nn.functional.pad(sl.v[0], (0, 0, 0, pad)).view(HKV, nblk[b], BLOCK, D)
+        ids = perm[at:at + nblk[b]]
+        at += nblk[b]
+        table[b, :nblk[b]] = ids.to(torch.int32)
+        k_pages[ids.to(dev)] = kk.transpose(0, 1)
+        v_pages[ids.to(dev)] = vv.transpose(0, 1)
+        kbar[b, :, :n // BLOCK] = sala.block_compress(sl.k, stream=stream)[0, :, :n // BLOCK]
+        qs.append(sl.q[0, :, 0])
+        del sl
+    q = torch.stack(qs).contiguous()
+    table = table.to(dev)
+    pos = torch.tensor([n - 1 for n in lengths], dtype=torch.int32, device=dev)
+    max_pos = max(lengths) - 1
+    need = sala.sparse_decode_paged_workspace_bytes(B, H, HKV, max_pos, TOPK, N_INIT, N_LOCAL, D)
+    ws = torch.zeros(max(need, 256), dtype=torch.uint8, device=dev)
+    o = torch.empty_like(q)
+    flush = torch.empty(512 << 20, device=dev, dtype=torch.uint8)
+    call = lambda: sala.sparse_decode_paged(q, k_pages, v_pages, table, kbar, pos, max_pos, TOPK,
+                                            N_INIT, N_LOCAL, o=o, workspace=ws, stream=stream)
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            call()
+        torch.cuda.synchronize()
+        sala.check_status(stream)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            call()
+        times = []
+        for _ in range(max(steps, 20)):
+            flush.zero_()
+            a, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            g.replay()
+            e.record(stream)
+            times.append((a, e))
+        torch.cuda.synchronize()
+    sala.check_status(stream)
+    us = sorted(a.elapsed_time(e) * 1000.0 for a, e in times)[len(times) // 2]
+    slots = N_INIT + N_LOCAL + TOPK
+    nbytes = sum(HKV * (n // BLOCK) * D * 2 + HKV * slots * BLOCK * D * 2 * 2 + 2 * H * D * 2
+                 for n in lengths)
+    del g, k_pages, v_pages, kbar, flush
+    torch.cuda.empty_cache()
+    return {"us_per_call": us, "bytes": nbytes, "lengths": lengths}
+
+
 def run_decode(sala, synth, torch, steps, warmup, stream, T=DECODE_T):
     """Decode at a T-token context (2^20 by default), 24 linear + 8 sparse layers per token, L2
     flushed."""
@@ -598,7 +663,7 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=0.0,
                     help="seconds of oracle work per CPU-baseline sample (0: the default sizing)")
     ap.add_argument("--phases", default="prefill,decode,e2e,cpu",
-                    help="comma list of prefill,decode,e2e,cpu (default: all)")
+                    help="comma list of prefill,decode,e2e,cpu,paged (default: all but paged)")
     ap.add_argument("--decode-steps", type=int, default=200)
     ap.add_argument("--decode-t", type=int, default=DECODE_T,
                     help="decode context length (default 2^20, the benchmark; smaller only for profiles)")
@@ -701,6 +766,15 @@ def main():
                                     "peak_source": f"{peaks['source']} HBM copy",
                                     "algorithmic_bytes_per_launch": linear_layer_bytes(n_tok),
                                     "mean_launch_ms": pre["linear_ms"]}
+    if "paged" in phases:
+        pg = run_decode_paged(sala, synth, torch, args.decode_steps, max(3, args.warmup), stream)
+        gbs = pg["bytes"] / (pg["us_per_call"] * 1e-6) / 1e9
+        line["decode_paged"] = {"metric": "paged sparse decode us per call (8 sequences, own positions)",
+                                "us_per_call": pg["us_per_call"], "sequence_tokens": pg["lengths"],
+                                "bytes_per_call": pg["bytes"], "achieved_gbs": gbs,
+                                "hbm_frac": gbs / peaks["hbm_gbs"],
+                                "timing": "CUDA events around one CUDA-graph replay, L2 flushed "
+                                          "before each, median"}
     if "decode" in phases:
         dec = run_decode(sala, synth, torch, args.decode_steps, max(3, args.warmup), stream, args.decode_t)
         db = decode_bytes(args.decode_t)
