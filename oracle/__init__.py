@@ -60,6 +60,7 @@ def _load():
             lib.orc_block_scores_at.argtypes = [_D, _D, _I64, _l, _D, _i, _i, _i, _i, _i]
             lib.orc_block_select.argtypes = [_D, _D, _I32, _D, _i, _i, _i, _i, _i, _i, _i, _i, _i,
                                              _i, _i, _i, _i]
+            lib.orc_block_select_qblock.argtypes = [_D, _D, _I32, _D] + [_i] * 12
             lib.orc_sparse_attention.argtypes = [_D, _D, _D, _I32, _D, _i, _i, _i, _i, _i, _i, _i,
                                                  _i, _i, ctypes.c_double, _I64, _l, _i]
             lib.orc_dense_causal_attention.argtypes = [_D, _D, _D, _D, _i, _i, _i, _i, _i, _i, _i,
@@ -197,6 +198,32 @@ def block_select(q, kbar, block, topk, n_init, n_local, q_pos0=0, slots=None, th
                              int(q_pos0), nb, d, block, topk, n_init, n_local, slots,
                              threads or default_threads())
     return idx, kth
+
+
+def block_select_qblock(q, kbar, block, topk, n_init, n_local, slots=None, threads=None):
+    """One selection per (batch, KV group, query block of `block` tokens), written to every token
+    row of the block.  Returns (idx int32 [B,Hkv,Nq,slots], kth_score [B,Hkv,Nq])."""
+    q, kbar = _f64(q), _f64(kbar)
+    B, H, Nq, d = q.shape
+    Hkv, nb = kbar.shape[1], kbar.shape[2]
+    slots = slots or (n_init + n_local + topk)
+    idx = np.empty((B, Hkv, Nq, slots), dtype=np.int32)
+    kth = np.empty((B, Hkv, Nq))
+    _load().orc_block_select_qblock(_p(q), _p(kbar), idx.ctypes.data_as(_I32), _p(kth), B, H, Hkv,
+                                    Nq, nb, d, block, topk, n_init, n_local, slots,
+                                    threads or default_threads())
+    return idx, kth
+
+
+def qblock_sum(q, block):
+    """q with every token replaced by the per-head sum of q over its query block (plain numpy):
+    the query tensor whose per-token selection is the query-block selection."""
+    q = _f64(q)
+    B, H, Nq, d = q.shape
+    out = np.empty_like(q)
+    for r0 in range(0, Nq, block):
+        out[:, :, r0:r0 + block] = q[:, :, r0:r0 + block].sum(axis=2, keepdims=True)
+    return out
 
 
 def block_scores_at(q, kbar, quads):

@@ -399,4 +399,52 @@ void orc_rope(double* x, int B, int H, int N, int d, int64_t pos0, double base) 
         }
 }
 
+// Query-block-granular selection: one selection per (batch, KV group, query block of T tokens),
+// shared by the block's tokens.  A variant the contract lists next to the per-token selection
+// (the pages describe InfLLM-V2's block selection without fixing its granularity).  Reading: the
+// block's score vector is the sum over the group's heads and over the block's tokens (those
+// below Nq in a partial last block) of q, dotted with kbar; candidates, forced blocks, tie rule
+// and output layout as orc_block_select, every token row of the block receiving the same row.
+void orc_block_select_qblock(const double* q, const double* kbar, int32_t* idx, double* kth_score,
+                             int B, int H, int Hkv, int Nq, int nb, int d, int T, int topk,
+                             int n_init, int n_local, int slots, int nthreads) {
+    const int G = H / Hkv;
+    const int nqb = (Nq + T - 1) / T;
+    parallel_for((int64_t)B * Hkv * nqb, nthreads, [&](int64_t item) {
+        const int64_t b = item / ((int64_t)Hkv * nqb);
+        const int g = (int)((item / nqb) % Hkv);
+        const int c = (int)(item % nqb);
+        const int r0 = c * T, r1 = std::min(Nq, r0 + T);
+        std::vector<double> qs(d, 0.0);
+        for (int h = g * G; h < (g + 1) * G; ++h)
+            for (int r = r0; r < r1; ++r) {
+                const double* qr = q + (((int64_t)b * H + h) * Nq + r) * d;
+                for (int a = 0; a < d; ++a) qs[a] += qr[a];
+            }
+        std::vector<int> sel;
+        for (int blk = 0; blk < n_init && blk <= c; ++blk) sel.push_back(blk);
+        for (int blk = std::max(0, c - n_local + 1); blk <= c; ++blk)
+            if (blk >= n_init) sel.push_back(blk);
+        std::vector<std::pair<double, int>> cand;
+        for (int blk = n_init; blk <= c - n_local; ++blk)
+            cand.push_back({dot(qs.data(), kbar + (((int64_t)b * Hkv + g) * nb + blk) * d, d), blk});
+        std::sort(cand.begin(), cand.end(), [](const auto& x, const auto& y) {
+            if (x.first != y.first) return x.first > y.first;
+            return x.second < y.second;
+        });
+        const int take = std::min<int>(topk, (int)cand.size());
+        for (int e = 0; e < take; ++e) sel.push_back(cand[e].second);
+        std::sort(sel.begin(), sel.end());
+        const double kth = ((int)cand.size() >= topk && topk > 0)
+                               ? cand[topk - 1].first
+                               : -std::numeric_limits<double>::infinity();
+        for (int r = r0; r < r1; ++r) {
+            const int64_t row = ((int64_t)b * Hkv + g) * Nq + r;
+            int32_t* out = idx + row * slots;
+            for (int e = 0; e < slots; ++e) out[e] = e < (int)sel.size() ? sel[e] : -1;
+            if (kth_score) kth_score[row] = kth;
+        }
+    });
+}
+
 }  // extern "C"
