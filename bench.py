@@ -236,6 +236,8 @@ WORKLOADS = {
     "linear_prefill_n256k": (N_TOK, ["linear"]),
     # a linear layer with its RoPE (HyPE) fused into the load path, base 10000, positions 0..N-1
     "linear_rope_prefill_n256k": (N_TOK, ["linear_rope"]),
+    # a sparse layer whose 64-token query blocks each share one selection (the variant)
+    "sparse_qblock_prefill_n256k": (N_TOK, ["sparse_qblock"]),
 }
 
 
@@ -246,9 +248,9 @@ def run_prefill(sala, synth, torch, steps, warmup, stream, workload="hybrid_pref
     lam = synth.decays(H).to(dev)
     layers = []
     for l, kind in enumerate(kinds):
-        if kind == "sparse":
+        if kind in ("sparse", "sparse_qblock"):
             sl = synth.sparse_layer(1, H, HKV, n_tok, D, torch.bfloat16, dev, layer=l)
-            layers.append(("sparse", sl.q, sl.k, sl.v))
+            layers.append((kind, sl.q, sl.k, sl.v))
         else:
             q, k, v = synth.linear_layer(1, H, n_tok, D, torch.bfloat16, dev, layer=l)
             layers.append((kind, q, k, v))
@@ -282,7 +284,10 @@ def run_prefill(sala, synth, torch, steps, warmup, stream, workload="hybrid_pref
                 t0, t1 = (ev(), ev()) if record else (None, None)
                 if record: t0.record(stream)
                 sala.block_compress(k, kbar, stream=stream)
-                sala.block_topk(q, kbar, TOPK, N_INIT, N_LOCAL, idx=idx, stream=stream)
+                if kind == "sparse":
+                    sala.block_topk(q, kbar, TOPK, N_INIT, N_LOCAL, idx=idx, stream=stream)
+                else:
+                    sala.block_topk_qblock(q, kbar, TOPK, N_INIT, N_LOCAL, idx=idx, stream=stream)
                 if record: t1.record(stream); topk_ev.append((t0, t1))
                 e0, e1 = (ev(), ev()) if record else (None, None)
                 if record: e0.record(stream)
@@ -316,9 +321,12 @@ def run_prefill(sala, synth, torch, steps, warmup, stream, workload="hybrid_pref
     union, n_sp = 0, 0
     with torch.cuda.stream(stream):
         for kind, q, k, v in layers:
-            if kind == "sparse":
+            if kind in ("sparse", "sparse_qblock"):
                 sala.block_compress(k, kbar, stream=stream)
-                sala.block_topk(q, kbar, TOPK, N_INIT, N_LOCAL, idx=idx, stream=stream)
+                if kind == "sparse":
+                    sala.block_topk(q, kbar, TOPK, N_INIT, N_LOCAL, idx=idx, stream=stream)
+                else:
+                    sala.block_topk_qblock(q, kbar, TOPK, N_INIT, N_LOCAL, idx=idx, stream=stream)
                 union += tile_union_blocks(torch, idx)
                 n_sp += 1
     res["sparse_exec_flops"] = EXEC_FLOPS_PER_TILE_BLOCK * union / max(1, n_sp)
@@ -739,14 +747,15 @@ def main():
             line["config"]["workload"] = f"{args.workload}: {len(kinds)} x {kinds[0]} layer, N={n_tok}"
             line["config"]["seq_len"] = n_tok
         line["kernels"] = {}
-        if "sparse" in kinds:
+        if "sparse" in kinds or "sparse_qblock" in kinds:
             fl = sparse_layer_flops(n_tok)
             achieved = fl / (pre["sparse_ms"] / 1000.0) / 1e12
             executed = pre["sparse_exec_flops"] / (pre["sparse_ms"] / 1000.0) / 1e12
             peak = peaks["bf16_tflops_sustained"]
             line["roofline"] = {"kernel": "sparse_prefill_tc_kernel", "bound": "tensor",
                                 "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                                "frac": achieved / peak, "traffic": sparse_traffic(n_tok),
+                                "frac": achieved / peak,
+                                "traffic": sparse_traffic(n_tok) if "sparse" in kinds else None,
                                 "peak_source": f"{peaks['source']} bf16 sustained",
                                 "algorithmic_flops_per_launch": fl,
                                 "mean_launch_ms": pre["sparse_ms"],

@@ -315,6 +315,23 @@ sala_status sala_block_topk(const void* q, const void* kbar, int32_t* idx, int B
                     "block_topk");
 }
 
+sala_status sala_block_topk_qblock(const void* q, const void* kbar, int32_t* idx, int B, int H,
+                                   int Hkv, int Nq, int nb, int d, int block, int topk, int n_init,
+                                   int n_local, sala_dtype dt, sala_stream stream) {
+    sala_status s = check_select_args(B, H, Hkv, Nq, 0, nb, d, block, topk, n_init, n_local, dt);
+    if (s != SALA_OK) return s;
+    if (B == 0 || H == 0 || Nq == 0) return SALA_OK;
+    REQ_PTR(q); REQUIRE(idx != nullptr, SALA_ERR_INVALID_ARG, "idx must be a device pointer");
+    if (nb > 0) REQ_PTR(kbar);
+    sala::DevCtx ctx;
+    s = get_ctx(&ctx);
+    if (s != SALA_OK) return s;
+    return launched(sala::launch_block_topk_qblock(to_dt(dt), q, kbar, idx, B, H, Hkv, Nq, nb, d,
+                                                   topk, n_init, n_local,
+                                                   static_cast<cudaStream_t>(stream), ctx),
+                    "block_topk_qblock");
+}
+
 // ----------------------------------------------------------------------------------------------
 sala_status sala_sparse_prefill(const void* q, const void* k, const void* v, const int32_t* idx,
                                 void* o, int B, int H, int Hkv, int N, int d, int block,

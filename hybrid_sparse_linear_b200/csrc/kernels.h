@@ -39,6 +39,11 @@ cudaError_t launch_linear_decode(DType dt, const void* q, const void* k, const v
 cudaError_t launch_block_compress(DType dt, const void* k, void* kbar, int B, int Hkv, int N,
                                   int d, int first_block, int n_blocks, int nb_cap,
                                   cudaStream_t st, DevCtx ctx);
+// Query-block-granular selection: one row per (batch, KV group, 64-token query block), written
+// to every token row of the block.
+cudaError_t launch_block_topk_qblock(DType dt, const void* q, const void* kbar, int32_t* idx, int B,
+                                     int H, int Hkv, int Nq, int nb, int d, int topk, int n_init,
+                                     int n_local, cudaStream_t st, DevCtx ctx);
 cudaError_t launch_block_topk_tiled(DType dt, const void* q, const void* kbar, int32_t* idx,
                                     int B, int H, int Hkv, int Nq, int q_pos0, int nb, int d,
                                     int topk, int n_init, int n_local, cudaStream_t st,

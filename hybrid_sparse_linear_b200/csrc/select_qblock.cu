@@ -1,0 +1,226 @@
+// Query-block-granular block selection (the variant of the selection step in which the tokens of
+// one query block share one selection): per (batch, KV group, query block c of 64 tokens) the
+// score vector is the sum of q over the group's G heads and the block's tokens, the candidates are
+// the blocks n_init .. c - n_local, the best k by (score, lower block first) join the forced init
+// and local blocks, and the resulting ascending row is written to every token row of the block,
+// in the layout of the per-token selection (so the sparse prefill takes it unchanged).
+//
+// One CTA per (batch, group, query block), 256 threads, on the CUDA cores (the scoring is a
+// matrix-vector product per block, ~0.5 % of the per-token selection's work):
+//   1. the summed query in fp32: thread = (4 columns, a stride of the G * 64 rows), partials
+//      reduced through shared memory;
+//   2. scores: one warp per candidate row of kbar (coalesced), four rows in flight per warp;
+//   3. the exact best k: chunks of kChunk candidates plus the best k so far, radix select
+//      (blocksel.cuh), winners carried to the next chunk;
+//   4. the winners sorted ascending by one warp, the slot row written to the block's token rows.
+#include "blocksel.cuh"
+#include "kernels.h"
+
+namespace sala {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kQB = 64;                    // tokens per query block (= key block)
+constexpr int kCapK = 64;                  // largest k that ranks
+constexpr int kE = 16;                     // keys per thread in one radix select
+constexpr int kChunk = kE * kThreads;      // keys per select: new candidates + carried winners
+constexpr int kNew = kChunk - kCapK;
+
+template <int D>
+struct QbSmem {
+    float part[kThreads / (D / 4)][D];     // partial sums of the query block
+    float qs[D];                           // the summed query
+    uint64_t keys[kChunk];                 // one chunk's keys, then the carried winners
+    uint64_t carry[kCapK];
+    int win[kCapK];
+    int n_win;
+    RadixSelSmem rs;
+};
+
+// Ascending bitonic sort of 64 ints held two per lane (position 2 * lane + j).
+__device__ __forceinline__ void sort64_asc(int& x0, int& x1, int lane) {
+#pragma unroll
+    for (int k = 2; k <= 64; k <<= 1) {
+#pragma unroll
+        for (int s = k >> 1; s > 0; s >>= 1) {
+            if (s == 1) {
+                const bool asc = ((2 * lane) & k) == 0;
+                const int lo = min(x0, x1), hi = max(x0, x1);
+                x0 = asc ? lo : hi;
+                x1 = asc ? hi : lo;
+            } else {
+                const int lm = s >> 1;
+                const int y0 = __shfl_xor_sync(0xffffffffu, x0, lm);
+                const int y1 = __shfl_xor_sync(0xffffffffu, x1, lm);
+                const int p0 = 2 * lane, p1 = 2 * lane + 1;
+                const bool asc0 = (p0 & k) == 0, low0 = (p0 & s) == 0;
+                const bool asc1 = (p1 & k) == 0, low1 = (p1 & s) == 0;
+                x0 = (low0 == asc0) ? min(x0, y0) : max(x0, y0);
+                x1 = (low1 == asc1) ? min(x1, y1) : max(x1, y1);
+            }
+        }
+    }
+}
+
+template <typename T>
+__device__ __forceinline__ void load4(const T* p, float (&f)[4]);
+template <>
+__device__ __forceinline__ void load4<float>(const float* p, float (&f)[4]) {
+    const float4 v = *reinterpret_cast<const float4*>(p);
+    f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
+}
+template <>
+__device__ __forceinline__ void load4<__nv_bfloat16>(const __nv_bfloat16* p, float (&f)[4]) {
+    const uint2 v = *reinterpret_cast<const uint2*>(p);
+    f[0] = __uint_as_float(v.x << 16);
+    f[1] = __uint_as_float(v.x & 0xffff0000u);
+    f[2] = __uint_as_float(v.y << 16);
+    f[3] = __uint_as_float(v.y & 0xffff0000u);
+}
+
+// Partial dot product of a kbar row with the summed query: lane covers D / 32 elements.
+template <typename T, int D>
+__device__ __forceinline__ float dot_lane(const T* row, const float* qs, int lane) {
+    if constexpr (D == 128) {
+        float f[4];
+        load4<T>(row + 4 * lane, f);
+        return f[0] * qs[4 * lane] + f[1] * qs[4 * lane + 1] + f[2] * qs[4 * lane + 2] +
+               f[3] * qs[4 * lane + 3];
+    } else {
+        return to_f(row[2 * lane]) * qs[2 * lane] + to_f(row[2 * lane + 1]) * qs[2 * lane + 1];
+    }
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kThreads)
+topk_qblock_kernel(const T* __restrict__ q, const T* __restrict__ kbar, int32_t* __restrict__ idx,
+                   int H, int Hkv, int Nq, int nb, int topk, int n_init, int n_local, int slots) {
+    extern __shared__ __align__(16) unsigned char smraw[];
+    QbSmem<D>& sm = *reinterpret_cast<QbSmem<D>*>(smraw);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int nqb = (Nq + kQB - 1) / kQB;
+    const int64_t bg = blockIdx.x / nqb;
+    const int c = (int)(blockIdx.x % nqb);
+    const int64_t b = bg / Hkv;
+    const int g = (int)(bg % Hkv);
+    const int G = H / Hkv;
+    const int r0 = c * kQB, nr = min(Nq, r0 + kQB) - r0;
+    const int lo = n_init, hi = c - n_local;
+    const int ncand = hi - lo + 1;
+    int32_t* out = idx + (bg * Nq + r0) * (int64_t)slots;  // the block's first token row
+    if (ncand <= topk) {  // every candidate taken: blocks 0 .. c
+        for (int e = tid; e < nr * slots; e += kThreads) out[e] = (e % slots) <= c ? e % slots : -1;
+        return;
+    }
+    const int K = min(topk, kCapK);  // a ranking k is at most 64 (validated by the caller)
+
+    // 1. the summed query (fp32)
+    {
+        constexpr int kCG = D / 4, kRL = kThreads / kCG;
+        const int cg = tid % kCG, rl = tid / kCG;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        const int nrows = G * nr;
+#pragma unroll 4
+        for (int e = rl; e < nrows; e += kRL) {
+            const int h = e / nr, r = r0 + e % nr;
+            float f[4];
+            load4<T>(q + ((b * H + (int64_t)g * G + h) * Nq + r) * D + 4 * cg, f);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc[i] += f[i];
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) sm.part[rl][4 * cg + i] = acc[i];
+        if (tid < kCapK) sm.carry[tid] = 0ull;
+        __syncthreads();
+        if (tid < D) {
+            float s = 0.f;
+#pragma unroll
+            for (int w = 0; w < kRL; ++w) s += sm.part[w][tid];
+            sm.qs[tid] = s;
+        }
+        __syncthreads();
+    }
+
+    // 2.-3. scores chunk by chunk, the best K carried through a radix select per chunk
+    const T* kb = kbar + bg * (int64_t)nb * D;
+    auto sync = [] { __syncthreads(); };
+    for (int cb = 0; cb < ncand; cb += kNew) {
+        const int nc = min(kNew, ncand - cb);
+        for (int i0 = warp * 4; i0 < nc; i0 += (kThreads / 32) * 4) {
+            float dv[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                dv[u] = i0 + u < nc ? dot_lane<T, D>(kb + (int64_t)(lo + cb + i0 + u) * D, sm.qs, lane) : 0.f;
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) dv[u] += __shfl_xor_sync(0xffffffffu, dv[u], off);
+            if (lane < 4 && i0 + lane < nc) {
+                const float d = lane == 0 ? dv[0] : lane == 1 ? dv[1] : lane == 2 ? dv[2] : dv[3];
+                sm.keys[i0 + lane] = sel_key(d, lo + cb + i0 + lane);
+            }
+        }
+        for (int i = nc + tid; i < kNew; i += kThreads) sm.keys[i] = 0ull;
+        if (tid < kCapK) sm.keys[kNew + tid] = sm.carry[tid];
+        __syncthreads();
+        uint64_t key[kE];
+#pragma unroll
+        for (int e = 0; e < kE; ++e) key[e] = sm.keys[e * kThreads + tid];
+        if (tid == 0) sm.n_win = 0;
+        uint64_t prefix, mask;
+        radix_kth<kE>(key, K, sm.rs, prefix, mask, tid, sync);
+#pragma unroll
+        for (int e = 0; e < kE; ++e)
+            if (key[e] && (key[e] & mask) >= prefix) sm.carry[atomicAdd(&sm.n_win, 1)] = key[e];
+        __syncthreads();
+    }
+
+    // 4. winners ascending, then the slot row for every token of the block
+    if (warp == 0) {
+        int x0 = 2 * lane < K ? key_block(sm.carry[2 * lane]) : 0x7fffffff;
+        int x1 = 2 * lane + 1 < K ? key_block(sm.carry[2 * lane + 1]) : 0x7fffffff;
+        sort64_asc(x0, x1, lane);
+        sm.win[2 * lane] = x0;
+        sm.win[2 * lane + 1] = x1;
+    }
+    __syncthreads();
+    for (int e = tid; e < nr * slots; e += kThreads) {
+        const int s = e % slots;
+        int v;
+        if (s < n_init) v = s;
+        else if (s < n_init + K) v = sm.win[s - n_init];
+        else if (s < n_init + K + n_local) v = c - n_local + 1 + (s - n_init - K);
+        else v = -1;
+        out[e] = v;
+    }
+}
+
+template <typename T, int D>
+cudaError_t launch_qb(const void* q, const void* kbar, int32_t* idx, int B, int H, int Hkv, int Nq,
+                      int nb, int topk, int n_init, int n_local, cudaStream_t st) {
+    const int nqb = (Nq + kQB - 1) / kQB;
+    const int64_t grid = (int64_t)B * Hkv * nqb;
+    if (grid == 0) return cudaSuccess;
+    if (grid > 0x7fffffff) return cudaErrorNotSupported;
+    const int smem = (int)sizeof(QbSmem<D>);
+    cudaError_t e = ensure_smem<topk_qblock_kernel<T, D>>(smem);
+    if (e != cudaSuccess) return e;
+    topk_qblock_kernel<T, D><<<(unsigned)grid, kThreads, smem, st>>>(
+        static_cast<const T*>(q), static_cast<const T*>(kbar), idx, H, Hkv, Nq, nb, topk, n_init,
+        n_local, n_init + n_local + topk);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_block_topk_qblock(DType dt, const void* q, const void* kbar, int32_t* idx, int B,
+                                     int H, int Hkv, int Nq, int nb, int d, int topk, int n_init,
+                                     int n_local, cudaStream_t st, DevCtx) {
+    if (dt == DType::F32)
+        return d == 64 ? launch_qb<float, 64>(q, kbar, idx, B, H, Hkv, Nq, nb, topk, n_init, n_local, st)
+                       : launch_qb<float, 128>(q, kbar, idx, B, H, Hkv, Nq, nb, topk, n_init, n_local, st);
+    return d == 64 ? launch_qb<__nv_bfloat16, 64>(q, kbar, idx, B, H, Hkv, Nq, nb, topk, n_init, n_local, st)
+                   : launch_qb<__nv_bfloat16, 128>(q, kbar, idx, B, H, Hkv, Nq, nb, topk, n_init, n_local, st);
+}
+
+}  // namespace sala

@@ -38,6 +38,7 @@ _lib.sala_block_compress.argtypes = [_vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _
 _lib.sala_block_topk.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp,
                                  _st, _i, _vp]
 _lib.sala_block_topk_workspace.argtypes = [_i, _i, _i, _i, _i, _i, _i]
+_lib.sala_block_topk_qblock.argtypes = [_vp, _vp, _vp] + [_i] * 11 + [_vp]
 _lib.sala_block_topk_workspace.restype = _st
 _lib.sala_sparse_prefill.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i,
                                      ctypes.c_float, _i, _vp]
@@ -57,7 +58,8 @@ _lib.sala_last_error.restype = ctypes.c_char_p
 _lib.sala_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
 _lib.sala_selftest_wait_timeout.argtypes = [_vp]
 for _f in ("sala_linear_prefill", "sala_linear_decode", "sala_linear_prefill_rope",
-           "sala_linear_decode_rope", "sala_sparse_decode_paged", "sala_block_compress",
+           "sala_linear_decode_rope", "sala_sparse_decode_paged", "sala_block_topk_qblock",
+           "sala_block_compress",
            "sala_block_topk",
            "sala_sparse_prefill", "sala_sparse_decode", "sala_check_status",
            "sala_selftest_wait_timeout"):
@@ -196,6 +198,22 @@ def block_topk(q, kbar, topk, n_init=1, n_local=1, block=64, q_pos0=0, idx=None,
                                 block, topk, n_init, n_local, _ptr(workspace),
                                 0 if workspace is None else workspace.numel(), _dt(q),
                                 _stream(stream)), "sala_block_topk")
+    return idx
+
+
+def block_topk_qblock(q, kbar, topk, n_init, n_local, idx=None, block=64, stream=None):
+    """Query-block-granular selection (one selection per KV group and query block, written to
+    every token row).  q: [B,H,Nq,d]; kbar [B,Hkv,nb,d].  Returns idx [B,Hkv,Nq,slots] int32."""
+    B, H, Nq, d = q.shape
+    Hkv, nb = kbar.shape[1], kbar.shape[2]
+    slots = n_init + n_local + topk
+    _need(q, "q"); _need(kbar, "kbar", dtype=q.dtype)
+    if idx is None:
+        idx = torch.empty((B, Hkv, Nq, slots), dtype=torch.int32, device=q.device)
+    _need(idx, "idx", (B, Hkv, Nq, slots), torch.int32)
+    _check(_lib.sala_block_topk_qblock(_ptr(q), _ptr(kbar), _ptr(idx), B, H, Hkv, Nq, nb, d, block,
+                                       topk, n_init, n_local, _dt(q), _stream(stream)),
+           "sala_block_topk_qblock")
     return idx
 
 

@@ -171,6 +171,21 @@ sala_status sala_block_topk(const void* q, const void* kbar, int32_t* idx, int B
                             sala_stream stream);
 size_t sala_block_topk_workspace(int B, int Hkv, int Nq, int q_pos0, int nb, int block, int topk);
 
+/* Query-block-granular selection: the tokens of one query block share one selection.  A variant of
+ * the selection step, which the pages describe (InfLLM-V2 selects blocks by a coarse score) without
+ * fixing its granularity.  For each (batch, KV group, query block c of `block` tokens, the last one
+ * possibly partial) the score of candidate b is (sum over the group's heads and the block's tokens
+ * of q) . kbar_b; candidates, forced blocks, ties and the row layout are those of sala_block_topk
+ * with q_pos0 = 0, and the row is written to every token of the block, so sala_sparse_prefill takes
+ * idx unchanged.  The scores are fp32 on CUDA cores.
+ * q   : [B, H, Nq, d] device, dt.   kbar : [B, Hkv, nb, d] device, dt.
+ * idx : [B, Hkv, Nq, n_init + n_local + topk] int32 device (output).
+ * Validation and errors as sala_block_topk (block = 64; topk <= 64 whenever a block has more
+ * than topk candidates). */
+sala_status sala_block_topk_qblock(const void* q, const void* kbar, int32_t* idx, int B, int H,
+                                   int Hkv, int Nq, int nb, int d, int block, int topk, int n_init,
+                                   int n_local, sala_dtype dt, sala_stream stream);
+
 /* ------------------------------------------------------------------------------------------
  * Sparse attention prefill: exact causal softmax over the selected blocks.  Pages: sparse
  * layers compute on selected parts but keep the dense KV cache ("sparse compute, dense

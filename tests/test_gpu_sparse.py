@@ -285,3 +285,49 @@ def test_sparse_decode_paged_bad_page_is_flagged(sala):
     table[0, 0] = 0 if int(table[1, 0]) != 0 else 1
     sala.sparse_decode_paged(q, kp, vp, table, kbar, pos, max(lengths) - 1, 16, 1, 2)
     sala.check_status()
+
+
+# ---------------------------------------------------------------------------------------------
+# Query-block-granular selection (sala_block_topk_qblock)
+
+@pytest.mark.parametrize("N,topk,dtype,d,H,Hkv", [
+    (64 * 200 + 7, 64, torch.bfloat16, 128, 32, 2),   # 16 heads per group, partial last block
+    (64 * 30 + 5, 8, torch.float32, 64, 8, 2),        # fp32, d 64
+    (64 * 4500 + 9, 64, torch.bfloat16, 128, 2, 1),   # > 4032 candidates: winners carried over chunks
+])
+def test_qblock_selection(sala, N, topk, dtype, d, H, Hkv):
+    from hybrid_sparse_linear_b200 import synth
+    layer = synth.sparse_layer(1, H, Hkv, N, d, dtype, layer=13, shift_frac=0.05)
+    kind = "bf16" if dtype == torch.bfloat16 else "f32"
+    q, k = layer.q.cuda(), layer.k.cuda()
+    kbar = sala.block_compress(k)
+    idx = sala.block_topk_qblock(q, kbar, topk, 1, 2)
+    sala.check_status()
+    kbar_ref = oracle.block_compress(_f64(layer.k), 64, round_to_bf16=(kind == "bf16"))
+    if kind == "f32":
+        kbar_ref = kbar_ref.astype(np.float32).astype(np.float64)
+    np.testing.assert_array_equal(_f64(kbar), kbar_ref)
+    q64 = _f64(layer.q)
+    ref, kth = oracle.block_select_qblock(q64, kbar_ref, 64, topk, 1, 2)
+    got = idx.cpu().numpy()
+    for r0 in range(0, N, 64):   # one row per query block on the GPU too
+        assert (got[:, :, r0:r0 + 64] == got[:, :, r0:r0 + 1]).all(), r0
+    check_selection(got, ref, oracle.qblock_sum(q64, 64), kbar_ref, kth, topk, 1, 2)
+
+
+def test_qblock_pipeline(sala):
+    # sparse prefill over query-block selections (every unit of 16 tokens shares one selection)
+    from hybrid_sparse_linear_b200 import synth
+    N, topk = 64 * 90 + 21, 32
+    layer = synth.sparse_layer(1, 32, 2, N, 128, torch.bfloat16, layer=14, shift_frac=0.05)
+    q, k, v = layer.q.cuda(), layer.k.cuda(), layer.v.cuda()
+    kbar = sala.block_compress(k)
+    idx = sala.block_topk_qblock(q, kbar, topk, 1, 2)
+    o = sala.sparse_prefill(q, k, v, idx)
+    sala.check_status()
+    q64, k64, v64 = _f64(layer.q), _f64(layer.k), _f64(layer.v)
+    kbar_ref = oracle.block_compress(k64, 64, round_to_bf16=True)
+    ref, kth = oracle.block_select_qblock(q64, kbar_ref, 64, topk, 1, 2)
+    got = idx.cpu().numpy()
+    check_selection(got, ref, oracle.qblock_sum(q64, 64), kbar_ref, kth, topk, 1, 2)
+    assert_close(_f64(o), oracle.sparse_attention(q64, k64, v64, got, 64), "bf16", "o")
