@@ -144,6 +144,26 @@ def linear_chunked(q, k, v, lam, chunk, s_in=None, threads=None):
     return o, s_out
 
 
+def linear_backward(q, k, v, lam, do):
+    """Gradients (dq, dk, dv) of sum(o * do), o the linear attention of a fresh sequence (no
+    carried state), by fp64 autograd through the plain quadratic form
+    o = ((Q K^T) * Dmask) V with Dmask[i, j] = lam^(i - j) for j <= i, 0 above the diagonal.
+    (plain PyTorch CPU ops; the contract's backward pass of the linear layers.)"""
+    import torch
+    t = lambda x: torch.tensor(_f64(x), dtype=torch.float64)
+    Q, K, V, dO = (t(x).requires_grad_(r) for x, r in ((q, True), (k, True), (v, True), (do, False)))
+    lam_t = t(lam)
+    N = Q.shape[2]
+    i = torch.arange(N, dtype=torch.float64)
+    diff = i[:, None] - i[None, :]
+    causal = diff >= 0
+    Dm = torch.where(causal, lam_t[:, None, None] ** diff.clamp(min=0), torch.zeros(()))  # [H, N, N]
+    A = (Q @ K.transpose(-1, -2)) * Dm
+    O = A @ V
+    (O * dO).sum().backward()
+    return Q.grad.numpy(), K.grad.numpy(), V.grad.numpy()
+
+
 def linear_decode(q, k, v, lam, state):
     """One decode step.  q,k: [B,H,dk]; v: [B,H,dv]; state [B,H,dk,dv].  Returns (o, new_state)."""
     q, k, v, lam = _f64(q), _f64(k), _f64(v), _f64(lam)
