@@ -400,6 +400,31 @@ def run_decode_paged(sala, synth, torch, steps, warmup, stream, B=8):
     return {"us_per_call": us, "bytes": nbytes, "lengths": lengths}
 
 
+def run_linear_backward(sala, synth, torch, steps, warmup, stream, n_tok=N_TOK):
+    """The backward pass of one linear layer (dq, dk, dv from dout) at N tokens, 32 heads."""
+    dev = torch.device("cuda")
+    q, k, v = synth.linear_layer(1, H, n_tok, D, torch.bfloat16, dev, layer=0)
+    dout = synth.linear_layer(1, H, n_tok, D, torch.bfloat16, dev, layer=1)[0]
+    lam = synth.decays(H).to(dev)
+    ws = torch.empty(max(sala._lib.sala_linear_backward_workspace(1, H, n_tok, D, 1), 16),
+                     dtype=torch.uint8, device=dev)
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            sala.linear_backward(q, k, v, lam, dout, workspace=ws, stream=stream)
+        torch.cuda.synchronize()
+        a, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(steps):
+            sala.linear_backward(q, k, v, lam, dout, workspace=ws, stream=stream)
+        e.record(stream)
+        torch.cuda.synchronize()
+    sala.check_status(stream)
+    ms = a.elapsed_time(e) / steps
+    del q, k, v, dout, ws
+    torch.cuda.empty_cache()
+    return {"ms": ms, "bytes": 7.0 * H * n_tok * D * 2}  # read q, k, v, dout; write dq, dk, dv
+
+
 def run_decode(sala, synth, torch, steps, warmup, stream, T=DECODE_T):
     """Decode at a T-token context (2^20 by default), 24 linear + 8 sparse layers per token, L2
     flushed."""
@@ -671,7 +696,7 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=0.0,
                     help="seconds of oracle work per CPU-baseline sample (0: the default sizing)")
     ap.add_argument("--phases", default="prefill,decode,e2e,cpu",
-                    help="comma list of prefill,decode,e2e,cpu,paged (default: all but paged)")
+                    help="comma list of prefill,decode,e2e,cpu,paged,backward (default: the first four)")
     ap.add_argument("--decode-steps", type=int, default=200)
     ap.add_argument("--decode-t", type=int, default=DECODE_T,
                     help="decode context length (default 2^20, the benchmark; smaller only for profiles)")
@@ -775,6 +800,14 @@ def main():
                                     "peak_source": f"{peaks['source']} HBM copy",
                                     "algorithmic_bytes_per_launch": linear_layer_bytes(n_tok),
                                     "mean_launch_ms": pre["linear_ms"]}
+    if "backward" in phases:
+        bw = run_linear_backward(sala, synth, torch, max(args.steps, 3), max(3, args.warmup), stream)
+        gbs = bw["bytes"] / (bw["ms"] * 1e-3) / 1e9
+        line["linear_backward"] = {"metric": "linear-attention backward ms per layer @256K (dq, dk, dv)",
+                                   "ms": bw["ms"], "algorithmic_bytes": bw["bytes"],
+                                   "achieved_gbs": gbs, "hbm_frac": gbs / peaks["hbm_gbs"],
+                                   "composition": "three forward linear attentions (two of the "
+                                                  "reversed sequence) and six row reversals"}
     if "paged" in phases:
         pg = run_decode_paged(sala, synth, torch, args.decode_steps, max(3, args.warmup), stream)
         gbs = pg["bytes"] / (pg["us_per_call"] * 1e-6) / 1e9

@@ -5,7 +5,9 @@
 #include <string.h>
 
 #include <atomic>
+#include <initializer_list>
 #include <mutex>
+#include <utility>
 
 #include "../../include/sala.h"
 #include "kernels.h"
@@ -189,6 +191,71 @@ sala_status sala_linear_prefill_rope(const void* q, const void* k, const void* v
             "rope_base %g (must lie in (1, 1e30))", rope_base);
     return linear_prefill_impl(q, k, v, decay, o, state_in, state_out, B, H, N, d, 0, workspace,
                                workspace_bytes, sala::Rope{rope_base, pos0}, dt, stream);
+}
+
+// Backward pass of the linear attention of a fresh sequence: with o_i = sum_{j<=i} lambda^{i-j}
+// (q_i . k_j) v_j and the upstream gradient do,
+//   dq_i = sum_{j<=i} lambda^{i-j} (do_i . v_j) k_j          = LA(q: do, k: v, v: k)_i
+//   dk_j = sum_{i>=j} lambda^{i-j} (do_i . v_j) q_i          = flip(LA(flip v, flip do, flip q))_j
+//   dv_j = sum_{i>=j} lambda^{i-j} (q_i . k_j) do_i          = flip(LA(flip k, flip q, flip do))_j
+// (the anti-causal sums are causal sums of the reversed sequence), so the forward kernels compute
+// all three; the workspace holds the reversed copies.
+size_t sala_linear_backward_workspace(int B, int H, int N, int d, sala_dtype dt) {
+    if (B <= 0 || H <= 0 || N <= 0 || (d != 64 && d != 128)) return 0;
+    auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    const size_t t = up((size_t)B * H * N * d * (dt == SALA_F32 ? 4 : 2));
+    return 5 * t + up(sala_linear_prefill_workspace(B, H, N, d, dt));
+}
+
+sala_status sala_linear_backward(const void* q, const void* k, const void* v, const float* decay,
+                                 const void* dout, void* dq, void* dk, void* dv, int B, int H, int N,
+                                 int d, void* workspace, size_t workspace_bytes, sala_dtype dt,
+                                 sala_stream stream) {
+    REQUIRE(B >= 0 && H >= 0 && N >= 0, SALA_ERR_INVALID_ARG, "negative size (B=%d H=%d N=%d)", B, H, N);
+    REQUIRE(dt == SALA_F32 || dt == SALA_BF16, SALA_ERR_INVALID_ARG, "unknown dtype %d", (int)dt);
+    REQUIRE(d == 64 || d == 128, SALA_ERR_UNSUPPORTED, "head dim %d (supported: 64, 128)", d);
+    if (B == 0 || H == 0 || N == 0) return SALA_OK;
+    REQ_PTR(q); REQ_PTR(k); REQ_PTR(v); REQ_PTR(dout); REQ_PTR(dq); REQ_PTR(dk); REQ_PTR(dv);
+    REQUIRE(decay != nullptr, SALA_ERR_INVALID_ARG, "decay must be a device pointer");
+    const size_t need = sala_linear_backward_workspace(B, H, N, d, dt);
+    REQUIRE(workspace != nullptr && aligned16(workspace) && workspace_bytes >= need,
+            SALA_ERR_INVALID_ARG, "workspace of %zu bytes (16-byte aligned) required, got %zu",
+            need, workspace_bytes);
+    sala::DevCtx ctx;
+    sala_status s = get_ctx(&ctx);
+    if (s != SALA_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    const size_t t = up((size_t)B * H * N * d * (dt == SALA_F32 ? 4 : 2));
+    char* w = static_cast<char*>(workspace);
+    void* fv = w;
+    void* fdo = w + t;
+    void* fq = w + 2 * t;
+    void* fk = w + 3 * t;
+    void* fo = w + 4 * t;
+    void* lws = w + 5 * t;
+    const size_t lws_bytes = workspace_bytes - 5 * t;
+    const sala::DType tdt = to_dt(dt);
+    const int64_t BH = (int64_t)B * H;
+    auto la = [&](const void* a, const void* b_, const void* c, void* o) {
+        return linear_prefill_impl(a, b_, c, decay, o, nullptr, nullptr, B, H, N, d, 0, lws,
+                                   lws_bytes, sala::Rope{0.0, 0}, dt, stream);
+    };
+    s = la(dout, v, k, dq);
+    if (s != SALA_OK) return s;
+    for (auto pr : {std::make_pair(v, fv), std::make_pair(dout, fdo), std::make_pair(q, fq),
+                    std::make_pair(k, fk)}) {
+        const cudaError_t e = sala::launch_flip_rows(tdt, pr.first, pr.second, BH, N, d, st);
+        if (e != cudaSuccess) return launched(e, "linear_backward flip");
+    }
+    s = la(fv, fdo, fq, fo);
+    if (s != SALA_OK) return s;
+    cudaError_t e = sala::launch_flip_rows(tdt, fo, dk, BH, N, d, st);
+    if (e != cudaSuccess) return launched(e, "linear_backward flip");
+    s = la(fk, fq, fdo, fo);
+    if (s != SALA_OK) return s;
+    e = sala::launch_flip_rows(tdt, fo, dv, BH, N, d, st);
+    return launched(e, "linear_backward flip");
 }
 
 static sala_status linear_decode_impl(const void* q, const void* k, const void* v,

@@ -97,6 +97,10 @@ cudaError_t launch_sparse_decode_attn(DType dt, const void* q, const void* kc, c
                                       int pos, int Tmax, int d, int slots, float scale, void* ws,
                                       cudaStream_t st, DevCtx ctx);
 
+// Row reversal of [BH][N][d] tensors (out must not overlap in).
+cudaError_t launch_flip_rows(DType dt, const void* in, void* out, int64_t BH, int N, int d,
+                             cudaStream_t st);
+
 // Diagnostics.
 cudaError_t launch_selftest_wait(cudaStream_t st, DevCtx ctx);
 

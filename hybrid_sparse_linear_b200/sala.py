@@ -31,6 +31,9 @@ _lib.sala_linear_prefill_ws.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _
 _lib.sala_linear_prefill_workspace.argtypes = [_i, _i, _i, _i, _i]
 _lib.sala_linear_prefill_workspace.restype = ctypes.c_size_t
 _lib.sala_linear_decode.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp]
+_lib.sala_linear_backward.argtypes = [_vp] * 8 + [_i] * 4 + [_vp, _st, _i, _vp]
+_lib.sala_linear_backward_workspace.argtypes = [_i] * 5
+_lib.sala_linear_backward_workspace.restype = _st
 _lib.sala_linear_prefill_rope.argtypes = [_vp] * 7 + [_i] * 4 + [ctypes.c_int64, ctypes.c_double,
                                                               _vp, _st, _i, _vp]
 _lib.sala_linear_decode_rope.argtypes = [_vp] * 6 + [_i] * 3 + [ctypes.c_int64, ctypes.c_double, _i, _vp]
@@ -59,6 +62,7 @@ _lib.sala_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
 _lib.sala_selftest_wait_timeout.argtypes = [_vp]
 for _f in ("sala_linear_prefill", "sala_linear_decode", "sala_linear_prefill_rope",
            "sala_linear_decode_rope", "sala_sparse_decode_paged", "sala_block_topk_qblock",
+           "sala_linear_backward",
            "sala_block_compress",
            "sala_block_topk",
            "sala_sparse_prefill", "sala_sparse_decode", "sala_check_status",
@@ -144,6 +148,24 @@ def linear_prefill(q, k, v, decay, o=None, state_in=None, state_out=None, chunk=
                                            _ptr(workspace), workspace.numel(), _dt(q),
                                            _stream(stream)), "sala_linear_prefill_ws")
     return o
+
+
+def linear_backward(q, k, v, decay, dout, workspace=None, stream=None):
+    """Gradients (dq, dk, dv) of sum(o * dout) for the linear attention of a fresh sequence.
+    q, k, v, dout: [B,H,N,d]; decay [H] fp32."""
+    B, H, N, d = q.shape
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (dout, "dout")):
+        _need(t, n, q.shape, q.dtype)
+    _need(decay, "decay", (H,), torch.float32)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    need = _lib.sala_linear_backward_workspace(B, H, N, d, _dt(q))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    _check(_lib.sala_linear_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(decay), _ptr(dout), _ptr(dq),
+                                     _ptr(dk), _ptr(dv), B, H, N, d, _ptr(workspace),
+                                     workspace.numel(), _dt(q), _stream(stream)),
+           "sala_linear_backward")
+    return dq, dk, dv
 
 
 def linear_decode(q, k, v, decay, state, o=None, stream=None, rope_base=None, pos=0):

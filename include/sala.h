@@ -124,6 +124,24 @@ sala_status sala_linear_prefill_rope(const void* q, const void* k, const void* v
                                      double rope_base, void* workspace, size_t workspace_bytes,
                                      sala_dtype dt, sala_stream stream);
 
+/* Backward pass of the linear attention of a fresh sequence (no carried state): the gradients of
+ * sum(o * dout) with respect to q, k and v, o as in sala_linear_prefill.  (The method is produced
+ * by continual training through these layers: MiniCPM-SALA summaries, JA section 2 "Method", DE
+ * section 3 on the training stages.)  With the upstream gradient dout:
+ *   dq_i = sum_{j<=i} lambda^{i-j} (dout_i . v_j) k_j
+ *   dk_j = sum_{i>=j} lambda^{i-j} (dout_i . v_j) q_i
+ *   dv_j = sum_{i>=j} lambda^{i-j} (q_i . k_j) dout_i
+ * Each is a linear attention (the anti-causal ones of the reversed sequence), computed by the
+ * forward kernels; the decay is not differentiated (it is a fixed per-head constant here).
+ * q, k, v, dout, dq, dk, dv : [B, H, N, d] device, dt (outputs must not overlap the inputs).
+ * workspace : at least sala_linear_backward_workspace(B, H, N, d, dt) bytes (16-byte aligned).
+ * Validation and errors as sala_linear_prefill. */
+sala_status sala_linear_backward(const void* q, const void* k, const void* v, const float* decay,
+                                 const void* dout, void* dq, void* dk, void* dv, int B, int H, int N,
+                                 int d, void* workspace, size_t workspace_bytes, sala_dtype dt,
+                                 sala_stream stream);
+size_t sala_linear_backward_workspace(int B, int H, int N, int d, sala_dtype dt);
+
 /* sala_linear_decode with q and k rotated at position pos (>= 0), as sala_linear_prefill_rope. */
 sala_status sala_linear_decode_rope(const void* q, const void* k, const void* v,
                                     const float* decay, float* state, void* o, int B, int H,

@@ -250,3 +250,27 @@ def test_rope_decode_fp32(sala, d):
     o_ref, s_ref = oracle.linear_decode(rq, rk, _f64(v), _f64(lam), _f64(S0))
     assert_close(_f64(o), o_ref, "f32", "rope decode o")
     assert_close(_f64(S), s_ref, "f32", "rope decode state")
+
+
+# ---------------------------------------------------------------------------------------------
+# Backward pass of the linear attention (sala_linear_backward)
+
+@pytest.mark.parametrize("d,N,B,H,dtype", [
+    (128, 333, 2, 3, torch.bfloat16),    # tensor cores, one pass
+    (128, 3000, 1, 4, torch.bfloat16),   # tensor cores, parallel segments
+    (64, 150, 1, 2, torch.float32),      # CUDA cores, fp32
+    (128, 65, 1, 2, torch.float32),
+])
+def test_linear_backward(sala, d, N, B, H, dtype):
+    from hybrid_sparse_linear_b200 import synth
+    q, k, v = _inputs(B, H, N, d, dtype, 700 + N)
+    g = torch.Generator().manual_seed(7)
+    dout = (torch.randn((B, H, N, d), generator=g) / math.sqrt(d)).to(dtype)
+    lam = synth.decays(H)
+    dq, dk, dv = sala.linear_backward(q.cuda(), k.cuda(), v.cuda(), lam.cuda(), dout.cuda())
+    sala.check_status()
+    rq, rk, rv = oracle.linear_backward(_f64(q), _f64(k), _f64(v), _f64(lam), _f64(dout))
+    kind = "bf16" if dtype == torch.bfloat16 else "f32"
+    assert_close(_f64(dq), rq, kind, "dq")
+    assert_close(_f64(dk), rk, kind, "dk")
+    assert_close(_f64(dv), rv, kind, "dv")
