@@ -56,6 +56,7 @@ def _load():
             lib.orc_linear_chunked.argtypes = [_D, _D, _D, _D, _D, _D, _D, _i, _i, _i, _i, _i, _i, _i]
             lib.orc_linear_decode.argtypes = [_D, _D, _D, _D, _D, _D, _i, _i, _i, _i]
             lib.orc_rope.argtypes = [_D, _i, _i, _i, _i, _l, ctypes.c_double]
+            lib.orc_qk_norm.argtypes = [_D, _l, _i, ctypes.c_double]
             lib.orc_block_compress.argtypes = [_D, _D, _i, _i, _i, _i, _i, _i, _i, _i]
             lib.orc_block_scores_at.argtypes = [_D, _D, _I64, _l, _D, _i, _i, _i, _i, _i]
             lib.orc_block_select.argtypes = [_D, _D, _I32, _D, _i, _i, _i, _i, _i, _i, _i, _i, _i,
@@ -66,7 +67,7 @@ def _load():
             lib.orc_dense_causal_attention.argtypes = [_D, _D, _D, _D, _i, _i, _i, _i, _i, _i, _i,
                                                        ctypes.c_double, _i]
             for name in ("orc_linear_recurrent", "orc_linear_quadratic", "orc_linear_chunked",
-                         "orc_linear_decode", "orc_block_compress", "orc_block_scores_at",
+                         "orc_linear_decode", "orc_qk_norm", "orc_block_compress", "orc_block_scores_at",
                          "orc_block_select", "orc_sparse_attention", "orc_dense_causal_attention"):
                 getattr(lib, name).restype = None
             _lib = lib
@@ -181,6 +182,15 @@ def rope(x, pos0=0, base=10000.0):
     B, H, N, d = x.shape
     assert d % 2 == 0
     _load().orc_rope(_p(x), B, H, N, d, int(pos0), float(base))
+    return x
+
+
+def qk_norm(x, eps=1e-6):
+    """Weight-free RMS normalisation of every head row of x [..., d] (QK normalisation); a
+    normalised copy."""
+    x = _f64(x).copy()
+    d = x.shape[-1]
+    _load().orc_qk_norm(_p(x), int(x.size // d), d, float(eps))
     return x
 
 

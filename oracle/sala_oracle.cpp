@@ -447,4 +447,21 @@ void orc_block_select_qblock(const double* q, const double* kbar, int32_t* idx, 
     });
 }
 
+// Weight-free RMS normalisation of every head row, in place on x [rows, d]:
+//   x'_c = x_c / sqrt((1/d) sum_e x_e^2 + eps).
+// MiniCPM-SALA summaries, DE section 2 "additional improvements": the model normalises queries
+// and keys (QK normalisation) to keep the activations stable.  The pages name the step without a
+// formula; the reading taken is an RMS norm over each head's d elements with no learned scale
+// (a learned per-channel scale, where a model has one, is an elementwise product after this),
+// applied to q and k of every layer before RoPE, block compression and selection.
+void orc_qk_norm(double* x, int64_t rows, int d, double eps) {
+    for (int64_t r = 0; r < rows; ++r) {
+        double* row = x + r * d;
+        double ss = 0.0;
+        for (int c = 0; c < d; ++c) ss += row[c] * row[c];
+        const double inv = 1.0 / std::sqrt(ss / d + eps);
+        for (int c = 0; c < d; ++c) row[c] *= inv;
+    }
+}
+
 }  // extern "C"
