@@ -425,6 +425,29 @@ def run_linear_backward(sala, synth, torch, steps, warmup, stream, n_tok=N_TOK):
     return {"ms": ms, "bytes": 7.0 * H * n_tok * D * 2}  # read q, k, v, dout; write dq, dk, dv
 
 
+def run_qk_norm(sala, synth, torch, steps, warmup, stream, n_tok=N_TOK):
+    """QK normalisation of one linear layer's q and k (32 heads each, d 128) at N tokens, in
+    place, one launch per call."""
+    dev = torch.device("cuda")
+    q = synth.prenorm((1, H, n_tok, D), synth.seed(0, synth.Q), dev, torch.bfloat16)
+    k = synth.prenorm((1, H, n_tok, D), synth.seed(0, synth.K), dev, torch.bfloat16)
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            sala.qk_norm(q, k, q_out=q, k_out=k, stream=stream)
+        torch.cuda.synchronize()
+        a, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(steps):
+            sala.qk_norm(q, k, q_out=q, k_out=k, stream=stream)
+        e.record(stream)
+        torch.cuda.synchronize()
+    sala.check_status(stream)
+    ms = a.elapsed_time(e) / steps
+    del q, k
+    torch.cuda.empty_cache()
+    return {"ms": ms, "bytes": 2.0 * 2 * H * n_tok * D * 2}  # q and k read once, written once
+
+
 def run_decode(sala, synth, torch, steps, warmup, stream, T=DECODE_T):
     """Decode at a T-token context (2^20 by default), 24 linear + 8 sparse layers per token, L2
     flushed."""
@@ -808,6 +831,15 @@ def main():
                                    "achieved_gbs": gbs, "hbm_frac": gbs / peaks["hbm_gbs"],
                                    "composition": "three forward linear attentions (two of the "
                                                   "reversed sequence) and six row reversals"}
+    if "qknorm" in phases:
+        qn = run_qk_norm(sala, synth, torch, max(args.steps, 5), max(3, args.warmup), stream)
+        gbs = qn["bytes"] / (qn["ms"] * 1e-3) / 1e9
+        line["qk_norm"] = {"metric": "QK normalisation ms per layer @256K (q and k, 32 heads each, "
+                                     "in place)",
+                           "ms": qn["ms"], "algorithmic_bytes": qn["bytes"], "achieved_gbs": gbs,
+                           "hbm_frac": gbs / peaks["hbm_gbs"],
+                           "timing": "CUDA events around back-to-back launches; 8.6 GB moved per "
+                                     "launch, far above L2"}
     if "paged" in phases:
         pg = run_decode_paged(sala, synth, torch, args.decode_steps, max(3, args.warmup), stream)
         gbs = pg["bytes"] / (pg["us_per_call"] * 1e-6) / 1e9

@@ -101,6 +101,11 @@ cudaError_t launch_sparse_decode_attn(DType dt, const void* q, const void* kc, c
 cudaError_t launch_flip_rows(DType dt, const void* in, void* out, int64_t BH, int N, int d,
                              cudaStream_t st);
 
+// Weight-free RMS normalisation of q rows [0, q_rows) and k rows [0, k_rows), d elements each;
+// outputs may alias their inputs exactly.
+cudaError_t launch_qk_norm(DType dt, const void* q, void* q_out, int64_t q_rows, const void* k,
+                           void* k_out, int64_t k_rows, int d, float eps, cudaStream_t st);
+
 // Diagnostics.
 cudaError_t launch_selftest_wait(cudaStream_t st, DevCtx ctx);
 

@@ -37,6 +37,8 @@ _lib.sala_linear_backward_workspace.restype = _st
 _lib.sala_linear_prefill_rope.argtypes = [_vp] * 7 + [_i] * 4 + [ctypes.c_int64, ctypes.c_double,
                                                               _vp, _st, _i, _vp]
 _lib.sala_linear_decode_rope.argtypes = [_vp] * 6 + [_i] * 3 + [ctypes.c_int64, ctypes.c_double, _i, _vp]
+_lib.sala_qk_norm.argtypes = [_vp, _vp, ctypes.c_int64, _vp, _vp, ctypes.c_int64, _i,
+                              ctypes.c_double, _i, _vp]
 _lib.sala_block_compress.argtypes = [_vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp]
 _lib.sala_block_topk.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp,
                                  _st, _i, _vp]
@@ -62,7 +64,7 @@ _lib.sala_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
 _lib.sala_selftest_wait_timeout.argtypes = [_vp]
 for _f in ("sala_linear_prefill", "sala_linear_decode", "sala_linear_prefill_rope",
            "sala_linear_decode_rope", "sala_sparse_decode_paged", "sala_block_topk_qblock",
-           "sala_linear_backward",
+           "sala_linear_backward", "sala_qk_norm",
            "sala_block_compress",
            "sala_block_topk",
            "sala_sparse_prefill", "sala_sparse_decode", "sala_check_status",
@@ -186,6 +188,28 @@ def linear_decode(q, k, v, decay, state, o=None, stream=None, rope_base=None, po
     _check(_lib.sala_linear_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(decay), _ptr(state), _ptr(o),
                                    B, H, d, _dt(q), _stream(stream)), "sala_linear_decode")
     return o
+
+
+def qk_norm(q, k=None, q_out=None, k_out=None, eps=1e-6, stream=None):
+    """Weight-free RMS normalisation of every head row (last dim d) of q and, if given, k, in
+    one launch.  Pass q_out=q / k_out=k to normalise in place.  Returns (q_out, k_out)."""
+    d = q.shape[-1]
+    _need(q, "q")
+    if q_out is None:
+        q_out = torch.empty_like(q)
+    _need(q_out, "q_out", q.shape, q.dtype)
+    k_rows = 0
+    if k is not None:
+        _need(k, "k", dtype=q.dtype)
+        if k.shape[-1] != d:
+            raise ValueError(f"k has head dim {k.shape[-1]}, q has {d}")
+        if k_out is None:
+            k_out = torch.empty_like(k)
+        _need(k_out, "k_out", k.shape, k.dtype)
+        k_rows = k.numel() // d
+    _check(_lib.sala_qk_norm(_ptr(q), _ptr(q_out), q.numel() // d, _ptr(k), _ptr(k_out), k_rows,
+                             d, float(eps), _dt(q), _stream(stream)), "sala_qk_norm")
+    return q_out, k_out
 
 
 def block_compress(k, kbar=None, block=64, first_block=0, n_blocks=None, stream=None):

@@ -61,6 +61,14 @@ def normal(shape, s: int, device="cpu", dtype=torch.float32, scale: float = 1.0,
     return out
 
 
+def prenorm(shape, s: int, device="cpu", dtype=torch.float32, spread: float = 3.0) -> torch.Tensor:
+    """q or k ahead of the QK normalisation: [B, heads, rows, d] standard normals, each row
+    scaled by e^u with u uniform in [-spread, spread] (row magnitudes from e^-3 to e^3)."""
+    x = normal(shape, s, device, torch.float32)
+    u = (torch.rand(tuple(shape[:-1]) + (1,), generator=_gen("cpu", s * 7919 + 1)) * 2 - 1) * spread
+    return (x * torch.exp(u).to(device)).to(dtype)
+
+
 def decays(H: int, kind: str = "geometric") -> torch.Tensor:
     """Per-head decay lambda_h as fp32 (an input of the method, not part of it)."""
     if kind == "tiny":

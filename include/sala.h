@@ -149,6 +149,26 @@ sala_status sala_linear_decode_rope(const void* q, const void* k, const void* v,
                                     sala_stream stream);
 
 /* ------------------------------------------------------------------------------------------
+ * QK normalisation (weight-free RMS norm of every head row).  Pages: MiniCPM-SALA normalises
+ * queries and keys to keep the activations stable (DE technical summary section 2, "additional
+ * improvements"); no formula is given, the reading taken is
+ *
+ *   y[r, c] = x[r, c] / sqrt( (1/d) * sum_e x[r, e]^2 + eps )
+ *
+ * over each row of d elements, no learned scale (a per-channel scale is an elementwise product
+ * the caller applies after this), for q and k of every layer ahead of RoPE, block compression
+ * and selection.  Squares are summed in fp32, the result rounded once to dt.
+ *   q, q_out   device, q_rows rows of d elements ([B, H, N, d] is B*H*N rows), dt
+ *   k, k_out   device, k_rows rows of d elements; may be NULL when k_rows == 0
+ *   eps        > 0 and finite
+ * Outputs may alias their inputs exactly (in place); partial overlap is not allowed.  All four
+ * pointers 16-byte aligned.  One launch covers both tensors.  d in {64, 128}.
+ * Errors: SALA_ERR_INVALID_ARG (negative rows, bad eps or pointer), SALA_ERR_UNSUPPORTED (d).
+ * ---------------------------------------------------------------------------------------- */
+sala_status sala_qk_norm(const void* q, void* q_out, int64_t q_rows, const void* k, void* k_out,
+                         int64_t k_rows, int d, double eps, sala_dtype dt, sala_stream stream);
+
+/* ------------------------------------------------------------------------------------------
  * Block compression of the keys of a sparse layer (mean pooling).  Pages: InfLLM-V2 selects
  * the relevant context parts without extra parameters (JA technical summary section 2.1); the
  * pooling itself is the plain reading of "mean-pooled block keys".
