@@ -296,3 +296,69 @@ def dense_causal_attention(q, k, v, scale=None, q_pos0=0, threads=None):
     _load().orc_dense_causal_attention(_p(q), _p(k), _p(v), _p(o), B, H, Hkv, Nq, int(q_pos0), Nk,
                                        d, scale, threads or default_threads())
     return o
+
+
+def _visible(idx_bg, N, block):
+    """[N, N] bool: key j visible to query row i (prefill, rows at positions 0..N-1) iff j's block
+    is in row i's selection and j <= i."""
+    import torch
+    nb = (N + block - 1) // block
+    sel = torch.zeros((N, nb + 1), dtype=torch.bool)
+    ids = torch.as_tensor(np.asarray(idx_bg, dtype=np.int64))
+    ids = torch.where(ids >= 0, ids, torch.full_like(ids, nb))  # padding -> a dummy column
+    sel.scatter_(1, ids, True)
+    j = torch.arange(N)
+    return sel[:, j // block] & (j[None, :] <= j[:, None])
+
+
+def sparse_lse(q, k, idx, block, scale=None):
+    """Natural log-sum-exp of each prefill row's visible logits scale * (q_i . k_j): [B, H, N]
+    (-inf where a row sees no key).  Plain PyTorch fp64."""
+    import torch
+    q, k = _f64(q), _f64(k)
+    B, H, N, d = q.shape
+    Hkv = k.shape[1]
+    G = H // Hkv
+    scale = (1.0 / np.sqrt(d)) if scale is None else float(scale)
+    out = np.empty((B, H, N))
+    for b in range(B):
+        for g in range(Hkv):
+            vis = _visible(idx[b, g], N, block)
+            K = torch.from_numpy(k[b, g])
+            for h in range(g * G, (g + 1) * G):
+                s = scale * (torch.from_numpy(q[b, h]) @ K.T)
+                out[b, h] = torch.logsumexp(s.masked_fill(~vis, -np.inf), dim=1).numpy()
+    return out
+
+
+def sparse_attention_backward(q, k, v, idx, do, block, scale=None):
+    """Gradients (dq, dk, dv) of sum(o * do), o the sparse attention of a prefill (rows at
+    positions 0..N-1) over the selected blocks idx [B, Hkv, N, slots], the selection held fixed
+    (the top-k choice is piecewise constant in q and k and passes no gradient).  fp64 autograd
+    through the plain masked softmax o_i = softmax_j(scale q_i . k_j, j visible) V, one query
+    head at a time; dk and dv sum the G heads of a KV group.  Every row must see a key.
+    (plain PyTorch CPU ops; the backward pass of the sparse layers.)"""
+    import torch
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    B, H, N, d = q.shape
+    Hkv = k.shape[1]
+    G = H // Hkv
+    scale = (1.0 / np.sqrt(d)) if scale is None else float(scale)
+    dq = np.empty_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    for b in range(B):
+        for g in range(Hkv):
+            vis = _visible(idx[b, g], N, block)
+            assert bool(vis.any(dim=1).all()), "a query row sees no key"
+            for h in range(g * G, (g + 1) * G):
+                Q = torch.tensor(q[b, h], requires_grad=True)
+                K = torch.tensor(k[b, g], requires_grad=True)
+                V = torch.tensor(v[b, g], requires_grad=True)
+                s = (scale * (Q @ K.T)).masked_fill(~vis, -np.inf)
+                o = torch.softmax(s, dim=1) @ V
+                gq, gk, gv = torch.autograd.grad((o * torch.from_numpy(do[b, h])).sum(), (Q, K, V))
+                dq[b, h] = gq.numpy()
+                dk[b, g] += gk.numpy()
+                dv[b, g] += gv.numpy()
+    return dq, dk, dv
