@@ -458,8 +458,9 @@ sala_status sala_sparse_prefill(const void* q, const void* k, const void* v, con
     if (s != SALA_OK) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (dt == SALA_BF16 && sala::sparse_prefill_tc_supported(H, Hkv, d))
-        return launched(sala::launch_sparse_prefill_tc(q, k, v, idx, o, B, H, Hkv, N, d, slots,
-                                                       scale, st, ctx), "sparse_prefill_tc");
+        return launched(sala::launch_sparse_prefill_tc(q, k, v, idx, o, nullptr, B, H, Hkv, N, d,
+                                                       slots, scale, st, ctx),
+                        "sparse_prefill_tc");
     return launched(sala::launch_sparse_prefill_simt(to_dt(dt), q, k, v, idx, o, B, H, Hkv, N, d,
                                                      slots, scale, st, ctx),
                     "sparse_prefill");
@@ -477,6 +478,100 @@ size_t sala_sparse_decode_workspace(int B, int H, int Hkv, int pos, int block, i
     const size_t multi = 256 + up(a) + up(sel) + up(idx_bytes);
     const size_t fused = up(sala::sparse_decode_fused_workspace(B, H, Hkv, pos, topk, n_init, n_local, d));
     return multi > fused ? multi : fused;
+}
+
+// Forward with the row statistic the backward needs (bf16, d 128, 16 query heads per KV head).
+sala_status sala_sparse_prefill_lse(const void* q, const void* k, const void* v,
+                                    const int32_t* idx, void* o, float* lse, int B, int H, int Hkv,
+                                    int N, int d, int block, int slots, float scale, sala_dtype dt,
+                                    sala_stream stream) {
+    REQUIRE(B >= 0 && H >= 0 && Hkv > 0 && N >= 0 && slots >= 1, SALA_ERR_INVALID_ARG,
+            "bad sizes (B=%d H=%d Hkv=%d N=%d slots=%d)", B, H, Hkv, N, slots);
+    REQUIRE(dt == SALA_F32 || dt == SALA_BF16, SALA_ERR_INVALID_ARG, "unknown dtype %d", (int)dt);
+    REQUIRE(isfinite(scale) && scale >= 0.f, SALA_ERR_INVALID_ARG, "scale must be finite and >= 0");
+    REQUIRE(dt == SALA_BF16 && d == 128 && H == 16 * Hkv && block == 64 && slots <= 80,
+            SALA_ERR_UNSUPPORTED, "the lse forward takes bf16, d 128, 16 query heads per KV head, "
+            "block 64 and at most 80 slots (got d=%d H=%d Hkv=%d block=%d slots=%d)", d, H, Hkv,
+            block, slots);
+    if (B == 0 || H == 0 || N == 0) return SALA_OK;
+    REQ_PTR(q); REQ_PTR(k); REQ_PTR(v); REQ_PTR(o);
+    REQUIRE(idx != nullptr && lse != nullptr, SALA_ERR_INVALID_ARG, "idx and lse must be device pointers");
+    if (scale == 0.f) scale = 1.0f / sqrtf((float)d);
+    sala::DevCtx ctx;
+    sala_status s = get_ctx(&ctx);
+    if (s != SALA_OK) return s;
+    return launched(sala::launch_sparse_prefill_tc(q, k, v, idx, o, lse, B, H, Hkv, N, d, slots,
+                                                   scale, static_cast<cudaStream_t>(stream), ctx),
+                    "sparse_prefill_lse");
+}
+
+// Backward pass of the sparse attention: the transposed selection, the query-side pass (D rows,
+// then dq), the key-side pass, then dk / dv rounded from their fp32 sums.
+static size_t sparse_bwd_ws_parts(int B, int H, int Hkv, int N, int slots, size_t* o_csr,
+                                  size_t* o_dk, size_t* o_dv) {
+    auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    const size_t delta = up((size_t)B * H * N * 4);
+    const size_t csr = up(sala::sparse_bwd_csr_layout(nullptr, B, Hkv, N, slots).bytes);
+    const size_t acc = up((size_t)B * Hkv * N * 128 * 4);
+    *o_csr = delta;
+    *o_dk = delta + csr;
+    *o_dv = delta + csr + acc;
+    return delta + csr + 2 * acc;
+}
+
+size_t sala_sparse_backward_workspace(int B, int H, int Hkv, int N, int d, int slots) {
+    if (B <= 0 || H <= 0 || Hkv <= 0 || N <= 0 || d != 128 || slots < 1) return 0;
+    size_t a, b, c;
+    return sparse_bwd_ws_parts(B, H, Hkv, N, slots, &a, &b, &c);
+}
+
+sala_status sala_sparse_backward(const void* q, const void* k, const void* v, const int32_t* idx,
+                                 const float* lse, const void* dout, void* dq,
+                                 void* dk, void* dv, int B, int H, int Hkv, int N, int d, int block,
+                                 int slots, float scale, void* workspace, size_t workspace_bytes,
+                                 sala_dtype dt, sala_stream stream) {
+    REQUIRE(B >= 0 && H >= 0 && Hkv > 0 && N >= 0 && slots >= 1, SALA_ERR_INVALID_ARG,
+            "bad sizes (B=%d H=%d Hkv=%d N=%d slots=%d)", B, H, Hkv, N, slots);
+    REQUIRE(dt == SALA_F32 || dt == SALA_BF16, SALA_ERR_INVALID_ARG, "unknown dtype %d", (int)dt);
+    REQUIRE(isfinite(scale) && scale >= 0.f, SALA_ERR_INVALID_ARG, "scale must be finite and >= 0");
+    REQUIRE(dt == SALA_BF16 && d == 128 && H == 16 * Hkv && block == 64 && slots <= 80,
+            SALA_ERR_UNSUPPORTED, "the sparse backward takes bf16, d 128, 16 query heads per KV "
+            "head, block 64 and at most 80 slots (got d=%d H=%d Hkv=%d block=%d slots=%d)", d, H,
+            Hkv, block, slots);
+    REQUIRE((int64_t)B * Hkv * N * slots < ((int64_t)1 << 31), SALA_ERR_UNSUPPORTED,
+            "B * Hkv * N * slots must stay below 2^31");
+    if (B == 0 || H == 0 || N == 0) return SALA_OK;
+    REQ_PTR(q); REQ_PTR(k); REQ_PTR(v); REQ_PTR(dout); REQ_PTR(dq); REQ_PTR(dk); REQ_PTR(dv);
+    REQUIRE(idx != nullptr && lse != nullptr, SALA_ERR_INVALID_ARG, "idx and lse must be device pointers");
+    size_t o_csr, o_dk, o_dv;
+    const size_t need = sparse_bwd_ws_parts(B, H, Hkv, N, slots, &o_csr, &o_dk, &o_dv);
+    REQUIRE(workspace != nullptr && aligned16(workspace) && workspace_bytes >= need,
+            SALA_ERR_INVALID_ARG, "workspace of %zu bytes (16-byte aligned) required, got %zu",
+            need, workspace_bytes);
+    if (scale == 0.f) scale = 1.0f / sqrtf((float)d);
+    sala::DevCtx ctx;
+    sala_status s = get_ctx(&ctx);
+    if (s != SALA_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    char* w = static_cast<char*>(workspace);
+    float* delta = reinterpret_cast<float*>(w);
+    const sala::SparseBwdCsr csr = sala::sparse_bwd_csr_layout(w + o_csr, B, Hkv, N, slots);
+    float* dk_acc = reinterpret_cast<float*>(w + o_dk);
+    float* dv_acc = reinterpret_cast<float*>(w + o_dv);
+    const size_t acc_bytes = (size_t)B * Hkv * N * 128 * 4;
+    cudaError_t e = sala::launch_sparse_bwd_csr(idx, B, Hkv, N, slots, csr, st, ctx);
+    if (e == cudaSuccess) e = cudaMemsetAsync(dk_acc, 0, acc_bytes, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(dv_acc, 0, acc_bytes, st);
+    if (e != cudaSuccess) return launched(e, "sparse_backward prologue");
+    e = sala::launch_sparse_dq_tc(q, k, v, dout, idx, lse, delta, dq, B, H, Hkv, N, slots, scale,
+                                  st, ctx);
+    if (e != cudaSuccess) return launched(e, "sparse_backward dq");
+    e = sala::launch_sparse_dkv_tc(q, k, v, dout, lse, delta, csr, dk_acc, dv_acc, B, H, Hkv, N,
+                                   scale, st, ctx);
+    if (e != cudaSuccess) return launched(e, "sparse_backward dk dv");
+    return launched(sala::launch_sparse_bwd_finish(dk_acc, dv_acc, dk, dv,
+                                                   (int64_t)B * Hkv * N * 128, scale, st),
+                    "sparse_backward finish");
 }
 
 sala_status sala_sparse_decode(const void* q, const void* kcache, const void* vcache,

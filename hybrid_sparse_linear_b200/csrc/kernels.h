@@ -64,9 +64,38 @@ cudaError_t launch_sparse_prefill_simt(DType dt, const void* q, const void* k, c
                                        const int32_t* idx, void* o, int B, int H, int Hkv, int N,
                                        int d, int slots, float scale, cudaStream_t st,
                                        DevCtx ctx);
+// lse (may be null): per query row, the natural log-sum-exp of its visible scaled logits.
 cudaError_t launch_sparse_prefill_tc(const void* q, const void* k, const void* v,
-                                     const int32_t* idx, void* o, int B, int H, int Hkv, int N,
-                                     int d, int slots, float scale, cudaStream_t st, DevCtx ctx);
+                                     const int32_t* idx, void* o, float* lse, int B, int H,
+                                     int Hkv, int N, int d, int slots, float scale, cudaStream_t st,
+                                     DevCtx ctx);
+
+// Sparse attention backward (bf16, G = 16, d = 128), selection held fixed.
+// The transposed selection: for key k = (b * Hkv + g) * nb + j, list[off[k] .. off[k+1]) holds
+// the query tokens whose selection row holds block j; off[n_keys] is the total.
+struct SparseBwdCsr {
+    int nb, n_keys;
+    int *cnt, *cur, *off, *list;
+    size_t bytes;  // workspace bytes the four arrays take
+};
+SparseBwdCsr sparse_bwd_csr_layout(void* ws, int B, int Hkv, int N, int slots);
+cudaError_t launch_sparse_bwd_csr(const int32_t* idx, int B, int Hkv, int N, int slots,
+                                  const SparseBwdCsr& c, cudaStream_t st, DevCtx ctx);
+// dq (bf16) from the query side: the forward's units walking the union of their selections
+// twice, first for D_i = sum_j P_ij dP_ij (written to delta, fp32 per query row), then for dq.
+cudaError_t launch_sparse_dq_tc(const void* q, const void* k, const void* v, const void* dout,
+                                const int32_t* idx, const float* lse, float* delta, void* dq,
+                                int B, int H, int Hkv, int N, int slots, float scale,
+                                cudaStream_t st, DevCtx ctx);
+// dk_acc, dv_acc (fp32, zeroed by the caller) += the key side: key blocks walking their
+// transposed lists; unscaled (dk_acc holds sum_i dS_ij q_i).
+cudaError_t launch_sparse_dkv_tc(const void* q, const void* k, const void* v, const void* dout,
+                                 const float* lse, const float* delta, const SparseBwdCsr& c,
+                                 float* dk_acc, float* dv_acc, int B, int H, int Hkv, int N,
+                                 float scale, cudaStream_t st, DevCtx ctx);
+// dk = bf16(scale * dk_acc), dv = bf16(dv_acc); n elements, a multiple of 4.
+cudaError_t launch_sparse_bwd_finish(const float* dk_acc, const float* dv_acc, void* dk, void* dv,
+                                     int64_t n, float scale, cudaStream_t st);
 bool sparse_prefill_tc_supported(int H, int Hkv, int d);
 size_t sparse_decode_attn_workspace(int B, int H, int Hkv, int slots, int d);
 // Sparse decode in one cooperative launch (scoring, top-k, attention, combine).  Returns

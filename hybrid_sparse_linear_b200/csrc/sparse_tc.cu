@@ -166,8 +166,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 sparse_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                          const __grid_constant__ CUtensorMap tmK,
                          const __grid_constant__ CUtensorMap tmV,
-                         const int32_t* __restrict__ idx, __nv_bfloat16* __restrict__ out, int H,
-                         int Hkv, int N, int slots, float sl2, int n_units, DevCtx ctx) {
+                         const int32_t* __restrict__ idx, __nv_bfloat16* __restrict__ out,
+                         float* __restrict__ lse, int H, int Hkv, int N, int slots, float sl2,
+                         int n_units, DevCtx ctx) {
     extern __shared__ uint8_t smraw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smraw) + 1023) &
                                              ~uintptr_t(1023));
@@ -531,8 +532,13 @@ sparse_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                 last = (int)a;
                 ++a;
             }
-            // Epilogue: O_x / l -> bf16 -> global (zeros when the tile saw no block).
+            // Epilogue: O_x / l -> bf16 -> global (zeros when the tile saw no block); with lse,
+            // the row's natural log-sum-exp ln(sum_j e^(scale s_j)) = (m_run + log2 l) ln 2.
             const int64_t orow = (((bg / Hkv) * H + (bg % Hkv) * kG + hh) * (int64_t)N + i) * kD;
+            if (lse != nullptr && i < N && !dead)
+                lse[orow / kD] = (last >= 0 && m_run != -INFINITY && l > 0.f)
+                                     ? (m_run + log2f(l)) * 0.69314718055994531f
+                                     : -INFINITY;
             if (last >= 0) {
                 if (!dead && !mbar_wait(&bars.pv_done[x][last & 1], ((uint32_t)last >> 1) & 1u, ctx)) fail();
                 if (!__any_sync(0xffffffffu, dead)) {
@@ -584,8 +590,9 @@ bool sparse_prefill_tc_supported(int H, int Hkv, int d) {
 }
 
 cudaError_t launch_sparse_prefill_tc(const void* q, const void* k, const void* v,
-                                     const int32_t* idx, void* o, int B, int H, int Hkv, int N,
-                                     int d, int slots, float scale, cudaStream_t st, DevCtx ctx) {
+                                     const int32_t* idx, void* o, float* lse, int B, int H,
+                                     int Hkv, int N, int d, int slots, float scale, cudaStream_t st,
+                                     DevCtx ctx) {
     if (d != kD || H != Hkv * kG || slots > kMaxSlots) return cudaErrorNotSupported;
     CUtensorMap tmQ, tmK, tmV;
     EncodeTiledFn fn = encode_tiled_fn();
@@ -618,7 +625,8 @@ cudaError_t launch_sparse_prefill_tc(const void* q, const void* k, const void* v
     const int grid = n_units < num_sms ? n_units : num_sms;
     const float sl2 = scale * 1.4426950408889634f;
     sparse_prefill_tc_kernel<<<grid, kThreads, kSmemBytes, st>>>(
-        tmQ, tmK, tmV, idx, static_cast<__nv_bfloat16*>(o), H, Hkv, N, slots, sl2, n_units, ctx);
+        tmQ, tmK, tmV, idx, static_cast<__nv_bfloat16*>(o), lse, H, Hkv, N, slots, sl2, n_units,
+        ctx);
     return cudaGetLastError();
 }
 

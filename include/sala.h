@@ -245,6 +245,45 @@ sala_status sala_sparse_prefill(const void* q, const void* k, const void* v, con
                                 int slots, float scale, sala_dtype dt, sala_stream stream);
 
 /* ------------------------------------------------------------------------------------------
+ * Training path of the sparse layers: the forward with its row statistic, and the backward pass.
+ * The method reaches its sparse layers by continual training through them (JA technical summary
+ * section 2, training phases; DE section 3 "Trainingsstrategie"); the pages give no formula, and
+ * the reading is the gradient of the sparse attention with the block selection held fixed (the
+ * top-k choice is piecewise constant in q and k and passes no gradient):
+ *   P_ij = exp(scale q_i.k_j - lse_i) over the visible keys j of row i,  D_i = do_i . o_i
+ *   dq_i = scale sum_j P_ij (do_i.v_j - D_i) k_j
+ *   dk_j = scale sum_i P_ij (do_i.v_j - D_i) q_i      (i over the KV group's query rows)
+ *   dv_j = sum_i P_ij do_i
+ *
+ * sala_sparse_prefill_lse: sala_sparse_prefill plus lse [B, H, N] fp32 (device, output), the
+ *   natural log of sum_j exp(scale q_i.k_j) over row i's visible keys (-inf for a row that sees
+ *   none).  Takes bf16, d 128, H = 16 Hkv, block 64, slots <= 80 (else SALA_ERR_UNSUPPORTED).
+ *
+ * sala_sparse_backward: q [B,H,N,d], k, v [B,Hkv,N,d], dout [B,H,N,d] (bf16, device), idx
+ *   [B,Hkv,N,slots] (the selection the forward used: ascending distinct block ids, -1 padded,
+ *   none in the future of its token), lse from sala_sparse_prefill_lse.  D_i is computed here
+ *   as sum_j P_ij dP_ij from the same fp32 P and dP that form dS (not as do_i . o_i from the
+ *   forward's bf16 o, whose rounding -- and that of the forward's bf16 P -- reaches every
+ *   dS_ij = P_ij (dP_ij - D_i) through the cancellation in dP_ij - D_i).  Writes dq [B,H,N,d] and
+ *   dk, dv [B,Hkv,N,d] (bf16, device, outputs; they must not alias the inputs).  scale 0 = 1/sqrt(d).
+ *   workspace: >= sala_sparse_backward_workspace(...) bytes, 16-byte aligned, not shared with a
+ *   concurrent call.  dk and dv are sums of fp32 atomic additions, so their last bits may vary
+ *   from run to run.  Same shape limits as above, and B * Hkv * N * slots < 2^31.  A selection
+ *   entry in the future of its token, past the last block or repeated is reported as
+ *   SALA_ERR_BOUNDS by sala_check_status and skipped.
+ * ---------------------------------------------------------------------------------------- */
+sala_status sala_sparse_prefill_lse(const void* q, const void* k, const void* v,
+                                    const int32_t* idx, void* o, float* lse, int B, int H, int Hkv,
+                                    int N, int d, int block, int slots, float scale, sala_dtype dt,
+                                    sala_stream stream);
+size_t sala_sparse_backward_workspace(int B, int H, int Hkv, int N, int d, int slots);
+sala_status sala_sparse_backward(const void* q, const void* k, const void* v, const int32_t* idx,
+                                 const float* lse, const void* dout, void* dq,
+                                 void* dk, void* dv, int B, int H, int Hkv, int N, int d, int block,
+                                 int slots, float scale, void* workspace, size_t workspace_bytes,
+                                 sala_dtype dt, sala_stream stream);
+
+/* ------------------------------------------------------------------------------------------
  * Sparse attention decode: one query token per (batch, head) at absolute position pos, over
  * a dense KV cache that holds rows 0 .. pos (capacity Tmax rows).
  *

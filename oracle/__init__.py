@@ -362,3 +362,26 @@ def sparse_attention_backward(q, k, v, idx, do, block, scale=None):
                 dk[b, g] += gk.numpy()
                 dv[b, g] += gv.numpy()
     return dq, dk, dv
+
+
+def sparse_dq_rows(q, k, v, idx, do, block, rows, scale=None):
+    """dq of selected prefill rows only, rows: [n, 3] of (b, h, i): for each, fp64 autograd of
+    o_i . do_i through the softmax over row i's visible keys (its selected blocks, keys <= i).
+    Equals the rows of sparse_attention_backward's dq; cheap at any N."""
+    import torch
+    B, H, N, d = q.shape
+    Hkv = k.shape[1]
+    G = H // Hkv
+    scale = (1.0 / np.sqrt(d)) if scale is None else float(scale)
+    out = np.empty((len(rows), d))
+    for n, (b, h, i) in enumerate(np.asarray(rows, dtype=np.int64)):
+        g = h // G
+        blks = [int(x) for x in np.asarray(idx[b, g, i]) if x >= 0]
+        keys = np.concatenate([np.arange(x * block, min((x + 1) * block, i + 1)) for x in blks])
+        Q = torch.tensor(_f64(q[b, h, i]), requires_grad=True)
+        K = torch.from_numpy(_f64(k[b, g, keys]))
+        V = torch.from_numpy(_f64(v[b, g, keys]))
+        o = torch.softmax(scale * (K @ Q), dim=0) @ V
+        (gq,) = torch.autograd.grad((o * torch.from_numpy(_f64(do[b, h, i]))).sum(), (Q,))
+        out[n] = gq.numpy()
+    return out

@@ -95,3 +95,12 @@ def test_lse_reproduces_forward():
             p = np.where(vis, np.exp(scale * q[b, h] @ k[b, g].T - lse[b, h][:, None]), 0.0)
             np.testing.assert_allclose(p @ v[b, g], o_ref[b, h], rtol=1e-12, atol=1e-12)
             assert lse[b, h, 0] == pytest.approx(scale * q[b, h, 0] @ k[b, g, 0], rel=1e-14)
+
+
+def test_sampled_dq_rows_equal_full_backward():
+    B, H, Hkv, N, d, block = 2, 4, 2, 80, 8, 16
+    q, k, v, do, idx = _case(B, H, Hkv, N, d, block, 2, 51)
+    dq = oracle.sparse_attention_backward(q, k, v, idx, do, block)[0]
+    rows = np.array([[0, 0, 0], [1, 3, 79], [0, 2, 40], [1, 1, 17], [0, 3, 63], [1, 0, 64]])
+    got = oracle.sparse_dq_rows(q, k, v, idx, do, block, rows)
+    np.testing.assert_allclose(got, dq[rows[:, 0], rows[:, 1], rows[:, 2]], rtol=1e-12, atol=1e-13)
