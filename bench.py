@@ -425,6 +425,50 @@ def run_linear_backward(sala, synth, torch, steps, warmup, stream, n_tok=N_TOK):
     return {"ms": ms, "bytes": 7.0 * H * n_tok * D * 2}  # read q, k, v, dout; write dq, dk, dv
 
 
+def run_sparse_backward(sala, synth, torch, steps, warmup, stream, n_tok=N_TOK):
+    """Training step of one sparse layer at N tokens (32 query / 2 KV heads, top-64 + 1 init +
+    2 local): the forward with its row log-sum-exp, then the backward (dq, dk, dv), each timed
+    with CUDA events over `steps` back-to-back calls.  Executed FLOPs are counted from the
+    selection: the query-side pass runs 6 MMAs of 2.10 MFLOP per (8-token tile, union block), the
+    key-side pass 4 per 8-token tile of each block's token list."""
+    dev = torch.device("cuda")
+    sl = synth.sparse_layer(1, H, HKV, n_tok, D, torch.bfloat16, dev, layer=3)
+    dout = synth.normal((1, H, n_tok, D), synth.seed(3, 7), dev, torch.bfloat16)
+    kbar = sala.block_compress(sl.k, stream=stream)
+    idx = sala.block_topk(sl.q, kbar, TOPK, N_INIT, N_LOCAL, stream=stream)
+    o, lse = sala.sparse_prefill(sl.q, sl.k, sl.v, idx, lse=True, stream=stream)
+    ws = torch.empty(sala.sparse_backward_workspace_bytes(1, H, HKV, n_tok, D, idx.shape[3]),
+                     dtype=torch.uint8, device=dev)
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            sala.sparse_prefill(sl.q, sl.k, sl.v, idx, o=o, lse=lse, stream=stream)
+            sala.sparse_backward(sl.q, sl.k, sl.v, idx, lse, dout, workspace=ws, stream=stream)
+        torch.cuda.synchronize()
+        a, b, c = ev(), ev(), ev()
+        a.record(stream)
+        for _ in range(steps):
+            sala.sparse_prefill(sl.q, sl.k, sl.v, idx, o=o, lse=lse, stream=stream)
+        b.record(stream)
+        for _ in range(steps):
+            sala.sparse_backward(sl.q, sl.k, sl.v, idx, lse, dout, workspace=ws, stream=stream)
+        c.record(stream)
+        torch.cuda.synchronize()
+    sala.check_status(stream)
+    mma = 2.0 * 128 * 64 * 128
+    union = tile_union_blocks(torch, idx)
+    nb = (n_tok + BLOCK - 1) // BLOCK
+    keys = (idx + torch.arange(HKV, device=dev, dtype=torch.int32).view(1, HKV, 1, 1) * nb)[idx >= 0]
+    cnt = torch.bincount(keys.long(), minlength=HKV * nb)
+    kv_tiles = int(((cnt + 7) // 8).sum().item())
+    out = {"fwd_ms": a.elapsed_time(b) / steps, "bwd_ms": b.elapsed_time(c) / steps,
+           "alg_flops": 10.0 * D * H * attended_keys(n_tok),
+           "exec_flops_dq": 6 * mma * union, "exec_flops_dkv": 4 * mma * kv_tiles}
+    del sl, dout, kbar, idx, o, lse, ws
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_qk_norm(sala, synth, torch, steps, warmup, stream, n_tok=N_TOK):
     """QK normalisation of one linear layer's q and k (32 heads each, d 128) at N tokens, in
     place, one launch per call."""
@@ -719,10 +763,16 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=0.0,
                     help="seconds of oracle work per CPU-baseline sample (0: the default sizing)")
     ap.add_argument("--phases", default="prefill,decode,e2e,cpu",
-                    help="comma list of prefill,decode,e2e,cpu,paged,backward (default: the first four)")
+                    help="comma list of prefill,decode,e2e,cpu,paged,backward,qknorm,sparse_bwd "
+                         "(default: the first four)")
     ap.add_argument("--decode-steps", type=int, default=200)
     ap.add_argument("--decode-t", type=int, default=DECODE_T,
                     help="decode context length (default 2^20, the benchmark; smaller only for profiles)")
+    ap.add_argument("--wait-limit-s", type=float, default=0.0,
+                    help="bound of the kernels' device-side waits in seconds (0: the library's 2 s; "
+                         "a profiler replaying kernels pass by pass needs more)")
+    ap.add_argument("--bwd-n", type=int, default=N_TOK,
+                    help="sequence length of the sparse_bwd phase (a smaller one for profiling)")
     ap.add_argument("--workload", default="hybrid_prefill_n256k", choices=sorted(WORKLOADS),
                     help="prefill workload (default: the 32-layer hybrid stack at 256K)")
     args = ap.parse_args()
@@ -770,6 +820,8 @@ def main():
     torch.cuda.set_device(local)
     init_dist("nccl")
     from hybrid_sparse_linear_b200 import sala, synth
+    if args.wait_limit_s > 0:
+        sala.set_wait_limit_ns(int(args.wait_limit_s * 1e9))
     stream = torch.cuda.Stream()
     peaks = measured_peaks()
     line = {"metric": METRIC, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
@@ -831,6 +883,20 @@ def main():
                                    "achieved_gbs": gbs, "hbm_frac": gbs / peaks["hbm_gbs"],
                                    "composition": "three forward linear attentions (two of the "
                                                   "reversed sequence) and six row reversals"}
+    if "sparse_bwd" in phases:
+        sb = run_sparse_backward(sala, synth, torch, max(args.steps, 3), max(3, args.warmup), stream,
+                                 args.bwd_n)
+        ex = sb["exec_flops_dq"] + sb["exec_flops_dkv"]
+        line["sparse_backward"] = {
+            "metric": f"sparse-attention training step ms per layer @{args.bwd_n} (forward with "
+                      "lse, then dq, dk, dv)",
+            "forward_ms": sb["fwd_ms"], "backward_ms": sb["bwd_ms"],
+            "algorithmic_tflops": sb["alg_flops"] / (sb["bwd_ms"] * 1e-3) / 1e12,
+            "executed_tflops": ex / (sb["bwd_ms"] * 1e-3) / 1e12,
+            "executed_tflop": {"dq_pass": sb["exec_flops_dq"] / 1e12, "dkv_pass": sb["exec_flops_dkv"] / 1e12},
+            "algorithmic_tflop": sb["alg_flops"] / 1e12,
+            "peak_tflops": peaks["bf16_tflops_sustained"],
+            "timing": "CUDA events around back-to-back calls on resident inputs"}
     if "qknorm" in phases:
         qn = run_qk_norm(sala, synth, torch, max(args.steps, 5), max(3, args.warmup), stream)
         gbs = qn["bytes"] / (qn["ms"] * 1e-3) / 1e9

@@ -561,6 +561,25 @@ struct Walk {
     }
 };
 
+// A tile cursor over the same walk: tile = up to kTok consecutive list positions of one segment.
+struct Cursor {
+    Walk w;
+    int64_t pos;
+    bool ok;
+    __device__ void start(const int* off, int n_keys, int64_t t0, int64_t t1) {
+        ok = w.start(off, n_keys, t0, t1);
+        pos = w.p0;
+    }
+    __device__ int n() const { return (int)min((int64_t)kTok, w.p1 - pos); }
+    __device__ void advance() {
+        pos += kTok;
+        if (pos >= w.p1) {
+            ok = ok && w.next();
+            pos = w.p0;
+        }
+    }
+};
+
 }  // namespace dkvp
 
 __global__ void __launch_bounds__(dkvp::kThreads, 1)
@@ -618,6 +637,7 @@ sparse_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         // last token; those rows are masked), 16 heads x 128 B per box.
         uint32_t seg = 0, t = 0, kv_iss = 0;  // segments walked, tiles and K|V pairs issued
         bool stop = false;
+        int tok_next = 0;
         for (bool more = wk.start(off, n_keys, t0, t1); more && !stop; more = wk.next(), ++seg) {
             const int64_t bg = wk.key / nb;
             const int j = wk.key % nb;
@@ -639,7 +659,11 @@ sparse_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             stop = __shfl_sync(0xffffffffu, stop ? 1 : 0, 0) != 0;
             for (int64_t pos = wk.p0; pos < wk.p1 && !stop; pos += kTok, ++t) {
                 const int n = (int)min((int64_t)kTok, wk.p1 - pos);
-                const int tok = lane < kTok ? __ldg(list + pos + min(lane, n - 1)) : 0;
+                // this tile's tokens came one tile ahead (positions pos .. pos + 7, clamped to the
+                // share); a short tile repeats its last token
+                const int raw = t == 0 ? (lane < kTok ? __ldg(list + min(pos + lane, t1 - 1)) : 0) : tok_next;
+                const int tok = __shfl_sync(0xffffffffu, raw, min(lane, n - 1));
+                tok_next = lane < kTok ? __ldg(list + min(pos + n + lane, t1 - 1)) : 0;
                 if (lane == 0) {
                     if (t >= 2 && !wait_or_abort(&bars.ring_empty[t & 1], ((t - 2) >> 1) & 1, ctx, abort))
                         stop = true;
@@ -755,21 +779,44 @@ sparse_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         // Thread = tile row r = TMEM lane r: token slot r / 16, head r % 16.  P and dS go to
         // shared memory as 128-byte rows with the 128-byte swizzle (16-byte chunk c of row r at
         // chunk c ^ (r & 7)), the layout the dK | dV issuer's descriptors read.
+        // The row's token, lse and D are global loads, the latter two dependent on the first:
+        // tokens are fetched two tiles ahead and lse, D one tile ahead of their use.
         const int r = tid, slot = r >> 4, hh = r & 15;
         const uint32_t lane_base = tmem_lane_base(warp);
-        uint32_t seg = 0, t = 0;
+        auto row_of = [&](const Cursor& c) {
+            const int64_t bg = c.w.key / nb;
+            return ((bg / Hkv) * H + (bg % Hkv) * kG + hh) * (int64_t)N;
+        };
+        auto tok_at = [&](const Cursor& c) {
+            return (c.ok && slot < c.n()) ? __ldg(list + c.pos + slot) : -1;
+        };
+        Cursor cur, c1, c2;
+        cur.start(off, n_keys, t0, t1);
+        c1 = cur;
+        c1.advance();
+        c2 = c1;
+        c2.advance();
+        int tok0 = tok_at(cur), tok1 = tok_at(c1);
+        float nl0 = 0.f, dv0 = 0.f;
+        if (tok0 >= 0) {
+            nl0 = -__ldg(lse + row_of(cur) + tok0) * kLog2e;
+            dv0 = __ldg(delta + row_of(cur) + tok0);
+        }
+        uint32_t t = 0;
         bool ok = true;
-        for (bool more = wk.start(off, n_keys, t0, t1); more && ok; more = wk.next(), ++seg) {
-            const int64_t bg = wk.key / nb;
-            const int j = wk.key % nb;
-            const int64_t row0 = ((bg / Hkv) * H + (bg % Hkv) * kG + hh) * (int64_t)N;
-            for (int64_t pos = wk.p0; pos < wk.p1; pos += kTok, ++t) {
+        for (; cur.ok && ok; ++t) {
+            float nl1 = 0.f, dv1 = 0.f;
+            if (tok1 >= 0) {
+                const int64_t r1 = row_of(c1) + tok1;
+                nl1 = -__ldg(lse + r1) * kLog2e;
+                dv1 = __ldg(delta + r1);
+            }
+            const int tok2 = tok_at(c2);
+            {
+                const int j = cur.w.key % nb;
                 const uint32_t u = t & 1;
-                const bool valid = slot < wk.p1 - pos;
-                const int i = valid ? __ldg(list + pos + slot) : 0;
-                const float nl = valid ? -__ldg(lse + row0 + i) * kLog2e : 0.f;
-                const float dv = valid ? __ldg(delta + row0 + i) : 0.f;
-                const int lim = valid ? min(kBlk - 1, i - j * kBlk) : -1;
+                const float nl = nl0, dv = dv0;
+                const int lim = tok0 >= 0 ? min(kBlk - 1, tok0 - j * kBlk) : -1;
                 if (!(ok = wait_or_abort(&bars.s_full[u], (t >> 1) & 1, ctx, abort))) break;
                 // the previous tile's dK | dV MMAs are done with the P and dS rows
                 if (t >= 1 && !(ok = wait_or_abort(&bars.pds_free, (t - 1) & 1, ctx, abort))) break;
@@ -805,6 +852,13 @@ sparse_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars.p_full);
             }
+            cur = c1;
+            c1 = c2;
+            c2.advance();
+            tok0 = tok1;
+            tok1 = tok2;
+            nl0 = nl1;
+            dv0 = dv1;
         }
     } else if (warp < 8) {
         // ---------------------------------------------------------------- epilogue
