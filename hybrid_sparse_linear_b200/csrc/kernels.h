@@ -71,12 +71,16 @@ cudaError_t launch_sparse_prefill_tc(const void* q, const void* k, const void* v
                                      DevCtx ctx);
 
 // Sparse attention backward (bf16, G = 16, d = 128), selection held fixed.
-// The transposed selection: for key k = (b * Hkv + g) * nb + j, list[off[k] .. off[k+1]) holds
-// the query tokens whose selection row holds block j; off[n_keys] is the total.
+// The transposed selection: for key k = ((b * Hkv + g) * n_chunks + chunk) * nb + j,
+// list[off[k] .. off[k+1]) holds the query tokens of the chunk (kChunkTok tokens) whose selection
+// row holds block j; off[n_keys] is the total.  item_key[it] is the list holding position
+// it * kItem (the key side's unit of work).
+constexpr int kChunkTok = 8192;
+constexpr int kItem = 512;
 struct SparseBwdCsr {
-    int nb, n_keys;
-    int *cnt, *cur, *off, *list;
-    size_t bytes;  // workspace bytes the four arrays take
+    int nb, n_chunks, n_keys, n_items;
+    int *cnt, *cur, *off, *list, *item_key, *bsum;
+    size_t bytes;  // workspace bytes the arrays take
 };
 SparseBwdCsr sparse_bwd_csr_layout(void* ws, int B, int Hkv, int N, int slots);
 cudaError_t launch_sparse_bwd_csr(const int32_t* idx, int B, int Hkv, int N, int slots,

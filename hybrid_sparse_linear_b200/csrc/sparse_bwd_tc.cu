@@ -23,7 +23,7 @@
 //
 // dk / dv pass (key side): one persistent CTA per SM takes an equal share of the transposed
 // selection (all (batch, group, key block) token lists laid end to end).  A segment is the part
-// of one block's list inside the share; its K and V sit in one of two shared buffers, and its
+// of one block's list inside the share; its K and V sit in a shared buffer, and its
 // tokens go in tiles of 8 (16 heads each: row = slot * 16 + head), their Q and dO rows gathered
 // by TMA, 16 rows per token.  Per tile:
 //   S = Q K_b^T, dP = dO V_b^T                       (M=128 N=64 K=128, K-major operands)
@@ -507,57 +507,64 @@ namespace dkvp {
 constexpr int kThreads = 352;  // warps 0-3 dS, 4-7 epilogue, 8 producer, 9 S|dP issuer, 10 dK|dV
 constexpr int kTok = 8;        // tokens per tile (x 16 heads = 128 rows)
 constexpr int kRingBytes = 2 * kTileBytes;          // Q tile then dO tile
-constexpr int kOffRing = 2 * kKVBytes;              // after the two K|V buffers
-constexpr int kOffP = kOffRing + 2 * kRingBytes;    // P [128 rows x 128 B], then dS
+constexpr int kOffRing = kKVBytes;                  // after the K|V buffer
+constexpr int kOffP = kOffRing + 2 * kRingBytes;    // two buffers of P [128 rows x 128 B] + dS
 constexpr int kPBytes = 16384;
-constexpr int kSmemBytes = kOffP + 2 * kPBytes + 1024;
+constexpr int kSmemBytes = kOffP + 4 * kPBytes + 1024;
 static_assert(kSmemBytes <= 232448 - 512, "shared memory");
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColAcc = 256;  // dK^T at kColAcc + 128 w, dV^T at +64; S_u at 128 u, dP_u +64
 
 struct Bars {
-    uint64_t kv_full[2], kv_empty[2];
+    uint64_t kv_full, kv_empty;
     uint64_t ring_full[2], ring_empty[2];
     uint64_t s_full[2], s_free[2];
-    uint64_t p_full, pds_free;
+    uint64_t p_full[2], pds_free[2];
     uint64_t acc_full[2], acc_empty[2];
     uint64_t fin[2];
     uint32_t tmem_base;
     int abort;
 };
 
-// The CTA's share [t0, t1) of the concatenated token lists, segment by segment: key = the list
-// (b * Hkv + g) * nb + j, [p0, p1) its part inside the share.  Every role walks it alike.
-struct Walk {
+// The CTA's work: items of kItem consecutive positions of the concatenated token lists, taken
+// in turn (item blockIdx.x, + gridDim.x, ...) so that all CTAs move through the lists together,
+// one chunk of query tokens at a time; within an item, segment by segment: key = the list
+// ((b * Hkv + g) * n_chunks + chunk) * nb + j, [p0, p1) its part inside the item.  Every role
+// walks it alike.
+struct WalkCtx {
     const int* off;
-    int n_keys;
-    int64_t t1;
+    const int* item_key;
+    int64_t T;
+    int stride;
+};
+struct Walk {
+    int item;
     int key;
-    int64_t p0, p1;
-    __device__ bool start(const int* off_, int n_keys_, int64_t t0, int64_t t1_) {
-        off = off_;
-        n_keys = n_keys_;
-        t1 = t1_;
-        if (t0 >= t1) return false;
-        int lo = 0, hi = n_keys - 1;  // the last list starting at or before t0 (a non-empty one)
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (__ldg(off + mid) <= t0) lo = mid;
-            else hi = mid - 1;
-        }
-        key = lo;
+    int64_t t1, p0, p1;
+    __device__ bool enter(const WalkCtx& c) {
+        const int64_t t0 = (int64_t)item * kItem;
+        if (t0 >= c.T) return false;
+        t1 = min(c.T, t0 + kItem);
+        key = __ldg(c.item_key + item);
         p0 = t0;
-        p1 = min((int64_t)__ldg(off + key + 1), t1);
+        p1 = min((int64_t)__ldg(c.off + key + 1), t1);
         return true;
     }
-    __device__ bool next() {
-        if (p1 >= t1) return false;
-        p0 = p1;
-        do {
-            ++key;
-        } while (__ldg(off + key + 1) <= p0);
-        p1 = min((int64_t)__ldg(off + key + 1), t1);
-        return true;
+    __device__ bool start(const WalkCtx& c, int first) {
+        item = first;
+        return enter(c);
+    }
+    __device__ bool next(const WalkCtx& c) {
+        if (p1 < t1) {
+            p0 = p1;
+            do {
+                ++key;
+            } while (__ldg(c.off + key + 1) <= p0);
+            p1 = min((int64_t)__ldg(c.off + key + 1), t1);
+            return true;
+        }
+        item += c.stride;
+        return enter(c);
     }
 };
 
@@ -566,15 +573,15 @@ struct Cursor {
     Walk w;
     int64_t pos;
     bool ok;
-    __device__ void start(const int* off, int n_keys, int64_t t0, int64_t t1) {
-        ok = w.start(off, n_keys, t0, t1);
+    __device__ void start(const WalkCtx& c, int first) {
+        ok = w.start(c, first);
         pos = w.p0;
     }
     __device__ int n() const { return (int)min((int64_t)kTok, w.p1 - pos); }
-    __device__ void advance() {
+    __device__ void advance(const WalkCtx& c) {
         pos += kTok;
         if (pos >= w.p1) {
-            ok = ok && w.next();
+            ok = ok && w.next(c);
             pos = w.p0;
         }
     }
@@ -585,10 +592,11 @@ struct Cursor {
 __global__ void __launch_bounds__(dkvp::kThreads, 1)
 sparse_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
                      const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                     const int* __restrict__ off, const int* __restrict__ list,
+                     const int* __restrict__ off, const int* __restrict__ item_key,
+                     const int* __restrict__ list,
                      const float* __restrict__ lse, const float* __restrict__ delta,
                      float* __restrict__ dk_acc, float* __restrict__ dv_acc, int H, int Hkv, int N,
-                     int nb, int n_keys, float sl2, DevCtx ctx) {
+                     int nb, int n_chunks, int n_keys, float sl2, DevCtx ctx) {
     using namespace dkvp;
     extern __shared__ uint8_t smraw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smraw) + 1023) &
@@ -602,9 +610,11 @@ sparse_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         tmem_relinquish();
     }
     if (tid == 0) {
+        mbar_init(&bars.kv_full, 1);
+        mbar_init(&bars.kv_empty, 1);
         for (int b = 0; b < 2; ++b) {
-            mbar_init(&bars.kv_full[b], 1);
-            mbar_init(&bars.kv_empty[b], 1);
+            mbar_init(&bars.p_full[b], 4);
+            mbar_init(&bars.pds_free[b], 1);
             mbar_init(&bars.ring_full[b], 1);
             mbar_init(&bars.ring_empty[b], 2);  // both issuers read a tile
             mbar_init(&bars.s_full[b], 1);
@@ -613,8 +623,6 @@ sparse_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             mbar_init(&bars.acc_empty[b], 4);
             mbar_init(&bars.fin[b], 1);
         }
-        mbar_init(&bars.p_full, 4);
-        mbar_init(&bars.pds_free, 1);
         bars.abort = 0;
         fence_mbar_init();
     }
@@ -622,12 +630,11 @@ sparse_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = bars.tmem_base;
-    const int64_t T = __ldg(off + n_keys);
-    const int64_t t0 = T * blockIdx.x / gridDim.x, t1 = T * (blockIdx.x + 1) / gridDim.x;
+    const WalkCtx wc{off, item_key, (int64_t)__ldg(off + n_keys), (int)gridDim.x};
     auto ring = [&](uint32_t t) { return sm + kOffRing + (t & 1) * kRingBytes; };
-    auto kvbuf = [&](uint32_t s) { return sm + (s & 1) * kKVBytes; };
-    uint8_t* sP = sm + kOffP;
-    uint8_t* sDS = sm + kOffP + kPBytes;
+    auto kvbuf = [&](uint32_t) { return sm; };
+    auto sP = [&](uint32_t t) { return sm + kOffP + (t & 1) * 2 * kPBytes; };
+    auto sDS = [&](uint32_t t) { return sm + kOffP + (t & 1) * 2 * kPBytes + kPBytes; };
     Walk wk;
 
     if (warp == 8) {
@@ -638,16 +645,17 @@ sparse_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         uint32_t seg = 0, t = 0, kv_iss = 0;  // segments walked, tiles and K|V pairs issued
         bool stop = false;
         int tok_next = 0;
-        for (bool more = wk.start(off, n_keys, t0, t1); more && !stop; more = wk.next(), ++seg) {
-            const int64_t bg = wk.key / nb;
+        bool have_next = false;
+        for (bool more = wk.start(wc, blockIdx.x); more && !stop; more = wk.next(wc), ++seg) {
+            const int64_t bg = wk.key / (nb * n_chunks);
             const int j = wk.key % nb;
             const int z = (int)((bg / Hkv) * H + (bg % Hkv) * kG);
             if (lane == 0) {
-                if (seg >= 2 && !wait_or_abort(&bars.kv_empty[seg & 1], ((seg - 2) >> 1) & 1, ctx, abort))
+                if (seg >= 1 && !wait_or_abort(&bars.kv_empty, (seg - 1) & 1, ctx, abort))
                     stop = true;
                 if (!stop) {
                     uint8_t* kv = kvbuf(seg);
-                    uint64_t* fb = &bars.kv_full[seg & 1];
+                    uint64_t* fb = &bars.kv_full;
                     mbar_arrive_expect_tx(fb, kKVBytes);
                     tma_load_3d(kv, &tmK, fb, 0, j * kBlk, (int)bg);
                     tma_load_3d(kv + kHalfBlk, &tmK, fb, 64, j * kBlk, (int)bg);
@@ -659,11 +667,13 @@ sparse_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             stop = __shfl_sync(0xffffffffu, stop ? 1 : 0, 0) != 0;
             for (int64_t pos = wk.p0; pos < wk.p1 && !stop; pos += kTok, ++t) {
                 const int n = (int)min((int64_t)kTok, wk.p1 - pos);
-                // this tile's tokens came one tile ahead (positions pos .. pos + 7, clamped to the
-                // share); a short tile repeats its last token
-                const int raw = t == 0 ? (lane < kTok ? __ldg(list + min(pos + lane, t1 - 1)) : 0) : tok_next;
+                // this tile's tokens came one tile ahead when it is not an item's first (positions
+                // pos .. pos + 7, clamped to the item); a short tile repeats its last token
+                const int raw = !have_next ? (lane < kTok ? __ldg(list + min(pos + lane, wk.t1 - 1)) : 0)
+                                           : tok_next;
                 const int tok = __shfl_sync(0xffffffffu, raw, min(lane, n - 1));
-                tok_next = lane < kTok ? __ldg(list + min(pos + n + lane, t1 - 1)) : 0;
+                have_next = pos + n < wk.t1;
+                tok_next = (lane < kTok && have_next) ? __ldg(list + min(pos + n + lane, wk.t1 - 1)) : 0;
                 if (lane == 0) {
                     if (t >= 2 && !wait_or_abort(&bars.ring_empty[t & 1], ((t - 2) >> 1) & 1, ctx, abort))
                         stop = true;
@@ -684,8 +694,7 @@ sparse_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             if (*abort) stop = true;
         }
         if (lane == 0) {  // every copy this warp started has landed before the block exits
-            for (uint32_t e = kv_iss > 2 ? kv_iss - 2 : 0; e < kv_iss; ++e)
-                (void)mbar_wait(&bars.kv_full[e & 1], (e >> 1) & 1, ctx);
+            if (kv_iss > 0) (void)mbar_wait(&bars.kv_full, (kv_iss - 1) & 1, ctx);
             for (uint32_t e = t > 2 ? t - 2 : 0; e < t; ++e)
                 (void)mbar_wait(&bars.ring_full[e & 1], (e >> 1) & 1, ctx);
         }
@@ -696,8 +705,8 @@ sparse_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             const uint32_t dhi = sdesc_sw128_hi(1024);
             uint32_t seg = 0, t = 0;
             bool ok = true;
-            for (bool more = wk.start(off, n_keys, t0, t1); more && ok; more = wk.next(), ++seg) {
-                if (!(ok = wait_or_abort(&bars.kv_full[seg & 1], (seg >> 1) & 1, ctx, abort))) break;
+            for (bool more = wk.start(wc, blockIdx.x); more && ok; more = wk.next(wc), ++seg) {
+                if (!(ok = wait_or_abort(&bars.kv_full, seg & 1, ctx, abort))) break;
                 const uint32_t k_lo = sdesc_sw128_lo(smem_u32(kvbuf(seg)), 16);
                 const uint32_t v_lo = sdesc_sw128_lo(smem_u32(kvbuf(seg) + 2 * kHalfBlk), 16);
                 for (int64_t pos = wk.p0; pos < wk.p1; pos += kTok, ++t) {
@@ -722,7 +731,7 @@ sparse_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                     }
                     mma_commit(&bars.s_full[u]);
                     mma_commit(&bars.ring_empty[u]);
-                    if (pos + kTok >= wk.p1) mma_commit(&bars.kv_empty[seg & 1]);
+                    if (pos + kTok >= wk.p1) mma_commit(&bars.kv_empty);
                 }
             }
             mma_commit(&bars.fin[0]);
@@ -737,24 +746,25 @@ sparse_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         if (lane == 0) {
             const uint32_t idD = idesc_bf16_f32(128, kBlk, true, true);
             const uint32_t dhi = sdesc_sw128_hi(1024);
-            const uint32_t p_lo = sdesc_sw128_lo(smem_u32(sP), kHalfQ);
-            const uint32_t ds_lo = sdesc_sw128_lo(smem_u32(sDS), kHalfQ);
+
             uint32_t seg = 0, t = 0;
             bool ok = true;
-            for (bool more = wk.start(off, n_keys, t0, t1); more && ok; more = wk.next(), ++seg) {
+            for (bool more = wk.start(wc, blockIdx.x); more && ok; more = wk.next(wc), ++seg) {
                 const uint32_t w = seg & 1;
                 const uint32_t tK = tmem + kColAcc + w * 128, tV = tK + 64;
                 for (int64_t pos = wk.p0; pos < wk.p1; pos += kTok, ++t) {
                     const uint32_t u = t & 1;
                     const bool first = pos == wk.p0;
                     if (!(ok = wait_or_abort(&bars.ring_full[u], (t >> 1) & 1, ctx, abort))) break;
-                    if (!(ok = wait_or_abort(&bars.p_full, t & 1, ctx, abort))) break;
+                    if (!(ok = wait_or_abort(&bars.p_full[u], (t >> 1) & 1, ctx, abort))) break;
                     if (first && seg >= 2 &&
                         !(ok = wait_or_abort(&bars.acc_empty[w], ((seg - 2) >> 1) & 1, ctx, abort)))
                         break;
                     tc_fence_after();
                     const uint32_t q_lo = sdesc_sw128_lo(smem_u32(ring(t)), kHalfQ);
                     const uint32_t do_lo = sdesc_sw128_lo(smem_u32(ring(t) + kTileBytes), kHalfQ);
+                    const uint32_t p_lo = sdesc_sw128_lo(smem_u32(sP(t)), kHalfQ);
+                    const uint32_t ds_lo = sdesc_sw128_lo(smem_u32(sDS(t)), kHalfQ);
 #pragma unroll
                     for (int ks = 0; ks < 128 / 16; ++ks) {
                         const uint32_t o = (ks * 16 * 128) >> 4;
@@ -765,7 +775,7 @@ sparse_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                         const uint32_t o = (ks * 16 * 128) >> 4;
                         mma_ss_lohi(tK, q_lo + o, ds_lo + o, dhi, idD, (first && ks == 0) ? 0u : 1u);
                     }
-                    mma_commit(&bars.pds_free);
+                    mma_commit(&bars.pds_free[u]);
                     mma_commit(&bars.ring_empty[u]);
                     if (pos + kTok >= wk.p1) mma_commit(&bars.acc_full[w]);
                 }
@@ -784,18 +794,23 @@ sparse_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         const int r = tid, slot = r >> 4, hh = r & 15;
         const uint32_t lane_base = tmem_lane_base(warp);
         auto row_of = [&](const Cursor& c) {
-            const int64_t bg = c.w.key / nb;
+            const int64_t bg = c.w.key / (nb * n_chunks);
             return ((bg / Hkv) * H + (bg % Hkv) * kG + hh) * (int64_t)N;
         };
         auto tok_at = [&](const Cursor& c) {
             return (c.ok && slot < c.n()) ? __ldg(list + c.pos + slot) : -1;
         };
-        Cursor cur, c1, c2;
-        cur.start(off, n_keys, t0, t1);
+        // the tile after c1 starts at c1.pos + c1.n() when that is inside c1's item; its token
+        // is fetched from there and kept if that tile turns out to start there
+        auto pos_after = [&](const Cursor& c) { return c.ok ? c.pos + c.n() : (int64_t)-1; };
+        auto tok_ahead = [&](const Cursor& c) {
+            const int64_t p = pos_after(c);
+            return (p >= 0 && p + slot < c.w.t1) ? __ldg(list + p + slot) : -1;
+        };
+        Cursor cur, c1;
+        cur.start(wc, blockIdx.x);
         c1 = cur;
-        c1.advance();
-        c2 = c1;
-        c2.advance();
+        c1.advance(wc);
         int tok0 = tok_at(cur), tok1 = tok_at(c1);
         float nl0 = 0.f, dv0 = 0.f;
         if (tok0 >= 0) {
@@ -811,18 +826,19 @@ sparse_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                 nl1 = -__ldg(lse + r1) * kLog2e;
                 dv1 = __ldg(delta + r1);
             }
-            const int tok2 = tok_at(c2);
+            const int64_t p2 = pos_after(c1);
+            const int tok2 = tok_ahead(c1);
             {
                 const int j = cur.w.key % nb;
                 const uint32_t u = t & 1;
                 const float nl = nl0, dv = dv0;
                 const int lim = tok0 >= 0 ? min(kBlk - 1, tok0 - j * kBlk) : -1;
                 if (!(ok = wait_or_abort(&bars.s_full[u], (t >> 1) & 1, ctx, abort))) break;
-                // the previous tile's dK | dV MMAs are done with the P and dS rows
-                if (t >= 1 && !(ok = wait_or_abort(&bars.pds_free, (t - 1) & 1, ctx, abort))) break;
+                // the dK | dV MMAs of the tile two back are done with this P | dS buffer
+                if (t >= 2 && !(ok = wait_or_abort(&bars.pds_free[u], ((t - 2) >> 1) & 1, ctx, abort))) break;
                 tc_fence_after();
-                uint4* prow = reinterpret_cast<uint4*>(sP + r * 128);
-                uint4* srow = reinterpret_cast<uint4*>(sDS + r * 128);
+                uint4* prow = reinterpret_cast<uint4*>(sP(t) + r * 128);
+                uint4* srow = reinterpret_cast<uint4*>(sDS(t) + r * 128);
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     uint32_t sr[32], pr[32], pkP[16], pkS[16];
@@ -850,13 +866,12 @@ sparse_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                 if (lane == 0) mbar_arrive(&bars.s_free[u]);
                 fence_proxy_async_smem();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&bars.p_full);
+                if (lane == 0) mbar_arrive(&bars.p_full[u]);
             }
             cur = c1;
-            c1 = c2;
-            c2.advance();
+            c1.advance(wc);
             tok0 = tok1;
-            tok1 = tok2;
+            tok1 = (c1.ok && c1.pos == p2) ? (slot < c1.n() ? tok2 : -1) : tok_at(c1);
             nl0 = nl1;
             dv0 = dv1;
         }
@@ -868,8 +883,8 @@ sparse_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         const uint32_t lane_base = tmem_lane_base(warp);
         uint32_t seg = 0;
         bool ok = true;
-        for (bool more = wk.start(off, n_keys, t0, t1); more && ok; more = wk.next(), ++seg) {
-            const int64_t bg = wk.key / nb;
+        for (bool more = wk.start(wc, blockIdx.x); more && ok; more = wk.next(wc), ++seg) {
+            const int64_t bg = wk.key / (nb * n_chunks);
             const int j = wk.key % nb;
             const uint32_t w = seg & 1;
             if (!(ok = wait_or_abort(&bars.acc_full[w], (seg >> 1) & 1, ctx, abort))) break;
@@ -967,8 +982,8 @@ cudaError_t launch_sparse_dkv_tc(const void* q, const void* k, const void* v, co
     cudaError_t e = ensure_smem<sparse_dkv_tc_kernel>(dkvp::kSmemBytes);
     if (e != cudaSuccess) return e;
     sparse_dkv_tc_kernel<<<num_sms(), dkvp::kThreads, dkvp::kSmemBytes, st>>>(
-        tmQ, tmDO, tmK, tmV, c.off, c.list, lse, delta, dk_acc, dv_acc, H, Hkv, N, c.nb, c.n_keys,
-        scale * kLog2e, ctx);
+        tmQ, tmDO, tmK, tmV, c.off, c.item_key, c.list, lse, delta, dk_acc, dv_acc, H, Hkv, N, c.nb,
+        c.n_chunks, c.n_keys, scale * kLog2e, ctx);
     return cudaGetLastError();
 }
 
