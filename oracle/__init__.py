@@ -62,6 +62,8 @@ def _load():
             lib.orc_block_select.argtypes = [_D, _D, _I32, _D, _i, _i, _i, _i, _i, _i, _i, _i, _i,
                                              _i, _i, _i, _i]
             lib.orc_block_select_qblock.argtypes = [_D, _D, _I32, _D] + [_i] * 12
+            lib.orc_block_select_qblock_softmax.argtypes = [_D, _D, _I32, _D] + [_i] * 11 + [
+                ctypes.c_double, _i]
             lib.orc_sparse_attention.argtypes = [_D, _D, _D, _I32, _D, _i, _i, _i, _i, _i, _i, _i,
                                                  _i, _i, ctypes.c_double, _I64, _l, _i]
             lib.orc_dense_causal_attention.argtypes = [_D, _D, _D, _D, _i, _i, _i, _i, _i, _i, _i,
@@ -242,6 +244,25 @@ def block_select_qblock(q, kbar, block, topk, n_init, n_local, slots=None, threa
     _load().orc_block_select_qblock(_p(q), _p(kbar), idx.ctypes.data_as(_I32), _p(kth), B, H, Hkv,
                                     Nq, nb, d, block, topk, n_init, n_local, slots,
                                     threads or default_threads())
+    return idx, kth
+
+
+def block_select_qblock_softmax(q, kbar, block, topk, n_init, n_local, slots=None, scale=None,
+                                threads=None):
+    """Query-block selection scored by softmax-probability group aggregation: per head, the
+    block's mean query gives logits scale * (u_h . kbar_j) over the candidates, a softmax over
+    them, the probabilities summed over the group's heads.  Returns (idx, kth_score) as
+    block_select_qblock; scale defaults to 1/sqrt(d)."""
+    q, kbar = _f64(q), _f64(kbar)
+    B, H, Nq, d = q.shape
+    Hkv, nb = kbar.shape[1], kbar.shape[2]
+    slots = slots or (n_init + n_local + topk)
+    scale = (1.0 / np.sqrt(d)) if scale is None else float(scale)
+    idx = np.empty((B, Hkv, Nq, slots), dtype=np.int32)
+    kth = np.empty((B, Hkv, Nq))
+    _load().orc_block_select_qblock_softmax(_p(q), _p(kbar), idx.ctypes.data_as(_I32), _p(kth), B,
+                                            H, Hkv, Nq, nb, d, block, topk, n_init, n_local, slots,
+                                            scale, threads or default_threads())
     return idx, kth
 
 

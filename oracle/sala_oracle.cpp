@@ -464,4 +464,68 @@ void orc_qk_norm(double* x, int64_t rows, int d, double eps) {
     }
 }
 
+// Query-block selection with softmax-probability group aggregation (a variant the selection
+// step leaves open: InfLLM-V2's block scores are not fixed by the pages).  Reading: for each
+// (batch, KV group g, query block c of T tokens) and each head h of the group, the mean query
+// u_h over the block's tokens scores every candidate block j (n_init .. c - n_local) with the
+// logit scale * (u_h . kbar_j); the logits of a head go through a softmax over the candidates;
+// the block's score is the sum over the group's heads of those probabilities.  The best topk by
+// (score, lower block first) join the forced blocks; layout and kth_score as
+// orc_block_select_qblock.  Optionally the candidates' scores of one (b, g, c) are returned.
+void orc_block_select_qblock_softmax(const double* q, const double* kbar, int32_t* idx,
+                                     double* kth_score, int B, int H, int Hkv, int Nq, int nb,
+                                     int d, int T, int topk, int n_init, int n_local, int slots,
+                                     double scale, int nthreads) {
+    const int G = H / Hkv;
+    const int nqb = (Nq + T - 1) / T;
+    parallel_for((int64_t)B * Hkv * nqb, nthreads, [&](int64_t item) {
+        const int64_t b = item / ((int64_t)Hkv * nqb);
+        const int g = (int)((item / nqb) % Hkv);
+        const int c = (int)(item % nqb);
+        const int r0 = c * T, r1 = std::min(Nq, r0 + T);
+        std::vector<int> sel;
+        for (int blk = 0; blk < n_init && blk <= c; ++blk) sel.push_back(blk);
+        for (int blk = std::max(0, c - n_local + 1); blk <= c; ++blk)
+            if (blk >= n_init) sel.push_back(blk);
+        const int lo = n_init, hi = c - n_local;
+        const int nc = std::max(0, hi - lo + 1);
+        std::vector<double> score(nc, 0.0), logit(nc);
+        std::vector<double> u(d);
+        for (int h = g * G; h < (g + 1) * G; ++h) {
+            std::fill(u.begin(), u.end(), 0.0);
+            for (int r = r0; r < r1; ++r) {
+                const double* qr = q + (((int64_t)b * H + h) * Nq + r) * d;
+                for (int a = 0; a < d; ++a) u[a] += qr[a];
+            }
+            for (int a = 0; a < d; ++a) u[a] /= (double)(r1 - r0);
+            double mx = -std::numeric_limits<double>::infinity();
+            for (int e = 0; e < nc; ++e) {
+                logit[e] = scale * dot(u.data(), kbar + (((int64_t)b * Hkv + g) * nb + lo + e) * d, d);
+                mx = std::max(mx, logit[e]);
+            }
+            double den = 0.0;
+            for (int e = 0; e < nc; ++e) den += std::exp(logit[e] - mx);
+            for (int e = 0; e < nc; ++e) score[e] += std::exp(logit[e] - mx) / den;
+        }
+        std::vector<std::pair<double, int>> cand;
+        for (int e = 0; e < nc; ++e) cand.push_back({score[e], lo + e});
+        std::sort(cand.begin(), cand.end(), [](const auto& x, const auto& y) {
+            if (x.first != y.first) return x.first > y.first;
+            return x.second < y.second;
+        });
+        const int take = std::min<int>(topk, (int)cand.size());
+        for (int e = 0; e < take; ++e) sel.push_back(cand[e].second);
+        std::sort(sel.begin(), sel.end());
+        const double kth = ((int)cand.size() >= topk && topk > 0)
+                               ? cand[topk - 1].first
+                               : -std::numeric_limits<double>::infinity();
+        for (int r = r0; r < r1; ++r) {
+            const int64_t row = ((int64_t)b * Hkv + g) * Nq + r;
+            int32_t* out = idx + row * slots;
+            for (int e = 0; e < slots; ++e) out[e] = e < (int)sel.size() ? sel[e] : -1;
+            if (kth_score) kth_score[row] = kth;
+        }
+    });
+}
+
 }  // extern "C"
