@@ -238,6 +238,7 @@ WORKLOADS = {
     "linear_rope_prefill_n256k": (N_TOK, ["linear_rope"]),
     # a sparse layer whose 64-token query blocks each share one selection (the variant)
     "sparse_qblock_prefill_n256k": (N_TOK, ["sparse_qblock"]),
+    "sparse_qblock_softmax_prefill_n256k": (N_TOK, ["sparse_qsoft"]),
 }
 
 
@@ -248,7 +249,7 @@ def run_prefill(sala, synth, torch, steps, warmup, stream, workload="hybrid_pref
     lam = synth.decays(H).to(dev)
     layers = []
     for l, kind in enumerate(kinds):
-        if kind in ("sparse", "sparse_qblock"):
+        if kind in ("sparse", "sparse_qblock", "sparse_qsoft"):
             sl = synth.sparse_layer(1, H, HKV, n_tok, D, torch.bfloat16, dev, layer=l)
             layers.append((kind, sl.q, sl.k, sl.v))
         else:
@@ -286,8 +287,11 @@ def run_prefill(sala, synth, torch, steps, warmup, stream, workload="hybrid_pref
                 sala.block_compress(k, kbar, stream=stream)
                 if kind == "sparse":
                     sala.block_topk(q, kbar, TOPK, N_INIT, N_LOCAL, idx=idx, stream=stream)
-                else:
+                elif kind == "sparse_qblock":
                     sala.block_topk_qblock(q, kbar, TOPK, N_INIT, N_LOCAL, idx=idx, stream=stream)
+                else:
+                    sala.block_topk_qblock_softmax(q, kbar, TOPK, N_INIT, N_LOCAL, idx=idx,
+                                                   stream=stream)
                 if record: t1.record(stream); topk_ev.append((t0, t1))
                 e0, e1 = (ev(), ev()) if record else (None, None)
                 if record: e0.record(stream)
@@ -321,12 +325,15 @@ def run_prefill(sala, synth, torch, steps, warmup, stream, workload="hybrid_pref
     union, n_sp = 0, 0
     with torch.cuda.stream(stream):
         for kind, q, k, v in layers:
-            if kind in ("sparse", "sparse_qblock"):
+            if kind in ("sparse", "sparse_qblock", "sparse_qsoft"):
                 sala.block_compress(k, kbar, stream=stream)
                 if kind == "sparse":
                     sala.block_topk(q, kbar, TOPK, N_INIT, N_LOCAL, idx=idx, stream=stream)
-                else:
+                elif kind == "sparse_qblock":
                     sala.block_topk_qblock(q, kbar, TOPK, N_INIT, N_LOCAL, idx=idx, stream=stream)
+                else:
+                    sala.block_topk_qblock_softmax(q, kbar, TOPK, N_INIT, N_LOCAL, idx=idx,
+                                                   stream=stream)
                 union += tile_union_blocks(torch, idx)
                 n_sp += 1
     res["sparse_exec_flops"] = EXEC_FLOPS_PER_TILE_BLOCK * union / max(1, n_sp)
@@ -847,7 +854,7 @@ def main():
             line["config"]["workload"] = f"{args.workload}: {len(kinds)} x {kinds[0]} layer, N={n_tok}"
             line["config"]["seq_len"] = n_tok
         line["kernels"] = {}
-        if "sparse" in kinds or "sparse_qblock" in kinds:
+        if "sparse" in kinds or "sparse_qblock" in kinds or "sparse_qsoft" in kinds:
             fl = sparse_layer_flops(n_tok)
             achieved = fl / (pre["sparse_ms"] / 1000.0) / 1e12
             executed = pre["sparse_exec_flops"] / (pre["sparse_ms"] / 1000.0) / 1e12

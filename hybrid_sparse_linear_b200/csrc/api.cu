@@ -419,6 +419,27 @@ sala_status sala_block_topk(const void* q, const void* kbar, int32_t* idx, int B
                     "block_topk");
 }
 
+sala_status sala_block_topk_qblock_softmax(const void* q, const void* kbar, int32_t* idx, int B,
+                                           int H, int Hkv, int Nq, int nb, int d, int block,
+                                           int topk, int n_init, int n_local, float scale,
+                                           sala_dtype dt, sala_stream stream) {
+    sala_status s = check_select_args(B, H, Hkv, Nq, 0, nb, d, block, topk, n_init, n_local, dt);
+    if (s != SALA_OK) return s;
+    REQUIRE(Hkv > 0 && H / Hkv <= 16, SALA_ERR_UNSUPPORTED, "more than 16 query heads per KV head");
+    REQUIRE(isfinite(scale) && scale >= 0.f, SALA_ERR_INVALID_ARG, "scale must be finite and >= 0");
+    if (B == 0 || H == 0 || Nq == 0) return SALA_OK;
+    REQ_PTR(q); REQUIRE(idx != nullptr, SALA_ERR_INVALID_ARG, "idx must be a device pointer");
+    if (nb > 0) REQ_PTR(kbar);
+    if (scale == 0.f) scale = 1.0f / sqrtf((float)d);
+    sala::DevCtx ctx;
+    s = get_ctx(&ctx);
+    if (s != SALA_OK) return s;
+    return launched(sala::launch_block_topk_qblock_softmax(to_dt(dt), q, kbar, idx, B, H, Hkv, Nq,
+                                                           nb, d, topk, n_init, n_local, scale,
+                                                           static_cast<cudaStream_t>(stream), ctx),
+                    "block_topk_qblock_softmax");
+}
+
 sala_status sala_block_topk_qblock(const void* q, const void* kbar, int32_t* idx, int B, int H,
                                    int Hkv, int Nq, int nb, int d, int block, int topk, int n_init,
                                    int n_local, sala_dtype dt, sala_stream stream) {

@@ -44,6 +44,11 @@ cudaError_t launch_block_compress(DType dt, const void* k, void* kbar, int B, in
 cudaError_t launch_block_topk_qblock(DType dt, const void* q, const void* kbar, int32_t* idx, int B,
                                      int H, int Hkv, int Nq, int nb, int d, int topk, int n_init,
                                      int n_local, cudaStream_t st, DevCtx ctx);
+// The same granularity scored by softmax-probability group aggregation (G <= 16).
+cudaError_t launch_block_topk_qblock_softmax(DType dt, const void* q, const void* kbar, int32_t* idx,
+                                             int B, int H, int Hkv, int Nq, int nb, int d, int topk,
+                                             int n_init, int n_local, float scale, cudaStream_t st,
+                                             DevCtx ctx);
 cudaError_t launch_block_topk_tiled(DType dt, const void* q, const void* kbar, int32_t* idx,
                                     int B, int H, int Hkv, int Nq, int q_pos0, int nb, int d,
                                     int topk, int n_init, int n_local, cudaStream_t st,

@@ -195,6 +195,191 @@ topk_qblock_kernel(const T* __restrict__ q, const T* __restrict__ kbar, int32_t*
     }
 }
 
+// ---------------------------------------------------------------------------------------------
+// Softmax-probability group aggregation (same granularity and output): head h of the group scores
+// candidate j with the logit scale * (u_h . kbar_j), u_h the mean of the block's queries of head
+// h; each head's logits go through a softmax over the candidates, and a block's score is the sum
+// over the heads of its probabilities.
+//   1. u_h for the G <= 16 heads (fp32, scaled by scale * log2 e: logits in log2 units);
+//   2. pass 1: lane pair (h, half) holds u_h's half in registers and dots it with each
+//      candidate's k-bar half (every lane of a half reads the same row: one load per address),
+//      the pair combines, and keeps a running max and sum of 2^logit; the warps' partial
+//      (max, sum) pairs are merged per head;
+//   3. pass 2: the same dots, 2^(logit - M_h) / S_h summed over the heads, then the chunked exact
+//      top k of the plain query-block kernel.
+constexpr int kGmax = 16;
+
+template <int D>
+struct QsSmem {
+    float u[kGmax][D];
+    float m[kThreads / 32][kGmax], s[kThreads / 32][kGmax];
+    float M[kGmax], S[kGmax];
+    uint64_t keys[kChunk];
+    uint64_t carry[kCapK];
+    int win[kCapK];
+    int n_win;
+    RadixSelSmem rs;
+};
+
+// Dot of the lane's half of u_h (registers) with the same half of a k-bar row, both halves
+// summed (lane pairs 2h, 2h + 1).
+template <typename T, int D>
+__device__ __forceinline__ float pair_dot(const T* row, const float (&uh)[D / 2], int half) {
+    float acc = 0.f;
+    const T* p = row + half * (D / 2);
+#pragma unroll
+    for (int e = 0; e < D / 2; e += 4) {
+        float f[4];
+        load4<T>(p + e, f);
+        acc = fmaf(f[0], uh[e], acc);
+        acc = fmaf(f[1], uh[e + 1], acc);
+        acc = fmaf(f[2], uh[e + 2], acc);
+        acc = fmaf(f[3], uh[e + 3], acc);
+    }
+    return acc + __shfl_xor_sync(0xffffffffu, acc, 1);
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kThreads)
+topk_qblock_softmax_kernel(const T* __restrict__ q, const T* __restrict__ kbar,
+                           int32_t* __restrict__ idx, int H, int Hkv, int Nq, int nb, int topk,
+                           int n_init, int n_local, int slots, float sl2) {
+    extern __shared__ __align__(16) unsigned char smraw[];
+    QsSmem<D>& sm = *reinterpret_cast<QsSmem<D>*>(smraw);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    constexpr int kWarps = kThreads / 32;
+    const int nqb = (Nq + kQB - 1) / kQB;
+    const int64_t bg = blockIdx.x / nqb;
+    const int c = (int)(blockIdx.x % nqb);
+    const int64_t b = bg / Hkv;
+    const int g = (int)(bg % Hkv);
+    const int G = H / Hkv;
+    const int r0 = c * kQB, nr = min(Nq, r0 + kQB) - r0;
+    const int lo = n_init, hi = c - n_local;
+    const int ncand = hi - lo + 1;
+    int32_t* out = idx + (bg * Nq + r0) * (int64_t)slots;
+    if (ncand <= topk) {  // every candidate taken: blocks 0 .. c
+        for (int e = tid; e < nr * slots; e += kThreads) out[e] = (e % slots) <= c ? e % slots : -1;
+        return;
+    }
+    const int K = min(topk, kCapK);
+
+    // 1. scaled mean queries
+    for (int e = tid; e < kGmax * (D / 4); e += kThreads) {
+        const int h = e / (D / 4), c4 = e % (D / 4);
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        if (h < G) {
+            const T* qh = q + ((b * H + (int64_t)g * G + h) * Nq + r0) * D + 4 * c4;
+            for (int r = 0; r < nr; ++r) {
+                float f[4];
+                load4<T>(qh + (int64_t)r * D, f);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) acc[i] += f[i];
+            }
+        }
+        const float w = sl2 / (float)nr;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) sm.u[h][4 * c4 + i] = acc[i] * w;
+    }
+    if (tid < kCapK) sm.carry[tid] = 0ull;
+    __syncthreads();
+    const int h = lane >> 1, half = lane & 1;
+    const bool live = h < G;
+    float uh[D / 2];
+#pragma unroll
+    for (int e = 0; e < D / 2; ++e) uh[e] = sm.u[h][half * (D / 2) + e];
+    const T* kb = kbar + bg * (int64_t)nb * D;
+
+    // 2. per-head max and sum of 2^logit over the candidates
+    float m = -INFINITY, sum = 0.f;
+    for (int i = warp; i < ncand; i += kWarps) {
+        const float l = pair_dot<T, D>(kb + (int64_t)(lo + i) * D, uh, half);
+        if (l > m) {
+            sum = sum * exp2f(m - l) + 1.f;
+            m = l;
+        } else {
+            sum += exp2f(l - m);
+        }
+    }
+    if (half == 0 && live) {
+        sm.m[warp][h] = m;
+        sm.s[warp][h] = sum;
+    }
+    __syncthreads();
+    if (tid < G) {
+        float M = -INFINITY;
+        for (int w = 0; w < kWarps; ++w) M = fmaxf(M, sm.m[w][tid]);
+        float S = 0.f;
+        for (int w = 0; w < kWarps; ++w)
+            if (sm.m[w][tid] != -INFINITY) S += sm.s[w][tid] * exp2f(sm.m[w][tid] - M);
+        sm.M[tid] = M;
+        sm.S[tid] = S;
+    }
+    __syncthreads();
+    const float Mh = live ? sm.M[h] : 0.f, invS = live ? 1.f / sm.S[h] : 0.f;
+
+    // 3. scores chunk by chunk, the best K carried through a radix select per chunk
+    auto sync = [] { __syncthreads(); };
+    for (int cb = 0; cb < ncand; cb += kNew) {
+        const int nc = min(kNew, ncand - cb);
+        for (int i = warp; i < nc; i += kWarps) {
+            const float l = pair_dot<T, D>(kb + (int64_t)(lo + cb + i) * D, uh, half);
+            float p = (live && half == 0) ? exp2f(l - Mh) * invS : 0.f;
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) p += __shfl_xor_sync(0xffffffffu, p, off);
+            if (lane == 0) sm.keys[i] = sel_key(p, lo + cb + i);
+        }
+        for (int i = nc + tid; i < kNew; i += kThreads) sm.keys[i] = 0ull;
+        if (tid < kCapK) sm.keys[kNew + tid] = sm.carry[tid];
+        __syncthreads();
+        uint64_t key[kE];
+#pragma unroll
+        for (int e = 0; e < kE; ++e) key[e] = sm.keys[e * kThreads + tid];
+        if (tid == 0) sm.n_win = 0;
+        uint64_t prefix, mask;
+        radix_kth<kE>(key, K, sm.rs, prefix, mask, tid, sync);
+#pragma unroll
+        for (int e = 0; e < kE; ++e)
+            if (key[e] && (key[e] & mask) >= prefix) sm.carry[atomicAdd(&sm.n_win, 1)] = key[e];
+        __syncthreads();
+    }
+
+    // 4. winners ascending, then the slot row for every token of the block
+    if (warp == 0) {
+        int x0 = 2 * lane < K ? key_block(sm.carry[2 * lane]) : 0x7fffffff;
+        int x1 = 2 * lane + 1 < K ? key_block(sm.carry[2 * lane + 1]) : 0x7fffffff;
+        sort64_asc(x0, x1, lane);
+        sm.win[2 * lane] = x0;
+        sm.win[2 * lane + 1] = x1;
+    }
+    __syncthreads();
+    for (int e = tid; e < nr * slots; e += kThreads) {
+        const int s = e % slots;
+        int v;
+        if (s < n_init) v = s;
+        else if (s < n_init + K) v = sm.win[s - n_init];
+        else if (s < n_init + K + n_local) v = c - n_local + 1 + (s - n_init - K);
+        else v = -1;
+        out[e] = v;
+    }
+}
+
+template <typename T, int D>
+cudaError_t launch_qbs(const void* q, const void* kbar, int32_t* idx, int B, int H, int Hkv, int Nq,
+                       int nb, int topk, int n_init, int n_local, float scale, cudaStream_t st) {
+    const int nqb = (Nq + kQB - 1) / kQB;
+    const int64_t grid = (int64_t)B * Hkv * nqb;
+    if (grid == 0) return cudaSuccess;
+    if (grid > 0x7fffffff || H / Hkv > kGmax) return cudaErrorNotSupported;
+    const int smem = (int)sizeof(QsSmem<D>);
+    cudaError_t e = ensure_smem<topk_qblock_softmax_kernel<T, D>>(smem);
+    if (e != cudaSuccess) return e;
+    topk_qblock_softmax_kernel<T, D><<<(unsigned)grid, kThreads, smem, st>>>(
+        static_cast<const T*>(q), static_cast<const T*>(kbar), idx, H, Hkv, Nq, nb, topk, n_init,
+        n_local, n_init + n_local + topk, scale * 1.4426950408889634f);
+    return cudaGetLastError();
+}
+
 template <typename T, int D>
 cudaError_t launch_qb(const void* q, const void* kbar, int32_t* idx, int B, int H, int Hkv, int Nq,
                       int nb, int topk, int n_init, int n_local, cudaStream_t st) {
@@ -221,6 +406,17 @@ cudaError_t launch_block_topk_qblock(DType dt, const void* q, const void* kbar, 
                        : launch_qb<float, 128>(q, kbar, idx, B, H, Hkv, Nq, nb, topk, n_init, n_local, st);
     return d == 64 ? launch_qb<__nv_bfloat16, 64>(q, kbar, idx, B, H, Hkv, Nq, nb, topk, n_init, n_local, st)
                    : launch_qb<__nv_bfloat16, 128>(q, kbar, idx, B, H, Hkv, Nq, nb, topk, n_init, n_local, st);
+}
+
+cudaError_t launch_block_topk_qblock_softmax(DType dt, const void* q, const void* kbar, int32_t* idx,
+                                             int B, int H, int Hkv, int Nq, int nb, int d, int topk,
+                                             int n_init, int n_local, float scale, cudaStream_t st,
+                                             DevCtx) {
+    if (dt == DType::F32)
+        return d == 64 ? launch_qbs<float, 64>(q, kbar, idx, B, H, Hkv, Nq, nb, topk, n_init, n_local, scale, st)
+                       : launch_qbs<float, 128>(q, kbar, idx, B, H, Hkv, Nq, nb, topk, n_init, n_local, scale, st);
+    return d == 64 ? launch_qbs<__nv_bfloat16, 64>(q, kbar, idx, B, H, Hkv, Nq, nb, topk, n_init, n_local, scale, st)
+                   : launch_qbs<__nv_bfloat16, 128>(q, kbar, idx, B, H, Hkv, Nq, nb, topk, n_init, n_local, scale, st);
 }
 
 }  // namespace sala

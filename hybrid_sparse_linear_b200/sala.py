@@ -44,6 +44,7 @@ _lib.sala_block_topk.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, 
                                  _st, _i, _vp]
 _lib.sala_block_topk_workspace.argtypes = [_i, _i, _i, _i, _i, _i, _i]
 _lib.sala_block_topk_qblock.argtypes = [_vp, _vp, _vp] + [_i] * 11 + [_vp]
+_lib.sala_block_topk_qblock_softmax.argtypes = [_vp, _vp, _vp] + [_i] * 10 + [ctypes.c_float, _i, _vp]
 _lib.sala_block_topk_workspace.restype = _st
 _lib.sala_sparse_prefill.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i,
                                      ctypes.c_float, _i, _vp]
@@ -69,6 +70,7 @@ _lib.sala_selftest_wait_timeout.argtypes = [_vp]
 for _f in ("sala_linear_prefill", "sala_linear_decode", "sala_linear_prefill_rope",
            "sala_linear_decode_rope", "sala_sparse_decode_paged", "sala_block_topk_qblock",
            "sala_linear_backward", "sala_qk_norm", "sala_sparse_prefill_lse", "sala_sparse_backward",
+           "sala_block_topk_qblock_softmax",
            "sala_block_compress",
            "sala_block_topk",
            "sala_sparse_prefill", "sala_sparse_decode", "sala_check_status",
@@ -264,6 +266,24 @@ def block_topk_qblock(q, kbar, topk, n_init, n_local, idx=None, block=64, stream
     _check(_lib.sala_block_topk_qblock(_ptr(q), _ptr(kbar), _ptr(idx), B, H, Hkv, Nq, nb, d, block,
                                        topk, n_init, n_local, _dt(q), _stream(stream)),
            "sala_block_topk_qblock")
+    return idx
+
+
+def block_topk_qblock_softmax(q, kbar, topk, n_init, n_local, idx=None, block=64, scale=0.0,
+                              stream=None):
+    """Query-block-granular selection scored by softmax-probability group aggregation.
+    q: [B,H,Nq,d]; kbar [B,Hkv,nb,d].  Returns idx [B,Hkv,Nq,slots] int32."""
+    B, H, Nq, d = q.shape
+    Hkv, nb = kbar.shape[1], kbar.shape[2]
+    slots = n_init + n_local + topk
+    _need(q, "q"); _need(kbar, "kbar", dtype=q.dtype)
+    if idx is None:
+        idx = torch.empty((B, Hkv, Nq, slots), dtype=torch.int32, device=q.device)
+    _need(idx, "idx", (B, Hkv, Nq, slots), torch.int32)
+    _check(_lib.sala_block_topk_qblock_softmax(_ptr(q), _ptr(kbar), _ptr(idx), B, H, Hkv, Nq, nb,
+                                               d, block, topk, n_init, n_local, float(scale),
+                                               _dt(q), _stream(stream)),
+           "sala_block_topk_qblock_softmax")
     return idx
 
 

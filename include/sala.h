@@ -224,6 +224,19 @@ sala_status sala_block_topk_qblock(const void* q, const void* kbar, int32_t* idx
                                    int Hkv, int Nq, int nb, int d, int block, int topk, int n_init,
                                    int n_local, sala_dtype dt, sala_stream stream);
 
+/* Query-block-granular selection scored by softmax-probability group aggregation (another reading
+ * of the open scoring step).  For each (batch, KV group, query block c) and each of the group's
+ * heads h: u_h = the mean of the block's queries of head h, logits scale * (u_h . kbar_j) over the
+ * candidates j, a softmax over them; score(j) = the sum over the group's heads of the
+ * probabilities.  Candidates, forced blocks, ties, output layout and validation as
+ * sala_block_topk_qblock; scale 0 = 1/sqrt(d); at most 16 query heads per KV head.  The scores
+ * are fp32 on CUDA cores (two passes over the candidates: per-head max and sum, then the sum of
+ * probabilities and the top k). */
+sala_status sala_block_topk_qblock_softmax(const void* q, const void* kbar, int32_t* idx, int B,
+                                           int H, int Hkv, int Nq, int nb, int d, int block,
+                                           int topk, int n_init, int n_local, float scale,
+                                           sala_dtype dt, sala_stream stream);
+
 /* ------------------------------------------------------------------------------------------
  * Sparse attention prefill: exact causal softmax over the selected blocks.  Pages: sparse
  * layers compute on selected parts but keep the dense KV cache ("sparse compute, dense

@@ -406,3 +406,18 @@ def sparse_dq_rows(q, k, v, idx, do, block, rows, scale=None):
         (gq,) = torch.autograd.grad((o * torch.from_numpy(_f64(do[b, h, i]))).sum(), (Q,))
         out[n] = gq.numpy()
     return out
+
+
+def qblock_softmax_scores(q, kbar, block, b, g, c, n_init, n_local, scale=None):
+    """Scores of block_select_qblock_softmax's candidates n_init .. c - n_local for one (batch,
+    KV group, query block), plain numpy fp64: (candidate block ids, scores)."""
+    q, kbar = _f64(q), _f64(kbar)
+    B, H, Nq, d = q.shape
+    Hkv = kbar.shape[1]
+    G = H // Hkv
+    scale = (1.0 / np.sqrt(d)) if scale is None else float(scale)
+    u = q[b, g * G:(g + 1) * G, c * block:min(Nq, (c + 1) * block)].mean(axis=1)   # [G, d]
+    ids = np.arange(n_init, c - n_local + 1)
+    logits = scale * u @ kbar[b, g, ids].T                                          # [G, nc]
+    p = np.exp(logits - logits.max(axis=1, keepdims=True))
+    return ids, (p / p.sum(axis=1, keepdims=True)).sum(axis=0)

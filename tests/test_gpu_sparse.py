@@ -331,3 +331,64 @@ def test_qblock_pipeline(sala):
     got = idx.cpu().numpy()
     check_selection(got, ref, oracle.qblock_sum(q64, 64), kbar_ref, kth, topk, 1, 2)
     assert_close(_f64(o), oracle.sparse_attention(q64, k64, v64, got, 64), "bf16", "o")
+
+
+# ---------------------------------------------------------------------------------------------
+# Query-block selection scored by softmax-probability group aggregation
+
+def _check_softmax_selection(got, ref, kth, q64, kbar_ref, topk, n_init, n_local, rel=1e-3):
+    """Rows may differ only by near-ties: every block in the symmetric difference scores within
+    rel of the oracle's k-th score (scores from the oracle's fp64 helper)."""
+    B, Hkv, N, _ = got.shape
+    for b in range(B):
+        for g in range(Hkv):
+            for r0 in range(0, N, 64):
+                a, e = got[b, g, r0], ref[b, g, r0]
+                assert (got[b, g, r0:r0 + 64] == a).all(), (b, g, r0)
+                if (a == e).all():
+                    continue
+                c = r0 // 64
+                ids, sc = oracle.qblock_softmax_scores(q64, kbar_ref, 64, b, g, c, n_init, n_local)
+                score = dict(zip(ids.tolist(), sc.tolist()))
+                sa, se = {x for x in a if x >= 0}, {x for x in e if x >= 0}
+                assert len(sa) == len(se), (b, g, c)
+                k = kth[b, g, r0]
+                for x in sa ^ se:
+                    assert x in score, f"block {x} is not a candidate of query block {c}"
+                    assert abs(score[x] - k) <= rel * max(abs(score[x]), abs(k)), \
+                        f"query block {c}: block {x} scores {score[x]}, k-th {k}"
+
+
+@pytest.mark.parametrize("N,topk,dtype,d,H,Hkv", [
+    (64 * 200 + 7, 64, torch.bfloat16, 128, 32, 2),   # 16 heads per group, partial last block
+    (64 * 30 + 5, 8, torch.float32, 64, 8, 2),        # fp32, d 64
+    (64 * 4500 + 9, 64, torch.bfloat16, 128, 4, 2),   # > 4032 candidates: winners carried over chunks
+])
+def test_qblock_softmax_selection(sala, N, topk, dtype, d, H, Hkv):
+    from hybrid_sparse_linear_b200 import synth
+    layer = synth.sparse_layer(1, H, Hkv, N, d, dtype, layer=15, shift_frac=0.05)
+    kind = "bf16" if dtype == torch.bfloat16 else "f32"
+    q, k = layer.q.cuda(), layer.k.cuda()
+    kbar = sala.block_compress(k)
+    idx = sala.block_topk_qblock_softmax(q, kbar, topk, 1, 2)
+    sala.check_status()
+    kbar_ref = _f64(kbar)
+    q64 = _f64(layer.q)
+    ref, kth = oracle.block_select_qblock_softmax(q64, kbar_ref, 64, topk, 1, 2)
+    _check_softmax_selection(idx.cpu().numpy(), ref, kth, q64, kbar_ref, topk, 1, 2)
+
+
+def test_qblock_softmax_pipeline(sala):
+    from hybrid_sparse_linear_b200 import synth
+    N, topk = 64 * 90 + 21, 32
+    layer = synth.sparse_layer(1, 32, 2, N, 128, torch.bfloat16, layer=16, shift_frac=0.05)
+    q, k, v = layer.q.cuda(), layer.k.cuda(), layer.v.cuda()
+    kbar = sala.block_compress(k)
+    idx = sala.block_topk_qblock_softmax(q, kbar, topk, 1, 2)
+    o = sala.sparse_prefill(q, k, v, idx)
+    sala.check_status()
+    q64, k64, v64 = _f64(layer.q), _f64(layer.k), _f64(layer.v)
+    ref, kth = oracle.block_select_qblock_softmax(q64, _f64(kbar), 64, topk, 1, 2)
+    got = idx.cpu().numpy()
+    _check_softmax_selection(got, ref, kth, q64, _f64(kbar), topk, 1, 2)
+    assert_close(_f64(o), oracle.sparse_attention(q64, k64, v64, got, 64), "bf16", "o")

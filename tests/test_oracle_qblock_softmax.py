@@ -67,3 +67,22 @@ def test_zero_scale_ties_to_lowest_blocks():
     # block c = 11: candidates 1 .. 9, all scoring G / 9; the lowest three win
     assert list(idx[0, 0, 64 * 11]) == [0, 1, 2, 3, 10, 11]
     assert abs(kth[0, 0, 64 * 11] - 2 / 9) < 1e-12
+
+
+def test_numpy_scores_agree_with_the_selection():
+    q = _rand((2, 6, 64 * 20 + 9, 16), 10)
+    kbar = _rand((2, 2, 21, 16), 11)
+    topk, n_init, n_local = 4, 1, 2
+    idx, kth = oracle.block_select_qblock_softmax(q, kbar, 64, topk, n_init, n_local)
+    for b in range(2):
+        for g in range(2):
+            for c in (3, 9, 20):
+                ids, sc = oracle.qblock_softmax_scores(q, kbar, 64, b, g, c, n_init, n_local)
+                assert abs(sc.sum() - 3.0) < 1e-12  # G heads, each a distribution
+                best = ids[np.lexsort((ids, -sc))][:topk]
+                forced = {0} | set(range(c - n_local + 1, c + 1))
+                assert sorted(forced | set(best.tolist())) == [x for x in idx[b, g, 64 * c] if x >= 0]
+                if len(ids) >= topk:
+                    assert abs(np.sort(sc)[::-1][topk - 1] - kth[b, g, 64 * c]) < 1e-12
+                else:
+                    assert kth[b, g, 64 * c] == -np.inf
