@@ -525,7 +525,9 @@ def run_decode(sala, synth, torch, steps, warmup, stream, T=DECODE_T):
     flush = torch.empty(512 << 20, device=dev, dtype=torch.uint8)
     torch.cuda.synchronize()
 
-    def one_token():
+    # Linear layers launch as programmatic dependents of the kernel before them (each reads its
+    # own state while the previous layer finishes); the token is also timed without that.
+    def one_token(pdl=True):
         for l in range(N_LAYERS):
             if l in SPARSE_LAYERS:
                 q, kc, vc, kbar = sp[SPARSE_LAYERS.index(l)]
@@ -533,7 +535,7 @@ def run_decode(sala, synth, torch, steps, warmup, stream, T=DECODE_T):
                                    stream=stream)
             else:
                 S, q, k, v = lin[l - sum(1 for s in SPARSE_LAYERS if s < l)]
-                sala.linear_decode(q, k, v, lam, S, o=o, stream=stream)
+                sala.linear_decode(q, k, v, lam, S, o=o, stream=stream, pdl=pdl)
 
     times = []
     with torch.cuda.stream(stream):
@@ -546,18 +548,25 @@ def run_decode(sala, synth, torch, steps, warmup, stream, T=DECODE_T):
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph, stream=stream):
             one_token()
+        graph_plain = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph_plain, stream=stream):
+            one_token(pdl=False)
         for _ in range(warmup):
             graph.replay()
+            graph_plain.replay()
+        times_plain = []
         for _ in range(steps):
-            flush.zero_()
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            graph.replay()
-            b.record(stream)
-            times.append((a, b))
+            for g_, ts_ in ((graph, times), (graph_plain, times_plain)):
+                flush.zero_()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                g_.replay()
+                b.record(stream)
+                ts_.append((a, b))
         torch.cuda.synchronize()
     sala.check_status(stream)
     us = [a.elapsed_time(b) * 1000.0 for a, b in times]
+    us_plain = [a.elapsed_time(b) * 1000.0 for a, b in times_plain]
 
     def per_layer(kind):
         # The same calls of one kind only, captured and replayed the same way: where the time goes.
@@ -572,7 +581,7 @@ def run_decode(sala, synth, torch, steps, warmup, stream, T=DECODE_T):
                                            workspace=ws, stream=stream)
                     else:
                         S, q, k, v = lin[l - sum(1 for s in SPARSE_LAYERS if s < l)]
-                        sala.linear_decode(q, k, v, lam, S, o=o, stream=stream)
+                        sala.linear_decode(q, k, v, lam, S, o=o, stream=stream, pdl=True)
             for _ in range(warmup):
                 g.replay()
             ts = []
@@ -589,11 +598,12 @@ def run_decode(sala, synth, torch, steps, warmup, stream, T=DECODE_T):
 
     lin_us, sp_us = per_layer("linear"), per_layer("sparse")
     sala.check_status(stream)
-    del graph, lin, sp, ws, flush
+    del graph, graph_plain, lin, sp, ws, flush
     torch.cuda.empty_cache()
     # launches per token: linear 1 each; sparse 1 each (scoring, top-k, attention and combine in
     # one cooperative launch)
     return {"us_per_token": statistics.median(us), "us_min": min(us), "samples": len(us),
+            "us_per_token_without_pdl": statistics.median(us_plain),
             "launches_per_token": 24 * 1 + 8 * 1,
             "us_per_linear_layer": lin_us, "us_per_sparse_layer": sp_us}
 
@@ -934,9 +944,12 @@ def main():
                           "launches_per_token": dec["launches_per_token"],
                           "us_per_linear_layer": dec["us_per_linear_layer"],
                           "us_per_sparse_layer": dec["us_per_sparse_layer"],
+                          "us_per_token_without_pdl": dec["us_per_token_without_pdl"],
                           "timing": "CUDA events around one CUDA-graph replay of a token's 32 layer "
-                                    "calls, L2 flushed before each token, median; per-layer figures "
-                                    "from graphs of one kind of call only"}
+                                    "calls, L2 flushed before each token, median; linear layers "
+                                    "launched as programmatic dependents (state read overlapping "
+                                    "the previous layer); per-layer figures from graphs of one kind "
+                                    "of call only"}
     if "e2e" in phases:
         e = run_e2e(sala, synth, torch, max(1, min(args.steps, 2)), 1)
         line["e2e"] = {"value": ws * N_TOK / (max_over_ranks(e["ms_per_step"], "cuda") / 1000.0),

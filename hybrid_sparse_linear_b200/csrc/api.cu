@@ -260,7 +260,8 @@ sala_status sala_linear_backward(const void* q, const void* k, const void* v, co
 
 static sala_status linear_decode_impl(const void* q, const void* k, const void* v,
                                       const float* decay, float* state, void* o, int B, int H,
-                                      int d, sala::Rope rope, sala_dtype dt, sala_stream stream) {
+                                      int d, sala::Rope rope, bool pdl, sala_dtype dt,
+                                      sala_stream stream) {
     REQUIRE(B >= 0 && H >= 0, SALA_ERR_INVALID_ARG, "negative size (B=%d H=%d)", B, H);
     REQUIRE(dt == SALA_F32 || dt == SALA_BF16, SALA_ERR_INVALID_ARG, "unknown dtype %d", (int)dt);
     REQUIRE(d == 64 || d == 128, SALA_ERR_UNSUPPORTED, "head dim %d (supported: 64, 128)", d);
@@ -271,14 +272,25 @@ static sala_status linear_decode_impl(const void* q, const void* k, const void* 
     sala_status s = get_ctx(&ctx);
     if (s != SALA_OK) return s;
     return launched(sala::launch_linear_decode(to_dt(dt), q, k, v, decay, state, o, B, H, d,
-                                               rope, static_cast<cudaStream_t>(stream), ctx),
+                                               rope, pdl, static_cast<cudaStream_t>(stream), ctx),
                     "linear_decode");
 }
 
 sala_status sala_linear_decode(const void* q, const void* k, const void* v, const float* decay,
                                float* state, void* o, int B, int H, int d, sala_dtype dt,
                                sala_stream stream) {
-    return linear_decode_impl(q, k, v, decay, state, o, B, H, d, sala::Rope{0.0, 0}, dt, stream);
+    return linear_decode_impl(q, k, v, decay, state, o, B, H, d, sala::Rope{0.0, 0}, false, dt,
+                              stream);
+}
+
+sala_status sala_linear_decode_pdl(const void* q, const void* k, const void* v, const float* decay,
+                                   float* state, void* o, int B, int H, int d, int64_t pos,
+                                   double rope_base, sala_dtype dt, sala_stream stream) {
+    REQUIRE(pos >= 0, SALA_ERR_INVALID_ARG, "pos %lld is negative", (long long)pos);
+    REQUIRE(rope_base == 0.0 || (rope_base > 1.0 && rope_base < 1e30), SALA_ERR_INVALID_ARG,
+            "rope_base %g (0, or in (1, 1e30))", rope_base);
+    return linear_decode_impl(q, k, v, decay, state, o, B, H, d, sala::Rope{rope_base, pos}, true,
+                              dt, stream);
 }
 
 sala_status sala_linear_decode_rope(const void* q, const void* k, const void* v,
@@ -288,8 +300,8 @@ sala_status sala_linear_decode_rope(const void* q, const void* k, const void* v,
     REQUIRE(pos >= 0, SALA_ERR_INVALID_ARG, "pos %lld is negative", (long long)pos);
     REQUIRE(rope_base > 1.0 && rope_base < 1e30, SALA_ERR_INVALID_ARG,
             "rope_base %g (must lie in (1, 1e30))", rope_base);
-    return linear_decode_impl(q, k, v, decay, state, o, B, H, d, sala::Rope{rope_base, pos}, dt,
-                              stream);
+    return linear_decode_impl(q, k, v, decay, state, o, B, H, d, sala::Rope{rope_base, pos}, false,
+                              dt, stream);
 }
 
 // ----------------------------------------------------------------------------------------------

@@ -31,9 +31,11 @@ cudaError_t launch_linear_prefill_tc(const void* q, const void* k, const void* v
                                      float* s_out, int B, int H, int N, int d, void* ws,
                                      size_t ws_bytes, Rope rope, cudaStream_t st, DevCtx ctx);
 bool linear_prefill_tc_supported(int d);
+// pdl: launched as a programmatic dependent of the previous kernel in the stream (the state is
+// read before that kernel completes; it must not write this state).
 cudaError_t launch_linear_decode(DType dt, const void* q, const void* k, const void* v,
                                  const float* decay, float* state, void* o, int B, int H, int d,
-                                 Rope rope, cudaStream_t st, DevCtx ctx);
+                                 Rope rope, bool pdl, cudaStream_t st, DevCtx ctx);
 
 // Sparse attention.
 cudaError_t launch_block_compress(DType dt, const void* k, void* kbar, int B, int Hkv, int N,

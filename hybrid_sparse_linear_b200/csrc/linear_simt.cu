@@ -163,7 +163,11 @@ cudaError_t prefill_simt(const void* q, const void* k, const void* v, const floa
 // ---------------------------------------------------------------------------------------------
 // Decode: S <- lambda S + k^T v ; o = q S.  One CTA per (batch*head, 16-column slice); thread
 // (a, half) owns row a of the slice, 8 columns, loaded and stored as two float4.
-template <typename T, int D, bool kRope>
+// kPdl: launched as a programmatic dependent of the previous kernel in the stream.  The state
+// row is requested first, while that kernel may still run (the caller guarantees it does not
+// write this state); q, k, v and the decays are read after griddepcontrol.wait, i.e. after it
+// has completed and its writes are visible.  The next kernel may launch at once.
+template <typename T, int D, bool kRope, bool kPdl>
 __global__ void __launch_bounds__(2 * D)
 linear_decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                      const float* __restrict__ decay, float* __restrict__ state,
@@ -175,6 +179,10 @@ linear_decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* 
     const int a = tid >> 1, half = tid & 1;
     const int64_t bh = blockIdx.y;
     const int c0 = blockIdx.x * kCols + half * 8;
+    if constexpr (kPdl) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    float4* row = reinterpret_cast<float4*>(state + (bh * D + a) * D + c0);
+    float4 s0 = row[0], s1 = row[1];
+    if constexpr (kPdl) asm volatile("griddepcontrol.wait;" ::: "memory");
     const float lam = decay[bh % H];
     float ka = to_f(k[bh * D + a]);
     float qa = to_f(q[bh * D + a]);
@@ -190,8 +198,6 @@ linear_decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* 
     float vv[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) vv[j] = to_f(v[bh * D + c0 + j]);
-    float4* row = reinterpret_cast<float4*>(state + (bh * D + a) * D + c0);
-    float4 s0 = row[0], s1 = row[1];
     float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
     float part[8];
 #pragma unroll
@@ -218,16 +224,38 @@ linear_decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* 
     }
 }
 
+template <typename T, int D, bool kRope>
+cudaError_t decode_launch_pdl(const void* q, const void* k, const void* v, const float* decay,
+                              float* state, void* o, int H, Rope rope, dim3 grid, cudaStream_t st) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(2 * D);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, linear_decode_kernel<T, D, kRope, true>,
+                              static_cast<const T*>(q), static_cast<const T*>(k),
+                              static_cast<const T*>(v), decay, state, static_cast<T*>(o), H, rope);
+}
+
 template <typename T, int D>
 cudaError_t decode_launch(const void* q, const void* k, const void* v, const float* decay,
-                          float* state, void* o, int B, int H, Rope rope, cudaStream_t st) {
+                          float* state, void* o, int B, int H, Rope rope, bool pdl,
+                          cudaStream_t st) {
     dim3 grid(D / 16, (unsigned)(B * H));
+    if (pdl)
+        return rope.base > 0.0 ? decode_launch_pdl<T, D, true>(q, k, v, decay, state, o, H, rope, grid, st)
+                               : decode_launch_pdl<T, D, false>(q, k, v, decay, state, o, H, rope, grid, st);
     if (rope.base > 0.0)
-        linear_decode_kernel<T, D, true><<<grid, 2 * D, 0, st>>>(
+        linear_decode_kernel<T, D, true, false><<<grid, 2 * D, 0, st>>>(
             static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), decay,
             state, static_cast<T*>(o), H, rope);
     else
-        linear_decode_kernel<T, D, false><<<grid, 2 * D, 0, st>>>(
+        linear_decode_kernel<T, D, false, false><<<grid, 2 * D, 0, st>>>(
             static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), decay,
             state, static_cast<T*>(o), H, rope);
     return cudaGetLastError();
@@ -256,12 +284,12 @@ cudaError_t launch_linear_prefill_simt(DType dt, const void* q, const void* k, c
 
 cudaError_t launch_linear_decode(DType dt, const void* q, const void* k, const void* v,
                                  const float* decay, float* state, void* o, int B, int H, int d,
-                                 Rope rope, cudaStream_t st, DevCtx) {
+                                 Rope rope, bool pdl, cudaStream_t st, DevCtx) {
     if (dt == DType::F32)
-        return d == 64 ? decode_launch<float, 64>(q, k, v, decay, state, o, B, H, rope, st)
-                       : decode_launch<float, 128>(q, k, v, decay, state, o, B, H, rope, st);
-    return d == 64 ? decode_launch<__nv_bfloat16, 64>(q, k, v, decay, state, o, B, H, rope, st)
-                   : decode_launch<__nv_bfloat16, 128>(q, k, v, decay, state, o, B, H, rope, st);
+        return d == 64 ? decode_launch<float, 64>(q, k, v, decay, state, o, B, H, rope, pdl, st)
+                       : decode_launch<float, 128>(q, k, v, decay, state, o, B, H, rope, pdl, st);
+    return d == 64 ? decode_launch<__nv_bfloat16, 64>(q, k, v, decay, state, o, B, H, rope, pdl, st)
+                   : decode_launch<__nv_bfloat16, 128>(q, k, v, decay, state, o, B, H, rope, pdl, st);
 }
 
 }  // namespace sala

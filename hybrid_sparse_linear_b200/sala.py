@@ -37,6 +37,7 @@ _lib.sala_linear_backward_workspace.restype = _st
 _lib.sala_linear_prefill_rope.argtypes = [_vp] * 7 + [_i] * 4 + [ctypes.c_int64, ctypes.c_double,
                                                               _vp, _st, _i, _vp]
 _lib.sala_linear_decode_rope.argtypes = [_vp] * 6 + [_i] * 3 + [ctypes.c_int64, ctypes.c_double, _i, _vp]
+_lib.sala_linear_decode_pdl.argtypes = [_vp] * 6 + [_i] * 3 + [ctypes.c_int64, ctypes.c_double, _i, _vp]
 _lib.sala_qk_norm.argtypes = [_vp, _vp, ctypes.c_int64, _vp, _vp, ctypes.c_int64, _i,
                               ctypes.c_double, _i, _vp]
 _lib.sala_block_compress.argtypes = [_vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp]
@@ -70,7 +71,7 @@ _lib.sala_selftest_wait_timeout.argtypes = [_vp]
 for _f in ("sala_linear_prefill", "sala_linear_decode", "sala_linear_prefill_rope",
            "sala_linear_decode_rope", "sala_sparse_decode_paged", "sala_block_topk_qblock",
            "sala_linear_backward", "sala_qk_norm", "sala_sparse_prefill_lse", "sala_sparse_backward",
-           "sala_block_topk_qblock_softmax",
+           "sala_block_topk_qblock_softmax", "sala_linear_decode_pdl",
            "sala_block_compress",
            "sala_block_topk",
            "sala_sparse_prefill", "sala_sparse_decode", "sala_check_status",
@@ -176,9 +177,11 @@ def linear_backward(q, k, v, decay, dout, workspace=None, stream=None):
     return dq, dk, dv
 
 
-def linear_decode(q, k, v, decay, state, o=None, stream=None, rope_base=None, pos=0):
+def linear_decode(q, k, v, decay, state, o=None, stream=None, rope_base=None, pos=0, pdl=False):
     """One decode step.  q,k,v: [B,H,d]; state [B,H,d,d] fp32 (updated in place).  Returns o.
-    rope_base: rotate q and k at position pos first (sala_linear_decode_rope)."""
+    rope_base: rotate q and k at position pos first (sala_linear_decode_rope).  pdl: launch as a
+    programmatic dependent of the previous kernel in the stream (sala_linear_decode_pdl; that
+    kernel must not write `state`)."""
     B, H, d = q.shape
     _need(q, "q"); _need(k, "k", q.shape, q.dtype); _need(v, "v", q.shape, q.dtype)
     _need(decay, "decay", (H,), torch.float32)
@@ -186,6 +189,12 @@ def linear_decode(q, k, v, decay, state, o=None, stream=None, rope_base=None, po
     if o is None:
         o = torch.empty_like(q)
     _need(o, "o", q.shape, q.dtype)
+    if pdl:
+        _check(_lib.sala_linear_decode_pdl(_ptr(q), _ptr(k), _ptr(v), _ptr(decay), _ptr(state),
+                                           _ptr(o), B, H, d, int(pos),
+                                           float(rope_base) if rope_base is not None else 0.0,
+                                           _dt(q), _stream(stream)), "sala_linear_decode_pdl")
+        return o
     if rope_base is not None:
         _check(_lib.sala_linear_decode_rope(_ptr(q), _ptr(k), _ptr(v), _ptr(decay), _ptr(state),
                                             _ptr(o), B, H, d, int(pos), float(rope_base), _dt(q),

@@ -148,6 +148,18 @@ sala_status sala_linear_decode_rope(const void* q, const void* k, const void* v,
                                     int d, int64_t pos, double rope_base, sala_dtype dt,
                                     sala_stream stream);
 
+/* sala_linear_decode (rope_base == 0) or sala_linear_decode_rope (rope_base in (1, 1e30)),
+ * launched as a programmatic dependent of the previous kernel in the stream: the kernel starts
+ * while that kernel is still running and requests `state` at once; q, k, v and decay are read
+ * only after that kernel has completed and its writes are visible.  A decode step of many
+ * layers thus overlaps each layer's state read with the layer before (the state of a layer does
+ * not depend on the previous layer's output).  Contract: the previous kernel in the stream does
+ * not write `state` (e.g. two steps of the same layer back to back need sala_linear_decode).
+ * Captures into CUDA graphs.  Arguments, layouts and errors as sala_linear_decode_rope. */
+sala_status sala_linear_decode_pdl(const void* q, const void* k, const void* v, const float* decay,
+                                   float* state, void* o, int B, int H, int d, int64_t pos,
+                                   double rope_base, sala_dtype dt, sala_stream stream);
+
 /* ------------------------------------------------------------------------------------------
  * QK normalisation (weight-free RMS norm of every head row).  Pages: MiniCPM-SALA normalises
  * queries and keys to keep the activations stable (DE technical summary section 2, "additional

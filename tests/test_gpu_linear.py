@@ -274,3 +274,57 @@ def test_linear_backward(sala, d, N, B, H, dtype):
     assert_close(_f64(dq), rq, kind, "dq")
     assert_close(_f64(dk), rk, kind, "dk")
     assert_close(_f64(dv), rv, kind, "dv")
+
+
+# ---------------------------------------------------------------------------------------------
+# Decode steps launched as programmatic dependents (sala_linear_decode_pdl)
+
+@pytest.mark.parametrize("graph", [False, True])
+def test_pdl_decode_chain_of_layers(sala, graph):
+    # Three layers' decode steps back to back, each launched while the previous one may still run
+    # (it reads only its own state early); then a second token.  Every output and state against
+    # the oracle.  The middle layer rotates q and k (RoPE), the others do not.
+    from hybrid_sparse_linear_b200 import synth
+    B, H, d, L = 2, 32, 128, 3
+    g = torch.Generator().manual_seed(77)
+    lam = synth.decays(H)
+    states = [torch.randn((B, H, d, d), generator=g) / d for _ in range(L)]
+    toks = [[(torch.randn((B, H, d), generator=g) / 4).to(torch.bfloat16) for _ in range(3)]
+            for _ in range(2 * L)]
+    S_dev = [s.clone().cuda() for s in states]
+    outs = [torch.empty((B, H, d), device="cuda", dtype=torch.bfloat16) for _ in range(2 * L)]
+    qkv = [[x.cuda() for x in t] for t in toks]
+    lam_d = lam.cuda()
+    pos = 4097
+    stream = torch.cuda.Stream()
+
+    def run():
+        for step in range(2):
+            for l in range(L):
+                q, k, v = qkv[step * L + l]
+                sala.linear_decode(q, k, v, lam_d, S_dev[l], o=outs[step * L + l], stream=stream,
+                                   pdl=True, rope_base=10000.0 if l == 1 else None, pos=pos + step)
+
+    with torch.cuda.stream(stream):
+        if graph:
+            G = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(G, stream=stream):
+                run()
+            for l in range(L):  # capture ran nothing: start from the initial states
+                S_dev[l].copy_(states[l])
+            G.replay()
+        else:
+            run()
+    torch.cuda.synchronize()
+    sala.check_status(stream)
+    S_ref = [_f64(s) for s in states]
+    for step in range(2):
+        for l in range(L):
+            q, k, v = (_f64(x) for x in toks[step * L + l])
+            if l == 1:
+                q = oracle.rope(q[:, :, None], pos + step, 10000.0)[:, :, 0]
+                k = oracle.rope(k[:, :, None], pos + step, 10000.0)[:, :, 0]
+            o_ref, S_ref[l] = oracle.linear_decode(q, k, v, _f64(lam), S_ref[l])
+            assert_close(_f64(outs[step * L + l]), o_ref, "bf16", f"o step {step} layer {l}")
+    for l in range(L):
+        assert_close(_f64(S_dev[l]), S_ref[l], "bf16", f"state layer {l}")
