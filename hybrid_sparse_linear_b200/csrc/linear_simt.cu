@@ -166,7 +166,8 @@ cudaError_t prefill_simt(const void* q, const void* k, const void* v, const floa
 // kPdl: launched as a programmatic dependent of the previous kernel in the stream.  The state
 // row is requested first, while that kernel may still run (the caller guarantees it does not
 // write this state); q, k, v and the decays are read after griddepcontrol.wait, i.e. after it
-// has completed and its writes are visible.  The next kernel may launch at once.
+// has completed and its writes are visible.  Only then may the next kernel launch, so a
+// dependent's early reads overlap this kernel alone, never the one before it.
 template <typename T, int D, bool kRope, bool kPdl>
 __global__ void __launch_bounds__(2 * D)
 linear_decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
@@ -179,10 +180,12 @@ linear_decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* 
     const int a = tid >> 1, half = tid & 1;
     const int64_t bh = blockIdx.y;
     const int c0 = blockIdx.x * kCols + half * 8;
-    if constexpr (kPdl) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     float4* row = reinterpret_cast<float4*>(state + (bh * D + a) * D + c0);
     float4 s0 = row[0], s1 = row[1];
-    if constexpr (kPdl) asm volatile("griddepcontrol.wait;" ::: "memory");
+    if constexpr (kPdl) {
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    }
     const float lam = decay[bh % H];
     float ka = to_f(k[bh * D + a]);
     float qa = to_f(q[bh * D + a]);

@@ -229,7 +229,8 @@ sparse_decode_fused_kernel(const T* __restrict__ q, const T* __restrict__ kc,
     extern __shared__ __align__(16) unsigned char dsm_raw[];
     DecSmem<D>& sm = *reinterpret_cast<DecSmem<D>*>(dsm_raw);
     // A kernel launched after this one as its programmatic dependent (sala_linear_decode_pdl)
-    // may start now: it reads only its own state until this grid has completed.
+    // may start now: it reads only its own state until this grid has completed.  (This kernel is
+    // not itself a programmatic dependent, so everything launched before it has completed.)
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int G = H / Hkv;
