@@ -434,31 +434,33 @@ def run_linear_backward(sala, synth, torch, steps, warmup, stream, n_tok=N_TOK):
 
 def run_sparse_backward(sala, synth, torch, steps, warmup, stream, n_tok=N_TOK):
     """Training step of one sparse layer at N tokens (32 query / 2 KV heads, top-64 + 1 init +
-    2 local): the forward with its row log-sum-exp, then the backward (dq, dk, dv), each timed
-    with CUDA events over `steps` back-to-back calls.  Executed FLOPs are counted from the
-    selection: the query-side pass runs 6 MMAs of 2.10 MFLOP per (8-token tile, union block), the
+    2 local): the training forward (lse, o's residual), then the backward (dq, dk, dv), each
+    timed with CUDA events over `steps` back-to-back calls.  Executed FLOPs are counted from the
+    selection: the query-side pass runs 4 MMAs of 2.10 MFLOP per (8-token tile, union block), the
     key-side pass 4 per 8-token tile of each block's token list."""
     dev = torch.device("cuda")
     sl = synth.sparse_layer(1, H, HKV, n_tok, D, torch.bfloat16, dev, layer=3)
     dout = synth.normal((1, H, n_tok, D), synth.seed(3, 7), dev, torch.bfloat16)
     kbar = sala.block_compress(sl.k, stream=stream)
     idx = sala.block_topk(sl.q, kbar, TOPK, N_INIT, N_LOCAL, stream=stream)
-    o, lse = sala.sparse_prefill(sl.q, sl.k, sl.v, idx, lse=True, stream=stream)
+    o, lse, o_lo = sala.sparse_prefill(sl.q, sl.k, sl.v, idx, lse=True, o_lo=True, stream=stream)
     ws = torch.empty(sala.sparse_backward_workspace_bytes(1, H, HKV, n_tok, D, idx.shape[3]),
                      dtype=torch.uint8, device=dev)
     ev = lambda: torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
         for _ in range(warmup):
-            sala.sparse_prefill(sl.q, sl.k, sl.v, idx, o=o, lse=lse, stream=stream)
-            sala.sparse_backward(sl.q, sl.k, sl.v, idx, lse, dout, workspace=ws, stream=stream)
+            sala.sparse_prefill(sl.q, sl.k, sl.v, idx, o=o, lse=lse, o_lo=o_lo, stream=stream)
+            sala.sparse_backward(sl.q, sl.k, sl.v, idx, o, lse, dout, o_lo=o_lo, workspace=ws,
+                                 stream=stream)
         torch.cuda.synchronize()
         a, b, c = ev(), ev(), ev()
         a.record(stream)
         for _ in range(steps):
-            sala.sparse_prefill(sl.q, sl.k, sl.v, idx, o=o, lse=lse, stream=stream)
+            sala.sparse_prefill(sl.q, sl.k, sl.v, idx, o=o, lse=lse, o_lo=o_lo, stream=stream)
         b.record(stream)
         for _ in range(steps):
-            sala.sparse_backward(sl.q, sl.k, sl.v, idx, lse, dout, workspace=ws, stream=stream)
+            sala.sparse_backward(sl.q, sl.k, sl.v, idx, o, lse, dout, o_lo=o_lo, workspace=ws,
+                                 stream=stream)
         c.record(stream)
         torch.cuda.synchronize()
     sala.check_status(stream)
@@ -470,8 +472,8 @@ def run_sparse_backward(sala, synth, torch, steps, warmup, stream, n_tok=N_TOK):
     kv_tiles = int(((cnt + 7) // 8).sum().item())
     out = {"fwd_ms": a.elapsed_time(b) / steps, "bwd_ms": b.elapsed_time(c) / steps,
            "alg_flops": 10.0 * D * H * attended_keys(n_tok),
-           "exec_flops_dq": 6 * mma * union, "exec_flops_dkv": 4 * mma * kv_tiles}
-    del sl, dout, kbar, idx, o, lse, ws
+           "exec_flops_dq": 4 * mma * union, "exec_flops_dkv": 4 * mma * kv_tiles}
+    del sl, dout, kbar, idx, o, lse, o_lo, ws
     torch.cuda.empty_cache()
     return out
 

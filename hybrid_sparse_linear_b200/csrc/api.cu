@@ -491,8 +491,8 @@ sala_status sala_sparse_prefill(const void* q, const void* k, const void* v, con
     if (s != SALA_OK) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (dt == SALA_BF16 && sala::sparse_prefill_tc_supported(H, Hkv, d))
-        return launched(sala::launch_sparse_prefill_tc(q, k, v, idx, o, nullptr, B, H, Hkv, N, d,
-                                                       slots, scale, st, ctx),
+        return launched(sala::launch_sparse_prefill_tc(q, k, v, idx, o, nullptr, nullptr, B, H,
+                                                       Hkv, N, d, slots, scale, st, ctx),
                         "sparse_prefill_tc");
     return launched(sala::launch_sparse_prefill_simt(to_dt(dt), q, k, v, idx, o, B, H, Hkv, N, d,
                                                      slots, scale, st, ctx),
@@ -515,9 +515,9 @@ size_t sala_sparse_decode_workspace(int B, int H, int Hkv, int pos, int block, i
 
 // Forward with the row statistic the backward needs (bf16, d 128, 16 query heads per KV head).
 sala_status sala_sparse_prefill_lse(const void* q, const void* k, const void* v,
-                                    const int32_t* idx, void* o, float* lse, int B, int H, int Hkv,
-                                    int N, int d, int block, int slots, float scale, sala_dtype dt,
-                                    sala_stream stream) {
+                                    const int32_t* idx, void* o, float* lse, void* o_lo, int B,
+                                    int H, int Hkv, int N, int d, int block, int slots, float scale,
+                                    sala_dtype dt, sala_stream stream) {
     REQUIRE(B >= 0 && H >= 0 && Hkv > 0 && N >= 0 && slots >= 1, SALA_ERR_INVALID_ARG,
             "bad sizes (B=%d H=%d Hkv=%d N=%d slots=%d)", B, H, Hkv, N, slots);
     REQUIRE(dt == SALA_F32 || dt == SALA_BF16, SALA_ERR_INVALID_ARG, "unknown dtype %d", (int)dt);
@@ -529,17 +529,18 @@ sala_status sala_sparse_prefill_lse(const void* q, const void* k, const void* v,
     if (B == 0 || H == 0 || N == 0) return SALA_OK;
     REQ_PTR(q); REQ_PTR(k); REQ_PTR(v); REQ_PTR(o);
     REQUIRE(idx != nullptr && lse != nullptr, SALA_ERR_INVALID_ARG, "idx and lse must be device pointers");
+    REQUIRE(o_lo == nullptr || aligned16(o_lo), SALA_ERR_INVALID_ARG, "o_lo must be 16-byte aligned");
     if (scale == 0.f) scale = 1.0f / sqrtf((float)d);
     sala::DevCtx ctx;
     sala_status s = get_ctx(&ctx);
     if (s != SALA_OK) return s;
-    return launched(sala::launch_sparse_prefill_tc(q, k, v, idx, o, lse, B, H, Hkv, N, d, slots,
+    return launched(sala::launch_sparse_prefill_tc(q, k, v, idx, o, lse, o_lo, B, H, Hkv, N, d, slots,
                                                    scale, static_cast<cudaStream_t>(stream), ctx),
                     "sparse_prefill_lse");
 }
 
-// Backward pass of the sparse attention: the transposed selection, the query-side pass (D rows,
-// then dq), the key-side pass, then dk / dv rounded from their fp32 sums.
+// Backward pass of the sparse attention: D rows, the transposed selection, the query-side and
+// key-side passes, then dk / dv rounded from their fp32 sums.
 static size_t sparse_bwd_ws_parts(int B, int H, int Hkv, int N, int slots, size_t* o_csr,
                                   size_t* o_dk, size_t* o_dv) {
     auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
@@ -559,7 +560,8 @@ size_t sala_sparse_backward_workspace(int B, int H, int Hkv, int N, int d, int s
 }
 
 sala_status sala_sparse_backward(const void* q, const void* k, const void* v, const int32_t* idx,
-                                 const float* lse, const void* dout, void* dq,
+                                 const void* o, const void* o_lo, const float* lse,
+                                 const void* dout, void* dq,
                                  void* dk, void* dv, int B, int H, int Hkv, int N, int d, int block,
                                  int slots, float scale, void* workspace, size_t workspace_bytes,
                                  sala_dtype dt, sala_stream stream) {
@@ -574,8 +576,10 @@ sala_status sala_sparse_backward(const void* q, const void* k, const void* v, co
     REQUIRE((int64_t)B * Hkv * N * slots < ((int64_t)1 << 31), SALA_ERR_UNSUPPORTED,
             "B * Hkv * N * slots must stay below 2^31");
     if (B == 0 || H == 0 || N == 0) return SALA_OK;
-    REQ_PTR(q); REQ_PTR(k); REQ_PTR(v); REQ_PTR(dout); REQ_PTR(dq); REQ_PTR(dk); REQ_PTR(dv);
+    REQ_PTR(q); REQ_PTR(k); REQ_PTR(v); REQ_PTR(o); REQ_PTR(dout); REQ_PTR(dq); REQ_PTR(dk);
+    REQ_PTR(dv);
     REQUIRE(idx != nullptr && lse != nullptr, SALA_ERR_INVALID_ARG, "idx and lse must be device pointers");
+    REQUIRE(o_lo == nullptr || aligned16(o_lo), SALA_ERR_INVALID_ARG, "o_lo must be 16-byte aligned");
     size_t o_csr, o_dk, o_dv;
     const size_t need = sparse_bwd_ws_parts(B, H, Hkv, N, slots, &o_csr, &o_dk, &o_dv);
     REQUIRE(workspace != nullptr && aligned16(workspace) && workspace_bytes >= need,
@@ -592,7 +596,8 @@ sala_status sala_sparse_backward(const void* q, const void* k, const void* v, co
     float* dk_acc = reinterpret_cast<float*>(w + o_dk);
     float* dv_acc = reinterpret_cast<float*>(w + o_dv);
     const size_t acc_bytes = (size_t)B * Hkv * N * 128 * 4;
-    cudaError_t e = sala::launch_sparse_bwd_csr(idx, B, Hkv, N, slots, csr, st, ctx);
+    cudaError_t e = sala::launch_sparse_bwd_delta(o, o_lo, dout, delta, (int64_t)B * H * N, st);
+    if (e == cudaSuccess) e = sala::launch_sparse_bwd_csr(idx, B, Hkv, N, slots, csr, st, ctx);
     if (e == cudaSuccess) e = cudaMemsetAsync(dk_acc, 0, acc_bytes, st);
     if (e == cudaSuccess) e = cudaMemsetAsync(dv_acc, 0, acc_bytes, st);
     if (e != cudaSuccess) return launched(e, "sparse_backward prologue");

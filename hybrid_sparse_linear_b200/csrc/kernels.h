@@ -71,11 +71,13 @@ cudaError_t launch_sparse_prefill_simt(DType dt, const void* q, const void* k, c
                                        const int32_t* idx, void* o, int B, int H, int Hkv, int N,
                                        int d, int slots, float scale, cudaStream_t st,
                                        DevCtx ctx);
-// lse (may be null): per query row, the natural log-sum-exp of its visible scaled logits.
+// lse (may be null): the training forward -- per query row the natural log-sum-exp of its
+// visible scaled logits, P V taken as P_hi V + P_lo V, and (o_lo, may be null) the bf16 rounding
+// residual of o.
 cudaError_t launch_sparse_prefill_tc(const void* q, const void* k, const void* v,
-                                     const int32_t* idx, void* o, float* lse, int B, int H,
-                                     int Hkv, int N, int d, int slots, float scale, cudaStream_t st,
-                                     DevCtx ctx);
+                                     const int32_t* idx, void* o, float* lse, void* o_lo, int B,
+                                     int H, int Hkv, int N, int d, int slots, float scale,
+                                     cudaStream_t st, DevCtx ctx);
 
 // Sparse attention backward (bf16, G = 16, d = 128), selection held fixed.
 // The transposed selection: for key k = ((b * Hkv + g) * n_chunks + chunk) * nb + j,
@@ -92,10 +94,13 @@ struct SparseBwdCsr {
 SparseBwdCsr sparse_bwd_csr_layout(void* ws, int B, int Hkv, int N, int slots);
 cudaError_t launch_sparse_bwd_csr(const int32_t* idx, int B, int Hkv, int N, int slots,
                                   const SparseBwdCsr& c, cudaStream_t st, DevCtx ctx);
-// dq (bf16) from the query side: the forward's units walking the union of their selections
-// twice, first for D_i = sum_j P_ij dP_ij (written to delta, fp32 per query row), then for dq.
+// delta[row] = sum_c (o + o_lo)[row, c] * dout[row, c] in fp32, rows of 128 bf16 (o_lo may be
+// null).
+cudaError_t launch_sparse_bwd_delta(const void* o, const void* o_lo, const void* dout,
+                                    float* delta, int64_t rows, cudaStream_t st);
+// dq (bf16) from the query side: the forward's units walking the union of their selections.
 cudaError_t launch_sparse_dq_tc(const void* q, const void* k, const void* v, const void* dout,
-                                const int32_t* idx, const float* lse, float* delta, void* dq,
+                                const int32_t* idx, const float* lse, const float* delta, void* dq,
                                 int B, int H, int Hkv, int N, int slots, float scale,
                                 cudaStream_t st, DevCtx ctx);
 // dk_acc, dv_acc (fp32, zeroed by the caller) += the key side: key blocks walking their

@@ -1,10 +1,14 @@
 // CUDA-core pieces of the sparse attention backward (the tensor-core passes are in
 // sparse_bwd_tc.cu).  With the selection held fixed, o_i = sum_j P_ij v_j over the visible keys,
 // P_ij = exp(scale q_i.k_j - lse_i), and for the upstream gradient do:
-//   dP_ij = do_i . v_j,   D_i = sum_j P_ij dP_ij (= do_i . o_i),   dS_ij = P_ij (dP_ij - D_i)
+//   dP_ij = do_i . v_j,   D_i = sum_j P_ij dP_ij = do_i . o_i,   dS_ij = P_ij (dP_ij - D_i)
 //   dq_i = scale sum_j dS_ij k_j,   dk_j = scale sum_i dS_ij q_i,   dv_j = sum_i P_ij do_i
 // where i runs over the query rows of the KV group's G heads.
 //
+//   * delta: D_i = do_i . (o_i + o_lo_i) per query row (fp32).  D_i enters every dS_ij through
+//     dP_ij - D_i, which cancels on peaked softmaxes, so it needs o far beyond bf16: the training
+//     forward returns o's bf16 rounding residual o_lo (o + o_lo carries it to ~2^-16, its P V
+//     having taken P as bf16 hi + lo);
 //   * the transposed selection (CSR): for every (batch, KV group, chunk of kChunkTok query
 //     tokens, key block j) the chunk's tokens whose selection holds j, so the dk / dv pass can
 //     walk key blocks and gather their rows.  Keyed chunk-major, the lists laid end to end visit
@@ -25,6 +29,58 @@ constexpr int kThreads = 256;
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// ---------------------------------------------------------------------------------- delta
+// Rows of 128 bf16: 16 lanes of 16 bytes per row, two rows per warp instruction, four such
+// loads in flight per lane per tensor.  o + o_lo is exact in fp32 (at most 17 significant bits).
+__global__ void __launch_bounds__(kThreads)
+delta_kernel(const uint4* __restrict__ o, const uint4* __restrict__ o_lo,
+             const uint4* __restrict__ dout, float* __restrict__ delta, int64_t rows) {
+    constexpr int kU = 4;
+    const int lane = threadIdx.x & 31, sub = lane >> 4, col = lane & 15;
+    const int64_t warp = (blockIdx.x * (int64_t)kThreads + threadIdx.x) >> 5;
+    const int64_t n_warps = ((int64_t)gridDim.x * kThreads) >> 5;
+    for (int64_t r0 = warp * 2 * kU; r0 < rows; r0 += n_warps * 2 * kU) {
+        uint4 a[kU], b[kU], c[kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            const int64_t r = r0 + 2 * u + sub;
+            a[u] = b[u] = c[u] = make_uint4(0u, 0u, 0u, 0u);
+            if (r < rows) {
+                a[u] = __ldcs(o + r * 16 + col);
+                b[u] = __ldcs(dout + r * 16 + col);
+                if (o_lo != nullptr) c[u] = __ldcs(o_lo + r * 16 + col);
+            }
+        }
+        float s[kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            const uint32_t x[4] = {a[u].x, a[u].y, a[u].z, a[u].w};
+            const uint32_t y[4] = {b[u].x, b[u].y, b[u].z, b[u].w};
+            const uint32_t z[4] = {c[u].x, c[u].y, c[u].z, c[u].w};
+            float acc = 0.f;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float o0 = __uint_as_float(x[e] << 16) + __uint_as_float(z[e] << 16);
+                const float o1 = __uint_as_float(x[e] & 0xffff0000u) + __uint_as_float(z[e] & 0xffff0000u);
+                acc = fmaf(o0, __uint_as_float(y[e] << 16), acc);
+                acc = fmaf(o1, __uint_as_float(y[e] & 0xffff0000u), acc);
+            }
+            s[u] = acc;
+        }
+#pragma unroll
+        for (int off = 8; off > 0; off >>= 1)
+#pragma unroll
+            for (int u = 0; u < kU; ++u) s[u] += __shfl_xor_sync(0xffffffffu, s[u], off);
+        if (col == 0) {
+#pragma unroll
+            for (int u = 0; u < kU; ++u) {
+                const int64_t r = r0 + 2 * u + sub;
+                if (r < rows) delta[r] = s[u];
+            }
+        }
+    }
 }
 
 // ---------------------------------------------------------------------------------- CSR
@@ -207,6 +263,24 @@ SparseBwdCsr sparse_bwd_csr_layout(void* ws, int B, int Hkv, int N, int slots) {
     c.bsum = reinterpret_cast<int*>(base + o_bsum);
     c.bytes = o_bsum + up((size_t)n_blk * 4);
     return c;
+}
+
+cudaError_t launch_sparse_bwd_delta(const void* o, const void* o_lo, const void* dout,
+                                    float* delta, int64_t rows, cudaStream_t st) {
+    if (rows == 0) return cudaSuccess;
+    static int wave = 0;
+    if (!wave) {
+        int dev = 0, n_sm = 0, per_sm = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, delta_kernel, kThreads, 0);
+        wave = std::max(1, n_sm * std::max(1, per_sm));
+    }
+    const int64_t blocks = std::min<int64_t>((rows + 63) / 64, wave);
+    delta_kernel<<<(unsigned)blocks, kThreads, 0, st>>>(static_cast<const uint4*>(o),
+                                                        static_cast<const uint4*>(o_lo),
+                                                        static_cast<const uint4*>(dout), delta, rows);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_sparse_bwd_csr(const int32_t* idx, int B, int Hkv, int N, int slots,

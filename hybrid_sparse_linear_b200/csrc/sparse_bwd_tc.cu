@@ -5,16 +5,14 @@
 //
 // dq pass (query side): the forward's work units.  A unit is 16 consecutive tokens of one KV
 // group as two 128-row tiles (row = head * 8 + token) walking the union of their selections, K
-// and V of each union block loaded once for both tiles -- twice over: the first walk sums
-// D_i = sum_j P_ij dP_ij for every row (written out for the key side), the second forms dS
-// with it.  D is taken from the same fp32 P and dP as dS, not as do_i . o_i from the forward's
-// bf16 output: dP_ij - D_i cancels where the softmax is peaked, and the rounding of o (and of
-// the forward's bf16 P) would reach every dS_ij.  Per block and active tile X:
+// and V of each union block loaded once for both tiles.  D_i = do_i . o_i comes from the training
+// forward's output carried to ~2^-16 (o plus its bf16 residual, P taken as hi + lo in its P V):
+// dP_ij - D_i cancels where the softmax is peaked, so D must match the P the backward forms
+// (from the same lse and ex2) far better than a bf16 o does.  Per block and active tile X:
 //   S_X  = Q_X K_b^T      M=128 N=64 K=128    (TMEM)
 //   dP_X = dO_X V_b^T     M=128 N=64 K=128    (TMEM)
-//   first walk: D += sum_k P dP;   second walk: dS_X = P (dP - D) as two bf16 terms hi + lo
-//   (hi over S_X's columns, lo over dP_X's), and dQ_X += hi K_b + lo K_b   M=128 N=128 K=64
-//   (A from TMEM, B = K_b N-major).  The rows of dS sum to zero while the keys of a group share
+//   dS_X = P (dP - D) as two bf16 terms hi + lo (hi over S_X's columns, lo over dP_X's), and
+//   dQ_X += hi K_b + lo K_b   M=128 N=128 K=64   (A from TMEM, B = K_b N-major).  The rows of dS sum to zero while the keys of a group share
 //   a large common part, so dq = scale sum_j dS_ij k_j cancels: one bf16 term would leave an
 //   error of ~2^-9 sum_j |dS_ij| |k_j|, near 1 % of max |dq| on peaked selections.
 // TMEM holds dQ_A, dQ_B (128 columns each) and one S | dP pair per tile (128 columns each), so
@@ -124,7 +122,7 @@ __global__ void __launch_bounds__(dqp::kThreads, 1)
 sparse_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
                     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                     const int32_t* __restrict__ idx, const float* __restrict__ lse,
-                    float* __restrict__ delta, __nv_bfloat16* __restrict__ dq, int H,
+                    const float* __restrict__ delta, __nv_bfloat16* __restrict__ dq, int H,
                     int Hkv, int N, int slots, float sl2, float scale, int n_units, DevCtx ctx) {
     using namespace dqp;
     extern __shared__ uint8_t smraw[];
@@ -265,7 +263,7 @@ sparse_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                         }
                         ++kq;
                     }
-                    for (int e = 0; e < 2 * n && !stop; ++e, ++rc) {  // the union, twice
+                    for (int e = 0; e < n && !stop; ++e, ++rc) {
                         if (rc >= kStages && !wait_or_abort(empty_bar(rc), round_of(rc - kStages), ctx, abort)) {
                             stop = 1;
                             break;
@@ -273,7 +271,7 @@ sparse_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                         uint8_t* st = stage_ptr(rc);
                         uint64_t* fb = full_bar(rc);
                         mbar_arrive_expect_tx(fb, kKVBytes);
-                        const int y = list_id(lb)[e < n ? e : e - n] * kBlk;
+                        const int y = list_id(lb)[e] * kBlk;
                         tma_load_3d(st, &tmK, fb, 0, y, (int)bg);
                         tma_load_3d(st + kHalfBlk, &tmK, fb, 64, y, (int)bg);
                         tma_load_3d(st + 2 * kHalfBlk, &tmV, fb, 0, y, (int)bg);
@@ -295,9 +293,8 @@ sparse_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     } else if (warp == 9 || warp == 10) {
         // ---------------------------------------------------------------- MMA issuers
         // Warp 9 issues tile A's MMAs, warp 10 tile B's (one thread each).  Per active block:
-        // S and dP; on the second walk, once the tile's softmax has written dS, dQ += dS K; the
-        // stage goes back after the softmax is done with S and dP (first walk) or after the dQ
-        // MMA (second); a block the tile did not choose goes back at once.  An issuer holds no stage
+        // S and dP, then, once the tile's softmax has written dS, dQ += dS K and the stage goes
+        // back; a block the tile did not choose goes back at once.  An issuer holds no stage
         // while it waits for another, and its S of the next block is issued after the dQ that
         // reads this block's dS from the same TMEM columns (MMAs of one thread run in order).
         const int x = warp - 9;
@@ -325,10 +322,9 @@ sparse_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                     ++kq;
                     tc_fence_after();
                     bool accum = false;
-                    for (int b = 0; b < 2 * n && ok; ++b) {
+                    for (int b = 0; b < n && ok; ++b) {
                         const uint32_t e = rc + b;
-                        const bool second = b >= n;
-                        const bool act = ((list_mask(lb)[second ? b - n : b] >> (8 * x)) & 0xffu) != 0;
+                        const bool act = ((list_mask(lb)[b] >> (8 * x)) & 0xffu) != 0;
                         if (!(ok = wait_or_abort(full_bar(e), round_of(e), ctx, abort))) break;
                         if (!act) {
                             mbar_arrive(empty_bar(e));
@@ -350,7 +346,7 @@ sparse_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                         }
                         mma_commit(&bars.s_full[x]);
                         if (!(ok = wait_or_abort(&bars.p_full[x], a & 1u, ctx, abort))) break;
-                        if (second) {
+                        {
                             tc_fence_after();
 #pragma unroll
                             for (int ks = 0; ks < kBlk / 16; ++ks)
@@ -367,7 +363,7 @@ sparse_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                         ++a;
                     }
                     mma_commit(&bars.q_empty);
-                    rc += 2 * n;
+                    rc += n;
                 }
                 mbar_arrive(&bars.list_empty[lb]);
             }
@@ -408,53 +404,34 @@ sparse_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             const int i = i0 + t;
             const int64_t row = ((bg / Hkv) * H + (bg % Hkv) * kG + hh) * (int64_t)N + i;
             const float nl = i < N ? -__ldg(lse + row) * kLog2e : 0.f;
-            float dsum = 0.f;  // D_i, summed on the first walk
-            int last = -1;     // the tile's last dQ round (its dq_done phase)
-            for (int walk = 0; walk < 2; ++walk) {
-                for (int b = 0; b < n; ++b) {
-                    const unsigned msk = msks[b];
-                    if (((msk >> (8 * x)) & 0xffu) == 0) continue;
-                    const int blk = ids[b];
-                    const bool sel = (msk >> t) & 1u;
-                    const int lim = (!sel || i >= N) ? -1 : (blk == c ? i - blk * kBlk : kBlk - 1);
-                    if (!dead && !mbar_wait(&bars.s_full[x], a & 1u, ctx)) fail();
-                    tc_fence_after();
-                    if (!__any_sync(0xffffffffu, dead)) {
+            const float dv = i < N ? __ldg(delta + row) : 0.f;
+            int last = -1;  // the tile's last dQ round (its dq_done phase)
+            for (int b = 0; b < n; ++b) {
+                const unsigned msk = msks[b];
+                if (((msk >> (8 * x)) & 0xffu) == 0) continue;
+                const int blk = ids[b];
+                const bool sel = (msk >> t) & 1u;
+                const int lim = (!sel || i >= N) ? -1 : (blk == c ? i - blk * kBlk : kBlk - 1);
+                if (!dead && !mbar_wait(&bars.s_full[x], a & 1u, ctx)) fail();
+                tc_fence_after();
+                if (!__any_sync(0xffffffffu, dead)) {
 #pragma unroll
-                        for (int h = 0; h < 2; ++h) {
-                            uint32_t sr[32], pr[32];
-                            tmem_ld32(colS + 32 * h, sr);
-                            tmem_ld32(colP + 32 * h, pr);
-                            tmem_ld_wait();
-                            if (walk == 0) {
-                                float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-                                for (int q = 0; q < 16; ++q) {
-                                    const int k = 32 * h + 2 * q;
-                                    const float p0 = k <= lim ? ex2(fmaf(__uint_as_float(sr[2 * q]), sl2, nl)) : 0.f;
-                                    const float p1 = k + 1 <= lim ? ex2(fmaf(__uint_as_float(sr[2 * q + 1]), sl2, nl)) : 0.f;
-                                    s0 = fmaf(p0, __uint_as_float(pr[2 * q]), s0);
-                                    s1 = fmaf(p1, __uint_as_float(pr[2 * q + 1]), s1);
-                                }
-                                dsum += s0 + s1;
-                            } else {
-                                uint32_t hi[16], lo[16];
-                                ds_half(sr, pr, 32 * h, lim, sl2, nl, dsum, hi, lo);
-                                tmem_st16(colS + 16 * h, hi);  // columns already read
-                                tmem_st16(colP + 16 * h, lo);
-                            }
-                        }
+                    for (int h = 0; h < 2; ++h) {
+                        uint32_t sr[32], pr[32], hi[16], lo[16];
+                        tmem_ld32(colS + 32 * h, sr);
+                        tmem_ld32(colP + 32 * h, pr);
+                        tmem_ld_wait();
+                        ds_half(sr, pr, 32 * h, lim, sl2, nl, dv, hi, lo);
+                        tmem_st16(colS + 16 * h, hi);  // columns already read
+                        tmem_st16(colP + 16 * h, lo);
                     }
-                    if (walk == 1) {
-                        tmem_st_wait();
-                        ++last;
-                    }
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&bars.p_full[x]);
-                    ++a;
                 }
-                if (walk == 0 && i < N && !dead) delta[row] = dsum;
+                tmem_st_wait();
+                ++last;
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars.p_full[x]);
+                ++a;
             }
             last = last >= 0 ? (int)(ndq + last) : -1;
             ndq = last >= 0 ? (uint32_t)last + 1 : ndq;
@@ -943,7 +920,7 @@ int num_sms() {
 }  // namespace
 
 cudaError_t launch_sparse_dq_tc(const void* q, const void* k, const void* v, const void* dout,
-                                const int32_t* idx, const float* lse, float* delta, void* dq,
+                                const int32_t* idx, const float* lse, const float* delta, void* dq,
                                 int B, int H, int Hkv, int N, int slots, float scale,
                                 cudaStream_t st, DevCtx ctx) {
     if (H != Hkv * kG || slots > dqp::kMaxSlots) return cudaErrorNotSupported;

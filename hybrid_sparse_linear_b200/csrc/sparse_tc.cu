@@ -128,21 +128,24 @@ constexpr int kPolyEvery = 4;
 
 // p = 2^(s * sl2 + nb) for 64 keys, packed to 32 bf16 pairs and stored to TMEM columns
 // taddr .. taddr+31 in two pieces of 16; sums added to a0..a3.  kMasked zeroes the keys past lim
-// (the causal edge) and uses ex2.approx throughout, so masked keys give exact zeros.
-template <bool kMasked>
+// (the causal edge) and uses ex2.approx throughout, so masked keys give exact zeros.  kTrain (the
+// training forward) takes every key through ex2.approx, as the backward recomputes P, and stores
+// the bf16 rounding residual p - bf16(p) to columns taddr+32 .. taddr+63 (the S values there are
+// already in registers), so P V can be taken as P_hi V + P_lo V.
+template <bool kMasked, bool kTrain>
 __device__ __forceinline__ void exp_block(const uint32_t* s, float sl2, float nb, int lim,
                                           uint32_t taddr, float& a0, float& a1, float& a2,
                                           float& a3) {
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-        uint32_t pk[16];
+        uint32_t pk[16], lo[16];
 #pragma unroll
         for (int q = 0; q < 16; ++q) {
             const int k = 32 * h + 2 * q;
             float y0, y1;
             fma2_bcast(y0, y1, __uint_as_float(s[k]), __uint_as_float(s[k + 1]), sl2, nb);
             float p0, p1;
-            if (!kMasked && q % kPolyEvery == kPolyEvery - 1) {
+            if (!kMasked && !kTrain && q % kPolyEvery == kPolyEvery - 1) {
                 p0 = y0;
                 p1 = y1;
                 exp2_poly2(p0, p1);
@@ -157,17 +160,23 @@ __device__ __forceinline__ void exp_block(const uint32_t* s, float sl2, float nb
             if (q & 1) add2(a2, a3, p0, p1);
             else add2(a0, a1, p0, p1);
             pk[q] = pack_bf16x2(p0, p1);
+            if (kTrain)
+                lo[q] = pack_bf16x2(p0 - __uint_as_float(pk[q] << 16),
+                                    p1 - __uint_as_float(pk[q] & 0xffff0000u));
         }
         tmem_st16(taddr + 16 * h, pk);
+        if (kTrain) tmem_st16(taddr + 32 + 16 * h, lo);
     }
 }
 
+template <bool kTrain>
 __global__ void __launch_bounds__(kThreads, 1)
 sparse_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                          const __grid_constant__ CUtensorMap tmK,
                          const __grid_constant__ CUtensorMap tmV,
                          const int32_t* __restrict__ idx, __nv_bfloat16* __restrict__ out,
-                         float* __restrict__ lse, int H, int Hkv, int N, int slots, float sl2,
+                         float* __restrict__ lse, __nv_bfloat16* __restrict__ out_lo, int H,
+                         int Hkv, int N, int slots, float sl2,
                          int n_units, DevCtx ctx) {
     extern __shared__ uint8_t smraw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smraw) + 1023) &
@@ -390,6 +399,12 @@ sparse_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                         for (int ks = 0; ks < kBlk / 16; ++ks)
                             mma_ts_lohi(dO, aP + ks * 8, v_lo + ((ks * 16 * 128) >> 4), dhi, idPV,
                                         (accum || ks > 0) ? 1u : 0u);
+                        if constexpr (kTrain) {  // + P_lo V: the residual columns of the same buffer
+#pragma unroll
+                            for (int ks = 0; ks < kBlk / 16; ++ks)
+                                mma_ts_lohi(dO, aP + 32 + ks * 8, v_lo + ((ks * 16 * 128) >> 4), dhi,
+                                            idPV, 1u);
+                        }
                         mma_commit(&bars.pv_done[x][k & 1]);
                         mma_commit(empty_bar(e));
                         accum = true;
@@ -502,8 +517,8 @@ sparse_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                 if (go) {
                     const float nb = lim >= 0 ? -m_run : -INFINITY;
                     float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-                    if (diag) exp_block<true>(sr, sl2, nb, lim, colS, a0, a1, a2, a3);
-                    else exp_block<false>(sr, sl2, nb, lim, colS, a0, a1, a2, a3);
+                    if (diag) exp_block<true, kTrain>(sr, sl2, nb, lim, colS, a0, a1, a2, a3);
+                    else exp_block<false, kTrain>(sr, sl2, nb, lim, colS, a0, a1, a2, a3);
                     l += (a0 + a1) + (a2 + a3);
                 }
                 // Rescale O_x by 2^(m_old - m_new) where the max grew past the threshold (before
@@ -533,9 +548,10 @@ sparse_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                 ++a;
             }
             // Epilogue: O_x / l -> bf16 -> global (zeros when the tile saw no block); with lse,
-            // the row's natural log-sum-exp ln(sum_j e^(scale s_j)) = (m_run + log2 l) ln 2.
+            // the row's natural log-sum-exp ln(sum_j e^(scale s_j)) = (m_run + log2 l) ln 2; with
+            // out_lo, the bf16 rounding residual of each output element.
             const int64_t orow = (((bg / Hkv) * H + (bg % Hkv) * kG + hh) * (int64_t)N + i) * kD;
-            if (lse != nullptr && i < N && !dead)
+            if (kTrain && lse != nullptr && i < N && !dead)
                 lse[orow / kD] = (last >= 0 && m_run != -INFINITY && l > 0.f)
                                      ? (m_run + log2f(l)) * 0.69314718055994531f
                                      : -INFINITY;
@@ -560,6 +576,18 @@ sparse_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                             uint4* d4 = reinterpret_cast<uint4*>(out + orow + c0);
 #pragma unroll
                             for (int q = 0; q < 4; ++q) d4[q] = w[q];
+                            if (kTrain && out_lo != nullptr) {
+#pragma unroll
+                                for (int q = 0; q < 16; ++q) {
+                                    const float x0 = __uint_as_float(orr[2 * q]) * inv;
+                                    const float x1 = __uint_as_float(orr[2 * q + 1]) * inv;
+                                    wp[q] = pack_bf16x2(x0 - __uint_as_float(wp[q] << 16),
+                                                        x1 - __uint_as_float(wp[q] & 0xffff0000u));
+                                }
+                                uint4* l4 = reinterpret_cast<uint4*>(out_lo + orow + c0);
+#pragma unroll
+                                for (int q = 0; q < 4; ++q) l4[q] = w[q];
+                            }
                         }
                     }
                     tc_fence_before();
@@ -567,6 +595,10 @@ sparse_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
             } else if (i < N && !dead) {
                 uint4* d4 = reinterpret_cast<uint4*>(out + orow);
                 for (int q = 0; q < kD / 8; ++q) d4[q] = make_uint4(0, 0, 0, 0);
+                if (kTrain && out_lo != nullptr) {
+                    uint4* l4 = reinterpret_cast<uint4*>(out_lo + orow);
+                    for (int q = 0; q < kD / 8; ++q) l4[q] = make_uint4(0, 0, 0, 0);
+                }
             }
             asm volatile("bar.sync 1, 256;" ::: "memory");
             ++nbar;
@@ -590,9 +622,9 @@ bool sparse_prefill_tc_supported(int H, int Hkv, int d) {
 }
 
 cudaError_t launch_sparse_prefill_tc(const void* q, const void* k, const void* v,
-                                     const int32_t* idx, void* o, float* lse, int B, int H,
-                                     int Hkv, int N, int d, int slots, float scale, cudaStream_t st,
-                                     DevCtx ctx) {
+                                     const int32_t* idx, void* o, float* lse, void* o_lo, int B,
+                                     int H, int Hkv, int N, int d, int slots, float scale,
+                                     cudaStream_t st, DevCtx ctx) {
     if (d != kD || H != Hkv * kG || slots > kMaxSlots) return cudaErrorNotSupported;
     CUtensorMap tmQ, tmK, tmV;
     EncodeTiledFn fn = encode_tiled_fn();
@@ -618,15 +650,22 @@ cudaError_t launch_sparse_prefill_tc(const void* q, const void* k, const void* v
         cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
         if (num_sms <= 0) num_sms = 148;
     }
-    cudaError_t e = ensure_smem<sparse_prefill_tc_kernel>(kSmemBytes);
+    const bool train = lse != nullptr;
+    cudaError_t e = train ? ensure_smem<sparse_prefill_tc_kernel<true>>(kSmemBytes)
+                          : ensure_smem<sparse_prefill_tc_kernel<false>>(kSmemBytes);
     if (e != cudaSuccess) return e;
     const int units_per_seq = (N + kUT - 1) / kUT;
     const int n_units = units_per_seq * B * Hkv;
     const int grid = n_units < num_sms ? n_units : num_sms;
     const float sl2 = scale * 1.4426950408889634f;
-    sparse_prefill_tc_kernel<<<grid, kThreads, kSmemBytes, st>>>(
-        tmQ, tmK, tmV, idx, static_cast<__nv_bfloat16*>(o), lse, H, Hkv, N, slots, sl2, n_units,
-        ctx);
+    if (train)
+        sparse_prefill_tc_kernel<true><<<grid, kThreads, kSmemBytes, st>>>(
+            tmQ, tmK, tmV, idx, static_cast<__nv_bfloat16*>(o), lse,
+            static_cast<__nv_bfloat16*>(o_lo), H, Hkv, N, slots, sl2, n_units, ctx);
+    else
+        sparse_prefill_tc_kernel<false><<<grid, kThreads, kSmemBytes, st>>>(
+            tmQ, tmK, tmV, idx, static_cast<__nv_bfloat16*>(o), nullptr, nullptr, H, Hkv, N, slots,
+            sl2, n_units, ctx);
     return cudaGetLastError();
 }
 

@@ -58,10 +58,10 @@ _lib.sala_sparse_decode_paged.argtypes = [_vp, _vp, _vp, _i, _vp, _i, _vp, _i, _
                                           _i, _vp]
 _lib.sala_sparse_decode_paged_workspace.argtypes = [_i] * 9
 _lib.sala_sparse_decode_paged_workspace.restype = _st
-_lib.sala_sparse_prefill_lse.argtypes = [_vp] * 6 + [_i] * 7 + [ctypes.c_float, _i, _vp]
+_lib.sala_sparse_prefill_lse.argtypes = [_vp] * 7 + [_i] * 7 + [ctypes.c_float, _i, _vp]
 _lib.sala_sparse_backward_workspace.argtypes = [_i] * 6
 _lib.sala_sparse_backward_workspace.restype = _st
-_lib.sala_sparse_backward.argtypes = [_vp] * 9 + [_i] * 7 + [ctypes.c_float, _vp, _st, _i, _vp]
+_lib.sala_sparse_backward.argtypes = [_vp] * 11 + [_i] * 7 + [ctypes.c_float, _vp, _st, _i, _vp]
 _lib.sala_check_status.argtypes = [_vp]
 _lib.sala_status_string.argtypes = [_i]
 _lib.sala_status_string.restype = ctypes.c_char_p
@@ -296,10 +296,11 @@ def block_topk_qblock_softmax(q, kbar, topk, n_init, n_local, idx=None, block=64
     return idx
 
 
-def sparse_prefill(q, k, v, idx, o=None, block=64, scale=0.0, stream=None, lse=None):
+def sparse_prefill(q, k, v, idx, o=None, block=64, scale=0.0, stream=None, lse=None, o_lo=None):
     """Softmax attention over the selected blocks.  q: [B,H,N,d]; k,v: [B,Hkv,N,d].
     Training forward (sala_sparse_prefill_lse): lse = an fp32 [B,H,N] tensor, or True to allocate
-    one, receives each row's log-sum-exp; then (o, lse) is returned."""
+    one, receives each row's log-sum-exp; o_lo (a tensor like q, or True to allocate; None for
+    none) o's bf16 rounding residual.  Then (o, lse, o_lo) is returned."""
     B, H, N, d = q.shape
     Hkv = k.shape[1]
     _need(q, "q"); _need(k, "k", (B, Hkv, N, d), q.dtype); _need(v, "v", (B, Hkv, N, d), q.dtype)
@@ -313,10 +314,14 @@ def sparse_prefill(q, k, v, idx, o=None, block=64, scale=0.0, stream=None, lse=N
         if lse is True:
             lse = torch.empty((B, H, N), device=q.device, dtype=torch.float32)
         _need(lse, "lse", (B, H, N), torch.float32)
+        if o_lo is True:
+            o_lo = torch.empty_like(q)
+        _need(o_lo, "o_lo", q.shape, q.dtype)
         _check(_lib.sala_sparse_prefill_lse(_ptr(q), _ptr(k), _ptr(v), _ptr(idx), _ptr(o), _ptr(lse),
-                                            B, H, Hkv, N, d, block, idx.shape[3], float(scale),
-                                            _dt(q), _stream(stream)), "sala_sparse_prefill_lse")
-        return o, lse
+                                            _ptr(o_lo), B, H, Hkv, N, d, block, idx.shape[3],
+                                            float(scale), _dt(q), _stream(stream)),
+               "sala_sparse_prefill_lse")
+        return o, lse, o_lo
     _check(_lib.sala_sparse_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(idx), _ptr(o), B, H, Hkv, N, d,
                                     block, idx.shape[3], float(scale), _dt(q), _stream(stream)),
            "sala_sparse_prefill")
@@ -327,13 +332,15 @@ def sparse_backward_workspace_bytes(B, H, Hkv, N, d, slots):
     return _lib.sala_sparse_backward_workspace(B, H, Hkv, N, d, slots)
 
 
-def sparse_backward(q, k, v, idx, lse, dout, block=64, scale=0.0, workspace=None, stream=None):
+def sparse_backward(q, k, v, idx, o, lse, dout, o_lo=None, block=64, scale=0.0, workspace=None,
+                    stream=None):
     """Gradients (dq, dk, dv) of sum(o * dout) for the sparse attention with the selection idx
-    held fixed.  lse: from sparse_prefill(..., lse=True)."""
+    held fixed.  o, lse, o_lo: from sparse_prefill(..., lse=True, o_lo=True)."""
     B, H, N, d = q.shape
     Hkv = k.shape[1]
     _need(q, "q"); _need(k, "k", (B, Hkv, N, d), q.dtype); _need(v, "v", (B, Hkv, N, d), q.dtype)
-    _need(dout, "dout", q.shape, q.dtype)
+    _need(o, "o", q.shape, q.dtype); _need(dout, "dout", q.shape, q.dtype)
+    _need(o_lo, "o_lo", q.shape, q.dtype)
     _need(lse, "lse", (B, H, N), torch.float32)
     _need(idx, "idx", dtype=torch.int32)
     if idx.shape[:3] != (B, Hkv, N):
@@ -343,7 +350,8 @@ def sparse_backward(q, k, v, idx, lse, dout, block=64, scale=0.0, workspace=None
     need = _lib.sala_sparse_backward_workspace(B, H, Hkv, N, d, slots)
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
-    _check(_lib.sala_sparse_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(idx), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), B, H, Hkv, N, d,
+    _check(_lib.sala_sparse_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(idx), _ptr(o), _ptr(o_lo),
+                                     _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), B, H, Hkv, N, d,
                                      block, slots, float(scale), _ptr(workspace),
                                      workspace.numel(), _dt(q), _stream(stream)),
            "sala_sparse_backward")

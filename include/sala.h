@@ -282,14 +282,18 @@ sala_status sala_sparse_prefill(const void* q, const void* k, const void* v, con
  *
  * sala_sparse_prefill_lse: sala_sparse_prefill plus lse [B, H, N] fp32 (device, output), the
  *   natural log of sum_j exp(scale q_i.k_j) over row i's visible keys (-inf for a row that sees
- *   none).  Takes bf16, d 128, H = 16 Hkv, block 64, slots <= 80 (else SALA_ERR_UNSUPPORTED).
+ *   none).  This training forward takes P V as P_hi V + P_lo V (P split into two bf16 terms) and
+ *   every exponential through the same ex2 the backward uses, so o is exact to ~2^-16 before its
+ *   rounding; when o_lo is not NULL it receives [B, H, N, d] bf16 (device, output), the rounding
+ *   residual o - bf16(o), so o + o_lo carries that accuracy to the backward.  Takes bf16, d 128,
+ *   H = 16 Hkv, block 64, slots <= 80 (else SALA_ERR_UNSUPPORTED).
  *
- * sala_sparse_backward: q [B,H,N,d], k, v [B,Hkv,N,d], dout [B,H,N,d] (bf16, device), idx
+ * sala_sparse_backward: q [B,H,N,d], k, v [B,Hkv,N,d], o, o_lo, dout [B,H,N,d] (bf16, device), idx
  *   [B,Hkv,N,slots] (the selection the forward used: ascending distinct block ids, -1 padded,
- *   none in the future of its token), lse from sala_sparse_prefill_lse.  D_i is computed here
- *   as sum_j P_ij dP_ij from the same fp32 P and dP that form dS (not as do_i . o_i from the
- *   forward's bf16 o, whose rounding -- and that of the forward's bf16 P -- reaches every
- *   dS_ij = P_ij (dP_ij - D_i) through the cancellation in dP_ij - D_i).  Writes dq [B,H,N,d] and
+ *   none in the future of its token), o, o_lo and lse from sala_sparse_prefill_lse.  D_i =
+ *   do_i . (o_i + o_lo_i) enters every dS_ij = P_ij (dP_ij - D_i), a difference that cancels on
+ *   peaked softmaxes: o_lo may be NULL, but D then carries bf16 o's rounding (~1 % of max |dq|
+ *   on peaked selections).  Writes dq [B,H,N,d] and
  *   dk, dv [B,Hkv,N,d] (bf16, device, outputs; they must not alias the inputs).  scale 0 = 1/sqrt(d).
  *   workspace: >= sala_sparse_backward_workspace(...) bytes, 16-byte aligned, not shared with a
  *   concurrent call.  dk and dv are sums of fp32 atomic additions, so their last bits may vary
@@ -298,12 +302,13 @@ sala_status sala_sparse_prefill(const void* q, const void* k, const void* v, con
  *   SALA_ERR_BOUNDS by sala_check_status and skipped.
  * ---------------------------------------------------------------------------------------- */
 sala_status sala_sparse_prefill_lse(const void* q, const void* k, const void* v,
-                                    const int32_t* idx, void* o, float* lse, int B, int H, int Hkv,
-                                    int N, int d, int block, int slots, float scale, sala_dtype dt,
-                                    sala_stream stream);
+                                    const int32_t* idx, void* o, float* lse, void* o_lo, int B,
+                                    int H, int Hkv, int N, int d, int block, int slots, float scale,
+                                    sala_dtype dt, sala_stream stream);
 size_t sala_sparse_backward_workspace(int B, int H, int Hkv, int N, int d, int slots);
 sala_status sala_sparse_backward(const void* q, const void* k, const void* v, const int32_t* idx,
-                                 const float* lse, const void* dout, void* dq,
+                                 const void* o, const void* o_lo, const float* lse,
+                                 const void* dout, void* dq,
                                  void* dk, void* dv, int B, int H, int Hkv, int N, int d, int block,
                                  int slots, float scale, void* workspace, size_t workspace_bytes,
                                  sala_dtype dt, sala_stream stream);

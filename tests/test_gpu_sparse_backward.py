@@ -39,18 +39,23 @@ def _run(sala, q, k, v, dout, topk, n_local=2):
     qd, kd, vd, dd = q.cuda(), k.cuda(), v.cuda(), dout.cuda()
     kbar = sala.block_compress(kd)
     idx = sala.block_topk(qd, kbar, topk, 1, n_local)
-    o, lse = sala.sparse_prefill(qd, kd, vd, idx, lse=True)
-    dq, dk, dv = sala.sparse_backward(qd, kd, vd, idx, lse, dd)
+    o, lse, o_lo = sala.sparse_prefill(qd, kd, vd, idx, lse=True, o_lo=True)
+    dq, dk, dv = sala.sparse_backward(qd, kd, vd, idx, o, lse, dd, o_lo=o_lo)
     sala.check_status()
-    return idx.cpu().numpy(), o, lse, dq, dk, dv
+    return idx.cpu().numpy(), o, lse, dq, dk, dv, o_lo
 
 
 @pytest.mark.parametrize("B,Hkv,N,topk", [(1, 2, 1000, 4), (1, 2, 333, 64), (2, 1, 200, 2),
                                           (1, 1, 40, 4), (1, 2, 2048, 8)])
 def test_backward_matches_oracle(sala, B, Hkv, N, topk):
     q, k, v, dout = _layer(B, Hkv, N, 5 + N % 7)
-    idx, o, lse, dq, dk, dv = _run(sala, q, k, v, dout, topk)
+    idx, o, lse, dq, dk, dv, o_lo = _run(sala, q, k, v, dout, topk)
     q64, k64, v64, do64 = _f64(q), _f64(k), _f64(v), _f64(dout)
+    # the training forward's o + o_lo carries o to ~2^-16 (P V as P_hi V + P_lo V)
+    o_ref = oracle.sparse_attention(q64, k64, v64, idx, 64)
+    err = np.abs(_f64(o) + _f64(o_lo) - o_ref).max()
+    assert err <= 2e-4 * np.abs(o_ref).max(), f"o + o_lo max error {err}"
+    assert_close(_f64(o), o_ref, "bf16", "o")
     lse_ref = oracle.sparse_lse(q64, k64, idx, 64)
     err = np.abs(_f64(lse) - lse_ref)
     assert err.max() <= 2e-3, f"lse max error {err.max()}"
@@ -64,11 +69,11 @@ def test_future_block_is_flagged(sala):
     q, k, v, dout = _layer(1, 1, 256, 3)
     qd, kd, vd, dd = q.cuda(), k.cuda(), v.cuda(), dout.cuda()
     idx = sala.block_topk(qd, sala.block_compress(kd), 2, 1, 1)
-    o, lse = sala.sparse_prefill(qd, kd, vd, idx, lse=True)
+    o, lse, _ = sala.sparse_prefill(qd, kd, vd, idx, lse=True)
     sala.check_status()
     bad = idx.clone()
     bad[0, 0, 5, 2] = 3  # token 5 sits in block 0; block 3 is in its future
-    sala.sparse_backward(qd, kd, vd, bad, lse, dd)
+    sala.sparse_backward(qd, kd, vd, bad, o, lse, dd)
     with pytest.raises(sala.SalaError) as e:
         sala.check_status()
     assert e.value.code == sala.ERR_BOUNDS
@@ -77,7 +82,7 @@ def test_future_block_is_flagged(sala):
 def test_full_size_32k_sampled(sala):
     B, Hkv, N, topk = 1, 2, 32768, 64
     q, k, v, dout = _layer(B, Hkv, N, 9)
-    idx, o, lse, dq, dk, dv = _run(sala, q, k, v, dout, topk)
+    idx, o, lse, dq, dk, dv, _ = _run(sala, q, k, v, dout, topk)
     g = np.random.default_rng(4)
     rows = np.stack([np.zeros(48, dtype=np.int64), g.integers(0, 32, 48), g.integers(0, N, 48)], 1)
     rows[:4, 2] = [0, 63, 64, N - 1]
