@@ -71,8 +71,8 @@ def sparse_layer_flops(N: int) -> float:
 # ncu capture of the single-layer N = 131072 case, 2.319e9 bytes per launch, scaled by the tokens
 # processed to N = 262144 (Q reads, O writes and the K/V re-reads per 16-token unit all grow with N).
 # Valid only for the kernel source it was taken on: any change to it reports null.
-SPARSE_TRAFFIC = {"bytes_per_token": 2.318987776e9 / 131072,
-                  "sources": {"sparse_tc.cu": "1edc311bc80f3f0a15fa6418d666272925abf14f8568caeed0ade12fc70503f8",
+SPARSE_TRAFFIC = {"bytes_per_token": 2.316974848e9 / 131072,
+                  "sources": {"sparse_tc.cu": "4405ca3c032055be662e5ac02a49fd91f6a3ff7d78ca482c32d5fd612f22b580",
                               "fastexp.cuh": "b6d9ae064f35b9fd752ec893180eaf72ade6f0495d57f5699832618f42784c06"}}
 
 
