@@ -481,7 +481,9 @@ sparse_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
 // ================================================================================== dk / dv pass
 namespace dkvp {
 
-constexpr int kThreads = 352;  // warps 0-3 dS, 4-7 epilogue, 8 producer, 9 S|dP issuer, 10 dK|dV
+// warps 0-7 dS (two per row: keys 0-31 and 32-63), 8-11 epilogue, 12 producer, 13 S|dP issuer
+// (and TMEM owner), 14 dV issuer, 15 dK issuer
+constexpr int kThreads = 512;
 constexpr int kTok = 8;        // tokens per tile (x 16 heads = 128 rows)
 constexpr int kRingBytes = 2 * kTileBytes;          // Q tile then dO tile
 constexpr int kOffRing = kKVBytes;                  // after the K|V buffer
@@ -498,7 +500,7 @@ struct Bars {
     uint64_t s_full[2], s_free[2];
     uint64_t p_full[2], pds_free[2];
     uint64_t acc_full[2], acc_empty[2];
-    uint64_t fin[2];
+    uint64_t fin[3];
     uint32_t tmem_base;
     int abort;
 };
@@ -582,7 +584,7 @@ sparse_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     volatile int* abort = &bars.abort;
 
-    if (warp == 9) {
+    if (warp == 13) {
         tmem_alloc(&bars.tmem_base, kTmemCols);
         tmem_relinquish();
     }
@@ -590,16 +592,16 @@ sparse_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
         mbar_init(&bars.kv_full, 1);
         mbar_init(&bars.kv_empty, 1);
         for (int b = 0; b < 2; ++b) {
-            mbar_init(&bars.p_full[b], 4);
-            mbar_init(&bars.pds_free[b], 1);
+            mbar_init(&bars.p_full[b], 8);       // eight dS warps
+            mbar_init(&bars.pds_free[b], 2);     // the dV and dK issuers
             mbar_init(&bars.ring_full[b], 1);
-            mbar_init(&bars.ring_empty[b], 2);  // both issuers read a tile
+            mbar_init(&bars.ring_empty[b], 3);   // all three issuers read a tile
             mbar_init(&bars.s_full[b], 1);
-            mbar_init(&bars.s_free[b], 4);
-            mbar_init(&bars.acc_full[b], 1);
+            mbar_init(&bars.s_free[b], 8);
+            mbar_init(&bars.acc_full[b], 2);     // dK and dV of a segment
             mbar_init(&bars.acc_empty[b], 4);
-            mbar_init(&bars.fin[b], 1);
         }
+        for (int b = 0; b < 3; ++b) mbar_init(&bars.fin[b], 1);
         bars.abort = 0;
         fence_mbar_init();
     }
@@ -614,7 +616,7 @@ sparse_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
     auto sDS = [&](uint32_t t) { return sm + kOffP + (t & 1) * 2 * kPBytes + kPBytes; };
     Walk wk;
 
-    if (warp == 8) {
+    if (warp == 12) {
         // ---------------------------------------------------------------- producer
         // Per segment its K and V (once the buffer's segment two back is done), then per tile the
         // Q and dO rows of its tokens: lane u < 8 gathers token u (a short last tile repeats its
@@ -675,7 +677,7 @@ sparse_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             for (uint32_t e = t > 2 ? t - 2 : 0; e < t; ++e)
                 (void)mbar_wait(&bars.ring_full[e & 1], (e >> 1) & 1, ctx);
         }
-    } else if (warp == 9) {
+    } else if (warp == 13) {
         // ---------------------------------------------------------------- S | dP issuer
         if (lane == 0) {
             const uint32_t idS = idesc_bf16_f32(128, kBlk, false, false);
@@ -715,11 +717,13 @@ sparse_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             (void)mbar_wait(&bars.fin[0], 0, ctx);
         }
         __syncwarp();
-    } else if (warp == 10) {
-        // ---------------------------------------------------------------- dK | dV issuer
-        // dV^T += dO^T P and dK^T += Q^T dS: A is the tile read M-major (d contiguous, the two
-        // 64-column halves 16 KiB apart), B the P / dS rows read N-major; K runs over the 128
-        // rows in steps of 16 (2 KiB).
+    } else if (warp == 14 || warp == 15) {
+        // ---------------------------------------------------------------- dV, dK issuers
+        // Warp 14: dV^T += dO^T P; warp 15: dK^T += Q^T dS (one thread each, separate TMEM
+        // accumulators).  A is the tile read M-major (d contiguous, the two 64-column halves
+        // 16 KiB apart), B the P / dS rows read N-major; K runs over the 128 rows in steps of 16
+        // (2 KiB).
+        const bool isV = warp == 14;
         if (lane == 0) {
             const uint32_t idD = idesc_bf16_f32(128, kBlk, true, true);
             const uint32_t dhi = sdesc_sw128_hi(1024);
@@ -742,33 +746,31 @@ sparse_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                     const uint32_t do_lo = sdesc_sw128_lo(smem_u32(ring(t) + kTileBytes), kHalfQ);
                     const uint32_t p_lo = sdesc_sw128_lo(smem_u32(sP(t)), kHalfQ);
                     const uint32_t ds_lo = sdesc_sw128_lo(smem_u32(sDS(t)), kHalfQ);
+                    const uint32_t tD = isV ? tV : tK;
+                    const uint32_t a_lo = isV ? do_lo : q_lo, b_lo = isV ? p_lo : ds_lo;
 #pragma unroll
                     for (int ks = 0; ks < 128 / 16; ++ks) {
                         const uint32_t o = (ks * 16 * 128) >> 4;
-                        mma_ss_lohi(tV, do_lo + o, p_lo + o, dhi, idD, (first && ks == 0) ? 0u : 1u);
-                    }
-#pragma unroll
-                    for (int ks = 0; ks < 128 / 16; ++ks) {
-                        const uint32_t o = (ks * 16 * 128) >> 4;
-                        mma_ss_lohi(tK, q_lo + o, ds_lo + o, dhi, idD, (first && ks == 0) ? 0u : 1u);
+                        mma_ss_lohi(tD, a_lo + o, b_lo + o, dhi, idD, (first && ks == 0) ? 0u : 1u);
                     }
                     mma_commit(&bars.pds_free[u]);
                     mma_commit(&bars.ring_empty[u]);
                     if (pos + kTok >= wk.p1) mma_commit(&bars.acc_full[w]);
                 }
             }
-            mma_commit(&bars.fin[1]);
-            (void)mbar_wait(&bars.fin[1], 0, ctx);
+            mma_commit(&bars.fin[isV ? 1 : 2]);
+            (void)mbar_wait(&bars.fin[isV ? 1 : 2], 0, ctx);
         }
         __syncwarp();
-    } else if (warp < 4) {
+    } else if (warp < 8) {
         // ---------------------------------------------------------------- P and dS rows
-        // Thread = tile row r = TMEM lane r: token slot r / 16, head r % 16.  P and dS go to
+        // Thread = tile row r = TMEM lane r (token slot r / 16, head r % 16), keys 32 kh ..
+        // 32 kh + 31 of it: warps 0-3 take the first half of every row, warps 4-7 the second.  P and dS go to
         // shared memory as 128-byte rows with the 128-byte swizzle (16-byte chunk c of row r at
         // chunk c ^ (r & 7)), the layout the dK | dV issuer's descriptors read.
         // The row's token, lse and D are global loads, the latter two dependent on the first:
         // tokens are fetched two tiles ahead and lse, D one tile ahead of their use.
-        const int r = tid, slot = r >> 4, hh = r & 15;
+        const int r = tid & 127, slot = r >> 4, hh = r & 15, kh = warp >> 2;
         const uint32_t lane_base = tmem_lane_base(warp);
         auto row_of = [&](const Cursor& c) {
             const int64_t bg = c.w.key / (nb * n_chunks);
@@ -816,8 +818,8 @@ sparse_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
                 tc_fence_after();
                 uint4* prow = reinterpret_cast<uint4*>(sP(t) + r * 128);
                 uint4* srow = reinterpret_cast<uint4*>(sDS(t) + r * 128);
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
+                {
+                    const int h = kh;
                     uint32_t sr[32], pr[32], pkP[16], pkS[16];
                     tmem_ld32(tmem + lane_base + u * 128 + 32 * h, sr);
                     tmem_ld32(tmem + lane_base + u * 128 + 64 + 32 * h, pr);
@@ -852,11 +854,11 @@ sparse_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
             nl0 = nl1;
             dv0 = dv1;
         }
-    } else if (warp < 8) {
+    } else if (warp < 12) {
         // ---------------------------------------------------------------- epilogue
         // Thread = TMEM lane = column d of dK_b^T / dV_b^T; key by key, a warp adds 32
         // consecutive floats (128 bytes) of one key row into the fp32 accumulators.
-        const int d = tid - 128;
+        const int d = tid - 256;
         const uint32_t lane_base = tmem_lane_base(warp);
         uint32_t seg = 0;
         bool ok = true;
@@ -887,7 +889,7 @@ sparse_dkv_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_const
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 9) {
+    if (warp == 13) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
