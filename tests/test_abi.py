@@ -120,3 +120,40 @@ def test_product_never_imports_the_oracle():
             text = open(os.path.join(ROOT, "oracle", f)).read()
             assert not re.search(r"^\s*(import|from)\s+hybrid_sparse_linear_b200|libsala|sala\.h",
                                  text, re.M), f
+
+
+def test_host_validation_of_the_training_and_variant_calls(lib):
+    vp, i64, f32, f64 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_float, ctypes.c_double
+    lib.sala_last_error.restype = ctypes.c_char_p
+    good = vp(1 << 20)
+    # QK normalisation: head dim 96, eps 0, negative rows, an output overlapping its input
+    lib.sala_qk_norm.argtypes = [vp, vp, i64, vp, vp, i64, ctypes.c_int, f64, ctypes.c_int, vp]
+    assert lib.sala_qk_norm(good, good, 4, None, None, 0, 96, 1e-6, 1, None) == 2
+    assert lib.sala_qk_norm(good, good, 4, None, None, 0, 128, 0.0, 1, None) == 1
+    assert lib.sala_qk_norm(good, good, -1, None, None, 0, 128, 1e-6, 1, None) == 1
+    assert lib.sala_qk_norm(good, vp((1 << 20) + 256), 4, None, None, 0, 128, 1e-6, 1, None) == 1
+    assert b"overlaps" in lib.sala_last_error()
+    assert lib.sala_qk_norm(None, None, 0, None, None, 0, 128, 1e-6, 1, None) == 0  # nothing to do
+    # sparse training calls: only bf16, d 128, 16 query heads per KV head
+    lib.sala_sparse_prefill_lse.argtypes = [vp] * 7 + [ctypes.c_int] * 7 + [f32, ctypes.c_int, vp]
+    assert lib.sala_sparse_prefill_lse(good, good, good, good, good, good, None, 1, 8, 2, 128, 128,
+                                       64, 67, f32(0.0), 1, None) == 2
+    lib.sala_sparse_backward.argtypes = [vp] * 11 + [ctypes.c_int] * 7 + [f32, vp, ctypes.c_size_t,
+                                                                          ctypes.c_int, vp]
+    assert lib.sala_sparse_backward(good, good, good, good, good, None, good, good, good, good, good,
+                                    1, 32, 2, 128, 64, 64, 67, f32(0.0), good, 1 << 30, 1,
+                                    None) == 2                       # d 64
+    assert lib.sala_sparse_backward(good, good, good, good, good, None, good, good, good, good, good,
+                                    1, 32, 2, 128, 128, 64, 67, f32(0.0), good, 16, 1, None) == 1
+    assert b"workspace" in lib.sala_last_error()                    # workspace too small
+    lib.sala_sparse_backward_workspace.restype = ctypes.c_size_t
+    assert lib.sala_sparse_backward_workspace(1, 32, 2, 262144, 128, 67) > 2 * 2 * 262144 * 128 * 4
+    # softmax-aggregated selection: more than 16 query heads per KV head
+    lib.sala_block_topk_qblock_softmax.argtypes = [vp, vp, vp] + [ctypes.c_int] * 10 + [
+        f32, ctypes.c_int, vp]
+    assert lib.sala_block_topk_qblock_softmax(good, good, good, 1, 34, 2, 640, 10, 128, 64, 4, 1, 2,
+                                              f32(0.0), 1, None) == 2
+    # programmatic-dependent decode: a RoPE base in (0, 1] is rejected
+    lib.sala_linear_decode_pdl.argtypes = [vp] * 6 + [ctypes.c_int] * 3 + [i64, f64, ctypes.c_int, vp]
+    assert lib.sala_linear_decode_pdl(good, good, good, good, good, good, 1, 4, 128, 5, 0.5, 1,
+                                      None) == 1
