@@ -239,6 +239,7 @@ WORKLOADS = {
     # a sparse layer whose 64-token query blocks each share one selection (the variant)
     "sparse_qblock_prefill_n256k": (N_TOK, ["sparse_qblock"]),
     "sparse_qblock_softmax_prefill_n256k": (N_TOK, ["sparse_qsoft"]),
+    "linear_rope_prologue_prefill_n256k": (N_TOK, ["linear_rope_pro"]),
 }
 
 
@@ -263,6 +264,11 @@ def run_prefill(sala, synth, torch, steps, warmup, stream, workload="hybrid_pref
     # scratch of the sequence-parallel linear prefill (the segments' states)
     lws = torch.empty(max(sala.linear_prefill_workspace_bytes(1, H, n_tok, D), 16), device=dev,
                       dtype=torch.uint8)
+    # rotated q and k of a RoPE layer run as the one-pass prologue + the plain prefill
+    qr = kr = None
+    if "linear_rope_pro" in kinds:
+        qr = torch.empty((1, H, n_tok, D), device=dev, dtype=torch.bfloat16)
+        kr = torch.empty_like(qr)
     torch.cuda.synchronize()
 
     ev = lambda: torch.cuda.Event(enable_timing=True)
@@ -271,16 +277,21 @@ def run_prefill(sala, synth, torch, steps, warmup, stream, workload="hybrid_pref
     def one_step(record):
         launches = 0
         for kind, q, k, v in layers:
-            if kind in ("linear", "linear_rope"):
+            if kind in ("linear", "linear_rope", "linear_rope_pro"):
                 e0, e1 = (ev(), ev()) if record else (None, None)
                 if record: e0.record(stream)
                 if kind == "linear":
                     sala.linear_prefill(q, k, v, lam, o=out, workspace=lws, stream=stream)
-                else:
+                elif kind == "linear_rope":
                     sala.linear_prefill(q, k, v, lam, o=out, workspace=lws, stream=stream,
                                         rope_base=10000.0, pos0=0)
+                else:
+                    sala.qk_prologue(q, k, q_out=qr, k_out=kr, rope_base=10000.0, pos0=0,
+                                     stream=stream)
+                    sala.linear_prefill(qr, kr, v, lam, o=out, workspace=lws, stream=stream)
+                    launches += 1
                 if record: e1.record(stream); linear_ev.append((e0, e1))
-                launches += 1
+                launches += 3  # segment states, their chain, the output pass
             else:
                 t0, t1 = (ev(), ev()) if record else (None, None)
                 if record: t0.record(stream)
@@ -883,7 +894,7 @@ def main():
             line["kernels"]["sparse_prefill"] = {"mean_ms": pre["sparse_ms"], "achieved_tflops": achieved,
                                                  "executed_tflops": executed}
             line["kernels"]["compress_plus_select"] = {"mean_ms": pre["select_ms"]}
-        if "linear" in kinds or "linear_rope" in kinds:
+        if "linear" in kinds or "linear_rope" in kinds or "linear_rope_pro" in kinds:
             lin_gbs = linear_layer_bytes(n_tok) / (pre["linear_ms"] / 1000.0) / 1e9
             line["kernels"]["linear_prefill"] = {"mean_ms": pre["linear_ms"], "achieved_gbs": lin_gbs,
                                                  "hbm_frac": lin_gbs / peaks["hbm_gbs"]}

@@ -341,6 +341,50 @@ sala_status sala_qk_norm(const void* q, void* q_out, int64_t q_rows, const void*
                     "qk_norm");
 }
 
+sala_status sala_qk_prologue(const void* q, void* q_out, int64_t q_rows, const void* k,
+                             void* k_out, int64_t k_rows, int d, int N, double eps,
+                             int64_t pos0, double rope_base, sala_dtype dt, sala_stream stream) {
+    REQUIRE(q_rows >= 0 && k_rows >= 0, SALA_ERR_INVALID_ARG, "negative row count (q %lld, k %lld)",
+            (long long)q_rows, (long long)k_rows);
+    REQUIRE(dt == SALA_F32 || dt == SALA_BF16, SALA_ERR_INVALID_ARG, "unknown dtype %d", (int)dt);
+    REQUIRE(d == 64 || d == 128, SALA_ERR_UNSUPPORTED, "head dim %d (supported: 64, 128)", d);
+    REQUIRE(eps == 0.0 || (eps > 0.0 && eps < 1e30), SALA_ERR_INVALID_ARG,
+            "eps %g (0 for no norm, else positive and finite)", eps);
+    REQUIRE(rope_base == 0.0 || (rope_base > 1.0 && rope_base < 1e30), SALA_ERR_INVALID_ARG,
+            "rope_base %g (0 for no rotation, else in (1, 1e30))", rope_base);
+    REQUIRE(eps > 0.0 || rope_base > 0.0, SALA_ERR_INVALID_ARG, "neither a norm nor a rotation asked");
+    REQUIRE(N >= 1 && pos0 >= 0, SALA_ERR_INVALID_ARG, "N %d, pos0 %lld", N, (long long)pos0);
+    REQUIRE(q_rows % N == 0 && k_rows % N == 0, SALA_ERR_INVALID_ARG,
+            "row counts (q %lld, k %lld) must be multiples of N = %d", (long long)q_rows,
+            (long long)k_rows, N);
+    if (q_rows == 0 && k_rows == 0) return SALA_OK;
+    if (q_rows > 0) {
+        REQ_PTR(q); REQ_PTR(q_out);
+    }
+    if (k_rows > 0) {
+        REQ_PTR(k); REQ_PTR(k_out);
+    }
+    const int esize = dt == SALA_F32 ? 4 : 2;
+    auto overlap = [&](const void* a, const void* b, int64_t rows) {
+        const char* x = static_cast<const char*>(a);
+        const char* y = static_cast<const char*>(b);
+        const int64_t n = rows * d * esize;
+        return x != y && x < y + n && y < x + n;
+    };
+    REQUIRE(q_rows == 0 || !overlap(q, q_out, q_rows), SALA_ERR_INVALID_ARG,
+            "q_out overlaps q without being the same buffer");
+    REQUIRE(k_rows == 0 || !overlap(k, k_out, k_rows), SALA_ERR_INVALID_ARG,
+            "k_out overlaps k without being the same buffer");
+    sala::DevCtx ctx;
+    sala_status s = get_ctx(&ctx);
+    if (s != SALA_OK) return s;
+    return launched(sala::launch_qk_prologue(to_dt(dt), q_rows ? q : nullptr, q_rows ? q_out : nullptr,
+                                             q_rows, k_rows ? k : nullptr, k_rows ? k_out : nullptr,
+                                             k_rows, d, (float)eps, N, pos0, rope_base,
+                                             static_cast<cudaStream_t>(stream)),
+                    "qk_prologue");
+}
+
 // ----------------------------------------------------------------------------------------------
 sala_status sala_block_compress(const void* k, void* kbar, int B, int Hkv, int N, int d,
                                 int block, int first_block, int n_blocks, int nb_cap,

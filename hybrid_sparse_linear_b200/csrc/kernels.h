@@ -150,6 +150,11 @@ cudaError_t launch_flip_rows(DType dt, const void* in, void* out, int64_t BH, in
 // outputs may alias their inputs exactly.
 cudaError_t launch_qk_norm(DType dt, const void* q, void* q_out, int64_t q_rows, const void* k,
                            void* k_out, int64_t k_rows, int d, float eps, cudaStream_t st);
+// The same pass with an optional RoPE: eps > 0 normalises, rope_base > 0 rotates (row r of a
+// [B, heads, N, d] tensor at position pos0 + r % N); at least one of the two.
+cudaError_t launch_qk_prologue(DType dt, const void* q, void* q_out, int64_t q_rows, const void* k,
+                               void* k_out, int64_t k_rows, int d, float eps, int N, int64_t pos0,
+                               double rope_base, cudaStream_t st);
 
 // Diagnostics.
 cudaError_t launch_selftest_wait(cudaStream_t st, DevCtx ctx);

@@ -40,6 +40,8 @@ _lib.sala_linear_decode_rope.argtypes = [_vp] * 6 + [_i] * 3 + [ctypes.c_int64, 
 _lib.sala_linear_decode_pdl.argtypes = [_vp] * 6 + [_i] * 3 + [ctypes.c_int64, ctypes.c_double, _i, _vp]
 _lib.sala_qk_norm.argtypes = [_vp, _vp, ctypes.c_int64, _vp, _vp, ctypes.c_int64, _i,
                               ctypes.c_double, _i, _vp]
+_lib.sala_qk_prologue.argtypes = [_vp, _vp, ctypes.c_int64, _vp, _vp, ctypes.c_int64, _i, _i,
+                                  ctypes.c_double, ctypes.c_int64, ctypes.c_double, _i, _vp]
 _lib.sala_block_compress.argtypes = [_vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp]
 _lib.sala_block_topk.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _vp,
                                  _st, _i, _vp]
@@ -71,7 +73,7 @@ _lib.sala_selftest_wait_timeout.argtypes = [_vp]
 for _f in ("sala_linear_prefill", "sala_linear_decode", "sala_linear_prefill_rope",
            "sala_linear_decode_rope", "sala_sparse_decode_paged", "sala_block_topk_qblock",
            "sala_linear_backward", "sala_qk_norm", "sala_sparse_prefill_lse", "sala_sparse_backward",
-           "sala_block_topk_qblock_softmax", "sala_linear_decode_pdl",
+           "sala_block_topk_qblock_softmax", "sala_linear_decode_pdl", "sala_qk_prologue",
            "sala_block_compress",
            "sala_block_topk",
            "sala_sparse_prefill", "sala_sparse_decode", "sala_check_status",
@@ -224,6 +226,30 @@ def qk_norm(q, k=None, q_out=None, k_out=None, eps=1e-6, stream=None):
         k_rows = k.numel() // d
     _check(_lib.sala_qk_norm(_ptr(q), _ptr(q_out), q.numel() // d, _ptr(k), _ptr(k_out), k_rows,
                              d, float(eps), _dt(q), _stream(stream)), "sala_qk_norm")
+    return q_out, k_out
+
+
+def qk_prologue(q, k=None, q_out=None, k_out=None, eps=0.0, rope_base=0.0, pos0=0, stream=None):
+    """One pass over q [B,H,N,d] and k [B,Hk,N,d]: the QK normalisation (eps > 0) and/or the
+    linear layers' RoPE (rope_base > 0, row n at position pos0 + n).  Pass q_out=q / k_out=k to
+    work in place.  Returns (q_out, k_out)."""
+    N, d = q.shape[-2], q.shape[-1]
+    _need(q, "q")
+    if q_out is None:
+        q_out = torch.empty_like(q)
+    _need(q_out, "q_out", q.shape, q.dtype)
+    k_rows = 0
+    if k is not None:
+        _need(k, "k", dtype=q.dtype)
+        if k.shape[-2:] != q.shape[-2:]:
+            raise ValueError(f"k has rows x dim {tuple(k.shape[-2:])}, q has {tuple(q.shape[-2:])}")
+        if k_out is None:
+            k_out = torch.empty_like(k)
+        _need(k_out, "k_out", k.shape, k.dtype)
+        k_rows = k.numel() // d
+    _check(_lib.sala_qk_prologue(_ptr(q), _ptr(q_out), q.numel() // d, _ptr(k), _ptr(k_out), k_rows,
+                                 d, N, float(eps), int(pos0), float(rope_base), _dt(q),
+                                 _stream(stream)), "sala_qk_prologue")
     return q_out, k_out
 
 

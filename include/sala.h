@@ -180,6 +180,18 @@ sala_status sala_linear_decode_pdl(const void* q, const void* k, const void* v, 
 sala_status sala_qk_norm(const void* q, void* q_out, int64_t q_rows, const void* k, void* k_out,
                          int64_t k_rows, int d, double eps, sala_dtype dt, sala_stream stream);
 
+/* The prologue of a layer in one pass over q and k: the QK normalisation above (eps > 0; eps 0
+ * skips it) and/or the rotary embedding of the linear layers (rope_base > 0, as in
+ * sala_linear_prefill_rope: rotate-half pairs, theta_i = base^(-2i/d); row r of a [B, heads, N, d]
+ * tensor at position pos0 + r % N; rope_base 0 skips it), at least one of the two.  The norm is
+ * applied first; a rotation keeps each row's RMS, so the order matters only at rounding level.
+ * A linear layer with RoPE can then run the plain sala_linear_prefill on the rotated q and k
+ * (one more read and write of them, against the fused rotation's issue cost).  q_rows and
+ * k_rows are multiples of N; other arguments and errors as sala_qk_norm. */
+sala_status sala_qk_prologue(const void* q, void* q_out, int64_t q_rows, const void* k,
+                             void* k_out, int64_t k_rows, int d, int N, double eps,
+                             int64_t pos0, double rope_base, sala_dtype dt, sala_stream stream);
+
 /* ------------------------------------------------------------------------------------------
  * Block compression of the keys of a sparse layer (mean pooling).  Pages: InfLLM-V2 selects
  * the relevant context parts without extra parameters (JA technical summary section 2.1); the

@@ -109,3 +109,45 @@ def test_full_size_sampled(sala):
         xs = rows.index_select(0, idx).cpu()
         ys = y.reshape(-1, 128).index_select(0, idx).cpu()
         _check(ys, xs, torch.bfloat16)
+
+
+# ---------------------------------------------------------------------------------------------
+# The layer prologue (sala_qk_prologue): QK norm and/or RoPE in one pass
+
+@pytest.mark.parametrize("dtype,d,norm,rope", [(torch.bfloat16, 128, False, True),
+                                               (torch.bfloat16, 128, True, True),
+                                               (torch.bfloat16, 64, True, True),
+                                               (torch.float32, 128, False, True),
+                                               (torch.float32, 64, True, False)])
+def test_prologue_matches_oracle(sala, dtype, d, norm, rope):
+    N, pos0, base = 333, 4099, 10000.0
+    q = _pre((2, 3, N, d), 41, dtype)
+    k = _pre((2, 1, N, d), 42, dtype)
+    qo, ko = sala.qk_prologue(q.cuda(), k.cuda(), eps=EPS if norm else 0.0,
+                              rope_base=base if rope else 0.0, pos0=pos0)
+    sala.check_status()
+    kind = "bf16" if dtype == torch.bfloat16 else "f32"
+    for x, y in ((q, qo), (k, ko)):
+        ref = oracle.from_tensor(x)
+        if norm:
+            ref = oracle.qk_norm(ref, EPS)
+        if rope:
+            ref = oracle.rope(ref, pos0, base)
+        assert_close(oracle.from_tensor(y.cpu()), ref, kind)
+
+
+def test_rope_layer_as_prologue_plus_plain_prefill(sala):
+    # a linear layer with RoPE: rotate q, k in one pass, then the plain (tensor-core) prefill
+    from hybrid_sparse_linear_b200 import synth
+    B, H, N, d = 1, 4, 64 * 37 + 11, 128
+    q, k, v = synth.linear_layer(B, H, N, d, torch.bfloat16, "cpu", layer=5)
+    lam = synth.decays(H)
+    qd, kd = q.cuda(), k.cuda()
+    qr, kr = sala.qk_prologue(qd, kd, rope_base=10000.0, pos0=0)
+    ws = torch.empty(max(sala.linear_prefill_workspace_bytes(B, H, N, d), 16), device="cuda",
+                     dtype=torch.uint8)
+    o = sala.linear_prefill(qr, kr, v.cuda(), lam.cuda(), workspace=ws)
+    sala.check_status()
+    f = oracle.from_tensor
+    ref, _ = oracle.linear_chunked_rope(f(q), f(k), f(v), f(lam), 64, 0, 10000.0)
+    assert_close(f(o.cpu()), ref, "bf16", "o")
