@@ -25,9 +25,9 @@
 // warps 0-3 softmax + epilogue of tile A, warps 4-7 of tile B (thread = row = TMEM lane); warp 11
 // stages the next unit's 16 selection rows and merges them into its union list (double-buffered,
 // one unit ahead); warp 8 issues the TMA loads (Q tiles, then the ring); warp 9 allocates TMEM and
-// issues the MMAs of tile A, warp 10 those of tile B (one thread each).  Every wait is bounded; a timeout sets the
-// status word, the roles wind down, and the kernel waits (bounded) for its own copies and MMAs
-// before it frees TMEM.
+// issues the MMAs of tile A, warp 10 those of tile B (one elected lane of each converged warp).
+// Every wait is bounded; a timeout sets the status word, the roles wind down, and the kernel waits
+// (bounded) for its own copies and MMAs before it frees TMEM.
 #include "fastexp.cuh"
 #include "kernels.h"
 #include "ptx.cuh"
@@ -350,9 +350,10 @@ sparse_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
         }
     } else if (warp == 9 || warp == 10) {
         // ---------------------------------------------------------------- MMA issuers
-        // Warp 9 issues the MMAs of tile A, warp 10 those of tile B (one thread each): a single
-        // thread needs ~50 cycles per tcgen05.mma, more than the 32 of math in an N=64 S MMA, so
-        // two issuers keep the tensor pipe fed and the tiles' chains never wait on each other.
+        // Warp 9 issues the MMAs of tile A, warp 10 those of tile B.  The whole warp runs the loop
+        // converged with warp-uniform operands and one elected lane issues each instruction (a
+        // single-lane branch ran the same loop ~3 % slower).  Two issuers keep the tensor pipe
+        // fed and the tiles' chains never wait on each other.
         // Order per tile: S of round k+1 is issued before PV of round k (two S buffers), so the
         // tensor core computes the next S while the softmax works on this one.  Each issuer
         // observes every ring entry in order (so its parity waits never run two uses ahead of a
@@ -360,96 +361,98 @@ sparse_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
         // for a block it did not.  Before it waits for an entry whose stage still holds a block of
         // its own, it issues that block's PV, so it never holds a stage the producer needs.
         const int x = warp - 9;
-        if (lane == 0) {
-            const uint32_t idS = idesc_bf16_f32(128, kBlk, false, false);
-            const uint32_t idPV = idesc_bf16_f32(128, kD, false, true);
-            const uint32_t dO = tmem + kColO + x * 128;
-            // Shared-memory descriptors by halves: one high half for every operand here (stride
-            // 1024 B, 128-byte swizzle); low halves = address | leading offset, plus the K step.
-            const uint32_t dhi = sdesc_sw128_hi(1024);
-            const uint32_t q_lo = sdesc_sw128_lo(smem_u32(sm + x * kQBytes), 16);
-            const uint32_t ring_lo = sdesc_sw128_lo(smem_u32(sm + kOffRing), 16);
-            const uint32_t ring_v_lo = sdesc_sw128_lo(smem_u32(sm + kOffRing + 2 * kHalfBlk), kHalfBlk);
-            int it = 0;
-            uint32_t rc = 0, kq = 0, a = 0;  // ring entries seen, Q tile pairs used, S rounds issued
-            bool ok = true;
-            for (int unit = blockIdx.x; unit < n_units && ok; unit += gridDim.x, ++it) {
-                const int lb = it & 1;
-                ok = wait_or_abort(&bars.list_full[lb], (it >> 1) & 1, ctx, abort);
-                if (!ok) break;
-                const int n = bars.list_n[lb];
-                if (n > 0) {
-                    ok = wait_or_abort(&bars.q_full, kq & 1, ctx, abort);
-                    ++kq;
+        auto wait_w = [&](uint64_t* bar, uint32_t parity) -> bool {  // warp-uniform outcome
+            const bool r = wait_or_abort(bar, parity, ctx, abort);
+            return __shfl_sync(0xffffffffu, r ? 1 : 0, 0) != 0;
+        };
+        const uint32_t tm = __shfl_sync(0xffffffffu, tmem, 0);
+        const uint32_t idS = idesc_bf16_f32(128, kBlk, false, false);
+        const uint32_t idPV = idesc_bf16_f32(128, kD, false, true);
+        const uint32_t dO = tm + kColO + x * 128;
+        // Shared-memory descriptors: one high half for every operand here (stride 1024 B, 128-byte
+        // swizzle); low halves = address | leading offset, plus the K step.
+        const uint64_t dhi = (uint64_t)sdesc_sw128_hi(1024) << 32;
+        const uint64_t q_d = dhi | sdesc_sw128_lo(smem_u32(sm + x * kQBytes), 16);
+        const uint64_t ring_d = dhi | sdesc_sw128_lo(smem_u32(sm + kOffRing), 16);
+        const uint64_t ring_v_d = dhi | sdesc_sw128_lo(smem_u32(sm + kOffRing + 2 * kHalfBlk), kHalfBlk);
+        int it = 0;
+        uint32_t rc = 0, kq = 0, a = 0;  // ring entries seen, Q tile pairs used, S rounds issued
+        bool ok = true;
+        for (int unit = blockIdx.x; unit < n_units && ok; unit += gridDim.x, ++it) {
+            const int lb = it & 1;
+            ok = wait_w(&bars.list_full[lb], (it >> 1) & 1);
+            if (!ok) break;
+            const int n = bars.list_n[lb];
+            if (n > 0) {
+                ok = wait_w(&bars.q_full, kq & 1);
+                ++kq;
+                tc_fence_after();
+                // Rounds whose S is issued and whose PV is not: at most two, oldest first.
+                int np = 0;
+                uint32_t pe0 = 0, pk0 = 0, pe1 = 0, pk1 = 0;  // ring entry, round
+                bool accum = false;
+                auto flush_pv = [&]() -> bool {
+                    const uint32_t e = pe0, k = pk0;
+                    pe0 = pe1;
+                    pk0 = pk1;
+                    --np;
+                    if (!wait_w(&bars.p_full[x][k & 1], (k >> 1) & 1)) return false;
                     tc_fence_after();
-                    // Rounds whose S is issued and whose PV is not: at most two, oldest first.
-                    int np = 0;
-                    uint32_t pe0 = 0, pk0 = 0, pe1 = 0, pk1 = 0;  // ring entry, round
-                    bool accum = false;
-                    auto flush_pv = [&]() -> bool {
-                        const uint32_t e = pe0, k = pk0;
-                        pe0 = pe1;
-                        pk0 = pk1;
-                        --np;
-                        if (!wait_or_abort(&bars.p_full[x][k & 1], (k >> 1) & 1, ctx, abort)) return false;
-                        tc_fence_after();
-                        const uint32_t aP = tmem + kColS + x * 128 + (k & 1) * 64;
-                        const uint32_t v_lo = ring_v_lo + (e % kStages) * (kStageBytes >> 4);
+                    const uint32_t aP = tm + kColS + x * 128 + (k & 1) * 64;
+                    const uint64_t v_d = ring_v_d + (e % kStages) * (kStageBytes >> 4);
+#pragma unroll
+                    for (int ks = 0; ks < kBlk / 16; ++ks)
+                        mma_ts_elect(dO, aP + ks * 8, v_d + ((ks * 16 * 128) >> 4), idPV,
+                                     (accum || ks > 0) ? 1u : 0u);
+                    if constexpr (kTrain) {  // + P_lo V: the residual columns of the same buffer
 #pragma unroll
                         for (int ks = 0; ks < kBlk / 16; ++ks)
-                            mma_ts_lohi(dO, aP + ks * 8, v_lo + ((ks * 16 * 128) >> 4), dhi, idPV,
-                                        (accum || ks > 0) ? 1u : 0u);
-                        if constexpr (kTrain) {  // + P_lo V: the residual columns of the same buffer
-#pragma unroll
-                            for (int ks = 0; ks < kBlk / 16; ++ks)
-                                mma_ts_lohi(dO, aP + 32 + ks * 8, v_lo + ((ks * 16 * 128) >> 4), dhi,
-                                            idPV, 1u);
-                        }
-                        mma_commit(&bars.pv_done[x][k & 1]);
-                        mma_commit(empty_bar(e));
-                        accum = true;
-                        return true;
-                    };
-                    for (int b = 0; b < n && ok; ++b) {
-                        const uint32_t e = rc + b;
-                        const bool act = ((list_mask(lb)[b] >> (8 * x)) & 0xffu) != 0;
-                        while (ok && np > 0 && pe0 + kStages <= e) ok = flush_pv();
-                        if (ok && np == 2) ok = flush_pv();
-                        if (!ok) break;
-                        if (!(ok = wait_or_abort(full_bar(e), round_of(e), ctx, abort))) break;
-                        if (!act) {  // no token of this tile chose the block
-                            mbar_arrive(empty_bar(e));
-                            continue;
-                        }
-                        tc_fence_after();
-                        const uint32_t dS = tmem + kColS + x * 128 + (a & 1) * 64;
-                        const uint32_t k_lo = ring_lo + (e % kStages) * (kStageBytes >> 4);
-#pragma unroll
-                        for (int ks = 0; ks < kD / 16; ++ks)
-                            mma_ss_lohi(dS, q_lo + (((ks >> 2) * kHalfQ + (ks & 3) * 32) >> 4),
-                                        k_lo + (((ks >> 2) * kHalfBlk + (ks & 3) * 32) >> 4), dhi, idS,
-                                        ks > 0 ? 1u : 0u);
-                        mma_commit(&bars.s_full[x][a & 1]);
-                        if (np == 0) {
-                            pe0 = e;
-                            pk0 = a;
-                        } else {
-                            pe1 = e;
-                            pk1 = a;
-                        }
-                        ++np;
-                        ++a;
-                        if (np == 2) ok = flush_pv();
+                            mma_ts_elect(dO, aP + 32 + ks * 8, v_d + ((ks * 16 * 128) >> 4), idPV, 1u);
                     }
-                    mma_commit(&bars.q_empty);  // every S MMA reading this unit's Q is issued
-                    while (ok && np > 0) ok = flush_pv();
-                    rc += n;
+                    mma_commit_elect(&bars.pv_done[x][k & 1]);
+                    mma_commit_elect(empty_bar(e));
+                    accum = true;
+                    return true;
+                };
+                for (int b = 0; b < n && ok; ++b) {
+                    const uint32_t e = rc + b;
+                    const bool act = ((list_mask(lb)[b] >> (8 * x)) & 0xffu) != 0;
+                    while (ok && np > 0 && pe0 + kStages <= e) ok = flush_pv();
+                    if (ok && np == 2) ok = flush_pv();
+                    if (!ok) break;
+                    if (!(ok = wait_w(full_bar(e), round_of(e)))) break;
+                    if (!act) {  // no token of this tile chose the block
+                        mbar_arrive_elect(empty_bar(e));
+                        continue;
+                    }
+                    tc_fence_after();
+                    const uint32_t dS = tm + kColS + x * 128 + (a & 1) * 64;
+                    const uint64_t k_d = ring_d + (e % kStages) * (kStageBytes >> 4);
+#pragma unroll
+                    for (int ks = 0; ks < kD / 16; ++ks)
+                        mma_ss_elect(dS, q_d + (((ks >> 2) * kHalfQ + (ks & 3) * 32) >> 4),
+                                     k_d + (((ks >> 2) * kHalfBlk + (ks & 3) * 32) >> 4), idS,
+                                     ks > 0 ? 1u : 0u);
+                    mma_commit_elect(&bars.s_full[x][a & 1]);
+                    if (np == 0) {
+                        pe0 = e;
+                        pk0 = a;
+                    } else {
+                        pe1 = e;
+                        pk1 = a;
+                    }
+                    ++np;
+                    ++a;
+                    if (np == 2) ok = flush_pv();
                 }
-                mbar_arrive(&bars.list_empty[lb]);
+                mma_commit_elect(&bars.q_empty);  // every S MMA reading this unit's Q is issued
+                while (ok && np > 0) ok = flush_pv();
+                rc += n;
             }
-            mma_commit(&bars.fin[x]);
-            (void)mbar_wait(&bars.fin[x], 0, ctx);
+            mbar_arrive_elect(&bars.list_empty[lb]);
         }
+        mma_commit_elect(&bars.fin[x]);
+        (void)mbar_wait(&bars.fin[x], 0, ctx);
         __syncwarp();
     } else {
         // ---------------------------------------------------------------- softmax + epilogue
