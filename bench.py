@@ -68,12 +68,13 @@ def sparse_layer_flops(N: int) -> float:
 
 
 # DRAM traffic of the sparse prefill kernel (dram__bytes_read.sum + dram__bytes_write.sum) from one
-# ncu capture of the single-layer N = 131072 case, 2.319e9 bytes per launch, scaled by the tokens
+# ncu capture of the single-layer N = 131072 case, 2.317e9 bytes per launch, scaled by the tokens
 # processed to N = 262144 (Q reads, O writes and the K/V re-reads per 16-token unit all grow with N).
-# Valid only for the kernel source it was taken on: any change to it reports null.
-SPARSE_TRAFFIC = {"bytes_per_token": 2.316974848e9 / 131072,
-                  "sources": {"sparse_tc.cu": "4405ca3c032055be662e5ac02a49fd91f6a3ff7d78ca482c32d5fd612f22b580",
-                              "fastexp.cuh": "b6d9ae064f35b9fd752ec893180eaf72ade6f0495d57f5699832618f42784c06"}}
+# Valid only for the kernel sources it was taken on: any change to them reports null.
+SPARSE_TRAFFIC = {"bytes_per_token": 2.31670912e9 / 131072,
+                  "sources": {"sparse_tc.cu": "197c07812f3e1039106bc2a1e2262b5b5d9e92f6a70a88d57aae48dea8a1e9ce",
+                              "fastexp.cuh": "b6d9ae064f35b9fd752ec893180eaf72ade6f0495d57f5699832618f42784c06",
+                              "ptx.cuh": "4958f3527272a2b6168ae878bd0b9208adb2bddd1e7053b6eaae10a36fd1d5fb"}}
 
 
 def sparse_traffic(N: int):
