@@ -656,12 +656,17 @@ sala_status sala_sparse_backward(const void* q, const void* k, const void* v, co
                     "sparse_backward finish");
 }
 
-sala_status sala_sparse_decode(const void* q, const void* kcache, const void* vcache,
-                               const void* kbar, const int32_t* idx_in, int32_t* idx_out, void* o,
-                               int B, int H, int Hkv, int pos, int Tmax, int nb_cap, int d,
-                               int block, int topk, int n_init, int n_local, float scale,
-                               void* workspace, size_t workspace_bytes, sala_dtype dt,
-                               sala_stream stream) {
+}  // extern "C"
+
+// sala_sparse_decode, optionally zeroing the workspace's barrier counters on the stream once the
+// arguments have passed validation (the allocation-free entry point, whose callers cannot reach
+// its built-in area to clear them after a timed-out call).
+sala_status sala::sparse_decode_impl(const void* q, const void* kcache, const void* vcache,
+                                     const void* kbar, const int32_t* idx_in, int32_t* idx_out,
+                                     void* o, int B, int H, int Hkv, int pos, int Tmax, int nb_cap,
+                                     int d, int block, int topk, int n_init, int n_local,
+                                     float scale, void* workspace, size_t workspace_bytes,
+                                     sala_dtype dt, sala_stream stream, bool zero_barrier) {
     REQUIRE(pos >= 0 && pos < Tmax, SALA_ERR_INVALID_ARG, "pos %d outside the cache (Tmax %d)", pos, Tmax);
     sala_status s = check_select_args(B, H, Hkv, 1, pos, nb_cap, d, block, topk, n_init,
                                       n_local, dt);
@@ -680,6 +685,10 @@ sala_status sala_sparse_decode(const void* q, const void* kcache, const void* vc
     s = get_ctx(&ctx);
     if (s != SALA_OK) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (zero_barrier) {
+        const cudaError_t e = cudaMemsetAsync(workspace, 0, 256, st);
+        if (e != cudaSuccess) return launched(e, "sparse_decode barrier reset");
+    }
     {
         const cudaError_t e = sala::launch_sparse_decode_fused(
             to_dt(dt), q, kcache, vcache, kbar, idx_in, idx_out, o, B, H, Hkv, pos, Tmax, nb_cap, d,
@@ -712,6 +721,19 @@ sala_status sala_sparse_decode(const void* q, const void* kcache, const void* vc
                                                     Hkv, pos, Tmax, d, slots, scale, ws_attn, st,
                                                     ctx),
                     "sparse_decode");
+}
+
+extern "C" {
+
+sala_status sala_sparse_decode(const void* q, const void* kcache, const void* vcache,
+                               const void* kbar, const int32_t* idx_in, int32_t* idx_out, void* o,
+                               int B, int H, int Hkv, int pos, int Tmax, int nb_cap, int d,
+                               int block, int topk, int n_init, int n_local, float scale,
+                               void* workspace, size_t workspace_bytes, sala_dtype dt,
+                               sala_stream stream) {
+    return sala::sparse_decode_impl(q, kcache, vcache, kbar, idx_in, idx_out, o, B, H, Hkv, pos,
+                                    Tmax, nb_cap, d, block, topk, n_init, n_local, scale,
+                                    workspace, workspace_bytes, dt, stream, false);
 }
 
 size_t sala_sparse_decode_paged_workspace(int B, int H, int Hkv, int max_pos, int block, int topk,

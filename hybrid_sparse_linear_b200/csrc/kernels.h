@@ -6,6 +6,7 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "../../include/sala.h"
 #include "common.cuh"
 
 namespace sala {
@@ -161,5 +162,14 @@ cudaError_t launch_selftest_wait(cudaStream_t st, DevCtx ctx);
 
 // Sets the calling thread's sala_last_error() message (printf-style).
 void set_last_error(const char* fmt, ...);
+
+// Body of sala_sparse_decode; zero_barrier additionally zeroes the workspace's first 256 bytes on
+// the stream after validation, before the kernels.
+sala_status sparse_decode_impl(const void* q, const void* kcache, const void* vcache,
+                               const void* kbar, const int32_t* idx_in, int32_t* idx_out, void* o,
+                               int B, int H, int Hkv, int pos, int Tmax, int nb_cap, int d,
+                               int block, int topk, int n_init, int n_local, float scale,
+                               void* workspace, size_t workspace_bytes, sala_dtype dt,
+                               sala_stream stream, bool zero_barrier);
 
 }  // namespace sala

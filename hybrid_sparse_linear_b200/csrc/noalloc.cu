@@ -13,9 +13,12 @@
 // until the process exits.  All calls on a GPU share it, so two calls that may run at the same
 // time on that GPU (different streams, no ordering between them) race on it and must not be made.
 // The area keeps whatever the previous call left there.  Its first 256 bytes are the counters of
-// the one-launch path's grid barrier: zero when the library loads (a __device__ array starts
-// zeroed) and put back to zero by every call that completes; every other byte a call reads it has
-// written earlier in the same call.
+// the one-launch path's grid barrier, which must read zero when a call starts.  A call that gave
+// up on a wait (SALA_ERR_TIMEOUT) can leave them nonzero, and no caller can reach the area to
+// clear them, so every call, once its arguments have passed validation, first zeroes those 256 bytes on its
+// own stream (cudaMemsetAsync, which allocates nothing): each call starts from clean counters
+// whatever the previous call did.  Every
+// other byte a call reads it has written earlier in the same call.
 #include <mutex>
 
 #include "../../include/sala.h"
@@ -81,7 +84,7 @@ extern "C" sala_status sala_sparse_decode_noalloc(const void* q, const void* kca
     void* scratch = nullptr;
     sala_status s = scratch_on_current_device(&scratch);
     if (s != SALA_OK) return s;
-    return sala_sparse_decode(q, kcache, vcache, kbar, idx_in, idx_out, o, B, H, Hkv, pos, Tmax,
-                              nb_cap, d, block, topk, n_init, n_local, scale, scratch,
-                              kNoallocScratchBytes, dt, stream);
+    return sala::sparse_decode_impl(q, kcache, vcache, kbar, idx_in, idx_out, o, B, H, Hkv, pos,
+                                    Tmax, nb_cap, d, block, topk, n_init, n_local, scale, scratch,
+                                    kNoallocScratchBytes, dt, stream, /*zero_barrier=*/true);
 }

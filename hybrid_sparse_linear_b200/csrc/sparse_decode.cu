@@ -729,20 +729,32 @@ cudaError_t fused(const void* q, const void* kc, const void* vc, const void* kba
         return cudaErrorNotSupported;
     auto kern = sparse_decode_fused_kernel<T, D>;
     const int smem = (int)sizeof(DecSmem<D>);
+    // resident CTAs per SM and SM count, per device (a process may drive several GPUs from
+    // several threads); read into locals under the lock
+    constexpr int kMaxDev = 64;
     static std::mutex mu;
-    static int occ_dev = -1, occ = 0, nsm = 0;
+    static int occ_of[kMaxDev] = {}, nsm_of[kMaxDev] = {};
+    int occ = 0, nsm = 0;
     {
-        std::lock_guard<std::mutex> lk(mu);
         int dev = 0;
-        cudaGetDevice(&dev);
-        if (occ_dev != dev) {
-            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e != cudaSuccess) return e;
+        if (dev < 0 || dev >= kMaxDev) return cudaErrorNotSupported;
+        std::lock_guard<std::mutex> lk(mu);
+        if (occ_of[dev] == 0) {
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
             if (e != cudaSuccess) return e;
-            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kThreads, smem);
+            int o = 0, n = 0;
+            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, kern, kThreads, smem);
             if (e != cudaSuccess) return e;
-            cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-            occ_dev = dev;
+            e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+            if (e != cudaSuccess) return e;
+            if (o < 1) return cudaErrorNotSupported;
+            occ_of[dev] = o;
+            nsm_of[dev] = n;
         }
+        occ = occ_of[dev];
+        nsm = nsm_of[dev];
     }
     const int groups = B * Hkv;
     const int cap = occ * nsm / groups;

@@ -93,8 +93,11 @@ sala_status sala_linear_prefill_ws(const void* q, const void* k, const void* v, 
                                    size_t workspace_bytes, sala_dtype dt, sala_stream stream);
 size_t sala_linear_prefill_workspace(int B, int H, int N, int d, sala_dtype dt);
 
-/* One decode step of the linear attention for every (batch, head): the state is updated first
- * and then read, so the current token attends to itself with lambda^0:
+/* One decode step of the linear attention for every (batch, head).  Pages: the linear layers keep
+ * O(1) memory per token through a recursive form (DE technical summary section 2, "recursive
+ * formulations"; JA technical summary section 2.1, linear attention at O(N) compute and memory);
+ * this is that recursion for one new token.  The state is updated first and then read, so the
+ * current token attends to itself with lambda^0:
  *   S <- lambda_h S + k^T v ;  o = q S
  * q, k, v, o : [B, H, d] device, dt.   state : [B, H, d, d] fp32 device, updated in place.
  */
@@ -211,8 +214,11 @@ sala_status sala_block_compress(const void* k, void* kbar, int B, int Hkv, int N
                                 sala_dtype dt, sala_stream stream);
 
 /* ------------------------------------------------------------------------------------------
- * Block selection (scoring + top-k).  Query row r sits at absolute position p = q_pos0 + r in
- * block c = p / block.  For KV group g:
+ * Block selection (scoring + top-k).  Pages: InfLLM-V2 picks, for each query, the context parts
+ * that matter, with no extra parameters (JA technical summary section 2.1 "hybrid attention";
+ * abstract on fugumt.com: sparse attention for local detail and key information); the scoring
+ * and the forced init/local blocks are the plain reading of that selection step.  Query row r
+ * sits at absolute position p = q_pos0 + r in block c = p / block.  For KV group g:
  *   forced     F = {0 .. n_init-1} U {max(0, c-n_local+1) .. c}          (init + local blocks)
  *   candidates   = {n_init .. c-n_local}                                 (complete, past)
  *   score(j)     = (sum over the group's query heads of q[b, h, r]) . kbar[b, g, j]
@@ -327,7 +333,12 @@ sala_status sala_sparse_backward(const void* q, const void* k, const void* v, co
 
 /* ------------------------------------------------------------------------------------------
  * Sparse attention decode: one query token per (batch, head) at absolute position pos, over
- * a dense KV cache that holds rows 0 .. pos (capacity Tmax rows).
+ * a dense KV cache that holds rows 0 .. pos (capacity Tmax rows).  Pages: the sparse layers keep
+ * the whole KV cache and compute on the selected parts only (JA technical summary section 1,
+ * "sparse compute, dense storage"), and the model decodes with contexts up to 1M tokens on one
+ * GPU (JA technical summary section 4.3; fugumt.com abstract).  The step is block selection as
+ * in sala_block_topk for the one query row, then sala_sparse_prefill's softmax over the chosen
+ * blocks.
  *
  * q, o          : [B, H, d] device, dt.
  * kcache, vcache: [B, Hkv, Tmax, d] device, dt.
@@ -402,10 +413,10 @@ size_t sala_sparse_decode_paged_workspace(int B, int H, int Hkv, int max_pos, in
  *     that GPU current) and caches it; make that first call before any stream capture.
  *   - All calls on a GPU share the one area: calls that can run concurrently on the same GPU
  *     race on it and must not be made.  The area keeps the previous call's contents.  Its first
- *     256 bytes are the barrier counters described under sala_sparse_decode: zero when the
- *     library loads and left zero by every call that completes (a call that reported
- *     SALA_ERR_TIMEOUT may leave them nonzero, after which later calls also time out instead of
- *     completing); nothing else in it needs a starting value.
+ *     256 bytes are the barrier counters described under sala_sparse_decode; every call zeroes
+ *     them on `stream` before its kernels run (a memset, which allocates nothing), so each call
+ *     starts from clean counters and a call that reported SALA_ERR_TIMEOUT does not affect the
+ *     calls after it.  Nothing else in the area needs a starting value.
  * Other arguments, validation and errors are those of sala_sparse_decode. */
 sala_status sala_sparse_decode_noalloc(const void* q, const void* kcache, const void* vcache,
                                        const void* kbar, const int32_t* idx_in, int32_t* idx_out,

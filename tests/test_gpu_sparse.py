@@ -89,7 +89,8 @@ def test_bf16_selection_weak_pilot(sala, topk):
     kbar = sala.block_compress(layer.k.cuda())
     idx = sala.block_topk(q.cuda(), kbar, topk, 1, 2)
     sala.check_status()
-    kbar_ref = _f64(kbar)
+    kbar_ref = oracle.block_compress(_f64(layer.k), 64, round_to_bf16=True)
+    np.testing.assert_array_equal(_f64(kbar), kbar_ref)
     idx_ref, kth = oracle.block_select(_f64(q), kbar_ref, 64, topk, 1, 2)
     check_selection(idx.cpu().numpy(), idx_ref, _f64(q), kbar_ref, kth, topk, 1, 2)
 
@@ -143,6 +144,7 @@ def _decode_case(sala, T, topk, n_init, n_local, dtype, layer_id, given_idx=Fals
     kbar_ref = oracle.block_compress(_f64(layer.k), 64, round_to_bf16=(kind == "bf16"))
     if kind == "f32":
         kbar_ref = kbar_ref.astype(np.float32).astype(np.float64)
+    np.testing.assert_array_equal(_f64(kbar)[:, :, :kbar_ref.shape[2]], kbar_ref)
     idx_ref, kth = oracle.block_select(q64, kbar_ref, 64, topk, n_init, n_local, q_pos0=pos)
     idx_in = torch.from_numpy(idx_ref[:, :, 0]).cuda() if given_idx else None
     o = sala.sparse_decode(qd, kc, vc, kbar, pos, topk, n_init, n_local, idx_in=idx_in,
@@ -327,6 +329,7 @@ def test_qblock_pipeline(sala):
     sala.check_status()
     q64, k64, v64 = _f64(layer.q), _f64(layer.k), _f64(layer.v)
     kbar_ref = oracle.block_compress(k64, 64, round_to_bf16=True)
+    np.testing.assert_array_equal(_f64(kbar), kbar_ref)
     ref, kth = oracle.block_select_qblock(q64, kbar_ref, 64, topk, 1, 2)
     got = idx.cpu().numpy()
     check_selection(got, ref, oracle.qblock_sum(q64, 64), kbar_ref, kth, topk, 1, 2)
@@ -372,7 +375,10 @@ def test_qblock_softmax_selection(sala, N, topk, dtype, d, H, Hkv):
     kbar = sala.block_compress(k)
     idx = sala.block_topk_qblock_softmax(q, kbar, topk, 1, 2)
     sala.check_status()
-    kbar_ref = _f64(kbar)
+    kbar_ref = oracle.block_compress(_f64(layer.k), 64, round_to_bf16=(kind == "bf16"))
+    if kind == "f32":
+        kbar_ref = kbar_ref.astype(np.float32).astype(np.float64)
+    np.testing.assert_array_equal(_f64(kbar), kbar_ref)
     q64 = _f64(layer.q)
     ref, kth = oracle.block_select_qblock_softmax(q64, kbar_ref, 64, topk, 1, 2)
     _check_softmax_selection(idx.cpu().numpy(), ref, kth, q64, kbar_ref, topk, 1, 2)
@@ -388,7 +394,9 @@ def test_qblock_softmax_pipeline(sala):
     o = sala.sparse_prefill(q, k, v, idx)
     sala.check_status()
     q64, k64, v64 = _f64(layer.q), _f64(layer.k), _f64(layer.v)
-    ref, kth = oracle.block_select_qblock_softmax(q64, _f64(kbar), 64, topk, 1, 2)
+    kbar_ref = oracle.block_compress(k64, 64, round_to_bf16=True)
+    np.testing.assert_array_equal(_f64(kbar), kbar_ref)
+    ref, kth = oracle.block_select_qblock_softmax(q64, kbar_ref, 64, topk, 1, 2)
     got = idx.cpu().numpy()
-    _check_softmax_selection(got, ref, kth, q64, _f64(kbar), topk, 1, 2)
+    _check_softmax_selection(got, ref, kth, q64, kbar_ref, topk, 1, 2)
     assert_close(_f64(o), oracle.sparse_attention(q64, k64, v64, got, 64), "bf16", "o")

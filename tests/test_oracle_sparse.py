@@ -118,6 +118,56 @@ def test_selection_properties(G, topk, n_init, n_local):
     _check_selection_properties(q, kbar, idx, T, topk, n_init, n_local)
 
 
+def test_block_scores_at_matches_group_summed_products():
+    # The near-tie rule of the GPU parity tests judges differing blocks by these scores, so the
+    # scorer is pinned on its own: every (b, g, r, block) quadruple against a numpy einsum of the
+    # group-summed query with the block key.  Shapes are chosen with B, Hkv, Nq and nb pairwise
+    # different so that a swapped quadruple field (g <-> r, b <-> g) indexes a different value.
+    rng = np.random.default_rng(77)
+    B, Hkv, G, Nq, nb, d = 2, 3, 4, 5, 7, 6
+    q = rng.standard_normal((B, Hkv * G, Nq, d))
+    kbar = rng.standard_normal((B, Hkv, nb, d))
+    quads = np.array([(b, g, r, j) for b in range(B) for g in range(Hkv) for r in range(Nq)
+                      for j in range(nb)], dtype=np.int64)
+    rng.shuffle(quads)
+    got = oracle.block_scores_at(q, kbar, quads)
+    qs = q.reshape(B, Hkv, G, Nq, d).sum(axis=2)
+    full = np.einsum("bgnd,bgkd->bgnk", qs, kbar)
+    want = full[quads[:, 0], quads[:, 1], quads[:, 2], quads[:, 3]]
+    np.testing.assert_allclose(got, want, rtol=1e-13, atol=1e-13)
+    # the block_select k-th score is one of these scores
+    # (block size 1, rows at positions 2..6: row r has candidates 1 .. r + 1, n_local 1)
+    idx, kth = oracle.block_select(q, kbar, 1, 2, 1, 1, q_pos0=2)
+    for b in range(B):
+        for g in range(Hkv):
+            for r in range(Nq):
+                c = 2 + r
+                chosen = [x for x in idx[b, g, r] if 1 <= x <= c - 1]
+                if c - 1 < 2:
+                    assert kth[b, g, r] == -np.inf
+                    continue
+                s = oracle.block_scores_at(q, kbar, np.array([(b, g, r, x) for x in chosen]))
+                assert len(chosen) == 2 and kth[b, g, r] == s.min()
+
+
+def test_block_scores_at_hand_case():
+    # two KV groups of two heads, d = 2, worked by hand:
+    #   group 1, row 1: q heads 2, 3 = (1, 2) and (3, -1) -> sum (4, 1); block 2 key (0.5, 2)
+    #   score = 4 * 0.5 + 1 * 2 = 4
+    q = np.zeros((1, 4, 2, 2))
+    q[0, 2, 1] = (1.0, 2.0)
+    q[0, 3, 1] = (3.0, -1.0)
+    q[0, 0, 1] = (100.0, 100.0)   # group 0, same row: must not enter group 1's score
+    q[0, 2, 0] = (-50.0, 7.0)     # group 1, other row
+    kbar = np.zeros((1, 2, 3, 2))
+    kbar[0, 1, 2] = (0.5, 2.0)
+    kbar[0, 0, 2] = (9.0, 9.0)
+    kbar[0, 1, 1] = (-3.0, 1.0)
+    s = oracle.block_scores_at(q, kbar, np.array([(0, 1, 1, 2), (0, 1, 1, 1), (0, 0, 1, 2),
+                                                  (0, 1, 0, 2)]))
+    assert list(s) == [4.0, 4 * -3.0 + 1 * 1.0, 100 * 9.0 + 100 * 9.0, -50 * 0.5 + 7 * 2.0]
+
+
 def test_selection_with_query_offset():
     rng = np.random.default_rng(31)
     B, H, Hkv, T, d = 1, 4, 2, 4, 5

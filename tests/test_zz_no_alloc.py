@@ -63,6 +63,46 @@ def test_noalloc_matches_workspace_version_twice(T):
                      f"no-alloc call {call}")
 
 
+def test_noalloc_recovers_after_a_timed_out_call():
+    # The built-in area carries the grid barrier's counters from call to call, and no caller can
+    # reach it to clear them.  Make one call give up on its waits (a 1 ns wait limit: every CTA
+    # but the last to arrive stops waiting at once, records SALA_ERR_TIMEOUT and returns; nothing
+    # faults), then check that the next call with the normal limit gives exactly the result of
+    # sala_sparse_decode with its own workspace.
+    from hybrid_sparse_linear_b200 import sala, synth
+    lib = _lib()
+    lib.sala_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+    lib.sala_check_status.argtypes = [ctypes.c_void_p]
+    lib.sala_check_status.restype = ctypes.c_int
+    T, topk, n_init, n_local, H, Hkv, d = 1 << 20, 64, 1, 2, 32, 2, 128
+    slots = n_init + n_local + topk
+    layer = synth.sparse_layer(1, H, Hkv, T, d, torch.bfloat16, "cuda", layer=12, q_rows=1)
+    kbar = sala.block_compress(layer.k)
+    q = layer.q[:, :, 0].contiguous()
+    idx_ref = torch.empty((1, Hkv, slots), dtype=torch.int32, device="cuda")
+    o_ref = sala.sparse_decode(q, layer.k, layer.v, kbar, T - 1, topk, n_init, n_local,
+                               idx_out=idx_ref)
+    sala.check_status()
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    o = torch.empty_like(o_ref)
+    idx = torch.empty_like(idx_ref)
+    lib.sala_set_wait_limit_ns(1)
+    try:
+        r = _call(lib, q, layer.k, layer.v, kbar, idx, o, T - 1, topk, n_init, n_local)
+        assert r == 0, lib.sala_last_error()
+        assert lib.sala_check_status(stream) == 4  # SALA_ERR_TIMEOUT
+    finally:
+        lib.sala_set_wait_limit_ns(2_000_000_000)
+    for call in range(2):
+        o = torch.full_like(o_ref, float("nan"))
+        idx = torch.full_like(idx_ref, -7)
+        r = _call(lib, q, layer.k, layer.v, kbar, idx, o, T - 1, topk, n_init, n_local)
+        assert r == 0, lib.sala_last_error()
+        assert lib.sala_check_status(stream) == 0, f"call {call} after the timeout did not complete"
+        assert torch.equal(idx, idx_ref), f"call {call} after the timeout: selection differs"
+        assert torch.equal(o, o_ref), f"call {call} after the timeout: output differs"
+
+
 def test_noalloc_refuses_oversized_problem():
     lib = _lib()
     vp = ctypes.c_void_p
