@@ -539,14 +539,15 @@ def run_decode(sala, synth, torch, steps, warmup, stream, T=DECODE_T):
     flush = torch.empty(512 << 20, device=dev, dtype=torch.uint8)
     torch.cuda.synchronize()
 
-    # Linear layers launch as programmatic dependents of the kernel before them (each reads its
-    # own state while the previous layer finishes); the token is also timed without that.
+    # Every layer launches as a programmatic dependent of the kernel before it (a linear layer
+    # reads its own state, a sparse layer its share of k_bar, while the previous layer finishes);
+    # the token is also timed without that.
     def one_token(pdl=True):
         for l in range(N_LAYERS):
             if l in SPARSE_LAYERS:
                 q, kc, vc, kbar = sp[SPARSE_LAYERS.index(l)]
                 sala.sparse_decode(q, kc, vc, kbar, pos, TOPK, N_INIT, N_LOCAL, o=o, workspace=ws,
-                                   stream=stream)
+                                   stream=stream, pdl=pdl)
             else:
                 S, q, k, v = lin[l - sum(1 for s in SPARSE_LAYERS if s < l)]
                 sala.linear_decode(q, k, v, lam, S, o=o, stream=stream, pdl=pdl)
@@ -592,7 +593,7 @@ def run_decode(sala, synth, torch, steps, warmup, stream, T=DECODE_T):
                     if kind == "sparse":
                         q, kc, vc, kbar = sp[SPARSE_LAYERS.index(l)]
                         sala.sparse_decode(q, kc, vc, kbar, pos, TOPK, N_INIT, N_LOCAL, o=o,
-                                           workspace=ws, stream=stream)
+                                           workspace=ws, stream=stream, pdl=True)
                     else:
                         S, q, k, v = lin[l - sum(1 for s in SPARSE_LAYERS if s < l)]
                         sala.linear_decode(q, k, v, lam, S, o=o, stream=stream, pdl=True)
@@ -960,10 +961,10 @@ def main():
                           "us_per_sparse_layer": dec["us_per_sparse_layer"],
                           "us_per_token_without_pdl": dec["us_per_token_without_pdl"],
                           "timing": "CUDA events around one CUDA-graph replay of a token's 32 layer "
-                                    "calls, L2 flushed before each token, median; linear layers "
-                                    "launched as programmatic dependents (state read overlapping "
-                                    "the previous layer); per-layer figures from graphs of one kind "
-                                    "of call only"}
+                                    "calls, L2 flushed before each token, median; every layer "
+                                    "launched as a programmatic dependent (linear state and sparse "
+                                    "k_bar reads overlapping the previous layer); per-layer figures "
+                                    "from graphs of one kind of call only"}
     if "e2e" in phases:
         e = run_e2e(sala, synth, torch, max(1, min(args.steps, 2)), 1)
         line["e2e"] = {"value": ws * N_TOK / (max_over_ranks(e["ms_per_step"], "cuda") / 1000.0),

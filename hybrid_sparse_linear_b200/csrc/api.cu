@@ -543,19 +543,25 @@ sala_status sala_sparse_prefill(const void* q, const void* k, const void* v, con
                     "sparse_prefill");
 }
 
+// Sparse decode workspace: [0, 256) the cooperative one-launch path's barrier words and [256, 512)
+// the prefetching one-launch path's epoch word, in every layout; from 512 on, the data of whichever
+// path a call takes (the prefetching path's tagged words may share bytes with the other paths'
+// data: no value those store looks like a tag).
 size_t sala_sparse_decode_workspace(int B, int H, int Hkv, int pos, int block, int topk,
                                     int n_init, int n_local, int d) {
     if (B <= 0 || H <= 0 || Hkv <= 0 || pos < 0 || block <= 0) return 0;
     const int slots = n_init + n_local + topk;
-    size_t a = sala::sparse_decode_attn_workspace(B, H, Hkv, slots, d);
-    size_t sel = sala::rowwise_topk_workspace(B, Hkv, 1, pos, topk);
-    size_t idx_bytes = (size_t)B * Hkv * slots * sizeof(int32_t);
     auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
-    // [0, 256) holds the one-launch path's barrier words in every layout.
-    const size_t multi = 256 + up(a) + up(sel) + up(idx_bytes);
+    const size_t multi = 512 + up(sala::sparse_decode_attn_workspace(B, H, Hkv, slots, d)) +
+                         up(sala::rowwise_topk_workspace(B, Hkv, 1, pos, topk)) +
+                         up((size_t)B * Hkv * slots * sizeof(int32_t));
     const size_t fused = up(sala::sparse_decode_fused_workspace(B, H, Hkv, pos, topk, n_init, n_local, d));
-    return multi > fused ? multi : fused;
+    const size_t pf = 512 + sala::sparse_decode_pf_workspace(B, H, Hkv, pos, topk, n_init, n_local, d);
+    const size_t m = multi > fused ? multi : fused;
+    return m > pf ? m : pf;
 }
+
+
 
 // Forward with the row statistic the backward needs (bf16, d 128, 16 query heads per KV head).
 sala_status sala_sparse_prefill_lse(const void* q, const void* k, const void* v,
@@ -666,7 +672,8 @@ sala_status sala::sparse_decode_impl(const void* q, const void* kcache, const vo
                                      void* o, int B, int H, int Hkv, int pos, int Tmax, int nb_cap,
                                      int d, int block, int topk, int n_init, int n_local,
                                      float scale, void* workspace, size_t workspace_bytes,
-                                     sala_dtype dt, sala_stream stream, bool zero_barrier) {
+                                     sala_dtype dt, sala_stream stream, bool zero_barrier,
+                                     bool pdl) {
     REQUIRE(pos >= 0 && pos < Tmax, SALA_ERR_INVALID_ARG, "pos %d outside the cache (Tmax %d)", pos, Tmax);
     sala_status s = check_select_args(B, H, Hkv, 1, pos, nb_cap, d, block, topk, n_init,
                                       n_local, dt);
@@ -690,6 +697,14 @@ sala_status sala::sparse_decode_impl(const void* q, const void* kcache, const vo
         if (e != cudaSuccess) return launched(e, "sparse_decode barrier reset");
     }
     {
+        const size_t base = 512;
+        const cudaError_t e = sala::launch_sparse_decode_pf(
+            to_dt(dt), q, kcache, vcache, kbar, idx_in, idx_out, o, B, H, Hkv, pos, Tmax, nb_cap, d,
+            topk, n_init, n_local, scale, static_cast<unsigned*>(static_cast<void*>(static_cast<char*>(workspace) + 256)),
+            static_cast<char*>(workspace) + base, workspace_bytes - base, pdl, st, ctx);
+        if (e != cudaErrorNotSupported) return launched(e, "sparse_decode");
+    }
+    {
         const cudaError_t e = sala::launch_sparse_decode_fused(
             to_dt(dt), q, kcache, vcache, kbar, idx_in, idx_out, o, B, H, Hkv, pos, Tmax, nb_cap, d,
             topk, n_init, n_local, scale, workspace, workspace_bytes,
@@ -698,7 +713,7 @@ sala_status sala::sparse_decode_impl(const void* q, const void* kcache, const vo
     }
     const int slots = n_init + n_local + topk;
     auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
-    char* w = static_cast<char*>(workspace) + 256;  // [0, 256): the one-launch path's barrier words
+    char* w = static_cast<char*>(workspace) + 512;  // [0, 512): the one-launch paths' words
     void* ws_attn = w;
     w += up(sala::sparse_decode_attn_workspace(B, H, Hkv, slots, d));
     void* ws_sel = w;
@@ -733,7 +748,18 @@ sala_status sala_sparse_decode(const void* q, const void* kcache, const void* vc
                                sala_stream stream) {
     return sala::sparse_decode_impl(q, kcache, vcache, kbar, idx_in, idx_out, o, B, H, Hkv, pos,
                                     Tmax, nb_cap, d, block, topk, n_init, n_local, scale,
-                                    workspace, workspace_bytes, dt, stream, false);
+                                    workspace, workspace_bytes, dt, stream, false, false);
+}
+
+sala_status sala_sparse_decode_pdl(const void* q, const void* kcache, const void* vcache,
+                                   const void* kbar, const int32_t* idx_in, int32_t* idx_out,
+                                   void* o, int B, int H, int Hkv, int pos, int Tmax, int nb_cap,
+                                   int d, int block, int topk, int n_init, int n_local, float scale,
+                                   void* workspace, size_t workspace_bytes, sala_dtype dt,
+                                   sala_stream stream) {
+    return sala::sparse_decode_impl(q, kcache, vcache, kbar, idx_in, idx_out, o, B, H, Hkv, pos,
+                                    Tmax, nb_cap, d, block, topk, n_init, n_local, scale,
+                                    workspace, workspace_bytes, dt, stream, false, true);
 }
 
 size_t sala_sparse_decode_paged_workspace(int B, int H, int Hkv, int max_pos, int block, int topk,

@@ -138,6 +138,23 @@ cudaError_t launch_sparse_decode_fused(DType dt, const void* q, const void* kc, 
                                        int nb_cap, int d, int topk, int n_init, int n_local,
                                        float scale, void* ws, size_t ws_bytes, DecodePaging pg, cudaStream_t st,
                                        DevCtx ctx);
+// Sparse decode in one launch with k_bar prefetched into shared memory (bf16, d 64 or 128, dense
+// cache, one position): each CTA scores its share of the rows out of shared memory, ranks its own
+// best keys among the group's published ones and attends the blocks it wins.  pdl: launched as a
+// programmatic dependent of the previous kernel (k_bar is read before that kernel completes).
+// Returns cudaErrorNotSupported, launching nothing, when the problem does not fit it (k > 64, more
+// than 80 slots, more than 16 heads per group, more than 64 groups, a CTA's share of k_bar above
+// its shared-memory rows, or a smaller workspace).  epoch: a word that stays at one place for every
+// call on the same workspace; ws: the path's own region of tagged words (both zero before the
+// first call).
+size_t sparse_decode_pf_workspace(int B, int H, int Hkv, int pos, int topk, int n_init, int n_local,
+                                  int d);
+cudaError_t launch_sparse_decode_pf(DType dt, const void* q, const void* kc, const void* vc,
+                                    const void* kbar, const int32_t* idx_in, int32_t* idx_out,
+                                    void* o, int B, int H, int Hkv, int pos, int Tmax, int nb_cap,
+                                    int d, int topk, int n_init, int n_local, float scale,
+                                    unsigned* epoch, void* ws, size_t ws_bytes, bool pdl,
+                                    cudaStream_t st, DevCtx ctx);
 cudaError_t launch_sparse_decode_attn(DType dt, const void* q, const void* kc, const void* vc,
                                       const int32_t* idx, void* o, int B, int H, int Hkv,
                                       int pos, int Tmax, int d, int slots, float scale, void* ws,
@@ -164,12 +181,13 @@ cudaError_t launch_selftest_wait(cudaStream_t st, DevCtx ctx);
 void set_last_error(const char* fmt, ...);
 
 // Body of sala_sparse_decode; zero_barrier additionally zeroes the workspace's first 256 bytes on
-// the stream after validation, before the kernels.
+// the stream after validation, before the kernels; pdl launches the prefetching one-launch kernel
+// as a programmatic dependent of the previous kernel (other paths launch as usual).
 sala_status sparse_decode_impl(const void* q, const void* kcache, const void* vcache,
                                const void* kbar, const int32_t* idx_in, int32_t* idx_out, void* o,
                                int B, int H, int Hkv, int pos, int Tmax, int nb_cap, int d,
                                int block, int topk, int n_init, int n_local, float scale,
                                void* workspace, size_t workspace_bytes, sala_dtype dt,
-                               sala_stream stream, bool zero_barrier);
+                               sala_stream stream, bool zero_barrier, bool pdl);
 
 }  // namespace sala

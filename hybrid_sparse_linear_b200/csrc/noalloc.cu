@@ -86,5 +86,6 @@ extern "C" sala_status sala_sparse_decode_noalloc(const void* q, const void* kca
     if (s != SALA_OK) return s;
     return sala::sparse_decode_impl(q, kcache, vcache, kbar, idx_in, idx_out, o, B, H, Hkv, pos,
                                     Tmax, nb_cap, d, block, topk, n_init, n_local, scale, scratch,
-                                    kNoallocScratchBytes, dt, stream, /*zero_barrier=*/true);
+                                    kNoallocScratchBytes, dt, stream, /*zero_barrier=*/true,
+                                    /*pdl=*/false);
 }

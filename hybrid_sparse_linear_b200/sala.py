@@ -53,6 +53,7 @@ _lib.sala_sparse_prefill.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i
                                      ctypes.c_float, _i, _vp]
 _lib.sala_sparse_decode.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i,
                                     _i, _i, _i, _i, ctypes.c_float, _vp, _st, _i, _vp]
+_lib.sala_sparse_decode_pdl.argtypes = _lib.sala_sparse_decode.argtypes
 _lib.sala_sparse_decode_workspace.argtypes = [_i, _i, _i, _i, _i, _i, _i, _i, _i]
 _lib.sala_sparse_decode_workspace.restype = _st
 _lib.sala_sparse_decode_paged.argtypes = [_vp, _vp, _vp, _i, _vp, _i, _vp, _i, _vp, _i, _vp, _vp,
@@ -76,7 +77,7 @@ for _f in ("sala_linear_prefill", "sala_linear_decode", "sala_linear_prefill_rop
            "sala_block_topk_qblock_softmax", "sala_linear_decode_pdl", "sala_qk_prologue",
            "sala_block_compress",
            "sala_block_topk",
-           "sala_sparse_prefill", "sala_sparse_decode", "sala_check_status",
+           "sala_sparse_prefill", "sala_sparse_decode", "sala_sparse_decode_pdl", "sala_check_status",
            "sala_selftest_wait_timeout"):
     getattr(_lib, _f).restype = _i
 
@@ -389,8 +390,10 @@ def sparse_decode_workspace_bytes(B, H, Hkv, pos, topk, n_init, n_local, d, bloc
 
 
 def sparse_decode(q, kcache, vcache, kbar, pos, topk, n_init=1, n_local=2, idx_in=None,
-                  idx_out=None, o=None, block=64, scale=0.0, workspace=None, stream=None):
-    """One query token per head at position pos over a dense KV cache.  q: [B,H,d]."""
+                  idx_out=None, o=None, block=64, scale=0.0, workspace=None, stream=None, pdl=False):
+    """One query token per head at position pos over a dense KV cache.  q: [B,H,d].
+    pdl=True launches it as a programmatic dependent of the previous kernel in the stream
+    (sala_sparse_decode_pdl: k_bar is read while that kernel finishes, so it must not write it)."""
     B, H, d = q.shape
     Hkv, Tmax = kcache.shape[1], kcache.shape[2]
     _need(q, "q"); _need(kcache, "kcache", dtype=q.dtype); _need(vcache, "vcache", kcache.shape, q.dtype)
@@ -404,11 +407,11 @@ def sparse_decode(q, kcache, vcache, kbar, pos, topk, n_init=1, n_local=2, idx_i
     need = sparse_decode_workspace_bytes(B, H, Hkv, pos, topk, n_init, n_local, d, block)
     if workspace is None:  # zero-filled: its first words are counters that must start at zero
         workspace = torch.zeros(max(need, 256), device=q.device, dtype=torch.uint8)
-    _check(_lib.sala_sparse_decode(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(kbar), _ptr(idx_in),
-                                   _ptr(idx_out), _ptr(o), B, H, Hkv, pos, Tmax, kbar.shape[2], d,
-                                   block, topk, n_init, n_local, float(scale), _ptr(workspace),
-                                   workspace.numel(), _dt(q), _stream(stream)),
-           "sala_sparse_decode")
+    fn = _lib.sala_sparse_decode_pdl if pdl else _lib.sala_sparse_decode
+    _check(fn(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(kbar), _ptr(idx_in), _ptr(idx_out),
+              _ptr(o), B, H, Hkv, pos, Tmax, kbar.shape[2], d, block, topk, n_init, n_local,
+              float(scale), _ptr(workspace), workspace.numel(), _dt(q), _stream(stream)),
+           "sala_sparse_decode_pdl" if pdl else "sala_sparse_decode")
     return o
 
 

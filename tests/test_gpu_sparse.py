@@ -214,6 +214,147 @@ def test_sparse_decode_workspace_reused_across_calls_and_shapes(sala):
                 assert torch.equal(o, first[0]) and torch.equal(idx, first[1])
 
 
+def test_sparse_decode_bf16_d64_four_heads_per_group(sala):
+    # bf16 d = 64 with G = 4: the prefetching one-launch kernel with padding heads in its tiles
+    _decode_case(sala, 64 * 900 + 33, 32, 1, 2, torch.bfloat16, 14, H=8, Hkv=2, d=64)
+
+
+def test_sparse_decode_bf16_given_idx(sala):
+    # a given selection: the one-launch kernel attends slots j, j + cpg, ... of the list
+    _decode_case(sala, 64 * 500 + 7, 64, 1, 2, torch.bfloat16, 15, given_idx=True)
+
+
+def test_sparse_decode_clustered_winners_take_the_exact_fallback(sala):
+    """The prefetching kernel ranks each CTA's best 8 keys among the group's published ones; when a
+    CTA holds more than 8 winners it must fall back to an exact selection over all keys.  The
+    candidates are dealt to the group's CTAs in 4-block chunks round robin (74 CTAs per group on a
+    148-SM B200 with 2 groups), so planting the 80 best blocks in chunks 0, 74, 148, ... puts all of
+    them in one CTA.  Selection and output are checked against the oracle on the planted k-bar."""
+    from hybrid_sparse_linear_b200 import synth
+    T, topk, n_init, n_local, H, Hkv, d = 1 << 20, 64, 1, 2, 32, 2, 128
+    layer = synth.sparse_layer(1, H, Hkv, T, d, torch.bfloat16, device="cuda", layer=17,
+                               shift_frac=0.02, q_rows=1)
+    kbar = sala.block_compress(layer.k)
+    q64 = _f64(layer.q)
+    qbar = q64[0].reshape(Hkv, H // Hkv, d).sum(axis=1)                    # [Hkv, d]
+    kb = _f64(kbar)
+    planted = []
+    for t in range(20):
+        for r in range(4):
+            cand = 74 * 4 * t + r
+            blk = n_init + cand
+            planted.append(blk)
+            i = len(planted)
+            for g in range(Hkv):
+                kb[0, g, blk] += (20000.0 + 97.0 * i) * qbar[g] / float(qbar[g] @ qbar[g])
+    kbar_p = torch.from_numpy(kb).to(torch.bfloat16)
+    kb_ref = _f64(kbar_p)
+    kbar_p = kbar_p.cuda()
+    slots = n_init + n_local + topk
+    idx_out = torch.empty((1, Hkv, slots), dtype=torch.int32, device="cuda")
+    qd = layer.q[:, :, 0].contiguous()
+    o = sala.sparse_decode(qd, layer.k, layer.v, kbar_p, T - 1, topk, n_init, n_local,
+                           idx_out=idx_out)
+    sala.check_status()
+    idx_ref, kth = oracle.block_select(q64, kb_ref, 64, topk, n_init, n_local, q_pos0=T - 1)
+    got = idx_out.cpu().numpy()[:, :, None, :]
+    check_selection(got, idx_ref, q64, kb_ref, kth, topk, n_init, n_local, q_pos0=T - 1,
+                    row_ids=np.array([0]))
+    assert set(got[0, 0, 0, n_init:n_init + topk]) <= set(planted)
+    o_ref = oracle.sparse_attention(q64, _f64(layer.k), _f64(layer.v), got, 64, q_pos0=T - 1)
+    assert_close(_f64(o), o_ref[:, :, 0], "bf16", "decode o")
+
+
+@pytest.mark.parametrize("graph", [False, True])
+def test_hybrid_decode_chain_programmatic_dependents(sala, graph):
+    """One token through linear, linear, sparse, linear, sparse layers, every call launched as a
+    programmatic dependent of the one before (the linear ones read their state early, the sparse
+    ones their share of k-bar); eagerly and replayed from a CUDA graph.  Every layer's output
+    against the oracle (the sparse ones through the selection check)."""
+    from hybrid_sparse_linear_b200 import synth
+    H, Hkv, d, topk, n_init, n_local = 32, 2, 128, 64, 1, 2
+    kinds = ["lin", "lin", "sparse", "lin", "sparse"]
+    gen = torch.Generator().manual_seed(91)
+    lam = synth.decays(H)
+    lam_d = lam.cuda()
+    layers = []
+    for li, kind in enumerate(kinds):
+        if kind == "lin":
+            S0 = torch.randn((1, H, d, d), generator=gen) / d
+            qkv = [(torch.randn((1, H, d), generator=gen) / 4).to(torch.bfloat16) for _ in range(3)]
+            layers.append(("lin", S0, [x.cuda() for x in qkv], qkv, S0.clone().cuda()))
+        else:
+            T = 64 * (1500 + 700 * li) + 11
+            sl = synth.sparse_layer(1, H, Hkv, T, d, torch.bfloat16, device="cuda", layer=30 + li,
+                                    q_rows=1)
+            kbar = sala.block_compress(sl.k)
+            ws = torch.zeros(sala.sparse_decode_workspace_bytes(1, H, Hkv, T - 1, topk, n_init,
+                                                                n_local, d), dtype=torch.uint8,
+                             device="cuda")
+            idx = torch.empty((1, Hkv, n_init + n_local + topk), dtype=torch.int32, device="cuda")
+            layers.append(("sparse", T, sl, kbar, ws, idx))
+    outs = [torch.empty((1, H, d), dtype=torch.bfloat16, device="cuda") for _ in kinds]
+    stream = torch.cuda.Stream()
+
+    def run():
+        for li, L in enumerate(layers):
+            if L[0] == "lin":
+                q, k, v = L[2]
+                sala.linear_decode(q, k, v, lam_d, L[4], o=outs[li], stream=stream, pdl=True)
+            else:
+                _, T, sl, kbar, ws, idx = L
+                sala.sparse_decode(sl.q[:, :, 0].contiguous(), sl.k, sl.v, kbar, T - 1, topk,
+                                   n_init, n_local, idx_out=idx, o=outs[li], workspace=ws,
+                                   stream=stream, pdl=True)
+
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        if graph:
+            G = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(G, stream=stream):
+                run()
+            for L in layers:  # capture ran nothing; start from the initial states anyway
+                if L[0] == "lin":
+                    L[4].copy_(L[1])
+            G.replay()
+        else:
+            run()
+    torch.cuda.synchronize()
+    sala.check_status(stream)
+    for li, L in enumerate(layers):
+        if L[0] == "lin":
+            q, k, v = (_f64(x) for x in L[3])
+            o_ref, _ = oracle.linear_decode(q, k, v, _f64(lam), _f64(L[1]))
+            assert_close(_f64(outs[li]), o_ref, "bf16", f"layer {li} (linear)")
+        else:
+            _, T, sl, kbar, ws, idx = L
+            q64 = _f64(sl.q)
+            kb_ref = oracle.block_compress(_f64(sl.k), 64)
+            np.testing.assert_array_equal(_f64(kbar), kb_ref)
+            idx_ref, kth = oracle.block_select(q64, kb_ref, 64, topk, n_init, n_local, q_pos0=T - 1)
+            got = idx.cpu().numpy()[:, :, None, :]
+            check_selection(got, idx_ref, q64, kb_ref, kth, topk, n_init, n_local, q_pos0=T - 1,
+                            row_ids=np.array([0]))
+            o_ref = oracle.sparse_attention(q64, _f64(sl.k), _f64(sl.v), got, 64, q_pos0=T - 1)
+            assert_close(_f64(outs[li]), o_ref[:, :, 0], "bf16", f"layer {li} (sparse)")
+
+
+def test_sparse_decode_run_twice_bitwise(sala):
+    # the same call twice on fresh workspaces gives the same bits (selection and output)
+    from hybrid_sparse_linear_b200 import synth
+    T = 1 << 19
+    sl = synth.sparse_layer(1, 32, 2, T, 128, torch.bfloat16, device="cuda", layer=18, q_rows=1)
+    kbar = sala.block_compress(sl.k)
+    res = []
+    for _ in range(2):
+        idx = torch.empty((1, 2, 67), dtype=torch.int32, device="cuda")
+        o = sala.sparse_decode(sl.q[:, :, 0].contiguous(), sl.k, sl.v, kbar, T - 1, 64, 1, 2,
+                               idx_out=idx)
+        sala.check_status()
+        res.append((o, idx))
+    assert torch.equal(res[0][1], res[1][1]) and torch.equal(res[0][0], res[1][0])
+
+
 # ---------------------------------------------------------------------------------------------
 # Paged KV cache, one position per sequence (sala_sparse_decode_paged)
 
