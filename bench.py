@@ -707,15 +707,13 @@ def run_e2e(sala, synth, torch, steps, warmup):
 
 
 # ----------------------------------------------------------------------------------------------
-# CPU baseline: the fp64 oracle on a bounded sample, scaled to the full workload.
+# CPU baseline: the fp64 oracle on bounded samples, scaled to the full workloads.
 
-def cpu_baseline(torch, synth, budget_s: float = 20.0):
-    import numpy as np
+def oracle_linear_layer(torch, synth, n_tok, budget_s):
+    """Seconds of one linear layer (32 heads x n_tok tokens) in the oracle's chunked form, from a
+    sample of `cores` heads; a 4096-token pilot sizes it to about 40 % of the budget."""
     import oracle
     cores = oracle.default_threads()
-    t_start = time.time()
-    # Linear layers: `cores` heads x n_lin tokens (the chunked form is O(N) per head).
-    # A pilot of 4096 tokens sizes the sample to about 40 % of the budget (at most the full length).
     hs = min(cores, H)
     lam = synth.decays(H)[:hs]
     f = oracle.from_tensor
@@ -726,15 +724,24 @@ def cpu_baseline(torch, synth, budget_s: float = 20.0):
         oracle.linear_chunked(f(q), f(k), f(v), f(lam), 64, threads=cores)
         return time.perf_counter() - t0
 
-    n_lin = 4096
+    n_lin = min(4096, n_tok)
     t_lin = lin_sample(n_lin)
-    grow = int(min(N_TOK // n_lin, max(1.0, 0.4 * budget_s / max(t_lin, 1e-6))))
+    grow = int(min(n_tok // n_lin, max(1.0, 0.4 * budget_s / max(t_lin, 1e-6))))
     if grow > 1:
         n_lin *= 1 << (grow.bit_length() - 1)
         t_lin = lin_sample(n_lin)
-    lin_layer_s = t_lin * (H / hs) * (N_TOK / n_lin)
-    # Sparse layers: selection + attention for sampled query rows spread over the sequence; the
-    # attention cost is proportional to the attended keys, the selection cost to the candidates.
+    return {"s": t_lin * (H / hs) * (n_tok / n_lin), "cores": cores,
+            "sample": f"{hs} heads x {n_lin} tokens (scaled x{H / hs:.0f} heads, x{n_tok / n_lin:g} length)"}
+
+
+def oracle_sparse_layer(torch, synth, n_tok, budget_s):
+    """Seconds of one sparse layer (selection + attention, 32 query heads over 2 KV heads) at n_tok
+    tokens: sampled query rows from the second half of a 32768-token layer, the attention scaled by
+    attended keys and the selection by candidate blocks."""
+    import numpy as np
+    import oracle
+    cores = oracle.default_threads()
+    f = oracle.from_tensor
     n_s = 32768
     sl = synth.sparse_layer(1, H, HKV, n_s, D, torch.bfloat16, "cpu", layer=3)
     q64, k64, v64 = f(sl.q), f(sl.k), f(sl.v)
@@ -763,29 +770,134 @@ def cpu_baseline(torch, synth, budget_s: float = 20.0):
     grow = int(min((n_s // 2) // n_rows, max(1.0, 0.4 * budget_s / max(t_sel + t_att, 1e-6))))
     if grow > 1:
         rows_tok, t_sel, t_att = sparse_sample(n_rows * grow)
-    # scale: attention by attended keys, selection by candidate count
-    keys_sample = 0
-    cand_sample = 0
+    keys_sample = cand_sample = 0
     for r in rows_tok:
         c = r // BLOCK
         ncand = max(0, c - N_LOCAL + 1 - N_INIT)
         full_before = c if ncand <= TOPK else N_INIT + TOPK + N_LOCAL - 1
         keys_sample += full_before * BLOCK + (r % BLOCK) + 1
         cand_sample += ncand
-    keys_full = attended_keys(N_TOK)
-    cand_full = sum(max(0, i // BLOCK - N_LOCAL + 1 - N_INIT) for i in range(0, N_TOK, BLOCK)) * BLOCK
-    sparse_layer_s = t_att * keys_full / keys_sample + t_sel * (cand_full * HKV) / (cand_sample * HKV)
-    step_s = 24 * lin_layer_s + 8 * sparse_layer_s
-    return {"value": N_TOK / step_s, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-            "sample": (f"linear: {hs} heads x {n_lin} tokens (scaled x{H / hs:.0f} heads, "
-                       f"x{N_TOK // n_lin} length); sparse: selection + attention of {len(rows_tok)} "
-                       f"query tokens x {H} heads sampled from the second half of a {n_s}-token "
-                       f"layer (scaled by attended keys and candidate blocks); "
+    keys_full = attended_keys(n_tok)
+    cand_full = sum(max(0, i // BLOCK - N_LOCAL + 1 - N_INIT) for i in range(0, n_tok, BLOCK)) * BLOCK
+    return {"s": t_att * keys_full / keys_sample + t_sel * cand_full / cand_sample, "cores": cores,
+            "sample": (f"selection + attention of {len(rows_tok)} query tokens x {H} heads sampled "
+                       f"from the second half of a {n_s}-token layer (scaled to {n_tok} tokens by "
+                       f"attended keys and candidate blocks)")}
+
+
+def oracle_decode_token(torch, synth, T):
+    """Seconds of one decode token at a T-token context in the oracle, at full size: a linear decode
+    step (32 heads, 128 x 128 state) counted 24 times, and a sparse step counted 8 times --
+    selection over the T/64 blocks' k_bar, then softmax attention over 67 blocks (a cache holding
+    exactly those blocks' keys, so the attended work is that of the real step)."""
+    import numpy as np
+    import oracle
+    f = oracle.from_tensor
+    cores = oracle.default_threads()
+    g = torch.Generator().manual_seed(5)
+    lam = f(synth.decays(H))
+    t_lin = 0.0
+    for _ in range(2):
+        S = torch.randn((1, H, D, D), generator=g, dtype=torch.float64).numpy() / D
+        q, k, v = (f(torch.randn((1, H, D), generator=g).to(torch.bfloat16)) for _ in range(3))
+        t0 = time.perf_counter()
+        oracle.linear_decode(q, k, v, lam, S)
+        t_lin += (time.perf_counter() - t0) / 2
+    nb = T // BLOCK
+    kbar = f(torch.randn((1, HKV, nb, D), generator=g).to(torch.bfloat16))
+    qd = f(torch.randn((1, H, 1, D), generator=g).to(torch.bfloat16))
+    t0 = time.perf_counter()
+    oracle.block_select(qd, kbar, BLOCK, TOPK, N_INIT, N_LOCAL, q_pos0=T - 1, threads=cores)
+    t_sel = time.perf_counter() - t0
+    slots = N_INIT + N_LOCAL + TOPK
+    n_c = slots * BLOCK
+    kc = f(torch.randn((1, HKV, n_c, D), generator=g).to(torch.bfloat16))
+    vc = f(torch.randn((1, HKV, n_c, D), generator=g).to(torch.bfloat16))
+    idx = np.tile(np.arange(slots, dtype=np.int32), (1, HKV, 1, 1))
+    t0 = time.perf_counter()
+    oracle.sparse_attention(qd, kc, vc, idx, BLOCK, q_pos0=n_c - 1, threads=cores)
+    t_att = time.perf_counter() - t0
+    s = 24 * t_lin + 8 * (t_sel + t_att)
+    return {"s": s, "cores": cores,
+            "sample": (f"one token at full size, each kind of step timed once and counted per "
+                       f"layer: 24 x linear decode step ({t_lin * 1e3:.2f} ms, mean of 2) + 8 x "
+                       f"(selection over {nb} blocks {t_sel * 1e3:.1f} ms + attention over {slots} "
+                       f"blocks {t_att * 1e3:.1f} ms)")}
+
+
+def cpu_baseline(torch, synth, budget_s: float = 20.0):
+    t_start = time.time()
+    lin = oracle_linear_layer(torch, synth, N_TOK, budget_s)
+    sp = oracle_sparse_layer(torch, synth, N_TOK, budget_s)
+    step_s = 24 * lin["s"] + 8 * sp["s"]
+    return {"value": N_TOK / step_s, "unit": "tokens/s", "cores": lin["cores"], "kind": "oracle",
+            "sample": (f"linear: {lin['sample']}; sparse: {sp['sample']}; "
                        f"{time.time() - t_start:.1f} s of CPU work"),
             "step_s_extrapolated": step_s}
 
 
+def config_lines(sala, synth, torch, stream, peaks, steps, warmup, decode=None, cpu=True,
+                 budget_s=8.0):
+    """One record per further benchmark configuration: the 32K linear prefill, the 128K sparse
+    prefill and the 1M-context decode -- absolute throughput, roofline fraction and, on rank 0, the
+    oracle timed on the host cores beside it."""
+    out = {}
+    hbm, tc = peaks["hbm_gbs"], peaks["bf16_tflops_sustained"]
+    n = 32768
+    pre = run_prefill(sala, synth, torch, steps, warmup, stream, "linear_prefill_n32k")
+    ms = pre["total_ms"] / steps
+    gbs = linear_layer_bytes(n) / (ms * 1e-3) / 1e9
+    rec = {"workload": "linear_prefill_n32k: B=1, 32 heads, d=128, N=32768, bf16, chunk 64",
+           "tokens_per_s": n / (ms * 1e-3), "ms": ms, "bound": "hbm", "achieved_gbs": gbs,
+           "roofline_frac": gbs / hbm, "algorithmic_bytes": linear_layer_bytes(n)}
+    if cpu:
+        o = oracle_linear_layer(torch, synth, n, budget_s)
+        rec["oracle"] = {"tokens_per_s": n / o["s"], "s": o["s"], "cores": o["cores"],
+                         "sample": o["sample"]}
+    out["linear_prefill_n32k"] = rec
+    n = 131072
+    pre = run_prefill(sala, synth, torch, steps, warmup, stream, "sparse_prefill_n128k")
+    ms = pre["total_ms"] / steps
+    fl = sparse_layer_flops(n)
+    rec = {"workload": "sparse_prefill_n128k: B=1, 32 query / 2 KV heads, d=128, N=131072, bf16, "
+                       "block 64, top-64 + init + 2 local (compress, select, attend)",
+           "tokens_per_s": n / (ms * 1e-3), "ms": ms, "bound": "tensor",
+           "attention_ms": pre["sparse_ms"], "selection_ms": pre["select_ms"],
+           "achieved_tflops": fl / (pre["sparse_ms"] * 1e-3) / 1e12,
+           "roofline_frac": fl / (pre["sparse_ms"] * 1e-3) / 1e12 / tc,
+           "executed_frac": pre["sparse_exec_flops"] / (pre["sparse_ms"] * 1e-3) / 1e12 / tc,
+           "algorithmic_flops": fl, "peak": f"{tc} TFLOP/s bf16 sustained ({peaks['source']})"}
+    if cpu:
+        o = oracle_sparse_layer(torch, synth, n, budget_s)
+        rec["oracle"] = {"tokens_per_s": n / o["s"], "s": o["s"], "cores": o["cores"],
+                         "sample": o["sample"]}
+    out["sparse_prefill_n128k"] = rec
+    if decode is not None:
+        us = decode["us_per_token"]
+        db = decode_bytes(DECODE_T)
+        rec = {"workload": "decode_1m: one token through 24 linear + 8 sparse layers at a 2^20-token "
+                           "context, batch 1",
+               "tokens_per_s": 1e6 / us, "us_per_token": us, "bound": "hbm",
+               "achieved_gbs": db["step"] / (us * 1e-6) / 1e9,
+               "roofline_frac": db["step"] / (us * 1e-6) / 1e9 / hbm, "bytes_per_token": db["step"]}
+        if cpu:
+            o = oracle_decode_token(torch, synth, DECODE_T)
+            rec["oracle"] = {"tokens_per_s": 1.0 / o["s"], "s": o["s"], "cores": o["cores"],
+                             "sample": o["sample"]}
+        out["decode_1m"] = rec
+    return out
+
+
 # ----------------------------------------------------------------------------------------------
+def bench_config(ws: int) -> dict:
+    return {"workload": "hybrid_prefill_n256k: 24 linear + 8 sparse layers, N=262144, "
+                        "32 heads (2 KV heads in sparse layers), d=128, chunk 64, "
+                        "block 64, top-64 + init + 2 local",
+            "global_batch": ws, "seq_len": N_TOK,
+            "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU",
+            "l2": "inputs larger than L2 (2 GiB per tensor); decode flushes L2 per step"}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -794,9 +906,9 @@ def main():
     ap.add_argument("--impl", choices=["sala", "reference"], default="sala")
     ap.add_argument("--cpu-budget", type=float, default=0.0,
                     help="seconds of oracle work per CPU-baseline sample (0: the default sizing)")
-    ap.add_argument("--phases", default="prefill,decode,e2e,cpu",
-                    help="comma list of prefill,decode,e2e,cpu,paged,backward,qknorm,sparse_bwd "
-                         "(default: the first four)")
+    ap.add_argument("--phases", default="prefill,decode,e2e,cpu,configs",
+                    help="comma list of prefill,decode,e2e,cpu,configs,paged,backward,qknorm,"
+                         "sparse_bwd (default: the first five)")
     ap.add_argument("--decode-steps", type=int, default=200)
     ap.add_argument("--decode-t", type=int, default=DECODE_T,
                     help="decode context length (default 2^20, the benchmark; smaller only for profiles)")
@@ -830,13 +942,13 @@ def main():
             if i >= args.warmup:
                 vals.append(r)
         v = statistics.median(x["value"] for x in vals)
+        # each step is a bounded sample scaled to the full step: ms_per_step is extrapolated
         line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s",
                 "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-                "ms_per_step": 1000.0 * N_TOK / v, "higher_is_better": True, "scaling": "weak",
+                "ms_per_step": 1000.0 * N_TOK / v, "extrapolated": True,
+                "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-                "config": {"workload": "hybrid_prefill_n256k: 24 linear + 8 sparse layers, "
-                                       "N=262144, 32 heads (2 KV heads in sparse layers), d=128",
-                           "global_batch": 1, "seq_len": N_TOK, "parallelism": "replicas"},
+                "config": bench_config(ws),
                 "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": vals[-1]["cores"],
                                  "kind": "oracle", "sample": vals[-1]["sample"]},
                 "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -859,12 +971,7 @@ def main():
     line = {"metric": METRIC, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded normal Q/K/V per layer)",
-            "config": {"workload": "hybrid_prefill_n256k: 24 linear + 8 sparse layers, N=262144, "
-                                   "32 heads (2 KV heads in sparse layers), d=128, chunk 64, "
-                                   "block 64, top-64 + init + 2 local",
-                       "global_batch": ws, "seq_len": N_TOK,
-                       "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU",
-                       "l2": "inputs larger than L2 (2 GiB per tensor); decode flushes L2 per step"}}
+            "config": bench_config(ws)}
     if "prefill" in phases:
         vis = [x for x in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if x.strip()]
         sampler = ClockSampler(vis[local] if local < len(vis) else str(local))
@@ -965,6 +1072,13 @@ def main():
                                     "launched as a programmatic dependent (linear state and sparse "
                                     "k_bar reads overlapping the previous layer); per-layer figures "
                                     "from graphs of one kind of call only"}
+    dec_result = None
+    if "decode" in phases:
+        dec_result = {"us_per_token": line["decode"]["us_per_token"]}
+    if "configs" in phases and args.workload == "hybrid_prefill_n256k":
+        line["configs"] = config_lines(sala, synth, torch, stream, peaks, max(args.steps, 3),
+                                       max(args.warmup, 3), dec_result,
+                                       cpu=(rank == 0 and ws == 1), budget_s=args.cpu_budget or 8.0)
     if "e2e" in phases:
         e = run_e2e(sala, synth, torch, max(1, min(args.steps, 2)), 1)
         line["e2e"] = {"value": ws * N_TOK / (max_over_ranks(e["ms_per_step"], "cuda") / 1000.0),

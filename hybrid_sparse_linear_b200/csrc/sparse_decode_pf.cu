@@ -110,15 +110,20 @@ constexpr size_t pf_smem_bytes(int rcap, int nstages) { return pf_region_off<D>(
 // ---------------------------------------------------------------- tagged words
 __device__ __forceinline__ uint64_t ll_word(uint32_t v, uint32_t tag) { return ((uint64_t)v << 32) | tag; }
 __device__ __forceinline__ void ll_st(uint64_t* p, uint64_t w) {
-    asm volatile("st.volatile.global.u64 [%0], %1;" ::"l"(p), "l"(w) : "memory");
+    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(w) : "memory");
 }
 __device__ __forceinline__ void ll_st2(uint64_t* p, uint64_t a, uint64_t b) {  // p 16-byte aligned
-    asm volatile("st.volatile.global.v2.u64 [%0], {%1, %2};" ::"l"(p), "l"(a), "l"(b) : "memory");
+    asm volatile("st.relaxed.gpu.global.v2.u64 [%0], {%1, %2};" ::"l"(p), "l"(a), "l"(b) : "memory");
 }
+// Reads of other CTAs' words are strong (gpu-scope relaxed): a weak load may be served from a copy
+// that is never refreshed and would not see the writer's update.
 __device__ __forceinline__ uint64_t ll_ld(const uint64_t* p) {
     uint64_t w;
-    asm volatile("ld.volatile.global.u64 %0, [%1];" : "=l"(w) : "l"(p) : "memory");
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(w) : "l"(p) : "memory");
     return w;
+}
+__device__ __forceinline__ void ll_ld2(const uint64_t* p, uint64_t& a, uint64_t& b) {  // p 16-byte aligned
+    asm volatile("ld.relaxed.gpu.global.v2.u64 {%0, %1}, [%2];" : "=l"(a), "=l"(b) : "l"(p) : "memory");
 }
 __device__ __forceinline__ bool ll_ok(uint64_t w, uint32_t tag) { return (uint32_t)w == tag; }
 __device__ __forceinline__ uint32_t ll_val(uint64_t w) { return (uint32_t)(w >> 32); }
@@ -504,11 +509,23 @@ sparse_decode_pf_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16
         if (tid < cpg) {
             uint64_t w[2 * (kPub + 1)];
             const uint64_t* lst = part + ((int64_t)(j % kPubCopies) * kMaxCpg + tid) * kPubWords;
-            {  // one word per round until the list shows up, then the whole list
-                uint64_t w1[1];
-                ll_wait_all([&](int) { return lst + 2 * kPub + 1; }, 1, w1, tag, ctx, bad);
+            {  // the list's words are their own readiness flags: one round trip after they land
+                uint64_t t0 = 0;
+                while (true) {
+#pragma unroll
+                    for (int i = 0; i <= kPub; ++i) ll_ld2(lst + 2 * i, w[2 * i], w[2 * i + 1]);
+                    unsigned miss = 0u;
+#pragma unroll
+                    for (int i = 0; i < 2 * (kPub + 1); ++i) miss |= (unsigned)((uint32_t)w[i] != tag);
+                    if (miss == 0u) break;
+                    const uint64_t t = globaltimer_ns();
+                    if (t0 == 0) t0 = t;
+                    if (*bad || t - t0 > ctx.wait_limit_ns) {
+                        *bad = 1;
+                        break;
+                    }
+                }
             }
-            ll_wait_all([&](int i) -> const uint64_t* { return lst + i; }, 2 * (kPub + 1), w, tag, ctx, bad);
             uint64_t mine[kPub];
 #pragma unroll
             for (int qq = 0; qq < kPub; ++qq) mine[qq] = sm.own[qq];
@@ -665,6 +682,10 @@ sparse_decode_pf_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16
     }
     __syncthreads();  // also: every thread is done with the k_bar rows the stages now overwrite
 
+    // CTA 0 requests every CTA's alive word now and looks at them at the end (see there)
+    uint64_t alive_w = 0;
+    if (blockIdx.x == 0 && tid < (int)gridDim.x) alive_w = ll_ld(alive + tid);
+
     // ---------------------------------------------------------------- C: per-slot partials
     // Warp w < nstages attends items w, w + nstages, ... in its own stage: its lanes request the
     // block's K and V rows (16-byte asynchronous copies; rows past the query zero-filled), wait for
@@ -708,7 +729,8 @@ sparse_decode_pf_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16
     }
 
     // ---------------------------------------------------------------- D: combine, idx_out
-    if (idx_out && j == 0) {
+    // idx_out comes from a CTA without a combine item when there is one
+    if (idx_out && j == (cpg > G * (D / 32) ? cpg - 1 : 0)) {
         if (owner && !fallback) {
             if (warp == 0) {
                 uint64_t ww[2];
@@ -798,6 +820,7 @@ sparse_decode_pf_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16
     // reading it), so the next call on this workspace uses a new tag.
     if (blockIdx.x == 0) {
         for (int i0 = 0; i0 < (int)gridDim.x; i0 += kThreads) {
+            if (i0 == 0 && (tid >= (int)gridDim.x || ll_ok(alive_w, tag))) continue;
             uint64_t ww[1];
             ll_wait_all([&](int) { return alive + min(i0 + tid, (int)gridDim.x - 1); }, 1, ww, tag, ctx, bad);
         }

@@ -308,6 +308,38 @@ def sparse_attention(q, k, v, idx, block, scale=None, q_pos0=0, rows=None, threa
     return o
 
 
+def block_select_per_head(q, kbar, block, topk, n_init, n_local, q_pos0=0, slots=None, threads=None):
+    """Per-query-head block selection (a listed variant of the selection step): every query head h
+    chooses its own blocks, scored with its own query, score_h(j) = q_h . kbar_{g(h), j}; forced
+    blocks, candidates, ties and the row layout as block_select.  This is block_select with groups of
+    one head: each head gets its KV head's kbar.  Returns (idx [B, H, Nq, slots] int32, kth_score
+    [B, H, Nq])."""
+    q, kbar = _f64(q), _f64(kbar)
+    B, H, Nq, d = q.shape
+    Hkv = kbar.shape[1]
+    G = H // Hkv
+    kbar_h = np.ascontiguousarray(np.repeat(kbar, G, axis=1))   # [B, H, nb, d]: head h -> kbar of h // G
+    return block_select(q, kbar_h, block, topk, n_init, n_local, q_pos0=q_pos0, slots=slots,
+                        threads=threads)
+
+
+def sparse_attention_per_head(q, k, v, idx_h, block, scale=None, q_pos0=0, threads=None):
+    """Softmax attention over per-head selections: idx_h [B, H, Nq, slots] gives query head h its
+    own blocks (of its KV head's keys).  One sparse_attention per head, each a group of one head."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H, Nq, d = q.shape
+    Hkv = k.shape[1]
+    G = H // Hkv
+    idx_h = np.ascontiguousarray(idx_h, dtype=np.int32)
+    o = np.empty((B, H, Nq, d))
+    for h in range(H):
+        g = h // G
+        o[:, h:h + 1] = sparse_attention(q[:, h:h + 1], k[:, g:g + 1], v[:, g:g + 1],
+                                         idx_h[:, h:h + 1], block, scale=scale, q_pos0=q_pos0,
+                                         threads=threads)
+    return o
+
+
 def dense_causal_attention(q, k, v, scale=None, q_pos0=0, threads=None):
     q, k, v = _f64(q), _f64(k), _f64(v)
     B, H, Nq, d = q.shape
