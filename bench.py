@@ -615,11 +615,11 @@ def run_decode(sala, synth, torch, steps, warmup, stream, T=DECODE_T):
     sala.check_status(stream)
     del graph, graph_plain, lin, sp, ws, flush
     torch.cuda.empty_cache()
-    # launches per token: linear 1 each; sparse 1 each (scoring, top-k, attention and combine in
-    # one cooperative launch)
+    # launches per token: linear 1 each; sparse 2 each (the score kernel over every SM, then the
+    # attend kernel of one cluster per KV group)
     return {"us_per_token": statistics.median(us), "us_min": min(us), "samples": len(us),
             "us_per_token_without_pdl": statistics.median(us_plain),
-            "launches_per_token": 24 * 1 + 8 * 1,
+            "launches_per_token": 24 * 1 + 8 * 2,
             "us_per_linear_layer": lin_us, "us_per_sparse_layer": sp_us}
 
 

@@ -543,10 +543,9 @@ sala_status sala_sparse_prefill(const void* q, const void* k, const void* v, con
                     "sparse_prefill");
 }
 
-// Sparse decode workspace: [0, 256) the cooperative one-launch path's barrier words and [256, 512)
-// the prefetching one-launch path's epoch word, in every layout; from 512 on, the data of whichever
-// path a call takes (the prefetching path's tagged words may share bytes with the other paths'
-// data: no value those store looks like a tag).
+// Sparse decode workspace: [0, 256) the cooperative one-launch path's barrier words, [256, 512)
+// unused; from 512 on, the data of whichever path a call takes (every path writes what it reads
+// there within the call).
 size_t sala_sparse_decode_workspace(int B, int H, int Hkv, int pos, int block, int topk,
                                     int n_init, int n_local, int d) {
     if (B <= 0 || H <= 0 || Hkv <= 0 || pos < 0 || block <= 0) return 0;
@@ -700,8 +699,8 @@ sala_status sala::sparse_decode_impl(const void* q, const void* kcache, const vo
         const size_t base = 512;
         const cudaError_t e = sala::launch_sparse_decode_pf(
             to_dt(dt), q, kcache, vcache, kbar, idx_in, idx_out, o, B, H, Hkv, pos, Tmax, nb_cap, d,
-            topk, n_init, n_local, scale, static_cast<unsigned*>(static_cast<void*>(static_cast<char*>(workspace) + 256)),
-            static_cast<char*>(workspace) + base, workspace_bytes - base, pdl, st, ctx);
+            topk, n_init, n_local, scale, static_cast<char*>(workspace) + base,
+            workspace_bytes - base, pdl, st, ctx);
         if (e != cudaErrorNotSupported) return launched(e, "sparse_decode");
     }
     {

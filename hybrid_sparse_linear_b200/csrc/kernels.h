@@ -138,23 +138,22 @@ cudaError_t launch_sparse_decode_fused(DType dt, const void* q, const void* kc, 
                                        int nb_cap, int d, int topk, int n_init, int n_local,
                                        float scale, void* ws, size_t ws_bytes, DecodePaging pg, cudaStream_t st,
                                        DevCtx ctx);
-// Sparse decode in one launch with k_bar prefetched into shared memory (bf16, d 64 or 128, dense
-// cache, one position): each CTA scores its share of the rows out of shared memory, ranks its own
-// best keys among the group's published ones and attends the blocks it wins.  pdl: launched as a
-// programmatic dependent of the previous kernel (k_bar is read before that kernel completes).
-// Returns cudaErrorNotSupported, launching nothing, when the problem does not fit it (k > 64, more
-// than 80 slots, more than 16 heads per group, more than 64 groups, a CTA's share of k_bar above
-// its shared-memory rows, or a smaller workspace).  epoch: a word that stays at one place for every
-// call on the same workspace; ws: the path's own region of tagged words (both zero before the
-// first call).
+// Sparse decode in two launches (bf16, d 64 or 128, dense cache, one position): a score kernel over
+// every SM (k_bar prefetched into shared memory, each CTA's best keys stored) and an attend kernel of
+// one 16-CTA cluster per (batch, KV group) that ranks the stored keys, attends the winners and
+// combines the partials in distributed shared memory.  pdl: the first launch is a programmatic
+// dependent of the previous kernel (k_bar is read before that kernel completes).  Returns
+// cudaErrorNotSupported, launching nothing, when the problem does not fit (k > 64, more than 80
+// slots, more than 16 heads per group, more than 16 groups or more than the GPU holds clusters, a
+// scoring CTA's share of k_bar above its shared memory, or a smaller workspace).  ws: the path's own
+// bytes, written before they are read within each call (no initial value needed).
 size_t sparse_decode_pf_workspace(int B, int H, int Hkv, int pos, int topk, int n_init, int n_local,
                                   int d);
 cudaError_t launch_sparse_decode_pf(DType dt, const void* q, const void* kc, const void* vc,
                                     const void* kbar, const int32_t* idx_in, int32_t* idx_out,
                                     void* o, int B, int H, int Hkv, int pos, int Tmax, int nb_cap,
-                                    int d, int topk, int n_init, int n_local, float scale,
-                                    unsigned* epoch, void* ws, size_t ws_bytes, bool pdl,
-                                    cudaStream_t st, DevCtx ctx);
+                                    int d, int topk, int n_init, int n_local, float scale, void* ws,
+                                    size_t ws_bytes, bool pdl, cudaStream_t st, DevCtx ctx);
 cudaError_t launch_sparse_decode_attn(DType dt, const void* q, const void* kc, const void* vc,
                                       const int32_t* idx, void* o, int B, int H, int Hkv,
                                       int pos, int Tmax, int d, int slots, float scale, void* ws,

@@ -98,6 +98,10 @@ __device__ __forceinline__ void bulk_load_g2s(void* dst, const void* src, uint32
         "l"(src), "r"(bytes), "r"(smem_u32(bar))
         : "memory");
 }
+// Hint: bring [src, src + bytes) into L2 (src 16-byte aligned, bytes a multiple of 16).
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
 // 16-byte asynchronous copy global -> shared memory; with valid == false the 16 bytes are
 // zero-filled and global memory is not read.
 __device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {

@@ -1,46 +1,37 @@
-// Sparse decode with the block-key table prefetched: block scoring, top-k selection and attention
-// for one query token per (batch, KV group) in one launch, bf16, d = 64 or 128.
+// Sparse decode in two launches for bf16, d = 64 or 128: the block-key table k_bar is prefetched
+// and scored by every SM, then one thread-block cluster per (batch, KV group) attends the selected
+// blocks and combines the partials in distributed shared memory.
 //
-// The step reads two things: the whole block-key table k_bar of the group (8 MiB at 2^20 tokens
-// and 2 KV heads) to score the candidates, and the ~67 selected K/V blocks (4 MiB) to attend.  The
-// k_bar table does not depend on the query, so each CTA starts copying its share of it into shared
-// memory (16-byte asynchronous copies from every thread) as soon as it runs -- before
-// griddepcontrol.wait when the call is launched as a programmatic dependent, i.e. while the
-// previous layer's kernel is still running.  Rows are dealt to the group's `cpg` CTAs in 4-row
-// chunks, round robin, so blocks that are chosen together (recent context, a run of related
-// blocks) land in different CTAs.
+// The step reads the whole block-key table of the group (8 MiB at 2^20 tokens and 2 KV heads) to
+// score the candidates, and then only the ~67 selected K/V blocks (4 MiB).  Exchanging data between
+// CTAs through global memory costs a round trip to the memory's home (on a two-die B200 often the
+// other die) every time, so the design keeps exactly one global exchange, the one between the two
+// kernels, where the kernel boundary itself makes the data visible:
 //
-//   A  every CTA scores its rows on the tensor cores (the group-summed query split into bf16
-//      hi + lo rows of an m16n8k16 tile against 8 k_bar rows at a time), keeps its best kPub + 1
-//      selection keys (orderable score above the inverted block index: distinct, larger = better,
-//      ties to the lower block) by counting ranks, and publishes them.
-//   B  every CTA reads the group's published lists U (kPub keys per CTA) and ranks its own kPub
-//      keys within U: a key of rank r < k is the group's (r+1)-th best block.  This is exact unless
-//      some CTA has more than kPub winners: with X = the largest (kPub+1)-th key of any CTA, no
-//      unpublished key can beat X, so when fewer than k keys of U exceed X (X would win), the lists
-//      may hide winners and all CTAs of the group (they see the same U) take the fallback: all keys
-//      published, an exact radix select over them.  Otherwise every published key of rank < k is a
-//      winner and every other key is not.
-//   C  each CTA attends the blocks it owns -- its own winners (record slot = rank) and, in the
-//      last CTAs, the init and local blocks (slots k ..) -- or, on the list paths (given
-//      selection, at most k candidates, k = 0, fallback), slots j, j + cpg, ...: the K and V of
-//      every owned block requested at once (16-byte asynchronous copies into stages that reuse the
-//      k_bar rows' shared memory), the G heads' logits and p v on warp-level tensor-core tiles, a
-//      per-head softmax partial (max, sum, sum of p v) per slot.
-//   D  the group's CTAs combine the partials, one (head, 32-column) piece each, in slot order;
-//      CTA 0 writes idx_out (blocks ascending).
+//   score kernel (groups x cpg CTAs, no waits between CTAs).  Each CTA copies its share of k_bar --
+//      4-block chunks dealt round robin, so blocks chosen together land in different CTAs -- into
+//      shared memory as soon as it runs (16-byte asynchronous copies; before griddepcontrol.wait
+//      when the call is a programmatic dependent, so the copy overlaps the previous layer's kernel).
+//      It then scores its rows on the tensor cores (the group-summed query as bf16 hi + lo rows of
+//      an m16n8k16 tile against 8 k_bar rows at a time), keeps its best kPub + 1 selection keys
+//      (orderable score above the inverted block index: distinct, larger = better, ties to the lower
+//      block) by counting ranks, and stores them, and all its keys, for the attend kernel.
+//   attend kernel (groups clusters of CS CTAs), launched as a programmatic dependent of the score
+//      kernel: before griddepcontrol.wait it loads the query rows and starts copying the init and
+//      local blocks; after it, every CTA reads the group's lists U (kPub keys per scoring CTA) and
+//      ranks its share of U's keys: a key of rank r < k is the group's (r+1)-th best block.  This is
+//      exact unless some scoring CTA had more than kPub winners: with X = the largest (kPub+1)-th
+//      key of any CTA, no unlisted key can beat X, so when fewer than k keys of U exceed X the
+//      cluster instead takes an exact radix select over all the group's keys.  The winners, by rank,
+//      are broadcast to the cluster through distributed shared memory.  CTA r then attends slots
+//      r, r + CS, ... (a warp per slot: K and V of the block by 16-byte asynchronous copies, the
+//      G heads' logits and p v on warp-level tensor-core tiles, a softmax partial per head), folds
+//      its slots into one partial per head, and after a cluster barrier combines the partials of
+//      every CTA of the cluster for its heads into the output.
 //
-// The exchanges between A and B and between C and D need no barrier: every word another CTA
-// reads is a tagged 8-byte word (32 bits of data above a 32-bit tag, written and read as one
-// single-copy-atomic access), and a reader spins, bounded, until every word it needs carries this
-// call's tag.  The tag is a signalling-NaN bit pattern (0x7F800001 + epoch mod 2^22 - 1); the epoch
-// is a word at a fixed place in the workspace that every CTA reads after griddepcontrol.wait and
-// CTA 0 advances once it has seen every CTA's tagged word (each CTA tags one word right after
-// reading the epoch), so the next call on the workspace uses a new tag; a CTA that gives up on a
-// wait advances it too.  A stale word therefore never carries the current tag, whatever layout the
-// call that wrote it had (within 2^22 - 1 calls), and no value the other decode paths store in the
-// same bytes (fp32 results, which arithmetic never makes signalling NaNs, block indices, counts)
-// looks like a tag, so this path's region may overlap theirs.
+// With a given selection (idx_in), or at most k candidates, or k = 0, only the attend kernel runs.
+#include <cooperative_groups.h>
+
 #include <mutex>
 
 #include "blocksel.cuh"
@@ -51,106 +42,58 @@
 namespace sala {
 namespace {
 
+namespace cg = cooperative_groups;
 using namespace dec;
 
 constexpr int kBlk = 64;
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int kCap = 64;         // largest k
-constexpr int kMaxSlots = 80;    // n_init + n_local + k
+constexpr int kCap = 64;            // largest k
+constexpr int kMaxSlots = 80;       // n_init + n_local + k
 constexpr int kMaxG = 16;
-constexpr int kPub = 8;          // keys per CTA ranked on the fast path
-constexpr int kPubWords = 32;    // tagged words per CTA's list: 2 per key (kPub + 1 keys), padding
-constexpr int kPubCopies = 8;    // copies of every list, so that no line is read by every CTA
-constexpr int kMaxCpg = 160;     // CTAs per group (a B200 has 148 SMs)
-constexpr int kMaxGroups = 64;
-constexpr int kChunk = 4;        // rows per round-robin chunk
-constexpr int kMaxStages = 5;    // K|V stages of phase C
+constexpr int kPub = 8;             // keys per scoring CTA in U
+constexpr int kListWords = 10;      // per list: kPub keys, the next key, padding
+constexpr int kMaxCpg = 160;        // scoring CTAs per group (a B200 has 148 SMs)
+constexpr int kMaxGroups = 16;
+constexpr int kChunk = 4;           // k_bar rows per round-robin chunk
+constexpr int kRowsMax = kThreads;  // k_bar rows a scoring CTA holds: 32 per warp (four 8-row tiles)
+constexpr int kStages = 5;          // K|V stages of an attend CTA (one per warp 0 .. 4)
+constexpr int kCS = 16;             // CTAs per attend cluster
 
-constexpr int kRowsMax = kThreads;  // k_bar rows a CTA scores: 32 per warp (four 8-row tiles)
 template <int D>
 constexpr int row_elems() { return D + 8; }  // padded rows: conflict-free ldmatrix
 template <int D>
 constexpr size_t stage_bytes() { return (size_t)2 * kBlk * row_elems<D>() * 2; }
 
 template <int D>
-struct PfSmem {
-    __nv_bfloat16 Qb[kMaxG][D + 8];
-    __nv_bfloat16 QS[16][D + 8];  // scoring A tile: row 0 bf16(qbar), row 1 the bf16 residual, others 0
+struct ScoreSmem {
+    __nv_bfloat16 QS[16][D + 8];      // A tile: row 0 bf16(sum of the group's queries), row 1 the residual
     uint64_t wtop[kWarps][kPub + 1];  // per-warp best keys, largest first (0: none)
     uint64_t own[kPub + 1];           // this CTA's best keys, largest first
-    uint64_t query[kPub + 1];         // keys ranked in phase B (own[0 .. kPub-1], X)
-    int rpart[kWarps][kPub + 1];
-    int rank[kPub + 1];
-    uint64_t xmax[kWarps];
-    int work_slot[kMaxSlots], work_blk[kMaxSlots];
-    int nwork;
-    int sel[kMaxSlots];
+    alignas(16) uint64_t keys[kRowsMax];  // read two at a time (16-byte loads)
+    alignas(128) __nv_bfloat16 rows[kRowsMax][D + 8];  // k_bar rows (rows past the CTA's share unused)
+};
+
+template <int D>
+struct AttendSmem {
+    __nv_bfloat16 Qb[kMaxG][D + 8];
+    uint64_t u[kMaxCpg * kPub];       // the group's lists
+    int cnt_part[kWarps][kPub * 2 + 1];
+    uint64_t xpart[kWarps];
+    int sel[kMaxSlots];               // slot -> block (-1: empty)
+    int overflow;
     uint64_t wkeys[kCap];
     int nwin;
     RadixSelSmem ss;
-    int bad;
-    float cm[8][32], cl[8][32], co[8][32];
+    float wt[kStages][kMaxG];         // fold: weight of each slot's partial per head
+    float fm[kMaxG], fl[kMaxG];       // fold: largest maximum and weighted sum per head
+    float recv[kMaxG / kCS][kCS][D + 2];  // partials of the heads this CTA combines, from every CTA
+    alignas(128) unsigned char stages[kStages * stage_bytes<D>()];
 };
-// After the fixed part: the CTA's keys (kRowsMax of them), then one region holding first its
-// k_bar rows (kRowsMax padded rows; rows past rcap are read by the scoring tiles but never kept)
-// and later the K|V stages of phase C.
-template <int D>
-constexpr size_t pf_keys_off() { return (sizeof(PfSmem<D>) + 15) & ~(size_t)15; }
-template <int D>
-constexpr size_t pf_region_off() { return (pf_keys_off<D>() + (size_t)kRowsMax * 8 + 127) & ~(size_t)127; }
-template <int D>
-constexpr size_t pf_region_bytes(int rcap, int nstages) {
-    const size_t a = (size_t)(rcap > 0 ? kRowsMax : 0) * row_elems<D>() * 2, b = (size_t)nstages * stage_bytes<D>();
-    return a > b ? a : b;
-}
-template <int D>
-constexpr size_t pf_smem_bytes(int rcap, int nstages) { return pf_region_off<D>() + pf_region_bytes<D>(rcap, nstages); }
 
-// ---------------------------------------------------------------- tagged words
-__device__ __forceinline__ uint64_t ll_word(uint32_t v, uint32_t tag) { return ((uint64_t)v << 32) | tag; }
-__device__ __forceinline__ void ll_st(uint64_t* p, uint64_t w) {
-    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(w) : "memory");
-}
-__device__ __forceinline__ void ll_st2(uint64_t* p, uint64_t a, uint64_t b) {  // p 16-byte aligned
-    asm volatile("st.relaxed.gpu.global.v2.u64 [%0], {%1, %2};" ::"l"(p), "l"(a), "l"(b) : "memory");
-}
-// Reads of other CTAs' words are strong (gpu-scope relaxed): a weak load may be served from a copy
-// that is never refreshed and would not see the writer's update.
-__device__ __forceinline__ uint64_t ll_ld(const uint64_t* p) {
-    uint64_t w;
-    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(w) : "l"(p) : "memory");
-    return w;
-}
-__device__ __forceinline__ void ll_ld2(const uint64_t* p, uint64_t& a, uint64_t& b) {  // p 16-byte aligned
-    asm volatile("ld.relaxed.gpu.global.v2.u64 {%0, %1}, [%2];" : "=l"(a), "=l"(b) : "l"(p) : "memory");
-}
-__device__ __forceinline__ bool ll_ok(uint64_t w, uint32_t tag) { return (uint32_t)w == tag; }
-__device__ __forceinline__ uint32_t ll_val(uint64_t w) { return (uint32_t)(w >> 32); }
-
-// Spins until every word addr(i) (i < n, n <= N) carries the tag; fills w[]; on expiry sets *bad
-// and returns false.  Every round issues all n loads before looking at any of them (no branch on a
-// loaded value between the loads: a GPU does not run past such a branch, so checking each word as
-// it arrives would serialise the round trips).
-template <int N, typename Addr>
-__device__ __forceinline__ bool ll_wait_all(Addr addr, int n, uint64_t (&w)[N], uint32_t tag, const DevCtx& ctx,
-                                            int* bad) {
-    if (n <= 0) return true;
-    uint64_t t0 = 0;
-    while (true) {
-#pragma unroll
-        for (int i = 0; i < N; ++i) w[i] = ll_ld(addr(i < n ? i : n - 1));
-        unsigned miss = 0u;
-#pragma unroll
-        for (int i = 0; i < N; ++i) miss |= (unsigned)((uint32_t)w[i] != tag);
-        if (miss == 0u) return true;
-        const uint64_t t = globaltimer_ns();
-        if (t0 == 0) t0 = t;
-        if (*bad || t - t0 > ctx.wait_limit_ns) {
-            *bad = 1;
-            return false;
-        }
-    }
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&h);
 }
 
 __device__ __forceinline__ uint64_t warp_max_u64(uint64_t x) {
@@ -162,19 +105,14 @@ __device__ __forceinline__ uint64_t warp_max_u64(uint64_t x) {
     return x;
 }
 
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-    const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<const uint32_t*>(&h);
-}
-
-// Exact k-th largest nonzero key among n keys in global memory (the fallback of phase B): one byte
-// at a time from the top, as radix_kth, streaming the keys from memory on every pass.  On return
-// winner(key) = key != 0 && (key & mask) >= prefix picks min(K, #nonzero) keys.
+// Exact k-th largest nonzero key among n keys in global memory (the fallback): one byte at a time
+// from the top, streaming the keys on every pass.  On return winner(key) = key != 0 &&
+// (key & mask) >= prefix picks min(K, #nonzero) keys.
 __device__ void radix_kth_stream(const uint64_t* keys, int n, int K, RadixSelSmem& s, uint64_t& prefix,
                                  uint64_t& mask, int t) {
     const int lane = t & 31, warp = t >> 5;
     int nv = 0;
-    for (int e = t; e < n; e += kThreads) nv += __ldcg(keys + e) != 0ull;
+    for (int e = t; e < n; e += kThreads) nv += keys[e] != 0ull;
     if (t == 0) s.nvalid = 0;
     __syncthreads();
     nv = __reduce_add_sync(0xffffffffu, nv);
@@ -192,7 +130,7 @@ __device__ void radix_kth_stream(const uint64_t* keys, int n, int K, RadixSelSme
         s.hist[t] = 0;
         __syncthreads();
         for (int e = t; e < n; e += kThreads) {
-            const uint64_t key = __ldcg(keys + e);
+            const uint64_t key = keys[e];
             if (key && (key & mask) == prefix) atomicAdd(&s.hist[(key >> shift) & 255u], 1u);
         }
         __syncthreads();
@@ -232,34 +170,16 @@ __device__ void radix_kth_stream(const uint64_t* keys, int n, int K, RadixSelSme
     }
 }
 
-// Workspace region of this path (zeroed before its first use): one tagged word per CTA (it has
-// read the epoch), the published lists, the fallback's keys and arrival words, the owners' block
-// ids per slot and the per-slot partial records, all tagged but the fallback keys.
-struct PfLayout {
-    size_t alive, part, keys, fb, blkid, rec, total;
-};
-PfLayout pf_layout(int groups, int ncand, int slots, int G, int d) {
-    auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
-    PfLayout L;
-    L.alive = 0;
-    L.part = L.alive + up((size_t)groups * kMaxCpg * 8);
-    L.keys = L.part + up((size_t)groups * kPubCopies * kMaxCpg * kPubWords * 8);
-    L.fb = L.keys + up((size_t)groups * (ncand > 0 ? ncand : 1) * 8);
-    L.blkid = L.fb + up((size_t)groups * kMaxCpg * 8);
-    L.rec = L.blkid + up((size_t)groups * kMaxSlots * 8);
-    L.total = L.rec + (size_t)groups * slots * G * (d + 2) * 8;
-    return L;
-}
-
 // One slot's softmax partial, computed by one warp: the block's K and V rows (64 x D, padded rows)
-// in shared memory, the G <= 16 query rows in sm.Qb (padded to 16 with zeros).  The logits are an
+// in shared memory, the G <= 16 query rows in Qs (padded to 16 with zeros).  The logits are an
 // m16n8k16 tile row per head (16 x 64), the softmax runs in registers (a head's row lives in the 4
 // lanes of a quad), and P -- rounded to bf16 -- becomes the A fragments of P V directly.  Writes
-// the record [G][m, l, o_0 .. o_{D-1}] as tagged words, o unnormalised.
+// out[h][0] = the head's maximum logit (log2 units), out[h][1] = the sum of its probabilities and
+// out[h][2 ..] = the unnormalised sum of p v, for heads h < G.
 template <int D>
 __device__ __forceinline__ void slot_partial(const __nv_bfloat16* __restrict__ Qs, const __nv_bfloat16* __restrict__ Ks,
                                              const __nv_bfloat16* __restrict__ Vs, int lim, float scale_log2, int G,
-                                             uint64_t* r, uint32_t tag, int lane) {
+                                             float* out, int lane) {
     constexpr int RE = row_elems<D>();
     const int gq = lane >> 2, t2 = 2 * (lane & 3), mi = lane >> 3, r8 = lane & 7;
     float sc[8][4];
@@ -313,8 +233,8 @@ __device__ __forceinline__ void slot_partial(const __nv_bfloat16* __restrict__ Q
         l0 += __shfl_xor_sync(0xffffffffu, l0, off);
         l1 += __shfl_xor_sync(0xffffffffu, l1, off);
     }
-    // P V in halves of D/2 columns (or all of D = 64): ldmatrix.trans of V gives both B fragments
-    // of two column tiles at once
+    // P V in halves of 64 columns (or all of D = 64): ldmatrix.trans of V gives the B fragments of
+    // two column tiles at once
     constexpr int kHalf = D >= 128 ? 64 : D;
 #pragma unroll
     for (int h0 = 0; h0 < D; h0 += kHalf) {
@@ -335,297 +255,267 @@ __device__ __forceinline__ void slot_partial(const __nv_bfloat16* __restrict__ Q
 #pragma unroll
         for (int n = 0; n < kHalf / 8; ++n) {
             const int col = h0 + 8 * n + t2;
-            if (gq < G)
-                ll_st2(r + gq * (D + 2) + 2 + col, ll_word(__float_as_uint(ov[n][0]), tag),
-                       ll_word(__float_as_uint(ov[n][1]), tag));
+            if (gq < G) *reinterpret_cast<float2*>(out + gq * (D + 2) + 2 + col) = make_float2(ov[n][0], ov[n][1]);
             if (gq + 8 < G)
-                ll_st2(r + (gq + 8) * (D + 2) + 2 + col, ll_word(__float_as_uint(ov[n][2]), tag),
-                       ll_word(__float_as_uint(ov[n][3]), tag));
+                *reinterpret_cast<float2*>(out + (gq + 8) * (D + 2) + 2 + col) = make_float2(ov[n][2], ov[n][3]);
         }
     }
-    // the running maximum is kept in log2 units; the combine takes exponents base 2
     if ((lane & 3) == 0) {
-        if (gq < G) ll_st2(r + gq * (D + 2), ll_word(__float_as_uint(mx0), tag), ll_word(__float_as_uint(l0), tag));
-        if (gq + 8 < G)
-            ll_st2(r + (gq + 8) * (D + 2), ll_word(__float_as_uint(mx1), tag), ll_word(__float_as_uint(l1), tag));
+        if (gq < G) *reinterpret_cast<float2*>(out + gq * (D + 2)) = make_float2(mx0, l0);
+        if (gq + 8 < G) *reinterpret_cast<float2*>(out + (gq + 8) * (D + 2)) = make_float2(mx1, l1);
     }
+}
+
+// Round-robin dealing of a group's candidates to its scoring CTAs: row r of CTA j holds candidate
+// (j + (r / kChunk) * cpg) * kChunk + r % kChunk (block n_init + candidate).
+__device__ __forceinline__ int cand_of_row(int j, int r, int cpg) {
+    return (j + (r / kChunk) * cpg) * kChunk + r % kChunk;
 }
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 2)
-sparse_decode_pf_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kc,
-                        const __nv_bfloat16* __restrict__ vc, const __nv_bfloat16* __restrict__ kbar,
-                        const int32_t* __restrict__ idx_in, int32_t* __restrict__ idx_out,
-                        __nv_bfloat16* __restrict__ o, int H, int Hkv, int pos, int Tmax, int nb_cap,
-                        int topk, int n_init, int n_local, int slots, float scale, int cpg, int rcap,
-                        int nstages, unsigned* epoch, unsigned char* ws, PfLayout lay, DevCtx ctx) {
-    extern __shared__ __align__(128) unsigned char pf_smem_raw[];
-    PfSmem<D>& sm = *reinterpret_cast<PfSmem<D>*>(pf_smem_raw);
-    uint64_t* s_keys = reinterpret_cast<uint64_t*>(pf_smem_raw + pf_keys_off<D>());
-    __nv_bfloat16* s_region = reinterpret_cast<__nv_bfloat16*>(pf_smem_raw + pf_region_off<D>());
-    constexpr int RE = row_elems<D>();
+decode_score_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kbar,
+                    const __nv_bfloat16* __restrict__ kc, const __nv_bfloat16* __restrict__ vc, int H, int Hkv,
+                    int pos, int Tmax, int nb_cap, int n_init, int n_local, int cpg, uint64_t* __restrict__ lists,
+                    uint64_t* __restrict__ allkeys) {
+    extern __shared__ __align__(128) unsigned char score_smem_raw[];
+    ScoreSmem<D>& sm = *reinterpret_cast<ScoreSmem<D>*>(score_smem_raw);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int G = H / Hkv;
     const int bg = blockIdx.x / cpg, j = blockIdx.x % cpg;
     const int64_t b = bg / Hkv;
     const int g = bg % Hkv;
     const int c = pos / kBlk;
-    const int lo = n_init, hi = c - n_local;
-    const int ncand = hi - lo + 1;
-    const int K = topk;
-    // owner mode: the selection is made here and the CTAs attend their own winners
-    const bool owner = idx_in == nullptr && K > 0 && ncand > K;
-    const int nchunks = owner ? (ncand + kChunk - 1) / kChunk : 0;
+    const int lo = n_init;
+    const int ncand = c - n_local - lo + 1;  // > topk >= 1 on this path
+    const int nchunks = (ncand + kChunk - 1) / kChunk;
     const int my_chunks = j < nchunks ? (nchunks - 1 - j) / cpg + 1 : 0;
-    const int nrows = my_chunks * kChunk;  // <= rcap <= kRowsMax
-    const __nv_bfloat16* qg = q + (b * H + (int64_t)g * G) * D;
-    uint64_t* alive = reinterpret_cast<uint64_t*>(ws + lay.alive);
-    uint64_t* part = reinterpret_cast<uint64_t*>(ws + lay.part) + (int64_t)bg * kPubCopies * kMaxCpg * kPubWords;
-    uint64_t* gkeys = reinterpret_cast<uint64_t*>(ws + lay.keys) + (int64_t)bg * (ncand > 0 ? ncand : 1);
-    uint64_t* fbw = reinterpret_cast<uint64_t*>(ws + lay.fb) + (int64_t)bg * kMaxCpg;
-    uint64_t* done = reinterpret_cast<uint64_t*>(ws + lay.blkid) + (int64_t)bg * kMaxSlots;
-    uint64_t* rec = reinterpret_cast<uint64_t*>(ws + lay.rec) + (int64_t)bg * slots * G * (D + 2);
+    const int nrows = my_chunks * kChunk;  // <= kRowsMax (checked at launch)
 
-    // ---------------------------------------------------------------- prefetch of k_bar
-    if (owner && my_chunks > 0) {
-        const __nv_bfloat16* kb = kbar + ((int64_t)bg * nb_cap + lo) * D;
-        for (int e = tid; e < nrows * (D / 8); e += kThreads) {
-            const int r = e / (D / 8), piece = e % (D / 8);
-            const int cand = (j + (r / kChunk) * cpg) * kChunk + r % kChunk;
-            const bool ok = cand < ncand;
-            ptx::cp_async16(s_region + (size_t)r * RE + piece * 8,
-                            kb + (ok ? (int64_t)cand * D + piece * 8 : 0), ok);
-        }
+    // k_bar rows first: they do not depend on the previous kernel
+    const __nv_bfloat16* kb = kbar + ((int64_t)bg * nb_cap + lo) * D;
+    for (int e = tid; e < nrows * (D / 8); e += kThreads) {
+        const int r = e / (D / 8), piece = e % (D / 8);
+        const int cand = cand_of_row(j, r, cpg);
+        const bool ok = cand < ncand;
+        ptx::cp_async16(&sm.rows[r][piece * 8], kb + (ok ? (int64_t)cand * D + piece * 8 : 0), ok);
     }
     ptx::cp_async_commit();
-    // The next kernel in the stream may start now (it waits for this grid before reading anything
-    // this grid writes); this kernel's own reads of q, the cache, idx_in and the workspace wait for
-    // the previous kernel when it was launched as a programmatic dependent.
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    // the attend kernel may start now: its own early reads come after the previous kernel
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
-    const uint32_t tag = 0x7F800001u + __ldcg(epoch) % 0x3FFFFFu;  // 0x7F800001 .. 0x7FBFFFFF
-    if (tid == 0) {
-        sm.bad = 0;
-        ll_st(alive + blockIdx.x, ll_word(1u, tag));
+    if (tid < D) {
+        // every head's load in flight at once (a loop over a runtime G would wait for each load
+        // before issuing the next)
+        const __nv_bfloat16* qg = q + (b * H + (int64_t)g * G) * D + tid;
+        float qv[kMaxG];
+#pragma unroll
+        for (int h = 0; h < kMaxG; ++h) qv[h] = h < G ? __bfloat162float(qg[h * D]) : 0.f;
+        float s = 0.f;
+#pragma unroll
+        for (int h = 0; h < kMaxG; ++h) s += qv[h];
+        const __nv_bfloat16 hi = __float2bfloat16_rn(s);
+        sm.QS[0][tid] = hi;
+        sm.QS[1][tid] = __float2bfloat16_rn(s - __bfloat162float(hi));
     }
-    int* bad = &sm.bad;
-    // ---------------------------------------------------------------- the group's query rows
-    for (int e = tid; e < kMaxG * (D / 8); e += kThreads) {
-        const int h = e / (D / 8), c8 = (e % (D / 8)) * 8;
-        *reinterpret_cast<uint4*>(&sm.Qb[h][c8]) = h < G ? ld16(qg + h * D + c8) : make_uint4(0u, 0u, 0u, 0u);
-    }
+    for (int e = tid; e < 14 * (D / 8); e += kThreads)
+        *reinterpret_cast<uint4*>(&sm.QS[2 + e / (D / 8)][(e % (D / 8)) * 8]) = make_uint4(0u, 0u, 0u, 0u);
+    if (tid <= kPub) sm.own[tid] = 0ull;
+    if (lane <= kPub) sm.wtop[warp][lane] = 0ull;
+    ptx::cp_async_wait<0>();
     __syncthreads();
 
-    bool fallback = false;
-    if (owner) {
-        if (tid < D) {
-            float s = 0.f;
-            for (int h = 0; h < G; ++h) s += __bfloat162float(sm.Qb[h][tid]);
-            const __nv_bfloat16 hi = __float2bfloat16_rn(s);
-            sm.QS[0][tid] = hi;
-            sm.QS[1][tid] = __float2bfloat16_rn(s - __bfloat162float(hi));
-        }
-        for (int e = tid; e < 14 * (D / 8); e += kThreads)
-            *reinterpret_cast<uint4*>(&sm.QS[2 + e / (D / 8)][(e % (D / 8)) * 8]) = make_uint4(0u, 0u, 0u, 0u);
-        if (tid <= kPub) sm.own[tid] = 0ull;
-        if (lane <= kPub) sm.wtop[warp][lane] = 0ull;
-        ptx::cp_async_wait<0>();
-        __syncthreads();
-        // ------------------------------------------------------------ A: scores of this CTA's rows
-        // Warp w scores rows 32w .. 32w+31 as four 8-row tiles at once.  A operand: the QS tile
-        // (row 0 = bf16(qbar), row 1 = bf16(qbar - row 0), the other rows zero), so the two rows
-        // of the result hold the hi and lo parts of each score.
-        {
-            float acc[4][4];
+    // scores: warp w takes rows 32w .. 32w+31 as four 8-row tiles at once; the two rows of each
+    // result hold the hi and lo parts of the scores
+    {
+        float acc[4][4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+        for (int i = 0; i < 4; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
 #pragma unroll
-            for (int ks = 0; ks < D / 16; ++ks) {
-                uint32_t af[4];
-                ldsm_x4(af, &sm.QS[lane & 15][16 * ks + (lane >> 4) * 8]);
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    uint32_t bfr[2];
-                    ldsm_x2(bfr, s_region + (size_t)(32 * warp + 8 * i + (lane & 7)) * RE + 16 * ks + ((lane >> 3) & 1) * 8);
-                    mma16816(acc[i], af, bfr);
-                }
-            }
-            // lanes 0-3: row 0 (hi) at columns 2t, 2t+1 of each tile; lanes 4-7: row 1 (lo)
+        for (int ks = 0; ks < D / 16; ++ks) {
+            uint32_t af[4];
+            ldsm_x4(af, &sm.QS[lane & 15][16 * ks + (lane >> 4) * 8]);
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                const float s0 = acc[i][0] + __shfl_down_sync(0xffffffffu, acc[i][0], 4);
-                const float s1 = acc[i][1] + __shfl_down_sync(0xffffffffu, acc[i][1], 4);
-                if (lane < 4) {
+                uint32_t bfr[2];
+                ldsm_x2(bfr, &sm.rows[32 * warp + 8 * i + (lane & 7)][16 * ks + ((lane >> 3) & 1) * 8]);
+                mma16816(acc[i], af, bfr);
+            }
+        }
 #pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const int r = 32 * warp + 8 * i + 2 * lane + u;
-                        const int cand = (j + (r / kChunk) * cpg) * kChunk + r % kChunk;
-                        s_keys[r] = r < nrows && cand < ncand ? sel_key(u ? s1 : s0, lo + cand) : 0ull;
-                    }
+        for (int i = 0; i < 4; ++i) {
+            const float s0 = acc[i][0] + __shfl_down_sync(0xffffffffu, acc[i][0], 4);
+            const float s1 = acc[i][1] + __shfl_down_sync(0xffffffffu, acc[i][1], 4);
+            if (lane < 4) {
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const int r = 32 * warp + 8 * i + 2 * lane + u;
+                    const int cand = cand_of_row(j, r, cpg);
+                    sm.keys[r] = r < nrows && cand < ncand ? sel_key(u ? s1 : s0, lo + cand) : 0ull;
                 }
             }
         }
-        __syncwarp();
-        // best kPub + 1 keys of the warp's 32 by counting ranks (keys are distinct), then of the
-        // CTA from the warps' lists
-        {
-            const uint64_t x = s_keys[32 * warp + lane];
-            const ulonglong2* kv = reinterpret_cast<const ulonglong2*>(s_keys + 32 * warp);
-            int n = 0;
+    }
+    __syncwarp();
+    // best kPub + 1 keys of the warp's 32 by counting ranks (keys are distinct), then of the CTA
+    {
+        const uint64_t x = sm.keys[32 * warp + lane];
+        const ulonglong2* kv = reinterpret_cast<const ulonglong2*>(sm.keys + 32 * warp);
+        int n = 0;
 #pragma unroll
-            for (int y = 0; y < 16; ++y) {
-                const ulonglong2 pr = kv[y];
-                n += (pr.x > x) + (pr.y > x);
-            }
-            if (x != 0ull && n <= kPub) sm.wtop[warp][n] = x;
+        for (int y = 0; y < 16; ++y) {
+            const ulonglong2 pr = kv[y];
+            n += (pr.x > x) + (pr.y > x);
         }
-        __syncthreads();
-        if (tid < kWarps * (kPub + 1)) {
-            const uint64_t* wt = &sm.wtop[0][0];
-            const uint64_t x = wt[tid];
-            int n = 0;
+        if (x != 0ull && n <= kPub) sm.wtop[warp][n] = x;
+    }
+    __syncthreads();
+    if (tid < kWarps * (kPub + 1)) {
+        const uint64_t* wt = &sm.wtop[0][0];
+        const uint64_t x = wt[tid];
+        int n = 0;
 #pragma unroll 8
-            for (int y = 0; y < kWarps * (kPub + 1); ++y) n += wt[y] > x;
-            if (x != 0ull && n <= kPub) sm.own[n] = x;
-        }
-        __syncthreads();
-        if (tid < kPubCopies * (kPub + 1)) {  // publish: two tagged words per key, in every copy
-            const int t = tid % (kPub + 1), cp = tid / (kPub + 1);
-            const uint64_t x = sm.own[t];
-            ll_st2(part + ((int64_t)cp * kMaxCpg + j) * kPubWords + 2 * t, ll_word((uint32_t)(x >> 32), tag),
-                   ll_word((uint32_t)x, tag));
-        }
+        for (int y = 0; y < kWarps * (kPub + 1); ++y) n += wt[y] > x;
+        if (x != 0ull && n <= kPub) sm.own[n] = x;
+    }
+    __syncthreads();
+    if (tid <= kPub) lists[(int64_t)blockIdx.x * kListWords + tid] = sm.own[tid];
+    // the CTA's two best blocks are likely winners: their K and V rows start towards L2 now, so the
+    // attend kernel finds most of its blocks there (a hint; the selection does not depend on it)
+    if (tid < 4 && sm.own[tid >> 1] != 0ull) {
+        const int blk = key_block(sm.own[tid >> 1]);
+        const __nv_bfloat16* base = (tid & 1) ? vc : kc;
+        ptx::bulk_prefetch_l2(base + ((int64_t)bg * Tmax + (int64_t)blk * kBlk) * D, kBlk * D * 2);
+    }
+    uint64_t* gk = allkeys + (int64_t)bg * ncand;
+    for (int r = tid; r < nrows; r += kThreads) {
+        const int cand = cand_of_row(j, r, cpg);
+        if (cand < ncand) gk[cand] = sm.keys[r];
+    }
+}
 
-        // ------------------------------------------------------------ B: rank own keys within U
-        // thread i < cpg reads list i (its kPub keys and the next one), polling until every word
-        // carries this call's tag, and counts its keys above each of this CTA's keys
-        int cnt[kPub + 1];
-        uint64_t x = 0, ukey[kPub];
-#pragma unroll
-        for (int qq = 0; qq <= kPub; ++qq) cnt[qq] = 0;
-#pragma unroll
-        for (int t = 0; t < kPub; ++t) ukey[t] = 0ull;
-        if (tid < cpg) {
-            uint64_t w[2 * (kPub + 1)];
-            const uint64_t* lst = part + ((int64_t)(j % kPubCopies) * kMaxCpg + tid) * kPubWords;
-            {  // the list's words are their own readiness flags: one round trip after they land
-                uint64_t t0 = 0;
-                while (true) {
-#pragma unroll
-                    for (int i = 0; i <= kPub; ++i) ll_ld2(lst + 2 * i, w[2 * i], w[2 * i + 1]);
-                    unsigned miss = 0u;
-#pragma unroll
-                    for (int i = 0; i < 2 * (kPub + 1); ++i) miss |= (unsigned)((uint32_t)w[i] != tag);
-                    if (miss == 0u) break;
-                    const uint64_t t = globaltimer_ns();
-                    if (t0 == 0) t0 = t;
-                    if (*bad || t - t0 > ctx.wait_limit_ns) {
-                        *bad = 1;
-                        break;
-                    }
-                }
-            }
-            uint64_t mine[kPub];
-#pragma unroll
-            for (int qq = 0; qq < kPub; ++qq) mine[qq] = sm.own[qq];
-#pragma unroll
-            for (int t = 0; t < kPub; ++t) {
-                ukey[t] = ((uint64_t)ll_val(w[2 * t]) << 32) | ll_val(w[2 * t + 1]);
-#pragma unroll
-                for (int qq = 0; qq < kPub; ++qq) cnt[qq] += ukey[t] > mine[qq];
-            }
-            x = ((uint64_t)ll_val(w[2 * kPub]) << 32) | ll_val(w[2 * kPub + 1]);
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+decode_attend_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kc,
+                     const __nv_bfloat16* __restrict__ vc, const int32_t* __restrict__ idx_in,
+                     int32_t* __restrict__ idx_out, __nv_bfloat16* __restrict__ o, int H, int Hkv, int pos,
+                     int Tmax, int topk, int n_init, int n_local, int slots, float scale, int cpg, bool early,
+                     const uint64_t* __restrict__ lists, const uint64_t* __restrict__ allkeys, DevCtx ctx) {
+    extern __shared__ __align__(128) unsigned char attend_smem_raw[];
+    AttendSmem<D>& sm = *reinterpret_cast<AttendSmem<D>*>(attend_smem_raw);
+    constexpr int RE = row_elems<D>();
+    cg::cluster_group cl = cg::this_cluster();
+    constexpr int CS = kCS;  // the launch's cluster size
+    const int rk = (int)cl.block_rank();
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int G = H / Hkv;
+    const int bg = blockIdx.x / CS;
+    const int64_t b = bg / Hkv;
+    const int g = bg % Hkv;
+    const int c = pos / kBlk;
+    const int lo = n_init;
+    const int ncand = c - n_local - lo + 1;
+    const int K = topk;
+    const bool owner = cpg > 0;  // the score kernel ran: the selection is made here
+    const int nitems = rk < slots ? (slots - 1 - rk) / CS + 1 : 0;  // slots rk, rk + CS, ... (<= kStages)
+    const __nv_bfloat16* qg = q + (b * H + (int64_t)g * G) * D;
+    const float scale_log2 = scale * 1.4426950408889634f;
+    auto stage_k = [&](int w) { return reinterpret_cast<__nv_bfloat16*>(sm.stages + (size_t)w * stage_bytes<D>()); };
+    auto issue = [&](int w, int blk) {  // warp w's lanes copy block blk's K and V rows into stage w
+        __nv_bfloat16* sk = stage_k(w);
+        __nv_bfloat16* sv = sk + kBlk * RE;
+        const __nv_bfloat16* kb = kc + ((int64_t)bg * Tmax + (int64_t)blk * kBlk) * D;
+        const __nv_bfloat16* vb = vc + ((int64_t)bg * Tmax + (int64_t)blk * kBlk) * D;
+        const int lim = min(kBlk - 1, pos - blk * kBlk);
+        for (int e = lane; e < kBlk * (D / 8); e += 32) {
+            const int row = e / (D / 8), c8 = (e % (D / 8)) * 8;
+            const bool ok = row <= lim;
+            ptx::cp_async16(sk + row * RE + c8, kb + (ok ? (int64_t)row * D + c8 : 0), ok);
+            ptx::cp_async16(sv + row * RE + c8, vb + (ok ? (int64_t)row * D + c8 : 0), ok);
         }
+        ptx::cp_async_commit();
+    };
+    // init and local blocks: slots K .. K + n_init + n_local - 1 on the rank path
+    auto forced_block = [&](int s) { const int f = s - K; return f < n_init ? f : c - n_local + 1 + (f - n_init); };
+
+    // ---------------------------------------------------------------- before the score kernel ends
+    // (only when it ran: its predecessor has then completed, so q and the cache are final)
+    bool preloaded = false;
+    if (early) {
+        for (int e = tid; e < kMaxG * (D / 8); e += kThreads) {
+            const int h = e / (D / 8), c8 = (e % (D / 8)) * 8;
+            *reinterpret_cast<uint4*>(&sm.Qb[h][c8]) = h < G ? ld16(qg + h * D + c8) : make_uint4(0u, 0u, 0u, 0u);
+        }
+        if (warp < nitems && rk + warp * CS >= K) {
+            issue(warp, forced_block(rk + warp * CS));
+            preloaded = true;
+        }
+    }
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    cl.sync();  // every CTA of the cluster runs before any reaches into another's shared memory
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (!early) {
+        for (int e = tid; e < kMaxG * (D / 8); e += kThreads) {
+            const int h = e / (D / 8), c8 = (e % (D / 8)) * 8;
+            *reinterpret_cast<uint4*>(&sm.Qb[h][c8]) = h < G ? ld16(qg + h * D + c8) : make_uint4(0u, 0u, 0u, 0u);
+        }
+    }
+
+    // ---------------------------------------------------------------- the slot list
+    bool rank_layout = false;  // slots 0 .. K-1: the winners ascending by block, then the forced blocks
+    if (owner) {
+        // U, the group's lists, in registers; the K-th largest key of U by a radix select
+        const int nu = cpg * kPub;
+        const uint64_t* gl = lists + (int64_t)bg * cpg * kListWords;
+        constexpr int kU = (kMaxCpg * kPub + kThreads - 1) / kThreads;
+        uint64_t uv[kU];
+#pragma unroll
+        for (int i = 0; i < kU; ++i) {
+            const int e = tid + kThreads * i;
+            uv[i] = e < nu ? gl[(e / kPub) * kListWords + e % kPub] : 0ull;
+        }
+        uint64_t x = tid < cpg ? gl[tid * kListWords + kPub] : 0ull;  // cpg <= kThreads
         x = warp_max_u64(x);
-        if (lane == 0) sm.xmax[warp] = x;
+        if (lane == 0) sm.xpart[warp] = x;
+        if (tid == 0) sm.nwin = 0;
+        uint64_t prefix, mask;
+        radix_kth<kU>(uv, K, sm.ss, prefix, mask, tid, [] { __syncthreads(); });
+        uint64_t X = 0ull;
 #pragma unroll
-        for (int qq = 0; qq < kPub; ++qq) {
-            const int n = __reduce_add_sync(0xffffffffu, cnt[qq]);
-            if (lane == 0) sm.rpart[warp][qq] = n;
-        }
-        __syncthreads();
-        if (sm.bad) {
-            if (tid == 0) {
-                flag(ctx, kStatusTimeout);
-                atomicAdd(epoch, 1u);
+        for (int w = 0; w < kWarps; ++w) X = sm.xpart[w] > X ? sm.xpart[w] : X;
+        // X, the largest key a list left out, would be a winner: the lists may hide winners.  (With
+        // fewer than K keys in U every key of U wins, and some list left keys out.)
+        const bool all_win = mask == ~0ull && prefix == 1ull;
+        rank_layout = all_win ? X == 0ull : !(X != 0ull && (X & mask) >= prefix);
+        if (rank_layout) {
+#pragma unroll
+            for (int i = 0; i < kU; ++i) {
+                if (uv[i] != 0ull && (uv[i] & mask) >= prefix) {
+                    const int w = atomicAdd(&sm.nwin, 1);
+                    if (w < kCap) sm.wkeys[w] = uv[i];
+                }
             }
-            return;
-        }
-        if (tid == 0) {
-            uint64_t m = 0;
-            for (int w = 0; w < kWarps; ++w) m = sm.xmax[w] > m ? sm.xmax[w] : m;
-            sm.query[kPub] = m;
-        }
-        __syncthreads();
-        // X, the largest next key of any list: the number of published keys above it
-        {
-            const uint64_t X = sm.query[kPub];
-#pragma unroll
-            for (int t = 0; t < kPub; ++t) cnt[kPub] += ukey[t] > X;
-        }
-        {
-            const int n = __reduce_add_sync(0xffffffffu, cnt[kPub]);
-            if (lane == 0) sm.rpart[warp][kPub] = n;
-        }
-        __syncthreads();
-        if (tid <= kPub) {
-            int n = 0;
-            for (int w = 0; w < kWarps; ++w) n += sm.rpart[w][tid];
-            sm.rank[tid] = n;
-        }
-        __syncthreads();
-        fallback = sm.query[kPub] != 0ull && sm.rank[kPub] < K;
-        if (!fallback) {
-            if (tid == 0) {
-                int n = 0;
-                for (int t = 0; t < kPub; ++t) {
-                    if (sm.own[t] != 0ull && sm.rank[t] < K) {
-                        sm.work_slot[n] = sm.rank[t];
-                        sm.work_blk[n] = key_block(sm.own[t]);
-                        ++n;
-                    }
-                }
-                // init and local blocks: slots K .. slots-1, one per CTA from the last CTA down
-                const int nf = n_init + n_local;
-                for (int f = 0; f < nf; ++f) {
-                    if ((cpg - 1 - (f % cpg)) != j) continue;
-                    sm.work_slot[n] = K + f;
-                    sm.work_blk[n] = f < n_init ? f : c - n_local + 1 + (f - n_init);
-                    ++n;
-                }
-                sm.nwork = n;
+            for (int f = tid; f < n_init + n_local; f += kThreads) sm.sel[K + f] = forced_block(K + f);
+            __syncthreads();
+            if (warp == 0) {
+                const int nw = min(sm.nwin, K);
+                int x0 = 2 * lane < nw ? key_block(sm.wkeys[2 * lane]) : 0x7fffffff;
+                int x1 = 2 * lane + 1 < nw ? key_block(sm.wkeys[2 * lane + 1]) : 0x7fffffff;
+                warp_sort64(x0, x1, lane);
+                if (2 * lane < K) sm.sel[2 * lane] = 2 * lane < nw ? x0 : -1;
+                if (2 * lane + 1 < K) sm.sel[2 * lane + 1] = 2 * lane + 1 < nw ? x1 : -1;
             }
         } else {
-            // every CTA publishes all its keys, then all meet (tagged arrival words); the winners of
-            // an exact top-k over all of them, ascending by block, fill the slots between the init
-            // and the local blocks
-            for (int r = tid; r < nrows; r += kThreads) {
-                const int cand = (j + (r / kChunk) * cpg) * kChunk + r % kChunk;
-                if (cand < ncand) gkeys[cand] = s_keys[r];
-            }
-            __threadfence();
-            __syncthreads();
-            if (tid == 0) ll_st(fbw + j, ll_word(1u, tag));
-            {
-                uint64_t ww[1];
-                ll_wait_all([&](int) { return fbw + min(tid, cpg - 1); }, 1, ww, tag, ctx, bad);
-            }
-            __threadfence();
-            __syncthreads();
-            if (sm.bad) {
-                if (tid == 0) {
-                    flag(ctx, kStatusTimeout);
-                    atomicAdd(epoch, 1u);
-                }
-                return;
-            }
+            // exact top-k over all the group's keys (written by the score kernel); the winners,
+            // ascending by block, fill the slots between the init and the local blocks
             uint64_t prefix, mask;
-            radix_kth_stream(gkeys, ncand, K, sm.ss, prefix, mask, tid);
+            const uint64_t* gk = allkeys + (int64_t)bg * ncand;
+            radix_kth_stream(gk, ncand, K, sm.ss, prefix, mask, tid);
             if (tid == 0) sm.nwin = 0;
             __syncthreads();
             for (int e = tid; e < ncand; e += kThreads) {
-                const uint64_t key = __ldcg(gkeys + e);
+                const uint64_t key = gk[e];
                 if (key && (key & mask) >= prefix) {
                     const int w = atomicAdd(&sm.nwin, 1);
                     if (w < kCap) sm.wkeys[w] = key;
@@ -644,296 +534,276 @@ sparse_decode_pf_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16
                 for (int s = n_init + K + n_local + lane; s < slots; s += 32) sm.sel[s] = -1;
             }
         }
+    } else if (idx_in) {
+        // a given selection: entries past the query's block are flagged and left out
+        for (int s = tid; s < slots; s += kThreads) {
+            int blk = idx_in[(int64_t)bg * slots + s];
+            if (blk > c) {
+                flag(ctx, kStatusBounds);
+                blk = -1;
+            }
+            sm.sel[s] = blk;
+        }
+    } else if (ncand <= K) {
+        for (int s = tid; s < slots; s += kThreads) sm.sel[s] = s <= c ? s : -1;  // every block 0 .. c
     } else {
-        // list paths: the given selection (entries past the query's block flagged and left out),
-        // or every block 0 .. c when there are at most k candidates, or the init and local blocks
-        // when k = 0
-        if (idx_in) {
-            for (int s = tid; s < slots; s += kThreads) {
-                int blk = idx_in[(int64_t)bg * slots + s];
-                if (blk > c) {
-                    flag(ctx, kStatusBounds);
-                    blk = -1;
-                }
-                sm.sel[s] = blk;
-            }
-        } else if (ncand <= K) {
-            for (int s = tid; s < slots; s += kThreads) sm.sel[s] = s <= c ? s : -1;
-        } else {
-            for (int s = tid; s < slots; s += kThreads) {
-                int blk = -1;
-                if (s < n_init) blk = s;
-                else if (s < n_init + n_local) blk = c - n_local + 1 + (s - n_init);
-                sm.sel[s] = blk;
-            }
+        for (int s = tid; s < slots; s += kThreads) {  // k = 0: the init and local blocks
+            int blk = -1;
+            if (s < n_init) blk = s;
+            else if (s < n_init + n_local) blk = c - n_local + 1 + (s - n_init);
+            sm.sel[s] = blk;
         }
     }
     __syncthreads();
-    if (!owner || fallback) {
-        if (tid == 0) {
-            int n = 0;
-            for (int s = j; s < slots; s += cpg) {
-                sm.work_slot[n] = s;
-                sm.work_blk[n] = sm.sel[s];
-                ++n;
-            }
-            sm.nwork = n;
-        }
-    }
-    __syncthreads();  // also: every thread is done with the k_bar rows the stages now overwrite
 
-    // CTA 0 requests every CTA's alive word now and looks at them at the end (see there)
-    uint64_t alive_w = 0;
-    if (blockIdx.x == 0 && tid < (int)gridDim.x) alive_w = ll_ld(alive + tid);
-
-    // ---------------------------------------------------------------- C: per-slot partials
-    // Warp w < nstages attends items w, w + nstages, ... in its own stage: its lanes request the
-    // block's K and V rows (16-byte asynchronous copies; rows past the query zero-filled), wait for
-    // their own copies, and compute the slot's partial.  The slot's done word (tagged, carrying the
-    // block id) follows its record.
-    const int nwork = sm.nwork;
-    const float scale_log2 = scale * 1.4426950408889634f;
-    if (warp < nstages) {
-        __nv_bfloat16* sk = s_region + (size_t)warp * (stage_bytes<D>() / 2);
-        __nv_bfloat16* sv = sk + kBlk * RE;
-        for (int w = warp; w < nwork; w += nstages) {
-            const int slot = sm.work_slot[w];
-            const int blk = sm.work_blk[w];
-            uint64_t* r = rec + (int64_t)slot * G * (D + 2);
-            if (blk < 0) {
-                for (int hh = 0; hh < G; ++hh) {
-                    for (int e = lane; e < D + 2; e += 32) {
-                        const float v = e == 0 ? -INFINITY : 0.f;
-                        ll_st(r + hh * (D + 2) + e, ll_word(__float_as_uint(v), tag));
-                    }
+    // ---------------------------------------------------------------- attention of this CTA's slots
+    // warp w < nitems attends slot rk + w CS in stage w and leaves the slot's partial (per head:
+    // max, sum, sum of p v) at the start of the stage
+    if (warp < nitems) {
+        const int blk = sm.sel[rk + warp * CS];
+        float* out = reinterpret_cast<float*>(stage_k(warp));
+        if (blk >= 0) {
+            if (!(preloaded && rank_layout)) {  // the early copy is this slot's block only on the rank path
+                if (preloaded) {
+                    ptx::cp_async_wait<0>();
+                    __syncwarp();
                 }
-            } else {
-                const __nv_bfloat16* kblk = kc + ((int64_t)bg * Tmax + (int64_t)blk * kBlk) * D;
-                const __nv_bfloat16* vblk = vc + ((int64_t)bg * Tmax + (int64_t)blk * kBlk) * D;
-                const int lim = min(kBlk - 1, pos - blk * kBlk);
-                for (int e = lane; e < kBlk * (D / 8); e += 32) {
-                    const int row = e / (D / 8), c8 = (e % (D / 8)) * 8;
-                    const bool ok = row <= lim;
-                    ptx::cp_async16(sk + row * RE + c8, kblk + (ok ? (int64_t)row * D + c8 : 0), ok);
-                    ptx::cp_async16(sv + row * RE + c8, vblk + (ok ? (int64_t)row * D + c8 : 0), ok);
-                }
-                ptx::cp_async_commit();
-                ptx::cp_async_wait<0>();
-                __syncwarp();
-                slot_partial<D>(&sm.Qb[0][0], sk, sv, lim, scale_log2, G, r, tag, lane);
-                __syncwarp();  // the stage is reloaded by the warp's next item
+                issue(warp, blk);
             }
+            ptx::cp_async_wait<0>();
             __syncwarp();
-            if (lane == 0) ll_st(done + slot, ll_word((uint32_t)blk, tag));
-        }
-    }
-
-    // ---------------------------------------------------------------- D: combine, idx_out
-    // idx_out comes from a CTA without a combine item when there is one
-    if (idx_out && j == (cpg > G * (D / 32) ? cpg - 1 : 0)) {
-        if (owner && !fallback) {
-            if (warp == 0) {
-                uint64_t ww[2];
-                ll_wait_all([&](int i) { return done + min(2 * lane + i, K - 1); }, 2, ww, tag, ctx, bad);
-                int x0 = 2 * lane < K ? (int)ll_val(ww[0]) : 0x7fffffff;
-                int x1 = 2 * lane + 1 < K ? (int)ll_val(ww[1]) : 0x7fffffff;
-                warp_sort64(x0, x1, lane);
-                int32_t* dst = idx_out + (int64_t)bg * slots;
-                for (int s = lane; s < n_init; s += 32) dst[s] = s;
-                if (2 * lane < K) dst[n_init + 2 * lane] = x0;
-                if (2 * lane + 1 < K) dst[n_init + 2 * lane + 1] = x1;
-                for (int t = lane; t < n_local; t += 32) dst[n_init + K + t] = c - n_local + 1 + t;
-                for (int s = n_init + K + n_local + lane; s < slots; s += 32) dst[s] = -1;
-            }
+            const __nv_bfloat16* sk = stage_k(warp);
+            const int lim = min(kBlk - 1, pos - blk * kBlk);
+            slot_partial<D>(&sm.Qb[0][0], sk, sk + kBlk * RE, lim, scale_log2, G, out, lane);
         } else {
-            for (int s = tid; s < slots; s += kThreads) idx_out[(int64_t)bg * slots + s] = sm.sel[s];
+            ptx::cp_async_wait<0>();
+            __syncwarp();
+            for (int e = lane; e < G * (D + 2); e += 32) out[e] = e % (D + 2) == 0 ? -INFINITY : 0.f;
         }
     }
-    constexpr int kPerWarp = (kMaxSlots + kWarps - 1) / kWarps;
-    const int nmine = warp < slots ? (slots - 1 - warp) / kWarps + 1 : 0;  // warp w folds slots w, w+8, ..
-    for (int item = j; item < G * (D / 32); item += cpg) {
-        const int hh = item / (D / 32), d0 = (item % (D / 32)) * 32;
-        // wait for the warp's slots (lane i polls the m word of slot warp + 8 i), then read their
-        // records (every word checked again; a word not yet visible is read again)
-        {
-            uint64_t ww[1];
-            if (lane < nmine)
-                ll_wait_all([&](int) { return rec + ((int64_t)(warp + kWarps * lane) * G + hh) * (D + 2); }, 1, ww,
-                            tag, ctx, bad);
-            __syncwarp();
-        }
-        float ms[kPerWarp], ls[kPerWarp], os[kPerWarp];
-        {
-            uint64_t ww[3 * kPerWarp];
-            auto addr = [&](int i) -> const uint64_t* {
-                const int s = warp + kWarps * (i / 3), part3 = i % 3;
-                return rec + ((int64_t)s * G + hh) * (D + 2) + (part3 < 2 ? part3 : 2 + d0 + lane);
-            };
-            ll_wait_all(addr, 3 * nmine, ww, tag, ctx, bad);
-#pragma unroll
-            for (int i = 0; i < kPerWarp; ++i) {
-                ms[i] = -INFINITY;
-                ls[i] = os[i] = 0.f;
-                if (i < nmine) {
-                    ms[i] = __uint_as_float(ll_val(ww[3 * i]));
-                    ls[i] = __uint_as_float(ll_val(ww[3 * i + 1]));
-                    os[i] = __uint_as_float(ll_val(ww[3 * i + 2]));
-                }
-            }
-        }
+    __syncthreads();
+    // fold the CTA's slots into one partial per head: per head the largest maximum over the slots
+    // and each slot's weight 2^(m - M), then the weighted sums; the partial of head h goes straight
+    // into the shared memory of CTA h mod kCS, which combines that head
+    if (tid < G) {
+        const int h = tid;
+        float m[kStages];
         float M = -INFINITY;
 #pragma unroll
-        for (int i = 0; i < kPerWarp; ++i) M = fmaxf(M, ms[i]);
-        float L = 0.f, acc = 0.f;
-        if (M != -INFINITY) {
-#pragma unroll
-            for (int i = 0; i < kPerWarp; ++i) {
-                if (ms[i] == -INFINITY) continue;
-                const float w8 = exp2f(ms[i] - M);
-                L = fmaf(ls[i], w8, L);
-                acc = fmaf(os[i], w8, acc);
-            }
+        for (int t = 0; t < kStages; ++t) {
+            m[t] = t < nitems ? reinterpret_cast<const float*>(stage_k(t))[h * (D + 2)] : -INFINITY;
+            M = fmaxf(M, m[t]);
         }
-        sm.cm[warp][lane] = M;
-        sm.cl[warp][lane] = L;
-        sm.co[warp][lane] = acc;
-        __syncthreads();
-        if (warp == 0 && !sm.bad) {
-            float Mt = -INFINITY;
+        float L = 0.f;
 #pragma unroll
-            for (int w = 0; w < kWarps; ++w) Mt = fmaxf(Mt, sm.cm[w][lane]);
-            float Lt = 0.f, At = 0.f;
-            if (Mt != -INFINITY) {
-#pragma unroll
-                for (int w = 0; w < kWarps; ++w) {
-                    if (sm.cm[w][lane] == -INFINITY) continue;
-                    const float a = exp2f(sm.cm[w][lane] - Mt);
-                    Lt += a * sm.cl[w][lane];
-                    At += a * sm.co[w][lane];
-                }
-            }
-            o[(b * H + (int64_t)g * G + hh) * D + d0 + lane] = __float2bfloat16_rn(Lt > 0.f ? At / Lt : 0.f);
+        for (int t = 0; t < kStages; ++t) {
+            const float w8 = m[t] == -INFINITY ? 0.f : exp2f(m[t] - M);
+            sm.wt[t][h] = w8;
+            if (t < nitems) L = fmaf(reinterpret_cast<const float*>(stage_k(t))[h * (D + 2) + 1], w8, L);
         }
-        __syncthreads();
-    }
-    // The epoch advances once every CTA of the grid has read it (each tagged its alive word after
-    // reading it), so the next call on this workspace uses a new tag.
-    if (blockIdx.x == 0) {
-        for (int i0 = 0; i0 < (int)gridDim.x; i0 += kThreads) {
-            if (i0 == 0 && (tid >= (int)gridDim.x || ll_ok(alive_w, tag))) continue;
-            uint64_t ww[1];
-            ll_wait_all([&](int) { return alive + min(i0 + tid, (int)gridDim.x - 1); }, 1, ww, tag, ctx, bad);
-        }
-        __syncthreads();
-        if (tid == 0 && !sm.bad) atomicAdd(epoch, 1u);
+        sm.fm[h] = M;
+        sm.fl[h] = L;
     }
     __syncthreads();
-    if (sm.bad && tid == 0) {
-        flag(ctx, kStatusTimeout);
-        atomicAdd(epoch, 1u);
+    for (int e = tid; e < G * (D + 2); e += kThreads) {
+        const int h = e / (D + 2), col = e % (D + 2);
+        float v;
+        if (col == 0) {
+            v = sm.fm[h];
+        } else if (col == 1) {
+            v = sm.fl[h];
+        } else {
+            float pv[kStages];
+#pragma unroll
+            for (int t = 0; t < kStages; ++t)
+                pv[t] = t < nitems ? reinterpret_cast<const float*>(stage_k(t))[h * (D + 2) + col] : 0.f;
+            v = 0.f;
+#pragma unroll
+            for (int t = 0; t < kStages; ++t) v = fmaf(pv[t], sm.wt[t][h], v);
+        }
+        *cl.map_shared_rank(&sm.recv[h / kCS][rk][col], h % kCS) = v;
     }
+    cl.sync();  // every CTA's partials have landed where they are combined
+    // CTA rk combines heads rk, rk + kCS, ... over the partials of every CTA of the cluster
+    for (int h = rk; h < G; h += kCS) {
+        if (tid < D) {
+            const int hh = h / kCS;
+            float mp[kCS], lp[kCS], op[kCS];
+#pragma unroll
+            for (int p = 0; p < kCS; ++p) {
+                mp[p] = sm.recv[hh][p][0];
+                lp[p] = sm.recv[hh][p][1];
+                op[p] = sm.recv[hh][p][2 + tid];
+            }
+            float M = -INFINITY;
+#pragma unroll
+            for (int p = 0; p < kCS; ++p) M = fmaxf(M, mp[p]);
+            float L = 0.f, A = 0.f;
+#pragma unroll
+            for (int p = 0; p < kCS; ++p) {
+                const float w8 = mp[p] == -INFINITY ? 0.f : exp2f(mp[p] - M);
+                L = fmaf(lp[p], w8, L);
+                A = fmaf(op[p], w8, A);
+            }
+            o[(b * H + (int64_t)g * G + h) * D + tid] = __float2bfloat16_rn(L > 0.f ? A / L : 0.f);
+        }
+    }
+    if (idx_out && rk == 0) {
+        int32_t* dst = idx_out + (int64_t)bg * slots;
+        if (rank_layout) {
+            for (int s = tid; s < n_init; s += kThreads) dst[s] = s;
+            for (int s = tid; s < K; s += kThreads) dst[n_init + s] = sm.sel[s];
+            for (int t = tid; t < n_local; t += kThreads) dst[n_init + K + t] = c - n_local + 1 + t;
+        } else {
+            for (int s = tid; s < slots; s += kThreads) dst[s] = sm.sel[s];
+        }
+    }
+}
+
+struct PfLayout {
+    size_t lists, keys, total;
+};
+PfLayout pf_layout(int groups, int ncand) {
+    auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    PfLayout L;
+    L.lists = 0;
+    L.keys = up((size_t)groups * kMaxCpg * kListWords * sizeof(uint64_t));
+    L.total = L.keys + (size_t)groups * (ncand > 0 ? ncand : 1) * sizeof(uint64_t);
+    return L;
+}
+
+struct DevInfo {
+    int nsm = 0, clusters = 0;
+};
+
+template <int D>
+cudaError_t dev_info(DevInfo* out) {
+    constexpr int kMaxDev = 64;
+    static std::mutex mu;
+    static DevInfo info[kMaxDev];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDev) return cudaErrorNotSupported;
+    std::lock_guard<std::mutex> lk(mu);
+    if (info[dev].nsm == 0) {
+        DevInfo d;
+        e = cudaDeviceGetAttribute(&d.nsm, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(decode_score_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)sizeof(ScoreSmem<D>));
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(decode_attend_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)sizeof(AttendSmem<D>));
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(decode_attend_kernel<D>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (e != cudaSuccess) return e;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(kCS);
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = sizeof(AttendSmem<D>);
+        cudaLaunchAttribute at[1];
+        at[0].id = cudaLaunchAttributeClusterDimension;
+        at[0].val.clusterDim.x = kCS;
+        at[0].val.clusterDim.y = 1;
+        at[0].val.clusterDim.z = 1;
+        cfg.attrs = at;
+        cfg.numAttrs = 1;
+        e = cudaOccupancyMaxActiveClusters(&d.clusters, decode_attend_kernel<D>, &cfg);
+        if (e != cudaSuccess) {
+            cudaGetLastError();
+            d.clusters = -1;  // no clusters of this size: this path is never taken
+        }
+        info[dev] = d;
+    }
+    *out = info[dev];
+    return cudaSuccess;
 }
 
 template <int D>
 cudaError_t pf(const void* q, const void* kc, const void* vc, const void* kbar, const int32_t* idx_in,
                int32_t* idx_out, void* o, int B, int H, int Hkv, int pos, int Tmax, int nb_cap, int topk,
-               int n_init, int n_local, float scale, unsigned* epoch, void* ws, size_t ws_bytes, bool pdl,
-               cudaStream_t st, DevCtx ctx) {
+               int n_init, int n_local, float scale, void* ws, size_t ws_bytes, bool pdl, cudaStream_t st,
+               DevCtx ctx) {
     const int slots = n_init + n_local + topk;
     const int G = H / Hkv;
     const int groups = B * Hkv;
-    const int c = pos / kBlk;
-    const int ncand = c - n_local - n_init + 1;
-    if (topk > kCap || slots > kMaxSlots || G > kMaxG || groups > kMaxGroups) return cudaErrorNotSupported;
-    auto kern = sparse_decode_pf_kernel<D>;
-    const int smem_max = (int)pf_smem_bytes<D>(kRowsMax, kMaxStages);
-    constexpr int kMaxDev = 64;
-    static std::mutex mu;
-    static int occ_of[kMaxDev] = {}, nsm_of[kMaxDev] = {};
-    int occ = 0, nsm = 0;
-    {
-        int dev = 0;
-        cudaError_t e = cudaGetDevice(&dev);
-        if (e != cudaSuccess) return e;
-        if (dev < 0 || dev >= kMaxDev) return cudaErrorNotSupported;
-        std::lock_guard<std::mutex> lk(mu);
-        if (occ_of[dev] == 0) {
-            e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_max);
-            if (e != cudaSuccess) return e;
-            int oc = 0, n = 0;
-            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&oc, kern, kThreads, smem_max);
-            if (e != cudaSuccess) return e;
-            e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-            if (e != cudaSuccess) return e;
-            if (oc < 1) return cudaErrorNotSupported;
-            occ_of[dev] = oc;
-            nsm_of[dev] = n;
-        }
-        occ = occ_of[dev];
-        nsm = nsm_of[dev];
-    }
-    int cpg = min(occ * nsm / groups, kMaxCpg);
-    if (cpg < 1) return cudaErrorNotSupported;
+    const int ncand = pos / kBlk - n_local - n_init + 1;
+    if (topk > kCap || slots > kMaxSlots || slots > kStages * kCS || G > kMaxG || groups > kMaxGroups)
+        return cudaErrorNotSupported;
+    DevInfo info;
+    cudaError_t e = dev_info<D>(&info);
+    if (e != cudaSuccess) return e;
+    if (info.clusters < groups) return cudaErrorNotSupported;  // every group's cluster resident at once
     const bool owner = idx_in == nullptr && topk > 0 && ncand > topk;
-    int rcap = 0, nstages = 1;  // k_bar rows a CTA holds (a multiple of 8), K|V stages
+    int cpg = 0;
     if (owner) {
+        cpg = min(kMaxCpg, info.nsm / groups);
+        if (cpg < 1) return cudaErrorNotSupported;
         const int nchunks = (ncand + kChunk - 1) / kChunk;
-        rcap = (nchunks + cpg - 1) / cpg * kChunk;
-        if (rcap > kRowsMax) return cudaErrorNotSupported;
-        nstages = kMaxStages;
-    } else {
-        cpg = min(cpg, max(slots, G * (D / 32)));
-        nstages = min(kMaxStages, (slots + cpg - 1) / cpg);
+        if ((nchunks + cpg - 1) / cpg * kChunk > kRowsMax) return cudaErrorNotSupported;
     }
-    const int smem = (int)pf_smem_bytes<D>(rcap, nstages);
-    const PfLayout lay = pf_layout(groups, ncand > 0 ? ncand : 0, slots, G, D);
+    const PfLayout lay = pf_layout(groups, ncand);
     if (lay.total > ws_bytes) return cudaErrorNotSupported;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(groups * cpg));
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = (size_t)smem;
-    cfg.stream = st;
-    // All CTAs must be resident at once (they wait for one another's words).  A plain call
-    // launches cooperatively.  A programmatic dependent launches with the grid sized to the
-    // occupancy instead: its CTAs may wait for resources that the previous kernel frees as it
-    // finishes, and every CTA of this grid runs before any kernel that waits for this one can
-    // start (those start only once all CTAs here have executed griddepcontrol.launch_dependents).
-    cudaLaunchAttribute attr[1];
-    if (pdl) {
-        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[0].val.programmaticStreamSerializationAllowed = 1;
-    } else {
-        attr[0].id = cudaLaunchAttributeCooperative;
-        attr[0].val.cooperative = 1;
+    unsigned char* w = static_cast<unsigned char*>(ws);
+    uint64_t* lists = reinterpret_cast<uint64_t*>(w + lay.lists);
+    uint64_t* keys = reinterpret_cast<uint64_t*>(w + lay.keys);
+    const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(q);
+    cudaLaunchAttribute pdl_attr;
+    pdl_attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl_attr.val.programmaticStreamSerializationAllowed = 1;
+    if (owner) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)(groups * cpg));
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = sizeof(ScoreSmem<D>);
+        cfg.stream = st;
+        cfg.attrs = &pdl_attr;
+        cfg.numAttrs = pdl ? 1 : 0;
+        e = cudaLaunchKernelEx(&cfg, decode_score_kernel<D>, qb, static_cast<const __nv_bfloat16*>(kbar),
+                               static_cast<const __nv_bfloat16*>(kc), static_cast<const __nv_bfloat16*>(vc), H,
+                               Hkv, pos, Tmax, nb_cap, n_init, n_local, cpg, lists, keys);
+        if (e != cudaSuccess) return e;
     }
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(kc),
-                              static_cast<const __nv_bfloat16*>(vc), static_cast<const __nv_bfloat16*>(kbar), idx_in,
-                              idx_out, static_cast<__nv_bfloat16*>(o), H, Hkv, pos, Tmax, nb_cap, topk, n_init,
-                              n_local, slots, scale, cpg, rcap, nstages, epoch, static_cast<unsigned char*>(ws), lay,
-                              ctx);
+    // the attend kernel: a programmatic dependent of the score kernel when that ran (its early
+    // reads come after the score kernel's own wait), else of the previous kernel when asked
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(groups * kCS));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = sizeof(AttendSmem<D>);
+    cfg.stream = st;
+    cudaLaunchAttribute at[2];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = kCS;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    at[1] = pdl_attr;
+    cfg.attrs = at;
+    cfg.numAttrs = (owner || pdl) ? 2 : 1;
+    return cudaLaunchKernelEx(&cfg, decode_attend_kernel<D>, qb, static_cast<const __nv_bfloat16*>(kc),
+                              static_cast<const __nv_bfloat16*>(vc), idx_in, idx_out, static_cast<__nv_bfloat16*>(o),
+                              H, Hkv, pos, Tmax, topk, n_init, n_local, slots, scale, cpg, owner,
+                              static_cast<const uint64_t*>(lists), static_cast<const uint64_t*>(keys), ctx);
 }
 
 }  // namespace
 
 size_t sparse_decode_pf_workspace(int B, int H, int Hkv, int pos, int topk, int n_init, int n_local, int d) {
     if (B <= 0 || H <= 0 || Hkv <= 0 || pos < 0) return 0;
-    const int slots = n_init + n_local + topk;
     const int ncand = pos / kBlk - n_local - n_init + 1;
-    return pf_layout(B * Hkv, ncand > 0 ? ncand : 0, slots, H / Hkv, d).total;
+    return pf_layout(B * Hkv, ncand > 0 ? ncand : 0).total;
 }
 
 cudaError_t launch_sparse_decode_pf(DType dt, const void* q, const void* kc, const void* vc, const void* kbar,
                                     const int32_t* idx_in, int32_t* idx_out, void* o, int B, int H, int Hkv,
                                     int pos, int Tmax, int nb_cap, int d, int topk, int n_init, int n_local,
-                                    float scale, unsigned* epoch, void* ws, size_t ws_bytes, bool pdl,
-                                    cudaStream_t st, DevCtx ctx) {
+                                    float scale, void* ws, size_t ws_bytes, bool pdl, cudaStream_t st,
+                                    DevCtx ctx) {
     if (dt != DType::BF16 || (d != 64 && d != 128)) return cudaErrorNotSupported;
     return d == 64 ? pf<64>(q, kc, vc, kbar, idx_in, idx_out, o, B, H, Hkv, pos, Tmax, nb_cap, topk, n_init,
-                            n_local, scale, epoch, ws, ws_bytes, pdl, st, ctx)
+                            n_local, scale, ws, ws_bytes, pdl, st, ctx)
                    : pf<128>(q, kc, vc, kbar, idx_in, idx_out, o, B, H, Hkv, pos, Tmax, nb_cap, topk, n_init,
-                             n_local, scale, epoch, ws, ws_bytes, pdl, st, ctx);
+                             n_local, scale, ws, ws_bytes, pdl, st, ctx);
 }
 
 }  // namespace sala

@@ -353,11 +353,16 @@ sala_status sala_sparse_backward(const void* q, const void* k, const void* v, co
  *                 workspace can serve call after call and CUDA-graph replays.  After a call that
  *                 reported an error (SALA_ERR_TIMEOUT from sala_check_status), zero them again.
  *                 The rest needs no initial value.
- * Implementation: when k <= 64, slots <= 80, H/Hkv <= 16 and the grid fits on the GPU at once,
- * the whole step (scoring, top-k, attention over the selected blocks, combine) is one cooperative
- * launch with two barriers per (batch, KV head) group; for bf16 with d 64 or 128 and at most 64
- * groups, each CTA holds its share of kbar in shared memory and attends the blocks it wins
- * (sala_sparse_decode_pdl).  Otherwise it runs as four launches.
+ * Implementation, by shape:
+ *   - bf16, d 64 or 128, k <= 64, slots <= 80, H/Hkv <= 16, at most 16 (batch, KV head) groups
+ *     (and as many 16-CTA clusters resident at once), contexts whose candidate blocks fit 256 per
+ *     SM: two launches -- a score kernel over every SM (each CTA's share of kbar in shared memory,
+ *     tensor-core scores, its best keys stored) and an attend kernel of one 16-CTA cluster per
+ *     group (exact top-k from the stored keys, attention over the winners, partials combined in
+ *     distributed shared memory).  No device-side waits.
+ *   - otherwise, when k <= 64, slots <= 80, H/Hkv <= 16 and the grid fits on the GPU at once: one
+ *     cooperative launch with two grid-wide barriers (the counters above).
+ *   - otherwise: four launches.
  */
 sala_status sala_sparse_decode(const void* q, const void* kcache, const void* vcache,
                                const void* kbar, const int32_t* idx_in, int32_t* idx_out, void* o,
@@ -369,16 +374,14 @@ size_t sala_sparse_decode_workspace(int B, int H, int Hkv, int pos, int block, i
                                     int n_init, int n_local, int d);
 
 /* sala_sparse_decode launched as a programmatic dependent of the previous kernel in the stream:
- * on its one-launch path (bf16, d 64 or 128, k <= 64, at most 80 slots and 16 query heads per KV
- * head, at most 64 (batch, KV head) groups, and each CTA's share of k_bar within its shared memory)
- * the kernel starts while that kernel still runs and copies its share of kbar -- the rows of the
- * candidate blocks n_init .. pos/block - n_local -- into shared memory at once; q, the KV cache
- * and idx_in are read only after that kernel has completed and its writes are visible.  A decode
- * step thus overlaps each sparse layer's kbar read (8 MiB at 2^20 tokens, 2 KV heads) with the
- * layer before.  Contract: the previous kernel in the stream does not write those kbar rows (the
- * block a token completes is a local block, never a candidate, so compressing it just before is
- * fine).  Other shapes run as sala_sparse_decode.  Arguments, workspace rules and errors as
- * sala_sparse_decode. */
+ * on its two-launch path (see sala_sparse_decode) the score kernel starts while that kernel still
+ * runs and copies its share of kbar -- the rows of the candidate blocks n_init ..
+ * pos/block - n_local -- into shared memory at once; q, the KV cache and idx_in are read only after
+ * that kernel has completed and its writes are visible.  A decode step thus overlaps each sparse
+ * layer's kbar read (8 MiB at 2^20 tokens, 2 KV heads) with the layer before.  Contract: the
+ * previous kernel in the stream does not write those kbar rows (the block a token completes is a
+ * local block, never a candidate, so compressing it just before is fine).  Other shapes run as
+ * sala_sparse_decode.  Arguments, workspace rules and errors as sala_sparse_decode. */
 sala_status sala_sparse_decode_pdl(const void* q, const void* kcache, const void* vcache,
                                    const void* kbar, const int32_t* idx_in, int32_t* idx_out,
                                    void* o, int B, int H, int Hkv, int pos, int Tmax, int nb_cap,

@@ -33,10 +33,11 @@ def _lib():
 def _call(lib, q, kc, vc, kbar, idx_out, o, pos, topk, n_init, n_local):
     B, H, d = q.shape
     Hkv, Tmax = kc.shape[1], kc.shape[2]
+    dt = 1 if q.dtype == torch.bfloat16 else 0
     return lib.sala_sparse_decode_noalloc(
         q.data_ptr(), kc.data_ptr(), vc.data_ptr(), kbar.data_ptr(), None, idx_out.data_ptr(),
         o.data_ptr(), B, H, Hkv, pos, Tmax, kbar.shape[2], d, 64, topk, n_init, n_local,
-        ctypes.c_float(0.0), 1, ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+        ctypes.c_float(0.0), dt, ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
 
 
 @pytest.mark.parametrize("T", [64 * 300 + 5, 1 << 20])
@@ -64,19 +65,20 @@ def test_noalloc_matches_workspace_version_twice(T):
 
 
 def test_noalloc_recovers_after_a_timed_out_call():
-    # The built-in area carries the grid barrier's counters from call to call, and no caller can
-    # reach it to clear them.  Make one call give up on its waits (a 1 ns wait limit: every CTA
-    # but the last to arrive stops waiting at once, records SALA_ERR_TIMEOUT and returns; nothing
-    # faults), then check that the next call with the normal limit gives exactly the result of
-    # sala_sparse_decode with its own workspace.
+    # The built-in area carries the grid barrier counters of the one-launch cooperative kernel
+    # (the fp32 decode takes it) from call to call, and no caller can reach the area to clear them.
+    # Make one call give up on its waits (a 1 ns wait limit: every CTA but the last to arrive stops
+    # waiting at once, records SALA_ERR_TIMEOUT and returns; nothing faults), then check that the
+    # next calls with the normal limit give exactly the result of sala_sparse_decode with its own
+    # workspace.
     from hybrid_sparse_linear_b200 import sala, synth
     lib = _lib()
     lib.sala_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
     lib.sala_check_status.argtypes = [ctypes.c_void_p]
     lib.sala_check_status.restype = ctypes.c_int
-    T, topk, n_init, n_local, H, Hkv, d = 1 << 20, 64, 1, 2, 32, 2, 128
+    T, topk, n_init, n_local, H, Hkv, d = 64 * 3000 + 5, 64, 1, 2, 32, 2, 128
     slots = n_init + n_local + topk
-    layer = synth.sparse_layer(1, H, Hkv, T, d, torch.bfloat16, "cuda", layer=12, q_rows=1)
+    layer = synth.sparse_layer(1, H, Hkv, T, d, torch.float32, "cuda", layer=12, q_rows=1)
     kbar = sala.block_compress(layer.k)
     q = layer.q[:, :, 0].contiguous()
     idx_ref = torch.empty((1, Hkv, slots), dtype=torch.int32, device="cuda")
