@@ -467,10 +467,10 @@ sala_status sala_block_topk(const void* q, const void* kbar, int32_t* idx, int B
                         "block_topk_rowwise");
     }
     if (dt == SALA_BF16 && sala::block_topk_tc_supported(H, Hkv, Nq, q_pos0, nb, d, topk))
-        return launched(sala::launch_block_topk_tc(q, kbar, idx, B, H, Hkv, Nq, nb, topk, n_init,
+        return launched(sala::launch_block_topk_tc(q, kbar, idx, B, H, Hkv, Hkv, Nq, nb, topk, n_init,
                                                    n_local, st, ctx),
                         "block_topk_tc");
-    return launched(sala::launch_block_topk_tiled(to_dt(dt), q, kbar, idx, B, H, Hkv, Nq, q_pos0,
+    return launched(sala::launch_block_topk_tiled(to_dt(dt), q, kbar, idx, B, H, Hkv, Hkv, Nq, q_pos0,
                                                   nb, d, topk, n_init, n_local, st, ctx),
                     "block_topk");
 }
@@ -513,6 +513,28 @@ sala_status sala_block_topk_qblock(const void* q, const void* kbar, int32_t* idx
                     "block_topk_qblock");
 }
 
+sala_status sala_block_topk_per_head(const void* q, const void* kbar, int32_t* idx, int B, int H,
+                                     int Hkv, int Nq, int nb, int d, int block, int topk,
+                                     int n_init, int n_local, sala_dtype dt, sala_stream stream) {
+    sala_status s = check_select_args(B, H, Hkv, Nq, 0, nb, d, block, topk, n_init, n_local, dt);
+    if (s != SALA_OK) return s;
+    if (B == 0 || H == 0 || Nq == 0) return SALA_OK;
+    REQ_PTR(q); REQUIRE(idx != nullptr, SALA_ERR_INVALID_ARG, "idx must be a device pointer");
+    if (nb > 0) REQ_PTR(kbar);
+    sala::DevCtx ctx;
+    s = get_ctx(&ctx);
+    if (s != SALA_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // One selection group per query head (Hs = H), each scored against its KV head's kbar.
+    if (dt == SALA_BF16 && sala::block_topk_tc_supported(H, Hkv, Nq, 0, nb, d, topk))
+        return launched(sala::launch_block_topk_tc(q, kbar, idx, B, H, Hkv, H, Nq, nb, topk, n_init,
+                                                   n_local, st, ctx),
+                        "block_topk_per_head_tc");
+    return launched(sala::launch_block_topk_tiled(to_dt(dt), q, kbar, idx, B, H, Hkv, H, Nq, 0, nb,
+                                                  d, topk, n_init, n_local, st, ctx),
+                    "block_topk_per_head");
+}
+
 // ----------------------------------------------------------------------------------------------
 sala_status sala_sparse_prefill(const void* q, const void* k, const void* v, const int32_t* idx,
                                 void* o, int B, int H, int Hkv, int N, int d, int block,
@@ -536,11 +558,41 @@ sala_status sala_sparse_prefill(const void* q, const void* k, const void* v, con
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (dt == SALA_BF16 && sala::sparse_prefill_tc_supported(H, Hkv, d))
         return launched(sala::launch_sparse_prefill_tc(q, k, v, idx, o, nullptr, nullptr, B, H,
-                                                       Hkv, N, d, slots, scale, st, ctx),
+                                                       Hkv, N, d, slots, scale, false, st, ctx),
                         "sparse_prefill_tc");
-    return launched(sala::launch_sparse_prefill_simt(to_dt(dt), q, k, v, idx, o, B, H, Hkv, N, d,
-                                                     slots, scale, st, ctx),
+    return launched(sala::launch_sparse_prefill_simt(to_dt(dt), q, k, v, idx, o, B, H, Hkv, Hkv, N,
+                                                     d, slots, scale, st, ctx),
                     "sparse_prefill");
+}
+
+sala_status sala_sparse_prefill_per_head(const void* q, const void* k, const void* v,
+                                         const int32_t* idx, void* o, int B, int H, int Hkv, int N,
+                                         int d, int block, int slots, float scale, sala_dtype dt,
+                                         sala_stream stream) {
+    REQUIRE(B >= 0 && H >= 0 && Hkv > 0 && N >= 0 && slots >= 1, SALA_ERR_INVALID_ARG,
+            "bad sizes (B=%d H=%d Hkv=%d N=%d slots=%d)", B, H, Hkv, N, slots);
+    REQUIRE(H % Hkv == 0, SALA_ERR_INVALID_ARG, "H=%d is not a multiple of Hkv=%d", H, Hkv);
+    REQUIRE(dt == SALA_F32 || dt == SALA_BF16, SALA_ERR_INVALID_ARG, "unknown dtype %d", (int)dt);
+    REQUIRE(d == 64 || d == 128, SALA_ERR_UNSUPPORTED, "head dim %d (supported: 64, 128)", d);
+    REQUIRE(block == 64, SALA_ERR_UNSUPPORTED, "block %d (supported: 64)", block);
+    REQUIRE(slots <= 1024, SALA_ERR_UNSUPPORTED, "more than 1024 slots");
+    REQUIRE(isfinite(scale) && scale >= 0.f, SALA_ERR_INVALID_ARG, "scale must be finite and >= 0");
+    if (B == 0 || H == 0 || N == 0) return SALA_OK;
+    REQ_PTR(q); REQ_PTR(k); REQ_PTR(v); REQ_PTR(o);
+    REQUIRE(idx != nullptr, SALA_ERR_INVALID_ARG, "idx must be a device pointer");
+    if (scale == 0.f) scale = 1.0f / sqrtf((float)d);
+    sala::DevCtx ctx;
+    sala_status s = get_ctx(&ctx);
+    if (s != SALA_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (dt == SALA_BF16 && sala::sparse_prefill_tc_supported(H, Hkv, d) && slots <= 80 &&
+        N <= (1 << 20))
+        return launched(sala::launch_sparse_prefill_tc(q, k, v, idx, o, nullptr, nullptr, B, H,
+                                                       Hkv, N, d, slots, scale, true, st, ctx),
+                        "sparse_prefill_per_head_tc");
+    return launched(sala::launch_sparse_prefill_simt(to_dt(dt), q, k, v, idx, o, B, H, Hkv, H, N,
+                                                     d, slots, scale, st, ctx),
+                    "sparse_prefill_per_head");
 }
 
 // Sparse decode workspace: [0, 256) the cooperative one-launch path's barrier words, [256, 512)
@@ -584,7 +636,8 @@ sala_status sala_sparse_prefill_lse(const void* q, const void* k, const void* v,
     sala_status s = get_ctx(&ctx);
     if (s != SALA_OK) return s;
     return launched(sala::launch_sparse_prefill_tc(q, k, v, idx, o, lse, o_lo, B, H, Hkv, N, d, slots,
-                                                   scale, static_cast<cudaStream_t>(stream), ctx),
+                                                   scale, false, static_cast<cudaStream_t>(stream),
+                                                   ctx),
                     "sparse_prefill_lse");
 }
 

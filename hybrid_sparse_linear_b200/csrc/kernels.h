@@ -52,15 +52,17 @@ cudaError_t launch_block_topk_qblock_softmax(DType dt, const void* q, const void
                                              int B, int H, int Hkv, int Nq, int nb, int d, int topk,
                                              int n_init, int n_local, float scale, cudaStream_t st,
                                              DevCtx ctx);
+// Hs = selection groups per batch: Hkv (the group-summed query of each KV group) or H (one
+// selection per query head, each scored with its KV head's kbar); idx is [B, Hs, Nq, slots].
 cudaError_t launch_block_topk_tiled(DType dt, const void* q, const void* kbar, int32_t* idx,
-                                    int B, int H, int Hkv, int Nq, int q_pos0, int nb, int d,
-                                    int topk, int n_init, int n_local, cudaStream_t st,
+                                    int B, int H, int Hkv, int Hs, int Nq, int q_pos0, int nb,
+                                    int d, int topk, int n_init, int n_local, cudaStream_t st,
                                     DevCtx ctx);
 // Tensor-core selection (bf16, d 128, prefill rows from position 0, topk <= 64).
 bool block_topk_tc_supported(int H, int Hkv, int Nq, int q_pos0, int nb, int d, int topk);
 cudaError_t launch_block_topk_tc(const void* q, const void* kbar, int32_t* idx, int B, int H,
-                                 int Hkv, int Nq, int nb, int topk, int n_init, int n_local,
-                                 cudaStream_t st, DevCtx ctx);
+                                 int Hkv, int Hs, int Nq, int nb, int topk, int n_init,
+                                 int n_local, cudaStream_t st, DevCtx ctx);
 // Row-wise selection for few query rows and many blocks: candidates split across CTAs, then a
 // merge.  Workspace = rowwise_topk_workspace(...) bytes.
 size_t rowwise_topk_workspace(int B, int Hkv, int Nq, int q_pos0, int topk);
@@ -68,17 +70,21 @@ cudaError_t launch_block_topk_rowwise(DType dt, const void* q, const void* kbar,
                                       int B, int H, int Hkv, int Nq, int q_pos0, int nb, int d,
                                       int topk, int n_init, int n_local, void* ws,
                                       cudaStream_t st, DevCtx ctx);
+// Hs as in the selection: idx [B, Hs, N, slots] is shared by the H / Hs heads of a selection
+// group (Hs = Hkv: the KV group; Hs = H: a selection per query head).
 cudaError_t launch_sparse_prefill_simt(DType dt, const void* q, const void* k, const void* v,
-                                       const int32_t* idx, void* o, int B, int H, int Hkv, int N,
-                                       int d, int slots, float scale, cudaStream_t st,
+                                       const int32_t* idx, void* o, int B, int H, int Hkv, int Hs,
+                                       int N, int d, int slots, float scale, cudaStream_t st,
                                        DevCtx ctx);
 // lse (may be null): the training forward -- per query row the natural log-sum-exp of its
 // visible scaled logits, P V taken as P_hi V + P_lo V, and (o_lo, may be null) the bf16 rounding
 // residual of o.
+// per_head: idx is [B, H, N, slots], a selection per query head (forward only: lse and o_lo
+// null); N <= 2^20.
 cudaError_t launch_sparse_prefill_tc(const void* q, const void* k, const void* v,
                                      const int32_t* idx, void* o, float* lse, void* o_lo, int B,
                                      int H, int Hkv, int N, int d, int slots, float scale,
-                                     cudaStream_t st, DevCtx ctx);
+                                     bool per_head, cudaStream_t st, DevCtx ctx);
 
 // Sparse attention backward (bf16, G = 16, d = 128), selection held fixed.
 // The transposed selection: for key k = ((b * Hkv + g) * n_chunks + chunk) * nb + j,

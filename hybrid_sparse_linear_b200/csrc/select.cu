@@ -114,17 +114,21 @@ struct TopkSmem {
 template <typename T, int D>
 __global__ void __launch_bounds__(kTThreads)
 topk_tiled_kernel(const T* __restrict__ q, const T* __restrict__ kbar, int32_t* __restrict__ idx,
-                  int H, int Hkv, int Nq, int q_pos0, int nb, int topk, int n_init, int n_local,
-                  int slots) {
+                  int H, int Hkv, int Hs, int Nq, int q_pos0, int nb, int topk, int n_init,
+                  int n_local, int slots) {
     extern __shared__ __align__(16) float smt[];
     float* QBt = smt;                          // [D][RT+4]  group-summed queries, transposed
     float* KBt = QBt + TopkSmem<D>::kQ;        // [D][CT+4]  block keys, transposed
     float* SC = KBt + TopkSmem<D>::kK;         // [RT][CT+1] scores
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int G = H / Hkv;
+    // Selection group bg = (b, g) of Hs per batch: the G = H / Hs query heads g*G .. g*G+G-1 are
+    // summed and scored against the kbar of their KV head (Hs = Hkv: the KV group; Hs = H: one
+    // head); idx rows are [B, Hs, Nq, slots].
+    const int G = H / Hs;
     const int64_t bg = blockIdx.y;
-    const int64_t b = bg / Hkv;
-    const int g = (int)(bg % Hkv);
+    const int64_t b = bg / Hs;
+    const int g = (int)(bg % Hs);
+    const int64_t kv_plane = b * Hkv + g / (Hs / Hkv);
     const int r0 = blockIdx.x * kRT;
     const int rend = min(Nq, r0 + kRT);
 
@@ -153,7 +157,7 @@ topk_tiled_kernel(const T* __restrict__ q, const T* __restrict__ kbar, int32_t* 
     }
     const int K = min(topk, kCap);
 
-    const T* kb = kbar + bg * (int64_t)nb * D;
+    const T* kb = kbar + kv_plane * (int64_t)nb * D;
     for (int j0 = cand_lo; j0 <= cand_hi; j0 += kCT) {
         __syncthreads();
         for (int e = tid; e < kCT * D; e += kTThreads) {
@@ -205,15 +209,15 @@ topk_tiled_kernel(const T* __restrict__ q, const T* __restrict__ kbar, int32_t* 
 }
 
 template <typename T, int D>
-cudaError_t tiled(const void* q, const void* kbar, int32_t* idx, int B, int H, int Hkv, int Nq,
-                  int q_pos0, int nb, int topk, int n_init, int n_local, cudaStream_t st) {
+cudaError_t tiled(const void* q, const void* kbar, int32_t* idx, int B, int H, int Hkv, int Hs,
+                  int Nq, int q_pos0, int nb, int topk, int n_init, int n_local, cudaStream_t st) {
     auto kern = topk_tiled_kernel<T, D>;
     const size_t smem = TopkSmem<D>::bytes;
     cudaError_t e = ensure_smem<topk_tiled_kernel<T, D>>((int)smem);
     if (e != cudaSuccess) return e;
-    dim3 grid(ceil_div(Nq, kRT), (unsigned)(B * Hkv));
+    dim3 grid(ceil_div(Nq, kRT), (unsigned)(B * Hs));
     kern<<<grid, kTThreads, smem, st>>>(static_cast<const T*>(q), static_cast<const T*>(kbar), idx,
-                                        H, Hkv, Nq, q_pos0, nb, topk, n_init, n_local,
+                                        H, Hkv, Hs, Nq, q_pos0, nb, topk, n_init, n_local,
                                         n_init + n_local + topk);
     return cudaGetLastError();
 }
@@ -330,13 +334,13 @@ size_t rowwise_topk_workspace(int B, int Hkv, int Nq, int q_pos0, int topk) {
 }
 
 cudaError_t launch_block_topk_tiled(DType dt, const void* q, const void* kbar, int32_t* idx, int B,
-                                    int H, int Hkv, int Nq, int q_pos0, int nb, int d, int topk,
-                                    int n_init, int n_local, cudaStream_t st, DevCtx) {
+                                    int H, int Hkv, int Hs, int Nq, int q_pos0, int nb, int d,
+                                    int topk, int n_init, int n_local, cudaStream_t st, DevCtx) {
     if (dt == DType::F32)
-        return d == 64 ? tiled<float, 64>(q, kbar, idx, B, H, Hkv, Nq, q_pos0, nb, topk, n_init, n_local, st)
-                       : tiled<float, 128>(q, kbar, idx, B, H, Hkv, Nq, q_pos0, nb, topk, n_init, n_local, st);
-    return d == 64 ? tiled<__nv_bfloat16, 64>(q, kbar, idx, B, H, Hkv, Nq, q_pos0, nb, topk, n_init, n_local, st)
-                   : tiled<__nv_bfloat16, 128>(q, kbar, idx, B, H, Hkv, Nq, q_pos0, nb, topk, n_init, n_local, st);
+        return d == 64 ? tiled<float, 64>(q, kbar, idx, B, H, Hkv, Hs, Nq, q_pos0, nb, topk, n_init, n_local, st)
+                       : tiled<float, 128>(q, kbar, idx, B, H, Hkv, Hs, Nq, q_pos0, nb, topk, n_init, n_local, st);
+    return d == 64 ? tiled<__nv_bfloat16, 64>(q, kbar, idx, B, H, Hkv, Hs, Nq, q_pos0, nb, topk, n_init, n_local, st)
+                   : tiled<__nv_bfloat16, 128>(q, kbar, idx, B, H, Hkv, Hs, Nq, q_pos0, nb, topk, n_init, n_local, st);
 }
 
 cudaError_t launch_block_topk_rowwise(DType dt, const void* q, const void* kbar, int32_t* idx,

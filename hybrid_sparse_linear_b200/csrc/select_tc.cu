@@ -141,21 +141,24 @@ __device__ __forceinline__ int keep_best(const uint64_t* buf, int n, int K, uint
 __global__ void __launch_bounds__(kThreads, 1)
 topk_tc_kernel(const __grid_constant__ CUtensorMap tmKb, const __nv_bfloat16* __restrict__ q,
                const __nv_bfloat16* __restrict__ kbar, int32_t* __restrict__ idx, int H, int Hkv,
-               int Nq, int nb, int topk, int n_init, int n_local, int slots, DevCtx ctx) {
+               int Hs, int Nq, int nb, int topk, int n_init, int n_local, int slots, DevCtx ctx) {
     extern __shared__ uint8_t smraw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smraw) + 1023) &
                                              ~uintptr_t(1023));
     __shared__ Bars bars;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int G = H / Hkv;
+    // Selection group (b, g) of Hs per batch: the G = H / Hs query heads g*G .. g*G+G-1, scored
+    // against their KV head's kbar (Hs = Hkv: the KV group; Hs = H: one query head).
+    const int G = H / Hs;
     // Heaviest tiles first: a tile's work grows with its candidate count, i.e. with its row
     // index, so the launch order walks row tiles from the last to the first (all groups of one
     // row tile together) and the lightest tiles fill the tail.
     const int n_rt = (Nq + kRows - 1) / kRows;
     const int n_bg = (int)(gridDim.x / n_rt);
     const int64_t bg = blockIdx.x % n_bg;
-    const int64_t b = bg / Hkv;
-    const int g = (int)(bg % Hkv);
+    const int64_t b = bg / Hs;
+    const int g = (int)(bg % Hs);
+    const int64_t kv_plane = b * Hkv + g / (Hs / Hkv);
     const int r0 = (n_rt - 1 - (int)(blockIdx.x / n_bg)) * kRows;
     const int nrows = min(kRows, Nq - r0);
     const int K = min(topk, kCap);
@@ -206,8 +209,8 @@ topk_tc_kernel(const __grid_constant__ CUtensorMap tmKb, const __nv_bfloat16* __
                 uint8_t* st = sm + kOffKb + s * 2 * kSub;
                 mbar_arrive_expect_tx(&bars.kv_full[s], 2 * kSub);
                 const int y = lo + t * kCand;
-                tma_load_3d(st, &tmKb, &bars.kv_full[s], 0, y, (int)bg);
-                tma_load_3d(st + kSub, &tmKb, &bars.kv_full[s], 64, y, (int)bg);
+                tma_load_3d(st, &tmKb, &bars.kv_full[s], 0, y, (int)kv_plane);
+                tma_load_3d(st + kSub, &tmKb, &bars.kv_full[s], 64, y, (int)kv_plane);
                 if (s == 0) issued0 = r; else issued1 = r;
             }
             if (issued0 >= 0) (void)mbar_wait(&bars.kv_full[0], issued0 & 1, ctx);
@@ -369,7 +372,7 @@ topk_tc_kernel(const __grid_constant__ CUtensorMap tmKb, const __nv_bfloat16* __
                     for (int st = 0; st < kBatch; ++st) {
                         const int i = it0 + st * 32 + warp * 4 + (lane >> 3);
                         const uint4* row = reinterpret_cast<const uint4*>(
-                            kbar + (bg * nb + lo + cb + i) * (int64_t)kD + part * 16);
+                            kbar + (kv_plane * nb + lo + cb + i) * (int64_t)kD + part * 16);
                         raw[st][0] = i < nc ? row[0] : make_uint4(0u, 0u, 0u, 0u);
                         raw[st][1] = i < nc ? row[1] : make_uint4(0u, 0u, 0u, 0u);
                     }
@@ -421,7 +424,7 @@ topk_tc_kernel(const __grid_constant__ CUtensorMap tmKb, const __nv_bfloat16* __
 #pragma unroll
             for (int u = 0; u < kPer; ++u) {
                 const int e = u * kWorkers + tid, j = e >> 4, cc = e & 15;
-                sv[u] = reinterpret_cast<const uint4*>(kbar + (bg * nb + bars.seeds[j]) * (int64_t)kD)[cc];
+                sv[u] = reinterpret_cast<const uint4*>(kbar + (kv_plane * nb + bars.seeds[j]) * (int64_t)kD)[cc];
             }
 #pragma unroll
             for (int u = 0; u < kPer; ++u) {
@@ -642,8 +645,8 @@ bool block_topk_tc_supported(int H, int Hkv, int Nq, int q_pos0, int nb, int d, 
 }
 
 cudaError_t launch_block_topk_tc(const void* q, const void* kbar, int32_t* idx, int B, int H,
-                                 int Hkv, int Nq, int nb, int topk, int n_init, int n_local,
-                                 cudaStream_t st, DevCtx ctx) {
+                                 int Hkv, int Hs, int Nq, int nb, int topk, int n_init,
+                                 int n_local, cudaStream_t st, DevCtx ctx) {
     EncodeTiledFn fn = encode_tiled_fn();
     if (!fn) return cudaErrorNotSupported;
     CUtensorMap tm;
@@ -658,10 +661,10 @@ cudaError_t launch_block_topk_tc(const void* q, const void* kbar, int32_t* idx, 
         return cudaErrorInvalidValue;
     cudaError_t e = ensure_smem<topk_tc_kernel>(kSmemBytes);
     if (e != cudaSuccess) return e;
-    dim3 grid((unsigned)(ceil_div(Nq, kRows) * B * Hkv));
+    dim3 grid((unsigned)(ceil_div(Nq, kRows) * B * Hs));
     topk_tc_kernel<<<grid, kThreads, kSmemBytes, st>>>(
         tm, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(kbar), idx, H,
-        Hkv, Nq, nb, topk, n_init, n_local, n_init + n_local + topk, ctx);
+        Hkv, Hs, Nq, nb, topk, n_init, n_local, n_init + n_local + topk, ctx);
     return cudaGetLastError();
 }
 

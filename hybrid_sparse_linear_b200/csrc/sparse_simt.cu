@@ -76,24 +76,27 @@ template <typename T, int D>
 __global__ void __launch_bounds__(kWarps * 32)
 sparse_prefill_simt_kernel(const T* __restrict__ q, const T* __restrict__ k,
                            const T* __restrict__ v, const int32_t* __restrict__ idx,
-                           T* __restrict__ o, int H, int Hkv, int N, int slots, float scale,
-                           DevCtx ctx) {
+                           T* __restrict__ o, int H, int Hkv, int Hs, int N, int slots,
+                           float scale, DevCtx ctx) {
     extern __shared__ float sms[];
     float* Kt = sms;
     float* Vs = Kt + D * (kBlk + 1);
     float* Qs = Vs + kBlk * D;  // [G][D]
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int G = H / Hkv;
+    // Selection group (b, g) of Hs per batch: heads g*G .. g*G+G-1 share idx row (b, g, i) and
+    // read the K/V of their KV head.
+    const int G = H / Hs;
     const int64_t i = blockIdx.x;
     const int64_t bg = blockIdx.y;
-    const int64_t b = bg / Hkv;
-    const int g = (int)(bg % Hkv);
+    const int64_t b = bg / Hs;
+    const int g = (int)(bg % Hs);
+    const int64_t kv_plane = b * Hkv + g / (Hs / Hkv);
     for (int e = threadIdx.x; e < G * D; e += blockDim.x) {
         const int hh = e / D, a = e % D;
         Qs[e] = to_f(q[((b * H + (int64_t)g * G + hh) * N + i) * D + a]);
     }
-    const T* kh = k + bg * (int64_t)N * D;
-    const T* vh = v + bg * (int64_t)N * D;
+    const T* kh = k + kv_plane * (int64_t)N * D;
+    const T* vh = v + kv_plane * (int64_t)N * D;
     const int32_t* sel = idx + (bg * N + i) * (int64_t)slots;
     const int max_blk = (int)(i / kBlk);
 
@@ -137,16 +140,17 @@ sparse_prefill_simt_kernel(const T* __restrict__ q, const T* __restrict__ k,
 
 template <typename T, int D>
 cudaError_t prefill(const void* q, const void* k, const void* v, const int32_t* idx, void* o, int B,
-                    int H, int Hkv, int N, int slots, float scale, cudaStream_t st, DevCtx ctx) {
+                    int H, int Hkv, int Hs, int N, int slots, float scale, cudaStream_t st,
+                    DevCtx ctx) {
     auto kern = sparse_prefill_simt_kernel<T, D>;
-    const int G = H / Hkv;
+    const int G = H / Hs;
     const size_t smem = BlockSmem<D>::bytes + sizeof(float) * G * D;
     cudaError_t e = ensure_smem<sparse_prefill_simt_kernel<T, D>>((int)(BlockSmem<D>::bytes + sizeof(float) * 2 * kWarps * D));
     if (e != cudaSuccess) return e;
-    dim3 grid((unsigned)N, (unsigned)(B * Hkv));
+    dim3 grid((unsigned)N, (unsigned)(B * Hs));
     kern<<<grid, kWarps * 32, smem, st>>>(static_cast<const T*>(q), static_cast<const T*>(k),
                                           static_cast<const T*>(v), idx, static_cast<T*>(o), H,
-                                          Hkv, N, slots, scale, ctx);
+                                          Hkv, Hs, N, slots, scale, ctx);
     return cudaGetLastError();
 }
 
@@ -250,14 +254,15 @@ cudaError_t decode(const void* q, const void* kc, const void* vc, const int32_t*
 }  // namespace
 
 cudaError_t launch_sparse_prefill_simt(DType dt, const void* q, const void* k, const void* v,
-                                       const int32_t* idx, void* o, int B, int H, int Hkv, int N,
-                                       int d, int slots, float scale, cudaStream_t st, DevCtx ctx) {
-    if (H / Hkv > 2 * kWarps) return cudaErrorNotSupported;
+                                       const int32_t* idx, void* o, int B, int H, int Hkv, int Hs,
+                                       int N, int d, int slots, float scale, cudaStream_t st,
+                                       DevCtx ctx) {
+    if (H / Hs > 2 * kWarps) return cudaErrorNotSupported;
     if (dt == DType::F32)
-        return d == 64 ? prefill<float, 64>(q, k, v, idx, o, B, H, Hkv, N, slots, scale, st, ctx)
-                       : prefill<float, 128>(q, k, v, idx, o, B, H, Hkv, N, slots, scale, st, ctx);
-    return d == 64 ? prefill<__nv_bfloat16, 64>(q, k, v, idx, o, B, H, Hkv, N, slots, scale, st, ctx)
-                   : prefill<__nv_bfloat16, 128>(q, k, v, idx, o, B, H, Hkv, N, slots, scale, st, ctx);
+        return d == 64 ? prefill<float, 64>(q, k, v, idx, o, B, H, Hkv, Hs, N, slots, scale, st, ctx)
+                       : prefill<float, 128>(q, k, v, idx, o, B, H, Hkv, Hs, N, slots, scale, st, ctx);
+    return d == 64 ? prefill<__nv_bfloat16, 64>(q, k, v, idx, o, B, H, Hkv, Hs, N, slots, scale, st, ctx)
+                   : prefill<__nv_bfloat16, 128>(q, k, v, idx, o, B, H, Hkv, Hs, N, slots, scale, st, ctx);
 }
 
 size_t sparse_decode_attn_workspace(int B, int H, int Hkv, int slots, int d) {

@@ -28,6 +28,14 @@
 // issues the MMAs of tile A, warp 10 those of tile B (one elected lane of each converged warp).
 // Every wait is bounded; a timeout sets the status word, the roles wind down, and the kernel waits
 // (bounded) for its own copies and MMAs before it frees TMEM.
+//
+// Per-head selections (kPerHead: idx is [B, H, N, slots], one row per query head and token): the
+// unit's union is over its 16 heads x 16 tokens.  The list warp sets one bit per chosen block in
+// two bitmaps (tile A's rows, tile B's rows), and every role walks the set bits of their OR in
+// ascending order; a tile skips the blocks its bitmap lacks, and each softmax thread decides its
+// row's mask by walking its own (ascending) selection row alongside the union.
+#include <climits>
+
 #include "fastexp.cuh"
 #include "kernels.h"
 #include "ptx.cuh"
@@ -59,6 +67,10 @@ constexpr int kOffList = kOffRing + kStages * kStageBytes;
 constexpr int kListBytes = kMaxList * 6;              // int32 ids + uint16 token masks
 constexpr int kOffStage = kOffList + 2 * kListBytes;  // staged selection rows of one unit
 constexpr int kSmemBytes = kOffStage + kUT * kMaxSlots * 4 + 1024;
+// Per-head mode keeps, in the list area, two bitmaps (tiles A, B) per list buffer over the
+// candidate blocks 0 .. c of the unit: up to 2^14 blocks, i.e. N <= 2^20.
+constexpr int kMaxBmWords = 512;
+static_assert(4 * kMaxBmWords * 4 <= 2 * kListBytes, "bitmaps exceed the list area");
 
 // TMEM columns: O_A [0,128), O_B [128,256), S_A two buffers [256,384), S_B two buffers [384,512).
 constexpr uint32_t kTmemCols = 512;
@@ -169,7 +181,41 @@ __device__ __forceinline__ void exp_block(const uint32_t* s, float sl2, float nb
     }
 }
 
-template <bool kTrain>
+// A unit's union in ascending block order.  Group selections: the list of (block, 16-bit token
+// mask) entries.  Per-head selections: the set bits of bitmap A | bitmap B over words 0 .. nw-1,
+// with m = bit 0 (a row of tile A chose the block) | bit 1 (a row of tile B did).
+template <bool kPerHead>
+struct UnionWalk {
+    const int32_t* ids;
+    const uint16_t* msks;
+    const uint32_t* bm_a;
+    const uint32_t* bm_b;
+    int pos, w, nw;
+    uint32_t bits;
+    __device__ __forceinline__ void next(int& blk, uint32_t& m) {
+        if constexpr (!kPerHead) {
+            blk = ids[pos];
+            m = msks[pos];
+            ++pos;
+        } else {
+            while (bits == 0u && w + 1 < nw) {
+                ++w;
+                bits = bm_a[w] | bm_b[w];
+            }
+            const int bit = __ffs((int)bits) - 1;  // callers take exactly the counted entries
+            bits &= bits - 1u;
+            blk = w * 32 + bit;
+            m = ((bm_a[w] >> bit) & 1u) | (((bm_b[w] >> bit) & 1u) << 1);
+        }
+    }
+    // Whether some row of tile x chose the block.
+    __device__ __forceinline__ static bool tile_active(uint32_t m, int x) {
+        if constexpr (kPerHead) return (m >> x) & 1u;
+        else return ((m >> (8 * x)) & 0xffu) != 0u;
+    }
+};
+
+template <bool kTrain, bool kPerHead>
 __global__ void __launch_bounds__(kThreads, 1)
 sparse_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                          const __grid_constant__ CUtensorMap tmK,
@@ -219,6 +265,22 @@ sparse_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
     auto list_mask = [&](int lb) {
         return reinterpret_cast<uint16_t*>(sm + kOffList + lb * kListBytes + kMaxList * 4);
     };
+    auto bitmap = [&](int lb, int x) {
+        return reinterpret_cast<uint32_t*>(sm + kOffList + (lb * 2 + x) * kMaxBmWords * 4);
+    };
+    // The union of list buffer lb for a unit whose tokens lie in query block c.
+    auto walk = [&](int lb, int c) {
+        UnionWalk<kPerHead> u;
+        u.ids = list_id(lb);
+        u.msks = list_mask(lb);
+        u.bm_a = bitmap(lb, 0);
+        u.bm_b = bitmap(lb, 1);
+        u.pos = 0;
+        u.w = -1;
+        u.nw = c / 32 + 1;
+        u.bits = 0u;
+        return u;
+    };
     // Ring entry e lives in stage e % kStages and is that stage's use number e / kStages.
     auto stage_ptr = [&](uint32_t e) { return sm + kOffRing + (e % kStages) * kStageBytes; };
     auto full_bar = [&](uint32_t e) { return &bars.kv_full[e % kStages]; };
@@ -230,7 +292,6 @@ sparse_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
         // Builds unit u+1's union list (double-buffered) while unit u is being consumed, so the
         // producer never stalls the ring on it: the unit's 16 selection rows (contiguous in
         // memory) are staged with all loads in flight, then merged.
-        int32_t* stage = reinterpret_cast<int32_t*>(sm + kOffStage);
         int it = 0;
         for (int unit = blockIdx.x; unit < n_units; unit += gridDim.x, ++it) {
             const int lb = it & 1;
@@ -240,51 +301,99 @@ sparse_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
             const int c = i0 / kBlk;
             const int n_act = min(kUT, N - i0);
             const int total = n_act * slots;
-            const int32_t* src = idx + (bg * N + i0) * (int64_t)slots;
-            {
-                constexpr int kPer = kMaxList / 32;  // entries per lane at most
-                int32_t v[kPer];
+            int n = 0;
+            if constexpr (!kPerHead) {
+                int32_t* stage = reinterpret_cast<int32_t*>(sm + kOffStage);
+                const int32_t* src = idx + (bg * N + i0) * (int64_t)slots;
+                {
+                    constexpr int kPer = kMaxList / 32;  // entries per lane at most
+                    int32_t v[kPer];
 #pragma unroll
-                for (int j = 0; j < kPer; ++j) {
-                    const int e = lane + 32 * j;
-                    v[j] = e < total ? __ldg(src + e) : -1;
-                }
+                    for (int j = 0; j < kPer; ++j) {
+                        const int e = lane + 32 * j;
+                        v[j] = e < total ? __ldg(src + e) : -1;
+                    }
 #pragma unroll
-                for (int j = 0; j < kPer; ++j) {
-                    const int e = lane + 32 * j;
-                    if (e < total) stage[e] = v[j];
-                }
-            }
-            __syncwarp();
-            // 16-way merge of the ascending rows, one lane per token.
-            const int32_t* row = stage + lane * slots;
-            const bool active = lane < n_act;
-            int p = 0, n = 0, prev = -1;
-            while (true) {
-                int head = 0x7fffffff;
-                if (active && p < slots) {
-                    const int v = row[p];
-                    if (v >= 0) head = v;
-                }
-                const int m = __reduce_min_sync(0xffffffffu, head);
-                if (m == 0x7fffffff) break;
-                const unsigned msk = __ballot_sync(0xffffffffu, head == m);
-                if (head == m) ++p;
-                if (m > c) {  // in the future of every token of the unit
-                    if (lane == 0) flag(ctx, kStatusBounds);
-                    continue;
-                }
-                if (lane == 0) {
-                    if (m == prev) {
-                        list_mask(lb)[n - 1] |= (uint16_t)msk;
-                    } else if (n < kMaxList) {
-                        list_id(lb)[n] = m;
-                        list_mask(lb)[n] = (uint16_t)msk;
-                        ++n;
+                    for (int j = 0; j < kPer; ++j) {
+                        const int e = lane + 32 * j;
+                        if (e < total) stage[e] = v[j];
                     }
                 }
-                n = __shfl_sync(0xffffffffu, n, 0);
-                prev = m;
+                __syncwarp();
+                // 16-way merge of the ascending rows, one lane per token.
+                const int32_t* row = stage + lane * slots;
+                const bool active = lane < n_act;
+                int p = 0, prev = -1;
+                while (true) {
+                    int head = 0x7fffffff;
+                    if (active && p < slots) {
+                        const int v = row[p];
+                        if (v >= 0) head = v;
+                    }
+                    const int m = __reduce_min_sync(0xffffffffu, head);
+                    if (m == 0x7fffffff) break;
+                    const unsigned msk = __ballot_sync(0xffffffffu, head == m);
+                    if (head == m) ++p;
+                    if (m > c) {  // in the future of every token of the unit
+                        if (lane == 0) flag(ctx, kStatusBounds);
+                        continue;
+                    }
+                    if (lane == 0) {
+                        if (m == prev) {
+                            list_mask(lb)[n - 1] |= (uint16_t)msk;
+                        } else if (n < kMaxList) {
+                            list_id(lb)[n] = m;
+                            list_mask(lb)[n] = (uint16_t)msk;
+                            ++n;
+                        }
+                    }
+                    n = __shfl_sync(0xffffffffu, n, 0);
+                    prev = m;
+                }
+            } else {
+                // Per-head rows: the unit's 16 heads, each a run of n_act rows of slots entries;
+                // entries of the first 8 tokens go to tile A's bitmap, the rest to tile B's.
+                uint32_t* bm_a = bitmap(lb, 0);
+                uint32_t* bm_b = bitmap(lb, 1);
+                const int nw = c / 32 + 1;
+                for (int w = lane; w < nw; w += 32) {
+                    bm_a[w] = 0u;
+                    bm_b[w] = 0u;
+                }
+                __syncwarp();
+                const int split = kTQ * slots;
+                bool bad = false;
+                constexpr int kPer = kMaxList / 32;
+                for (int h0 = 0; h0 < kG; h0 += 2) {
+                    int32_t v[2][kPer];
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const int64_t head = (bg / Hkv) * H + (bg % Hkv) * kG + h0 + u;
+                        const int32_t* src = idx + (head * N + i0) * (int64_t)slots;
+#pragma unroll
+                        for (int j = 0; j < kPer; ++j) {
+                            const int e = lane + 32 * j;
+                            v[u][j] = e < total ? __ldg(src + e) : -1;
+                        }
+                    }
+#pragma unroll
+                    for (int u = 0; u < 2; ++u)
+#pragma unroll
+                        for (int j = 0; j < kPer; ++j) {
+                            const int m = v[u][j];
+                            if (m > c) {  // in the future of every token of the unit
+                                bad = true;
+                            } else if (m >= 0) {
+                                const int e = lane + 32 * j;
+                                atomicOr((e < split ? bm_a : bm_b) + (m >> 5), 1u << (m & 31));
+                            }
+                        }
+                }
+                if (__any_sync(0xffffffffu, bad) && lane == 0) flag(ctx, kStatusBounds);
+                __syncwarp();
+                for (int w = lane; w < nw; w += 32) n += __popc(bm_a[w] | bm_b[w]);
+                n = __reduce_add_sync(0xffffffffu, n);
+                __threadfence_block();  // every lane's bitmap words before lane 0 publishes them
             }
             __syncwarp();
             if (lane == 0) {
@@ -308,6 +417,7 @@ sparse_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                 const int n = stop ? 0 : bars.list_n[lb];
                 const int64_t bg = unit / units_per_seq;
                 const int i0 = (unit % units_per_seq) * kUT;
+                UnionWalk<kPerHead> uw = walk(lb, i0 / kBlk);
                 if (n > 0) {
                     // Q_A, Q_B: 16 heads x 8 tokens x 128 columns each, once both issuers are
                     // done with the previous unit's S MMAs.
@@ -329,7 +439,10 @@ sparse_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                         uint8_t* st = stage_ptr(rc);
                         uint64_t* fb = full_bar(rc);
                         mbar_arrive_expect_tx(fb, kStageBytes);
-                        const int y = list_id(lb)[e] * kBlk;
+                        int blk;
+                        uint32_t m;
+                        uw.next(blk, m);
+                        const int y = blk * kBlk;
                         tma_load_3d(st, &tmK, fb, 0, y, (int)bg);
                         tma_load_3d(st + kHalfBlk, &tmK, fb, 64, y, (int)bg);
                         tma_load_3d(st + 2 * kHalfBlk, &tmV, fb, 0, y, (int)bg);
@@ -383,6 +496,7 @@ sparse_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
             ok = wait_w(&bars.list_full[lb], (it >> 1) & 1);
             if (!ok) break;
             const int n = bars.list_n[lb];
+            UnionWalk<kPerHead> uw = walk(lb, ((unit % units_per_seq) * kUT) / kBlk);
             if (n > 0) {
                 ok = wait_w(&bars.q_full, kq & 1);
                 ++kq;
@@ -416,7 +530,10 @@ sparse_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                 };
                 for (int b = 0; b < n && ok; ++b) {
                     const uint32_t e = rc + b;
-                    const bool act = ((list_mask(lb)[b] >> (8 * x)) & 0xffu) != 0;
+                    int blk;
+                    uint32_t m;
+                    uw.next(blk, m);
+                    const bool act = UnionWalk<kPerHead>::tile_active(m, x);
                     while (ok && np > 0 && pe0 + kStages <= e) ok = flush_pv();
                     if (ok && np == 2) ok = flush_pv();
                     if (!ok) break;
@@ -481,20 +598,46 @@ sparse_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
             const int lb = it & 1;
             if (!dead && !mbar_wait(&bars.list_full[lb], (it >> 1) & 1, ctx)) fail();
             const int n = dead ? 0 : bars.list_n[lb];
-            const int32_t* ids = list_id(lb);
-            const uint16_t* msks = list_mask(lb);
             const int64_t bg = unit / units_per_seq;
             const int i0 = (unit % units_per_seq) * kUT;
             const int c = i0 / kBlk;
             const int i = i0 + t;
+            UnionWalk<kPerHead> uw = walk(lb, c);
+            // Per-head: this row's own selection, read four entries ahead (own0 is the first entry
+            // not below the blocks walked so far; INT_MAX past the row's end).
+            const int32_t* own = nullptr;
+            int own0 = INT_MAX, own1 = INT_MAX, own2 = INT_MAX, own3 = INT_MAX, own_p = 0;
+            if constexpr (kPerHead) {
+                if (i < N) {
+                    own = idx + (((bg / Hkv) * H + (bg % Hkv) * kG + hh) * (int64_t)N + i) * slots;
+                    own0 = __ldg(own);
+                    own1 = slots > 1 ? __ldg(own + 1) : INT_MAX;
+                    own2 = slots > 2 ? __ldg(own + 2) : INT_MAX;
+                    own3 = slots > 3 ? __ldg(own + 3) : INT_MAX;
+                    own_p = 4;
+                }
+            }
             float m_run = -INFINITY, l = 0.f;  // running max (scaled log2 units), row sum
             int last = -1;
             for (int b = 0; b < n; ++b) {
-                const unsigned msk = msks[b];
-                if (((msk >> (8 * x)) & 0xffu) == 0) continue;  // no token of this tile chose it
-                const int blk = ids[b];
+                int blk;
+                uint32_t msk;
+                uw.next(blk, msk);
+                if (!UnionWalk<kPerHead>::tile_active(msk, x)) continue;  // no row of the tile chose it
                 const bool diag = blk == c;                      // uniform over the warpgroup
-                const bool sel = (msk >> t) & 1u;
+                bool sel;
+                if constexpr (kPerHead) {
+                    while (own0 < blk) {  // padding (-1) and blocks the walk has passed
+                        own0 = own1;
+                        own1 = own2;
+                        own2 = own3;
+                        own3 = own_p < slots ? __ldg(own + own_p) : INT_MAX;
+                        ++own_p;
+                    }
+                    sel = own0 == blk;
+                } else {
+                    sel = (msk >> t) & 1u;
+                }
                 const int lim = !sel ? -1 : (diag ? i - blk * kBlk : kBlk - 1);  // last visible key
                 const uint32_t j = a & 1u, colS = colS0 + j * 64;
                 if (!dead && !mbar_wait(&bars.s_full[x][j], (a >> 1) & 1u, ctx)) fail();
@@ -627,8 +770,10 @@ bool sparse_prefill_tc_supported(int H, int Hkv, int d) {
 cudaError_t launch_sparse_prefill_tc(const void* q, const void* k, const void* v,
                                      const int32_t* idx, void* o, float* lse, void* o_lo, int B,
                                      int H, int Hkv, int N, int d, int slots, float scale,
-                                     cudaStream_t st, DevCtx ctx) {
+                                     bool per_head, cudaStream_t st, DevCtx ctx) {
     if (d != kD || H != Hkv * kG || slots > kMaxSlots) return cudaErrorNotSupported;
+    if (per_head && (lse != nullptr || o_lo != nullptr || (N + kBlk - 1) / kBlk > 32 * kMaxBmWords))
+        return cudaErrorNotSupported;
     CUtensorMap tmQ, tmK, tmV;
     EncodeTiledFn fn = encode_tiled_fn();
     if (!fn) return cudaErrorNotSupported;
@@ -654,19 +799,24 @@ cudaError_t launch_sparse_prefill_tc(const void* q, const void* k, const void* v
         if (num_sms <= 0) num_sms = 148;
     }
     const bool train = lse != nullptr;
-    cudaError_t e = train ? ensure_smem<sparse_prefill_tc_kernel<true>>(kSmemBytes)
-                          : ensure_smem<sparse_prefill_tc_kernel<false>>(kSmemBytes);
+    cudaError_t e = train      ? ensure_smem<sparse_prefill_tc_kernel<true, false>>(kSmemBytes)
+                    : per_head ? ensure_smem<sparse_prefill_tc_kernel<false, true>>(kSmemBytes)
+                               : ensure_smem<sparse_prefill_tc_kernel<false, false>>(kSmemBytes);
     if (e != cudaSuccess) return e;
     const int units_per_seq = (N + kUT - 1) / kUT;
     const int n_units = units_per_seq * B * Hkv;
     const int grid = n_units < num_sms ? n_units : num_sms;
     const float sl2 = scale * 1.4426950408889634f;
     if (train)
-        sparse_prefill_tc_kernel<true><<<grid, kThreads, kSmemBytes, st>>>(
+        sparse_prefill_tc_kernel<true, false><<<grid, kThreads, kSmemBytes, st>>>(
             tmQ, tmK, tmV, idx, static_cast<__nv_bfloat16*>(o), lse,
             static_cast<__nv_bfloat16*>(o_lo), H, Hkv, N, slots, sl2, n_units, ctx);
+    else if (per_head)
+        sparse_prefill_tc_kernel<false, true><<<grid, kThreads, kSmemBytes, st>>>(
+            tmQ, tmK, tmV, idx, static_cast<__nv_bfloat16*>(o), nullptr, nullptr, H, Hkv, N, slots,
+            sl2, n_units, ctx);
     else
-        sparse_prefill_tc_kernel<false><<<grid, kThreads, kSmemBytes, st>>>(
+        sparse_prefill_tc_kernel<false, false><<<grid, kThreads, kSmemBytes, st>>>(
             tmQ, tmK, tmV, idx, static_cast<__nv_bfloat16*>(o), nullptr, nullptr, H, Hkv, N, slots,
             sl2, n_units, ctx);
     return cudaGetLastError();

@@ -48,9 +48,11 @@ _lib.sala_block_topk.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, 
 _lib.sala_block_topk_workspace.argtypes = [_i, _i, _i, _i, _i, _i, _i]
 _lib.sala_block_topk_qblock.argtypes = [_vp, _vp, _vp] + [_i] * 11 + [_vp]
 _lib.sala_block_topk_qblock_softmax.argtypes = [_vp, _vp, _vp] + [_i] * 10 + [ctypes.c_float, _i, _vp]
+_lib.sala_block_topk_per_head.argtypes = [_vp, _vp, _vp] + [_i] * 11 + [_vp]
 _lib.sala_block_topk_workspace.restype = _st
 _lib.sala_sparse_prefill.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i,
                                      ctypes.c_float, _i, _vp]
+_lib.sala_sparse_prefill_per_head.argtypes = _lib.sala_sparse_prefill.argtypes
 _lib.sala_sparse_decode.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i,
                                     _i, _i, _i, _i, ctypes.c_float, _vp, _st, _i, _vp]
 _lib.sala_sparse_decode_pdl.argtypes = _lib.sala_sparse_decode.argtypes
@@ -75,6 +77,7 @@ for _f in ("sala_linear_prefill", "sala_linear_decode", "sala_linear_prefill_rop
            "sala_linear_decode_rope", "sala_sparse_decode_paged", "sala_block_topk_qblock",
            "sala_linear_backward", "sala_qk_norm", "sala_sparse_prefill_lse", "sala_sparse_backward",
            "sala_block_topk_qblock_softmax", "sala_linear_decode_pdl", "sala_qk_prologue",
+           "sala_block_topk_per_head", "sala_sparse_prefill_per_head",
            "sala_block_compress",
            "sala_block_topk",
            "sala_sparse_prefill", "sala_sparse_decode", "sala_sparse_decode_pdl", "sala_check_status",
@@ -321,6 +324,41 @@ def block_topk_qblock_softmax(q, kbar, topk, n_init, n_local, idx=None, block=64
                                                _dt(q), _stream(stream)),
            "sala_block_topk_qblock_softmax")
     return idx
+
+
+def block_topk_per_head(q, kbar, topk, n_init, n_local, idx=None, block=64, stream=None):
+    """Per-query-head selection (each query head scores the candidates with its own query against
+    its KV head's kbar).  q: [B,H,Nq,d]; kbar [B,Hkv,nb,d].  Returns idx [B,H,Nq,slots] int32."""
+    B, H, Nq, d = q.shape
+    Hkv, nb = kbar.shape[1], kbar.shape[2]
+    slots = n_init + n_local + topk
+    _need(q, "q"); _need(kbar, "kbar", dtype=q.dtype)
+    if idx is None:
+        idx = torch.empty((B, H, Nq, slots), dtype=torch.int32, device=q.device)
+    _need(idx, "idx", (B, H, Nq, slots), torch.int32)
+    _check(_lib.sala_block_topk_per_head(_ptr(q), _ptr(kbar), _ptr(idx), B, H, Hkv, Nq, nb, d,
+                                         block, topk, n_init, n_local, _dt(q), _stream(stream)),
+           "sala_block_topk_per_head")
+    return idx
+
+
+def sparse_prefill_per_head(q, k, v, idx, o=None, block=64, scale=0.0, stream=None):
+    """Softmax attention over per-head selections.  q: [B,H,N,d]; k,v: [B,Hkv,N,d];
+    idx [B,H,N,slots] int32 (block_topk_per_head's output)."""
+    B, H, N, d = q.shape
+    Hkv = k.shape[1]
+    _need(q, "q"); _need(k, "k", (B, Hkv, N, d), q.dtype); _need(v, "v", (B, Hkv, N, d), q.dtype)
+    _need(idx, "idx", dtype=torch.int32)
+    if idx.shape[:3] != (B, H, N):
+        raise ValueError(f"idx has shape {tuple(idx.shape)}, expected ({B}, {H}, {N}, slots)")
+    if o is None:
+        o = torch.empty_like(q)
+    _need(o, "o", q.shape, q.dtype)
+    _check(_lib.sala_sparse_prefill_per_head(_ptr(q), _ptr(k), _ptr(v), _ptr(idx), _ptr(o), B, H,
+                                             Hkv, N, d, block, idx.shape[3], float(scale), _dt(q),
+                                             _stream(stream)),
+           "sala_sparse_prefill_per_head")
+    return o
 
 
 def sparse_prefill(q, k, v, idx, o=None, block=64, scale=0.0, stream=None, lse=None, o_lo=None):

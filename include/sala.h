@@ -267,6 +267,22 @@ sala_status sala_block_topk_qblock_softmax(const void* q, const void* kbar, int3
                                            int topk, int n_init, int n_local, float scale,
                                            sala_dtype dt, sala_stream stream);
 
+/* Per-query-head selection: every query head chooses its own blocks.  Another reading of the
+ * open selection step (the pages: InfLLM-V2 picks the relevant context blocks for each query,
+ * gist.science JA technical summary section 2.1, without saying whether a KV group's heads share
+ * the choice).  For each (batch, query head h, query row i) the score of candidate b is
+ * q[b,h,i] . kbar[b, h / (H/Hkv), b]; candidates (n_init .. c - n_local), forced blocks, ties
+ * (the lower block wins) and the row layout are those of sala_block_topk with q_pos0 = 0.  bf16
+ * with d 128, Nq > 16 and topk <= 64 scores on the tensor cores (the query split into two bf16
+ * terms, as sala_block_topk); other shapes and fp32 on CUDA cores.
+ * q   : [B, H, Nq, d] device, dt.   kbar : [B, Hkv, nb, d] device, dt.
+ * idx : [B, H, Nq, n_init + n_local + topk] int32 device (output), one row per query head.
+ * Validation and errors as sala_block_topk (block = 64; topk <= 64 whenever a row has more than
+ * topk candidates). */
+sala_status sala_block_topk_per_head(const void* q, const void* kbar, int32_t* idx, int B, int H,
+                                     int Hkv, int Nq, int nb, int d, int block, int topk,
+                                     int n_init, int n_local, sala_dtype dt, sala_stream stream);
+
 /* ------------------------------------------------------------------------------------------
  * Sparse attention prefill: exact causal softmax over the selected blocks.  Pages: sparse
  * layers compute on selected parts but keep the dense KV cache ("sparse compute, dense
@@ -286,6 +302,20 @@ sala_status sala_block_topk_qblock_softmax(const void* q, const void* kbar, int3
 sala_status sala_sparse_prefill(const void* q, const void* k, const void* v, const int32_t* idx,
                                 void* o, int B, int H, int Hkv, int N, int d, int block,
                                 int slots, float scale, sala_dtype dt, sala_stream stream);
+
+/* Sparse attention prefill over per-head selections (sala_block_topk_per_head's output):
+ *   J(b,h,i) = { j <= i : j / block in idx[b, h, i, :] },  o as sala_sparse_prefill.
+ * idx  : [B, H, N, slots] int32 device, each row ascending among its non-negative entries and -1
+ *        padded; entries past the row's query block are skipped and flagged SALA_ERR_BOUNDS.
+ * Other arguments, shapes and errors as sala_sparse_prefill.  bf16 with H = 16 Hkv, d 128,
+ * slots <= 80 and N <= 2^20 runs on the tensor cores: each 16-token unit of a KV group walks the
+ * union of its 16 heads' x 16 tokens' selections, and every row keeps only its own blocks; other
+ * shapes and fp32 run on CUDA cores, one query head per CTA.
+ */
+sala_status sala_sparse_prefill_per_head(const void* q, const void* k, const void* v,
+                                         const int32_t* idx, void* o, int B, int H, int Hkv, int N,
+                                         int d, int block, int slots, float scale, sala_dtype dt,
+                                         sala_stream stream);
 
 /* ------------------------------------------------------------------------------------------
  * Training path of the sparse layers: the forward with its row statistic, and the backward pass.

@@ -106,6 +106,26 @@ def test_empty_problems_are_noops(lib):
                                    ctypes.c_float(0.0), 1, None) == 0
     assert lib.sala_block_compress(None, None, 1, 2, 64, 128, 64, 0, 0, 1, 1, None) == 0
     assert lib.sala_block_topk(None, None, None, 1, 4, 2, 0, 0, 0, 128, 64, 2, 1, 1, None, 0, 1, None) == 0
+    assert lib.sala_block_topk_per_head(None, None, None, 1, 4, 2, 0, 0, 128, 64, 2, 1, 1, 1, None) == 0
+    assert lib.sala_sparse_prefill_per_head(None, None, None, None, None, 1, 4, 2, 0, 128, 64, 3,
+                                            ctypes.c_float(0.0), 1, None) == 0
+
+
+def test_per_head_calls_validate_before_launch(lib):
+    vp = ctypes.c_void_p
+    lib.sala_last_error.restype = ctypes.c_char_p
+    good = vp(1 << 20)  # never dereferenced: every case below fails validation first
+    # block 32 is unsupported
+    r = lib.sala_block_topk_per_head(good, good, good, 1, 4, 2, 64, 2, 128, 32, 2, 1, 1, 1, None)
+    assert r == 2
+    # H not a multiple of Hkv
+    r = lib.sala_sparse_prefill_per_head(good, good, good, good, good, 1, 5, 2, 64, 128, 64, 3,
+                                         ctypes.c_float(0.0), 1, None)
+    assert r == 1 and b"multiple" in lib.sala_last_error()
+    # NULL idx with work to do
+    r = lib.sala_sparse_prefill_per_head(good, good, good, None, good, 1, 4, 2, 64, 128, 64, 3,
+                                         ctypes.c_float(0.0), 1, None)
+    assert r == 1 and b"idx" in lib.sala_last_error()
 
 
 def test_product_never_imports_the_oracle():
