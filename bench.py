@@ -68,13 +68,13 @@ def sparse_layer_flops(N: int) -> float:
 
 
 # DRAM traffic of the sparse prefill kernel (dram__bytes_read.sum + dram__bytes_write.sum) from one
-# ncu capture of the single-layer N = 131072 case, 2.317e9 bytes per launch, scaled by the tokens
+# ncu capture of the single-layer N = 131072 case, 2.323e9 bytes per launch, scaled by the tokens
 # processed to N = 262144 (Q reads, O writes and the K/V re-reads per 16-token unit all grow with N).
 # Valid only for the kernel sources it was taken on: any change to them reports null.
-SPARSE_TRAFFIC = {"bytes_per_token": 2.31670912e9 / 131072,
-                  "sources": {"sparse_tc.cu": "197c07812f3e1039106bc2a1e2262b5b5d9e92f6a70a88d57aae48dea8a1e9ce",
+SPARSE_TRAFFIC = {"bytes_per_token": (1287155200 + 1035656960) / 131072,
+                  "sources": {"sparse_tc.cu": "71ff73bea6734e4ba25f214f086e3ad2f0bacd0a1b9d8d7c123393baa9edd39c",
                               "fastexp.cuh": "b6d9ae064f35b9fd752ec893180eaf72ade6f0495d57f5699832618f42784c06",
-                              "ptx.cuh": "4958f3527272a2b6168ae878bd0b9208adb2bddd1e7053b6eaae10a36fd1d5fb"}}
+                              "ptx.cuh": "fd104364a691e71bb755a0a84573920e3263e23dbfbee024db781170b73eb422"}}
 
 
 def sparse_traffic(N: int):
@@ -95,8 +95,15 @@ def sparse_traffic(N: int):
 EXEC_FLOPS_PER_TILE_BLOCK = 2.0 * 128 * 64 * 128 * 2
 
 
-def tile_union_blocks(torch, idx, tq: int = 8) -> int:
-    """Sum over 8-token tiles of |union of the tile's selections| (idx [B, Hkv, N, slots], -1 pad)."""
+def tile_union_blocks(torch, idx, tq: int = 8, heads: int = 1) -> int:
+    """Sum over 8-token tiles of |union of the tile's selections| (idx [B, Hkv, N, slots], -1 pad).
+    heads > 1: idx is [B, Hkv * heads, N, slots], one row per query head, and a tile's union runs
+    over its 8 tokens of all `heads` heads of the KV group (one KV group at a time)."""
+    if heads > 1:
+        B, Hq, N, S = idx.shape
+        return sum(tile_union_blocks(torch, idx[:, g * heads:(g + 1) * heads].permute(0, 2, 1, 3)
+                                     .reshape(B, 1, N, heads * S), tq)
+                   for g in range(Hq // heads))
     B, G, N, S = idx.shape
     pad = (-N) % tq
     if pad:
@@ -240,6 +247,8 @@ WORKLOADS = {
     # a sparse layer whose 64-token query blocks each share one selection (the variant)
     "sparse_qblock_prefill_n256k": (N_TOK, ["sparse_qblock"]),
     "sparse_qblock_softmax_prefill_n256k": (N_TOK, ["sparse_qsoft"]),
+    # a sparse layer whose query heads each choose their own blocks (the per-head variant)
+    "sparse_per_head_prefill_n256k": (N_TOK, ["sparse_per_head"]),
     "linear_rope_prologue_prefill_n256k": (N_TOK, ["linear_rope_pro"]),
 }
 
@@ -251,7 +260,7 @@ def run_prefill(sala, synth, torch, steps, warmup, stream, workload="hybrid_pref
     lam = synth.decays(H).to(dev)
     layers = []
     for l, kind in enumerate(kinds):
-        if kind in ("sparse", "sparse_qblock", "sparse_qsoft"):
+        if kind.startswith("sparse"):
             sl = synth.sparse_layer(1, H, HKV, n_tok, D, torch.bfloat16, dev, layer=l)
             layers.append((kind, sl.q, sl.k, sl.v))
         else:
@@ -261,7 +270,8 @@ def run_prefill(sala, synth, torch, steps, warmup, stream, workload="hybrid_pref
     nb = n_tok // BLOCK
     kbar = torch.empty((1, HKV, nb, D), device=dev, dtype=torch.bfloat16)
     slots = N_INIT + N_LOCAL + TOPK
-    idx = torch.empty((1, HKV, n_tok, slots), device=dev, dtype=torch.int32)
+    sel_heads = H if "sparse_per_head" in kinds else HKV   # selection rows per token
+    idx = torch.empty((1, sel_heads, n_tok, slots), device=dev, dtype=torch.int32)
     # scratch of the sequence-parallel linear prefill (the segments' states)
     lws = torch.empty(max(sala.linear_prefill_workspace_bytes(1, H, n_tok, D), 16), device=dev,
                       dtype=torch.uint8)
@@ -274,6 +284,16 @@ def run_prefill(sala, synth, torch, steps, warmup, stream, workload="hybrid_pref
 
     ev = lambda: torch.cuda.Event(enable_timing=True)
     sparse_ev, linear_ev, topk_ev = [], [], []
+
+    def select(kind, q):
+        if kind == "sparse":
+            sala.block_topk(q, kbar, TOPK, N_INIT, N_LOCAL, idx=idx, stream=stream)
+        elif kind == "sparse_qblock":
+            sala.block_topk_qblock(q, kbar, TOPK, N_INIT, N_LOCAL, idx=idx, stream=stream)
+        elif kind == "sparse_per_head":
+            sala.block_topk_per_head(q, kbar, TOPK, N_INIT, N_LOCAL, idx=idx, stream=stream)
+        else:
+            sala.block_topk_qblock_softmax(q, kbar, TOPK, N_INIT, N_LOCAL, idx=idx, stream=stream)
 
     def one_step(record):
         launches = 0
@@ -297,17 +317,14 @@ def run_prefill(sala, synth, torch, steps, warmup, stream, workload="hybrid_pref
                 t0, t1 = (ev(), ev()) if record else (None, None)
                 if record: t0.record(stream)
                 sala.block_compress(k, kbar, stream=stream)
-                if kind == "sparse":
-                    sala.block_topk(q, kbar, TOPK, N_INIT, N_LOCAL, idx=idx, stream=stream)
-                elif kind == "sparse_qblock":
-                    sala.block_topk_qblock(q, kbar, TOPK, N_INIT, N_LOCAL, idx=idx, stream=stream)
-                else:
-                    sala.block_topk_qblock_softmax(q, kbar, TOPK, N_INIT, N_LOCAL, idx=idx,
-                                                   stream=stream)
+                select(kind, q)
                 if record: t1.record(stream); topk_ev.append((t0, t1))
                 e0, e1 = (ev(), ev()) if record else (None, None)
                 if record: e0.record(stream)
-                sala.sparse_prefill(q, k, v, idx, o=out, stream=stream)
+                if kind == "sparse_per_head":
+                    sala.sparse_prefill_per_head(q, k, v, idx, o=out, stream=stream)
+                else:
+                    sala.sparse_prefill(q, k, v, idx, o=out, stream=stream)
                 if record: e1.record(stream); sparse_ev.append((e0, e1))
                 launches += 3
         return launches
@@ -337,16 +354,10 @@ def run_prefill(sala, synth, torch, steps, warmup, stream, workload="hybrid_pref
     union, n_sp = 0, 0
     with torch.cuda.stream(stream):
         for kind, q, k, v in layers:
-            if kind in ("sparse", "sparse_qblock", "sparse_qsoft"):
+            if kind.startswith("sparse"):
                 sala.block_compress(k, kbar, stream=stream)
-                if kind == "sparse":
-                    sala.block_topk(q, kbar, TOPK, N_INIT, N_LOCAL, idx=idx, stream=stream)
-                elif kind == "sparse_qblock":
-                    sala.block_topk_qblock(q, kbar, TOPK, N_INIT, N_LOCAL, idx=idx, stream=stream)
-                else:
-                    sala.block_topk_qblock_softmax(q, kbar, TOPK, N_INIT, N_LOCAL, idx=idx,
-                                                   stream=stream)
-                union += tile_union_blocks(torch, idx)
+                select(kind, q)
+                union += tile_union_blocks(torch, idx, heads=H // HKV if kind == "sparse_per_head" else 1)
                 n_sp += 1
     res["sparse_exec_flops"] = EXEC_FLOPS_PER_TILE_BLOCK * union / max(1, n_sp)
     del layers, out, kbar, idx
@@ -872,6 +883,20 @@ def config_lines(sala, synth, torch, stream, peaks, steps, warmup, decode=None, 
         rec["oracle"] = {"tokens_per_s": n / o["s"], "s": o["s"], "cores": o["cores"],
                          "sample": o["sample"]}
     out["sparse_prefill_n128k"] = rec
+    n = N_TOK
+    pre = run_prefill(sala, synth, torch, steps, warmup, stream, "sparse_per_head_prefill_n256k")
+    ms = pre["total_ms"] / steps
+    fl = sparse_layer_flops(n)
+    out["sparse_per_head_prefill_n256k"] = {
+        "workload": "sparse_per_head_prefill_n256k (selection variant): B=1, 32 query / 2 KV heads, "
+                    "d=128, N=262144, bf16, block 64, top-64 + init + 2 local chosen per query head",
+        "tokens_per_s": n / (ms * 1e-3), "ms": ms, "bound": "tensor",
+        "attention_ms": pre["sparse_ms"], "selection_ms": pre["select_ms"],
+        "achieved_tflops": fl / (pre["sparse_ms"] * 1e-3) / 1e12,
+        "roofline_frac": fl / (pre["sparse_ms"] * 1e-3) / 1e12 / tc,
+        "executed_frac": pre["sparse_exec_flops"] / (pre["sparse_ms"] * 1e-3) / 1e12 / tc,
+        "union_overhead": pre["sparse_exec_flops"] / fl,
+        "algorithmic_flops": fl, "peak": f"{tc} TFLOP/s bf16 sustained ({peaks['source']})"}
     if decode is not None:
         us = decode["us_per_token"]
         db = decode_bytes(DECODE_T)
@@ -986,7 +1011,7 @@ def main():
             line["config"]["workload"] = f"{args.workload}: {len(kinds)} x {kinds[0]} layer, N={n_tok}"
             line["config"]["seq_len"] = n_tok
         line["kernels"] = {}
-        if "sparse" in kinds or "sparse_qblock" in kinds or "sparse_qsoft" in kinds:
+        if any(k.startswith("sparse") for k in kinds):
             fl = sparse_layer_flops(n_tok)
             achieved = fl / (pre["sparse_ms"] / 1000.0) / 1e12
             executed = pre["sparse_exec_flops"] / (pre["sparse_ms"] / 1000.0) / 1e12
@@ -1001,7 +1026,8 @@ def main():
                                 "executed_flops_per_launch": pre["sparse_exec_flops"],
                                 "executed_tflops": executed, "executed_frac": executed / peak}
             line["kernels"]["sparse_prefill"] = {"mean_ms": pre["sparse_ms"], "achieved_tflops": achieved,
-                                                 "executed_tflops": executed}
+                                                 "executed_tflops": executed,
+                                                 "union_overhead": pre["sparse_exec_flops"] / fl}
             line["kernels"]["compress_plus_select"] = {"mean_ms": pre["select_ms"]}
         if "linear" in kinds or "linear_rope" in kinds or "linear_rope_pro" in kinds:
             lin_gbs = linear_layer_bytes(n_tok) / (pre["linear_ms"] / 1000.0) / 1e9
