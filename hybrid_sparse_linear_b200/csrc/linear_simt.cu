@@ -166,8 +166,11 @@ cudaError_t prefill_simt(const void* q, const void* k, const void* v, const floa
 // kPdl: launched as a programmatic dependent of the previous kernel in the stream.  The state
 // row is requested first, while that kernel may still run (the caller guarantees it does not
 // write this state); q, k, v and the decays are read after griddepcontrol.wait, i.e. after it
-// has completed and its writes are visible.  Only then may the next kernel launch, so a
-// dependent's early reads overlap this kernel alone, never the one before it.
+// has completed and its writes are visible.  Before the wait their lines are only pulled into
+// L2: L2 is where every SM's writes land, so a line fetched there early is updated by any later
+// write of the previous kernel, and nothing is held in this SM's L1 or registers.  Only after the
+// wait may the next kernel launch, so a dependent's early reads overlap this kernel alone, never
+// the one before it.
 template <typename T, int D, bool kRope, bool kPdl>
 __global__ void __launch_bounds__(2 * D)
 linear_decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
@@ -183,6 +186,13 @@ linear_decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* 
     float4* row = reinterpret_cast<float4*>(state + (bh * D + a) * D + c0);
     float4 s0 = row[0], s1 = row[1];
     if constexpr (kPdl) {
+        constexpr int kLines = D * (int)sizeof(T) / 128;  // 128-byte lines of a q or k row
+        const void* line = nullptr;
+        if (tid < kLines) line = reinterpret_cast<const char*>(q + bh * D) + 128 * tid;
+        else if (tid < 2 * kLines) line = reinterpret_cast<const char*>(k + bh * D) + 128 * (tid - kLines);
+        else if (tid == 2 * kLines) line = v + bh * D + blockIdx.x * kCols;
+        else if (tid == 2 * kLines + 1) line = decay + bh % H;
+        if (line != nullptr) asm volatile("prefetch.global.L2 [%0];" ::"l"(line));
         asm volatile("griddepcontrol.wait;" ::: "memory");
         asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     }

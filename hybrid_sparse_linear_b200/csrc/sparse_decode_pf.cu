@@ -301,6 +301,10 @@ decode_score_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __
         ptx::cp_async16(&sm.rows[r][piece * 8], kb + (ok ? (int64_t)cand * D + piece * 8 : 0), ok);
     }
     ptx::cp_async_commit();
+    // the group's query rows (G x D bf16, 128-byte lines) are pulled into L2 only: the previous
+    // kernel's writes land there, so they are read for real after the wait
+    if (tid < G * D / 64)
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(q + (b * H + (int64_t)g * G) * D + 64 * tid));
     asm volatile("griddepcontrol.wait;" ::: "memory");
     // the attend kernel may start now: its own early reads come after the previous kernel
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
