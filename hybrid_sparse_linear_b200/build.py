@@ -1,5 +1,6 @@
-"""Build libsala.so (the product kernels + C ABI) and libsala_selftest.so (tensor-core layout
-self-test used by the tests) in-tree, for sm_100a only.
+"""Build libsala.so (the product kernels + C ABI), libsala_debug.so (the same with the
+SALA_DEBUG_BOUNDS index checks) and libsala_selftest.so (tensor-core layout self-test used by the
+tests) in-tree, for sm_100a only.
 
     python -m hybrid_sparse_linear_b200.build [--force] [-j N]
 
@@ -22,6 +23,7 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libsala.so")
+DEBUG_LIB = os.path.join(HERE, "libsala_debug.so")   # the same kernels with -DSALA_DEBUG_BOUNDS
 SELFTEST_LIB = os.path.join(HERE, "libsala_selftest.so")
 SELFTEST_SRC = {"selftest_mma.cu"}
 
@@ -49,8 +51,8 @@ def _stale(target: str, deps) -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def _compile(src: str, force: bool, extra=()) -> str:
-    obj = os.path.join(BUILD, os.path.basename(src) + ".o")
+def _compile(src: str, force: bool, extra=(), tag: str = "") -> str:
+    obj = os.path.join(BUILD, os.path.basename(src) + tag + ".o")
     if force or _stale(obj, [src] + _headers()):
         cmd = [nvcc(), *ARCH, *NVCC_FLAGS, *extra, "-c", src, "-o", obj]
         r = subprocess.run(cmd, capture_output=True, text=True)
@@ -75,11 +77,16 @@ def build(force: bool = False, jobs: int | None = None, verbose_ptxas: bool = Fa
     os.makedirs(BUILD, exist_ok=True)
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     extra = ["-Xptxas", "-v"] if verbose_ptxas else []
+    lib_srcs = [s for s in srcs if os.path.basename(s) not in SELFTEST_SRC]
     with cf.ThreadPoolExecutor(max_workers=jobs or os.cpu_count() or 4) as ex:
         futs = {s: ex.submit(_compile, s, force, extra) for s in srcs}
+        dfuts = {s: ex.submit(_compile, s, force, [*extra, "-DSALA_DEBUG_BOUNDS"], ".dbg")
+                 for s in lib_srcs}
         objs = {os.path.basename(s): f.result() for s, f in futs.items()}
+        dobjs = [f.result() for f in dfuts.values()]
     _link([o for n, o in objs.items() if n not in SELFTEST_SRC], LIB, force)
     _link([o for n, o in objs.items() if n in SELFTEST_SRC], SELFTEST_LIB, force)
+    _link(dobjs, DEBUG_LIB, force)
     return LIB
 
 

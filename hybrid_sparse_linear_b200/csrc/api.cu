@@ -85,6 +85,8 @@ extern "C" {
 
 int sala_version(void) { return 100; }
 
+int sala_debug_bounds_build(void) { return sala::kDebugBounds ? 1 : 0; }
+
 const char* sala_status_string(sala_status s) {
     switch (s) {
         case SALA_OK: return "SALA_OK";

@@ -21,6 +21,25 @@ struct DevCtx {
 
 __device__ __forceinline__ void flag(const DevCtx& c, unsigned bits) { atomicOr(c.status, bits); }
 
+// Index checks of the debug build (compiled with -DSALA_DEBUG_BOUNDS into libsala_debug.so):
+// in_bounds(c, ok) records kStatusBounds when ok is false and returns ok, so the caller skips the
+// access instead of making it; the release build folds it to true and emits nothing.
+#ifdef SALA_DEBUG_BOUNDS
+constexpr bool kDebugBounds = true;
+#else
+constexpr bool kDebugBounds = false;
+#endif
+__device__ __forceinline__ bool in_bounds(const DevCtx& c, bool ok) {
+    if constexpr (kDebugBounds) {
+        if (!ok) flag(c, kStatusBounds);
+        return ok;
+    } else {
+        (void)c;
+        (void)ok;
+        return true;
+    }
+}
+
 __device__ __forceinline__ uint64_t globaltimer_ns() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

@@ -415,7 +415,10 @@ topk_tc_kernel(const __grid_constant__ CUtensorMap tmKb, const __nv_bfloat16* __
                     if (key[e] && (key[e] & mask) >= prefix) bars.carry[atomicAdd(&bars.n_win, 1)] = key[e];
                 sync_workers();
             }
-            if (tid < kSeeds) bars.seeds[tid] = key_block(bars.carry[tid]);
+            if (tid < kSeeds) {
+                const int sd = key_block(bars.carry[tid]);
+                bars.seeds[tid] = in_bounds(ctx, sd >= lo && sd <= hi_all) ? sd : lo;
+            }
             if (tid == 0) bars.n_seeds = kSeeds;
             sync_workers();
             // seed kbar rows -> B operand (K-major, 128-byte swizzle); all loads in flight first
@@ -528,7 +531,8 @@ topk_tc_kernel(const __grid_constant__ CUtensorMap tmKb, const __nv_bfloat16* __
                 auto append = [&](uint32_t msk) {
 #pragma unroll
                     for (int j = 0; j < 32; ++j)
-                        if ((msk >> j) & 1u) buf[n++] = sel_key(__uint_as_float(x[j]), jb + j);
+                        if (((msk >> j) & 1u) && in_bounds(ctx, n < kBufCap))
+                            buf[n++] = sel_key(__uint_as_float(x[j]), jb + j);
                 };
                 const uint32_t pass = passing(~0u);
                 if (__any_sync(0xffffffffu, n + __popc(pass) > kBufCap)) {

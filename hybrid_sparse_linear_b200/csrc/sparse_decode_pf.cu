@@ -564,7 +564,8 @@ decode_attend_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
     // warp w < nitems attends slot rk + w CS in stage w and leaves the slot's partial (per head:
     // max, sum, sum of p v) at the start of the stage
     if (warp < nitems) {
-        const int blk = sm.sel[rk + warp * CS];
+        int blk = sm.sel[rk + warp * CS];
+        if (blk >= 0 && !in_bounds(ctx, blk <= c)) blk = -1;
         float* out = reinterpret_cast<float*>(stage_k(warp));
         if (blk >= 0) {
             if (!(preloaded && rank_layout)) {  // the early copy is this slot's block only on the rank path

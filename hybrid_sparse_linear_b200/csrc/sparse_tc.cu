@@ -316,7 +316,7 @@ sparse_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
 #pragma unroll
                     for (int j = 0; j < kPer; ++j) {
                         const int e = lane + 32 * j;
-                        if (e < total) stage[e] = v[j];
+                        if (e < total && in_bounds(ctx, e < kUT * kMaxSlots)) stage[e] = v[j];
                     }
                 }
                 __syncwarp();
@@ -340,7 +340,7 @@ sparse_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                     }
                     if (lane == 0) {
                         if (m == prev) {
-                            list_mask(lb)[n - 1] |= (uint16_t)msk;
+                            if (in_bounds(ctx, n >= 1 && n <= kMaxList)) list_mask(lb)[n - 1] |= (uint16_t)msk;
                         } else if (n < kMaxList) {
                             list_id(lb)[n] = m;
                             list_mask(lb)[n] = (uint16_t)msk;
@@ -383,7 +383,7 @@ sparse_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                             const int m = v[u][j];
                             if (m > c) {  // in the future of every token of the unit
                                 bad = true;
-                            } else if (m >= 0) {
+                            } else if (m >= 0 && in_bounds(ctx, (m >> 5) < nw && nw <= kMaxBmWords)) {
                                 const int e = lane + 32 * j;
                                 atomicOr((e < split ? bm_a : bm_b) + (m >> 5), 1u << (m & 31));
                             }
@@ -442,6 +442,7 @@ sparse_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                         int blk;
                         uint32_t m;
                         uw.next(blk, m);
+                        if (!in_bounds(ctx, blk >= 0 && blk <= i0 / kBlk)) blk = 0;  // load a real block
                         const int y = blk * kBlk;
                         tma_load_3d(st, &tmK, fb, 0, y, (int)bg);
                         tma_load_3d(st + kHalfBlk, &tmK, fb, 64, y, (int)bg);

@@ -14,7 +14,10 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libsala.so")
+# SALA_LIBRARY=debug loads the bounds-checking build (libsala_debug.so: the same kernels, with
+# out-of-range indices recorded as SALA_ERR_BOUNDS and skipped); anything else the release build.
+LIB_PATH = os.path.join(_HERE, "libsala_debug.so" if os.environ.get("SALA_LIBRARY") == "debug"
+                        else "libsala.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is missing: build it with `python -m hybrid_sparse_linear_b200.build`")
@@ -68,6 +71,7 @@ _lib.sala_sparse_backward_workspace.argtypes = [_i] * 6
 _lib.sala_sparse_backward_workspace.restype = _st
 _lib.sala_sparse_backward.argtypes = [_vp] * 11 + [_i] * 7 + [ctypes.c_float, _vp, _st, _i, _vp]
 _lib.sala_check_status.argtypes = [_vp]
+_lib.sala_debug_bounds_build.restype = _i
 _lib.sala_status_string.argtypes = [_i]
 _lib.sala_status_string.restype = ctypes.c_char_p
 _lib.sala_last_error.restype = ctypes.c_char_p
@@ -486,6 +490,11 @@ def sparse_decode_paged(q, k_pages, v_pages, page_table, kbar, pos, max_pos, top
                                          ctypes.c_float(scale), _ptr(workspace), workspace.numel(),
                                          _dt(q), _stream(stream)), "sala_sparse_decode_paged")
     return o
+
+
+def debug_bounds_build() -> bool:
+    """Whether the loaded library is the bounds-checking build."""
+    return bool(_lib.sala_debug_bounds_build())
 
 
 def check_status(stream=None):

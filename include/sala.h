@@ -504,6 +504,14 @@ sala_status sala_selftest_wait_timeout(sala_stream stream);
 /* Library version (major * 10000 + minor * 100 + patch). */
 int sala_version(void);
 
+/* 1 in the bounds-checking build (libsala_debug.so, compiled with SALA_DEBUG_BOUNDS), 0 in the
+ * release build (libsala.so).  The debug build runs the same kernels with checks on the indices
+ * that come from data or counters (selection rows, union lists and bitmaps, row buffers, seeds,
+ * decode slots, compressed blocks): an index that would leave its buffer records SALA_ERR_BOUNDS
+ * in the status word and the access is skipped instead of made.  It stands in for a memory
+ * checker on tiny cases; it is slower and not for production. */
+int sala_debug_bounds_build(void);
+
 #ifdef __cplusplus
 }
 #endif

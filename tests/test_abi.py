@@ -10,6 +10,7 @@ import pytest
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "sala.h")
 LIB = os.path.join(ROOT, "hybrid_sparse_linear_b200", "libsala.so")
+DEBUG_LIB = os.path.join(ROOT, "hybrid_sparse_linear_b200", "libsala_debug.so")
 
 
 def _declared():
@@ -43,6 +44,17 @@ def test_every_declared_symbol_is_exported(lib):
     assert not missing, missing
     for n in _declared():
         assert hasattr(lib, n)
+
+
+def test_debug_build_exports_the_same_boundary(lib):
+    # the bounds-checking build is a drop-in for the release one, and each says which it is
+    out = subprocess.run(["nm", "-D", "--defined-only", DEBUG_LIB], capture_output=True, text=True,
+                         check=True).stdout
+    exported = set(re.findall(r"\bT (sala_\w+)", out))
+    assert not [n for n in _declared() if n not in exported]
+    dbg = ctypes.CDLL(DEBUG_LIB)
+    assert dbg.sala_debug_bounds_build() == 1
+    assert lib.sala_debug_bounds_build() == 0
 
 
 def test_library_is_sm100a_only():
