@@ -331,8 +331,10 @@ linear_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
         const int t = tid;
         const uint32_t lb = tmem_lane_base(warp);
         const float wq = bars.pw[t + 1];
-        // Tile c+1 is masked before tile c's output is written: MMA2(c) and MMA3(c) then run
-        // while this warp group works on the next tile's scores.
+        // Per tile the warp group reads O(c), masks tile c+1, then stores o(c): reading O before
+        // the mask frees O1 and O2 early, so MMA2(c+1) and MMA3(c+1) -- the last readers of the
+        // stage of tile c+1 -- issue right after the mask (with the mask first they waited for
+        // the whole output step, and the ring's refill with them).
         auto mask = [&](int c) -> bool {  // A' = A * lambda^{t-s} [s <= t], bf16, over A in TMEM
             const int s = c & 1;
             if (!wait_or_abort(&bars.qk_done[s], (c >> 1) & 1, ctx, abort)) return false;
@@ -367,7 +369,10 @@ linear_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
             if (lane == 0) mbar_arrive(&bars.a_ready[s]);
             return true;
         };
-        auto output = [&](int c) -> bool {  // o_t = O1 + lambda^{t+1} O2
+        // o_t = O1 + lambda^{t+1} O2 in two steps.  read_out takes O1 and O2 of tile c out of TMEM
+        // and frees them at once (MMA2(c+1) and MMA3(c+1) wait for that), keeping the packed bf16
+        // row; store_out writes it once the next tile's mask is done.
+        auto read_out = [&](int c, uint32_t (&wp)[32]) -> bool {
             if (!wait_or_abort(&bars.o_done, c & 1, ctx, abort)) return false;
             tc_fence_after();
             uint32_t o1[64], o2[64];
@@ -379,12 +384,13 @@ linear_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars.o_free);
-            uint4 w[8];
-            uint32_t* wp = reinterpret_cast<uint32_t*>(w);
 #pragma unroll
             for (int j = 0; j < 32; ++j)
                 wp[j] = pack_bf16x2(fmaf(wq, __uint_as_float(o2[2 * j]), __uint_as_float(o1[2 * j])),
                                     fmaf(wq, __uint_as_float(o2[2 * j + 1]), __uint_as_float(o1[2 * j + 1])));
+            return true;
+        };
+        auto store_out = [&](int c, const uint32_t (&wp)[32]) {
             // The warp's 32 rows go out as one TMA store from its own 4 KiB of the staging tile
             // (128-byte swizzle, as the tensor map reads it): the previous tile's store from the
             // same rows must have read them first.  Rows past the sequence end are clipped by the
@@ -394,19 +400,24 @@ linear_prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
             __syncwarp();
 #pragma unroll
             for (int cj = 0; cj < 8; ++cj)
-                *reinterpret_cast<uint4*>(stg + lane * 128 + ((cj ^ (lane & 7)) << 4)) = w[cj];
+                *reinterpret_cast<uint4*>(stg + lane * 128 + ((cj ^ (lane & 7)) << 4)) =
+                    make_uint4(wp[4 * cj], wp[4 * cj + 1], wp[4 * cj + 2], wp[4 * cj + 3]);
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0 && c * kC + warp * 32 < Ns) {  // no store starts past the end
                 tma_store_3d(&tmO, stg, slice * kDv, row0 + c * kC + warp * 32, (int)bh);
                 bulk_commit();
             }
-            return true;
         };
+        // Per tile c: O(c) out of TMEM, then the mask of tile c+1 (MMA2(c+1) and MMA3(c+1) can
+        // issue as soon as it is done, and the stage of tile c+1 goes back to the producer right
+        // after them), then the store of o(c).
         bool ok = n_tiles > 0 ? mask(0) : true;
         for (int c = 0; c < n_tiles && ok; ++c) {
+            uint32_t wp[32];
+            if (!read_out(c, wp)) break;
             if (c + 1 < n_tiles && !mask(c + 1)) break;
-            ok = output(c);
+            store_out(c, wp);
         }
         if (lane == 0) bulk_wait0();  // this warp's stores complete before the CTA retires
     } else if (warp < 8) {
