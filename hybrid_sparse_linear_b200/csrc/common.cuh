@@ -83,6 +83,20 @@ __device__ __forceinline__ int key_block(uint64_t key) { return (int)(~(uint32_t
 
 __host__ __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
+// The current device's SM count, read once per device (any host thread may call it; a failed
+// query counts as a B200's 148).
+inline int device_sm_count() {
+    constexpr int kMaxDev = 64;
+    static std::atomic<int> cache[kMaxDev];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return 148;
+    int n = cache[dev].load(std::memory_order_relaxed);
+    if (n > 0) return n;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cache[dev].store(n, std::memory_order_relaxed);
+    return n;
+}
+
 // Raises a kernel's dynamic shared memory limit once per device, so later launches (including
 // ones recorded into a CUDA graph) only enqueue work.
 template <auto Kern>

@@ -754,16 +754,7 @@ bool linear_prefill_tc_supported(int d) { return d == kD; }
 
 namespace {
 
-int sm_count() {
-    static int n = 0;
-    if (!n) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        if (n <= 0) n = 148;
-    }
-    return n;
-}
+int sm_count() { return device_sm_count(); }
 
 // Segments for the sequence-parallel form: the count that minimises (waves of output-pass CTAs) x
 // (rows per segment) plus a per-segment cost for the state chaining (a segment boundary costs about

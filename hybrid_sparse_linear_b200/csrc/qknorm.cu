@@ -225,11 +225,12 @@ cudaError_t launch_qn(const void* q, void* qo, int64_t nq, const void* k, void* 
     if (total == 0) return cudaSuccess;
     constexpr int64_t kRowsPerBlock = (kThreads / 32) * (32 / (D * (int)sizeof(T) / 16)) * kU;
     // one wave: the SMs times the blocks resident per SM, the rows striding over it
-    static int wave = 0;
+    // (any positive count is correct: it only sizes the grid)
+    static std::atomic<int> wave_cache{0};
+    int wave = wave_cache.load(std::memory_order_relaxed);
     if (!wave) {
-        int dev = 0, n_sm = 0, per_sm = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+        const int n_sm = device_sm_count();
+        int per_sm = 0;
         if constexpr (kRope)
             cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, qk_rope_kernel<T, D, kNorm>,
                                                           kThreads, 0);
@@ -237,6 +238,7 @@ cudaError_t launch_qn(const void* q, void* qo, int64_t nq, const void* k, void* 
             cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, qk_norm_kernel<T, D, kNorm, false>,
                                                           kThreads, 0);
         wave = std::max(1, n_sm * std::max(1, per_sm));
+        wave_cache.store(wave, std::memory_order_relaxed);
     }
     const int64_t blocks = std::min<int64_t>((total + kRowsPerBlock - 1) / kRowsPerBlock, wave);
     if constexpr (kRope)

@@ -268,13 +268,14 @@ SparseBwdCsr sparse_bwd_csr_layout(void* ws, int B, int Hkv, int N, int slots) {
 cudaError_t launch_sparse_bwd_delta(const void* o, const void* o_lo, const void* dout,
                                     float* delta, int64_t rows, cudaStream_t st) {
     if (rows == 0) return cudaSuccess;
-    static int wave = 0;
+    // one wave of resident blocks, the rows striding over it (any positive count is correct)
+    static std::atomic<int> wave_cache{0};
+    int wave = wave_cache.load(std::memory_order_relaxed);
     if (!wave) {
-        int dev = 0, n_sm = 0, per_sm = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+        int per_sm = 0;
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, delta_kernel, kThreads, 0);
-        wave = std::max(1, n_sm * std::max(1, per_sm));
+        wave = std::max(1, device_sm_count() * std::max(1, per_sm));
+        wave_cache.store(wave, std::memory_order_relaxed);
     }
     const int64_t blocks = std::min<int64_t>((rows + 63) / 64, wave);
     delta_kernel<<<(unsigned)blocks, kThreads, 0, st>>>(static_cast<const uint4*>(o),

@@ -792,13 +792,7 @@ cudaError_t launch_sparse_prefill_tc(const void* q, const void* k, const void* v
         !make3(&tmK, k, (uint64_t)N, (uint64_t)B * Hkv, kBlk, 1) ||
         !make3(&tmV, v, (uint64_t)N, (uint64_t)B * Hkv, kBlk, 1))
         return cudaErrorInvalidValue;
-    static int num_sms = 0;
-    if (!num_sms) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
-        if (num_sms <= 0) num_sms = 148;
-    }
+    const int num_sms = device_sm_count();
     const bool train = lse != nullptr;
     cudaError_t e = train      ? ensure_smem<sparse_prefill_tc_kernel<true, false>>(kSmemBytes)
                     : per_head ? ensure_smem<sparse_prefill_tc_kernel<false, true>>(kSmemBytes)
