@@ -1,6 +1,6 @@
 """Full-size parity in the launch configuration the benchmark times: one sparse layer at
-N = 131072 and 262144 (32 query heads, 2 KV heads, d 128, top-64 + init + 2 local) and one linear
-layer at N = 262144.  The oracle checks sampled outputs one by one (first/last rows, block and tile
+N = 131072 and 262144 (32 query heads, 2 KV heads, d 128, top-64 + init + 2 local), the same with
+per-head selections at 262144, and one linear layer at N = 262144.  The oracle checks sampled outputs one by one (first/last rows, block and tile
 boundaries, the row where top-k starts to bind, random rows); compression is checked on every
 block, selection on the sampled rows with the near-tie rule."""
 import numpy as np
@@ -46,6 +46,36 @@ def test_sparse_layer_full_size(N):
         ref.append(oracle.sparse_attention(q64, k64, v64, gidx[:, :, r:r + 1], 64, q_pos0=r)[0, :, 0])
         got.append(f(o[0, :, r]))
     assert_close(np.stack(got), np.stack(ref), "bf16", f"sparse N={N} sampled rows")
+
+
+def test_sparse_layer_per_head_full_size():
+    # the per-query-head variant at the benchmark's N = 262144: selection rows per head, each head
+    # checked against the oracle's per-head selection (a group of one, its KV head's kbar), and
+    # the attention over every head's own blocks on sampled rows
+    from hybrid_sparse_linear_b200 import sala, synth
+    N = 262144
+    layer = synth.sparse_layer(1, 32, 2, N, 128, torch.bfloat16, "cuda", layer=8)
+    kbar = sala.block_compress(layer.k)
+    idx = sala.block_topk_per_head(layer.q, kbar, TOPK, N_INIT, N_LOCAL)
+    o = sala.sparse_prefill_per_head(layer.q, layer.k, layer.v, idx)
+    sala.check_status()
+    f = oracle.from_tensor
+    k64, v64 = f(layer.k), f(layer.v)
+    kbar_ref = oracle.block_compress(k64, 64)
+    np.testing.assert_array_equal(f(kbar), kbar_ref)
+    kbar_h = np.repeat(kbar_ref, 16, axis=1)
+    rows = _rows(N, N + 1)
+    gidx = idx.cpu().numpy()
+    got, ref = [], []
+    for r in rows:
+        q64 = f(layer.q[:, :, r:r + 1])
+        ridx, kth = oracle.block_select_per_head(q64, kbar_ref, 64, TOPK, N_INIT, N_LOCAL, q_pos0=r)
+        check_selection(gidx[:, :, r:r + 1], ridx, q64, kbar_h, kth, TOPK, N_INIT, N_LOCAL,
+                        q_pos0=r, row_ids=np.array([0]))
+        ref.append(oracle.sparse_attention_per_head(q64, k64, v64, gidx[:, :, r:r + 1], 64,
+                                                    q_pos0=r)[0, :, 0])
+        got.append(f(o[0, :, r]))
+    assert_close(np.stack(got), np.stack(ref), "bf16", "per-head sparse N=262144 sampled rows")
 
 
 def test_linear_layer_full_size():
