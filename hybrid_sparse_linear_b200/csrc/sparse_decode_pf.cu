@@ -64,6 +64,10 @@ template <int D>
 constexpr int row_elems() { return D + 8; }  // padded rows: conflict-free ldmatrix
 template <int D>
 constexpr size_t stage_bytes() { return (size_t)2 * kBlk * row_elems<D>() * 2; }
+// A head's softmax partial: maximum, sum, two unused words, then the D sums of p v -- rows of
+// D + 4 floats, so the p v part is read and sent to the combining CTA 16 bytes at a time.
+template <int D>
+constexpr int part_row() { return D + 4; }
 
 template <int D>
 struct ScoreSmem {
@@ -77,17 +81,17 @@ struct ScoreSmem {
 template <int D>
 struct AttendSmem {
     __nv_bfloat16 Qb[kMaxG][D + 8];
-    uint64_t u[kMaxCpg * kPub];       // the group's lists
-    int cnt_part[kWarps][kPub * 2 + 1];
+    alignas(16) uint64_t u[kMaxCpg * kPub];  // the group's lists (read two at a time)
+    int cnt_part[kWarps][2];          // per warp: nonzero keys of U, keys of U above X
     uint64_t xpart[kWarps];
     int sel[kMaxSlots];               // slot -> block (-1: empty)
-    int overflow;
+    int wblk[kCap];                   // CTA 0, with idx_out: the winners' blocks by rank
     uint64_t wkeys[kCap];
     int nwin;
     RadixSelSmem ss;
     float wt[kStages][kMaxG];         // fold: weight of each slot's partial per head
     float fm[kMaxG], fl[kMaxG];       // fold: largest maximum and weighted sum per head
-    float recv[kMaxG / kCS][kCS][D + 2];  // partials of the heads this CTA combines, from every CTA
+    alignas(16) float recv[kMaxG / kCS][kCS][part_row<D>()];  // partials of the heads this CTA combines
     alignas(128) unsigned char stages[kStages * stage_bytes<D>()];
 };
 
@@ -175,7 +179,7 @@ __device__ void radix_kth_stream(const uint64_t* keys, int n, int K, RadixSelSme
 // m16n8k16 tile row per head (16 x 64), the softmax runs in registers (a head's row lives in the 4
 // lanes of a quad), and P -- rounded to bf16 -- becomes the A fragments of P V directly.  Writes
 // out[h][0] = the head's maximum logit (log2 units), out[h][1] = the sum of its probabilities and
-// out[h][2 ..] = the unnormalised sum of p v, for heads h < G.
+// out[h][4 ..] = the unnormalised sum of p v, for heads h < G (rows of part_row<D>() floats).
 template <int D>
 __device__ __forceinline__ void slot_partial(const __nv_bfloat16* __restrict__ Qs, const __nv_bfloat16* __restrict__ Ks,
                                              const __nv_bfloat16* __restrict__ Vs, int lim, float scale_log2, int G,
@@ -255,14 +259,14 @@ __device__ __forceinline__ void slot_partial(const __nv_bfloat16* __restrict__ Q
 #pragma unroll
         for (int n = 0; n < kHalf / 8; ++n) {
             const int col = h0 + 8 * n + t2;
-            if (gq < G) *reinterpret_cast<float2*>(out + gq * (D + 2) + 2 + col) = make_float2(ov[n][0], ov[n][1]);
+            if (gq < G) *reinterpret_cast<float2*>(out + gq * part_row<D>() + 4 + col) = make_float2(ov[n][0], ov[n][1]);
             if (gq + 8 < G)
-                *reinterpret_cast<float2*>(out + (gq + 8) * (D + 2) + 2 + col) = make_float2(ov[n][2], ov[n][3]);
+                *reinterpret_cast<float2*>(out + (gq + 8) * part_row<D>() + 4 + col) = make_float2(ov[n][2], ov[n][3]);
         }
     }
     if ((lane & 3) == 0) {
-        if (gq < G) *reinterpret_cast<float2*>(out + gq * (D + 2)) = make_float2(mx0, l0);
-        if (gq + 8 < G) *reinterpret_cast<float2*>(out + (gq + 8) * (D + 2)) = make_float2(mx1, l1);
+        if (gq < G) *reinterpret_cast<float2*>(out + gq * part_row<D>()) = make_float2(mx0, l0);
+        if (gq + 8 < G) *reinterpret_cast<float2*>(out + (gq + 8) * part_row<D>()) = make_float2(mx1, l1);
     }
 }
 
@@ -467,9 +471,10 @@ decode_attend_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
     }
 
     // ---------------------------------------------------------------- the slot list
-    bool rank_layout = false;  // slots 0 .. K-1: the winners ascending by block, then the forced blocks
+    bool rank_layout = false;  // slots 0 .. K-1: the winners by rank, then the forced blocks
+    int nwin = 0;              // winners on the rank path (min(K, nonzero keys of U))
     if (owner) {
-        // U, the group's lists, in registers; the K-th largest key of U by a radix select
+        // U, the group's lists, into shared memory; X, the largest key any list left out
         const int nu = cpg * kPub;
         const uint64_t* gl = lists + (int64_t)bg * cpg * kListWords;
         constexpr int kU = (kMaxCpg * kPub + kThreads - 1) / kThreads;
@@ -481,34 +486,69 @@ decode_attend_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
         }
         uint64_t x = tid < cpg ? gl[tid * kListWords + kPub] : 0ull;  // cpg <= kThreads
         x = warp_max_u64(x);
-        if (lane == 0) sm.xpart[warp] = x;
-        if (tid == 0) sm.nwin = 0;
-        uint64_t prefix, mask;
-        radix_kth<kU>(uv, K, sm.ss, prefix, mask, tid, [] { __syncthreads(); });
+        int nz = 0;
+#pragma unroll
+        for (int i = 0; i < kU; ++i) {
+            const int e = tid + kThreads * i;
+            if (e < nu) sm.u[e] = uv[i];
+            nz += uv[i] != 0ull;
+        }
+        nz = __reduce_add_sync(0xffffffffu, nz);
+        if (lane == 0) {
+            sm.xpart[warp] = x;
+            sm.cnt_part[warp][0] = nz;
+        }
+        __syncthreads();
         uint64_t X = 0ull;
+        int nvalid = 0;
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w) X = sm.xpart[w] > X ? sm.xpart[w] : X;
-        // X, the largest key a list left out, would be a winner: the lists may hide winners.  (With
-        // fewer than K keys in U every key of U wins, and some list left keys out.)
-        const bool all_win = mask == ~0ull && prefix == 1ull;
-        rank_layout = all_win ? X == 0ull : !(X != 0ull && (X & mask) >= prefix);
+        for (int w = 0; w < kWarps; ++w) {
+            X = sm.xpart[w] > X ? sm.xpart[w] : X;
+            nvalid += sm.cnt_part[w][0];
+        }
+        int above = 0;  // keys of U above X
+#pragma unroll
+        for (int i = 0; i < kU; ++i) above += uv[i] > X;
+        above = __reduce_add_sync(0xffffffffu, above);
+        if (lane == 0) sm.cnt_part[warp][1] = above;
+        __syncthreads();
+        int rank_x = 0;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) rank_x += sm.cnt_part[w][1];
+        // X would be a winner when fewer than K keys of U beat it: the lists may then hide winners
+        // (with fewer than K keys in U every key wins, and some list left keys out).
+        rank_layout = X == 0ull || rank_x >= K;
         if (rank_layout) {
-#pragma unroll
-            for (int i = 0; i < kU; ++i) {
-                if (uv[i] != 0ull && (uv[i] & mask) >= prefix) {
-                    const int w = atomicAdd(&sm.nwin, 1);
-                    if (w < kCap) sm.wkeys[w] = uv[i];
+            // Every key's rank (the keys of U above it; keys are distinct) decides its slot: the
+            // winner of rank r < K is attended in slot r by CTA r mod CS.  This CTA ranks its share
+            // of U, eight threads per key, and writes each winner's block into the slot list of
+            // the CTA that attends it (and, with idx_out, into CTA 0's list of winners).
+            nwin = min(nvalid, K);
+            const int per = (nu + CS - 1) / CS, e0 = rk * per, e1 = min(nu, e0 + per);
+            const int sub = tid & 7;
+            const ulonglong2* u2 = reinterpret_cast<const ulonglong2*>(sm.u);  // nu is a multiple of 8
+            for (int base = e0; base < e1; base += kThreads / 8) {
+                const int e = base + (tid >> 3);
+                const uint64_t key = e < e1 ? sm.u[e] : 0ull;
+                int r = 0;
+#pragma unroll 4
+                for (int j = sub; j < nu / 2; j += 8) {  // two keys per 16-byte load, loads in flight
+                    const ulonglong2 p2 = u2[j];
+                    r += (p2.x > key) + (p2.y > key);
+                }
+                r += __shfl_xor_sync(0xffffffffu, r, 1);
+                r += __shfl_xor_sync(0xffffffffu, r, 2);
+                r += __shfl_xor_sync(0xffffffffu, r, 4);
+                if (sub == 0 && key != 0ull && r < K) {
+                    const int blk = key_block(key);
+                    *cl.map_shared_rank(&sm.sel[r], r % CS) = blk;
+                    if (idx_out) *cl.map_shared_rank(&sm.wblk[r], 0) = blk;
                 }
             }
-            for (int f = tid; f < n_init + n_local; f += kThreads) sm.sel[K + f] = forced_block(K + f);
-            __syncthreads();
-            if (warp == 0) {
-                const int nw = min(sm.nwin, K);
-                int x0 = 2 * lane < nw ? key_block(sm.wkeys[2 * lane]) : 0x7fffffff;
-                int x1 = 2 * lane + 1 < nw ? key_block(sm.wkeys[2 * lane + 1]) : 0x7fffffff;
-                warp_sort64(x0, x1, lane);
-                if (2 * lane < K) sm.sel[2 * lane] = 2 * lane < nw ? x0 : -1;
-                if (2 * lane + 1 < K) sm.sel[2 * lane + 1] = 2 * lane + 1 < nw ? x1 : -1;
+            // this CTA's own slots that no winner fills: the forced blocks, and -1 past the winners
+            for (int s = rk; s < slots; s += CS) {
+                if (s >= K) sm.sel[s] = forced_block(s);
+                else if (s >= nwin) sm.sel[s] = -1;
             }
         } else {
             // exact top-k over all the group's keys (written by the score kernel); the winners,
@@ -558,7 +598,10 @@ decode_attend_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
             sm.sel[s] = blk;
         }
     }
-    __syncthreads();
+    // With the score kernel's lists, winners were written into other CTAs' slot lists: a cluster
+    // barrier (the same on both of that path's branches, so every CTA of the cluster meets it).
+    if (owner) cl.sync();
+    else __syncthreads();
 
     // ---------------------------------------------------------------- attention of this CTA's slots
     // warp w < nitems attends slot rk + w CS in stage w and leaves the slot's partial (per head:
@@ -583,7 +626,7 @@ decode_attend_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
         } else {
             ptx::cp_async_wait<0>();
             __syncwarp();
-            for (int e = lane; e < G * (D + 2); e += 32) out[e] = e % (D + 2) == 0 ? -INFINITY : 0.f;
+            for (int e = lane; e < G * part_row<D>(); e += 32) out[e] = e % part_row<D>() == 0 ? -INFINITY : 0.f;
         }
     }
     __syncthreads();
@@ -596,7 +639,7 @@ decode_attend_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
         float M = -INFINITY;
 #pragma unroll
         for (int t = 0; t < kStages; ++t) {
-            m[t] = t < nitems ? reinterpret_cast<const float*>(stage_k(t))[h * (D + 2)] : -INFINITY;
+            m[t] = t < nitems ? reinterpret_cast<const float*>(stage_k(t))[h * part_row<D>()] : -INFINITY;
             M = fmaxf(M, m[t]);
         }
         float L = 0.f;
@@ -604,29 +647,36 @@ decode_attend_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
         for (int t = 0; t < kStages; ++t) {
             const float w8 = m[t] == -INFINITY ? 0.f : exp2f(m[t] - M);
             sm.wt[t][h] = w8;
-            if (t < nitems) L = fmaf(reinterpret_cast<const float*>(stage_k(t))[h * (D + 2) + 1], w8, L);
+            if (t < nitems) L = fmaf(reinterpret_cast<const float*>(stage_k(t))[h * part_row<D>() + 1], w8, L);
         }
         sm.fm[h] = M;
         sm.fl[h] = L;
     }
     __syncthreads();
-    for (int e = tid; e < G * (D + 2); e += kThreads) {
-        const int h = e / (D + 2), col = e % (D + 2);
-        float v;
-        if (col == 0) {
-            v = sm.fm[h];
-        } else if (col == 1) {
-            v = sm.fl[h];
+    // per head: (maximum, sum) as one 8-byte store, then the weighted p v sums 16 bytes at a time
+    constexpr int kQ = D / 4 + 1;
+    for (int e = tid; e < G * kQ; e += kThreads) {
+        const int h = e / kQ, q4 = e % kQ;
+        float* dst = cl.map_shared_rank(&sm.recv[h / kCS][rk][0], h % kCS);
+        if (q4 == 0) {
+            *reinterpret_cast<float2*>(dst) = make_float2(sm.fm[h], sm.fl[h]);
         } else {
-            float pv[kStages];
+            const int col = 4 + 4 * (q4 - 1);
+            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-            for (int t = 0; t < kStages; ++t)
-                pv[t] = t < nitems ? reinterpret_cast<const float*>(stage_k(t))[h * (D + 2) + col] : 0.f;
-            v = 0.f;
-#pragma unroll
-            for (int t = 0; t < kStages; ++t) v = fmaf(pv[t], sm.wt[t][h], v);
+            for (int t = 0; t < kStages; ++t) {
+                if (t < nitems) {
+                    const float4 pv = *reinterpret_cast<const float4*>(
+                        reinterpret_cast<const float*>(stage_k(t)) + h * part_row<D>() + col);
+                    const float w8 = sm.wt[t][h];
+                    v.x = fmaf(pv.x, w8, v.x);
+                    v.y = fmaf(pv.y, w8, v.y);
+                    v.z = fmaf(pv.z, w8, v.z);
+                    v.w = fmaf(pv.w, w8, v.w);
+                }
+            }
+            *reinterpret_cast<float4*>(dst + col) = v;
         }
-        *cl.map_shared_rank(&sm.recv[h / kCS][rk][col], h % kCS) = v;
     }
     cl.sync();  // every CTA's partials have landed where they are combined
     // CTA rk combines heads rk, rk + kCS, ... over the partials of every CTA of the cluster
@@ -638,7 +688,7 @@ decode_attend_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
             for (int p = 0; p < kCS; ++p) {
                 mp[p] = sm.recv[hh][p][0];
                 lp[p] = sm.recv[hh][p][1];
-                op[p] = sm.recv[hh][p][2 + tid];
+                op[p] = sm.recv[hh][p][4 + tid];
             }
             float M = -INFINITY;
 #pragma unroll
@@ -655,9 +705,15 @@ decode_attend_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
     }
     if (idx_out && rk == 0) {
         int32_t* dst = idx_out + (int64_t)bg * slots;
-        if (rank_layout) {
+        if (rank_layout) {  // the winners ascending by block (k <= 64: one warp sorts them)
             for (int s = tid; s < n_init; s += kThreads) dst[s] = s;
-            for (int s = tid; s < K; s += kThreads) dst[n_init + s] = sm.sel[s];
+            if (warp == 0) {
+                int x0 = 2 * lane < nwin ? sm.wblk[2 * lane] : 0x7fffffff;
+                int x1 = 2 * lane + 1 < nwin ? sm.wblk[2 * lane + 1] : 0x7fffffff;
+                warp_sort64(x0, x1, lane);
+                if (2 * lane < K) dst[n_init + 2 * lane] = 2 * lane < nwin ? x0 : -1;
+                if (2 * lane + 1 < K) dst[n_init + 2 * lane + 1] = 2 * lane + 1 < nwin ? x1 : -1;
+            }
             for (int t = tid; t < n_local; t += kThreads) dst[n_init + K + t] = c - n_local + 1 + t;
         } else {
             for (int s = tid; s < slots; s += kThreads) dst[s] = sm.sel[s];
