@@ -86,6 +86,8 @@ struct AttendSmem {
     uint64_t xpart[kWarps];
     int sel[kMaxSlots];               // slot -> block (-1: empty)
     int wblk[kCap];                   // CTA 0, with idx_out: the winners' blocks by rank
+    int nloc;                         // winners among this CTA's share of U ...
+    int loc_rank[kMaxCpg * kPub / kCS], loc_blk[kMaxCpg * kPub / kCS];  // ... their ranks and blocks
     uint64_t wkeys[kCap];
     int nwin;
     RadixSelSmem ss;
@@ -511,6 +513,7 @@ decode_attend_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
         for (int i = 0; i < kU; ++i) above += uv[i] > X;
         above = __reduce_add_sync(0xffffffffu, above);
         if (lane == 0) sm.cnt_part[warp][1] = above;
+        if (tid == 0) sm.nloc = 0;
         __syncthreads();
         int rank_x = 0;
 #pragma unroll
@@ -527,23 +530,40 @@ decode_attend_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
             const int per = (nu + CS - 1) / CS, e0 = rk * per, e1 = min(nu, e0 + per);
             const int sub = tid & 7;
             const ulonglong2* u2 = reinterpret_cast<const ulonglong2*>(sm.u);  // nu is a multiple of 8
-            for (int base = e0; base < e1; base += kThreads / 8) {
-                const int e = base + (tid >> 3);
-                const uint64_t key = e < e1 ? sm.u[e] : 0ull;
-                int r = 0;
+            // the share holds at most kMaxCpg * kPub / CS = 80 keys: up to three per group of eight
+            // threads, all ranked against each pair of U's keys as it is read
+            constexpr int kPerThread = (kMaxCpg * kPub / kCS + kThreads / 8 - 1) / (kThreads / 8);
+            uint64_t key[kPerThread];
+            int r[kPerThread];
+#pragma unroll
+            for (int m = 0; m < kPerThread; ++m) {
+                const int e = e0 + (tid >> 3) + (kThreads / 8) * m;
+                key[m] = e < e1 ? sm.u[e] : 0ull;
+                r[m] = 0;
+            }
 #pragma unroll 4
-                for (int j = sub; j < nu / 2; j += 8) {  // two keys per 16-byte load, loads in flight
-                    const ulonglong2 p2 = u2[j];
-                    r += (p2.x > key) + (p2.y > key);
+            for (int j = sub; j < nu / 2; j += 8) {
+                const ulonglong2 p2 = u2[j];
+#pragma unroll
+                for (int m = 0; m < kPerThread; ++m) r[m] += (p2.x > key[m]) + (p2.y > key[m]);
+            }
+#pragma unroll
+            for (int m = 0; m < kPerThread; ++m) {
+                r[m] += __shfl_xor_sync(0xffffffffu, r[m], 1);
+                r[m] += __shfl_xor_sync(0xffffffffu, r[m], 2);
+                r[m] += __shfl_xor_sync(0xffffffffu, r[m], 4);
+                if (sub == 0 && key[m] != 0ull && r[m] < K) {
+                    const int w = atomicAdd(&sm.nloc, 1);
+                    sm.loc_rank[w] = r[m];
+                    sm.loc_blk[w] = key_block(key[m]);
                 }
-                r += __shfl_xor_sync(0xffffffffu, r, 1);
-                r += __shfl_xor_sync(0xffffffffu, r, 2);
-                r += __shfl_xor_sync(0xffffffffu, r, 4);
-                if (sub == 0 && key != 0ull && r < K) {
-                    const int blk = key_block(key);
-                    *cl.map_shared_rank(&sm.sel[r], r % CS) = blk;
-                    if (idx_out) *cl.map_shared_rank(&sm.wblk[r], 0) = blk;
-                }
+            }
+            // the share's winners, gathered above, go out together: one thread each
+            __syncthreads();
+            if (tid < sm.nloc) {
+                const int r = sm.loc_rank[tid], blk = sm.loc_blk[tid];
+                *cl.map_shared_rank(&sm.sel[r], r % CS) = blk;
+                if (idx_out) *cl.map_shared_rank(&sm.wblk[r], 0) = blk;
             }
             // this CTA's own slots that no winner fills: the forced blocks, and -1 past the winners
             for (int s = rk; s < slots; s += CS) {
