@@ -71,8 +71,8 @@ def sparse_layer_flops(N: int) -> float:
 # ncu capture of the single-layer N = 131072 case, 2.323e9 bytes per launch, scaled by the tokens
 # processed to N = 262144 (Q reads, O writes and the K/V re-reads per 16-token unit all grow with N).
 # Valid only for the kernel sources it was taken on: any change to them reports null.
-SPARSE_TRAFFIC = {"bytes_per_token": (1287155200 + 1035656960) / 131072,
-                  "sources": {"sparse_tc.cu": "71ff73bea6734e4ba25f214f086e3ad2f0bacd0a1b9d8d7c123393baa9edd39c",
+SPARSE_TRAFFIC = {"bytes_per_token": (1288783104 + 1033887232) / 131072,
+                  "sources": {"sparse_tc.cu": "0b1ebdf2db4727e0e23f510939c7096e1ceba114f6c618463cff01c4d788a173",
                               "fastexp.cuh": "b6d9ae064f35b9fd752ec893180eaf72ade6f0495d57f5699832618f42784c06",
                               "ptx.cuh": "fd104364a691e71bb755a0a84573920e3263e23dbfbee024db781170b73eb422"}}
 
