@@ -141,3 +141,19 @@ def test_per_head_out_of_range_index_is_flagged(sala):
     assert ei.value.code == sala.ERR_BOUNDS
     assert torch.isfinite(o.float()).all()
     sala.check_status()
+
+
+def test_bf16_per_head_batch2_tensor_core_paths(sala):
+    # batch 2 through the tensor-core selection (more than 16 rows) and attention
+    from hybrid_sparse_linear_b200 import synth
+    layer = synth.sparse_layer(2, 32, 2, 64 * 10 + 7, 128, torch.bfloat16, layer=28, shift_frac=0.1)
+    _per_head_pipeline(sala, layer, "bf16", 8, 1, 2)
+
+
+def test_per_head_top0_forced_blocks_only(sala):
+    # k = 0: rows of three slots (init + two local), shorter than the four-entry look-ahead each
+    # softmax thread keeps over its own row
+    from hybrid_sparse_linear_b200 import synth
+    layer = synth.sparse_layer(1, 32, 2, 64 * 7 + 33, 128, torch.bfloat16, layer=29)
+    got, _ = _per_head_pipeline(sala, layer, "bf16", 0, 1, 2)
+    assert got.shape[-1] == 3
