@@ -56,11 +56,17 @@ constexpr int kOffSeedB = kOffBuf + kPilotChunk * 8;   // [128 seeds x 128 d], 2
 constexpr int kOffSeedSc = kOffBuf;  // [128 rows][kSeeds + 1] seed scores, once the seed MMA is done
 static_assert(kOffSeedB + 2 * kSub <= kOffBuf + kBufBytes, "buffer area too small");
 static_assert(kRows * (kSeeds + 1) * 4 <= kBufBytes, "buffer area too small for the seed scores");
+// While the group sum runs, the A operand area and the buffer area hold four stages of one query
+// head's 128 rows each ([128 rows x 256 B], as in global memory): stages 0-1 in A, 2-3 in the
+// buffers.  A is written only once every head has been summed.
+constexpr int kQStages = 4, kQStageBytes = kRows * kD * 2;
+static_assert(2 * kQStageBytes == kOffKb - kOffAhi && 2 * kQStageBytes <= kBufBytes, "Q stages");
 
 constexpr uint32_t kColS0 = 0, kColSeed = 256, kTmemCols = 512;
 
 struct Bars {
     uint64_t a_ready, seed_ready, seed_done;
+    uint64_t q_full[kQStages], q_empty[kQStages];
     uint64_t kv_full[2], kv_empty[2], s_full[2], s_free[2];
     uint64_t fin;
     uint32_t tmem_base;
@@ -188,6 +194,10 @@ topk_tc_kernel(const __grid_constant__ CUtensorMap tmKb, const __nv_bfloat16* __
             mbar_init(&bars.s_free[s], 4);
         }
         mbar_init(&bars.fin, 1);
+        for (int s = 0; s < kQStages; ++s) {
+            mbar_init(&bars.q_full[s], 1);
+            mbar_init(&bars.q_empty[s], 8);  // the worker warps
+        }
         bars.abort = 0;
         bars.sm_stop = 0;
         bars.n_seeds = 0;
@@ -198,9 +208,23 @@ topk_tc_kernel(const __grid_constant__ CUtensorMap tmKb, const __nv_bfloat16* __
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = bars.tmem_base;
+    auto q_stage = [&](int s) { return sm + (s < 2 ? kOffAhi : kOffBuf - 2 * kQStageBytes) + s * kQStageBytes; };
 
     if (warp == 8) {
         // ------------------------------------------------------------------ TMA producer
+        // First the tile's rows of the G query heads, one head per stage, for the group sum; then
+        // the kbar tiles of the main pass.
+        int hq = 0;  // heads issued
+        if (lane == 0) {
+            const uint32_t qbytes = (uint32_t)nrows * kD * 2;
+            for (; hq < G; ++hq) {
+                const int s = hq % kQStages, u = hq / kQStages;
+                if (u >= 1 && !mbar_wait(&bars.q_empty[s], (u - 1) & 1, ctx)) { *abort = 1; break; }
+                mbar_arrive_expect_tx(&bars.q_full[s], qbytes);
+                bulk_load_g2s(q_stage(s), q + ((b * H + (int64_t)g * G + hq) * Nq + r0) * kD, qbytes,
+                              &bars.q_full[s]);
+            }
+        }
         if (lane == 0 && n_tiles > 0) {
             int issued0 = -1, issued1 = -1;
             for (int t = 0; t < n_tiles; ++t) {
@@ -215,6 +239,10 @@ topk_tc_kernel(const __grid_constant__ CUtensorMap tmKb, const __nv_bfloat16* __
             }
             if (issued0 >= 0) (void)mbar_wait(&bars.kv_full[0], issued0 & 1, ctx);
             if (issued1 >= 0) (void)mbar_wait(&bars.kv_full[1], issued1 & 1, ctx);
+        }
+        if (lane == 0) {  // drain: the last head copied into each stage has landed
+            for (int s = 0; s < min(hq, kQStages); ++s)
+                (void)mbar_wait(&bars.q_full[s], ((s + kQStages * ((hq - 1 - s) / kQStages)) / kQStages) & 1, ctx);
         }
         __syncwarp();
     } else if (warp == 9) {
@@ -277,66 +305,62 @@ topk_tc_kernel(const __grid_constant__ CUtensorMap tmKb, const __nv_bfloat16* __
             ++nbar;
         };
         auto stop_now = [&]() { const int v = *sm_stop; return v != 0 && v <= nbar; };
-        // (1) group-summed queries -> A (hi, lo), pilot partial sums.  Warp w: rows 16w..16w+15,
-        // two rows at a time with all their heads' loads in flight; lane l: columns 4l..4l+3.
+        // (1) group-summed queries -> A (hi, lo), pilot partial sums.  The G heads' rows arrive
+        // one head per stage; warp w sums rows 16w..16w+15, lane l columns 4l..4l+3, adding the
+        // heads in order (rows past the tile stay 0).
         {
+            float acc[16][4];
+#pragma unroll
+            for (int rr = 0; rr < 16; ++rr)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) acc[rr][e] = 0.f;
+            for (int h = 0; h < G; ++h) {
+                const int s = h % kQStages, u = h / kQStages;
+                const bool got = mbar_wait(&bars.q_full[s], u & 1, ctx);
+                if (!__all_sync(0xffffffffu, got)) {
+                    fail();
+                    break;
+                }
+                const uint8_t* st = q_stage(s);
+                uint2 v[16];
+#pragma unroll
+                for (int rr = 0; rr < 16; ++rr)
+                    v[rr] = *reinterpret_cast<const uint2*>(st + (warp * 16 + rr) * (kD * 2) + 8 * lane);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars.q_empty[s]);
+#pragma unroll
+                for (int rr = 0; rr < 16; ++rr) {
+                    if (warp * 16 + rr >= nrows) continue;
+                    acc[rr][0] += __uint_as_float(v[rr].x << 16);
+                    acc[rr][1] += __uint_as_float(v[rr].x & 0xffff0000u);
+                    acc[rr][2] += __uint_as_float(v[rr].y << 16);
+                    acc[rr][3] += __uint_as_float(v[rr].y & 0xffff0000u);
+                }
+            }
+            // A and the buffer area held the stages: every worker is done reading them
+            sync_workers();
             float* ppart = reinterpret_cast<float*>(sm + kOffPPart);
             float pp[4] = {0.f, 0.f, 0.f, 0.f};
             const int sub = lane >> 4, chunk = (lane & 15) >> 1, within = (lane & 1) * 8;
-            for (int rr = 0; rr < 16; rr += 2) {
-                float a[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-                if (G <= kMaxG) {
-                    uint2 v[2][kMaxG];
 #pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const int row = warp * 16 + rr + u;
+            for (int rr = 0; rr < 16; ++rr) {
+                const int row = warp * 16 + rr;
+                float a[4];
 #pragma unroll
-                        for (int h = 0; h < kMaxG; ++h)
-                            v[u][h] = (row < nrows && h < G)
-                                          ? *reinterpret_cast<const uint2*>(
-                                                q + ((b * H + (int64_t)g * G + h) * Nq + r0 + row) * kD + 4 * lane)
-                                          : make_uint2(0u, 0u);
-                    }
+                for (int e = 0; e < 4; ++e) a[e] = G < kMaxG ? acc[rr][e] + 0.f : acc[rr][e];  // -0 -> +0 below 16 heads
+                uint32_t hb[2], lb2[2];
 #pragma unroll
-                    for (int u = 0; u < 2; ++u)
-#pragma unroll
-                        for (int h = 0; h < kMaxG; ++h) {
-                            a[u][0] += __uint_as_float(v[u][h].x << 16);
-                            a[u][1] += __uint_as_float(v[u][h].x & 0xffff0000u);
-                            a[u][2] += __uint_as_float(v[u][h].y << 16);
-                            a[u][3] += __uint_as_float(v[u][h].y & 0xffff0000u);
-                        }
-                } else {
-                    for (int u = 0; u < 2; ++u) {
-                        const int row = warp * 16 + rr + u;
-                        if (row >= nrows) continue;
-                        for (int h = 0; h < G; ++h) {
-                            const uint2 w2 = *reinterpret_cast<const uint2*>(
-                                q + ((b * H + (int64_t)g * G + h) * Nq + r0 + row) * kD + 4 * lane);
-                            a[u][0] += __uint_as_float(w2.x << 16);
-                            a[u][1] += __uint_as_float(w2.x & 0xffff0000u);
-                            a[u][2] += __uint_as_float(w2.y << 16);
-                            a[u][3] += __uint_as_float(w2.y & 0xffff0000u);
-                        }
-                    }
+                for (int e = 0; e < 2; ++e) {
+                    const __nv_bfloat16 h0 = __float2bfloat16_rn(a[2 * e]), h1 = __float2bfloat16_rn(a[2 * e + 1]);
+                    const float d0 = a[2 * e] - __bfloat162float(h0), d1 = a[2 * e + 1] - __bfloat162float(h1);
+                    hb[e] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
+                    lb2[e] = pack_bf16x2(d0, d1);
                 }
+                const int off = sub * kSub + row * 128 + ((chunk ^ (row & 7)) << 4) + within;
+                *reinterpret_cast<uint2*>(sm + kOffAhi + off) = make_uint2(hb[0], hb[1]);
+                *reinterpret_cast<uint2*>(sm + kOffAlo + off) = make_uint2(lb2[0], lb2[1]);
 #pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    const int row = warp * 16 + rr + u;
-                    uint32_t hb[2], lb2[2];
-#pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const __nv_bfloat16 h0 = __float2bfloat16_rn(a[u][2 * e]), h1 = __float2bfloat16_rn(a[u][2 * e + 1]);
-                        const float d0 = a[u][2 * e] - __bfloat162float(h0), d1 = a[u][2 * e + 1] - __bfloat162float(h1);
-                        hb[e] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
-                        lb2[e] = pack_bf16x2(d0, d1);
-                    }
-                    const int off = sub * kSub + row * 128 + ((chunk ^ (row & 7)) << 4) + within;
-                    *reinterpret_cast<uint2*>(sm + kOffAhi + off) = make_uint2(hb[0], hb[1]);
-                    *reinterpret_cast<uint2*>(sm + kOffAlo + off) = make_uint2(lb2[0], lb2[1]);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) pp[e] += a[u][e];
-                }
+                for (int e = 0; e < 4; ++e) pp[e] += a[e];
             }
 #pragma unroll
             for (int e = 0; e < 4; ++e) ppart[warp * kD + 4 * lane + e] = pp[e];
