@@ -553,10 +553,17 @@ topk_tc_kernel(const __grid_constant__ CUtensorMap tmKb, const __nv_bfloat16* __
                     return msk & keep;
                 };
                 auto append = [&](uint32_t msk) {
+                    // A row passes ~1 candidate of 32: park the chunk in this thread's local memory
+                    // (L1-resident) and visit only the set bits, in ascending order.
+                    if (msk == 0u) return;
+                    uint32_t xs[32];
 #pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        if (((msk >> j) & 1u) && in_bounds(ctx, n < kBufCap))
-                            buf[n++] = sel_key(__uint_as_float(x[j]), jb + j);
+                    for (int j = 0; j < 32; ++j) xs[j] = x[j];
+                    do {
+                        const int j = __ffs(msk) - 1;
+                        msk &= msk - 1u;
+                        if (in_bounds(ctx, n < kBufCap)) buf[n++] = sel_key(__uint_as_float(xs[j]), jb + j);
+                    } while (msk);
                 };
                 const uint32_t pass = passing(~0u);
                 if (__any_sync(0xffffffffu, n + __popc(pass) > kBufCap)) {
