@@ -61,12 +61,18 @@ static_assert(kRows * (kSeeds + 1) * 4 <= kBufBytes, "buffer area too small for 
 // buffers.  A is written only once every head has been summed.
 constexpr int kQStages = 4, kQStageBytes = kRows * kD * 2;
 static_assert(2 * kQStageBytes == kOffKb - kOffAhi && 2 * kQStageBytes <= kBufBytes, "Q stages");
+// The pilot scores read the candidates' kbar rows in pieces of 128 rows ([128 rows x 256 B]),
+// copied into three stages: the two kbar tile stages (the main pass loads them afterwards) and
+// the seed operand area (written once every piece has been scored).
+constexpr int kSdStages = 3, kSdRows = 128, kSdStageBytes = kSdRows * kD * 2;
+static_assert(2 * kSdStageBytes == 4 * kSub && kSdStageBytes <= 2 * kSub, "seed stages");
 
 constexpr uint32_t kColS0 = 0, kColSeed = 256, kTmemCols = 512;
 
 struct Bars {
     uint64_t a_ready, seed_ready, seed_done;
     uint64_t q_full[kQStages], q_empty[kQStages];
+    uint64_t sd_full[kSdStages], sd_empty[kSdStages];
     uint64_t kv_full[2], kv_empty[2], s_full[2], s_free[2];
     uint64_t fin;
     uint32_t tmem_base;
@@ -177,6 +183,10 @@ topk_tc_kernel(const __grid_constant__ CUtensorMap tmKb, const __nv_bfloat16* __
     const int ncand_all = hi_all - lo + 1;
     const bool rank = (hi - lo + 1) > topk && K > 0;  // some row has more candidates than k
     const int n_tiles = rank ? (hi - lo + kCand) / kCand : 0;
+    // Seeds (the pilot's best kSeeds candidates of [lo, hi_all]) are used when every row may take
+    // that many; the pilot scores go through a radix select in chunks of kNew candidates.
+    const bool seeded = rank && ncand_all >= kSeeds;
+    constexpr int kNew = kPilotChunk - kSeeds;
     volatile int* abort = &bars.abort;
 
     if (warp == 9) {
@@ -198,6 +208,10 @@ topk_tc_kernel(const __grid_constant__ CUtensorMap tmKb, const __nv_bfloat16* __
             mbar_init(&bars.q_full[s], 1);
             mbar_init(&bars.q_empty[s], 8);  // the worker warps
         }
+        for (int s = 0; s < kSdStages; ++s) {
+            mbar_init(&bars.sd_full[s], 1);
+            mbar_init(&bars.sd_empty[s], 8);
+        }
         bars.abort = 0;
         bars.sm_stop = 0;
         bars.n_seeds = 0;
@@ -209,6 +223,7 @@ topk_tc_kernel(const __grid_constant__ CUtensorMap tmKb, const __nv_bfloat16* __
     tc_fence_after();
     const uint32_t tmem = bars.tmem_base;
     auto q_stage = [&](int s) { return sm + (s < 2 ? kOffAhi : kOffBuf - 2 * kQStageBytes) + s * kQStageBytes; };
+    auto sd_stage = [&](int s) { return sm + (s < 2 ? kOffKb + s * kSdStageBytes : kOffSeedB); };
 
     if (warp == 8) {
         // ------------------------------------------------------------------ TMA producer
@@ -225,6 +240,38 @@ topk_tc_kernel(const __grid_constant__ CUtensorMap tmKb, const __nv_bfloat16* __
                               &bars.q_full[s]);
             }
         }
+        // Then the candidates' kbar rows for the pilot scores, piece by piece, and once the pieces
+        // in the kbar tile stages have been read, the main pass's tiles.
+        int ksd = 0;  // pieces issued
+        if (lane == 0 && seeded) {
+            bool ok = true;
+            for (int cb = 0; cb < ncand_all && ok; cb += kNew) {
+                const int nc = min(kNew, ncand_all - cb);
+                for (int sc0 = 0; sc0 < nc; sc0 += kSdRows, ++ksd) {
+                    const int s = ksd % kSdStages, u = ksd / kSdStages;
+                    if (u >= 1 && !mbar_wait(&bars.sd_empty[s], (u - 1) & 1, ctx)) {
+                        *abort = 1;
+                        ok = false;
+                        break;
+                    }
+                    // seed stage 2 is query stage 3: its last head must have been read
+                    constexpr int kQ3 = kQStages - 1;
+                    static_assert(kSdStages == 3 && kOffSeedB == kOffBuf + kQStageBytes, "stage overlap");
+                    if (ksd == 2 && hq > kQ3 &&
+                        !mbar_wait(&bars.q_empty[kQ3], ((kQ3 + kQStages * ((hq - 1 - kQ3) / kQStages)) / kQStages) & 1, ctx)) {
+                        *abort = 1;
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t bytes = (uint32_t)min(kSdRows, nc - sc0) * kD * 2;
+                    mbar_arrive_expect_tx(&bars.sd_full[s], bytes);
+                    bulk_load_g2s(sd_stage(s), kbar + (kv_plane * nb + lo + cb + sc0) * (int64_t)kD, bytes,
+                                  &bars.sd_full[s]);
+                }
+            }
+            for (int s = 0; s < min(ksd, 2); ++s)
+                (void)mbar_wait(&bars.sd_empty[s], ((s + kSdStages * ((ksd - 1 - s) / kSdStages)) / kSdStages) & 1, ctx);
+        }
         if (lane == 0 && n_tiles > 0) {
             int issued0 = -1, issued1 = -1;
             for (int t = 0; t < n_tiles; ++t) {
@@ -240,9 +287,11 @@ topk_tc_kernel(const __grid_constant__ CUtensorMap tmKb, const __nv_bfloat16* __
             if (issued0 >= 0) (void)mbar_wait(&bars.kv_full[0], issued0 & 1, ctx);
             if (issued1 >= 0) (void)mbar_wait(&bars.kv_full[1], issued1 & 1, ctx);
         }
-        if (lane == 0) {  // drain: the last head copied into each stage has landed
+        if (lane == 0) {  // drain: the last copy into each stage has landed
             for (int s = 0; s < min(hq, kQStages); ++s)
                 (void)mbar_wait(&bars.q_full[s], ((s + kQStages * ((hq - 1 - s) / kQStages)) / kQStages) & 1, ctx);
+            for (int s = 0; s < min(ksd, kSdStages); ++s)
+                (void)mbar_wait(&bars.sd_full[s], ((s + kSdStages * ((ksd - 1 - s) / kSdStages)) / kSdStages) & 1, ctx);
         }
         __syncwarp();
     } else if (warp == 9) {
@@ -378,34 +427,46 @@ topk_tc_kernel(const __grid_constant__ CUtensorMap tmKb, const __nv_bfloat16* __
         }
         sync_workers();
         // (2) seeds: the best kSeeds candidates of [lo, hi_all] by the pilot score (every row may
-        // take them).  Pilot scores of a chunk of candidates (coalesced kbar rows, 8 lanes per row,
-        // eight rows per lane in flight) plus the winners so far, then a radix select.
-        const bool seeded = rank && ncand_all >= kSeeds;
+        // take them).  Pilot scores of a chunk of candidates, read from the staged kbar pieces (8
+        // lanes per row, lane l: columns 8(l%8)..+7 and 64+8(l%8)..+7), plus the winners so far,
+        // then a radix select.
         if (seeded) {
             uint64_t* pkeys = reinterpret_cast<uint64_t*>(sm + kOffPKeys);
             if (tid < kSeeds) bars.carry[tid] = 0ull;
             sync_workers();
-            constexpr int kNew = kPilotChunk - kSeeds, kBatch = 8;
             const int part = lane & 7;
-            const float* pv = bars.pilot + part * 16;
+            float pv[16];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                pv[e] = bars.pilot[part * 8 + e];
+                pv[8 + e] = bars.pilot[64 + part * 8 + e];
+            }
+            int ksd = 0;  // pieces consumed
             for (int cb = 0; cb < ncand_all; cb += kNew) {
                 const int nc = min(kNew, ncand_all - cb);
-                for (int it0 = 0; it0 < nc; it0 += 32 * kBatch) {
-                    uint4 raw[kBatch][2];
-#pragma unroll
-                    for (int st = 0; st < kBatch; ++st) {
-                        const int i = it0 + st * 32 + warp * 4 + (lane >> 3);
-                        const uint4* row = reinterpret_cast<const uint4*>(
-                            kbar + (kv_plane * nb + lo + cb + i) * (int64_t)kD + part * 16);
-                        raw[st][0] = i < nc ? row[0] : make_uint4(0u, 0u, 0u, 0u);
-                        raw[st][1] = i < nc ? row[1] : make_uint4(0u, 0u, 0u, 0u);
+                for (int sc0 = 0; sc0 < nc; sc0 += kSdRows, ++ksd) {
+                    const int s = ksd % kSdStages;
+                    const bool got = !dead && mbar_wait(&bars.sd_full[s], (ksd / kSdStages) & 1, ctx);
+                    if (!__all_sync(0xffffffffu, got)) {
+                        if (!dead) fail();
+                        continue;
                     }
+                    const uint8_t* st = sd_stage(s);
+                    uint4 raw[4][2];
 #pragma unroll
-                    for (int st = 0; st < kBatch; ++st) {
+                    for (int ps = 0; ps < 4; ++ps) {
+                        const uint8_t* row = st + (ps * 32 + warp * 4 + (lane >> 3)) * (kD * 2) + part * 16;
+                        raw[ps][0] = *reinterpret_cast<const uint4*>(row);
+                        raw[ps][1] = *reinterpret_cast<const uint4*>(row + 128);
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bars.sd_empty[s]);
+#pragma unroll
+                    for (int ps = 0; ps < 4; ++ps) {
                         float d0 = 0.f, d1 = 0.f;
 #pragma unroll
                         for (int u = 0; u < 2; ++u) {
-                            const uint4 v = raw[st][u];
+                            const uint4 v = raw[ps][u];
                             const float* p8 = pv + 8 * u;
                             d0 = fmaf(p8[0], __uint_as_float(v.x << 16), d0);
                             d1 = fmaf(p8[1], __uint_as_float(v.x & 0xffff0000u), d1);
@@ -420,7 +481,7 @@ topk_tc_kernel(const __grid_constant__ CUtensorMap tmKb, const __nv_bfloat16* __
                         d += __shfl_xor_sync(0xffffffffu, d, 1);
                         d += __shfl_xor_sync(0xffffffffu, d, 2);
                         d += __shfl_xor_sync(0xffffffffu, d, 4);
-                        const int i = it0 + st * 32 + warp * 4 + (lane >> 3);
+                        const int i = sc0 + ps * 32 + warp * 4 + (lane >> 3);
                         if (part == 0 && i < nc) pkeys[i] = sel_key(d, lo + cb + i);
                     }
                 }
