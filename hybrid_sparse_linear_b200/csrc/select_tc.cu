@@ -683,45 +683,68 @@ topk_tc_kernel(const __grid_constant__ CUtensorMap tmKb, const __nv_bfloat16* __
         }
         sync_workers();
         // (5) output rows: init ids, the top-k ids in ascending order, local ids, -1 padding.
-        // Warp w: rows 16w..16w+15, four at a time; a ranked row's k-th best score comes from a
-        // bitwise select over its buffer's scores, and its best k keys are taken in buffer (=
-        // block) order.
+        // Warp w: rows 16w..16w+15.  A ranked row keeps the K largest keys of its buffer (score,
+        // then the lower block), in buffer (= block) order.  The buffer holds n >= K keys, rarely
+        // many more: the d = n - K smallest are dropped one at a time (two warp-wide minima
+        // each); a row with more than kDrop extra keys takes the bitwise select of its K-th best
+        // score instead.  Both keep the same keys.
         if (!stop_now() && !dead) {
             const uint64_t* bufs = reinterpret_cast<const uint64_t*>(sm + kOffBuf);
+            constexpr int kDrop = 8;
+            const unsigned below = (1u << lane) - 1u;
 #pragma unroll 1
-            for (int i = 0; i < 16; i += 4) {
-                uint32_t v[4][4];
-                int nr[4];
-#pragma unroll
-                for (int r = 0; r < 4; ++r) {
-                    const int row = warp * 16 + i + r;
-                    const bool ranked = row < nrows && (r0 + row) / kBlk - n_local - n_init + 1 > topk;
-                    nr[r] = ranked ? min(bars.buf_n[row], kBufCap) : 0;
-#pragma unroll
-                    for (int u = 0; u < 4; ++u)
-                        v[r][u] = 4 * lane + u < nr[r] ? (uint32_t)(bufs[row * kBufCap + 4 * lane + u] >> 32) : 0u;
+            for (int i = 0; i < 16; ++i) {
+                const int row = warp * 16 + i;
+                if (row >= nrows) break;
+                const int rq = r0 + row;
+                const int c = rq / kBlk;
+                int32_t* out = idx + (bg * Nq + rq) * (int64_t)slots;
+                if (c - n_local - n_init + 1 <= topk) {
+                    for (int sl = lane; sl < slots; sl += 32) out[sl] = sl <= c ? sl : -1;
+                    continue;
                 }
-                uint32_t kth[4];
-                kth_largest<4, 32>(v, K, kth);
+                const int n = min(bars.buf_n[row], kBufCap);
+                const uint64_t* b = bufs + row * kBufCap;
+                int kept;
+                if (n - K > kDrop) {
+                    uint32_t v[1][4];
 #pragma unroll
-                for (int r = 0; r < 4; ++r) {
-                    const int row = warp * 16 + i + r;
-                    if (row >= nrows) continue;
-                    const int rq = r0 + row;
-                    const int c = rq / kBlk;
-                    int32_t* out = idx + (bg * Nq + rq) * (int64_t)slots;
-                    if (c - n_local - n_init + 1 <= topk) {
-                        for (int sl = lane; sl < slots; sl += 32) out[sl] = sl <= c ? sl : -1;
-                        continue;
+                    for (int u = 0; u < 4; ++u) v[0][u] = 4 * lane + u < n ? (uint32_t)(b[4 * lane + u] >> 32) : 0u;
+                    uint32_t t[1];
+                    kth_largest<1, 32>(v, K, t);
+                    kept = keep_best(b, n, K, t[0], lane,
+                                     [&](int pos, uint64_t key) { out[n_init + pos] = key_block(key); });
+                } else {
+                    uint64_t key[3];
+                    bool keep[3];
+#pragma unroll
+                    for (int j = 0; j < 3; ++j) {
+                        const int p = lane + 32 * j;
+                        keep[j] = p < n;
+                        key[j] = keep[j] ? b[p] : 0ull;
                     }
-                    const uint32_t s_k = kth[r];
-                    const int kept = keep_best(bufs + row * kBufCap, nr[r], K, s_k, lane,
-                                               [&](int pos, uint64_t key) { out[n_init + pos] = key_block(key); });
-                    for (int u = kept + lane; u < K; u += 32) out[n_init + u] = -1;  // unreachable: >= k kept
-                    for (int sl = lane; sl < n_init; sl += 32) out[sl] = sl;
-                    for (int u = lane; u < n_local; u += 32) out[n_init + K + u] = c - n_local + 1 + u;
-                    for (int sl = n_init + K + n_local + lane; sl < slots; sl += 32) out[sl] = -1;
+                    for (int it = K; it < n; ++it) {  // drop the smallest key still kept
+                        uint64_t m = ~0ull;
+#pragma unroll
+                        for (int j = 0; j < 3; ++j) m = keep[j] && key[j] < m ? key[j] : m;
+                        const uint32_t mh = __reduce_min_sync(0xffffffffu, (uint32_t)(m >> 32));
+                        const uint32_t ml = __reduce_min_sync(0xffffffffu, (uint32_t)(m >> 32) == mh ? (uint32_t)m : ~0u);
+                        const uint64_t mk = ((uint64_t)mh << 32) | ml;
+#pragma unroll
+                        for (int j = 0; j < 3; ++j) keep[j] = keep[j] && key[j] != mk;
+                    }
+                    kept = 0;
+#pragma unroll
+                    for (int j = 0; j < 3; ++j) {
+                        const unsigned ut = __ballot_sync(0xffffffffu, keep[j]);
+                        if (keep[j]) out[n_init + kept + __popc(ut & below)] = key_block(key[j]);
+                        kept += __popc(ut);
+                    }
                 }
+                for (int u = kept + lane; u < K; u += 32) out[n_init + u] = -1;  // unreachable: >= k kept
+                for (int sl = lane; sl < n_init; sl += 32) out[sl] = sl;
+                for (int u = lane; u < n_local; u += 32) out[n_init + K + u] = c - n_local + 1 + u;
+                for (int sl = n_init + K + n_local + lane; sl < slots; sl += 32) out[sl] = -1;
             }
         }
     }
