@@ -17,9 +17,14 @@
 // one thread per query row reads its 128 scores straight from TMEM, compares each with the row's
 // floor, and appends the few that pass to the row's buffer in shared memory, in ascending block
 // order.  A full buffer is cut back to its best k, order kept (the floor rises to the k-th
-// score); at the end each row's k-th best score is found by a bitwise select and the best k keys
-// are taken in buffer order.  Key = (orderable score, ~block), so ties go to the lower block
-// index.  Output as the CUDA-core path: init ids, top-k ids ascending, local ids.
+// score); at the end the buffer's smallest keys are dropped until k remain (a bitwise select of
+// the k-th best score when many more than k are left), and the rest are taken in buffer order.
+// Key = (orderable score, ~block), so ties go to the lower block index.  Output as the
+// CUDA-core path: init ids, top-k ids ascending, local ids.
+//
+// The producer warp also stages, by bulk copies, what the phases before the main pass read:
+// each query head's rows of the tile for the group sum, and the candidates' kbar rows for the
+// pilot scores, in areas the later phases take over.
 //
 // Roles (320 threads): warps 0-7 workers (the main pass runs on warps 0-3, thread = row = TMEM
 // lane), warp 8 TMA producer (kbar tiles), warp 9 TMEM owner and MMA issuer.  Every wait is
@@ -53,9 +58,7 @@ constexpr int kPilotChunk = 16 * kWorkers;             // keys per radix-select 
 constexpr int kOffPKeys = kOffBuf;                     // [kPilotChunk] keys
 constexpr int kSeeds = 2 * kCap;                       // pilot seeds (the floor uses the k-th)
 constexpr int kOffSeedB = kOffBuf + kPilotChunk * 8;   // [128 seeds x 128 d], 2 sub-tiles
-constexpr int kOffSeedSc = kOffBuf;  // [128 rows][kSeeds + 1] seed scores, once the seed MMA is done
 static_assert(kOffSeedB + 2 * kSub <= kOffBuf + kBufBytes, "buffer area too small");
-static_assert(kRows * (kSeeds + 1) * 4 <= kBufBytes, "buffer area too small for the seed scores");
 // While the group sum runs, the A operand area and the buffer area hold four stages of one query
 // head's 128 rows each ([128 rows x 256 B], as in global memory): stages 0-1 in A, 2-3 in the
 // buffers.  A is written only once every head has been summed.
@@ -524,40 +527,43 @@ topk_tc_kernel(const __grid_constant__ CUtensorMap tmKb, const __nv_bfloat16* __
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars.seed_ready);
-        // (3) per-row floors: the k-th best of the row's own seed scores.  Warps 0-3 (thread = row)
-        // park the scores in shared memory (the seed operand is consumed by then); each worker warp
-        // then sorts 16 rows' scores.
+        // (3) per-row floors: the k-th best of the row's own seed scores, to 16 bits of its
+        // orderable form.  Warps 0-3, thread = row = TMEM lane: the row's seed scores come into
+        // registers, and the bits of the k-th best are decided one at a time by counting, from the
+        // highest bit in which the row's largest and smallest seed scores differ (the bits above
+        // are common to all of them, hence to the k-th best).
         if (seeded && n_tiles > 0) {
-            float* sc = reinterpret_cast<float*>(sm + kOffSeedSc);  // [128][kSeeds + 1]
             if (warp < 4) {
                 if (!mbar_wait(&bars.seed_done, 0, ctx)) fail();
                 tc_fence_after();
+                float fl = -INFINITY;
                 if (!__any_sync(0xffffffffu, dead)) {
                     const uint32_t lb = tmem_lane_base(warp);
-#pragma unroll 1
-                    for (int c = 0; c < kSeeds; c += 32) {
-                        uint32_t x[32];
-                        tmem_ld32(tmem + lb + kColSeed + c, x);
-                        tmem_ld_wait();
+                    uint32_t x[kSeeds];
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) sc[tid * (kSeeds + 1) + c + j] = __uint_as_float(x[j]);
+                    for (int c = 0; c < kSeeds; c += 32)
+                        tmem_ld32(tmem + lb + kColSeed + c, *reinterpret_cast<uint32_t(*)[32]>(x + c));
+                    tmem_ld_wait();
+                    uint32_t omax = 0u, omin = ~0u;
+#pragma unroll
+                    for (int j = 0; j < kSeeds; ++j) {
+                        x[j] = orderable(__uint_as_float(x[j]));
+                        omax = max(omax, x[j]);
+                        omin = min(omin, x[j]);
                     }
-                }
-            }
-            sync_workers();
+                    const int p = __clz(omax ^ omin);  // 32 when all are equal
+                    uint32_t t = p >= 32 ? omax : omax & ~(0xffffffffu >> p);
 #pragma unroll 1
-            for (int i = 0; i < 16; i += 4) {
-                uint32_t v[4][4];
+                    for (int bit = 31 - p; bit >= 16; --bit) {
+                        const uint32_t c = t | (1u << bit);
+                        int cnt = 0;
 #pragma unroll
-                for (int r = 0; r < 4; ++r)
-#pragma unroll
-                    for (int u = 0; u < 4; ++u)
-                        v[r][u] = orderable(sc[(warp * 16 + i + r) * (kSeeds + 1) + 4 * lane + u]);
-                uint32_t t[4];
-                kth_largest<4, 16>(v, K, t);
-#pragma unroll
-                for (int r = 0; r < 4; ++r)
-                    if (lane == 0) bars.floor_s[warp * 16 + i + r] = from_orderable(t[r]);
+                        for (int j = 0; j < kSeeds; ++j) cnt += x[j] >= c ? 1 : 0;
+                        t = cnt >= K ? c : t;
+                    }
+                    fl = from_orderable(t & 0xffff0000u);
+                }
+                bars.floor_s[tid] = fl;
             }
         } else if (tid < kRows) {
             bars.floor_s[tid] = -INFINITY;
