@@ -235,9 +235,11 @@ def test_sparse_decode_clustered_winners_take_the_exact_fallback(sala):
     layer = synth.sparse_layer(1, H, Hkv, T, d, torch.bfloat16, device="cuda", layer=17,
                                shift_frac=0.02, q_rows=1)
     kbar = sala.block_compress(layer.k)
-    q64 = _f64(layer.q)
+    q64, k64 = _f64(layer.q), _f64(layer.k)
     qbar = q64[0].reshape(Hkv, H // Hkv, d).sum(axis=1)                    # [Hkv, d]
-    kb = _f64(kbar)
+    # the planted k-bar starts from the oracle's compression (the GPU's must equal it bitwise)
+    kb = oracle.block_compress(k64, 64, round_to_bf16=True)
+    np.testing.assert_array_equal(_f64(kbar)[:, :, :kb.shape[2]], kb)
     planted = []
     for t in range(20):
         for r in range(4):
@@ -261,7 +263,7 @@ def test_sparse_decode_clustered_winners_take_the_exact_fallback(sala):
     check_selection(got, idx_ref, q64, kb_ref, kth, topk, n_init, n_local, q_pos0=T - 1,
                     row_ids=np.array([0]))
     assert set(got[0, 0, 0, n_init:n_init + topk]) <= set(planted)
-    o_ref = oracle.sparse_attention(q64, _f64(layer.k), _f64(layer.v), got, 64, q_pos0=T - 1)
+    o_ref = oracle.sparse_attention(q64, k64, _f64(layer.v), got, 64, q_pos0=T - 1)
     assert_close(_f64(o), o_ref[:, :, 0], "bf16", "decode o")
 
 
