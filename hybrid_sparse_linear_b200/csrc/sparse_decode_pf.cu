@@ -18,11 +18,12 @@
 //      block) by counting ranks, and stores them, and all its keys, for the attend kernel.
 //   attend kernel (groups clusters of CS CTAs), launched as a programmatic dependent of the score
 //      kernel: before griddepcontrol.wait it loads the query rows and starts copying the init and
-//      local blocks; after it, every CTA reads the group's lists U (kPub keys per scoring CTA) and
-//      ranks its share of U's keys: a key of rank r < k is the group's (r+1)-th best block.  This is
-//      exact unless some scoring CTA had more than kPub winners: with X = the largest (kPub+1)-th
-//      key of any CTA, no unlisted key can beat X, so when fewer than k keys of U exceed X the
-//      cluster instead takes an exact radix select over all the group's keys.  The winners, by rank,
+//      local blocks; after it, every CTA reads the group's lists U (kPub keys per scoring CTA).
+//      With X = the largest (kPub+1)-th key of any CTA, no unlisted key can beat X; when at least
+//      k keys of U exceed X, the winners are among those keys C, and every CTA ranks its share of C
+//      against C: a key of rank r < k is the group's (r+1)-th best block.  When fewer than k keys
+//      of U exceed X (some scoring CTA had more than kPub winners), the cluster instead takes an
+//      exact radix select over all the group's keys.  The winners, by rank,
 //      are broadcast to the cluster through distributed shared memory.  CTA r then attends slots
 //      r, r + CS, ... (a warp per slot: K and V of the block by 16-byte asynchronous copies, the
 //      G heads' logits and p v on warp-level tensor-core tiles, a softmax partial per head), folds
@@ -81,8 +82,9 @@ struct ScoreSmem {
 template <int D>
 struct AttendSmem {
     __nv_bfloat16 Qb[kMaxG][D + 8];
-    alignas(16) uint64_t u[kMaxCpg * kPub];  // the group's lists (read two at a time)
-    int cnt_part[kWarps][2];          // per warp: nonzero keys of U, keys of U above X
+    alignas(16) uint64_t u[kMaxCpg * kPub];  // C, the keys of U above X (read two at a time)
+    int cnt_part[kWarps];             // per warp: nonzero keys of U
+    int cnt_c[(kMaxCpg * kPub + kThreads - 1) / kThreads][kWarps];  // per (key slot, warp): keys above X
     uint64_t xpart[kWarps];
     int sel[kMaxSlots];               // slot -> block (-1: empty)
     int wblk[kCap];                   // CTA 0, with idx_out: the winners' blocks by rank
@@ -476,7 +478,7 @@ decode_attend_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
     bool rank_layout = false;  // slots 0 .. K-1: the winners by rank, then the forced blocks
     int nwin = 0;              // winners on the rank path (min(K, nonzero keys of U))
     if (owner) {
-        // U, the group's lists, into shared memory; X, the largest key any list left out
+        // U, the group's lists, into registers; X, the largest key any list left out
         const int nu = cpg * kPub;
         const uint64_t* gl = lists + (int64_t)bg * cpg * kListWords;
         constexpr int kU = (kMaxCpg * kPub + kThreads - 1) / kThreads;
@@ -490,15 +492,11 @@ decode_attend_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
         x = warp_max_u64(x);
         int nz = 0;
 #pragma unroll
-        for (int i = 0; i < kU; ++i) {
-            const int e = tid + kThreads * i;
-            if (e < nu) sm.u[e] = uv[i];
-            nz += uv[i] != 0ull;
-        }
+        for (int i = 0; i < kU; ++i) nz += uv[i] != 0ull;
         nz = __reduce_add_sync(0xffffffffu, nz);
         if (lane == 0) {
             sm.xpart[warp] = x;
-            sm.cnt_part[warp][0] = nz;
+            sm.cnt_part[warp] = nz;
         }
         __syncthreads();
         uint64_t X = 0ull;
@@ -506,32 +504,55 @@ decode_attend_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
 #pragma unroll
         for (int w = 0; w < kWarps; ++w) {
             X = sm.xpart[w] > X ? sm.xpart[w] : X;
-            nvalid += sm.cnt_part[w][0];
+            nvalid += sm.cnt_part[w];
         }
-        int above = 0;  // keys of U above X
+        // C = the keys of U above X, in (key slot, thread) order.  A key at or below X has at
+        // least |C| keys above it, so when |C| >= K only keys of C can win, and a key of C has
+        // the same rank in C as in U (every key above it is in C).
+        unsigned ab[kU];
 #pragma unroll
-        for (int i = 0; i < kU; ++i) above += uv[i] > X;
-        above = __reduce_add_sync(0xffffffffu, above);
-        if (lane == 0) sm.cnt_part[warp][1] = above;
+        for (int i = 0; i < kU; ++i) ab[i] = __ballot_sync(0xffffffffu, uv[i] > X);
+        if (lane == 0) {
+#pragma unroll
+            for (int i = 0; i < kU; ++i) sm.cnt_c[i][warp] = __popc(ab[i]);
+        }
         if (tid == 0) sm.nloc = 0;
         __syncthreads();
-        int rank_x = 0;
+        const unsigned below = (1u << lane) - 1u;
+        int rank_x = 0;  // |C|: the keys of U above X
+        int pos[kU];
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w) rank_x += sm.cnt_part[w][1];
+        for (int i = 0; i < kU; ++i) {
+            int before = 0, tot = 0;
+#pragma unroll
+            for (int w = 0; w < kWarps; ++w) {
+                const int c = sm.cnt_c[i][w];
+                tot += c;
+                before += w < warp ? c : 0;
+            }
+            pos[i] = rank_x + before + __popc(ab[i] & below);
+            rank_x += tot;
+        }
         // X would be a winner when fewer than K keys of U beat it: the lists may then hide winners
         // (with fewer than K keys in U every key wins, and some list left keys out).
         rank_layout = X == 0ull || rank_x >= K;
         if (rank_layout) {
-            // Every key's rank (the keys of U above it; keys are distinct) decides its slot: the
+            // Every key's rank (the keys of C above it; keys are distinct) decides its slot: the
             // winner of rank r < K is attended in slot r by CTA r mod CS.  This CTA ranks its share
-            // of U, eight threads per key, and writes each winner's block into the slot list of
+            // of C, eight threads per key, and writes each winner's block into the slot list of
             // the CTA that attends it (and, with idx_out, into CTA 0's list of winners).
+#pragma unroll
+            for (int i = 0; i < kU; ++i)
+                if (uv[i] > X) sm.u[pos[i]] = uv[i];
+            if (tid == 0 && (rank_x & 1)) sm.u[rank_x] = 0ull;  // even length (rank_x < nu here)
+            __syncthreads();
             nwin = min(nvalid, K);
-            const int per = (nu + CS - 1) / CS, e0 = rk * per, e1 = min(nu, e0 + per);
+            const int nc = rank_x;
+            const int per = (nc + CS - 1) / CS, e0 = rk * per, e1 = min(nc, e0 + per);
             const int sub = tid & 7;
-            const ulonglong2* u2 = reinterpret_cast<const ulonglong2*>(sm.u);  // nu is a multiple of 8
+            const ulonglong2* u2 = reinterpret_cast<const ulonglong2*>(sm.u);
             // the share holds at most kMaxCpg * kPub / CS = 80 keys: up to three per group of eight
-            // threads, all ranked against each pair of U's keys as it is read
+            // threads, all ranked against each pair of C's keys as it is read
             constexpr int kPerThread = (kMaxCpg * kPub / kCS + kThreads / 8 - 1) / (kThreads / 8);
             uint64_t key[kPerThread];
             int r[kPerThread];
@@ -542,7 +563,7 @@ decode_attend_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
                 r[m] = 0;
             }
 #pragma unroll 4
-            for (int j = sub; j < nu / 2; j += 8) {
+            for (int j = sub; j < (nc + 1) / 2; j += 8) {
                 const ulonglong2 p2 = u2[j];
 #pragma unroll
                 for (int m = 0; m < kPerThread; ++m) r[m] += (p2.x > key[m]) + (p2.y > key[m]);
