@@ -273,8 +273,8 @@ sparse_decode_fused_kernel(const T* __restrict__ q, const T* __restrict__ kc,
                 block_sort_desc<2>(x, sm.cand);
                 if (tid == (K - 1) / 2) sm.cand[0] = ((K - 1) & 1) ? x[1] : x[0];  // buf is free again
                 __syncthreads();
-                const uint64_t T = sm.cand[0];
-                if (T == 0ull || (k8[0] && k8[0] >= T) || (k8[1] && k8[1] >= T)) sm.overflow = 1;
+                const uint64_t kth = sm.cand[0];  // the K-th best loaded key
+                if (kth == 0ull || (k8[0] && k8[0] >= kth) || (k8[1] && k8[1] >= kth)) sm.overflow = 1;
                 __syncthreads();
                 if (!sm.overflow) {
 #pragma unroll
